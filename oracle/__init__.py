@@ -1,0 +1,265 @@
+"""CPU oracle for the sparse-MoE SwiGLU layer forward (ctypes over moe_oracle.c).
+
+TEST INFRASTRUCTURE ONLY: imported by tests/, by the smoke check and by the
+CPU-baseline leg of bench.py.  The GPU product path never imports it.
+
+Every numerical function lives in moe_oracle.c; this module only marshals
+numpy arrays.  See the C file for the citations of each step.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+SO = os.path.join(_HERE, "_moe_oracle.so")
+SRC = os.path.join(_HERE, "moe_oracle.c")
+
+F32, BF16, F16, Q4_0 = 0, 1, 2, 3
+
+
+def build(force: bool = False) -> str:
+    if force or not os.path.exists(SO) or os.path.getmtime(SRC) > os.path.getmtime(SO):
+        subprocess.check_call(["gcc", "-O2", "-std=c11", "-fopenmp", "-ffp-contract=off", "-fPIC",
+                               "-shared", SRC, "-o", SO + ".tmp", "-lm"])
+        os.replace(SO + ".tmp", SO)
+    return SO
+
+
+class OrMat(ctypes.Structure):
+    _fields_ = [("dtype", ctypes.c_int), ("rows", ctypes.c_int64), ("cols", ctypes.c_int64),
+                ("data", ctypes.c_void_p), ("qs", ctypes.c_void_p), ("scales", ctypes.c_void_p)]
+
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        L = ctypes.CDLL(build())
+        i64, vp, dbl = ctypes.c_int64, ctypes.c_void_p, ctypes.c_double
+        L.or_bf16_to_f64.argtypes = [ctypes.c_uint16]
+        L.or_bf16_to_f64.restype = dbl
+        L.or_f16_to_f64.argtypes = [ctypes.c_uint16]
+        L.or_f16_to_f64.restype = dbl
+        L.or_round_bf16.argtypes = [dbl]
+        L.or_round_bf16.restype = dbl
+        L.or_mat_decode.argtypes = [ctypes.POINTER(OrMat), vp]
+        L.or_router_logit.argtypes = [vp, vp, i64]
+        L.or_router_logit.restype = ctypes.c_float
+        L.or_route.argtypes = [i64, i64, i64, i64, ctypes.c_int, vp, vp, vp, vp, vp, vp, vp]
+        L.or_route_from_logits.argtypes = [i64, i64, i64, ctypes.c_int, vp, vp, vp, vp]
+        L.or_aux_stats.argtypes = [i64, i64, i64, vp, vp, vp, vp, vp, vp]
+        L.or_capacity.argtypes = [i64, i64, i64, dbl]
+        L.or_capacity.restype = i64
+        L.or_permute.argtypes = [i64, i64, i64, i64, vp, vp, vp, vp, vp, vp, vp]
+        L.or_matvec.argtypes = [ctypes.POINTER(OrMat), vp, vp]
+        L.or_expert.argtypes = [ctypes.POINTER(OrMat)] * 3 + [vp, ctypes.c_int, dbl, dbl,
+                                                              ctypes.c_int, vp]
+        L.or_moe_tokens.argtypes = [i64, vp, vp, vp, vp, i64, vp, vp, vp, ctypes.c_int, dbl, dbl,
+                                    ctypes.c_int, vp, i64, vp]
+        L.or_moe_dense.argtypes = [i64, i64, i64, vp, vp, vp, vp, i64, vp, vp, ctypes.c_int, dbl,
+                                   dbl, ctypes.c_int, vp]
+        L.or_rmsnorm.argtypes = [i64, vp, dbl, vp]
+        L.or_ledger.argtypes = [i64, i64, i64, i64, vp, vp, vp, vp]
+        L.or_bandwidth_gain.argtypes = [i64, i64, i64]
+        L.or_bandwidth_gain.restype = dbl
+        for f in (L.or_mat_decode, L.or_route, L.or_route_from_logits, L.or_aux_stats,
+                  L.or_permute, L.or_matvec, L.or_expert, L.or_moe_tokens, L.or_moe_dense,
+                  L.or_rmsnorm, L.or_ledger):
+            f.restype = None
+        _lib = L
+    return _lib
+
+
+def _p(a):
+    return None if a is None else a.ctypes.data
+
+
+def _c(a, dt):
+    return np.ascontiguousarray(a, dtype=dt)
+
+
+# ------------------------------------------------------------------ matrices
+class Mat:
+    """A [rows][cols] matrix in f32 / bf16 / f16 / q4_0 storage (keeps arrays alive)."""
+
+    def __init__(self, dtype, rows, cols, data=None, qs=None, scales=None):
+        self.dtype, self.rows, self.cols = dtype, rows, cols
+        if dtype == F32:
+            self.data = _c(data, np.float32)
+        elif dtype in (BF16, F16):
+            self.data = _c(data, np.uint16)
+        else:
+            self.qs, self.scales, self.data = _c(qs, np.uint8), _c(scales, np.uint16), None
+        self.s = OrMat(dtype, rows, cols, _p(self.data),
+                       _p(getattr(self, "qs", None)) if dtype == Q4_0 else None,
+                       _p(getattr(self, "scales", None)) if dtype == Q4_0 else None)
+
+    def decode(self):
+        out = np.empty((self.rows, self.cols), dtype=np.float64)
+        lib().or_mat_decode(ctypes.byref(self.s), out.ctypes.data)
+        return out
+
+
+def mat_array(mats):
+    arr = (OrMat * len(mats))(*[m.s for m in mats])
+    return arr
+
+
+def bf16_to_f64(code: int) -> float:
+    return lib().or_bf16_to_f64(int(code))
+
+
+def f16_to_f64(code: int) -> float:
+    return lib().or_f16_to_f64(int(code))
+
+
+def round_bf16(x: float) -> float:
+    return lib().or_round_bf16(float(x))
+
+
+def decode(dtype, arr):
+    """Exact decode of an f32/bf16/f16 array to float64 (the oracle's own decoder)."""
+    arr = np.asarray(arr)
+    m = Mat(dtype, 1, arr.size, data=arr.reshape(-1))
+    return m.decode().reshape(arr.shape)
+
+
+def as_f32(dtype, arr):
+    """Exact conversion of an activation array to fp32 for the router dot products."""
+    return decode(dtype, arr).astype(np.float32)
+
+
+# -------------------------------------------------------------------- router
+def router_logit(w, u):
+    w, u = _c(w, np.float32), _c(u, np.float32)
+    return float(lib().or_router_logit(w.ctypes.data, u.ctypes.data, w.size))
+
+
+def route(u_f32, w_route, k, renorm=1, bias=None):
+    u_f32, w_route = _c(u_f32, np.float32), _c(w_route, np.float32)
+    T, d = u_f32.shape
+    N = w_route.shape[0]
+    bias = None if bias is None else _c(bias, np.float32)
+    logits = np.empty((T, N), np.float32)
+    probs = np.empty((T, N), np.float64)
+    idx = np.empty((T, k), np.int32)
+    w = np.empty((T, k), np.float64)
+    lib().or_route(T, d, N, k, renorm, u_f32.ctypes.data, w_route.ctypes.data, _p(bias),
+                   logits.ctypes.data, probs.ctypes.data, idx.ctypes.data, w.ctypes.data)
+    return logits, probs, idx, w
+
+
+def route_from_logits(logits, k, renorm=1):
+    logits = _c(logits, np.float32)
+    T, N = logits.shape
+    probs = np.empty((T, N), np.float64)
+    idx = np.empty((T, k), np.int32)
+    w = np.empty((T, k), np.float64)
+    lib().or_route_from_logits(T, N, k, renorm, logits.ctypes.data, probs.ctypes.data,
+                               idx.ctypes.data, w.ctypes.data)
+    return probs, idx, w
+
+
+def aux_stats(probs, idx):
+    probs, idx = _c(probs, np.float64), _c(idx, np.int32)
+    T, N = probs.shape
+    k = idx.shape[1]
+    f = np.empty(N, np.float64)
+    P = np.empty(N, np.float64)
+    nsum = np.empty(1, np.float64)
+    loads = np.empty(N, np.int32)
+    lib().or_aux_stats(T, N, k, probs.ctypes.data, idx.ctypes.data, f.ctypes.data, P.ctypes.data,
+                       nsum.ctypes.data, loads.ctypes.data)
+    return f, P, float(nsum[0]), loads
+
+
+def capacity(T, N, k, factor):
+    return int(lib().or_capacity(T, N, k, float(factor)))
+
+
+def permute(idx, N, C):
+    idx = _c(idx, np.int32)
+    T, k = idx.shape
+    counts = np.empty(N, np.int32)
+    offsets = np.empty(N + 1, np.int32)
+    perm_tok = np.full(T * k, -7, np.int32)
+    row_of = np.empty((T, k), np.int32)
+    overflow = np.empty(N, np.int32)
+    totals = np.empty(3, np.int64)
+    lib().or_permute(T, N, k, C, idx.ctypes.data, counts.ctypes.data, offsets.ctypes.data,
+                     perm_tok.ctypes.data, row_of.ctypes.data, overflow.ctypes.data,
+                     totals.ctypes.data)
+    return dict(counts=counts, offsets=offsets, perm_tok=perm_tok[: int(offsets[N])],
+                row_of=row_of, overflow=overflow, totals=totals)
+
+
+# -------------------------------------------------------------------- experts
+def matvec(W: Mat, x):
+    x = _c(x, np.float64)
+    y = np.empty(W.rows, np.float64)
+    lib().or_matvec(ctypes.byref(W.s), x.ctypes.data, y.ctypes.data)
+    return y
+
+
+def expert(Wg: Mat, Wu: Mat, Wd: Mat, u, act=0, beta_g=0.0, beta_u=0.0, round_h=0):
+    u = _c(u, np.float64)
+    out = np.empty(Wd.rows, np.float64)
+    lib().or_expert(ctypes.byref(Wg.s), ctypes.byref(Wu.s), ctypes.byref(Wd.s), u.ctypes.data,
+                    act, beta_g, beta_u, round_h, out.ctypes.data)
+    return out
+
+
+def moe_tokens(Wg, Wu, Wd, u, idx, top_w, row_of=None, tokens=None, act=0, beta_g=0.0,
+               beta_u=0.0, round_h=0):
+    """y_t = sum_kept a_{t,s} F_{idx}(u_t) for the listed tokens (all by default)."""
+    u = _c(u, np.float64)
+    idx, top_w = _c(idx, np.int32), _c(top_w, np.float64)
+    T, d_in = u.shape
+    k = idx.shape[1]
+    tokens = np.arange(T, dtype=np.int32) if tokens is None else _c(tokens, np.int32)
+    d_out = Wd[0].rows
+    y = np.empty((len(tokens), d_out), np.float64)
+    g, up, dn = mat_array(Wg), mat_array(Wu), mat_array(Wd)
+    row_of = None if row_of is None else _c(row_of, np.int32)
+    lib().or_moe_tokens(k, g, up, dn, u.ctypes.data, d_in, idx.ctypes.data, top_w.ctypes.data,
+                        _p(row_of), act, beta_g, beta_u, round_h, tokens.ctypes.data, len(tokens),
+                        y.ctypes.data)
+    return y
+
+
+def moe_dense(Wg, Wu, Wd, u, idx, top_w, act=0, beta_g=0.0, beta_u=0.0, round_h=0):
+    u = _c(u, np.float64)
+    idx, top_w = _c(idx, np.int32), _c(top_w, np.float64)
+    T, d_in = u.shape
+    k = idx.shape[1]
+    d_out = Wd[0].rows
+    y = np.empty((T, d_out), np.float64)
+    lib().or_moe_dense(T, len(Wg), k, mat_array(Wg), mat_array(Wu), mat_array(Wd), u.ctypes.data,
+                       d_in, idx.ctypes.data, top_w.ctypes.data, act, beta_g, beta_u, round_h,
+                       y.ctypes.data)
+    return y
+
+
+def rmsnorm(x, eps=1e-6):
+    x = _c(x, np.float64)
+    y = np.empty_like(x)
+    lib().or_rmsnorm(x.size, x.ctypes.data, eps, y.ctypes.data)
+    return y
+
+
+# -------------------------------------------------------------------- ledgers
+def ledger(d, h, N, k):
+    out = [np.zeros(1, np.int64) for _ in range(3)] + [np.zeros(1, np.float64)]
+    lib().or_ledger(d, h, N, k, *[o.ctypes.data for o in out])
+    return dict(one=int(out[0][0]), all=int(out[1][0]), active=int(out[2][0]),
+                bf16_gib=float(out[3][0]))
+
+
+def bandwidth_gain(ffn, top_k, ffn_e):
+    return float(lib().or_bandwidth_gain(ffn, top_k, ffn_e))

@@ -1,0 +1,401 @@
+/*
+ * CPU oracle for the sparse Mixture-of-Experts SwiGLU layer forward.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the tests, the smoke check and the CPU
+ * baseline leg of the benchmark may load this library.  The GPU product path
+ * never links, imports or calls it, and it shares no code with the GPU path.
+ *
+ * Sources, cited by page title and section:
+ *   [MoE tutorial]  "Mixture of Experts MoE: how sparse activation saves
+ *                   compute" (jefxiong.cn), §3.1-§3.8 and its appendix lab.
+ *   [MCU #13]       "Kestrel-MCU notes 13: the deployment gap between the
+ *                   converter and the inference kernel" (0539edu.com), §2, §4, §6.
+ *   [MCU #10]       "Kestrel-MCU notes 10: MoE sparsification in practice"
+ *                   (gsyq.cn), §3 (bandwidth gain table).
+ *   [LatentMoE]     "Stable LatentMoE interactive demo document" (cnblogs via
+ *                   82so.com): width separation, RMSNorm before up-projection,
+ *                   SiTU-GLU soft caps.
+ *
+ * Precision: every floating-point quantity is evaluated in double from the
+ * exact input values, except the router logits.  The tutorial's router works
+ * in fp32 (§3.2 and its code: softmax of logits.float()); the logits decide
+ * the discrete top-k, so they are formed in fp32 in one fixed summation order
+ * (or_router_logit below) which any implementation can reproduce bit for bit.
+ * Compiled with -ffp-contract=off so each operation rounds on its own.
+ *
+ * Parity pins: every function is checked against worked numbers printed on
+ * the pages, closed forms, brute force or textbook identities in
+ * tests/test_oracle_pins.py.  The softmax/SiLU/tanh transcendental values
+ * themselves have no printed example beyond the tutorial's aux-loss figures.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* ------------------------------------------------------------------ formats */
+
+/* bf16 bit pattern -> exact double (the upper half of an IEEE binary32). */
+double or_bf16_to_f64(uint16_t b) {
+  uint32_t u = (uint32_t)b << 16;
+  float f;
+  memcpy(&f, &u, 4);
+  return (double)f;
+}
+
+/* IEEE binary16 bit pattern -> exact double, decoded field by field.
+ * Subnormals are mantissa * 2^-24 (exponent field 0 means 2^(1-15) with no
+ * implicit bit).  [MCU #13] §6 reports a hand-written decoder whose subnormal
+ * branch was off by one in the exponent and halved 14.2% of the q4 scales. */
+double or_f16_to_f64(uint16_t h) {
+  int sign = (h >> 15) & 1;
+  int ex = (h >> 10) & 0x1F;
+  int man = h & 0x3FF;
+  double v;
+  if (ex == 0) {
+    v = ldexp((double)man, -24);
+  } else if (ex == 31) {
+    v = man ? NAN : INFINITY;
+  } else {
+    v = ldexp((double)(man | 0x400), ex - 25);
+  }
+  return sign ? -v : v;
+}
+
+/* Storage of an activation or weight tensor. */
+enum { OR_F32 = 0, OR_BF16 = 1, OR_F16 = 2, OR_Q4_0 = 3 };
+
+/* One [rows][cols] matrix in any storage type.  q4_0 (format named in
+ * [MCU #13] §4): blocks of 32 consecutive values along a row, one fp16 scale
+ * s per block, 4-bit codes q in 0..15, value (q - 8) * s; byte j (0..15) of a
+ * block holds element j in its low nibble and element j + 16 in its high
+ * nibble. */
+typedef struct {
+  int dtype;
+  int64_t rows, cols;
+  const void* data;       /* f32 / bf16 / f16 */
+  const uint8_t* qs;      /* q4_0: [rows][cols/2] */
+  const uint16_t* scales; /* q4_0: [rows][cols/32] fp16 codes */
+} or_mat;
+
+static inline double mat_get(const or_mat* m, int64_t r, int64_t c) {
+  switch (m->dtype) {
+    case OR_F32: return (double)((const float*)m->data)[r * m->cols + c];
+    case OR_BF16: return or_bf16_to_f64(((const uint16_t*)m->data)[r * m->cols + c]);
+    case OR_F16: return or_f16_to_f64(((const uint16_t*)m->data)[r * m->cols + c]);
+    default: {
+      int64_t b = c / 32, j = c % 32;
+      uint8_t byte = m->qs[r * (m->cols / 2) + b * 16 + (j & 15)];
+      int q = (j < 16) ? (byte & 0xF) : (byte >> 4);
+      return (double)(q - 8) * or_f16_to_f64(m->scales[r * (m->cols / 32) + b]);
+    }
+  }
+}
+
+/* Decode a whole matrix (or vector) to double. */
+void or_mat_decode(const or_mat* m, double* out) {
+  for (int64_t r = 0; r < m->rows; ++r)
+    for (int64_t c = 0; c < m->cols; ++c) out[r * m->cols + c] = mat_get(m, r, c);
+}
+
+/* Round a double to the nearest bf16 value through fp32 (the storage a GPU
+ * kernel uses for an intermediate it writes as bf16), returned as double. */
+double or_round_bf16(double x) {
+  float f = (float)x;
+  uint32_t u;
+  memcpy(&u, &f, 4);
+  u += 0x7FFFu + ((u >> 16) & 1u);
+  u &= 0xFFFF0000u;
+  memcpy(&f, &u, 4);
+  return (double)f;
+}
+
+/* ------------------------------------------------------------------- router */
+
+/* Router logit z = (W_route u)_i  [MoE tutorial] §3.2, formed in fp32.
+ * Fixed order: the d inputs are cut into chunks of 8 consecutive elements;
+ * chunk c belongs to partial sum c mod 32; each partial is a sequential
+ * single-rounding fused multiply-add chain from +0 over its chunks in
+ * ascending order; the 32 partials are then added pairwise at distance 16,
+ * 8, 4, 2, 1 (partial p + partial p+16 first).  d must be a multiple of 8. */
+float or_router_logit(const float* w, const float* u, int64_t d) {
+  float part[32];
+  for (int l = 0; l < 32; ++l) part[l] = 0.0f;
+  for (int64_t c = 0; c < d / 8; ++c) {
+    int l = (int)(c % 32);
+    for (int j = 0; j < 8; ++j) part[l] = fmaf(w[c * 8 + j], u[c * 8 + j], part[l]);
+  }
+  for (int dist = 16; dist >= 1; dist /= 2)
+    for (int l = 0; l < dist; ++l) part[l] = part[l] + part[l + dist];
+  return part[0];
+}
+
+/* Routing of T tokens  [MoE tutorial] §3.2:
+ *   z_{t,i} = (W_route u_t)_i (+ b_i),  p = softmax(z),
+ *   S_t = the k experts with the largest z (ties: lower expert index),
+ *   a_{t,i} = p_{t,i} / sum_{j in S_t} p_{t,j}  (renorm = 1, Mixtral style) or
+ *   a_{t,i} = p_{t,i} (renorm = 0, the top-1 Switch multiplier of §3.2).
+ * Selection by z equals selection by p (softmax is monotone) without the ties
+ * that rounding p could introduce.  Outputs: logits [T][N] fp32, probs and
+ * top_w in double, top_idx [T][k] ordered by descending z. */
+void or_route(int64_t T, int64_t d, int64_t N, int64_t k, int renorm, const float* u,
+              const float* w_route, const float* bias, float* logits, double* probs,
+              int32_t* top_idx, double* top_w) {
+#pragma omp parallel for schedule(dynamic, 16)
+  for (int64_t t = 0; t < T; ++t) {
+    float* z = logits + t * N;
+    for (int64_t i = 0; i < N; ++i) {
+      z[i] = or_router_logit(w_route + i * d, u + t * d, d);
+      if (bias) z[i] = z[i] + bias[i];
+    }
+    double zmax = -INFINITY;
+    for (int64_t i = 0; i < N; ++i) zmax = fmax(zmax, (double)z[i]);
+    double den = 0.0;
+    for (int64_t i = 0; i < N; ++i) den += exp((double)z[i] - zmax);
+    double* p = probs + t * N;
+    for (int64_t i = 0; i < N; ++i) p[i] = exp((double)z[i] - zmax) / den;
+    /* top-k by repeated selection of the best remaining (z desc, index asc) */
+    int32_t* sel = top_idx + t * k;
+    for (int64_t s = 0; s < k; ++s) {
+      int64_t best = -1;
+      for (int64_t i = 0; i < N; ++i) {
+        int taken = 0;
+        for (int64_t q = 0; q < s; ++q) taken |= (sel[q] == i);
+        if (taken) continue;
+        if (best < 0 || z[i] > z[best]) best = i;
+      }
+      sel[s] = (int32_t)best;
+    }
+    double ssum = 0.0;
+    for (int64_t s = 0; s < k; ++s) ssum += p[sel[s]];
+    for (int64_t s = 0; s < k; ++s) top_w[t * k + s] = renorm ? p[sel[s]] / ssum : p[sel[s]];
+  }
+}
+
+/* The same routing from given logits (the tutorial's controlled-logit
+ * experiments feed logits directly).  No fp32 dot product involved. */
+void or_route_from_logits(int64_t T, int64_t N, int64_t k, int renorm, const float* logits,
+                          double* probs, int32_t* top_idx, double* top_w) {
+  for (int64_t t = 0; t < T; ++t) {
+    const float* z = logits + t * N;
+    double zmax = -INFINITY, den = 0.0;
+    for (int64_t i = 0; i < N; ++i) zmax = fmax(zmax, (double)z[i]);
+    for (int64_t i = 0; i < N; ++i) den += exp((double)z[i] - zmax);
+    for (int64_t i = 0; i < N; ++i) probs[t * N + i] = exp((double)z[i] - zmax) / den;
+    int32_t* sel = top_idx + t * k;
+    for (int64_t s = 0; s < k; ++s) {
+      int64_t best = -1;
+      for (int64_t i = 0; i < N; ++i) {
+        int taken = 0;
+        for (int64_t q = 0; q < s; ++q) taken |= (sel[q] == i);
+        if (!taken && (best < 0 || z[i] > z[best])) best = i;
+      }
+      sel[s] = (int32_t)best;
+    }
+    double ssum = 0.0;
+    for (int64_t s = 0; s < k; ++s) ssum += probs[t * N + sel[s]];
+    for (int64_t s = 0; s < k; ++s)
+      top_w[t * k + s] = renorm ? probs[t * N + sel[s]] / ssum : probs[t * N + sel[s]];
+  }
+}
+
+/* --------------------------------------------------------------- aux stats */
+
+/* Switch balancing statistics  [MoE tutorial] §3.4:
+ *   f_i = (1/T) #{t : argmax_j p_{t,j} = i}   (argmax = slot 0 of the top-k)
+ *   P_i = (1/T) sum_t p_{t,i}
+ *   n_sum_fP = N * sum_i f_i P_i               (L_aux without alpha)
+ * plus the dispatch loads L_i = #{(t,s) : top_idx[t][s] = i}  (§3.6). */
+void or_aux_stats(int64_t T, int64_t N, int64_t k, const double* probs, const int32_t* top_idx,
+                  double* f, double* P, double* n_sum_fP, int32_t* loads) {
+  for (int64_t i = 0; i < N; ++i) {
+    f[i] = 0.0;
+    P[i] = 0.0;
+    loads[i] = 0;
+  }
+  for (int64_t t = 0; t < T; ++t) {
+    f[top_idx[t * k]] += 1.0;
+    for (int64_t s = 0; s < k; ++s) loads[top_idx[t * k + s]] += 1;
+    for (int64_t i = 0; i < N; ++i) P[i] += probs[t * N + i];
+  }
+  double acc = 0.0;
+  for (int64_t i = 0; i < N; ++i) {
+    f[i] /= (double)T;
+    P[i] /= (double)T;
+    acc += f[i] * P[i];
+  }
+  *n_sum_fP = (double)N * acc;
+}
+
+/* -------------------------------------------------------- capacity, permute */
+
+/* Expert capacity C = ceil(c * T / N)  [MoE tutorial] §3.5, with T counted as
+ * dispatches (k * T) for top-k as §3.5 requires. */
+int64_t or_capacity(int64_t T, int64_t N, int64_t k, double factor) {
+  return (int64_t)ceil(factor * (double)(k * T) / (double)N);
+}
+
+/* Group dispatches by expert  [MoE tutorial] §3.5, §3.6, §3.8.
+ * Dispatch (t, s) goes to expert top_idx[t][s].  Its rank is the number of
+ * dispatches to the same expert from lower token indices.  It is kept when
+ * C == 0 (unlimited) or rank < C; a dropped dispatch skips the expert
+ * (the residual path carries the token).  Grouped row of a kept dispatch:
+ * offsets[e] + rank, where offsets is the exclusive prefix sum of the kept
+ * counts.  Outputs:
+ *   counts[e]   = L_e (all dispatches, kept or not)
+ *   offsets[N+1]
+ *   perm_tok[r] = token of grouped row r   (r < offsets[N])
+ *   row_of[t][s] = grouped row, or -1 if dropped
+ *   overflow[e] = max(L_e - C, 0)
+ *   totals = {kept, sum overflow, sum empty slots max(C - L_e, 0)} */
+void or_permute(int64_t T, int64_t N, int64_t k, int64_t C, const int32_t* top_idx,
+                int32_t* counts, int32_t* offsets, int32_t* perm_tok, int32_t* row_of,
+                int32_t* overflow, int64_t* totals) {
+  int64_t* seen = (int64_t*)calloc((size_t)N, sizeof(int64_t));
+  for (int64_t e = 0; e < N; ++e) counts[e] = 0;
+  for (int64_t x = 0; x < T * k; ++x) counts[top_idx[x]] += 1;
+  int64_t run = 0, of = 0, empty = 0;
+  for (int64_t e = 0; e < N; ++e) {
+    offsets[e] = (int32_t)run;
+    int64_t kept = (C > 0 && counts[e] > C) ? C : counts[e];
+    run += kept;
+    overflow[e] = (int32_t)((C > 0 && counts[e] > C) ? counts[e] - C : 0);
+    of += overflow[e];
+    empty += (C > 0 && counts[e] < C) ? C - counts[e] : 0;
+  }
+  offsets[N] = (int32_t)run;
+  for (int64_t t = 0; t < T; ++t) {
+    for (int64_t s = 0; s < k; ++s) {
+      int32_t e = top_idx[t * k + s];
+      int64_t rank = seen[e]++;
+      if (C > 0 && rank >= C) {
+        row_of[t * k + s] = -1;
+      } else {
+        int64_t r = offsets[e] + rank;
+        row_of[t * k + s] = (int32_t)r;
+        perm_tok[r] = (int32_t)t;
+      }
+    }
+  }
+  totals[0] = run;
+  totals[1] = of;
+  totals[2] = empty;
+  free(seen);
+}
+
+/* ------------------------------------------------------------ expert FFN */
+
+/* y = W x for one [rows][cols] matrix, in double. */
+void or_matvec(const or_mat* W, const double* x, double* y) {
+  for (int64_t r = 0; r < W->rows; ++r) {
+    double acc = 0.0;
+    for (int64_t c = 0; c < W->cols; ++c) acc += mat_get(W, r, c) * x[c];
+    y[r] = acc;
+  }
+}
+
+static inline double silu(double g) { return g / (1.0 + exp(-g)); }
+
+/* One expert F(u) = W_down (SiLU(W_gate u) (*) W_up u)  [MoE tutorial] §3.1.
+ * act = 1 applies the SiTU-GLU soft caps of [LatentMoE]: the gate and up
+ * pre-activations become beta_g tanh(g / beta_g) and beta_u tanh(u / beta_u)
+ * before SiLU and the product.  round_h = 1 rounds the hidden vector to bf16
+ * (the storage of the intermediate in the bf16 layers).  W_gate, W_up:
+ * [h][d_in]; W_down: [d_out][h]. */
+void or_expert(const or_mat* Wg, const or_mat* Wu, const or_mat* Wd, const double* u, int act,
+               double beta_g, double beta_u, int round_h, double* out) {
+  int64_t h = Wg->rows;
+  double* g = (double*)malloc(sizeof(double) * (size_t)h);
+  double* v = (double*)malloc(sizeof(double) * (size_t)h);
+  or_matvec(Wg, u, g);
+  or_matvec(Wu, u, v);
+  for (int64_t i = 0; i < h; ++i) {
+    double gi = g[i], ui = v[i];
+    if (act == 1) {
+      gi = beta_g * tanh(gi / beta_g);
+      ui = beta_u * tanh(ui / beta_u);
+    }
+    double hi = silu(gi) * ui;
+    g[i] = round_h ? or_round_bf16(hi) : hi;
+  }
+  or_matvec(Wd, g, out);
+  free(g);
+  free(v);
+}
+
+/* Token outputs of the sparse layer  [MoE tutorial] §3.2:
+ *   y_t = sum over kept dispatches s of a_{t,s} F_{top_idx[t][s]}(u_t);
+ * a dropped dispatch (row_of = -1) contributes nothing and the remaining
+ * weights are not renormalised.  Experts are [N] arrays of matrices.  Only
+ * the n_sel tokens listed in tokens[] are evaluated (all of them when the
+ * caller lists every token).  u is [T][d_in] in double. */
+void or_moe_tokens(int64_t k, const or_mat* Wg, const or_mat* Wu, const or_mat* Wd,
+                   const double* u, int64_t d_in, const int32_t* top_idx, const double* top_w,
+                   const int32_t* row_of, int act, double beta_g, double beta_u, int round_h,
+                   const int32_t* tokens, int64_t n_sel, double* y) {
+  int64_t d_out = Wd[0].rows;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int64_t q = 0; q < n_sel; ++q) {
+    int64_t t = tokens[q];
+    double* acc = y + q * d_out;
+    double* tmp = (double*)malloc(sizeof(double) * (size_t)d_out);
+    for (int64_t m = 0; m < d_out; ++m) acc[m] = 0.0;
+    for (int64_t s = 0; s < k; ++s) {
+      if (row_of && row_of[t * k + s] < 0) continue;
+      int32_t e = top_idx[t * k + s];
+      or_expert(&Wg[e], &Wu[e], &Wd[e], u + t * d_in, act, beta_g, beta_u, round_h, tmp);
+      for (int64_t m = 0; m < d_out; ++m) acc[m] += top_w[t * k + s] * tmp[m];
+    }
+    free(tmp);
+  }
+}
+
+/* Dense brute-force reference  [MoE tutorial] appendix lab: every expert is
+ * evaluated for every token and multiplied by its combine weight, which is
+ * zero for the unselected experts.  Must equal or_moe_tokens exactly when
+ * nothing is dropped. */
+void or_moe_dense(int64_t T, int64_t N, int64_t k, const or_mat* Wg, const or_mat* Wu,
+                  const or_mat* Wd, const double* u, int64_t d_in, const int32_t* top_idx,
+                  const double* top_w, int act, double beta_g, double beta_u, int round_h,
+                  double* y) {
+  int64_t d_out = Wd[0].rows;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int64_t t = 0; t < T; ++t) {
+    double* tmp = (double*)malloc(sizeof(double) * (size_t)d_out);
+    for (int64_t m = 0; m < d_out; ++m) y[t * d_out + m] = 0.0;
+    for (int64_t e = 0; e < N; ++e) {
+      double w = 0.0;
+      for (int64_t s = 0; s < k; ++s)
+        if (top_idx[t * k + s] == e) w += top_w[t * k + s];
+      or_expert(&Wg[e], &Wu[e], &Wd[e], u + t * d_in, act, beta_g, beta_u, round_h, tmp);
+      for (int64_t m = 0; m < d_out; ++m) y[t * d_out + m] += w * tmp[m];
+    }
+    free(tmp);
+  }
+}
+
+/* RMSNorm without gain  [LatentMoE]: x / sqrt(mean(x^2) + eps). */
+void or_rmsnorm(int64_t n, const double* x, double eps, double* y) {
+  double ss = 0.0;
+  for (int64_t i = 0; i < n; ++i) ss += x[i] * x[i];
+  double r = sqrt(ss / (double)n + eps);
+  for (int64_t i = 0; i < n; ++i) y[i] = x[i] / r;
+}
+
+/* ------------------------------------------------------------------ ledgers */
+
+/* Expert parameter ledger  [MoE tutorial] §3.3 and §01:
+ * one SwiGLU expert has 3dh weights; N experts 3dhN; k active 3dhk. */
+void or_ledger(int64_t d, int64_t h, int64_t N, int64_t k, int64_t* one, int64_t* all,
+               int64_t* active, double* bf16_gib) {
+  *one = 3 * d * h;
+  *all = N * *one;
+  *active = k * *one;
+  *bf16_gib = (double)(*all) * 2.0 / 1073741824.0;
+}
+
+/* Expert-weight bandwidth gain of top-k lookup-loading  [MCU #10] §3 table,
+ * [MCU #13] §2: dense FFN width over the k selected expert widths. */
+double or_bandwidth_gain(int64_t ffn, int64_t top_k, int64_t ffn_e) {
+  return (double)ffn / (double)(top_k * ffn_e);
+}
