@@ -113,21 +113,13 @@ double or_round_bf16(double x) {
 /* ------------------------------------------------------------------- router */
 
 /* Router logit z = (W_route u)_i  [MoE tutorial] §3.2, formed in fp32.
- * Fixed order: the d inputs are cut into chunks of 8 consecutive elements;
- * chunk c belongs to partial sum c mod 32; each partial is a sequential
- * single-rounding fused multiply-add chain from +0 over its chunks in
- * ascending order; the 32 partials are then added pairwise at distance 16,
- * 8, 4, 2, 1 (partial p + partial p+16 first).  d must be a multiple of 8. */
+ * The page fixes fp32 but not the summation order; the order used is the
+ * plainest one: a single sequential chain of fused multiply-adds (one
+ * rounding each) over j = 0 .. d-1 in ascending order, starting from +0. */
 float or_router_logit(const float* w, const float* u, int64_t d) {
-  float part[32];
-  for (int l = 0; l < 32; ++l) part[l] = 0.0f;
-  for (int64_t c = 0; c < d / 8; ++c) {
-    int l = (int)(c % 32);
-    for (int j = 0; j < 8; ++j) part[l] = fmaf(w[c * 8 + j], u[c * 8 + j], part[l]);
-  }
-  for (int dist = 16; dist >= 1; dist /= 2)
-    for (int l = 0; l < dist; ++l) part[l] = part[l] + part[l + dist];
-  return part[0];
+  float acc = 0.0f;
+  for (int64_t j = 0; j < d; ++j) acc = fmaf(w[j], u[j], acc);
+  return acc;
 }
 
 /* Routing of T tokens  [MoE tutorial] §3.2:

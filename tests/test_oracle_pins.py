@@ -68,12 +68,13 @@ def _exact_dot(w, u):
 
 
 def test_router_logit_within_fp32_bound():
+    """Sequential fp32 summation error bound: |z - exact| <= d * u * sum|w u| (u = 2^-24)."""
     for d in (8, 64, 512, 4096):
         w = RNG.standard_normal(d).astype(np.float32)
         u = RNG.standard_normal(d).astype(np.float32)
         z = O.router_logit(w, u)
         exact = _exact_dot(w, u)
-        bound = (d / 32 * 8 + 5 + 1) * 2.0 ** -24 * float(np.sum(np.abs(w.astype(np.float64) * u)))
+        bound = (d + 1) * 2.0 ** -24 * float(np.sum(np.abs(w.astype(np.float64) * u)))
         assert abs(z - exact) <= bound
 
 
@@ -84,23 +85,21 @@ def test_router_logit_integer_inputs_exact():
 
 
 def test_router_logit_documented_order():
-    """Hand-worked values that only the documented order produces.
+    """Hand-worked values that only an ascending sequential sum produces.
 
-    d = 256: chunk c of 8 elements feeds partial c mod 32; partials are added
-    at distance 16 first.  +2^25 in chunk 0, +1 in chunk 1, -2^25 in chunk 16:
-    the tree gives (2^25 - 2^25) + 1 = 1, a left-to-right sum gives 0.
+    [2^25, -2^25, 1]: ascending gives (2^25 - 2^25) + 1 = 1; descending gives
+    (1 - 2^25) -> -2^25 (ulp 4) then + 2^25 = 0.
+    [2^25, 1, -2^25] spread over the positions 0, 8, 128 of d = 256: ascending
+    gives 2^25 + 1 -> 2^25 then 0; a pairwise tree over 8-element chunks
+    would cancel the two big terms first and give 1.
     """
+    w = np.ones(3, np.float32)
+    assert O.router_logit(w, np.array([2.0 ** 25, -(2.0 ** 25), 1.0], np.float32)) == 1.0
+    assert O.router_logit(w, np.array([1.0, -(2.0 ** 25), 2.0 ** 25], np.float32)) == 1.0 - 1.0
     d = 256
     w = np.ones(d, np.float32)
     u = np.zeros(d, np.float32)
     u[0], u[8], u[128] = 2.0 ** 25, 1.0, -(2.0 ** 25)
-    assert O.router_logit(w, u) == 1.0
-    # d = 512: chunk 32 shares partial 0 with chunk 0 and is added sequentially
-    # before the tree: 2^25 + 1 rounds to 2^25, then the tree cancels -> 0.
-    d = 512
-    w = np.ones(d, np.float32)
-    u = np.zeros(d, np.float32)
-    u[0], u[256], u[128] = 2.0 ** 25, 1.0, -(2.0 ** 25)
     assert O.router_logit(w, u) == 0.0
 
 
