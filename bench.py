@@ -1,0 +1,423 @@
+"""Benchmark of the sparse-MoE layer forward on B200 (tokens/s).
+
+One step = one full pass of the layer (router -> permutation -> gather ->
+grouped tcgen05 SwiGLU experts -> weighted combine) over one batch of seeded
+synthetic tokens already resident in HBM.  Default workload: the small-model
+layer (T=4096, d=512, N=8 experts, h=128, top-2, bf16).  Other workloads:
+--workload mixtral | tiny.
+
+Prints ONE JSON line (rank 0).  With torchrun (N > 1) every rank runs its own
+replica of the workload (the layer needs no collective: "replicas only",
+weak scaling) and the time is the max over ranks.
+--impl reference times the CPU oracle (the reference arm) on a bounded sample.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import synthetic as S  # noqa: E402
+from synthetic import workloads as W  # noqa: E402
+
+METRIC = "MoE-layer fwd tokens/s on 1 B200"
+L2_BYTES = 126 * 1024 * 1024
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return (float(d["hbm_gbs"]), float(d["bf16_tflops"]), float(d["bf16_tflops_sustained"]),
+                "measured")
+    return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+# --------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.out = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"], stdout=self.out,
+                stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.out.flush()
+        rows = []
+        with open(self.out.name) as f:
+            for ln in f:
+                parts = [x.strip() for x in ln.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.out.name)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": float(rows[0][2]) if rows[0][2].replace(".", "").isdigit() else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ------------------------------------------------------------ workload setup
+class Replica:
+    """Device inputs and weights of one copy of the workload."""
+
+    def __init__(self, wl: W.Workload, seed: int, torch):
+        self.wl = wl
+        st = torch.cuda.current_stream().cuda_stream
+        T, d, N, h = wl.T, wl.d, wl.N, wl.h
+        tdt = {S.DT_F32: torch.float32, S.DT_BF16: torch.bfloat16, S.DT_F16: torch.float16}
+        adt = tdt[wl.act_dtype]
+        wdt = tdt[W.w_storage(wl)]
+        self.u = torch.empty((T, d), dtype=adt, device="cuda")
+        if wl.rms_inputs:
+            S.rmsnorm_rows_dev(seed, W.TID_U, T, d, wl.act_dtype, self.u.data_ptr(), st)
+        else:
+            S.normal_dev(seed, W.TID_U, T * d, wl.u_sigma, wl.act_dtype, self.u.data_ptr(), st)
+        self.w_route = torch.empty((N, d), dtype=torch.float32, device="cuda")
+        S.normal_dev(seed, W.TID_WROUTE, N * d, W.SIGMA_W, S.DT_F32, self.w_route.data_ptr(), st)
+        b = wl.router_bias()
+        self.bias = None if b is None else torch.from_numpy(b).cuda()
+        self.w = []
+        for tid, shp in ((W.TID_WGATE, (N, h, d)), (W.TID_WUP, (N, h, d)),
+                         (W.TID_WDOWN, (N, d, h))):
+            t = torch.empty(shp, dtype=wdt, device="cuda")
+            S.normal_dev(seed, tid, t.numel(), W.SIGMA_W, W.w_storage(wl), t.data_ptr(), st)
+            self.w.append(t)
+
+    def nbytes(self):
+        return sum(t.numel() * t.element_size() for t in [self.u, self.w_route, *self.w])
+
+
+class Step:
+    """The layer step through the C ABI, split at the expert FFN so that the
+    tcgen05 GEMM launches can be timed on their own stream position."""
+
+    def __init__(self, wl: W.Workload, torch, moe):
+        self.wl, self.torch, self.moe = wl, torch, moe
+        T, d, N, k, h = wl.T, wl.d, wl.N, wl.k, wl.h
+        self.s = moe.shape(T, d, N, k, h, wl.renorm, wl.capacity())
+        i32 = dict(dtype=torch.int32, device="cuda")
+        adt = {S.DT_F32: torch.float32, S.DT_BF16: torch.bfloat16}[wl.act_dtype]
+        self.top_idx = torch.empty((T, k), **i32)
+        self.top_w = torch.empty((T, k), dtype=torch.float32, device="cuda")
+        self.logits = torch.empty((T, N), dtype=torch.float32, device="cuda")
+        self.counts = torch.empty(N, **i32)
+        self.offsets = torch.empty(N + 1, **i32)
+        self.perm = torch.empty(T * k, **i32)
+        self.row_of = torch.empty((T, k), **i32)
+        self.overflow = torch.empty(N, **i32)
+        self.totals = torch.empty(3, **i32)
+        self.x_rows = torch.empty((T * k, d), dtype=adt, device="cuda")
+        self.y_rows = torch.empty((T * k, d), dtype=torch.float32, device="cuda")
+        self.y = torch.empty((T, d), dtype=adt, device="cuda")
+        lib = moe._lib
+        import ctypes
+        pb = lib.moe_permute_workspace_bytes(ctypes.byref(self.s))
+        fb = lib.moe_expert_ffn_workspace_bytes(ctypes.byref(self.s), d, wl.act_dtype)
+        self.ws_perm = torch.empty(max(pb, 256), dtype=torch.uint8, device="cuda")
+        self.ws_ffn = torch.empty(max(fb, 256), dtype=torch.uint8, device="cuda")
+        self.act = moe.act()
+        self.launches_per_step = 2 + 3 + 1 + 2 + 1  # route, permute, gather, ffn, combine
+
+    def __call__(self, r: Replica, ev_ffn=None):
+        m = self.moe
+        m.moe_route(self.s, r.u, r.w_route, self.top_idx, self.top_w, bias=r.bias,
+                    logits=self.logits)
+        m.moe_permute(self.s, self.top_idx, self.counts, self.offsets, self.perm, self.row_of,
+                      self.overflow, self.totals, ws=self.ws_perm)
+        m.moe_gather(self.s, self.wl.d, r.u, self.perm, self.offsets, self.x_rows)
+        if ev_ffn:
+            ev_ffn[0].record()
+        m.moe_expert_ffn(self.s, self.wl.d, self.x_rows, self.offsets, *r.w, self.y_rows,
+                         self.act, ws=self.ws_ffn)
+        if ev_ffn:
+            ev_ffn[1].record()
+        m.moe_combine(self.s, self.wl.d, self.y_rows, self.row_of, self.top_w, self.y)
+
+
+def _algorithmic(wl: W.Workload, kept_rows: int):
+    """Algorithmic FLOPs and HBM bytes of one step (bf16 weights and activations)."""
+    el = 2 if wl.act_dtype != S.DT_F32 else 4
+    flops_router = 2.0 * wl.T * wl.N * wl.d
+    flops_experts = 6.0 * wl.d * wl.h * kept_rows
+    w_bytes = 3.0 * wl.N * wl.d * wl.h * el
+    act_bytes = 2.0 * wl.T * wl.d * el + wl.N * wl.d * 4
+    return flops_router, flops_experts, w_bytes, act_bytes
+
+
+# --------------------------------------------------------------- oracle legs
+def oracle_pass(wl: W.Workload, host, tokens):
+    """The oracle on the listed tokens (routing of all tokens when a capacity
+    makes drops depend on the whole batch)."""
+    import oracle as O
+    od = {S.DT_F32: O.F32, S.DT_BF16: O.BF16, S.DT_F16: O.F16}[wl.act_dtype]
+    u_codes, w_route, bias, mats = host
+    if wl.capacity():
+        route_rows = np.arange(wl.T)
+    else:
+        route_rows = tokens
+    _, _, idx, tw = O.route(O.as_f32(od, u_codes[route_rows]), w_route, wl.k, wl.renorm, bias)
+    C = wl.capacity()
+    perm = O.permute(idx, wl.N, C)
+    sel = tokens if wl.capacity() else np.arange(len(tokens))
+    O.moe_tokens([m[0] for m in mats], [m[1] for m in mats], [m[2] for m in mats],
+                 O.decode(od, u_codes[tokens]), idx[sel], tw[sel], row_of=perm["row_of"][sel],
+                 tokens=np.arange(len(tokens), dtype=np.int32),
+                 round_h=int(wl.act_dtype == S.DT_BF16))
+
+
+def oracle_host_inputs(wl: W.Workload):
+    import oracle as O
+    dt = W.w_storage(wl)
+    od = {S.DT_F32: O.F32, S.DT_BF16: O.BF16}[dt]
+    u = (S.rmsnorm_rows(wl.seed, W.TID_U, wl.T, wl.d, wl.act_dtype) if wl.rms_inputs
+         else S.normal(wl.seed, W.TID_U, (wl.T, wl.d), wl.u_sigma, wl.act_dtype))
+    w_route = S.normal(wl.seed, W.TID_WROUTE, (wl.N, wl.d), W.SIGMA_W, S.DT_F32)
+    mats = []
+    for e in range(wl.N):
+        g = S.normal(wl.seed, W.TID_WGATE, (wl.h, wl.d), W.SIGMA_W, dt, offset=e * wl.h * wl.d)
+        up = S.normal(wl.seed, W.TID_WUP, (wl.h, wl.d), W.SIGMA_W, dt, offset=e * wl.h * wl.d)
+        dn = S.normal(wl.seed, W.TID_WDOWN, (wl.d, wl.h), W.SIGMA_W, dt, offset=e * wl.d * wl.h)
+        mats.append((O.Mat(od, wl.h, wl.d, data=g), O.Mat(od, wl.h, wl.d, data=up),
+                     O.Mat(od, wl.d, wl.h, data=dn)))
+    return u, w_route, wl.router_bias(), mats
+
+
+def cpu_sample_tokens(wl: W.Workload) -> int:
+    """Tokens per oracle sample: about 10 s of host work on 8 cores."""
+    per_token = 6.0 * wl.d * wl.h * wl.k
+    return int(max(16, min(wl.T, 2.0e10 / per_token)))
+
+
+def run_cpu_baseline(wl: W.Workload, host, budget_s: float = 12.0):
+    n = cpu_sample_tokens(wl)
+    rng = np.random.default_rng(0)
+    done, t0 = 0, time.perf_counter()
+    while True:
+        tokens = np.sort(rng.choice(wl.T, n, replace=False)).astype(np.int32)
+        oracle_pass(wl, host, tokens)
+        done += n
+        el = time.perf_counter() - t0
+        if el >= budget_s:
+            break
+    return done / el, el, n
+
+
+def reference_arm(args, wl):
+    """--impl reference: the CPU oracle timed on this machine's host cores."""
+    host = oracle_host_inputs(wl)
+    n = cpu_sample_tokens(wl) // 4 or 1
+    rng = np.random.default_rng(1)
+    samples = [np.sort(rng.choice(wl.T, n, replace=False)).astype(np.int32)
+               for _ in range(args.warmup + args.steps)]
+    for i in range(args.warmup):
+        oracle_pass(wl, host, samples[i])
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        oracle_pass(wl, host, samples[args.warmup + i])
+    el = time.perf_counter() - t0
+    value = n * args.steps / el
+    cores = os.cpu_count()
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": el / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": wl.name, "T": wl.T, "d": wl.d, "N": wl.N, "k": wl.k,
+                       "h": wl.h},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores,
+                             "kind": "oracle",
+                             "sample": f"{n} random tokens of the {wl.name} batch per step"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------- main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="small", choices=["small", "mixtral", "tiny"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    wl = W.ALL[args.workload]()
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            reference_arm(args, wl)
+        return
+
+    import torch
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    import sparse_mixture_experts_15_b200 as moe
+
+    # replicas rotate so that the inputs of consecutive steps exceed L2
+    one = Replica(wl, wl.seed + 7919 * rank, torch)
+    n_rep = max(1, min(64, -(-2 * L2_BYTES // max(one.nbytes(), 1))))
+    reps = [one] + [Replica(wl, wl.seed + 7919 * (rank + world * i), torch)
+                    for i in range(1, n_rep)]
+    step = Step(wl, torch, moe)
+    stream = torch.cuda.current_stream()
+
+    for i in range(args.warmup):
+        step(reps[i % n_rep])
+    torch.cuda.synchronize()
+    kept = [0] * n_rep
+    for i in range(n_rep):
+        step(reps[i])
+        torch.cuda.synchronize()
+        kept[i] = int(step.totals[0].item())
+    assert moe.moe_device_status() == 0
+
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    t_start, t_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local) if rank == 0 else None
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    t_start.record(stream)
+    for i in range(args.steps):
+        step(reps[i % n_rep], ev[i])
+    t_stop.record(stream)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    clocks = sampler.stop() if sampler else None
+    ms = t_start.elapsed_time(t_stop)
+    ffn_ms = [a.elapsed_time(b) for a, b in ev]
+    if dist:
+        t = torch.tensor([ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    tokens = wl.T * args.steps * world
+    value = tokens / (ms / 1e3)
+
+    # roofline of the dominant kernel: the tcgen05 grouped GEMM (gate/up + down launches)
+    hbm, tf_burst, tf_sust, peak_src = _peaks()
+    kept_timed = [kept[i % n_rep] for i in range(args.steps)]
+    gemm_flops = sum(6.0 * wl.d * wl.h * kr for kr in kept_timed)
+    gemm_s = sum(ffn_ms) / 1e3
+    achieved_tf = gemm_flops / gemm_s / 1e12
+    roofline = {"bound": "tensor", "achieved": achieved_tf, "peak": tf_burst, "unit": "TFLOP/s",
+                "frac": achieved_tf / tf_burst, "traffic": None,
+                "kernel": "tc_grouped_gemm (gate/up + down, 2 launches per step)",
+                "peak_source": f"{peak_src} bf16_tflops (burst)",
+                "ms_per_launch_pair": gemm_s / args.steps * 1e3}
+
+    # end to end: pinned host input -> device -> layer -> pinned host output
+    e2e = None
+    if not args.no_e2e:
+        u_host = torch.empty_like(reps[0].u, device="cpu").pin_memory()
+        u_host.copy_(reps[0].u.cpu())
+        y_host = torch.empty_like(step.y, device="cpu").pin_memory()
+        u_dev = torch.empty_like(reps[0].u)
+        r0 = reps[0]
+        outs = {"top_idx": step.top_idx}
+        lws = torch.empty(moe.moe_layer_workspace_bytes(step.s, wl.act_dtype), dtype=torch.uint8,
+                          device="cuda")
+
+        def e2e_step():
+            u_dev.copy_(u_host, non_blocking=True)
+            moe.moe_layer_fwd(step.s, r0.w_route, *r0.w, u_dev, step.y, bias=r0.bias,
+                              outputs=outs, ws=lws)
+            y_host.copy_(step.y, non_blocking=True)
+
+        for _ in range(args.warmup):
+            e2e_step()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        e_ms = a.elapsed_time(b)
+        if dist:
+            t = torch.tensor([e_ms], device="cuda")
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t.item())
+        el = 2 if wl.act_dtype != S.DT_F32 else 4
+        e2e = {"value": tokens / (e_ms / 1e3), "unit": "tokens/s",
+               "h2d_bytes_per_step": wl.T * wl.d * el, "d2h_bytes_per_step": wl.T * wl.d * el}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        host = oracle_host_inputs(wl)
+        v, el_s, n = run_cpu_baseline(wl, host)
+        cpu = {"value": v, "unit": "tokens/s", "cores": os.cpu_count(), "kind": "oracle",
+               "sample": f"random samples of {n} tokens of the {wl.name} batch, "
+                         f"{el_s:.1f} s of CPU work"}
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "bf16" if wl.act_dtype == S.DT_BF16 else "f32", "data": "synthetic",
+                "config": {"workload": f"{wl.name}: T={wl.T} d={wl.d} N={wl.N} h={wl.h} "
+                                       f"top-{wl.k}", "global_batch": wl.T * world,
+                           "parallelism": f"replicas x{world}",
+                           "l2": f"inputs rotate over {n_rep} replicas "
+                                 f"({n_rep * one.nbytes() / 2**20:.0f} MiB > L2)",
+                           "capacity": wl.capacity()},
+                "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+                "gpu_launches": step.launches_per_step * args.steps, "clocks": clocks}
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

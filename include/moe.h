@@ -1,0 +1,222 @@
+/*
+ * moe.h -- C ABI of the B200 (sm_100a) sparse Mixture-of-Experts layer forward.
+ *
+ * The layer (tutorial "Mixture of Experts MoE: how sparse activation saves
+ * compute", §3.1-§3.8):
+ *   z_t = W_route u_t (+ b)          router logits, fp32          (§3.2 eq. z)
+ *   p_t = softmax(z_t)                                             (§3.2 eq. p)
+ *   S_t = top-k of z_t, ties to the lower expert index             (§3.2)
+ *   a_{t,i} = p_{t,i} / sum_{j in S_t} p_{t,j}   (renorm)          (§3.2 eq. a)
+ *   F_i(u) = W_down,i (SiLU(W_gate,i u) * W_up,i u)  SwiGLU expert (§3.1 eq. F)
+ *   y_t = sum_{i in S_t, kept} a_{t,i} F_i(u_t)                    (§3.2 eq. y)
+ * with tokens grouped by expert and a per-expert capacity C (§3.5, §3.6, §3.8).
+ *
+ * Conventions shared by every entry point:
+ *   - All tensor pointers are DEVICE pointers unless a parameter says "host".
+ *     The caller owns every buffer; the library never allocates device memory.
+ *     Scratch memory is passed as (ws, ws_bytes); its size comes from the
+ *     matching *_workspace_bytes query.  Pointers must be 16-byte aligned.
+ *   - Row-major layouts.  u [T][d]; W_route [N][d] fp32; bias [N] fp32;
+ *     expert weights expert-contiguous: W_gate [N][h][d], W_up [N][h][d],
+ *     W_down [N][d][h] (the expert-grouped storage of the deployment notes,
+ *     "Kestrel-MCU notes 13", §2).
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default).
+ *   - Return value: MOE_OK (0) or a negative MOE_ERR_*.  Argument errors are
+ *     detected on the host, synchronously, before anything is launched.
+ *     Errors found by a kernel (an index out of range, a bounded wait that
+ *     ran out) are recorded in a sticky device status word that
+ *     moe_device_status() reads.  No C++ exception crosses this boundary.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Every entry point is exported from the shared library. */
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+/* ---------------------------------------------------------------- status */
+#define MOE_OK 0
+#define MOE_ERR_INVALID_ARG (-1) /* null pointer, bad size, misalignment */
+#define MOE_ERR_UNSUPPORTED (-2) /* valid but not implemented combination */
+#define MOE_ERR_CUDA (-3)        /* a CUDA runtime call failed */
+#define MOE_ERR_TIMEOUT (-4)     /* device: a bounded wait ran out */
+#define MOE_ERR_BOUNDS (-5)      /* device: an index was out of range */
+#define MOE_ERR_WORKSPACE (-6)   /* ws_bytes smaller than the query returned */
+
+/* ------------------------------------------------------------ data types */
+#define MOE_F32 0
+#define MOE_BF16 1
+#define MOE_F16 2
+#define MOE_Q4_0 3
+
+/* Expert activation.  MOE_ACT_SWIGLU: H = SiLU(g) * v.  MOE_ACT_SITU_GLU:
+ * H = SiLU(beta_gate tanh(g / beta_gate)) * beta_up tanh(v / beta_up), the
+ * soft-capped gate and up of the Stable LatentMoE demo document (SiTU-GLU),
+ * whose product stays below beta_gate * beta_up. */
+#define MOE_ACT_SWIGLU 0
+#define MOE_ACT_SITU_GLU 1
+
+typedef struct {
+  int32_t kind;    /* MOE_ACT_* */
+  float beta_gate; /* SiTU-GLU only */
+  float beta_up;   /* SiTU-GLU only */
+} moe_act;
+
+/* Problem shape.  T tokens of width d, N experts, k experts per token,
+ * expert hidden width h.  renorm = 1 uses a = p_S / sum p_S (Mixtral-style
+ * top-k, tutorial §3.2); renorm = 0 keeps a = p_S (the Switch top-1
+ * multiplier, §3.2 caveat).  capacity = C slots per expert (0 = unlimited);
+ * the tutorial's C = ceil(c * dispatches / N) is what moe_capacity computes. */
+typedef struct {
+  int32_t T;
+  int32_t d;
+  int32_t N;
+  int32_t k;
+  int32_t h;
+  int32_t renorm;
+  int32_t capacity;
+} moe_shape;
+
+/* Limits checked on the host: 1 <= k <= min(N, 32); 1 <= N <= 1024;
+ * d % 8 == 0; h % 64 == 0 for the bf16 tensor-core experts; T * k < 2^31. */
+
+/* Host-only.  C = ceil(factor * k * T / N), tutorial §3.5 with the top-k
+ * dispatch count.  Writes *capacity (host pointer).  factor <= 0 gives 0. */
+MOE_API int moe_capacity(int64_t T, int32_t N, int32_t k, double factor, int32_t* capacity);
+
+/* ---------------------------------------------------------------- router */
+/* Router, softmax, top-k and combine weights (tutorial §3.2).
+ *   u        [T][d] in u_dtype (MOE_F32, MOE_BF16 or MOE_F16)
+ *   w_route  [N][d] fp32;  bias [N] fp32 or NULL (added to z after the dot)
+ *   top_idx  [T][k] int32 out: experts by descending z, ties to lower index
+ *   top_w    [T][k] fp32 out: a (renormalised when shape->renorm)
+ *   probs    [T][N] fp32 out or NULL: softmax p
+ *   logits   [T][N] fp32 out or NULL: z
+ * z is a sequential fp32 fused-multiply-add chain over j = 0..d-1 (then + b),
+ * so routing decisions are reproducible bit for bit.
+ * Needs ws of moe_route_workspace_bytes(shape) bytes (may be 0 -> ws NULL). */
+MOE_API size_t moe_route_workspace_bytes(const moe_shape* shape);
+MOE_API int moe_route(const moe_shape* shape, const void* u, int32_t u_dtype, const float* w_route,
+              const float* bias, int32_t* top_idx, float* top_w, float* probs, float* logits,
+              void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------- aux stats */
+/* Switch balancing statistics (tutorial §3.4) from probs [T][N] and top_idx:
+ *   f[i] = fraction of tokens whose argmax (slot 0) is i
+ *   P[i] = mean over tokens of p[t][i]
+ *   n_sum_fP[0] = N * sum_i f[i] P[i]   (L_aux without alpha)
+ *   loads[i] = dispatches to expert i over all k slots (L_i, §3.6)
+ * Any output may be NULL; probs may be NULL (P and n_sum_fP then read 0).
+ * ws: moe_aux_stats_workspace_bytes(N) bytes of scratch. */
+MOE_API size_t moe_aux_stats_workspace_bytes(int32_t N);
+MOE_API int moe_aux_stats(int32_t T, int32_t N, int32_t k, const float* probs, const int32_t* top_idx,
+                  float* f, float* P, float* n_sum_fP, int32_t* loads, void* ws, size_t ws_bytes,
+                  void* stream);
+
+/* --------------------------------------------------------------- permute */
+/* Group the T*k dispatches by expert (tutorial §3.5, §3.6, §3.8).
+ * Dispatch (t, s) -> expert top_idx[t][s]; its rank = dispatches to the same
+ * expert from lower tokens; kept iff capacity == 0 or rank < capacity.
+ *   counts   [N]   L_e, all dispatches
+ *   offsets  [N+1] exclusive prefix sum of the kept counts; offsets[N] = rows
+ *   perm_tok [T*k] token of grouped row r, for r < offsets[N]
+ *   row_of   [T][k] grouped row of (t, s), or -1 when dropped
+ *   overflow [N]   max(L_e - C, 0)
+ *   totals   [3]   {kept rows, overflowed dispatches, empty slots sum max(C - L_e, 0)}
+ * Bit-exact and deterministic.  ws: moe_permute_workspace_bytes(shape). */
+MOE_API size_t moe_permute_workspace_bytes(const moe_shape* shape);
+MOE_API int moe_permute(const moe_shape* shape, const int32_t* top_idx, int32_t* counts,
+                int32_t* offsets, int32_t* perm_tok, int32_t* row_of, int32_t* overflow,
+                int32_t* totals, void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------- gather */
+/* x_rows[r] = u[perm_tok[r]] for r < offsets[N] (tutorial §3.6: expert i
+ * receives its [L_i, d] rows).  u [T][width] in dtype; x_rows has room for
+ * T*k rows of width elements.  Rows >= offsets[N] are left untouched. */
+MOE_API int moe_gather(const moe_shape* shape, int32_t width, const void* u, int32_t dtype,
+               const int32_t* perm_tok, const int32_t* offsets, void* x_rows, void* stream);
+
+/* ------------------------------------------------------------ expert FFN */
+/* Grouped expert FFN on grouped rows (tutorial §3.1): for every grouped row
+ * r of expert e (offsets[e] <= r < offsets[e+1]):
+ *   y_rows[r] = W_down,e act(W_gate,e x_rows[r], W_up,e x_rows[r])
+ * unweighted, fp32 [T*k][width].  width is the expert input/output width (d,
+ * or the latent width of a latent-space layer); h = shape->h.
+ * dtype = w_dtype = MOE_F32 (SIMT fp32) or MOE_BF16 (tcgen05 tensor cores,
+ * fp32 accumulate, hidden stored as bf16).  ws: moe_expert_ffn_workspace_bytes. */
+MOE_API size_t moe_expert_ffn_workspace_bytes(const moe_shape* shape, int32_t width, int32_t dtype);
+MOE_API int moe_expert_ffn(const moe_shape* shape, int32_t width, const void* x_rows, int32_t dtype,
+                   const int32_t* offsets, const void* w_gate, const void* w_up,
+                   const void* w_down, int32_t w_dtype, const moe_act* act, float* y_rows,
+                   void* ws, size_t ws_bytes, void* stream);
+
+/* --------------------------------------------------------------- combine */
+/* y[t] = sum over kept slots s (row_of[t][s] >= 0, ascending s) of
+ * top_w[t][s] * y_rows[row_of[t][s]]  (tutorial §3.2 eq. y); dropped slots
+ * add nothing and the weights are not renormalised.  y [T][width] in y_dtype
+ * (MOE_F32, MOE_BF16 or MOE_F16), fully overwritten. */
+MOE_API int moe_combine(const moe_shape* shape, int32_t width, const float* y_rows,
+                const int32_t* row_of, const float* top_w, void* y, int32_t y_dtype,
+                void* stream);
+
+/* ------------------------------------------------------------ full layer */
+typedef struct {
+  const float* w_route; /* [N][d] fp32 */
+  const float* bias;    /* [N] fp32 or NULL */
+  const void* w_gate;   /* [N][h][d] */
+  const void* w_up;     /* [N][h][d] */
+  const void* w_down;   /* [N][d][h] */
+  int32_t w_dtype;      /* MOE_F32 or MOE_BF16 (same as the activations) */
+  moe_act act;
+} moe_layer_weights;
+
+/* Optional device outputs of moe_layer_fwd; every pointer may be NULL. */
+typedef struct {
+  int32_t* top_idx;  /* [T][k] */
+  float* top_w;      /* [T][k] */
+  float* probs;      /* [T][N] */
+  int32_t* counts;   /* [N] */
+  int32_t* offsets;  /* [N+1] */
+  int32_t* perm_tok; /* [T*k] */
+  int32_t* row_of;   /* [T][k] */
+  int32_t* overflow; /* [N] */
+  int32_t* totals;   /* [3] */
+  float* f;          /* [N] */
+  float* P;          /* [N] */
+  float* n_sum_fP;   /* [1] */
+} moe_layer_outputs;
+
+/* The whole forward: router -> permute -> gather -> grouped SwiGLU experts ->
+ * weighted combine, plus the aux statistics when out->f/P/n_sum_fP are set.
+ * u and y are [T][d] in act_dtype (MOE_F32 or MOE_BF16).  y excludes the
+ * residual: a dropped dispatch contributes zero (tutorial §3.5: the
+ * residual path carries it).  ws: moe_layer_workspace_bytes. */
+MOE_API size_t moe_layer_workspace_bytes(const moe_shape* shape, int32_t act_dtype);
+MOE_API int moe_layer_fwd(const moe_shape* shape, const moe_layer_weights* w, const void* u,
+                  int32_t act_dtype, void* y, const moe_layer_outputs* out, void* ws,
+                  size_t ws_bytes, void* stream);
+
+/* ----------------------------------------------------------- diagnostics */
+/* Human-readable name of a status code (static string). */
+MOE_API const char* moe_status_string(int32_t status);
+/* Synchronises `stream`, then copies the sticky device status word to
+ * *status (host pointer): MOE_OK or the first MOE_ERR_* a kernel recorded. */
+MOE_API int moe_device_status(void* stream, int32_t* status);
+/* Clears the device status word (asynchronous on stream). */
+MOE_API int moe_reset_device_status(void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

@@ -65,12 +65,13 @@ def lib():
         L.or_moe_dense.argtypes = [i64, i64, i64, vp, vp, vp, vp, i64, vp, vp, ctypes.c_int, dbl,
                                    dbl, ctypes.c_int, vp]
         L.or_rmsnorm.argtypes = [i64, vp, dbl, vp]
+        L.or_combine.argtypes = [i64, i64, i64, vp, vp, vp, vp]
         L.or_ledger.argtypes = [i64, i64, i64, i64, vp, vp, vp, vp]
         L.or_bandwidth_gain.argtypes = [i64, i64, i64]
         L.or_bandwidth_gain.restype = dbl
         for f in (L.or_mat_decode, L.or_route, L.or_route_from_logits, L.or_aux_stats,
                   L.or_permute, L.or_matvec, L.or_expert, L.or_moe_tokens, L.or_moe_dense,
-                  L.or_rmsnorm, L.or_ledger):
+                  L.or_rmsnorm, L.or_ledger, L.or_combine):
             f.restype = None
         _lib = L
     return _lib
@@ -243,6 +244,18 @@ def moe_dense(Wg, Wu, Wd, u, idx, top_w, act=0, beta_g=0.0, beta_u=0.0, round_h=
     lib().or_moe_dense(T, len(Wg), k, mat_array(Wg), mat_array(Wu), mat_array(Wd), u.ctypes.data,
                        d_in, idx.ctypes.data, top_w.ctypes.data, act, beta_g, beta_u, round_h,
                        y.ctypes.data)
+    return y
+
+
+def combine(rows, row_of, top_w):
+    """y_t = sum over kept slots of a_{t,s} * rows[row_of[t, s]] (float64)."""
+    rows = _c(rows, np.float64)
+    row_of, top_w = _c(row_of, np.int32), _c(top_w, np.float64)
+    T, k = row_of.shape
+    width = rows.shape[1]
+    y = np.empty((T, width), np.float64)
+    lib().or_combine(T, k, width, rows.ctypes.data, row_of.ctypes.data, top_w.ctypes.data,
+                     y.ctypes.data)
     return y
 
 

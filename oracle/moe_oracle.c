@@ -342,6 +342,21 @@ void or_moe_tokens(int64_t k, const or_mat* Wg, const or_mat* Wu, const or_mat* 
   }
 }
 
+/* Weighted combine of per-row expert outputs  [MoE tutorial] §3.2 eq. y and
+ * §3.6 (results added back to [T, d] by token index): for each token,
+ * y_t = sum over slots s with row_of[t][s] >= 0 of top_w[t][s] * rows[row_of[t][s]]. */
+void or_combine(int64_t T, int64_t k, int64_t width, const double* rows, const int32_t* row_of,
+                const double* top_w, double* y) {
+  for (int64_t t = 0; t < T; ++t) {
+    for (int64_t m = 0; m < width; ++m) y[t * width + m] = 0.0;
+    for (int64_t s = 0; s < k; ++s) {
+      int32_t r = row_of[t * k + s];
+      if (r < 0) continue;
+      for (int64_t m = 0; m < width; ++m) y[t * width + m] += top_w[t * k + s] * rows[r * width + m];
+    }
+  }
+}
+
 /* Dense brute-force reference  [MoE tutorial] appendix lab: every expert is
  * evaluated for every token and multiplied by its combine weight, which is
  * zero for the unselected experts.  Must equal or_moe_tokens exactly when

@@ -1,0 +1,206 @@
+"""Python binding of the sm_100a sparse-MoE layer library (libmoe.so).
+
+Argument marshalling only: every function here converts torch tensors to
+device pointers, calls the C entry point of the same name declared in
+include/moe.h, and raises MoeError on a non-zero status.  All compute runs in
+the library's CUDA kernels; there is no Python or CPU fallback.  Importing
+this package fails loudly when libmoe.so has not been built.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoe.so")
+
+F32, BF16, F16, Q4_0 = 0, 1, 2, 3
+ACT_SWIGLU, ACT_SITU_GLU = 0, 1
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with "
+                      "`python sparse_mixture_experts_15_b200/build.py` (nvcc, sm_100a)")
+_lib = ctypes.CDLL(LIB_PATH)
+
+_i32, _i64, _sz, _vp, _f32, _f64 = (ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t,
+                                    ctypes.c_void_p, ctypes.c_float, ctypes.c_double)
+
+
+class MoeShape(ctypes.Structure):
+    _fields_ = [("T", _i32), ("d", _i32), ("N", _i32), ("k", _i32), ("h", _i32),
+                ("renorm", _i32), ("capacity", _i32)]
+
+
+class MoeAct(ctypes.Structure):
+    _fields_ = [("kind", _i32), ("beta_gate", _f32), ("beta_up", _f32)]
+
+
+class MoeLayerWeights(ctypes.Structure):
+    _fields_ = [("w_route", _vp), ("bias", _vp), ("w_gate", _vp), ("w_up", _vp),
+                ("w_down", _vp), ("w_dtype", _i32), ("act", MoeAct)]
+
+
+class MoeLayerOutputs(ctypes.Structure):
+    _fields_ = [(n, _vp) for n in ("top_idx", "top_w", "probs", "counts", "offsets", "perm_tok",
+                                   "row_of", "overflow", "totals", "f", "P", "n_sum_fP")]
+
+
+_P_SHAPE = ctypes.POINTER(MoeShape)
+_PROTOS = {
+    "moe_capacity": (_i32, [_i64, _i32, _i32, _f64, ctypes.POINTER(_i32)]),
+    "moe_route_workspace_bytes": (_sz, [_P_SHAPE]),
+    "moe_route": (_i32, [_P_SHAPE, _vp, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "moe_aux_stats_workspace_bytes": (_sz, [_i32]),
+    "moe_aux_stats": (_i32, [_i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "moe_permute_workspace_bytes": (_sz, [_P_SHAPE]),
+    "moe_permute": (_i32, [_P_SHAPE, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "moe_gather": (_i32, [_P_SHAPE, _i32, _vp, _i32, _vp, _vp, _vp, _vp]),
+    "moe_expert_ffn_workspace_bytes": (_sz, [_P_SHAPE, _i32, _i32]),
+    "moe_expert_ffn": (_i32, [_P_SHAPE, _i32, _vp, _i32, _vp, _vp, _vp, _vp, _i32,
+                              ctypes.POINTER(MoeAct), _vp, _vp, _sz, _vp]),
+    "moe_combine": (_i32, [_P_SHAPE, _i32, _vp, _vp, _vp, _vp, _i32, _vp]),
+    "moe_layer_workspace_bytes": (_sz, [_P_SHAPE, _i32]),
+    "moe_layer_fwd": (_i32, [_P_SHAPE, ctypes.POINTER(MoeLayerWeights), _vp, _i32, _vp,
+                             ctypes.POINTER(MoeLayerOutputs), _vp, _sz, _vp]),
+    "moe_status_string": (ctypes.c_char_p, [_i32]),
+    "moe_device_status": (_i32, [_vp, ctypes.POINTER(_i32)]),
+    "moe_reset_device_status": (_i32, [_vp]),
+}
+for _name, (_res, _args) in _PROTOS.items():
+    _fn = getattr(_lib, _name)
+    _fn.restype, _fn.argtypes = _res, _args
+
+EXPORTED = tuple(_PROTOS)
+
+
+class MoeError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        msg = _lib.moe_status_string(status).decode()
+        super().__init__(f"{where}: {msg} ({status})")
+        self.status = status
+
+
+def _check(rc: int, where: str):
+    if rc != 0:
+        raise MoeError(rc, where)
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    return int(stream)
+
+
+def _dtype_code(t):
+    import torch
+    return {torch.float32: F32, torch.bfloat16: BF16, torch.float16: F16}[t.dtype]
+
+
+def _ws(nbytes, device, ws=None):
+    import torch
+    if ws is not None:
+        if ws.numel() * ws.element_size() < nbytes:
+            raise MoeError(-6, "workspace")
+        return ws, ws.numel() * ws.element_size()
+    n = max(int(nbytes), 256)
+    return torch.empty(n, dtype=torch.uint8, device=device), n
+
+
+def shape(T, d, N, k, h=0, renorm=1, capacity=0) -> MoeShape:
+    return MoeShape(T, d, N, k, h, renorm, capacity)
+
+
+def act(kind=ACT_SWIGLU, beta_gate=0.0, beta_up=0.0) -> MoeAct:
+    return MoeAct(kind, beta_gate, beta_up)
+
+
+# ------------------------------------------------------------- entry points
+def moe_capacity(T: int, N: int, k: int, factor: float) -> int:
+    out = _i32(0)
+    _check(_lib.moe_capacity(T, N, k, factor, ctypes.byref(out)), "moe_capacity")
+    return out.value
+
+
+def moe_route(s: MoeShape, u, w_route, top_idx, top_w, bias=None, probs=None, logits=None,
+              ws=None, stream=None):
+    nb = _lib.moe_route_workspace_bytes(ctypes.byref(s))
+    wbuf, wlen = (None, 0) if logits is not None else _ws(nb, u.device, ws)
+    _check(_lib.moe_route(ctypes.byref(s), _ptr(u), _dtype_code(u), _ptr(w_route), _ptr(bias),
+                          _ptr(top_idx), _ptr(top_w), _ptr(probs), _ptr(logits), _ptr(wbuf), wlen,
+                          _stream(stream)), "moe_route")
+
+
+def moe_aux_stats(probs, top_idx, f=None, P=None, n_sum_fP=None, loads=None, ws=None,
+                  stream=None):
+    T, k = top_idx.shape
+    N = f.shape[0] if f is not None else (P.shape[0] if P is not None else loads.shape[0])
+    wbuf, wlen = _ws(_lib.moe_aux_stats_workspace_bytes(N), top_idx.device, ws)
+    _check(_lib.moe_aux_stats(T, N, k, _ptr(probs), _ptr(top_idx), _ptr(f), _ptr(P),
+                              _ptr(n_sum_fP), _ptr(loads), _ptr(wbuf), wlen, _stream(stream)),
+           "moe_aux_stats")
+
+
+def moe_permute(s: MoeShape, top_idx, counts, offsets, perm_tok, row_of, overflow, totals,
+                ws=None, stream=None):
+    wbuf, wlen = _ws(_lib.moe_permute_workspace_bytes(ctypes.byref(s)), top_idx.device, ws)
+    _check(_lib.moe_permute(ctypes.byref(s), _ptr(top_idx), _ptr(counts), _ptr(offsets),
+                            _ptr(perm_tok), _ptr(row_of), _ptr(overflow), _ptr(totals), _ptr(wbuf),
+                            wlen, _stream(stream)), "moe_permute")
+
+
+def moe_gather(s: MoeShape, width: int, u, perm_tok, offsets, x_rows, stream=None):
+    _check(_lib.moe_gather(ctypes.byref(s), width, _ptr(u), _dtype_code(u), _ptr(perm_tok),
+                           _ptr(offsets), _ptr(x_rows), _stream(stream)), "moe_gather")
+
+
+def moe_expert_ffn(s: MoeShape, width: int, x_rows, offsets, w_gate, w_up, w_down, y_rows,
+                   a: MoeAct | None = None, ws=None, stream=None):
+    a = a or act()
+    dt = _dtype_code(x_rows)
+    nb = _lib.moe_expert_ffn_workspace_bytes(ctypes.byref(s), width, dt)
+    wbuf, wlen = _ws(nb, x_rows.device, ws)
+    _check(_lib.moe_expert_ffn(ctypes.byref(s), width, _ptr(x_rows), dt, _ptr(offsets),
+                               _ptr(w_gate), _ptr(w_up), _ptr(w_down), _dtype_code(w_gate),
+                               ctypes.byref(a), _ptr(y_rows), _ptr(wbuf), wlen, _stream(stream)),
+           "moe_expert_ffn")
+
+
+def moe_combine(s: MoeShape, width: int, y_rows, row_of, top_w, y, stream=None):
+    _check(_lib.moe_combine(ctypes.byref(s), width, _ptr(y_rows), _ptr(row_of), _ptr(top_w),
+                            _ptr(y), _dtype_code(y), _stream(stream)), "moe_combine")
+
+
+def moe_layer_workspace_bytes(s: MoeShape, act_dtype: int) -> int:
+    return int(_lib.moe_layer_workspace_bytes(ctypes.byref(s), act_dtype))
+
+
+def moe_layer_fwd(s: MoeShape, w_route, w_gate, w_up, w_down, u, y, bias=None, a=None,
+                  outputs: dict | None = None, ws=None, stream=None):
+    """The whole layer.  `outputs` maps moe_layer_outputs field names to tensors."""
+    a = a or act()
+    dt = _dtype_code(u)
+    W = MoeLayerWeights(_ptr(w_route), _ptr(bias), _ptr(w_gate), _ptr(w_up), _ptr(w_down),
+                        _dtype_code(w_gate), a)
+    O = MoeLayerOutputs(**{k: _ptr(v) for k, v in (outputs or {}).items()})
+    wbuf, wlen = _ws(moe_layer_workspace_bytes(s, dt), u.device, ws)
+    _check(_lib.moe_layer_fwd(ctypes.byref(s), ctypes.byref(W), _ptr(u), dt, _ptr(y),
+                              ctypes.byref(O), _ptr(wbuf), wlen, _stream(stream)), "moe_layer_fwd")
+
+
+def moe_device_status(stream=None) -> int:
+    out = _i32(0)
+    _check(_lib.moe_device_status(_stream(stream), ctypes.byref(out)), "moe_device_status")
+    return out.value
+
+
+def moe_reset_device_status(stream=None):
+    _check(_lib.moe_reset_device_status(_stream(stream)), "moe_reset_device_status")
+
+
+def status_string(code: int) -> str:
+    return _lib.moe_status_string(code).decode()

@@ -1,0 +1,140 @@
+// Shared helpers of the sm_100a MoE library: status reporting, number
+// conversions, vector loads and host-side argument checks.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/moe.h"
+
+namespace moe {
+
+// ------------------------------------------------------------- device status
+// The sticky status word lives in status.cu; kernels receive its address as an
+// argument and record the first error with atomicCAS (never trap).
+__device__ __forceinline__ void record_error(int* status, int code) {
+  if (status) atomicCAS(status, 0, code);
+}
+
+// Returns the device address of the status word of the current device.
+int* status_word();
+
+// ----------------------------------------------------------------- numbers
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+__device__ __forceinline__ float to_f32(__half x) { return __half2float(x); }
+
+template <typename T>
+__device__ __forceinline__ T from_f32(float x);
+template <>
+__device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <>
+__device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+  return __float2bfloat16_rn(x);
+}
+template <>
+__device__ __forceinline__ __half from_f32<__half>(float x) { return __float2half_rn(x); }
+
+// Load 8 consecutive elements (16 B for 16-bit types, 32 B for fp32) as fp32.
+__device__ __forceinline__ void load8(const float* p, float* o) {
+  float4 a = *reinterpret_cast<const float4*>(p);
+  float4 b = *reinterpret_cast<const float4*>(p + 4);
+  o[0] = a.x; o[1] = a.y; o[2] = a.z; o[3] = a.w;
+  o[4] = b.x; o[5] = b.y; o[6] = b.z; o[7] = b.w;
+}
+__device__ __forceinline__ void load8(const __nv_bfloat16* p, float* o) {
+  uint4 v = *reinterpret_cast<const uint4*>(p);
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    o[2 * i] = __uint_as_float(w[i] << 16);
+    o[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+  }
+}
+__device__ __forceinline__ void load8(const __half* p, float* o) {
+  uint4 v = *reinterpret_cast<const uint4*>(p);
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    __half2 h = *reinterpret_cast<const __half2*>(&w[i]);
+    float2 f = __half22float2(h);
+    o[2 * i] = f.x;
+    o[2 * i + 1] = f.y;
+  }
+}
+
+__device__ __forceinline__ float silu(float g) { return g / (1.0f + expf(-g)); }
+
+// ------------------------------------------------------------- host checks
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline bool valid_act_dtype(int32_t dt) {
+  return dt == MOE_F32 || dt == MOE_BF16 || dt == MOE_F16;
+}
+
+inline size_t dtype_bytes(int32_t dt) { return dt == MOE_F32 ? 4 : 2; }
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Basic shape validity shared by every entry point.
+inline bool shape_ok(const moe_shape* s) {
+  if (!s) return false;
+  if (s->T < 0 || s->d <= 0 || s->N <= 0 || s->N > 1024 || s->k <= 0 || s->k > 32) return false;
+  if (s->k > s->N || (s->d % 8) != 0 || s->capacity < 0) return false;
+  if ((int64_t)s->T * s->k >= (int64_t)1 << 31) return false;
+  return true;
+}
+
+inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+inline int cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+inline int launch_status() { return cuda_status(cudaGetLastError()); }
+
+// Carves sub-buffers out of a caller workspace (256-byte aligned pieces).
+struct Carver {
+  char* base;
+  size_t off = 0;
+  explicit Carver(void* b) : base(static_cast<char*>(b)) {}
+  template <typename T>
+  T* take(size_t count) {
+    off = align_up(off, 256);
+    T* p = base ? reinterpret_cast<T*>(base + off) : nullptr;
+    off += count * sizeof(T);
+    return p;
+  }
+  size_t used() const { return align_up(off, 256); }
+};
+
+// ------------------------------------------------------- internal launchers
+// (defined in the per-step .cu files; all asynchronous on `st`)
+size_t route_ws_bytes(const moe_shape& s);
+int launch_route(const moe_shape& s, const void* u, int32_t u_dtype, const float* w_route,
+                 const float* bias, int32_t* top_idx, float* top_w, float* probs, float* logits,
+                 void* ws, cudaStream_t st);
+size_t aux_stats_ws_bytes(int32_t N);
+int launch_aux_stats(int32_t T, int32_t N, int32_t k, const float* probs, const int32_t* top_idx,
+                     float* f, float* P, float* n_sum_fP, int32_t* loads, void* ws,
+                     cudaStream_t st);
+size_t permute_ws_bytes(const moe_shape& s);
+int launch_permute(const moe_shape& s, const int32_t* top_idx, int32_t* counts, int32_t* offsets,
+                   int32_t* perm_tok, int32_t* row_of, int32_t* overflow, int32_t* totals,
+                   void* ws, cudaStream_t st);
+int launch_gather(const moe_shape& s, int32_t width, const void* u, int32_t dtype,
+                  const int32_t* perm_tok, const int32_t* offsets, void* x_rows, cudaStream_t st);
+int launch_combine(const moe_shape& s, int32_t width, const float* y_rows, const int32_t* row_of,
+                   const float* top_w, void* y, int32_t y_dtype, cudaStream_t st);
+size_t ffn_simt_ws_bytes(const moe_shape& s);
+int launch_ffn_simt(const moe_shape& s, int32_t width, const float* x_rows, const int32_t* offsets,
+                    const float* w_gate, const float* w_up, const float* w_down,
+                    const moe_act& act, float* y_rows, void* ws, cudaStream_t st);
+size_t ffn_tc_ws_bytes(const moe_shape& s, int32_t width);
+int launch_ffn_tc(const moe_shape& s, int32_t width, const __nv_bfloat16* x_rows,
+                  const int32_t* offsets, const __nv_bfloat16* w_gate, const __nv_bfloat16* w_up,
+                  const __nv_bfloat16* w_down, const moe_act& act, float* y_rows, void* ws,
+                  cudaStream_t st);
+
+}  // namespace moe

@@ -1,0 +1,512 @@
+// Grouped expert GEMMs on the sm_100a tensor cores (tcgen05 + TMEM + TMA).
+//
+// Tutorial "Mixture of Experts MoE: how sparse activation saves compute",
+// §3.1 equation F and §3.6 (expert i works on its own [L_i, d] rows):
+//   gate/up:  H = act(X_e W_gate,e^T, X_e W_up,e^T)   -> bf16 [rows][h]
+//   down:     Y = H_e W_down,e^T                       -> fp32 [rows][width]
+//
+// Orientation: the expert WEIGHTS are the MMA's M operand (128 rows per tile)
+// and the expert's TOKENS are its N operand (up to BN per tile, rounded up to
+// 16), so a ragged last token tile of an expert costs only its own columns.
+// For gate/up the 128 weight rows of a tile are 64 gate rows stacked on the
+// 64 matching up rows (two TMA boxes), so one accumulator holds both halves
+// and the epilogue applies SiLU(g) * u (or the SiTU-GLU soft caps of the
+// Stable LatentMoE document) and stores bf16 H.
+//
+// Persistent kernel, one CTA per SM, 6 warps:
+//   warp 0    TMA producer (one elected lane), S-stage smem ring
+//   warp 1    TMEM allocator + single-thread tcgen05.mma issuer
+//   warps 2-5 epilogue: tcgen05.ld TMEM -> registers -> global
+// Two TMEM accumulators (2 x BN columns) let the epilogue of tile i overlap
+// the MMAs of tile i+1.  Every mbarrier wait is bounded; a wait that runs out
+// records MOE_ERR_TIMEOUT, stops all roles, drains in-flight TMA loads and
+// frees TMEM before the CTA exits.
+#include <cuda.h>
+
+#include "common.cuh"
+#include "tc_primitives.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kBM = 128;
+constexpr int kBK = 64;  // 64 bf16 = 128 bytes = one swizzle span
+constexpr int kThreads = 192;
+constexpr long long kWaitBudget = 4000000000LL;  // cycles (~2 s)
+constexpr int kEpiLd = 33;                       // padded row of the gate/up exchange tile
+
+enum { MODE_GATEUP = 0, MODE_STORE_F32 = 1, MODE_STORE_BF16 = 2 };
+
+struct TcParams {
+  CUtensorMap tmA0;  // weights (gate, or the single weight of a store mode)
+  CUtensorMap tmA1;  // up weights (gate/up mode)
+  CUtensorMap tmB;   // token rows
+  const int32_t* offsets;  // [G+1] token row ranges; nullptr: every group uses rows [0, T)
+  int T;
+  int G;
+  int K;                  // multiple of 64
+  int a_rows_per_group;   // rows of A owned by one group
+  int m_tiles;            // 128-row tiles of A per group
+  int mode;
+  int act_kind;
+  float beta_g, beta_u;
+  void* out;
+  int out_ld;             // elements per output row
+  int out_col_group;      // output column offset per group (groups sharing tokens)
+  int* status;
+};
+
+__device__ __forceinline__ float epi_act(float g, float v, int kind, float bg, float bu) {
+  if (kind == MOE_ACT_SITU_GLU) {
+    g = bg * tanhf(g / bg);
+    v = bu * tanhf(v / bu);
+  }
+  return silu(g) * v;
+}
+
+__device__ __forceinline__ void named_sync_epi() {
+  asm volatile("bar.sync 1, 128;" ::: "memory");
+}
+
+template <int BN, int S>
+struct Layout {
+  static constexpr int A_BYTES = kBM * kBK * 2;
+  static constexpr int B_BYTES = BN * kBK * 2;
+  static constexpr int STAGE = A_BYTES + B_BYTES;
+  static constexpr int EPI_BYTES = kBM * kEpiLd * 4;
+  static size_t bytes(int G) {
+    size_t b = 1024;  // alignment slack of the dynamic smem base
+    b += (size_t)S * STAGE + EPI_BYTES;
+    b += (size_t)3 * (G + 1) * 4;
+    b = align_up(b, 8);
+    b += (size_t)(2 * S + 5) * 8 + 16;
+    return b;
+  }
+};
+
+template <int BN, int S>
+__global__ void __launch_bounds__(kThreads, 1) tc_grouped_gemm(const __grid_constant__ TcParams p) {
+  using L = Layout<BN, S>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* stages = smem;
+  float* epi = reinterpret_cast<float*>(smem + S * L::STAGE);
+  int* grp_beg = reinterpret_cast<int*>(epi + kBM * kEpiLd);
+  int* grp_cnt = grp_beg + (p.G + 1);
+  int* grp_pre = grp_cnt + (p.G + 1);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(
+      (reinterpret_cast<uintptr_t>(grp_pre + p.G + 1) + 7) & ~static_cast<uintptr_t>(7));
+  uint64_t* full = bars;
+  uint64_t* empty = bars + S;
+  uint64_t* tfull = bars + 2 * S;
+  uint64_t* tempty = bars + 2 * S + 2;
+  uint64_t* drain = bars + 2 * S + 4;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 5);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const bool fused = p.mode == MODE_GATEUP;
+
+  // ---- group table: token range and tile prefix per group (warp 0 scans)
+  if (warp == 0) {
+    int carry = 0;
+    for (int base = 0; base < p.G; base += 32) {
+      const int g = base + lane;
+      int beg = 0, cnt = 0;
+      if (g < p.G) {
+        if (p.offsets) {
+          beg = p.offsets[g];
+          cnt = p.offsets[g + 1] - beg;
+          if (cnt < 0 || beg < 0) {
+            record_error(p.status, MOE_ERR_BOUNDS);
+            cnt = 0;
+          }
+        } else {
+          cnt = p.T;
+        }
+      }
+      const int t = g < p.G ? p.m_tiles * ((cnt + BN - 1) / BN) : 0;
+      int incl = t;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int n = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += n;
+      }
+      if (g < p.G) {
+        grp_beg[g] = beg;
+        grp_cnt[g] = cnt;
+        grp_pre[g] = carry + incl - t;
+      }
+      carry += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) {
+      grp_pre[p.G] = carry;
+      *abort_flag = 0;
+      for (int s = 0; s < S; ++s) {
+        tc::mbar_init(tc::smem_u32(&full[s]), 1);
+        tc::mbar_init(tc::smem_u32(&empty[s]), 1);
+      }
+      for (int b = 0; b < 2; ++b) {
+        tc::mbar_init(tc::smem_u32(&tfull[b]), 1);
+        tc::mbar_init(tc::smem_u32(&tempty[b]), 128);
+      }
+      tc::mbar_init(tc::smem_u32(drain), 1);
+      tc::fence_barrier_init();
+      tc::tma_prefetch_desc(&p.tmA0);
+      if (fused) tc::tma_prefetch_desc(&p.tmA1);
+      tc::tma_prefetch_desc(&p.tmB);
+    }
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(tc::smem_u32(tmem_slot), 2 * BN);
+    tc::tmem_relinquish();
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int total_tiles = grp_pre[p.G];
+  const int kblocks = p.K / kBK;
+
+  auto decode = [&](int tile, int& g, int& m, int& n) {
+    int lo = 0, hi = p.G;
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (grp_pre[mid] <= tile) lo = mid; else hi = mid;
+    }
+    g = lo;
+    const int local = tile - grp_pre[g];
+    const int nt = (grp_cnt[g] + BN - 1) / BN;
+    m = local / nt;
+    n = local - m * nt;
+  };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
+        int g, m, n;
+        decode(tile, g, m, n);
+        const int a_row = g * p.a_rows_per_group + m * (fused ? 64 : kBM);
+        const int b_row = grp_beg[g] + n * BN;
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!tc::mbar_wait(tc::smem_u32(&empty[stage]), phase ^ 1u, abort_flag, kWaitBudget)) {
+            ok = false;
+            break;
+          }
+          const uint32_t fb = tc::smem_u32(&full[stage]);
+          tc::mbar_arrive_expect_tx(fb, L::STAGE);
+          const uint32_t sa = tc::smem_u32(stages + stage * L::STAGE);
+          const uint32_t sb = sa + L::A_BYTES;
+          if (fused) {
+            tc::tma_load_2d(sa, &p.tmA0, fb, kb * kBK, a_row);
+            tc::tma_load_2d(sa + L::A_BYTES / 2, &p.tmA1, fb, kb * kBK, a_row);
+          } else {
+            tc::tma_load_2d(sa, &p.tmA0, fb, kb * kBK, a_row);
+          }
+          tc::tma_load_2d(sb, &p.tmB, fb, kb * kBK, b_row);
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok) {
+        record_error(p.status, MOE_ERR_TIMEOUT);
+        *abort_flag = 1;
+      }
+      // Drain: the last S issued stages may still have loads in flight.
+      for (int i = 0; i < S; ++i) {
+        if (--stage < 0) {
+          stage = S - 1;
+          phase ^= 1u;
+        }
+        tc::mbar_wait(tc::smem_u32(&full[stage]), phase, nullptr, kWaitBudget / 8);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ----------------------------------------------------------------- MMA
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      int it = 0;
+      for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x, ++it) {
+        int g, m, n;
+        decode(tile, g, m, n);
+        const int n_valid = min(BN, grp_cnt[g] - n * BN);
+        const uint32_t n_mma = (uint32_t)((n_valid + 15) & ~15);
+        const uint32_t idesc = tc::idesc_bf16_f32(kBM, n_mma);
+        const int b = it & 1;
+        const uint32_t use = (uint32_t)(it >> 1);
+        if (!tc::mbar_wait(tc::smem_u32(&tempty[b]), (use & 1u) ^ 1u, abort_flag, kWaitBudget)) {
+          ok = false;
+          break;
+        }
+        tc::tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(b * BN);
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!tc::mbar_wait(tc::smem_u32(&full[stage]), phase, abort_flag, kWaitBudget)) {
+            ok = false;
+            break;
+          }
+          tc::tc_fence_after();
+          const uint32_t sa = tc::smem_u32(stages + stage * L::STAGE);
+          const uint32_t sb = sa + L::A_BYTES;
+#pragma unroll
+          for (int k = 0; k < kBK / 16; ++k) {
+            tc::mma_bf16(d_tmem, tc::smem_desc_sw128(sa + k * 32), tc::smem_desc_sw128(sb + k * 32),
+                         idesc, (kb | k) != 0 ? 1u : 0u);
+          }
+          tc::mma_commit(tc::smem_u32(&empty[stage]));
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        tc::mma_commit(tc::smem_u32(&tfull[b]));
+      }
+      if (!ok) {
+        record_error(p.status, MOE_ERR_TIMEOUT);
+        *abort_flag = 1;
+        // Let every MMA issued so far finish before TMEM is released.
+        tc::mma_commit(tc::smem_u32(drain));
+        tc::mbar_wait(tc::smem_u32(drain), 0, nullptr, kWaitBudget / 8);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    const int row = q * 32 + lane;
+    int it = 0;
+    for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x, ++it) {
+      int g, m, n;
+      decode(tile, g, m, n);
+      const int n_valid = min(BN, grp_cnt[g] - n * BN);
+      const int tok0 = grp_beg[g] + n * BN;
+      const int b = it & 1;
+      const uint32_t use = (uint32_t)(it >> 1);
+      // The four epilogue warps share named barriers, so they take the
+      // give-up decision together.
+      const bool got = tc::mbar_wait(tc::smem_u32(&tfull[b]), use & 1u, abort_flag, kWaitBudget);
+      uint32_t all_ok;
+      asm volatile(
+          "{\n\t.reg .pred p, q;\n\t"
+          "setp.ne.u32 p, %1, 0;\n\t"
+          "bar.red.and.pred q, 1, 128, p;\n\t"
+          "selp.u32 %0, 1, 0, q;\n\t}"
+          : "=r"(all_ok)
+          : "r"((uint32_t)got)
+          : "memory");
+      if (!all_ok) {
+        record_error(p.status, MOE_ERR_TIMEOUT);
+        *abort_flag = 1;
+        break;
+      }
+      tc::tc_fence_after();
+      const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * BN);
+      for (int c = 0; c < n_valid; c += 32) {
+        float v[32];
+        tc::tmem_ld_32x32b_x32(t_row + (uint32_t)c, v);
+        if (p.mode == MODE_GATEUP) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) epi[row * kEpiLd + j] = v[j];
+          named_sync_epi();
+          const int tok = c + lane;
+          if (tok < n_valid) {
+            uint32_t packed[8];
+#pragma unroll
+            for (int i = 0; i < 16; i += 2) {
+              const float h0 = epi_act(epi[(q * 16 + i) * kEpiLd + lane],
+                                       epi[(64 + q * 16 + i) * kEpiLd + lane], p.act_kind,
+                                       p.beta_g, p.beta_u);
+              const float h1 = epi_act(epi[(q * 16 + i + 1) * kEpiLd + lane],
+                                       epi[(64 + q * 16 + i + 1) * kEpiLd + lane], p.act_kind,
+                                       p.beta_g, p.beta_u);
+              __nv_bfloat162 hv = __floats2bfloat162_rn(h0, h1);
+              packed[i >> 1] = *reinterpret_cast<uint32_t*>(&hv);
+            }
+            __nv_bfloat16* o = static_cast<__nv_bfloat16*>(p.out) +
+                               (size_t)(tok0 + tok) * p.out_ld + g * p.out_col_group + m * 64 +
+                               q * 16;
+            reinterpret_cast<uint4*>(o)[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+            reinterpret_cast<uint4*>(o)[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+          }
+          named_sync_epi();
+        } else {
+          const int col = g * p.out_col_group + m * kBM + row;
+          if (p.mode == MODE_STORE_F32) {
+            float* o = static_cast<float*>(p.out);
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (c + j < n_valid) o[(size_t)(tok0 + c + j) * p.out_ld + col] = v[j];
+          } else {
+            __nv_bfloat16* o = static_cast<__nv_bfloat16*>(p.out);
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (c + j < n_valid)
+                o[(size_t)(tok0 + c + j) * p.out_ld + col] = __float2bfloat16_rn(v[j]);
+          }
+        }
+      }
+      tc::tc_fence_before();
+      tc::mbar_arrive(tc::smem_u32(&tempty[b]));
+    }
+  }
+
+  tc::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc::tc_fence_after();
+    tc::tmem_dealloc(tmem_base, 2 * BN);
+  }
+}
+
+// ------------------------------------------------------------------- host
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+// Row-major bf16 matrix [rows][cols] viewed as a 2-D tensor, box 64 x box_rows,
+// 128-byte swizzle (the layout smem_desc_sw128 describes).
+bool make_tmap(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {(cuuint32_t)kBK, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int sm_count() {
+  static int cached[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) return 148;
+  if (!cached[dev]) {
+    int n = 0;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    cached[dev] = n > 0 ? n : 148;
+  }
+  return cached[dev];
+}
+
+template <int BN, int S>
+int launch_tc(const TcParams& p, int64_t tiles_upper, cudaStream_t st) {
+  const size_t smem = Layout<BN, S>::bytes(p.G);
+  static bool configured[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && !configured[dev]) {
+    if (cudaFuncSetAttribute(tc_grouped_gemm<BN, S>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)Layout<BN, S>::bytes(1024)) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    configured[dev] = true;
+  }
+  int64_t grid = sm_count();
+  if (tiles_upper < grid) grid = tiles_upper;
+  if (grid <= 0) return MOE_OK;
+  tc_grouped_gemm<BN, S><<<(unsigned)grid, kThreads, smem, st>>>(p);
+  return launch_status();
+}
+
+// Token tile width: 256 columns when that still gives at least two tiles per
+// SM, 128 otherwise (more, smaller tiles for small problems).
+int pick_bn(int m_tiles, int64_t max_rows, int G) {
+  const int64_t up256 = (int64_t)m_tiles * ((max_rows + 255) / 256 + G);
+  return up256 >= 2LL * sm_count() ? 256 : 128;
+}
+
+int launch_tc_bn(const TcParams& p, int64_t max_rows, int bn, cudaStream_t st) {
+  const int64_t upper = (int64_t)p.m_tiles * ((max_rows + bn - 1) / bn + p.G);
+  if (bn == 256) return launch_tc<256, 4>(p, upper, st);
+  return launch_tc<128, 6>(p, upper, st);
+}
+
+}  // namespace
+
+size_t ffn_tc_ws_bytes(const moe_shape& s, int32_t /*width*/) {
+  return align_up((size_t)s.T * s.k * s.h * 2, 256);
+}
+
+int launch_ffn_tc(const moe_shape& s, int32_t width, const __nv_bfloat16* x_rows,
+                  const int32_t* offsets, const __nv_bfloat16* w_gate, const __nv_bfloat16* w_up,
+                  const __nv_bfloat16* w_down, const moe_act& act, float* y_rows, void* ws,
+                  cudaStream_t st) {
+  const int64_t R = (int64_t)s.T * s.k;
+  if (R == 0) return MOE_OK;
+  __nv_bfloat16* H = static_cast<__nv_bfloat16*>(ws);
+  {  // gate/up with the fused activation -> H
+    TcParams p{};
+    const int64_t rows_w = (int64_t)s.N * s.h;
+    if (!make_tmap(&p.tmA0, w_gate, rows_w, width, 64) ||
+        !make_tmap(&p.tmA1, w_up, rows_w, width, 64))
+      return MOE_ERR_CUDA;
+    p.offsets = offsets;
+    p.T = s.T;
+    p.G = s.N;
+    p.K = width;
+    p.a_rows_per_group = s.h;
+    p.m_tiles = s.h / 64;
+    p.mode = MODE_GATEUP;
+    p.act_kind = act.kind;
+    p.beta_g = act.beta_gate;
+    p.beta_u = act.beta_up;
+    p.out = H;
+    p.out_ld = s.h;
+    p.out_col_group = 0;
+    p.status = status_word();
+    const int bn = pick_bn(p.m_tiles, R, p.G);
+    if (!make_tmap(&p.tmB, x_rows, R, width, bn)) return MOE_ERR_CUDA;
+    const int rc = launch_tc_bn(p, R, bn, st);
+    if (rc != MOE_OK) return rc;
+  }
+  {  // down projection -> unweighted fp32 rows
+    TcParams p{};
+    const int64_t rows_w = (int64_t)s.N * width;
+    if (!make_tmap(&p.tmA0, w_down, rows_w, s.h, kBM)) return MOE_ERR_CUDA;
+    p.tmA1 = p.tmA0;
+    p.offsets = offsets;
+    p.T = s.T;
+    p.G = s.N;
+    p.K = s.h;
+    p.a_rows_per_group = width;
+    p.m_tiles = width / kBM;
+    p.mode = MODE_STORE_F32;
+    p.out = y_rows;
+    p.out_ld = width;
+    p.out_col_group = 0;
+    p.status = status_word();
+    const int bn = pick_bn(p.m_tiles, R, p.G);
+    if (!make_tmap(&p.tmB, H, R, s.h, bn)) return MOE_ERR_CUDA;
+    const int rc = launch_tc_bn(p, R, bn, st);
+    if (rc != MOE_OK) return rc;
+  }
+  return MOE_OK;
+}
+
+}  // namespace moe

@@ -1,0 +1,190 @@
+// Token permutation: group the T*k dispatches by expert with a per-expert
+// capacity (tutorial "Mixture of Experts MoE: how sparse activation saves
+// compute", §3.5 capacity C, §3.6 grouping into per-expert [L_i, d] rows,
+// §3.8 overflow and empty slots).
+//
+// Three launches, all deterministic (atomics only count, ranks come from
+// scans):
+//   1. permute_hist:    block b counts the experts of dispatches
+//                       [256 b, 256 b + 256) -> hist[b][e]
+//   2. permute_scan:    one block; per expert an exclusive scan over blocks
+//                       (hist becomes the base rank of block b), L_e, the
+//                       kept counts, their exclusive scan -> offsets, overflow
+//                       and the totals
+//   3. permute_scatter: block b ranks its dispatches stably (warp match +
+//                       per-warp counts), keeps rank < C, writes row_of and
+//                       perm_tok
+#include "common.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kChunk = 256;  // dispatches per block = 8 warps x 32 lanes
+
+__global__ void __launch_bounds__(kChunk)
+    permute_hist(const int32_t* __restrict__ idx, int64_t total, int N, int32_t* __restrict__ hist,
+                 int* status) {
+  extern __shared__ int32_t cnt[];
+  for (int i = threadIdx.x; i < N; i += kChunk) cnt[i] = 0;
+  __syncthreads();
+  const int64_t x = (int64_t)blockIdx.x * kChunk + threadIdx.x;
+  if (x < total) {
+    const int e = idx[x];
+    if (e >= 0 && e < N) {
+      atomicAdd(&cnt[e], 1);
+    } else {
+      record_error(status, MOE_ERR_BOUNDS);
+    }
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < N; i += kChunk) hist[(size_t)blockIdx.x * N + i] = cnt[i];
+}
+
+// Block-wide exclusive scan of one int per thread (blockDim.x <= 1024).
+__device__ int block_exclusive_scan(int v, int* total) {
+  __shared__ int warp_sums[32];
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  int incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int n = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += n;
+  }
+  if (lane == 31) warp_sums[w] = incl;
+  __syncthreads();
+  if (w == 0) {
+    const int nw = (blockDim.x + 31) >> 5;
+    int s = lane < nw ? warp_sums[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int n = __shfl_up_sync(0xffffffffu, s, o);
+      if (lane >= o) s += n;
+    }
+    warp_sums[lane] = s;  // inclusive over warps
+  }
+  __syncthreads();
+  const int before = w > 0 ? warp_sums[w - 1] : 0;
+  if (total) *total = warp_sums[((blockDim.x + 31) >> 5) - 1];
+  __syncthreads();
+  return before + incl - v;
+}
+
+__device__ int block_sum(int v) {
+  int t;
+  block_exclusive_scan(v, &t);
+  return t;
+}
+
+__global__ void __launch_bounds__(1024)
+    permute_scan(int32_t* __restrict__ hist, int nblk, int N, int C, int32_t* __restrict__ counts,
+                 int32_t* __restrict__ offsets, int32_t* __restrict__ overflow,
+                 int32_t* __restrict__ totals) {
+  const int e = threadIdx.x;
+  int L = 0;
+  if (e < N) {
+    for (int b = 0; b < nblk; ++b) {
+      const int v = hist[(size_t)b * N + e];
+      hist[(size_t)b * N + e] = L;
+      L += v;
+    }
+  }
+  const int kept = e < N ? ((C > 0 && L > C) ? C : L) : 0;
+  const int of = (e < N && C > 0 && L > C) ? L - C : 0;
+  const int empty = (e < N && C > 0 && L < C) ? C - L : 0;
+  int kept_total = 0;
+  const int off = block_exclusive_scan(kept, &kept_total);
+  const int of_total = block_sum(of);
+  const int empty_total = block_sum(empty);
+  if (e < N) {
+    counts[e] = L;
+    offsets[e] = off;
+    overflow[e] = of;
+  }
+  if (e == 0) {
+    offsets[N] = kept_total;
+    totals[0] = kept_total;
+    totals[1] = of_total;
+    totals[2] = empty_total;
+  }
+}
+
+__global__ void __launch_bounds__(kChunk)
+    permute_scatter(const int32_t* __restrict__ idx, int64_t total, int k, int N, int C,
+                    const int32_t* __restrict__ base, const int32_t* __restrict__ offsets,
+                    int32_t* __restrict__ perm_tok, int32_t* __restrict__ row_of) {
+  extern __shared__ int32_t wcnt[];  // [8][N]
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  for (int i = threadIdx.x; i < 8 * N; i += kChunk) wcnt[i] = 0;
+  const int64_t x = (int64_t)blockIdx.x * kChunk + threadIdx.x;
+  int e = -1;
+  if (x < total) {
+    e = idx[x];
+    if (e < 0 || e >= N) e = -1;  // counted as an error by permute_hist
+  }
+  const unsigned peers = __match_any_sync(0xffffffffu, e);
+  const int in_warp = __popc(peers & ((1u << lane) - 1u));
+  __syncthreads();
+  if (e >= 0 && in_warp == 0) wcnt[w * N + e] = __popc(peers);
+  __syncthreads();
+  if (x >= total) return;
+  if (e < 0) {
+    row_of[x] = -1;
+    return;
+  }
+  int cross = 0;
+  for (int v = 0; v < w; ++v) cross += wcnt[v * N + e];
+  const int rank = base[(size_t)blockIdx.x * N + e] + cross + in_warp;
+  if (C > 0 && rank >= C) {
+    row_of[x] = -1;
+  } else {
+    const int r = offsets[e] + rank;
+    row_of[x] = r;
+    perm_tok[r] = (int32_t)(x / k);
+  }
+}
+
+}  // namespace
+
+size_t permute_ws_bytes(const moe_shape& s) {
+  const int64_t total = (int64_t)s.T * s.k;
+  const int64_t nblk = (total + kChunk - 1) / kChunk;
+  return align_up((size_t)(nblk > 0 ? nblk : 1) * s.N * 4, 256);
+}
+
+int launch_permute(const moe_shape& s, const int32_t* top_idx, int32_t* counts, int32_t* offsets,
+                   int32_t* perm_tok, int32_t* row_of, int32_t* overflow, int32_t* totals,
+                   void* ws, cudaStream_t st) {
+  const int64_t total = (int64_t)s.T * s.k;
+  const int nblk = (int)((total + kChunk - 1) / kChunk);
+  int32_t* hist = static_cast<int32_t*>(ws);
+  if (nblk > 0) {
+    permute_hist<<<nblk, kChunk, (size_t)s.N * 4, st>>>(top_idx, total, s.N, hist, status_word());
+  }
+  permute_scan<<<1, 1024, 0, st>>>(hist, nblk, s.N, s.capacity, counts, offsets, overflow, totals);
+  if (nblk > 0) {
+    permute_scatter<<<nblk, kChunk, (size_t)s.N * 8 * 4, st>>>(top_idx, total, s.k, s.N,
+                                                               s.capacity, hist, offsets,
+                                                               perm_tok, row_of);
+  }
+  return launch_status();
+}
+
+}  // namespace moe
+
+extern "C" size_t moe_permute_workspace_bytes(const moe_shape* shape) {
+  if (!moe::shape_ok(shape)) return 0;
+  return moe::permute_ws_bytes(*shape);
+}
+
+extern "C" int moe_permute(const moe_shape* shape, const int32_t* top_idx, int32_t* counts,
+                           int32_t* offsets, int32_t* perm_tok, int32_t* row_of,
+                           int32_t* overflow, int32_t* totals, void* ws, size_t ws_bytes,
+                           void* stream) {
+  using namespace moe;
+  if (!shape_ok(shape)) return MOE_ERR_INVALID_ARG;
+  if (!counts || !offsets || !overflow || !totals) return MOE_ERR_INVALID_ARG;
+  if (shape->T > 0 && (!top_idx || !perm_tok || !row_of)) return MOE_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < permute_ws_bytes(*shape)) return MOE_ERR_WORKSPACE;
+  return launch_permute(*shape, top_idx, counts, offsets, perm_tok, row_of, overflow, totals, ws,
+                        as_stream(stream));
+}

@@ -1,0 +1,234 @@
+// Router: logits z = W_route u (+ b), softmax, top-k, combine weights.
+// Tutorial "Mixture of Experts MoE: how sparse activation saves compute", §3.2
+// (equations z, p, a); the router runs in fp32 as its code's softmax of
+// logits.float() does.
+//
+// Logits are a register-tiled SIMT GEMM: each thread owns TM tokens x TN
+// experts and walks the input dimension in ascending order with one fused
+// multiply-add per step, so every logit is the same sequential fp32 chain
+// whatever the tiling (the reproducible order the routing decision needs).
+// Top-k runs one warp per token with the logits in registers.
+#include <cfloat>
+#include <climits>
+
+#include "common.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kBK = 32;
+
+template <int BT, int BN, int TM, int TN, typename TU>
+__global__ void __launch_bounds__((BT / TM) * (BN / TN))
+    router_logits_kernel(const TU* __restrict__ u, const float* __restrict__ w,
+                         const float* __restrict__ bias, float* __restrict__ z, int T, int d,
+                         int N) {
+  constexpr int NT = (BT / TM) * (BN / TN);
+  __shared__ __align__(16) float us[kBK][BT];
+  __shared__ __align__(16) float wsm[kBK][BN];
+  const int t0 = blockIdx.x * BT, n0 = blockIdx.y * BN;
+  const int tid = threadIdx.x;
+  const int tx = tid % (BN / TN);
+  const int ty = tid / (BN / TN);
+  float acc[TM][TN];
+#pragma unroll
+  for (int i = 0; i < TM; ++i)
+#pragma unroll
+    for (int j = 0; j < TN; ++j) acc[i][j] = 0.0f;
+
+  for (int k0 = 0; k0 < d; k0 += kBK) {
+    const int kw = min(kBK, d - k0);  // multiple of 8
+    for (int v = tid; v < BT * (kBK / 8); v += NT) {
+      const int r = v / (kBK / 8), c8 = (v % (kBK / 8)) * 8;
+      float tmp[8];
+      if (t0 + r < T && c8 < kw) {
+        load8(u + (size_t)(t0 + r) * d + k0 + c8, tmp);
+      } else {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) tmp[j] = 0.0f;
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j) us[c8 + j][r] = tmp[j];
+    }
+    for (int v = tid; v < BN * (kBK / 8); v += NT) {
+      const int r = v / (kBK / 8), c8 = (v % (kBK / 8)) * 8;
+      float tmp[8];
+      if (n0 + r < N && c8 < kw) {
+        load8(w + (size_t)(n0 + r) * d + k0 + c8, tmp);
+      } else {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) tmp[j] = 0.0f;
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j) wsm[c8 + j][r] = tmp[j];
+    }
+    __syncthreads();
+    for (int kk = 0; kk < kw; ++kk) {
+      float a[TM], b[TN];
+#pragma unroll
+      for (int i = 0; i < TM; ++i) a[i] = us[kk][ty * TM + i];
+#pragma unroll
+      for (int j = 0; j < TN; ++j) b[j] = wsm[kk][tx * TN + j];
+#pragma unroll
+      for (int i = 0; i < TM; ++i)
+#pragma unroll
+        for (int j = 0; j < TN; ++j) acc[i][j] = __fmaf_rn(b[j], a[i], acc[i][j]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < TM; ++i) {
+    const int t = t0 + ty * TM + i;
+    if (t >= T) continue;
+#pragma unroll
+    for (int j = 0; j < TN; ++j) {
+      const int n = n0 + tx * TN + j;
+      if (n < N) z[(size_t)t * N + n] = bias ? __fadd_rn(acc[i][j], bias[n]) : acc[i][j];
+    }
+  }
+}
+
+// (z, index) ordering of the top-k: larger z first, equal z -> lower index.
+__device__ __forceinline__ bool better(float za, int ia, float zb, int ib) {
+  return za > zb || (za == zb && ia < ib);
+}
+
+template <int PER>
+__global__ void __launch_bounds__(256)
+    router_topk_kernel(const float* __restrict__ z, int T, int N, int k, int renorm,
+                       int32_t* __restrict__ top_idx, float* __restrict__ top_w,
+                       float* __restrict__ probs) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (warp >= T) return;
+  const float* zt = z + (size_t)warp * N;
+  float zr[PER];
+  float zmax = -FLT_MAX;
+#pragma unroll
+  for (int q = 0; q < PER; ++q) {
+    const int j = lane + 32 * q;
+    zr[q] = j < N ? zt[j] : -FLT_MAX;
+    zmax = fmaxf(zmax, zr[q]);
+  }
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) zmax = fmaxf(zmax, __shfl_xor_sync(0xffffffffu, zmax, o));
+  float den = 0.0f;
+#pragma unroll
+  for (int q = 0; q < PER; ++q) {
+    const int j = lane + 32 * q;
+    if (j < N) den += expf(zr[q] - zmax);
+  }
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+  if (probs) {
+    float* pt = probs + (size_t)warp * N;
+#pragma unroll
+    for (int q = 0; q < PER; ++q) {
+      const int j = lane + 32 * q;
+      if (j < N) pt[j] = expf(zr[q] - zmax) / den;
+    }
+  }
+  uint32_t taken = 0;
+  float my_z = -FLT_MAX;
+  int my_i = INT_MAX;
+  for (int s = 0; s < k; ++s) {
+    float bz = -FLT_MAX;
+    int bi = INT_MAX;
+#pragma unroll
+    for (int q = 0; q < PER; ++q) {
+      const int j = lane + 32 * q;
+      if (j < N && !((taken >> q) & 1u) && better(zr[q], j, bz, bi)) {
+        bz = zr[q];
+        bi = j;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) {
+      const float oz = __shfl_xor_sync(0xffffffffu, bz, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      if (better(oz, oi, bz, bi)) {
+        bz = oz;
+        bi = oi;
+      }
+    }
+    if (bi != INT_MAX && (bi & 31) == lane) taken |= 1u << (bi >> 5);
+    if (lane == s) {
+      my_z = bz;
+      my_i = bi;
+    }
+  }
+  const float p = lane < k ? expf(my_z - zmax) / den : 0.0f;
+  float ps = p;
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, o);
+  if (lane < k) {
+    top_idx[(size_t)warp * k + lane] = my_i;
+    top_w[(size_t)warp * k + lane] = renorm ? p / ps : p;
+  }
+}
+
+template <typename TU>
+void launch_logits(const TU* u, const float* w, const float* bias, float* z, int T, int d, int N,
+                   cudaStream_t st) {
+  if (N <= 8) {
+    dim3 grid((T + 63) / 64, 1);
+    router_logits_kernel<64, 8, 2, 4, TU><<<grid, 64, 0, st>>>(u, w, bias, z, T, d, N);
+  } else if (N <= 16) {
+    dim3 grid((T + 63) / 64, 1);
+    router_logits_kernel<64, 16, 4, 4, TU><<<grid, 64, 0, st>>>(u, w, bias, z, T, d, N);
+  } else {
+    dim3 grid((T + 63) / 64, (N + 63) / 64);
+    router_logits_kernel<64, 64, 4, 4, TU><<<grid, 256, 0, st>>>(u, w, bias, z, T, d, N);
+  }
+}
+
+}  // namespace
+
+size_t route_ws_bytes(const moe_shape& s) { return align_up((size_t)s.T * s.N * 4, 256); }
+
+int launch_route(const moe_shape& s, const void* u, int32_t u_dtype, const float* w_route,
+                 const float* bias, int32_t* top_idx, float* top_w, float* probs, float* logits,
+                 void* ws, cudaStream_t st) {
+  if (s.T == 0) return MOE_OK;
+  float* z = logits ? logits : static_cast<float*>(ws);
+  if (u_dtype == MOE_F32) {
+    launch_logits(static_cast<const float*>(u), w_route, bias, z, s.T, s.d, s.N, st);
+  } else if (u_dtype == MOE_BF16) {
+    launch_logits(static_cast<const __nv_bfloat16*>(u), w_route, bias, z, s.T, s.d, s.N, st);
+  } else {
+    launch_logits(static_cast<const __half*>(u), w_route, bias, z, s.T, s.d, s.N, st);
+  }
+  const int blocks = (s.T + 7) / 8;
+  const int per = (s.N + 31) / 32;
+#define MOE_TOPK(P)                                                                          \
+  router_topk_kernel<P><<<blocks, 256, 0, st>>>(z, s.T, s.N, s.k, s.renorm, top_idx, top_w, \
+                                                probs)
+  if (per <= 1) MOE_TOPK(1);
+  else if (per <= 2) MOE_TOPK(2);
+  else if (per <= 4) MOE_TOPK(4);
+  else if (per <= 8) MOE_TOPK(8);
+  else if (per <= 16) MOE_TOPK(16);
+  else MOE_TOPK(32);
+#undef MOE_TOPK
+  return launch_status();
+}
+
+}  // namespace moe
+
+extern "C" size_t moe_route_workspace_bytes(const moe_shape* shape) {
+  if (!moe::shape_ok(shape)) return 0;
+  return moe::route_ws_bytes(*shape);
+}
+
+extern "C" int moe_route(const moe_shape* shape, const void* u, int32_t u_dtype,
+                         const float* w_route, const float* bias, int32_t* top_idx, float* top_w,
+                         float* probs, float* logits, void* ws, size_t ws_bytes, void* stream) {
+  using namespace moe;
+  if (!shape_ok(shape) || !valid_act_dtype(u_dtype)) return MOE_ERR_INVALID_ARG;
+  if (shape->T > 0 && (!u || !w_route || !top_idx || !top_w)) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(u) || !aligned16(w_route)) return MOE_ERR_INVALID_ARG;
+  if (!logits && shape->T > 0 && (!ws || ws_bytes < route_ws_bytes(*shape)))
+    return MOE_ERR_WORKSPACE;
+  return launch_route(*shape, u, u_dtype, w_route, bias, top_idx, top_w, probs, logits, ws,
+                      as_stream(stream));
+}

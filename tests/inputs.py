@@ -1,0 +1,96 @@
+"""Workload inputs for the parity tests, drawn from the shared seeded generator.
+
+Device tensors come from the generator's CUDA implementation, host arrays from
+its C implementation; the two are bit-identical (checked in the GPU tests).
+Nothing here computes any part of the MoE layer.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+import oracle as O
+import synthetic as S
+from synthetic import workloads as W
+
+TORCH_OF = {S.DT_F32: "float32", S.DT_BF16: "bfloat16", S.DT_F16: "float16"}
+ORACLE_DT = {S.DT_F32: O.F32, S.DT_BF16: O.BF16, S.DT_F16: O.F16}
+
+
+def torch_dtype(code):
+    import torch
+    return getattr(torch, TORCH_OF[code])
+
+
+def dev_normal(seed, tid, shape, sigma, dtype, device="cuda", offset=0):
+    import torch
+    t = torch.empty(shape, dtype=torch_dtype(dtype), device=device)
+    S.normal_dev(seed, tid, t.numel(), sigma, dtype, t.data_ptr(),
+                 torch.cuda.current_stream().cuda_stream, offset)
+    return t
+
+
+def dev_u(wl: W.Workload, T=None, device="cuda"):
+    import torch
+    T = wl.T if T is None else T
+    if wl.rms_inputs:
+        t = torch.empty((T, wl.d), dtype=torch_dtype(wl.act_dtype), device=device)
+        S.rmsnorm_rows_dev(wl.seed, W.TID_U, T, wl.d, wl.act_dtype, t.data_ptr(),
+                           torch.cuda.current_stream().cuda_stream)
+        return t
+    return dev_normal(wl.seed, W.TID_U, (T, wl.d), wl.u_sigma, wl.act_dtype, device)
+
+
+def host_u(wl: W.Workload, T=None):
+    T = wl.T if T is None else T
+    if wl.rms_inputs:
+        return S.rmsnorm_rows(wl.seed, W.TID_U, T, wl.d, wl.act_dtype)
+    return S.normal(wl.seed, W.TID_U, (T, wl.d), wl.u_sigma, wl.act_dtype)
+
+
+def dev_router(wl: W.Workload, device="cuda", layer=0):
+    import torch
+    w = dev_normal(wl.seed, W.tid(W.TID_WROUTE, layer), (wl.N, wl.d), W.SIGMA_W, S.DT_F32, device)
+    b = wl.router_bias()
+    return w, (None if b is None else torch.from_numpy(b).to(device))
+
+
+def host_router(wl: W.Workload, layer=0):
+    return (S.normal(wl.seed, W.tid(W.TID_WROUTE, layer), (wl.N, wl.d), W.SIGMA_W, S.DT_F32),
+            wl.router_bias())
+
+
+def dev_experts(wl: W.Workload, device="cuda"):
+    """W_gate [N][h][w], W_up [N][h][w], W_down [N][w][h] with w the expert width."""
+    w, h, N = wl.expert_in, wl.h, wl.N
+    dt = W.w_storage(wl)
+    return (dev_normal(wl.seed, W.TID_WGATE, (N, h, w), W.SIGMA_W, dt, device),
+            dev_normal(wl.seed, W.TID_WUP, (N, h, w), W.SIGMA_W, dt, device),
+            dev_normal(wl.seed, W.TID_WDOWN, (N, w, h), W.SIGMA_W, dt, device))
+
+
+def host_expert(wl: W.Workload, e: int):
+    """Oracle matrices of expert e, drawn directly at that expert's offset."""
+    w, h = wl.expert_in, wl.h
+    dt = W.w_storage(wl)
+    od = ORACLE_DT[dt]
+    g = S.normal(wl.seed, W.TID_WGATE, (h, w), W.SIGMA_W, dt, offset=e * h * w)
+    u = S.normal(wl.seed, W.TID_WUP, (h, w), W.SIGMA_W, dt, offset=e * h * w)
+    d = S.normal(wl.seed, W.TID_WDOWN, (w, h), W.SIGMA_W, dt, offset=e * w * h)
+    return O.Mat(od, h, w, data=g), O.Mat(od, h, w, data=u), O.Mat(od, w, h, data=d)
+
+
+def to_numpy_codes(t):
+    """Raw storage of a device tensor: uint16 codes for 16-bit types, else values."""
+    import torch
+    c = t.detach().cpu()
+    if c.dtype in (torch.bfloat16, torch.float16):
+        return c.view(torch.int16).numpy().view(np.uint16)
+    return c.numpy()
+
+
+def rel_err(got, ref):
+    """max |got - ref| / rms(ref), the layer's output tolerance measure."""
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    rms = float(np.sqrt(np.mean(ref * ref)))
+    return float(np.max(np.abs(got - ref))) / (rms if rms > 0 else 1.0)

@@ -1,0 +1,111 @@
+"""The C-ABI boundary without a GPU: the library loads, exports every entry
+point include/*.h declares, the Python binding covers them, and host-side
+argument checks reject bad calls before any device work."""
+import ctypes
+import glob
+import os
+import re
+import subprocess
+
+import pytest
+
+from conftest import ROOT
+
+import sparse_mixture_experts_15_b200 as moe
+
+
+def _declared():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        txt = open(h).read()
+        names |= set(re.findall(r"MOE_API\s+[\w\s\*]*?\b(moe_\w+)\s*\(", txt))
+    return sorted(names)
+
+
+def test_header_declares_entry_points():
+    names = _declared()
+    for required in ("moe_route", "moe_permute", "moe_expert_ffn", "moe_combine",
+                     "moe_layer_fwd", "moe_aux_stats", "moe_gather", "moe_capacity"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol():
+    out = subprocess.run(["nm", "-D", "--defined-only", moe.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = {ln.split()[-1] for ln in out.splitlines() if " T " in ln}
+    missing = [n for n in _declared() if n not in exported]
+    assert not missing, missing
+    lib = ctypes.CDLL(moe.LIB_PATH)
+    for n in _declared():
+        assert getattr(lib, n) is not None
+
+
+def test_binding_covers_every_symbol():
+    assert set(_declared()) <= set(moe.EXPORTED)
+
+
+def test_capacity_host_only():
+    """Tutorial §3.5: C = ceil(c * dispatches / N)."""
+    assert moe.moe_capacity(16, 4, 1, 1.0) == 4
+    assert moe.moe_capacity(16, 4, 1, 1.5) == 6
+    assert moe.moe_capacity(16, 4, 1, 2.5) == 10
+    assert moe.moe_capacity(8192, 8, 2, 1.25) == 2560
+    assert moe.moe_capacity(100, 8, 2, 0.0) == 0
+    with pytest.raises(moe.MoeError):
+        moe.moe_capacity(-1, 8, 2, 1.0)
+
+
+def test_status_strings():
+    assert moe.status_string(0) == "MOE_OK"
+    for code in range(-1, -7, -1):
+        assert moe.status_string(code).startswith("MOE_ERR_")
+
+
+def test_host_rejects_bad_shapes_before_device_work():
+    lib = moe._lib
+    bad = [moe.shape(16, 63, 4, 2, 128),   # d % 8 != 0
+           moe.shape(16, 64, 4, 5, 128),   # k > N
+           moe.shape(16, 64, 0, 1, 128),   # N = 0
+           moe.shape(16, 64, 2000, 2, 128),  # N > 1024
+           moe.shape(16, 64, 64, 33, 128)]   # k > 32
+    for s in bad:
+        assert lib.moe_route_workspace_bytes(ctypes.byref(s)) == 0
+        rc = lib.moe_route(ctypes.byref(s), None, 1, None, None, None, None, None, None, None, 0,
+                           None)
+        assert rc == -1
+        rc = lib.moe_permute(ctypes.byref(s), None, None, None, None, None, None, None, None, 0,
+                             None)
+        assert rc == -1
+
+
+def test_host_rejects_null_and_misaligned_pointers():
+    lib = moe._lib
+    s = moe.shape(16, 64, 4, 2, 128)
+    # null outputs
+    assert lib.moe_route(ctypes.byref(s), 4096, 0, 8192, None, None, None, None, None, None, 0,
+                         None) == -1
+    # misaligned activation pointer
+    assert lib.moe_route(ctypes.byref(s), 4098, 0, 8192, None, 12288, 16384, None, None, 20480,
+                         1 << 20, None) == -1
+    # workspace too small
+    assert lib.moe_route(ctypes.byref(s), 4096, 0, 8192, None, 12288, 16384, None, None, 20480,
+                         16, None) == -6
+    # unsupported expert dtype combination (fp32 activations, bf16 weights)
+    a = moe.act()
+    assert lib.moe_expert_ffn(ctypes.byref(s), 64, 4096, 0, 4096, 4096, 4096, 4096, 1,
+                              ctypes.byref(a), 4096, None, 0, None) == -2
+    # SiTU-GLU needs positive caps
+    a2 = moe.act(moe.ACT_SITU_GLU, 0.0, 25.0)
+    assert lib.moe_expert_ffn(ctypes.byref(s), 64, 4096, 1, 4096, 4096, 4096, 4096, 1,
+                              ctypes.byref(a2), 4096, None, 0, None) == -1
+
+
+def test_workspace_queries_are_host_only_and_monotone():
+    lib = moe._lib
+    small = moe.shape(1024, 512, 8, 2, 128)
+    big = moe.shape(8192, 512, 8, 2, 128)
+    for q in (lambda s: lib.moe_route_workspace_bytes(ctypes.byref(s)),
+              lambda s: lib.moe_permute_workspace_bytes(ctypes.byref(s)),
+              lambda s: lib.moe_layer_workspace_bytes(ctypes.byref(s), 1),
+              lambda s: lib.moe_expert_ffn_workspace_bytes(ctypes.byref(s), 512, 1)):
+        assert 0 < q(small) <= q(big)

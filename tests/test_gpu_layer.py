@@ -1,0 +1,190 @@
+"""GPU parity of the expert FFN and the whole layer forward against the CPU
+oracle, through the C ABI.  Tolerances (max|d|/rms(y)): 1e-4 for fp32
+layers, 2e-2 for bf16; routing, counts, permutation and overflow bit-exact."""
+import numpy as np
+import pytest
+
+import oracle as O
+import synthetic as S
+from synthetic import workloads as W
+
+from inputs import (dev_experts, dev_normal, dev_router, dev_u, host_expert, host_router, host_u,
+                    to_numpy_codes, ORACLE_DT, rel_err)
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+TOL_F32, TOL_BF16 = 1e-4, 2e-2
+
+if torch.cuda.is_available():
+    import sparse_mixture_experts_15_b200 as moe
+
+
+@pytest.fixture(autouse=True)
+def _clean_status():
+    moe.moe_reset_device_status()
+    yield
+    assert moe.moe_device_status() == 0
+
+
+def _ragged_offsets(counts):
+    return np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+
+
+def _ffn_case(counts, width, h, dtype, act_kind=0, x_sigma=1.0, sample=None, seed=21):
+    """Expert FFN on synthetic grouped rows with the given per-expert counts."""
+    N = len(counts)
+    R = int(sum(counts))
+    off = _ragged_offsets(counts)
+    s = moe.shape(R, width, N, 1, h, 1, 0)  # T*k = R rows of room
+    Tk = s.T * s.k
+    xr = dev_normal(seed, 1, (Tk, width), x_sigma, dtype)
+    wg = dev_normal(seed, 3, (N, h, width), W.SIGMA_W, dtype)
+    wu = dev_normal(seed, 4, (N, h, width), W.SIGMA_W, dtype)
+    wd = dev_normal(seed, 5, (N, width, h), W.SIGMA_W, dtype)
+    yr = torch.full((Tk, width), float("nan"), dtype=torch.float32, device="cuda")
+    a = moe.act(act_kind, 4.0, 25.0)
+    moe.moe_expert_ffn(s, width, xr, torch.from_numpy(off).cuda(), wg, wu, wd, yr, a)
+    torch.cuda.synchronize()
+    got = yr.cpu().numpy()
+    od = ORACLE_DT[dtype]
+    xh = O.decode(od, S.normal(seed, 1, (Tk, width), x_sigma, dtype))
+    rows = np.arange(R) if sample is None else np.sort(
+        np.random.default_rng(0).choice(R, min(sample, R), replace=False))
+    ref = np.empty((len(rows), width))
+    mats = {}
+    for i, r in enumerate(rows):
+        e = int(np.searchsorted(off, r, side="right") - 1)
+        if e not in mats:
+            g = S.normal(seed, 3, (h, width), W.SIGMA_W, dtype, offset=e * h * width)
+            u = S.normal(seed, 4, (h, width), W.SIGMA_W, dtype, offset=e * h * width)
+            d = S.normal(seed, 5, (width, h), W.SIGMA_W, dtype, offset=e * width * h)
+            mats[e] = (O.Mat(od, h, width, data=g), O.Mat(od, h, width, data=u),
+                       O.Mat(od, width, h, data=d))
+        ref[i] = O.expert(*mats[e], xh[r], act=act_kind, beta_g=4.0, beta_u=25.0,
+                          round_h=int(dtype == S.DT_BF16))
+    return got[rows], ref
+
+
+def test_expert_ffn_f32_simt():
+    got, ref = _ffn_case([3, 0, 9, 4], 64, 128, S.DT_F32, x_sigma=0.02)
+    assert rel_err(got, ref) < TOL_F32
+
+
+@pytest.mark.parametrize("counts,width,h", [
+    ([16], 128, 64),                                   # one tile, smallest shapes
+    ([0, 5, 130, 257, 16, 1, 300, 64], 512, 256),      # ragged tails, empty expert
+    ([1024] * 8, 512, 128),                            # the small-model layer's shape
+    ([700, 333, 1500, 410], 512, 1024),                # 256-token tiles
+])
+def test_expert_ffn_bf16_tensor_cores(counts, width, h):
+    got, ref = _ffn_case(counts, width, h, S.DT_BF16, sample=600)
+    assert np.all(np.isfinite(got))
+    assert rel_err(got, ref) < TOL_BF16
+
+
+def test_expert_ffn_bf16_situ_glu_soft_caps():
+    """SiTU-GLU epilogue with inputs large enough for the caps to bind."""
+    got, ref = _ffn_case([100, 37, 260], 256, 192, S.DT_BF16, act_kind=1, x_sigma=20.0)
+    assert rel_err(got, ref) < TOL_BF16
+
+
+# --------------------------------------------------------------- full layer
+def _layer_gpu(wl, outputs=True):
+    T = wl.T
+    s = moe.shape(T, wl.d, wl.N, wl.k, wl.h, wl.renorm, wl.capacity())
+    u = dev_u(wl)
+    w, b = dev_router(wl)
+    wg, wu, wd = dev_experts(wl)
+    y = torch.empty((T, wl.d), dtype=u.dtype, device="cuda")
+    outs = {}
+    if outputs:
+        i32 = dict(dtype=torch.int32, device="cuda")
+        outs = dict(top_idx=torch.empty((T, wl.k), **i32),
+                    top_w=torch.empty((T, wl.k), dtype=torch.float32, device="cuda"),
+                    counts=torch.empty(wl.N, **i32), offsets=torch.empty(wl.N + 1, **i32),
+                    row_of=torch.empty((T, wl.k), **i32), overflow=torch.empty(wl.N, **i32),
+                    totals=torch.empty(3, **i32))
+    moe.moe_layer_fwd(s, w, wg, wu, wd, u, y, bias=b, outputs=outs)
+    torch.cuda.synchronize()
+    return y, {k: v.cpu().numpy() for k, v in outs.items()}
+
+
+def _layer_oracle(wl, tokens):
+    u_codes = host_u(wl)
+    od = ORACLE_DT[wl.act_dtype]
+    w, b = host_router(wl)
+    _, probs, idx, tw = O.route(O.as_f32(od, u_codes), w, wl.k, wl.renorm, b)
+    perm = O.permute(idx, wl.N, wl.capacity())
+    mats = [host_expert(wl, e) for e in range(wl.N)]
+    y = O.moe_tokens([m[0] for m in mats], [m[1] for m in mats], [m[2] for m in mats],
+                     O.decode(od, u_codes), idx, tw, row_of=perm["row_of"], tokens=tokens,
+                     round_h=int(wl.act_dtype == S.DT_BF16))
+    return y, idx, tw, perm
+
+
+def _check_routing(outs, idx, tw, perm):
+    assert np.array_equal(outs["top_idx"], idx)
+    assert np.allclose(outs["top_w"], tw, rtol=2e-6, atol=1e-7)
+    for key in ("counts", "offsets", "row_of", "overflow"):
+        assert np.array_equal(outs[key], perm[key]), key
+    assert np.array_equal(outs["totals"], perm["totals"].astype(np.int32))
+
+
+def test_layer_tiny_fp32():
+    wl = W.tiny()
+    y, outs = _layer_gpu(wl)
+    ref, idx, tw, perm = _layer_oracle(wl, np.arange(wl.T, dtype=np.int32))
+    _check_routing(outs, idx, tw, perm)
+    assert rel_err(y.cpu().numpy(), ref) < TOL_F32
+    # brute force: all experts on every token, unselected weighted by zero
+    od = ORACLE_DT[wl.act_dtype]
+    mats = [host_expert(wl, e) for e in range(wl.N)]
+    dense = O.moe_dense([m[0] for m in mats], [m[1] for m in mats], [m[2] for m in mats],
+                        O.decode(od, host_u(wl)), idx, tw)
+    assert rel_err(y.cpu().numpy(), dense) < TOL_F32
+
+
+def test_layer_small_bf16_full():
+    wl = W.small()
+    y, outs = _layer_gpu(wl)
+    tokens = np.arange(wl.T, dtype=np.int32)
+    ref, idx, tw, perm = _layer_oracle(wl, tokens)
+    _check_routing(outs, idx, tw, perm)
+    assert outs["counts"].sum() == wl.k * wl.T
+    assert rel_err(y.float().cpu().numpy(), ref) < TOL_BF16
+
+
+def test_layer_small_bf16_ragged_T():
+    wl = W.small(T=777)
+    y, outs = _layer_gpu(wl)
+    ref, idx, tw, perm = _layer_oracle(wl, np.arange(wl.T, dtype=np.int32))
+    _check_routing(outs, idx, tw, perm)
+    assert rel_err(y.float().cpu().numpy(), ref) < TOL_BF16
+
+
+def test_layer_mixtral_full_size_sampled():
+    """Mixtral-shaped layer at full size with Zipf-skewed loads and capacity
+    1.25: routing, overflow and totals bit-exact on all 8192 tokens, outputs on
+    sampled tokens (including tokens with a dropped slot)."""
+    wl = W.mixtral()
+    y, outs = _layer_gpu(wl)
+    u_codes = host_u(wl)
+    od = ORACLE_DT[wl.act_dtype]
+    w, b = host_router(wl)
+    _, probs, idx, tw = O.route(O.as_f32(od, u_codes), w, wl.k, wl.renorm, b)
+    perm = O.permute(idx, wl.N, wl.capacity())
+    _check_routing(outs, idx, tw, perm)
+    assert int(perm["totals"][1]) > 0, "the skewed loads should overflow the capacity"
+    rng = np.random.default_rng(3)
+    dropped = np.where((perm["row_of"] < 0).any(1))[0]
+    tokens = np.sort(np.concatenate([rng.choice(wl.T, 12, replace=False),
+                                     rng.choice(dropped, min(4, len(dropped)), replace=False)]))
+    tokens = np.unique(tokens).astype(np.int32)
+    mats = [host_expert(wl, e) for e in range(wl.N)]
+    ref = O.moe_tokens([m[0] for m in mats], [m[1] for m in mats], [m[2] for m in mats],
+                       O.decode(od, u_codes[tokens]), idx[tokens], tw[tokens],
+                       row_of=perm["row_of"][tokens], tokens=np.arange(len(tokens), dtype=np.int32),
+                       round_h=1)
+    got = y[torch.from_numpy(tokens).long().cuda()].float().cpu().numpy()
+    assert rel_err(got, ref) < TOL_BF16

@@ -352,6 +352,28 @@ def test_dropped_dispatch_contributes_nothing():
     assert np.all(y[4:] == 0.0) and np.all(np.abs(y[:4]).sum(1) > 0)
 
 
+def test_combine_of_expert_rows_equals_sparse_layer():
+    """Grouping rows by expert, running experts per row and combining by row_of
+    gives the token-wise sparse layer (§3.6: split into [L_i, d], add back)."""
+    T, d, h, N, k, C = 20, 8, 12, 4, 2, 7
+    Wg = [_rand_mat(h, d) for _ in range(N)]
+    Wu = [_rand_mat(h, d) for _ in range(N)]
+    Wd = [_rand_mat(d, h) for _ in range(N)]
+    u = RNG.standard_normal((T, d))
+    W_route = RNG.standard_normal((N, d)).astype(np.float32)
+    _, _, idx, w = O.route(u.astype(np.float32), W_route, k)
+    out = O.permute(idx, N, C)
+    rows = np.zeros((len(out["perm_tok"]), d))
+    for e in range(N):
+        for r in range(out["offsets"][e], out["offsets"][e + 1]):
+            rows[r] = O.expert(Wg[e], Wu[e], Wd[e], u[out["perm_tok"][r]])
+    y = O.combine(rows, out["row_of"], w)
+    ref = O.moe_tokens(Wg, Wu, Wd, u, idx, w, row_of=out["row_of"])
+    assert np.allclose(y, ref, rtol=1e-13, atol=1e-15)
+    # a dropped slot adds nothing; an all-dropped token is exactly zero
+    assert np.all(O.combine(rows, -np.ones((T, k), np.int32), w) == 0.0)
+
+
 def test_q4_expert_equals_dequantised_f64():
     """Per-GEMV emulation with the same quantised weights (deployment notes §6)."""
     d, h = 64, 32
