@@ -327,10 +327,12 @@ def main():
     if sampler:
         sampler.start()
         time.sleep(0.3)
+    torch.cuda.nvtx.range_push("timed")
     t_start.record(stream)
     for i in range(args.steps):
         step(reps[i % n_rep], ev[i])
     t_stop.record(stream)
+    torch.cuda.nvtx.range_pop()
     torch.cuda.synchronize()
     if dist:
         dist.barrier()

@@ -237,7 +237,11 @@ def test_combine_vs_oracle(y_dtype):
                     torch.from_numpy(tw).cuda(), y)
     ref = O.combine(yr[:rows].astype(np.float64), p["row_of"], tw.astype(np.float64))
     got = y.float().cpu().numpy()
-    tol = 1e-6 if y_dtype == S.DT_F32 else 8e-3
-    assert rel_err(got, ref) < tol
+    if y_dtype == S.DT_F32:
+        assert rel_err(got, ref) < 1e-6
+    else:
+        # bf16 output: within the bf16 layers' 2e-2 and one bf16 ulp of each value
+        assert rel_err(got, ref) < 2e-2
+        assert np.all(np.abs(got - ref) <= np.abs(ref) * 2.0 ** -8 + 1e-6)
     dropped = np.all(p["row_of"] < 0, axis=1)
     assert np.all(got[dropped] == 0.0)
