@@ -139,6 +139,25 @@ MOE_API int moe_permute(const moe_shape* shape, const int32_t* top_idx, int32_t*
                 int32_t* offsets, int32_t* perm_tok, int32_t* row_of, int32_t* overflow,
                 int32_t* totals, void* ws, size_t ws_bytes, void* stream);
 
+/* Allocation-free moe_permute.  The pages have no counterpart: this entry
+ * point exists for callers that cannot allocate device memory when they call
+ * in (a C program that loads only this library and has no device allocator,
+ * or a framework whose memory planner forbids allocation at call time).
+ * Same arguments, results and errors as moe_permute, minus (ws, ws_bytes):
+ * the scratch is a fixed 1 MiB array inside the library, resident on every
+ * GPU that loads it until the process exits.  Limit: ceil(T*k / 256) * N
+ * <= 262144 (e.g. T*k = 65536 dispatches with N up to 1024 experts); larger
+ * problems return MOE_ERR_WORKSPACE before anything is launched.  The first
+ * call on a device looks up the array's device address (with that device
+ * current); make that first call before any stream capture.  All calls in
+ * the process share the one array, so calls whose work overlaps on the GPU
+ * (other streams, other host threads) race; serialise them.  Nothing in the
+ * array needs to start at zero: each call rewrites what it reads.  Never
+ * calls cudaMalloc, cudaFree or any allocating routine. */
+MOE_API int moe_permute_noalloc(const moe_shape* shape, const int32_t* top_idx, int32_t* counts,
+                                int32_t* offsets, int32_t* perm_tok, int32_t* row_of,
+                                int32_t* overflow, int32_t* totals, void* stream);
+
 /* ---------------------------------------------------------------- gather */
 /* x_rows[r] = u[perm_tok[r]] for r < offsets[N] (tutorial §3.6: expert i
  * receives its [L_i, d] rows).  u [T][width] in dtype; x_rows has room for

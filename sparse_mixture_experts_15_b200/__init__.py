@@ -54,6 +54,7 @@ _PROTOS = {
     "moe_aux_stats": (_i32, [_i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "moe_permute_workspace_bytes": (_sz, [_P_SHAPE]),
     "moe_permute": (_i32, [_P_SHAPE, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "moe_permute_noalloc": (_i32, [_P_SHAPE, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "moe_gather": (_i32, [_P_SHAPE, _i32, _vp, _i32, _vp, _vp, _vp, _vp]),
     "moe_expert_ffn_workspace_bytes": (_sz, [_P_SHAPE, _i32, _i32]),
     "moe_expert_ffn": (_i32, [_P_SHAPE, _i32, _vp, _i32, _vp, _vp, _vp, _vp, _i32,
@@ -151,6 +152,14 @@ def moe_permute(s: MoeShape, top_idx, counts, offsets, perm_tok, row_of, overflo
     _check(_lib.moe_permute(ctypes.byref(s), _ptr(top_idx), _ptr(counts), _ptr(offsets),
                             _ptr(perm_tok), _ptr(row_of), _ptr(overflow), _ptr(totals), _ptr(wbuf),
                             wlen, _stream(stream)), "moe_permute")
+
+
+def moe_permute_noalloc(s: MoeShape, top_idx, counts, offsets, perm_tok, row_of, overflow,
+                        totals, stream=None):
+    """moe_permute without a workspace (the library's fixed 1 MiB scratch)."""
+    _check(_lib.moe_permute_noalloc(ctypes.byref(s), _ptr(top_idx), _ptr(counts), _ptr(offsets),
+                                    _ptr(perm_tok), _ptr(row_of), _ptr(overflow), _ptr(totals),
+                                    _stream(stream)), "moe_permute_noalloc")
 
 
 def moe_gather(s: MoeShape, width: int, u, perm_tok, offsets, x_rows, stream=None):

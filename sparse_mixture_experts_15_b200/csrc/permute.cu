@@ -188,3 +188,49 @@ extern "C" int moe_permute(const moe_shape* shape, const int32_t* top_idx, int32
   return launch_permute(*shape, top_idx, counts, offsets, perm_tok, row_of, overflow, totals, ws,
                         as_stream(stream));
 }
+
+// ------------------------------------------------- allocation-free variant
+// Some callers cannot allocate device memory when they call in: a C program
+// that loads only this library and owns no device allocator, or a host
+// framework whose memory planner hands out every device byte in advance and
+// forbids allocation at call time.  moe_permute_noalloc serves them with the
+// same kernels as moe_permute, taking its block-count scratch from this fixed
+// array instead of a caller workspace.  Every GPU that loads the library
+// holds the array until the process exits.
+static __device__ __align__(256) int32_t g_permute_noalloc_scratch[262144];  // 1 MiB
+
+namespace moe {
+namespace {
+
+// Device address of the scratch array for the current device, looked up once
+// per device with that device current (in host code the array's name is only a
+// host-side stand-in and must not be handed to a kernel).
+int32_t* noalloc_scratch() {
+  static int32_t* addr[64] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  if (!addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_permute_noalloc_scratch) != cudaSuccess) return nullptr;
+    addr[dev] = static_cast<int32_t*>(p);
+  }
+  return addr[dev];
+}
+
+}  // namespace
+}  // namespace moe
+
+extern "C" int moe_permute_noalloc(const moe_shape* shape, const int32_t* top_idx,
+                                   int32_t* counts, int32_t* offsets, int32_t* perm_tok,
+                                   int32_t* row_of, int32_t* overflow, int32_t* totals,
+                                   void* stream) {
+  using namespace moe;
+  if (!shape_ok(shape)) return MOE_ERR_INVALID_ARG;
+  if (!counts || !offsets || !overflow || !totals) return MOE_ERR_INVALID_ARG;
+  if (shape->T > 0 && (!top_idx || !perm_tok || !row_of)) return MOE_ERR_INVALID_ARG;
+  if (permute_ws_bytes(*shape) > sizeof(g_permute_noalloc_scratch)) return MOE_ERR_WORKSPACE;
+  int32_t* scratch = noalloc_scratch();
+  if (!scratch) return MOE_ERR_CUDA;
+  return launch_permute(*shape, top_idx, counts, offsets, perm_tok, row_of, overflow, totals,
+                        scratch, as_stream(stream));
+}
