@@ -7,7 +7,8 @@
 // experts and walks the input dimension in ascending order with one fused
 // multiply-add per step, so every logit is the same sequential fp32 chain
 // whatever the tiling (the reproducible order the routing decision needs).
-// Top-k runs one warp per token with the logits in registers.
+// Top-k runs one warp per token with the logits in registers.  With at most
+// 16 experts a single fused kernel (router_fused_small) does all of it.
 #include <cfloat>
 #include <climits>
 
@@ -167,6 +168,93 @@ __global__ void __launch_bounds__(256)
   }
 }
 
+// Few experts (N <= NP <= 16): one thread per token keeps all N logits in
+// registers and finishes softmax, top-k and the combine weights itself, so
+// routing is a single launch.  W_route is staged in shared memory in slabs of
+// kSlab inputs as [j][NP] so every thread reads the same NP floats (broadcast).
+// Each logit is the same sequential FMA chain over j as in the tiled kernel.
+constexpr int kSlab = 512;
+
+template <int NP, typename TU>
+__global__ void __launch_bounds__(64)
+    router_fused_small(const TU* __restrict__ u, const float* __restrict__ w,
+                       const float* __restrict__ bias, int T, int d, int N, int k, int renorm,
+                       int32_t* __restrict__ top_idx, float* __restrict__ top_w,
+                       float* __restrict__ probs, float* __restrict__ logits) {
+  __shared__ __align__(16) float ws[kSlab][NP];
+  const int t = blockIdx.x * blockDim.x + threadIdx.x;
+  float acc[NP];
+#pragma unroll
+  for (int e = 0; e < NP; ++e) acc[e] = 0.0f;
+  for (int k0 = 0; k0 < d; k0 += kSlab) {
+    const int kw = min(kSlab, d - k0);
+    __syncthreads();
+    for (int i = threadIdx.x; i < kw * NP; i += blockDim.x) {
+      const int e = i / kw, j = i - e * kw;  // coalesced along j
+      ws[j][e] = e < N ? w[(size_t)e * d + k0 + j] : 0.0f;
+    }
+    __syncthreads();
+    if (t < T) {
+      const TU* ut = u + (size_t)t * d + k0;
+      for (int j = 0; j < kw; j += 8) {
+        float x[8];
+        load8(ut + j, x);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+#pragma unroll
+          for (int e = 0; e < NP; ++e) acc[e] = __fmaf_rn(ws[j + q][e], x[q], acc[e]);
+        }
+      }
+    }
+  }
+  if (t >= T) return;
+  float zmax = -FLT_MAX;
+#pragma unroll
+  for (int e = 0; e < NP; ++e) {
+    if (e < N) {
+      if (bias) acc[e] = __fadd_rn(acc[e], bias[e]);
+      zmax = fmaxf(zmax, acc[e]);
+    }
+  }
+  float den = 0.0f;
+#pragma unroll
+  for (int e = 0; e < NP; ++e)
+    if (e < N) den += expf(acc[e] - zmax);
+  if (logits) {
+#pragma unroll
+    for (int e = 0; e < NP; ++e)
+      if (e < N) logits[(size_t)t * N + e] = acc[e];
+  }
+  if (probs) {
+#pragma unroll
+    for (int e = 0; e < NP; ++e)
+      if (e < N) probs[(size_t)t * N + e] = expf(acc[e] - zmax) / den;
+  }
+  uint32_t taken = 0;
+  float psel[16];
+  int isel[16];
+  float ps = 0.0f;
+  for (int s = 0; s < k; ++s) {
+    float bz = -FLT_MAX;
+    int bi = -1;
+#pragma unroll
+    for (int e = 0; e < NP; ++e) {
+      if (e < N && !((taken >> e) & 1u) && (bi < 0 || acc[e] > bz)) {
+        bz = acc[e];
+        bi = e;
+      }
+    }
+    taken |= 1u << bi;
+    isel[s] = bi;
+    psel[s] = expf(bz - zmax) / den;
+    ps += psel[s];
+  }
+  for (int s = 0; s < k; ++s) {
+    top_idx[(size_t)t * k + s] = isel[s];
+    top_w[(size_t)t * k + s] = renorm ? psel[s] / ps : psel[s];
+  }
+}
+
 template <typename TU>
 void launch_logits(const TU* u, const float* w, const float* bias, float* z, int T, int d, int N,
                    cudaStream_t st) {
@@ -190,6 +278,22 @@ int launch_route(const moe_shape& s, const void* u, int32_t u_dtype, const float
                  const float* bias, int32_t* top_idx, float* top_w, float* probs, float* logits,
                  void* ws, cudaStream_t st) {
   if (s.T == 0) return MOE_OK;
+  if (s.N <= 16) {
+    const int blocks = (s.T + 63) / 64;
+#define MOE_FUSED(NP, TU)                                                                     \
+  router_fused_small<NP, TU><<<blocks, 64, 0, st>>>(static_cast<const TU*>(u), w_route, bias, \
+                                                    s.T, s.d, s.N, s.k, s.renorm, top_idx,     \
+                                                    top_w, probs, logits)
+    if (u_dtype == MOE_F32) {
+      if (s.N <= 8) MOE_FUSED(8, float); else MOE_FUSED(16, float);
+    } else if (u_dtype == MOE_BF16) {
+      if (s.N <= 8) MOE_FUSED(8, __nv_bfloat16); else MOE_FUSED(16, __nv_bfloat16);
+    } else {
+      if (s.N <= 8) MOE_FUSED(8, __half); else MOE_FUSED(16, __half);
+    }
+#undef MOE_FUSED
+    return launch_status();
+  }
   float* z = logits ? logits : static_cast<float*>(ws);
   if (u_dtype == MOE_F32) {
     launch_logits(static_cast<const float*>(u), w_route, bias, z, s.T, s.d, s.N, st);
