@@ -268,18 +268,158 @@ def reference_arm(args, wl):
 
 
 # ------------------------------------------------------------------- main
+# ----------------------------------------------------------- decode workload
+Q4_EXPERT_BYTES = lambda wl: 3 * wl.h * wl.d // 2 + 3 * wl.h * wl.d // 32 * 2  # qs + fp16 scales
+
+
+class DecodeReplica:
+    """24 layers of q4_0 experts (all N experts resident; only selected ones read)."""
+
+    def __init__(self, wl, seed, torch, moe):
+        st = torch.cuda.current_stream().cuda_stream
+        N, d, h = wl.N, wl.d, wl.h
+        self.layers, self.keep = [], []
+        for l in range(wl.n_layers):
+            wr = torch.empty((N, d), dtype=torch.float32, device="cuda")
+            S.normal_dev(seed, W.tid(W.TID_WROUTE, l), N * d, W.SIGMA_W, S.DT_F32,
+                         wr.data_ptr(), st)
+            mats = []
+            for base, rows, cols in ((W.TID_WGATE, h, d), (W.TID_WUP, h, d),
+                                     (W.TID_WDOWN, d, h)):
+                qs = torch.empty((N * rows, cols // 2), dtype=torch.uint8, device="cuda")
+                sc = torch.empty((N * rows, cols // 32), dtype=torch.int16, device="cuda")
+                S.q4_dev(seed, W.tid(base, l), N * rows, cols, qs.data_ptr(), sc.data_ptr(), st)
+                mats += [qs, sc]
+            self.keep += [wr, *mats]
+            self.layers.append(moe.q4_layer(wr, *mats))
+        self.u = torch.empty((wl.T, d), dtype=torch.float16, device="cuda")
+        S.normal_dev(seed, W.TID_U, wl.T * d, 1.0, S.DT_F16, self.u.data_ptr(), st)
+
+    def nbytes(self):
+        return sum(t.numel() * t.element_size() for t in self.keep)
+
+
+def decode_main(args, wl, torch, moe, rank, world, dist):
+    stream = torch.cuda.current_stream()
+    one = DecodeReplica(wl, wl.seed + 7919 * rank, torch, moe)
+    n_rep = max(1, -(-2 * L2_BYTES // one.nbytes()))
+    reps = [one] + [DecodeReplica(wl, wl.seed + 7919 * (rank + world * i), torch, moe)
+                    for i in range(1, n_rep)]
+    s = moe.shape(wl.T, wl.d, wl.N, wl.k, wl.h, 1, 0)
+    ws = torch.empty(moe.moe_decode_workspace_bytes(s), dtype=torch.uint8, device="cuda")
+    out = torch.empty((wl.T, wl.d), dtype=torch.float16, device="cuda")
+    idx_all = torch.empty((n_rep, wl.n_layers, wl.T, wl.k), dtype=torch.int32, device="cuda")
+
+    def step(i):
+        moe.moe_decode_step(s, reps[i].layers, reps[i].u, out, idx_all[i], ws=ws)
+
+    for i in range(max(args.warmup, n_rep)):
+        step(i % n_rep)
+    torch.cuda.synchronize()
+    assert moe.moe_device_status() == 0
+    graphs = []
+    cap = torch.cuda.Stream()
+    cap.wait_stream(stream)
+    with torch.cuda.stream(cap):
+        for i in range(n_rep):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=cap):
+                step(i)
+            graphs.append(g)
+    stream.wait_stream(cap)
+    for i in range(args.warmup):
+        graphs[i % n_rep].replay()
+    torch.cuda.synchronize()
+    # algorithmic bytes: router + the union of selected experts + u in/out, per layer
+    sel = idx_all.cpu().numpy()
+    ebytes = Q4_EXPERT_BYTES(wl)
+    step_bytes = []
+    for i in range(n_rep):
+        b = 0
+        for l in range(wl.n_layers):
+            b += wl.N * wl.d * 4 + len(np.unique(sel[i, l])) * ebytes + 2 * wl.T * wl.d * 2
+        step_bytes.append(b)
+    sampler = ClockSampler(int(os.environ.get("LOCAL_RANK", "0"))) if rank == 0 else None
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    torch.cuda.nvtx.range_push("timed")
+    a.record(stream)
+    for i in range(args.steps):
+        graphs[i % n_rep].replay()
+    b.record(stream)
+    torch.cuda.nvtx.range_pop()
+    torch.cuda.synchronize()
+    clocks = sampler.stop() if sampler else None
+    ms = a.elapsed_time(b)
+    if dist:
+        t = torch.tensor([ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    hbm, _, _, src = _peaks()
+    bytes_timed = sum(step_bytes[i % n_rep] for i in range(args.steps))
+    achieved = bytes_timed / (ms / 1e3) / 1e9
+    tokens = wl.T * args.steps * world
+    # end to end: pinned host u -> device -> 24 layers -> pinned host output
+    u_host = reps[0].u.cpu().pin_memory()
+    o_host = torch.empty_like(out, device="cpu").pin_memory()
+    u_dev = torch.empty_like(reps[0].u)
+    for _ in range(args.warmup):
+        u_dev.copy_(u_host, non_blocking=True)
+        moe.moe_decode_step(s, reps[0].layers, u_dev, out, ws=ws)
+        o_host.copy_(out, non_blocking=True)
+    torch.cuda.synchronize()
+    ea, eb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ea.record(stream)
+    for _ in range(args.steps):
+        u_dev.copy_(u_host, non_blocking=True)
+        moe.moe_decode_step(s, reps[0].layers, u_dev, out, ws=ws)
+        o_host.copy_(out, non_blocking=True)
+    eb.record(stream)
+    torch.cuda.synchronize()
+    e_ms = ea.elapsed_time(eb)
+    if rank == 0:
+        line = {"metric": METRIC, "value": tokens / (ms / 1e3), "unit": "tokens/s",
+                "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "q4_0 weights, fp16 activations, fp32 math",
+                "data": "synthetic",
+                "config": {"workload": f"decode: T={wl.T} d={wl.d} N={wl.N} h={wl.h} "
+                                       f"top-{wl.k}, {wl.n_layers} layers per step",
+                           "global_batch": wl.T * world, "parallelism": f"replicas x{world}",
+                           "l2": f"weights rotate over {n_rep} replicas "
+                                 f"({n_rep * one.nbytes() / 2**20:.0f} MiB > L2)"},
+                "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                             "frac": achieved / hbm, "traffic": None,
+                             "kernel": "decode_gateup + decode_down, whole 24-layer step",
+                             "bytes_per_step": bytes_timed / args.steps,
+                             "peak_source": f"{src} hbm_gbs"},
+                "cpu_baseline": None,
+                "e2e": {"value": tokens / (e_ms / 1e3), "unit": "tokens/s",
+                        "h2d_bytes_per_step": wl.T * wl.d * 2,
+                        "d2h_bytes_per_step": wl.T * wl.d * 2},
+                "gpu_launches": 2 * wl.n_layers * args.steps, "clocks": clocks}
+        print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="small", choices=["small", "mixtral", "tiny"])
+    ap.add_argument("--workload", default="small",
+                    choices=["small", "mixtral", "tiny", "decode"])
+    ap.add_argument("--decode-T", type=int, default=32, help="decode batch (1, 8 or 32)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
-    wl = W.ALL[args.workload]()
+    wl = W.decode(T=args.decode_T) if args.workload == "decode" else W.ALL[args.workload]()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -298,6 +438,13 @@ def main():
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     import sparse_mixture_experts_15_b200 as moe
+
+    if args.workload == "decode":
+        decode_main(args, wl, torch, moe, rank, world, dist)
+        if dist:
+            dist.barrier()
+            dist.destroy_process_group()
+        return
 
     # replicas rotate so that the inputs of consecutive steps exceed L2
     one = Replica(wl, wl.seed + 7919 * rank, torch)

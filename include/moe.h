@@ -225,6 +225,46 @@ MOE_API int moe_layer_fwd(const moe_shape* shape, const moe_layer_weights* w, co
                   int32_t act_dtype, void* y, const moe_layer_outputs* out, void* ws,
                   size_t ws_bytes, void* stream);
 
+/* ---------------------------------------------------------- q4_0 decode */
+/* Small-batch decode with q4_0 experts (deployment notes "Kestrel-MCU notes
+ * 13", §2 lookup loading of the selected experts only, §4 q4_0 experts with an
+ * fp32 router).  q4_0: blocks of 32 consecutive values along a row, one fp16
+ * scale s per block, 4-bit q in 0..15, w = (q - 8) s; byte j of a block holds
+ * element j (low nibble) and element j + 16 (high nibble).  A matrix
+ * [rows][cols] is qs [rows][cols/2] bytes plus scales [rows][cols/32] fp16.
+ * Per layer: gate, up [N][h][d]; down [N][d][h]; router [N][d] fp32. */
+typedef struct {
+  const float* w_route;        /* [N][d] fp32 */
+  const float* bias;           /* [N] fp32 or NULL */
+  const uint8_t* gate_qs;      /* [N][h][d/2] */
+  const uint16_t* gate_scales; /* [N][h][d/32] fp16 */
+  const uint8_t* up_qs;
+  const uint16_t* up_scales;
+  const uint8_t* down_qs;      /* [N][d][h/2] */
+  const uint16_t* down_scales; /* [N][d][h/32] fp16 */
+} moe_q4_layer;
+
+/* Limits: T <= 32, N <= 64, k <= 8, d % 32 == 0, h % 32 == 0, h / 32 a
+ * divisor of 32.  Returns 0 for shapes outside them. */
+MOE_API size_t moe_decode_workspace_bytes(const moe_shape* shape);
+
+/* One decode layer: u [T][d] fp16 (bit patterns) -> y [T][d] fp16, the
+ * layer output sum_s a_s F_{e_s}(u_t) with the hidden vector kept in fp32;
+ * u_next (nullable) = fp16(u + y), the next layer's input.  top_idx [T][k]
+ * and top_w [T][k] are optional outputs.  Only the experts some token
+ * selected are read.  `layer` is a host struct of device pointers. */
+MOE_API int moe_decode_layer(const moe_shape* shape, const moe_q4_layer* layer, const uint16_t* u,
+                             uint16_t* y, uint16_t* u_next, int32_t* top_idx, float* top_w,
+                             void* ws, size_t ws_bytes, void* stream);
+
+/* n_layers chained layers: u_{l+1} = fp16(u_l + y_l), u_out = u_{n_layers}.
+ * `layers` is a host array of n_layers structs.  top_idx_all [n_layers][T][k]
+ * (nullable) receives every layer's routing.  Same kernels as
+ * moe_decode_layer, so a chain equals the layer calls made one by one. */
+MOE_API int moe_decode_step(const moe_shape* shape, int32_t n_layers, const moe_q4_layer* layers,
+                            const uint16_t* u0, uint16_t* u_out, int32_t* top_idx_all, void* ws,
+                            size_t ws_bytes, void* stream);
+
 /* ----------------------------------------------------------- diagnostics */
 /* Human-readable name of a status code (static string). */
 MOE_API const char* moe_status_string(int32_t status);

@@ -48,6 +48,8 @@ def lib():
         L.or_f16_to_f64.restype = dbl
         L.or_round_bf16.argtypes = [dbl]
         L.or_round_bf16.restype = dbl
+        L.or_round_f16.argtypes = [dbl]
+        L.or_round_f16.restype = ctypes.c_uint16
         L.or_mat_decode.argtypes = [ctypes.POINTER(OrMat), vp]
         L.or_router_logit.argtypes = [vp, vp, i64]
         L.or_router_logit.restype = ctypes.c_float
@@ -122,6 +124,23 @@ def f16_to_f64(code: int) -> float:
 
 def round_bf16(x: float) -> float:
     return lib().or_round_bf16(float(x))
+
+
+def round_f16(x) -> np.ndarray:
+    """Round float64 values to fp16 bit patterns (round to nearest even)."""
+    x = np.asarray(x, np.float64)
+    out = np.array([lib().or_round_f16(float(v)) for v in x.ravel()], np.uint16)
+    return out.reshape(x.shape)
+
+
+def decode_layer(u_codes, w_route, mats, k, renorm=1, bias=None):
+    """One q4_0 decode layer on fp16 activations (deployment notes §2, §4):
+    routing, then y_t = sum_s a_s F_{e_s}(u_t) with the hidden vector unrounded;
+    returns (top_idx, top_w, y in float64, u_next = fp16(u + y) codes)."""
+    u = decode(F16, u_codes)
+    _, _, idx, tw = route(u.astype(np.float32), w_route, k, renorm, bias)
+    y = moe_tokens([m[0] for m in mats], [m[1] for m in mats], [m[2] for m in mats], u, idx, tw)
+    return idx, tw, y, round_f16(u + y)
 
 
 def decode(dtype, arr):

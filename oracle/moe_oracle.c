@@ -110,6 +110,15 @@ double or_round_bf16(double x) {
   return (double)f;
 }
 
+/* Round a double to the nearest IEEE binary16 (ties to even) and return its
+ * bit pattern: the storage of the fp16 decode activations between layers. */
+uint16_t or_round_f16(double x) {
+  _Float16 h = (_Float16)x;
+  uint16_t u;
+  memcpy(&u, &h, 2);
+  return u;
+}
+
 /* ------------------------------------------------------------------- router */
 
 /* Router logit z = (W_route u)_i  [MoE tutorial] §3.2, formed in fp32.

@@ -45,6 +45,11 @@ class MoeLayerOutputs(ctypes.Structure):
                                    "row_of", "overflow", "totals", "f", "P", "n_sum_fP")]
 
 
+class MoeQ4Layer(ctypes.Structure):
+    _fields_ = [(n, _vp) for n in ("w_route", "bias", "gate_qs", "gate_scales", "up_qs",
+                                   "up_scales", "down_qs", "down_scales")]
+
+
 _P_SHAPE = ctypes.POINTER(MoeShape)
 _PROTOS = {
     "moe_capacity": (_i32, [_i64, _i32, _i32, _f64, ctypes.POINTER(_i32)]),
@@ -63,6 +68,11 @@ _PROTOS = {
     "moe_layer_workspace_bytes": (_sz, [_P_SHAPE, _i32]),
     "moe_layer_fwd": (_i32, [_P_SHAPE, ctypes.POINTER(MoeLayerWeights), _vp, _i32, _vp,
                              ctypes.POINTER(MoeLayerOutputs), _vp, _sz, _vp]),
+    "moe_decode_workspace_bytes": (_sz, [_P_SHAPE]),
+    "moe_decode_layer": (_i32, [_P_SHAPE, ctypes.POINTER(MoeQ4Layer), _vp, _vp, _vp, _vp, _vp,
+                                _vp, _sz, _vp]),
+    "moe_decode_step": (_i32, [_P_SHAPE, _i32, ctypes.POINTER(MoeQ4Layer), _vp, _vp, _vp, _vp,
+                               _sz, _vp]),
     "moe_status_string": (ctypes.c_char_p, [_i32]),
     "moe_device_status": (_i32, [_vp, ctypes.POINTER(_i32)]),
     "moe_reset_device_status": (_i32, [_vp]),
@@ -199,6 +209,34 @@ def moe_layer_fwd(s: MoeShape, w_route, w_gate, w_up, w_down, u, y, bias=None, a
     wbuf, wlen = _ws(moe_layer_workspace_bytes(s, dt), u.device, ws)
     _check(_lib.moe_layer_fwd(ctypes.byref(s), ctypes.byref(W), _ptr(u), dt, _ptr(y),
                               ctypes.byref(O), _ptr(wbuf), wlen, _stream(stream)), "moe_layer_fwd")
+
+
+def q4_layer(w_route, gate_qs, gate_scales, up_qs, up_scales, down_qs, down_scales,
+             bias=None) -> MoeQ4Layer:
+    return MoeQ4Layer(_ptr(w_route), _ptr(bias), _ptr(gate_qs), _ptr(gate_scales), _ptr(up_qs),
+                      _ptr(up_scales), _ptr(down_qs), _ptr(down_scales))
+
+
+def moe_decode_workspace_bytes(s: MoeShape) -> int:
+    return int(_lib.moe_decode_workspace_bytes(ctypes.byref(s)))
+
+
+def moe_decode_layer(s: MoeShape, layer: MoeQ4Layer, u, y, u_next=None, top_idx=None,
+                     top_w=None, ws=None, stream=None):
+    """u, y, u_next: fp16 tensors [T][d]."""
+    wbuf, wlen = _ws(moe_decode_workspace_bytes(s), u.device, ws)
+    _check(_lib.moe_decode_layer(ctypes.byref(s), ctypes.byref(layer), _ptr(u), _ptr(y),
+                                 _ptr(u_next), _ptr(top_idx), _ptr(top_w), _ptr(wbuf), wlen,
+                                 _stream(stream)), "moe_decode_layer")
+
+
+def moe_decode_step(s: MoeShape, layers, u0, u_out, top_idx_all=None, ws=None, stream=None):
+    """`layers`: a sequence of MoeQ4Layer (host structs of device pointers)."""
+    arr = (MoeQ4Layer * len(layers))(*layers)
+    wbuf, wlen = _ws(moe_decode_workspace_bytes(s), u0.device, ws)
+    _check(_lib.moe_decode_step(ctypes.byref(s), len(layers), arr, _ptr(u0), _ptr(u_out),
+                                _ptr(top_idx_all), _ptr(wbuf), wlen, _stream(stream)),
+           "moe_decode_step")
 
 
 def moe_device_status(stream=None) -> int:

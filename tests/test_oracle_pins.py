@@ -416,3 +416,35 @@ def test_bandwidth_gain_printed_values(golden):
     for rec in golden("mcu_bandwidth_gain.txt"):
         g = O.bandwidth_gain(int(rec["ffn"]), int(rec["top_k"]), int(rec["ffn_e"]))
         assert f"{g:.2f}" == rec["gain"]
+
+
+def test_round_f16_matches_numpy():
+    x = np.concatenate([RNG.standard_normal(5000) * 10.0 ** RNG.integers(-8, 4, 5000),
+                        [0.0, 65504.0, 6.0e-8, 2.0 ** -25, 3 * 2.0 ** -26, 1.0 + 2.0 ** -11]])
+    ref = x.astype(np.float16).view(np.uint16)
+    assert np.array_equal(O.round_f16(x), ref)
+
+
+def test_decode_layer_q4_matches_dequantised_dense():
+    """A q4_0 layer equals the same layer with the dequantised weights in
+    float64 (the per-GEMV emulation of the deployment notes, §6)."""
+    T, d, h, N, k = 5, 64, 32, 4, 2
+    mats, dense = [], []
+    for e in range(N):
+        trip = []
+        for rows, cols in ((h, d), (h, d), (d, h)):
+            qs = RNG.integers(0, 256, (rows, cols // 2)).astype(np.uint8)
+            sc = np.array(RNG.choice([0x2000, 0x1C00, 0x0005, 0x9C00], (rows, cols // 32)),
+                          np.uint16)
+            trip.append(O.Mat(O.Q4_0, rows, cols, qs=qs, scales=sc))
+        mats.append(tuple(trip))
+        dense.append(tuple(O.Mat(O.F32, m.rows, m.cols, data=m.decode().astype(np.float32))
+                           for m in trip))
+    u = RNG.standard_normal((T, d)).astype(np.float16).view(np.uint16)
+    w_route = (RNG.standard_normal((N, d)) * 0.1).astype(np.float32)
+    idx, tw, y, un = O.decode_layer(u, w_route, mats, k)
+    # the q4 values are exactly representable in fp32, so the dense copy is exact
+    y2 = O.moe_tokens([m[0] for m in dense], [m[1] for m in dense], [m[2] for m in dense],
+                      O.decode(O.F16, u), idx, tw)
+    assert np.array_equal(y, y2)
+    assert np.array_equal(un, (O.decode(O.F16, u) + y).astype(np.float16).view(np.uint16))
