@@ -406,6 +406,128 @@ def decode_main(args, wl, torch, moe, rank, world, dist):
         print(json.dumps(line), flush=True)
 
 
+# ----------------------------------------------------------- latent workload
+def latent_main(args, wl, torch, moe, rank, world, dist):
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    stream = torch.cuda.current_stream()
+    st = stream.cuda_stream
+    E, d, l, h, n, sh = wl.N, wl.d, wl.latent, wl.h, wl.n_shared, wl.shared_hidden
+    seed = wl.seed + 7919 * rank
+
+    def normal(tid, shape, dt, tdt):
+        t = torch.empty(shape, dtype=tdt, device="cuda")
+        S.normal_dev(seed, tid, t.numel(), W.SIGMA_W, dt, t.data_ptr(), st)
+        return t
+
+    bf = torch.bfloat16
+    w_route = normal(W.TID_WROUTE, (E, d), S.DT_F32, torch.float32)
+    wg = normal(W.TID_WGATE, (E, h, l), S.DT_BF16, bf)
+    wu = normal(W.TID_WUP, (E, h, l), S.DT_BF16, bf)
+    wd = normal(W.TID_WDOWN, (E, l, h), S.DT_BF16, bf)
+    w_dp = normal(W.TID_WDP, (l, d), S.DT_BF16, bf)
+    w_upp = normal(W.TID_WUPP, (d, l), S.DT_BF16, bf)
+    sg = torch.empty((n, sh, d), dtype=bf, device="cuda")
+    su, sd = torch.empty_like(sg), torch.empty((n, d, sh), dtype=bf, device="cuda")
+    for j in range(n):
+        tg, tu, td = W.shared_tids(j)
+        S.normal_dev(seed, tg, sh * d, W.SIGMA_W, S.DT_BF16, sg[j].data_ptr(), st)
+        S.normal_dev(seed, tu, sh * d, W.SIGMA_W, S.DT_BF16, su[j].data_ptr(), st)
+        S.normal_dev(seed, td, d * sh, W.SIGMA_W, S.DT_BF16, sd[j].data_ptr(), st)
+    x = torch.empty((wl.T, d), dtype=bf, device="cuda")
+    S.rmsnorm_rows_dev(seed, W.TID_U, wl.T, d, S.DT_BF16, x.data_ptr(), st)
+    y = torch.empty_like(x)
+    s = moe.shape(wl.T, d, E, wl.k, h, 1, 0)
+    lw = moe.latent_weights(l, w_dp, w_upp, sg, su, sd, n, sh, 1e-6)
+    ws = torch.empty(moe.moe_latent_workspace_bytes(s, lw), dtype=torch.uint8, device="cuda")
+    counts = torch.empty(E, dtype=torch.int32, device="cuda")
+    act = moe.act(moe.ACT_SITU_GLU, wl.beta_gate, wl.beta_up)
+
+    def step():
+        moe.moe_latent_fwd(s, w_route, wg, wu, wd, lw, x, y, a=act,
+                           outputs={"counts": counts}, ws=ws)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert moe.moe_device_status() == 0
+    g = torch.cuda.CUDAGraph()
+    cap = torch.cuda.Stream()
+    cap.wait_stream(stream)
+    with torch.cuda.stream(cap):
+        with torch.cuda.graph(g, stream=cap):
+            step()
+    stream.wait_stream(cap)
+    g.replay()
+    torch.cuda.synchronize()
+    used = int((counts > 0).sum().item())
+    # algorithmic HBM bytes: router + touched routed experts + dense weights + activations
+    wbytes = (E * d * 4 + used * 3 * l * h * 2 + 2 * l * d * 2 + n * 3 * sh * d * 2)
+    abytes = 2 * wl.T * d * 2
+    step_bytes = wbytes + abytes
+    flops = (2.0 * wl.T * E * d + 2.0 * wl.T * l * d + 6.0 * l * h * wl.T * wl.k
+             + 2.0 * wl.T * d * l + n * 6.0 * wl.T * d * sh)
+    sampler = ClockSampler(int(os.environ.get("LOCAL_RANK", "0"))) if rank == 0 else None
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    torch.cuda.nvtx.range_push("timed")
+    a.record(stream)
+    for _ in range(args.steps):
+        g.replay()
+    b.record(stream)
+    torch.cuda.nvtx.range_pop()
+    torch.cuda.synchronize()
+    clocks = sampler.stop() if sampler else None
+    ms = a.elapsed_time(b)
+    if dist:
+        t = torch.tensor([ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    hbm, tf, _, src = _peaks()
+    per_step_s = ms / args.steps / 1e3
+    achieved = step_bytes / per_step_s / 1e9
+    # end to end: pinned host x -> device -> layer -> pinned host y
+    x_host = x.cpu().pin_memory()
+    y_host = torch.empty_like(y, device="cpu").pin_memory()
+    x_dev = torch.empty_like(x)
+    ea, eb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ea.record(stream)
+    for _ in range(args.steps):
+        x_dev.copy_(x_host, non_blocking=True)
+        moe.moe_latent_fwd(s, w_route, wg, wu, wd, lw, x_dev, y, a=act, ws=ws)
+        y_host.copy_(y, non_blocking=True)
+    eb.record(stream)
+    torch.cuda.synchronize()
+    e_ms = ea.elapsed_time(eb)
+    tokens = wl.T * args.steps * world
+    if rank == 0:
+        line = {"metric": METRIC, "value": tokens / (ms / 1e3), "unit": "tokens/s",
+                "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                "config": {"workload": f"latent: T={wl.T} d={d} l={l} E={E} H={h} top-{wl.k}, "
+                                       f"{n} shared of hidden {sh}, caps 4/25",
+                           "global_batch": wl.T * world, "parallelism": f"replicas x{world}",
+                           "l2": "routed expert weights 59 GB > L2",
+                           "experts_touched": used},
+                "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                             "frac": achieved / hbm, "traffic": None,
+                             "kernel": "whole layer step (routed tcgen05 GEMMs stream every "
+                                       "touched expert once)",
+                             "bytes_per_step": step_bytes,
+                             "tflops": flops / per_step_s / 1e12,
+                             "peak_source": f"{src} hbm_gbs"},
+                "cpu_baseline": None,
+                "e2e": {"value": tokens / (e_ms / 1e3), "unit": "tokens/s",
+                        "h2d_bytes_per_step": wl.T * d * 2, "d2h_bytes_per_step": wl.T * d * 2},
+                "gpu_launches": None, "clocks": clocks}
+        print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -413,7 +535,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="small",
-                    choices=["small", "mixtral", "tiny", "decode"])
+                    choices=["small", "mixtral", "tiny", "decode", "latent"])
     ap.add_argument("--decode-T", type=int, default=32, help="decode batch (1, 8 or 32)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -439,8 +561,9 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     import sparse_mixture_experts_15_b200 as moe
 
-    if args.workload == "decode":
-        decode_main(args, wl, torch, moe, rank, world, dist)
+    if args.workload in ("decode", "latent"):
+        (decode_main if args.workload == "decode" else latent_main)(args, wl, torch, moe, rank,
+                                                                    world, dist)
         if dist:
             dist.barrier()
             dist.destroy_process_group()

@@ -225,6 +225,38 @@ MOE_API int moe_layer_fwd(const moe_shape* shape, const moe_layer_weights* w, co
                   int32_t act_dtype, void* y, const moe_layer_outputs* out, void* ws,
                   size_t ws_bytes, void* stream);
 
+/* -------------------------------------------------------------- LatentMoE */
+/* Latent-space MoE layer (Stable LatentMoE demo document: width separation,
+ * RMSNorm before the up-projection, SiTU-GLU soft caps).  The routed experts
+ * work in a latent width l < d, the shared experts at full width d:
+ *   z = W_route x (+b) on the full-width x; top-k; a   (routing on x)
+ *   x_l = W_dp x                                 W_dp [l][d] bf16
+ *   m = sum_s a_s E_{e_s}(x_l)                   routed gate/up [N][h][l], down [N][l][h]
+ *   m^ = m / sqrt(mean(m^2) + rms_eps)           no gain
+ *   y = W_upp m^ + sum_j S_j(x)                  W_upp [d][l]; S_j SwiGLU d -> sh -> d
+ * The routed act is taken from moe_layer_weights.act (MOE_ACT_SITU_GLU with
+ * beta_gate, beta_up for the document's experts); shared experts are plain
+ * SwiGLU.  Capacity applies as in moe_layer_fwd. */
+typedef struct {
+  int32_t latent;          /* l, multiple of 128 */
+  int32_t n_shared;        /* 0..2 shared experts */
+  int32_t shared_hidden;   /* sh, multiple of 64 */
+  const void* w_down_proj; /* [l][d] bf16 */
+  const void* w_up_proj;   /* [d][l] bf16 */
+  const void* shared_gate; /* [n_shared][sh][d] bf16 */
+  const void* shared_up;   /* [n_shared][sh][d] bf16 */
+  const void* shared_down; /* [n_shared][d][sh] bf16 */
+  float rms_eps;
+} moe_latent_weights;
+
+MOE_API size_t moe_latent_workspace_bytes(const moe_shape* shape, const moe_latent_weights* lw);
+/* shape: T tokens, d model width, N routed experts, k, h routed hidden width.
+ * w: router [N][d] fp32 (+bias) and the routed experts (bf16, latent width),
+ * w->w_dtype == MOE_BF16.  x, y [T][d] bf16.  out: as for moe_layer_fwd. */
+MOE_API int moe_latent_fwd(const moe_shape* shape, const moe_layer_weights* w,
+                           const moe_latent_weights* lw, const void* x, void* y,
+                           const moe_layer_outputs* out, void* ws, size_t ws_bytes, void* stream);
+
 /* ---------------------------------------------------------- q4_0 decode */
 /* Small-batch decode with q4_0 experts (deployment notes "Kestrel-MCU notes
  * 13", §2 lookup loading of the selected experts only, §4 q4_0 experts with an

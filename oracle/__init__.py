@@ -48,6 +48,8 @@ def lib():
         L.or_f16_to_f64.restype = dbl
         L.or_round_bf16.argtypes = [dbl]
         L.or_round_bf16.restype = dbl
+        L.or_round_bf16_n.argtypes = [i64, vp, vp]
+        L.or_round_bf16_n.restype = None
         L.or_round_f16.argtypes = [dbl]
         L.or_round_f16.restype = ctypes.c_uint16
         L.or_mat_decode.argtypes = [ctypes.POINTER(OrMat), vp]
@@ -124,6 +126,39 @@ def f16_to_f64(code: int) -> float:
 
 def round_bf16(x: float) -> float:
     return lib().or_round_bf16(float(x))
+
+
+def round_bf16_array(x) -> np.ndarray:
+    x = _c(x, np.float64)
+    y = np.empty_like(x)
+    lib().or_round_bf16_n(x.size, x.ctypes.data, y.ctypes.data)
+    return y
+
+
+def latent_tokens(x_codes, w_route, k, W_dp, get_expert, W_upp, shared, beta_g, beta_u, eps,
+                  renorm=1, bias=None):
+    """LatentMoE forward for the given token rows (Stable LatentMoE demo document:
+    width separation, RMSNorm before the up-projection, SiTU-GLU soft caps):
+      routing on the full-width x; x_l = bf16(W_dp x); m = sum_s a_s E_s(x_l) with
+      the soft-capped routed experts (hidden stored as bf16);
+      m^ = bf16(m / sqrt(mean m^2 + eps)); y = W_upp m^ + sum_j S_j(x) (plain SwiGLU).
+    get_expert(e) returns the (gate, up, down) matrices of routed expert e.
+    Returns (top_idx, top_w, y in float64)."""
+    x = decode(BF16, x_codes)
+    _, _, idx, tw = route(x.astype(np.float32), w_route, k, renorm, bias)
+    y = np.zeros((x.shape[0], W_upp.rows))
+    for t in range(x.shape[0]):
+        xl = round_bf16_array(matvec(W_dp, x[t]))
+        m = np.zeros(W_dp.rows)
+        for s_ in range(k):
+            g, u, d = get_expert(int(idx[t, s_]))
+            m += tw[t, s_] * expert(g, u, d, xl, act=1, beta_g=beta_g, beta_u=beta_u, round_h=1)
+        mh = round_bf16_array(rmsnorm(m, eps))
+        yt = matvec(W_upp, mh)
+        for (g, u, d) in shared:
+            yt = yt + expert(g, u, d, x[t], act=0, round_h=1)
+        y[t] = yt
+    return idx, tw, y
 
 
 def round_f16(x) -> np.ndarray:

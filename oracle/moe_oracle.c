@@ -110,6 +110,11 @@ double or_round_bf16(double x) {
   return (double)f;
 }
 
+/* Element-wise or_round_bf16 over n values. */
+void or_round_bf16_n(int64_t n, const double* x, double* y) {
+  for (int64_t i = 0; i < n; ++i) y[i] = or_round_bf16(x[i]);
+}
+
 /* Round a double to the nearest IEEE binary16 (ties to even) and return its
  * bit pattern: the storage of the fp16 decode activations between layers. */
 uint16_t or_round_f16(double x) {

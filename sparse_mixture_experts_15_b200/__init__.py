@@ -50,6 +50,12 @@ class MoeQ4Layer(ctypes.Structure):
                                    "up_scales", "down_qs", "down_scales")]
 
 
+class MoeLatentWeights(ctypes.Structure):
+    _fields_ = [("latent", _i32), ("n_shared", _i32), ("shared_hidden", _i32),
+                ("w_down_proj", _vp), ("w_up_proj", _vp), ("shared_gate", _vp),
+                ("shared_up", _vp), ("shared_down", _vp), ("rms_eps", _f32)]
+
+
 _P_SHAPE = ctypes.POINTER(MoeShape)
 _PROTOS = {
     "moe_capacity": (_i32, [_i64, _i32, _i32, _f64, ctypes.POINTER(_i32)]),
@@ -68,6 +74,10 @@ _PROTOS = {
     "moe_layer_workspace_bytes": (_sz, [_P_SHAPE, _i32]),
     "moe_layer_fwd": (_i32, [_P_SHAPE, ctypes.POINTER(MoeLayerWeights), _vp, _i32, _vp,
                              ctypes.POINTER(MoeLayerOutputs), _vp, _sz, _vp]),
+    "moe_latent_workspace_bytes": (_sz, [_P_SHAPE, ctypes.POINTER(MoeLatentWeights)]),
+    "moe_latent_fwd": (_i32, [_P_SHAPE, ctypes.POINTER(MoeLayerWeights),
+                              ctypes.POINTER(MoeLatentWeights), _vp, _vp,
+                              ctypes.POINTER(MoeLayerOutputs), _vp, _sz, _vp]),
     "moe_decode_workspace_bytes": (_sz, [_P_SHAPE]),
     "moe_decode_layer": (_i32, [_P_SHAPE, ctypes.POINTER(MoeQ4Layer), _vp, _vp, _vp, _vp, _vp,
                                 _vp, _sz, _vp]),
@@ -209,6 +219,29 @@ def moe_layer_fwd(s: MoeShape, w_route, w_gate, w_up, w_down, u, y, bias=None, a
     wbuf, wlen = _ws(moe_layer_workspace_bytes(s, dt), u.device, ws)
     _check(_lib.moe_layer_fwd(ctypes.byref(s), ctypes.byref(W), _ptr(u), dt, _ptr(y),
                               ctypes.byref(O), _ptr(wbuf), wlen, _stream(stream)), "moe_layer_fwd")
+
+
+def latent_weights(latent, w_down_proj, w_up_proj, shared_gate=None, shared_up=None,
+                   shared_down=None, n_shared=0, shared_hidden=0, rms_eps=1e-6):
+    return MoeLatentWeights(latent, n_shared, shared_hidden, _ptr(w_down_proj), _ptr(w_up_proj),
+                            _ptr(shared_gate), _ptr(shared_up), _ptr(shared_down), rms_eps)
+
+
+def moe_latent_workspace_bytes(s: MoeShape, lw: MoeLatentWeights) -> int:
+    return int(_lib.moe_latent_workspace_bytes(ctypes.byref(s), ctypes.byref(lw)))
+
+
+def moe_latent_fwd(s: MoeShape, w_route, w_gate, w_up, w_down, lw: MoeLatentWeights, x, y,
+                   bias=None, a=None, outputs: dict | None = None, ws=None, stream=None):
+    """The LatentMoE layer; x, y bf16 [T][d]; routed experts at latent width."""
+    a = a or act()
+    W = MoeLayerWeights(_ptr(w_route), _ptr(bias), _ptr(w_gate), _ptr(w_up), _ptr(w_down), BF16,
+                        a)
+    O = MoeLayerOutputs(**{k: _ptr(v) for k, v in (outputs or {}).items()})
+    wbuf, wlen = _ws(moe_latent_workspace_bytes(s, lw), x.device, ws)
+    _check(_lib.moe_latent_fwd(ctypes.byref(s), ctypes.byref(W), ctypes.byref(lw), _ptr(x),
+                               _ptr(y), ctypes.byref(O), _ptr(wbuf), wlen, _stream(stream)),
+           "moe_latent_fwd")
 
 
 def q4_layer(w_route, gate_qs, gate_scales, up_qs, up_scales, down_qs, down_scales,

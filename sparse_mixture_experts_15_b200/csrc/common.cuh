@@ -137,4 +137,31 @@ int launch_ffn_tc(const moe_shape& s, int32_t width, const __nv_bfloat16* x_rows
                   const __nv_bfloat16* w_down, const moe_act& act, float* y_rows, void* ws,
                   cudaStream_t st);
 
+// Grouped tcgen05 GEMM helpers (gemm_tc.cu).
+enum TcMode { MODE_GATEUP = 0, MODE_STORE_F32 = 1, MODE_STORE_BF16 = 2 };
+
+// One K-segment of a store-mode GEMM: A rows (weights) and B rows (tokens).
+struct TcSeg {
+  const void* a;      // [a_rows][K] bf16
+  int64_t a_rows;
+  int K;              // multiple of 64
+  int arow;           // row offset into A added to the group's base row
+  const void* b;      // [b_rows][b_cols] bf16
+  int64_t b_rows;
+  int b_cols;
+  int bcol;           // column offset into B
+};
+
+// Gate/up GEMM with the fused activation: for group g and its rows of X,
+// out[row][g * out_col_group + j] = act(X W_gate[g]^T, X W_up[g]^T)[j] as bf16.
+// offsets == nullptr: every group uses rows [0, T) of X.
+int tc_gateup(const int32_t* offsets, int T, int G, const __nv_bfloat16* X, int64_t x_rows,
+              int K, const __nv_bfloat16* w_gate, const __nv_bfloat16* w_up, int hidden,
+              const moe_act& act, __nv_bfloat16* out, int out_ld, int out_col_group,
+              cudaStream_t st);
+// Store-mode GEMM over 1..3 K-segments accumulated into one fp32 tile:
+// out[row][g * m_rows + m] = sum_s A_s[g * a_rows + arow_s + m] . B_s[row][bcol_s ...].
+int tc_store(const int32_t* offsets, int T, int G, int m_rows, const TcSeg* segs, int nseg,
+             void* out, int mode, int out_ld, cudaStream_t st);
+
 }  // namespace moe

@@ -35,16 +35,23 @@ constexpr int kThreads = 192;
 constexpr long long kWaitBudget = 4000000000LL;  // cycles (~2 s)
 constexpr int kEpiLd = 33;                       // padded row of the gate/up exchange tile
 
-enum { MODE_GATEUP = 0, MODE_STORE_F32 = 1, MODE_STORE_BF16 = 2 };
 
+constexpr int kMaxSeg = 3;
+
+// One GEMM problem.  The reduction runs over up to kMaxSeg K-segments that
+// accumulate into the same tile; segment s reads A from maps[amap[s]] (rows
+// offset by arow[s]) and B from maps[bmap[s]] (columns offset by bcol[s]).
+// Gate/up mode has one segment: A rows 0-63 from maps[0] (gate), rows 64-127
+// from maps[1] (up), B from maps[2].
 struct TcParams {
-  CUtensorMap tmA0;  // weights (gate, or the single weight of a store mode)
-  CUtensorMap tmA1;  // up weights (gate/up mode)
-  CUtensorMap tmB;   // token rows
+  CUtensorMap maps[4];
   const int32_t* offsets;  // [G+1] token row ranges; nullptr: every group uses rows [0, T)
   int T;
   int G;
-  int K;                  // multiple of 64
+  int nseg;
+  int seg_end[kMaxSeg];   // cumulative 64-wide k-blocks at the end of each segment
+  int amap[kMaxSeg], bmap[kMaxSeg];
+  int arow[kMaxSeg], bcol[kMaxSeg];
   int a_rows_per_group;   // rows of A owned by one group
   int m_tiles;            // 128-row tiles of A per group
   int mode;
@@ -153,9 +160,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_grouped_gemm(const __grid_cons
       }
       tc::mbar_init(tc::smem_u32(drain), 1);
       tc::fence_barrier_init();
-      tc::tma_prefetch_desc(&p.tmA0);
-      if (fused) tc::tma_prefetch_desc(&p.tmA1);
-      tc::tma_prefetch_desc(&p.tmB);
+      for (int i = 0; i < 4; ++i) tc::tma_prefetch_desc(&p.maps[i]);
     }
   }
   if (warp == 1) {
@@ -167,7 +172,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_grouped_gemm(const __grid_cons
   tc::tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const int total_tiles = grp_pre[p.G];
-  const int kblocks = p.K / kBK;
+  const int kblocks = p.seg_end[p.nseg - 1];
 
   auto decode = [&](int tile, int& g, int& m, int& n) {
     int lo = 0, hi = p.G;
@@ -193,7 +198,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_grouped_gemm(const __grid_cons
         decode(tile, g, m, n);
         const int a_row = g * p.a_rows_per_group + m * (fused ? 64 : kBM);
         const int b_row = grp_beg[g] + n * BN;
+        int seg = 0, seg_start = 0;
         for (int kb = 0; kb < kblocks; ++kb) {
+          while (kb >= p.seg_end[seg]) seg_start = p.seg_end[seg++];
+          const int kx = (kb - seg_start) * kBK;
           if (!tc::mbar_wait(tc::smem_u32(&empty[stage]), phase ^ 1u, abort_flag, kWaitBudget)) {
             ok = false;
             break;
@@ -203,12 +211,13 @@ __global__ void __launch_bounds__(kThreads, 1) tc_grouped_gemm(const __grid_cons
           const uint32_t sa = tc::smem_u32(stages + stage * L::STAGE);
           const uint32_t sb = sa + L::A_BYTES;
           if (fused) {
-            tc::tma_load_2d(sa, &p.tmA0, fb, kb * kBK, a_row);
-            tc::tma_load_2d(sa + L::A_BYTES / 2, &p.tmA1, fb, kb * kBK, a_row);
+            tc::tma_load_2d(sa, &p.maps[0], fb, kx, a_row);
+            tc::tma_load_2d(sa + L::A_BYTES / 2, &p.maps[1], fb, kx, a_row);
+            tc::tma_load_2d(sb, &p.maps[2], fb, kx, b_row);
           } else {
-            tc::tma_load_2d(sa, &p.tmA0, fb, kb * kBK, a_row);
+            tc::tma_load_2d(sa, &p.maps[p.amap[seg]], fb, kx, a_row + p.arow[seg]);
+            tc::tma_load_2d(sb, &p.maps[p.bmap[seg]], fb, p.bcol[seg] + kx, b_row);
           }
-          tc::tma_load_2d(sb, &p.tmB, fb, kb * kBK, b_row);
           if (++stage == S) {
             stage = 0;
             phase ^= 1u;
@@ -370,6 +379,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_grouped_gemm(const __grid_cons
 }
 
 // ------------------------------------------------------------------- host
+
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                    const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
                                    const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
@@ -434,9 +444,11 @@ int launch_tc(const TcParams& p, int64_t tiles_upper, cudaStream_t st) {
   return launch_status();
 }
 
-// Token tile width: 256 columns when that still gives at least two tiles per
-// SM, 128 otherwise (more, smaller tiles for small problems).
+// Token tile width: 128 columns when groups average under 192 rows (a
+// 256-wide tile would be mostly padding) or when 256-wide tiles would not
+// give every SM two tiles; 256 otherwise.
 int pick_bn(int m_tiles, int64_t max_rows, int G) {
+  if (max_rows < 192LL * G) return 128;
   const int64_t up256 = (int64_t)m_tiles * ((max_rows + 255) / 256 + G);
   return up256 >= 2LL * sm_count() ? 256 : 128;
 }
@@ -460,53 +472,95 @@ int launch_ffn_tc(const moe_shape& s, int32_t width, const __nv_bfloat16* x_rows
   const int64_t R = (int64_t)s.T * s.k;
   if (R == 0) return MOE_OK;
   __nv_bfloat16* H = static_cast<__nv_bfloat16*>(ws);
-  {  // gate/up with the fused activation -> H
-    TcParams p{};
-    const int64_t rows_w = (int64_t)s.N * s.h;
-    if (!make_tmap(&p.tmA0, w_gate, rows_w, width, 64) ||
-        !make_tmap(&p.tmA1, w_up, rows_w, width, 64))
-      return MOE_ERR_CUDA;
-    p.offsets = offsets;
-    p.T = s.T;
-    p.G = s.N;
-    p.K = width;
-    p.a_rows_per_group = s.h;
-    p.m_tiles = s.h / 64;
-    p.mode = MODE_GATEUP;
-    p.act_kind = act.kind;
-    p.beta_g = act.beta_gate;
-    p.beta_u = act.beta_up;
-    p.out = H;
-    p.out_ld = s.h;
-    p.out_col_group = 0;
-    p.status = status_word();
-    const int bn = pick_bn(p.m_tiles, R, p.G);
-    if (!make_tmap(&p.tmB, x_rows, R, width, bn)) return MOE_ERR_CUDA;
-    const int rc = launch_tc_bn(p, R, bn, st);
-    if (rc != MOE_OK) return rc;
+  int rc = tc_gateup(offsets, (int)R, s.N, x_rows, R, width, w_gate, w_up, s.h, act, H, s.h, 0,
+                     st);
+  if (rc != MOE_OK) return rc;
+  TcSeg seg{w_down, (int64_t)s.N * width, s.h, 0, H, R, s.h, 0};
+  return tc_store(offsets, (int)R, s.N, width, &seg, 1, y_rows, MODE_STORE_F32, width, st);
+}
+
+// Gate/up GEMM with the fused activation: for group g and its rows of X,
+// out[row][g * out_col_group + j] = act(X W_gate[g]^T, X W_up[g]^T)[j], bf16.
+int tc_gateup(const int32_t* offsets, int T, int G, const __nv_bfloat16* X, int64_t x_rows,
+              int K, const __nv_bfloat16* w_gate, const __nv_bfloat16* w_up, int hidden,
+              const moe_act& act, __nv_bfloat16* out, int out_ld, int out_col_group,
+              cudaStream_t st) {
+  TcParams p{};
+  const int64_t rows_w = (int64_t)G * hidden;
+  const int64_t max_rows = offsets ? x_rows : (int64_t)T * G;
+  const int bn = pick_bn(hidden / 64, max_rows, G);
+  if (!make_tmap(&p.maps[0], w_gate, rows_w, K, 64) || !make_tmap(&p.maps[1], w_up, rows_w, K, 64) ||
+      !make_tmap(&p.maps[2], X, x_rows, K, bn))
+    return MOE_ERR_CUDA;
+  p.maps[3] = p.maps[2];
+  p.offsets = offsets;
+  p.T = T;
+  p.G = G;
+  p.nseg = 1;
+  p.seg_end[0] = K / kBK;
+  p.a_rows_per_group = hidden;
+  p.m_tiles = hidden / 64;
+  p.mode = MODE_GATEUP;
+  p.act_kind = act.kind;
+  p.beta_g = act.beta_gate;
+  p.beta_u = act.beta_up;
+  p.out = out;
+  p.out_ld = out_ld;
+  p.out_col_group = out_col_group;
+  p.status = status_word();
+  return launch_tc_bn(p, max_rows, bn, st);
+}
+
+// Plain GEMM over 1..3 K-segments accumulated into one output:
+// out[row][g * m_rows + m] = sum_s (A_s[g * a_rows_s + arow_s + m] . B_s[row][bcol_s + ...]).
+int tc_store(const int32_t* offsets, int T, int G, int m_rows, const TcSeg* segs, int nseg,
+             void* out, int mode, int out_ld, cudaStream_t st) {
+  if (nseg < 1 || nseg > kMaxSeg) return MOE_ERR_INVALID_ARG;
+  TcParams p{};
+  const int64_t max_rows = offsets ? segs[0].b_rows : (int64_t)T * G;
+  const int bn = pick_bn(m_rows / kBM, max_rows, G);
+  // distinct (pointer, rows, cols, box) tensor maps, at most four
+  const void* key_p[4];
+  int64_t key_r[4];
+  int key_c[4], key_box[4];
+  int nmaps = 0;
+  auto map_of = [&](const void* ptr, int64_t rows, int cols, int box) -> int {
+    for (int i = 0; i < nmaps; ++i)
+      if (key_p[i] == ptr && key_r[i] == rows && key_c[i] == cols && key_box[i] == box) return i;
+    if (nmaps >= 4) return -1;
+    if (!make_tmap(&p.maps[nmaps], ptr, rows, cols, box)) return -2;
+    key_p[nmaps] = ptr;
+    key_r[nmaps] = rows;
+    key_c[nmaps] = cols;
+    key_box[nmaps] = box;
+    return nmaps++;
+  };
+  int kb = 0;
+  for (int i = 0; i < nseg; ++i) {
+    const int ia = map_of(segs[i].a, segs[i].a_rows, segs[i].K, kBM);
+    const int ib = map_of(segs[i].b, segs[i].b_rows, segs[i].b_cols, bn);
+    if (ia == -1 || ib == -1) return MOE_ERR_UNSUPPORTED;
+    if (ia < 0 || ib < 0) return MOE_ERR_CUDA;
+    p.amap[i] = ia;
+    p.bmap[i] = ib;
+    kb += segs[i].K / kBK;
+    p.seg_end[i] = kb;
+    p.arow[i] = segs[i].arow;
+    p.bcol[i] = segs[i].bcol;
   }
-  {  // down projection -> unweighted fp32 rows
-    TcParams p{};
-    const int64_t rows_w = (int64_t)s.N * width;
-    if (!make_tmap(&p.tmA0, w_down, rows_w, s.h, kBM)) return MOE_ERR_CUDA;
-    p.tmA1 = p.tmA0;
-    p.offsets = offsets;
-    p.T = s.T;
-    p.G = s.N;
-    p.K = s.h;
-    p.a_rows_per_group = width;
-    p.m_tiles = width / kBM;
-    p.mode = MODE_STORE_F32;
-    p.out = y_rows;
-    p.out_ld = width;
-    p.out_col_group = 0;
-    p.status = status_word();
-    const int bn = pick_bn(p.m_tiles, R, p.G);
-    if (!make_tmap(&p.tmB, H, R, s.h, bn)) return MOE_ERR_CUDA;
-    const int rc = launch_tc_bn(p, R, bn, st);
-    if (rc != MOE_OK) return rc;
-  }
-  return MOE_OK;
+  for (int i = nmaps; i < 4; ++i) p.maps[i] = p.maps[0];
+  p.offsets = offsets;
+  p.T = T;
+  p.G = G;
+  p.nseg = nseg;
+  p.a_rows_per_group = m_rows;
+  p.m_tiles = m_rows / kBM;
+  p.mode = mode;
+  p.out = out;
+  p.out_ld = out_ld;
+  p.out_col_group = 0;
+  p.status = status_word();
+  return launch_tc_bn(p, max_rows, bn, st);
 }
 
 }  // namespace moe

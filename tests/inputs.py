@@ -94,3 +94,52 @@ def rel_err(got, ref):
     ref = np.asarray(ref, np.float64)
     rms = float(np.sqrt(np.mean(ref * ref)))
     return float(np.max(np.abs(got - ref))) / (rms if rms > 0 else 1.0)
+
+
+# ------------------------------------------------------------- LatentMoE
+def dev_latent(wl: W.Workload, device="cuda"):
+    """Device weights of a LatentMoE workload (bf16; router fp32)."""
+    import torch
+    E, d, l, h, n, sh = wl.N, wl.d, wl.latent, wl.h, wl.n_shared, wl.shared_hidden
+    st = torch.cuda.current_stream().cuda_stream
+    out = dict(
+        w_route=dev_normal(wl.seed, W.TID_WROUTE, (E, d), W.SIGMA_W, S.DT_F32, device),
+        w_gate=dev_normal(wl.seed, W.TID_WGATE, (E, h, l), W.SIGMA_W, S.DT_BF16, device),
+        w_up=dev_normal(wl.seed, W.TID_WUP, (E, h, l), W.SIGMA_W, S.DT_BF16, device),
+        w_down=dev_normal(wl.seed, W.TID_WDOWN, (E, l, h), W.SIGMA_W, S.DT_BF16, device),
+        w_dp=dev_normal(wl.seed, W.TID_WDP, (l, d), W.SIGMA_W, S.DT_BF16, device),
+        w_upp=dev_normal(wl.seed, W.TID_WUPP, (d, l), W.SIGMA_W, S.DT_BF16, device))
+    sg = torch.empty((max(n, 1), sh, d), dtype=torch.bfloat16, device=device)
+    su = torch.empty_like(sg)
+    sd = torch.empty((max(n, 1), d, sh), dtype=torch.bfloat16, device=device)
+    for j in range(n):
+        tg, tu, td = W.shared_tids(j)
+        S.normal_dev(wl.seed, tg, sh * d, W.SIGMA_W, S.DT_BF16, sg[j].data_ptr(), st)
+        S.normal_dev(wl.seed, tu, sh * d, W.SIGMA_W, S.DT_BF16, su[j].data_ptr(), st)
+        S.normal_dev(wl.seed, td, d * sh, W.SIGMA_W, S.DT_BF16, sd[j].data_ptr(), st)
+    out.update(shared_gate=sg, shared_up=su, shared_down=sd)
+    return out
+
+
+def host_latent_expert(wl: W.Workload, e: int):
+    l, h = wl.latent, wl.h
+    g = S.normal(wl.seed, W.TID_WGATE, (h, l), W.SIGMA_W, S.DT_BF16, offset=e * h * l)
+    u = S.normal(wl.seed, W.TID_WUP, (h, l), W.SIGMA_W, S.DT_BF16, offset=e * h * l)
+    d = S.normal(wl.seed, W.TID_WDOWN, (l, h), W.SIGMA_W, S.DT_BF16, offset=e * l * h)
+    return O.Mat(O.BF16, h, l, data=g), O.Mat(O.BF16, h, l, data=u), O.Mat(O.BF16, l, h, data=d)
+
+
+def host_latent_dense(wl: W.Workload):
+    d, l, sh = wl.d, wl.latent, wl.shared_hidden
+    W_dp = O.Mat(O.BF16, l, d, data=S.normal(wl.seed, W.TID_WDP, (l, d), W.SIGMA_W, S.DT_BF16))
+    W_upp = O.Mat(O.BF16, d, l, data=S.normal(wl.seed, W.TID_WUPP, (d, l), W.SIGMA_W, S.DT_BF16))
+    shared = []
+    for j in range(wl.n_shared):
+        tg, tu, td = W.shared_tids(j)
+        shared.append((O.Mat(O.BF16, sh, d, data=S.normal(wl.seed, tg, (sh, d), W.SIGMA_W,
+                                                            S.DT_BF16)),
+                       O.Mat(O.BF16, sh, d, data=S.normal(wl.seed, tu, (sh, d), W.SIGMA_W,
+                                                            S.DT_BF16)),
+                       O.Mat(O.BF16, d, sh, data=S.normal(wl.seed, td, (d, sh), W.SIGMA_W,
+                                                            S.DT_BF16))))
+    return W_dp, W_upp, shared

@@ -448,3 +448,65 @@ def test_decode_layer_q4_matches_dequantised_dense():
                       O.decode(O.F16, u), idx, tw)
     assert np.array_equal(y, y2)
     assert np.array_equal(un, (O.decode(O.F16, u) + y).astype(np.float16).view(np.uint16))
+
+
+def _latent_case(N=6, d=64, l=32, h=48, sh=40, n_sh=2, T=5, scale_down=1.0):
+    rng = np.random.default_rng(77)
+
+    def bf(rows, cols, sig=0.2):
+        v = (rng.standard_normal((rows, cols)) * sig).astype(np.float32)
+        return O.Mat(O.BF16, rows, cols, data=v.view(np.uint32) >> 16)
+
+    experts = [(bf(h, l), bf(h, l), bf(l, h)) for _ in range(N)]
+    if scale_down != 1.0:  # exact power-of-two rescale of every routed down matrix
+        experts = [(g, u, O.Mat(O.F32, l, h, data=(dn.decode() * scale_down).astype(np.float32)))
+                   for g, u, dn in experts]
+    shared = [(bf(sh, d), bf(sh, d), bf(d, sh)) for _ in range(n_sh)]
+    W_dp, W_upp = bf(l, d), bf(d, l)
+    w_route = rng.standard_normal((N, d)).astype(np.float32)
+    x = (rng.standard_normal((T, d)).astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
+    return x, w_route, W_dp, experts, W_upp, shared
+
+
+def test_latent_rmsnorm_removes_scale_of_routed_branch():
+    """LatentMoE document: RMSNorm before the up-projection makes the output
+    insensitive to the routed branch's scale.  An exact x8 on every routed
+    down matrix leaves y bit-identical when eps = 0."""
+    x, wr, W_dp, ex, W_upp, sh = _latent_case()
+    _, _, y1 = O.latent_tokens(x, wr, 2, W_dp, lambda e: ex[e], W_upp, sh, 4.0, 25.0, 0.0)
+    x, wr, W_dp, ex8, W_upp, sh = _latent_case(scale_down=8.0)
+    _, _, y8 = O.latent_tokens(x, wr, 2, W_dp, lambda e: ex8[e], W_upp, sh, 4.0, 25.0, 0.0)
+    assert np.array_equal(y1, y8)
+
+
+def test_latent_routed_experts_live_in_the_bottleneck():
+    """Routed experts see only x_l = W_dp x: with W_dp = 0 the routed branch is
+    zero and y is exactly the shared experts' output; routing (on x) is unchanged."""
+    x, wr, W_dp, ex, W_upp, sh = _latent_case()
+    zero = O.Mat(O.F32, W_dp.rows, W_dp.cols, data=np.zeros((W_dp.rows, W_dp.cols), np.float32))
+    idx0, _, y0 = O.latent_tokens(x, wr, 2, zero, lambda e: ex[e], W_upp, sh, 4.0, 25.0, 1e-6)
+    idx1, _, _ = O.latent_tokens(x, wr, 2, W_dp, lambda e: ex[e], W_upp, sh, 4.0, 25.0, 1e-6)
+    assert np.array_equal(idx0, idx1)
+    xd = O.decode(O.BF16, x)
+    ref = np.array([sum(O.expert(g, u, d, xd[t], round_h=1) for g, u, d in sh)
+                    for t in range(x.shape[0])])
+    assert np.array_equal(y0, ref)
+
+
+def test_latent_single_expert_closed_form():
+    """N = 1, k = 1, no shared experts: y = W_upp bf16(rms(F(bf16(W_dp x))))
+    restated with numpy and torch's bf16 rounding."""
+    x, wr, W_dp, ex, W_upp, sh = _latent_case(N=1, n_sh=0, T=3)
+    _, tw, y = O.latent_tokens(x, wr[:1], 1, W_dp, lambda e: ex[e], W_upp, [], 4.0, 25.0, 1e-6)
+    assert np.all(tw == 1.0)
+
+    def bf16(v):
+        return torch.tensor(v.astype(np.float32)).to(torch.bfloat16).double().numpy()
+
+    g, u, d = (m.decode() for m in ex[0])
+    for t, xt in enumerate(O.decode(O.BF16, x)):
+        xl = bf16(W_dp.decode() @ xt)
+        G, U = 4 * np.tanh(g @ xl / 4), 25 * np.tanh(u @ xl / 25)
+        m = d @ bf16(_silu(G) * U)
+        mh = bf16(m / np.sqrt(np.mean(m * m) + 1e-6))
+        assert np.allclose(y[t], W_upp.decode() @ mh, rtol=1e-11, atol=1e-12)
