@@ -68,6 +68,18 @@ __device__ __forceinline__ void load8(const __half* p, float* o) {
 
 __device__ __forceinline__ float silu(float g) { return g / (1.0f + expf(-g)); }
 
+// ------------------------------------------- programmatic dependent launch
+// Every kernel is launched with programmatic stream serialization: its CTAs
+// may be scheduled while the previous kernel on the stream drains, and they
+// wait in pdl_wait() (before their first global-memory access) until that
+// kernel has finished and its writes are visible.  pdl_allow_next() lets the
+// following kernel be scheduled early in turn.  Both are no-ops for a kernel
+// launched without the attribute.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_allow_next() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ------------------------------------------------------------- host checks
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -92,7 +104,54 @@ inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s
 
 inline int cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
-inline int launch_status() { return cuda_status(cudaGetLastError()); }
+// Launch errors reported by cudaLaunchKernelEx (launch_pdl) on this thread.
+inline cudaError_t& pdl_launch_error() {
+  static thread_local cudaError_t e = cudaSuccess;
+  return e;
+}
+
+inline int launch_status() {
+  const cudaError_t e = cudaGetLastError();
+  const cudaError_t p = pdl_launch_error();
+  pdl_launch_error() = cudaSuccess;
+  return (e == cudaSuccess && p == cudaSuccess) ? MOE_OK : MOE_ERR_CUDA;
+}
+
+// Every kernel of the library asks for the maximum shared-memory carve-out, so
+// consecutive launches on an SM never need a different L1/shared split (the
+// tensor-core kernels need ~215 KB of shared memory).  Once per device and
+// call site.
+#define MOE_PREFER_SHARED(kernel)                                                      \
+  do {                                                                                 \
+    static bool moe_done_[64] = {false};                                               \
+    int moe_dev_ = 0;                                                                  \
+    if (cudaGetDevice(&moe_dev_) == cudaSuccess && moe_dev_ >= 0 && moe_dev_ < 64 &&   \
+        !moe_done_[moe_dev_]) {                                                        \
+      cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,     \
+                           (int)cudaSharedmemCarveoutMaxShared);                       \
+      moe_done_[moe_dev_] = true;                                                      \
+    }                                                                                  \
+  } while (0)
+
+// Launches kernel<<<grid, block, smem, st>>>(args...) with programmatic
+// stream serialization (see pdl_wait).
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t st, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+  if (e != cudaSuccess) pdl_launch_error() = e;
+  return e;
+}
 
 // Carves sub-buffers out of a caller workspace (256-byte aligned pieces).
 struct Carver {

@@ -127,6 +127,8 @@ __global__ void __launch_bounds__(128)
                   const uint8_t* __restrict__ gq, const uint16_t* __restrict__ gs,
                   const uint8_t* __restrict__ uq, const uint16_t* __restrict__ us,
                   float* __restrict__ H, int32_t* __restrict__ top_idx, float* __restrict__ top_w) {
+  pdl_wait();
+  pdl_allow_next();
   extern __shared__ __align__(16) char dyn[];
   const int us_ld = d + 8, ws_ld = d + 4, nb = d / 32;
   __half* u_s = reinterpret_cast<__half*>(dyn);                          // [T][d+8]
@@ -220,6 +222,8 @@ __global__ void __launch_bounds__(128)
                 const uint8_t* __restrict__ dq, const uint16_t* __restrict__ dsc,
                 const float* __restrict__ H, __half* __restrict__ y, __half* __restrict__ u_next,
                 int* status) {
+  pdl_wait();
+  pdl_allow_next();
   extern __shared__ __align__(16) char dyn[];
   const int TKmax = T * k, h_ld = h + 4;
   float* hs = reinterpret_cast<float*>(dyn);  // [T*k][h+4]: H row of each (token, slot)
@@ -385,10 +389,12 @@ int launch_decode_layer(const moe_shape& s, const moe_q4_layer& L, const __half*
       return MOE_ERR_CUDA;
     configured[dev] = true;
   }
-  decode_gateup<<<s.N * (s.h / kRowsA), 128, gateup_smem(s), st>>>(
+  MOE_PREFER_SHARED((decode_gateup));
+  launch_pdl(decode_gateup, dim3(s.N * (s.h / kRowsA)), dim3(128), gateup_smem(s), st, 
       u, s.T, s.d, s.N, s.k, s.h, s.renorm, L.w_route, L.bias, L.gate_qs, L.gate_scales, L.up_qs,
       L.up_scales, H, idx, w);
-  decode_down<<<s.d / kRowsB, 128, down_smem(s), st>>>(u, s.T, s.d, s.N, s.k, s.h, idx, w,
+  MOE_PREFER_SHARED((decode_down));
+  launch_pdl(decode_down, dim3(s.d / kRowsB), dim3(128), down_smem(s), st, u, s.T, s.d, s.N, s.k, s.h, idx, w,
                                                        L.down_qs, L.down_scales, H, y, u_next,
                                                        status_word());
   return launch_status();

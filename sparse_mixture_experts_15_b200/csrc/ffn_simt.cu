@@ -32,6 +32,8 @@ __global__ void __launch_bounds__(256)
     ffn_gateup_simt(const float* __restrict__ x_rows, int width, int h,
                     const int32_t* __restrict__ offsets, int N, const float* __restrict__ wg,
                     const float* __restrict__ wu, moe_act act, float* __restrict__ H) {
+  pdl_wait();
+  pdl_allow_next();
   extern __shared__ float xs[];
   const int r = blockIdx.x;
   if (r >= offsets[N]) return;
@@ -56,6 +58,8 @@ __global__ void __launch_bounds__(256)
     ffn_down_simt(const float* __restrict__ H, int h, int width,
                   const int32_t* __restrict__ offsets, int N, const float* __restrict__ wd,
                   float* __restrict__ y_rows) {
+  pdl_wait();
+  pdl_allow_next();
   extern __shared__ float hs[];
   const int r = blockIdx.x;
   if (r >= offsets[N]) return;
@@ -83,9 +87,11 @@ int launch_ffn_simt(const moe_shape& s, int32_t width, const float* x_rows, cons
   const int64_t max_rows = (int64_t)s.T * s.k;
   if (max_rows == 0) return MOE_OK;
   float* H = static_cast<float*>(ws);
-  ffn_gateup_simt<<<(unsigned)max_rows, 256, (size_t)width * 4, st>>>(x_rows, width, s.h, offsets,
+  MOE_PREFER_SHARED((ffn_gateup_simt));
+  launch_pdl(ffn_gateup_simt, dim3((unsigned)max_rows), dim3(256), (size_t)width * 4, st, x_rows, width, s.h, offsets,
                                                                        s.N, w_gate, w_up, act, H);
-  ffn_down_simt<<<(unsigned)max_rows, 256, (size_t)s.h * 4, st>>>(H, s.h, width, offsets, s.N,
+  MOE_PREFER_SHARED((ffn_down_simt));
+  launch_pdl(ffn_down_simt, dim3((unsigned)max_rows), dim3(256), (size_t)s.h * 4, st, H, s.h, width, offsets, s.N,
                                                                   w_down, y_rows);
   return launch_status();
 }

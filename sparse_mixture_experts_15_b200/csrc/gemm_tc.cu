@@ -115,6 +115,29 @@ __global__ void __launch_bounds__(kThreads, 1) tc_grouped_gemm(const __grid_cons
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const bool fused = p.mode == MODE_GATEUP;
 
+  // ---- prologue that reads no data of the previous kernel: barriers, TMEM,
+  // tensor-map prefetch; it overlaps the previous kernel's tail (PDL)
+  if (warp == 0 && lane == 0) {
+    *abort_flag = 0;
+    for (int s = 0; s < S; ++s) {
+      tc::mbar_init(tc::smem_u32(&full[s]), 1);
+      tc::mbar_init(tc::smem_u32(&empty[s]), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      tc::mbar_init(tc::smem_u32(&tfull[b]), 1);
+      tc::mbar_init(tc::smem_u32(&tempty[b]), 128);
+    }
+    tc::mbar_init(tc::smem_u32(drain), 1);
+    tc::fence_barrier_init();
+    for (int i = 0; i < 4; ++i) tc::tma_prefetch_desc(&p.maps[i]);
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(tc::smem_u32(tmem_slot), 2 * BN);
+    tc::tmem_relinquish();
+  }
+  pdl_wait();
+  pdl_allow_next();
+
   // ---- group table: token range and tile prefix per group (warp 0 scans)
   if (warp == 0) {
     int carry = 0;
@@ -147,25 +170,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_grouped_gemm(const __grid_cons
       }
       carry += __shfl_sync(0xffffffffu, incl, 31);
     }
-    if (lane == 0) {
-      grp_pre[p.G] = carry;
-      *abort_flag = 0;
-      for (int s = 0; s < S; ++s) {
-        tc::mbar_init(tc::smem_u32(&full[s]), 1);
-        tc::mbar_init(tc::smem_u32(&empty[s]), 1);
-      }
-      for (int b = 0; b < 2; ++b) {
-        tc::mbar_init(tc::smem_u32(&tfull[b]), 1);
-        tc::mbar_init(tc::smem_u32(&tempty[b]), 128);
-      }
-      tc::mbar_init(tc::smem_u32(drain), 1);
-      tc::fence_barrier_init();
-      for (int i = 0; i < 4; ++i) tc::tma_prefetch_desc(&p.maps[i]);
-    }
-  }
-  if (warp == 1) {
-    tc::tmem_alloc(tc::smem_u32(tmem_slot), 2 * BN);
-    tc::tmem_relinquish();
+    if (lane == 0) grp_pre[p.G] = carry;
   }
   tc::tc_fence_before();
   __syncthreads();
@@ -440,7 +445,8 @@ int launch_tc(const TcParams& p, int64_t tiles_upper, cudaStream_t st) {
   int64_t grid = sm_count();
   if (tiles_upper < grid) grid = tiles_upper;
   if (grid <= 0) return MOE_OK;
-  tc_grouped_gemm<BN, S><<<(unsigned)grid, kThreads, smem, st>>>(p);
+  MOE_PREFER_SHARED((tc_grouped_gemm<BN, S>));
+  launch_pdl(tc_grouped_gemm<BN, S>, dim3((unsigned)grid), dim3(kThreads), smem, st, p);
   return launch_status();
 }
 

@@ -22,6 +22,8 @@ namespace {
 __global__ void __launch_bounds__(256)
     rmsnorm_rows(const float* __restrict__ m, int rows, int cols, float eps,
                  __nv_bfloat16* __restrict__ out) {
+  pdl_wait();
+  pdl_allow_next();
   const int lane = threadIdx.x & 31;
   for (int r = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; r < rows;
        r += (gridDim.x * blockDim.x) >> 5) {
@@ -185,7 +187,8 @@ extern "C" int moe_latent_fwd(const moe_shape* shape, const moe_layer_weights* w
   {
     int blocks = (s.T + 7) / 8;
     if (blocks > 148 * 16) blocks = 148 * 16;
-    rmsnorm_rows<<<blocks, 256, 0, st>>>(b.m, s.T, l, lw->rms_eps, b.m_hat);
+    MOE_PREFER_SHARED((rmsnorm_rows));
+    launch_pdl(rmsnorm_rows, dim3(blocks), dim3(256), 0, st, b.m, s.T, l, lw->rms_eps, b.m_hat);
     rc = launch_status();
     if (rc != MOE_OK) return rc;
   }

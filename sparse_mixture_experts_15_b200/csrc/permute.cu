@@ -24,6 +24,8 @@ constexpr int kChunk = 256;  // dispatches per block = 8 warps x 32 lanes
 __global__ void __launch_bounds__(kChunk)
     permute_hist(const int32_t* __restrict__ idx, int64_t total, int N, int32_t* __restrict__ hist,
                  int* status) {
+  pdl_wait();
+  pdl_allow_next();
   extern __shared__ int32_t cnt[];
   for (int i = threadIdx.x; i < N; i += kChunk) cnt[i] = 0;
   __syncthreads();
@@ -79,13 +81,22 @@ __global__ void __launch_bounds__(1024)
     permute_scan(int32_t* __restrict__ hist, int nblk, int N, int C, int32_t* __restrict__ counts,
                  int32_t* __restrict__ offsets, int32_t* __restrict__ overflow,
                  int32_t* __restrict__ totals) {
+  pdl_wait();
+  pdl_allow_next();
   const int e = threadIdx.x;
   int L = 0;
   if (e < N) {
-    for (int b = 0; b < nblk; ++b) {
-      const int v = hist[(size_t)b * N + e];
-      hist[(size_t)b * N + e] = L;
-      L += v;
+    // eight loads in flight per round (the loop rewrites what it reads, so
+    // the compiler would otherwise wait on each load)
+    for (int b0 = 0; b0 < nblk; b0 += 8) {
+      int v[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) v[j] = b0 + j < nblk ? hist[(size_t)(b0 + j) * N + e] : 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if (b0 + j < nblk) hist[(size_t)(b0 + j) * N + e] = L;
+        L += v[j];
+      }
     }
   }
   const int kept = e < N ? ((C > 0 && L > C) ? C : L) : 0;
@@ -112,6 +123,8 @@ __global__ void __launch_bounds__(kChunk)
     permute_scatter(const int32_t* __restrict__ idx, int64_t total, int k, int N, int C,
                     const int32_t* __restrict__ base, const int32_t* __restrict__ offsets,
                     int32_t* __restrict__ perm_tok, int32_t* __restrict__ row_of) {
+  pdl_wait();
+  pdl_allow_next();
   extern __shared__ int32_t wcnt[];  // [8][N]
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   for (int i = threadIdx.x; i < 8 * N; i += kChunk) wcnt[i] = 0;
@@ -158,11 +171,14 @@ int launch_permute(const moe_shape& s, const int32_t* top_idx, int32_t* counts, 
   const int nblk = (int)((total + kChunk - 1) / kChunk);
   int32_t* hist = static_cast<int32_t*>(ws);
   if (nblk > 0) {
-    permute_hist<<<nblk, kChunk, (size_t)s.N * 4, st>>>(top_idx, total, s.N, hist, status_word());
+    MOE_PREFER_SHARED((permute_hist));
+    launch_pdl(permute_hist, dim3(nblk), dim3(kChunk), (size_t)s.N * 4, st, top_idx, total, s.N, hist, status_word());
   }
-  permute_scan<<<1, 1024, 0, st>>>(hist, nblk, s.N, s.capacity, counts, offsets, overflow, totals);
+  MOE_PREFER_SHARED((permute_scan));
+  launch_pdl(permute_scan, dim3(1), dim3(1024), 0, st, hist, nblk, s.N, s.capacity, counts, offsets, overflow, totals);
   if (nblk > 0) {
-    permute_scatter<<<nblk, kChunk, (size_t)s.N * 8 * 4, st>>>(top_idx, total, s.k, s.N,
+    MOE_PREFER_SHARED((permute_scatter));
+    launch_pdl(permute_scatter, dim3(nblk), dim3(kChunk), (size_t)s.N * 8 * 4, st, top_idx, total, s.k, s.N,
                                                                s.capacity, hist, offsets,
                                                                perm_tok, row_of);
   }

@@ -24,6 +24,8 @@ __global__ void __launch_bounds__((BT / TM) * (BN / TN))
     router_logits_kernel(const TU* __restrict__ u, const float* __restrict__ w,
                          const float* __restrict__ bias, float* __restrict__ z, int T, int d,
                          int N) {
+  pdl_wait();
+  pdl_allow_next();
   constexpr int NT = (BT / TM) * (BN / TN);
   __shared__ __align__(16) float us[kBK][BT];
   __shared__ __align__(16) float wsm[kBK][BN];
@@ -99,6 +101,8 @@ __global__ void __launch_bounds__(256)
     router_topk_kernel(const float* __restrict__ z, int T, int N, int k, int renorm,
                        int32_t* __restrict__ top_idx, float* __restrict__ top_w,
                        float* __restrict__ probs) {
+  pdl_wait();
+  pdl_allow_next();
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (warp >= T) return;
@@ -170,39 +174,72 @@ __global__ void __launch_bounds__(256)
 
 // Few experts (N <= NP <= 16): one thread per token keeps all N logits in
 // registers and finishes softmax, top-k and the combine weights itself, so
-// routing is a single launch.  W_route is staged in shared memory in slabs of
-// kSlab inputs as [j][NP] so every thread reads the same NP floats (broadcast).
+// routing is a single launch.  Per slab of inputs, the router rows and the
+// block's 32 token rows are copied with cp.async (every copy issued before
+// one wait) into rows padded to 16 B past a multiple of 128 B: the threads'
+// 16-byte token reads hit distinct banks and the router reads are broadcasts.
 // Each logit is the same sequential FMA chain over j as in the tiled kernel.
-constexpr int kSlab = 512;
+constexpr int kTokPerBlock = 32;
+
+__device__ __forceinline__ void cp16_async(void* smem, const void* gmem) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
+                   static_cast<uint32_t>(__cvta_generic_to_shared(smem))),
+               "l"(gmem)
+               : "memory");
+}
 
 template <int NP, typename TU>
-__global__ void __launch_bounds__(64)
+__global__ void __launch_bounds__(kTokPerBlock)
     router_fused_small(const TU* __restrict__ u, const float* __restrict__ w,
                        const float* __restrict__ bias, int T, int d, int N, int k, int renorm,
                        int32_t* __restrict__ top_idx, float* __restrict__ top_w,
                        float* __restrict__ probs, float* __restrict__ logits) {
-  __shared__ __align__(16) float ws[kSlab][NP];
-  const int t = blockIdx.x * blockDim.x + threadIdx.x;
+  pdl_wait();
+  pdl_allow_next();
+  constexpr int kSlab = sizeof(TU) == 4 ? 128 : 256;  // 512-byte token slabs
+  constexpr int kRowBytes = kSlab * (int)sizeof(TU) + 16;
+  constexpr int kWld = kSlab + 4;                      // padded router row (floats)
+  __shared__ __align__(16) float ws[NP][kWld];
+  __shared__ __align__(16) char us[kTokPerBlock * kRowBytes];
+  const int t0 = blockIdx.x * kTokPerBlock;
+  const int t = t0 + threadIdx.x;
   float acc[NP];
 #pragma unroll
   for (int e = 0; e < NP; ++e) acc[e] = 0.0f;
   for (int k0 = 0; k0 < d; k0 += kSlab) {
-    const int kw = min(kSlab, d - k0);
+    const int kw = min(kSlab, d - k0);  // multiple of 8
+    const int chunks = kw * (int)sizeof(TU) / 16;
     __syncthreads();
-    for (int i = threadIdx.x; i < kw * NP; i += blockDim.x) {
-      const int e = i / kw, j = i - e * kw;  // coalesced along j
-      ws[j][e] = e < N ? w[(size_t)e * d + k0 + j] : 0.0f;
+    for (int i = threadIdx.x; i < kTokPerBlock * chunks; i += blockDim.x) {
+      const int r = i / chunks, c = i - r * chunks;
+      if (t0 + r < T)
+        cp16_async(us + r * kRowBytes + c * 16,
+                   reinterpret_cast<const char*>(u + (size_t)(t0 + r) * d + k0) + c * 16);
     }
+    const int wchunks = kw / 4;
+    for (int i = threadIdx.x; i < N * wchunks; i += blockDim.x) {
+      const int e = i / wchunks, c = i - e * wchunks;
+      cp16_async(&ws[e][c * 4], w + (size_t)e * d + k0 + c * 4);
+    }
+    asm volatile("cp.async.wait_all;" ::: "memory");
     __syncthreads();
     if (t < T) {
-      const TU* ut = u + (size_t)t * d + k0;
+      const TU* ut = reinterpret_cast<const TU*>(us + threadIdx.x * kRowBytes);
       for (int j = 0; j < kw; j += 8) {
         float x[8];
         load8(ut + j, x);
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
+        for (int h4 = 0; h4 < 8; h4 += 4) {
 #pragma unroll
-          for (int e = 0; e < NP; ++e) acc[e] = __fmaf_rn(ws[j + q][e], x[q], acc[e]);
+          for (int e = 0; e < NP; ++e) {
+            if (e < N) {
+              const float4 wv = *reinterpret_cast<const float4*>(&ws[e][j + h4]);
+              acc[e] = __fmaf_rn(wv.x, x[h4], acc[e]);
+              acc[e] = __fmaf_rn(wv.y, x[h4 + 1], acc[e]);
+              acc[e] = __fmaf_rn(wv.z, x[h4 + 2], acc[e]);
+              acc[e] = __fmaf_rn(wv.w, x[h4 + 3], acc[e]);
+            }
+          }
         }
       }
     }
@@ -260,13 +297,16 @@ void launch_logits(const TU* u, const float* w, const float* bias, float* z, int
                    cudaStream_t st) {
   if (N <= 8) {
     dim3 grid((T + 63) / 64, 1);
-    router_logits_kernel<64, 8, 2, 4, TU><<<grid, 64, 0, st>>>(u, w, bias, z, T, d, N);
+    MOE_PREFER_SHARED((router_logits_kernel<64, 8, 2, 4, TU>));
+    launch_pdl(router_logits_kernel<64, 8, 2, 4, TU>, dim3(grid), dim3(64), 0, st, u, w, bias, z, T, d, N);
   } else if (N <= 16) {
     dim3 grid((T + 63) / 64, 1);
-    router_logits_kernel<64, 16, 4, 4, TU><<<grid, 64, 0, st>>>(u, w, bias, z, T, d, N);
+    MOE_PREFER_SHARED((router_logits_kernel<64, 16, 4, 4, TU>));
+    launch_pdl(router_logits_kernel<64, 16, 4, 4, TU>, dim3(grid), dim3(64), 0, st, u, w, bias, z, T, d, N);
   } else {
     dim3 grid((T + 63) / 64, (N + 63) / 64);
-    router_logits_kernel<64, 64, 4, 4, TU><<<grid, 256, 0, st>>>(u, w, bias, z, T, d, N);
+    MOE_PREFER_SHARED((router_logits_kernel<64, 64, 4, 4, TU>));
+    launch_pdl(router_logits_kernel<64, 64, 4, 4, TU>, dim3(grid), dim3(256), 0, st, u, w, bias, z, T, d, N);
   }
 }
 
@@ -279,11 +319,15 @@ int launch_route(const moe_shape& s, const void* u, int32_t u_dtype, const float
                  void* ws, cudaStream_t st) {
   if (s.T == 0) return MOE_OK;
   if (s.N <= 16) {
-    const int blocks = (s.T + 63) / 64;
+    const int blocks = (s.T + kTokPerBlock - 1) / kTokPerBlock;
 #define MOE_FUSED(NP, TU)                                                                     \
-  router_fused_small<NP, TU><<<blocks, 64, 0, st>>>(static_cast<const TU*>(u), w_route, bias, \
-                                                    s.T, s.d, s.N, s.k, s.renorm, top_idx,     \
-                                                    top_w, probs, logits)
+  do {                                                                                        \
+    MOE_PREFER_SHARED((router_fused_small<NP, TU>));                                          \
+    launch_pdl(router_fused_small<NP, TU>, dim3(blocks), dim3(kTokPerBlock), 0, st, static_cast<const TU*>(u),     \
+                                                                w_route,                        \
+                                                      bias, s.T, s.d, s.N, s.k, s.renorm,     \
+                                                      top_idx, top_w, probs, logits);         \
+  } while (0)
     if (u_dtype == MOE_F32) {
       if (s.N <= 8) MOE_FUSED(8, float); else MOE_FUSED(16, float);
     } else if (u_dtype == MOE_BF16) {
@@ -305,8 +349,11 @@ int launch_route(const moe_shape& s, const void* u, int32_t u_dtype, const float
   const int blocks = (s.T + 7) / 8;
   const int per = (s.N + 31) / 32;
 #define MOE_TOPK(P)                                                                          \
-  router_topk_kernel<P><<<blocks, 256, 0, st>>>(z, s.T, s.N, s.k, s.renorm, top_idx, top_w, \
-                                                probs)
+  do {                                                                                       \
+    MOE_PREFER_SHARED((router_topk_kernel<P>));                                              \
+    launch_pdl(router_topk_kernel<P>, dim3(blocks), dim3(256), 0, st, z, s.T, s.N, s.k, s.renorm, top_idx,       \
+                                                  top_w, probs);                             \
+  } while (0)
   if (per <= 1) MOE_TOPK(1);
   else if (per <= 2) MOE_TOPK(2);
   else if (per <= 4) MOE_TOPK(4);

@@ -13,6 +13,8 @@ __global__ void __launch_bounds__(256)
     gather_rows(const uint4* __restrict__ u, int vec_per_row, const int32_t* __restrict__ perm_tok,
                 const int32_t* __restrict__ offsets, int N, int T, uint4* __restrict__ x_rows,
                 int* status) {
+  pdl_wait();
+  pdl_allow_next();
   const int rows = offsets[N];
   const int lane = threadIdx.x & 31;
   for (int r = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; r < rows;
@@ -56,6 +58,8 @@ template <typename TY>
 __global__ void __launch_bounds__(256)
     combine_rows(const float4* __restrict__ y_rows, int width4, const int32_t* __restrict__ row_of,
                  const float* __restrict__ top_w, int T, int k, TY* __restrict__ y) {
+  pdl_wait();
+  pdl_allow_next();
   const int lane = threadIdx.x & 31;
   for (int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; t < T;
        t += (gridDim.x * blockDim.x) >> 5) {
@@ -89,7 +93,8 @@ int launch_gather(const moe_shape& s, int32_t width, const void* u, int32_t dtyp
   const int vec = (int)((size_t)width * dtype_bytes(dtype) / 16);
   const int64_t max_rows = (int64_t)s.T * s.k;
   if (max_rows == 0) return MOE_OK;
-  gather_rows<<<grid_cap(max_rows), 256, 0, st>>>(static_cast<const uint4*>(u), vec, perm_tok,
+  MOE_PREFER_SHARED((gather_rows));
+  launch_pdl(gather_rows, dim3(grid_cap(max_rows)), dim3(256), 0, st, static_cast<const uint4*>(u), vec, perm_tok,
                                                   offsets, s.N, s.T,
                                                   static_cast<uint4*>(x_rows), status_word());
   return launch_status();
@@ -102,13 +107,16 @@ int launch_combine(const moe_shape& s, int32_t width, const float* y_rows, const
   const int grid = grid_cap(s.T);
   const float4* yr = reinterpret_cast<const float4*>(y_rows);
   if (y_dtype == MOE_F32) {
-    combine_rows<float><<<grid, 256, 0, st>>>(yr, w4, row_of, top_w, s.T, s.k,
+    MOE_PREFER_SHARED((combine_rows<float>));
+    launch_pdl(combine_rows<float>, dim3(grid), dim3(256), 0, st, yr, w4, row_of, top_w, s.T, s.k,
                                               static_cast<float*>(y));
   } else if (y_dtype == MOE_BF16) {
-    combine_rows<__nv_bfloat16><<<grid, 256, 0, st>>>(yr, w4, row_of, top_w, s.T, s.k,
+    MOE_PREFER_SHARED((combine_rows<__nv_bfloat16>));
+    launch_pdl(combine_rows<__nv_bfloat16>, dim3(grid), dim3(256), 0, st, yr, w4, row_of, top_w, s.T, s.k,
                                                       static_cast<__nv_bfloat16*>(y));
   } else {
-    combine_rows<__half><<<grid, 256, 0, st>>>(yr, w4, row_of, top_w, s.T, s.k,
+    MOE_PREFER_SHARED((combine_rows<__half>));
+    launch_pdl(combine_rows<__half>, dim3(grid), dim3(256), 0, st, yr, w4, row_of, top_w, s.T, s.k,
                                                static_cast<__half*>(y));
   }
   return launch_status();

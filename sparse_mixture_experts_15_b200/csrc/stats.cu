@@ -15,6 +15,8 @@ __global__ void __launch_bounds__(256)
     stats_accumulate(const float* __restrict__ probs, const int32_t* __restrict__ top_idx, int T,
                      int N, int k, int32_t* __restrict__ argmax_cnt, int32_t* __restrict__ loads,
                      float* __restrict__ Psum, int* status) {
+  pdl_wait();
+  pdl_allow_next();
   extern __shared__ char smem[];
   int32_t* c_arg = reinterpret_cast<int32_t*>(smem);
   int32_t* c_load = c_arg + N;
@@ -55,6 +57,8 @@ __global__ void stats_finish(const int32_t* __restrict__ argmax_cnt,
                              const int32_t* __restrict__ loads_in, const float* __restrict__ Psum,
                              int T, int N, int has_p, float* __restrict__ f, float* __restrict__ P,
                              float* __restrict__ n_sum_fP, int32_t* __restrict__ loads) {
+  pdl_wait();
+  pdl_allow_next();
   __shared__ float red[32];
   float acc = 0.0f;
   const float inv_t = T > 0 ? 1.0f / (float)T : 0.0f;
@@ -91,10 +95,12 @@ int launch_aux_stats(int32_t T, int32_t N, int32_t k, const float* probs, const 
   if (T > 0) {
     int blocks = (T + 63) / 64;
     if (blocks > 148) blocks = 148;
-    stats_accumulate<<<blocks, 256, (size_t)N * 12, st>>>(probs, top_idx, T, N, k, c_arg, c_load,
+    MOE_PREFER_SHARED((stats_accumulate));
+    launch_pdl(stats_accumulate, dim3(blocks), dim3(256), (size_t)N * 12, st, probs, top_idx, T, N, k, c_arg, c_load,
                                                           c_p, status_word());
   }
-  stats_finish<<<1, 1024, 0, st>>>(c_arg, c_load, c_p, T, N, probs != nullptr, f, P, n_sum_fP,
+  MOE_PREFER_SHARED((stats_finish));
+  launch_pdl(stats_finish, dim3(1), dim3(1024), 0, st, c_arg, c_load, c_p, T, N, probs != nullptr, f, P, n_sum_fP,
                                    loads);
   return launch_status();
 }
