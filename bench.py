@@ -44,6 +44,27 @@ def _peaks():
     return 6650.0, 1590.0, 1400.0, "fallback"
 
 
+# ------------------------------------------------------------ multi-rank
+def max_over_ranks(value: float, dist, device) -> float:
+    """The slowest rank's time: every rank's device-timed value, reduced by MAX."""
+    if dist is None:
+        return value
+    import torch
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(tokens_per_rank_step: int, steps: int, world: int, ms: float) -> float:
+    """Tokens/s of the whole job: all ranks' tokens over the slowest rank's time."""
+    return tokens_per_rank_step * steps * world / (ms / 1e3)
+
+
+def rank_seed(base_seed: int, rank: int, world: int, replica: int = 0) -> int:
+    """Seed of replica `replica` on rank `rank`: every rank draws its own batch."""
+    return base_seed + 7919 * (rank + world * replica)
+
+
 # --------------------------------------------------------------- clocks
 class ClockSampler:
     """nvidia-smi clocks and throttle reasons sampled during the timed region."""
@@ -152,8 +173,19 @@ class Step:
         self.ws_perm = torch.empty(max(pb, 256), dtype=torch.uint8, device="cuda")
         self.ws_ffn = torch.empty(max(fb, 256), dtype=torch.uint8, device="cuda")
         self.act = moe.act()
-        route_launches = 1 if N <= 16 else 2
-        self.launches_per_step = route_launches + 3 + 1 + 2 + 1  # route, permute, gather, ffn, combine
+        self.lws = torch.empty(moe.moe_layer_workspace_bytes(self.s, wl.act_dtype),
+                               dtype=torch.uint8, device="cuda")
+        self.outs = {"top_idx": self.top_idx, "top_w": self.top_w, "totals": self.totals}
+        tpb = 16 if N <= 8 else 8  # tokens per router block
+        small = N <= 16 and k <= 16 and ((T + tpb - 1) // tpb) * N <= 8192
+        # moe_layer_fwd: route (+counts), dispatch, gather, 2 GEMMs, combine for few
+        # experts; route (2), permute (3), gather, 2 GEMMs, combine otherwise
+        self.launches_per_step = 6 if small else 9
+
+    def layer(self, r: Replica):
+        """The product entry point: the whole layer in one C-ABI call."""
+        self.moe.moe_layer_fwd(self.s, r.w_route, *r.w, r.u, self.y, bias=r.bias,
+                               outputs=self.outs, ws=self.lws)
 
     def ffn(self, r: Replica):
         self.moe.moe_expert_ffn(self.s, self.wl.d, self.x_rows, self.offsets, *r.w, self.y_rows,
@@ -301,9 +333,9 @@ class DecodeReplica:
 
 def decode_main(args, wl, torch, moe, rank, world, dist):
     stream = torch.cuda.current_stream()
-    one = DecodeReplica(wl, wl.seed + 7919 * rank, torch, moe)
+    one = DecodeReplica(wl, rank_seed(wl.seed, rank, world), torch, moe)
     n_rep = max(1, -(-2 * L2_BYTES // one.nbytes()))
-    reps = [one] + [DecodeReplica(wl, wl.seed + 7919 * (rank + world * i), torch, moe)
+    reps = [one] + [DecodeReplica(wl, rank_seed(wl.seed, rank, world, i), torch, moe)
                     for i in range(1, n_rep)]
     s = moe.shape(wl.T, wl.d, wl.N, wl.k, wl.h, 1, 0)
     ws = torch.empty(moe.moe_decode_workspace_bytes(s), dtype=torch.uint8, device="cuda")
@@ -355,11 +387,7 @@ def decode_main(args, wl, torch, moe, rank, world, dist):
     torch.cuda.nvtx.range_pop()
     torch.cuda.synchronize()
     clocks = sampler.stop() if sampler else None
-    ms = a.elapsed_time(b)
-    if dist:
-        t = torch.tensor([ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(a.elapsed_time(b), dist, "cuda")
     hbm, _, _, src = _peaks()
     bytes_timed = sum(step_bytes[i % n_rep] for i in range(args.steps))
     achieved = bytes_timed / (ms / 1e3) / 1e9
@@ -381,9 +409,10 @@ def decode_main(args, wl, torch, moe, rank, world, dist):
         o_host.copy_(out, non_blocking=True)
     eb.record(stream)
     torch.cuda.synchronize()
-    e_ms = ea.elapsed_time(eb)
+    e_ms = max_over_ranks(ea.elapsed_time(eb), dist, "cuda")
     if rank == 0:
-        line = {"metric": METRIC, "value": tokens / (ms / 1e3), "unit": "tokens/s",
+        line = {"metric": METRIC, "value": whole_job_rate(wl.T, args.steps, world, ms),
+                "unit": "tokens/s",
                 "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
                 "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "q4_0 weights, fp16 activations, fp32 math",
@@ -412,7 +441,7 @@ def latent_main(args, wl, torch, moe, rank, world, dist):
     stream = torch.cuda.current_stream()
     st = stream.cuda_stream
     E, d, l, h, n, sh = wl.N, wl.d, wl.latent, wl.h, wl.n_shared, wl.shared_hidden
-    seed = wl.seed + 7919 * rank
+    seed = rank_seed(wl.seed, rank, world)
 
     def normal(tid, shape, dt, tdt):
         t = torch.empty(shape, dtype=tdt, device="cuda")
@@ -482,11 +511,7 @@ def latent_main(args, wl, torch, moe, rank, world, dist):
     torch.cuda.nvtx.range_pop()
     torch.cuda.synchronize()
     clocks = sampler.stop() if sampler else None
-    ms = a.elapsed_time(b)
-    if dist:
-        t = torch.tensor([ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(a.elapsed_time(b), dist, "cuda")
     hbm, tf, _, src = _peaks()
     per_step_s = ms / args.steps / 1e3
     achieved = step_bytes / per_step_s / 1e9
@@ -502,10 +527,11 @@ def latent_main(args, wl, torch, moe, rank, world, dist):
         y_host.copy_(y, non_blocking=True)
     eb.record(stream)
     torch.cuda.synchronize()
-    e_ms = ea.elapsed_time(eb)
+    e_ms = max_over_ranks(ea.elapsed_time(eb), dist, "cuda")
     tokens = wl.T * args.steps * world
     if rank == 0:
-        line = {"metric": METRIC, "value": tokens / (ms / 1e3), "unit": "tokens/s",
+        line = {"metric": METRIC, "value": whole_job_rate(wl.T, args.steps, world, ms),
+                "unit": "tokens/s",
                 "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
                 "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
@@ -570,25 +596,26 @@ def main():
         return
 
     # replicas rotate so that the inputs of consecutive steps exceed L2
-    one = Replica(wl, wl.seed + 7919 * rank, torch)
+    one = Replica(wl, rank_seed(wl.seed, rank, world), torch)
     n_rep = max(1, min(64, -(-2 * L2_BYTES // max(one.nbytes(), 1))))
-    reps = [one] + [Replica(wl, wl.seed + 7919 * (rank + world * i), torch)
+    reps = [one] + [Replica(wl, rank_seed(wl.seed, rank, world, i), torch)
                     for i in range(1, n_rep)]
     step = Step(wl, torch, moe)
     stream = torch.cuda.current_stream()
 
     for i in range(args.warmup):
-        step(reps[i % n_rep])
+        step.layer(reps[i % n_rep])
+    step(reps[0])  # the step split at the expert FFN: fills x_rows / offsets for the GEMM replay
     torch.cuda.synchronize()
     kept = [0] * n_rep
     for i in range(n_rep):
-        step(reps[i])
+        step.layer(reps[i])
         torch.cuda.synchronize()
         kept[i] = int(step.totals[0].item())
     assert moe.moe_device_status() == 0
 
-    # The step is device-only work (no host sync), so each replica's step is
-    # captured once as a CUDA graph and replayed: launch overhead off the host.
+    # The step (moe_layer_fwd) is device-only work (no host sync), so each
+    # replica's step is captured once as a CUDA graph and replayed.
     full_g, ffn_g = [], []
     cap = torch.cuda.Stream()
     cap.wait_stream(stream)
@@ -596,7 +623,7 @@ def main():
         for i in range(n_rep):
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g, stream=cap):
-                step(reps[i])
+                step.layer(reps[i])
             full_g.append(g)
             g2 = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g2, stream=cap):
@@ -625,7 +652,7 @@ def main():
     if dist:
         dist.barrier()
     clocks = sampler.stop() if sampler else None
-    ms = t_start.elapsed_time(t_stop)
+    ms = max_over_ranks(t_start.elapsed_time(t_stop), dist, "cuda")
     # the dominant kernel alone: the two tcgen05 GEMM launches of each step
     f_start, f_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     f_start.record(stream)
@@ -634,12 +661,8 @@ def main():
     f_stop.record(stream)
     torch.cuda.synchronize()
     ffn_ms = [f_start.elapsed_time(f_stop) / args.steps] * args.steps
-    if dist:
-        t = torch.tensor([ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
     tokens = wl.T * args.steps * world
-    value = tokens / (ms / 1e3)
+    value = whole_job_rate(wl.T, args.steps, world, ms)
 
     # roofline of the dominant kernel: the tcgen05 grouped GEMM (gate/up + down launches)
     hbm, tf_burst, tf_sust, peak_src = _peaks()
@@ -680,11 +703,7 @@ def main():
             e2e_step()
         b.record(stream)
         torch.cuda.synchronize()
-        e_ms = a.elapsed_time(b)
-        if dist:
-            t = torch.tensor([e_ms], device="cuda")
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e_ms = float(t.item())
+        e_ms = max_over_ranks(a.elapsed_time(b), dist, "cuda")
         el = 2 if wl.act_dtype != S.DT_F32 else 4
         e2e = {"value": tokens / (e_ms / 1e3), "unit": "tokens/s",
                "h2d_bytes_per_step": wl.T * wl.d * el, "d2h_bytes_per_step": wl.T * wl.d * el}

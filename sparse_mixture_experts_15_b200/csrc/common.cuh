@@ -171,9 +171,18 @@ struct Carver {
 // ------------------------------------------------------- internal launchers
 // (defined in the per-step .cu files; all asynchronous on `st`)
 size_t route_ws_bytes(const moe_shape& s);
+// hist (optional, N <= 16 only): per router block of route_tokens_per_block(N)
+// tokens, the count of its dispatches to each expert, [blocks][N].
 int launch_route(const moe_shape& s, const void* u, int32_t u_dtype, const float* w_route,
                  const float* bias, int32_t* top_idx, float* top_w, float* probs, float* logits,
-                 void* ws, cudaStream_t st);
+                 void* ws, cudaStream_t st, int32_t* hist = nullptr);
+int route_tokens_per_block(int N);
+// Permutation in one launch from the router's per-block counts (few experts;
+// dispatch_small_ok says when): see dispatch_small in permute.cu.
+bool dispatch_small_ok(const moe_shape& s);
+int launch_dispatch_small(const moe_shape& s, const int32_t* top_idx, const int32_t* hist,
+                          int32_t* counts, int32_t* offsets, int32_t* perm_tok, int32_t* row_of,
+                          int32_t* overflow, int32_t* totals, cudaStream_t st);
 size_t aux_stats_ws_bytes(int32_t N);
 int launch_aux_stats(int32_t T, int32_t N, int32_t k, const float* probs, const int32_t* top_idx,
                      float* f, float* P, float* n_sum_fP, int32_t* loads, void* ws,

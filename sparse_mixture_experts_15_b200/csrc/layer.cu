@@ -3,6 +3,8 @@
 // (tutorial "Mixture of Experts MoE: how sparse activation saves compute",
 // §3.1-§3.8).  Every step is one of this library's kernels, launched in order
 // on the caller's stream; nothing is read back to the host.
+#include <algorithm>
+
 #include "common.cuh"
 
 namespace moe {
@@ -51,7 +53,8 @@ LayerBufs carve_layer(const moe_shape& s, int32_t act_dtype, void* base) {
   b.row_of = c.take<int32_t>(Tk);
   b.overflow = c.take<int32_t>(s.N);
   b.totals = c.take<int32_t>(4);
-  b.permute_ws = c.take<char>(permute_ws_bytes(s));
+  b.permute_ws = c.take<char>(std::max(permute_ws_bytes(s),
+                                        align_up((size_t)(s.T / 8 + 1) * s.N * 4, 256)));
   b.x_rows = c.take<char>(Tk * s.d * dtype_bytes(act_dtype));
   b.ffn_ws = c.take<char>(ffn_ws_bytes(s, s.d, act_dtype));
   b.y_rows = c.take<float>(Tk * s.d);
@@ -144,18 +147,26 @@ extern "C" int moe_layer_fwd(const moe_shape* shape, const moe_layer_weights* w,
   int32_t* totals = o.totals ? o.totals : b.totals;
   cudaStream_t st = as_stream(stream);
 
+  // Few experts: the router also counts each block's dispatches, and one
+  // kernel then scans and scatters (2 launches instead of 4 before the gather).
+  const bool small = dispatch_small_ok(s);
+  int32_t* hist = small ? static_cast<int32_t*>(b.permute_ws) : nullptr;
   int rc = launch_route(s, u, act_dtype, w->w_route, w->bias, top_idx, top_w, probs, b.logits,
-                        nullptr, st);
+                        nullptr, st, hist);
   if (rc != MOE_OK) return rc;
   if (want_stats) {
     rc = launch_aux_stats(s.T, s.N, s.k, probs, top_idx, o.f, o.P, o.n_sum_fP, nullptr, b.stats_ws,
                           st);
     if (rc != MOE_OK) return rc;
   }
-  rc = launch_permute(s, top_idx, counts, offsets, perm_tok, row_of, overflow, totals,
-                      b.permute_ws, st);
-  if (rc != MOE_OK) return rc;
-  rc = launch_gather(s, s.d, u, act_dtype, perm_tok, offsets, b.x_rows, st);
+  if (small) {
+    rc = launch_dispatch_small(s, top_idx, hist, counts, offsets, perm_tok, row_of, overflow,
+                               totals, st);
+  } else {
+    rc = launch_permute(s, top_idx, counts, offsets, perm_tok, row_of, overflow, totals,
+                        b.permute_ws, st);
+  }
+  if (rc == MOE_OK) rc = launch_gather(s, s.d, u, act_dtype, perm_tok, offsets, b.x_rows, st);
   if (rc != MOE_OK) return rc;
   rc = run_ffn(s, s.d, b.x_rows, act_dtype, offsets, w->w_gate, w->w_up, w->w_down, w->act,
                b.y_rows, b.ffn_ws, st);

@@ -156,6 +156,107 @@ __global__ void __launch_bounds__(kChunk)
   }
 }
 
+// Permutation in one launch for few experts (N <= 16), from the per-block
+// expert counts the fused router wrote (router block r owns tokens
+// [tpb r, tpb (r+1)), i.e. dispatches [tpb k r, tpb k (r+1))).  Block b of
+// this kernel owns the dispatches of router blocks [R b, R (b+1)) (one thread
+// each; R tpb k is a multiple of 32 near 256).  It loads all the
+// counts into shared memory at once, sums those of the blocks before it (its
+// base ranks) and of all blocks (L_e, offsets), ranks its dispatches stably
+// as permute_scatter does and writes row_of / perm_tok.
+constexpr int kDispatchMaxHist = 8192;  // nblk * N ints held in shared memory
+
+__global__ void __launch_bounds__(512)
+    dispatch_small(const int32_t* __restrict__ idx, int64_t total, int k, int N, int C,
+                   const int32_t* __restrict__ hist, int nblk, int rblk_per_block,
+                   int32_t* __restrict__ counts,
+                   int32_t* __restrict__ offsets, int32_t* __restrict__ overflow,
+                   int32_t* __restrict__ totals, int32_t* __restrict__ perm_tok,
+                   int32_t* __restrict__ row_of, int* status) {
+  pdl_wait();
+  pdl_allow_next();
+  __shared__ int hist_s[kDispatchMaxHist];
+  __shared__ int base_s[16], L_s[16], off_s[17];
+  __shared__ int wcnt[16][16];
+  const int b = blockIdx.x, lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int nh = nblk * N;
+  for (int i0 = threadIdx.x; i0 < nh; i0 += 8 * blockDim.x) {
+    int v[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int i = i0 + j * blockDim.x;
+      v[j] = i < nh ? hist[i] : 0;
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int i = i0 + j * blockDim.x;
+      if (i < nh) hist_s[i] = v[j];
+    }
+  }
+  for (int i = threadIdx.x; i < 16 * 16; i += blockDim.x) (&wcnt[0][0])[i] = 0;
+  __syncthreads();
+  if (threadIdx.x < N) {
+    const int e = threadIdx.x;
+    const int first = b * rblk_per_block;  // first router block of this block's dispatches
+    int base = 0, tot = 0;
+    for (int i = 0; i < nblk; ++i) {
+      const int v = hist_s[i * N + e];
+      base += i < first ? v : 0;
+      tot += v;
+    }
+    base_s[e] = base;
+    L_s[e] = tot;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int run = 0, of = 0, empty = 0;
+    for (int e = 0; e < N; ++e) {
+      const int L = L_s[e];
+      off_s[e] = run;
+      run += (C > 0 && L > C) ? C : L;
+      if (C > 0 && L > C) of += L - C;
+      if (C > 0 && L < C) empty += C - L;
+    }
+    off_s[N] = run;
+    if (b == 0) {
+      for (int e = 0; e < N; ++e) {
+        counts[e] = L_s[e];
+        offsets[e] = off_s[e];
+        overflow[e] = (C > 0 && L_s[e] > C) ? L_s[e] - C : 0;
+      }
+      offsets[N] = run;
+      totals[0] = run;
+      totals[1] = of;
+      totals[2] = empty;
+    }
+  }
+  const int64_t x = (int64_t)b * blockDim.x + threadIdx.x;
+  int e = -1;
+  if (x < total) {
+    e = idx[x];
+    if (e < 0 || e >= N) {
+      record_error(status, MOE_ERR_BOUNDS);
+      e = -1;
+    }
+  }
+  const unsigned peers = __match_any_sync(0xffffffffu, e);
+  const int in_warp = __popc(peers & ((1u << lane) - 1u));
+  if (e >= 0 && in_warp == 0) wcnt[w][e] = __popc(peers);
+  __syncthreads();
+  if (x >= total) return;
+  int row = -1;
+  if (e >= 0) {
+    int cross = 0;
+    for (int v = 0; v < w; ++v) cross += wcnt[v][e];
+    const int rank = base_s[e] + cross + in_warp;
+    if (!(C > 0 && rank >= C)) {
+      row = off_s[e] + rank;
+      perm_tok[row] = (int32_t)(x / k);
+    }
+  }
+  row_of[x] = row;
+}
+
 }  // namespace
 
 size_t permute_ws_bytes(const moe_shape& s) {
@@ -182,6 +283,36 @@ int launch_permute(const moe_shape& s, const int32_t* top_idx, int32_t* counts, 
                                                                s.capacity, hist, offsets,
                                                                perm_tok, row_of);
   }
+  return launch_status();
+}
+
+bool dispatch_small_ok(const moe_shape& s) {
+  const int tpb = route_tokens_per_block(s.N);
+  const int64_t nblk = (s.T + tpb - 1) / tpb;
+  return s.N <= 16 && s.k <= 16 && nblk * s.N <= kDispatchMaxHist;
+}
+
+int launch_dispatch_small(const moe_shape& s, const int32_t* top_idx, const int32_t* hist,
+                          int32_t* counts, int32_t* offsets, int32_t* perm_tok, int32_t* row_of,
+                          int32_t* overflow, int32_t* totals, cudaStream_t st) {
+  const int tpb = route_tokens_per_block(s.N);
+  const int nblk = (s.T + tpb - 1) / tpb;
+  const int per = tpb * s.k;  // dispatches of one router block
+  int g = per, h = 32;        // lcm(per, 32)
+  while (h) {
+    const int t = g % h;
+    g = h;
+    h = t;
+  }
+  const int L = per / g * 32;
+  const int threads = L * (L < 256 ? 256 / L : 1);
+  const int rpb = threads / per;
+  const int64_t total = (int64_t)s.T * s.k;
+  const int blocks = (int)((total + threads - 1) / threads);
+  MOE_PREFER_SHARED((dispatch_small));
+  launch_pdl(dispatch_small, dim3(blocks > 0 ? blocks : 1), dim3(threads), 0, st, top_idx, total,
+             s.k, s.N, s.capacity, hist, nblk, rpb, counts, offsets, overflow, totals, perm_tok,
+             row_of, status_word());
   return launch_status();
 }
 

@@ -172,14 +172,16 @@ __global__ void __launch_bounds__(256)
   }
 }
 
-// Few experts (N <= NP <= 16): one thread per token keeps all N logits in
-// registers and finishes softmax, top-k and the combine weights itself, so
-// routing is a single launch.  Per slab of inputs, the router rows and the
-// block's 32 token rows are copied with cp.async (every copy issued before
-// one wait) into rows padded to 16 B past a multiple of 128 B: the threads'
-// 16-byte token reads hit distinct banks and the router reads are broadcasts.
-// Each logit is the same sequential FMA chain over j as in the tiled kernel.
-constexpr int kTokPerBlock = 32;
+// Few experts (N <= NP <= 16): a block routes 128 / NP tokens with one
+// thread per (token, expert) pair, each running its logit's sequential FMA
+// chain over j (the same order as the tiled kernel), then one thread per
+// token does softmax, top-k and the combine weights from shared memory, so
+// routing is a single launch.  Per slab of inputs the block's token rows and
+// the router rows are copied with cp.async (every copy issued before one
+// wait) into rows padded to 16 B past a multiple of 128 B, so the 16-byte
+// shared-memory reads of a warp hit distinct banks.  Optionally the block
+// also writes its expert counts (the first step of the permutation).
+constexpr int kRouteThreads = 128;
 
 __device__ __forceinline__ void cp16_async(void* smem, const void* gmem) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
@@ -189,28 +191,31 @@ __device__ __forceinline__ void cp16_async(void* smem, const void* gmem) {
 }
 
 template <int NP, typename TU>
-__global__ void __launch_bounds__(kTokPerBlock)
+__global__ void __launch_bounds__(kRouteThreads)
     router_fused_small(const TU* __restrict__ u, const float* __restrict__ w,
                        const float* __restrict__ bias, int T, int d, int N, int k, int renorm,
                        int32_t* __restrict__ top_idx, float* __restrict__ top_w,
-                       float* __restrict__ probs, float* __restrict__ logits) {
+                       float* __restrict__ probs, float* __restrict__ logits,
+                       int32_t* __restrict__ hist) {
   pdl_wait();
   pdl_allow_next();
+  constexpr int TPB = kRouteThreads / NP;               // tokens per block
   constexpr int kSlab = sizeof(TU) == 4 ? 128 : 256;  // 512-byte token slabs
   constexpr int kRowBytes = kSlab * (int)sizeof(TU) + 16;
-  constexpr int kWld = kSlab + 4;                      // padded router row (floats)
+  constexpr int kWld = kSlab + 4;  // padded router row (floats)
   __shared__ __align__(16) float ws[NP][kWld];
-  __shared__ __align__(16) char us[kTokPerBlock * kRowBytes];
-  const int t0 = blockIdx.x * kTokPerBlock;
-  const int t = t0 + threadIdx.x;
-  float acc[NP];
-#pragma unroll
-  for (int e = 0; e < NP; ++e) acc[e] = 0.0f;
+  __shared__ __align__(16) char us[TPB * kRowBytes];
+  __shared__ float zs[TPB][NP + 1];
+  __shared__ int cnt[NP];
+  const int t0 = blockIdx.x * TPB;
+  const int tl = threadIdx.x / NP, e = threadIdx.x - tl * NP;
+  const int t = t0 + tl;
+  float acc = 0.0f;
   for (int k0 = 0; k0 < d; k0 += kSlab) {
     const int kw = min(kSlab, d - k0);  // multiple of 8
     const int chunks = kw * (int)sizeof(TU) / 16;
     __syncthreads();
-    for (int i = threadIdx.x; i < kTokPerBlock * chunks; i += blockDim.x) {
+    for (int i = threadIdx.x; i < TPB * chunks; i += blockDim.x) {
       const int r = i / chunks, c = i - r * chunks;
       if (t0 + r < T)
         cp16_async(us + r * kRowBytes + c * 16,
@@ -218,77 +223,68 @@ __global__ void __launch_bounds__(kTokPerBlock)
     }
     const int wchunks = kw / 4;
     for (int i = threadIdx.x; i < N * wchunks; i += blockDim.x) {
-      const int e = i / wchunks, c = i - e * wchunks;
-      cp16_async(&ws[e][c * 4], w + (size_t)e * d + k0 + c * 4);
+      const int ee = i / wchunks, c = i - ee * wchunks;
+      cp16_async(&ws[ee][c * 4], w + (size_t)ee * d + k0 + c * 4);
     }
     asm volatile("cp.async.wait_all;" ::: "memory");
     __syncthreads();
-    if (t < T) {
-      const TU* ut = reinterpret_cast<const TU*>(us + threadIdx.x * kRowBytes);
+    if (t < T && e < N) {
+      const TU* ut = reinterpret_cast<const TU*>(us + tl * kRowBytes);
+      const float* wt = ws[e];
       for (int j = 0; j < kw; j += 8) {
         float x[8];
         load8(ut + j, x);
-#pragma unroll
-        for (int h4 = 0; h4 < 8; h4 += 4) {
-#pragma unroll
-          for (int e = 0; e < NP; ++e) {
-            if (e < N) {
-              const float4 wv = *reinterpret_cast<const float4*>(&ws[e][j + h4]);
-              acc[e] = __fmaf_rn(wv.x, x[h4], acc[e]);
-              acc[e] = __fmaf_rn(wv.y, x[h4 + 1], acc[e]);
-              acc[e] = __fmaf_rn(wv.z, x[h4 + 2], acc[e]);
-              acc[e] = __fmaf_rn(wv.w, x[h4 + 3], acc[e]);
-            }
-          }
-        }
+        const float4 w0 = *reinterpret_cast<const float4*>(wt + j);
+        const float4 w1 = *reinterpret_cast<const float4*>(wt + j + 4);
+        acc = __fmaf_rn(w0.x, x[0], acc);
+        acc = __fmaf_rn(w0.y, x[1], acc);
+        acc = __fmaf_rn(w0.z, x[2], acc);
+        acc = __fmaf_rn(w0.w, x[3], acc);
+        acc = __fmaf_rn(w1.x, x[4], acc);
+        acc = __fmaf_rn(w1.y, x[5], acc);
+        acc = __fmaf_rn(w1.z, x[6], acc);
+        acc = __fmaf_rn(w1.w, x[7], acc);
       }
     }
   }
-  if (t >= T) return;
-  float zmax = -FLT_MAX;
-#pragma unroll
-  for (int e = 0; e < NP; ++e) {
-    if (e < N) {
-      if (bias) acc[e] = __fadd_rn(acc[e], bias[e]);
-      zmax = fmaxf(zmax, acc[e]);
+  if (e < N) {
+    if (bias) acc = __fadd_rn(acc, bias[e]);
+    zs[tl][e] = acc;
+    if (logits && t < T) logits[(size_t)t * N + e] = acc;
+  }
+  if (hist && threadIdx.x < NP) cnt[threadIdx.x] = 0;
+  __syncthreads();
+  if (threadIdx.x < TPB && t0 + threadIdx.x < T) {
+    const int tt = t0 + threadIdx.x;
+    const float* z = zs[threadIdx.x];
+    float zmax = -FLT_MAX;
+    for (int i = 0; i < N; ++i) zmax = fmaxf(zmax, z[i]);
+    float den = 0.0f;
+    for (int i = 0; i < N; ++i) den += expf(z[i] - zmax);
+    if (probs)
+      for (int i = 0; i < N; ++i) probs[(size_t)tt * N + i] = expf(z[i] - zmax) / den;
+    uint32_t taken = 0;
+    float psel[16];
+    int isel[16];
+    float ps = 0.0f;
+    for (int s = 0; s < k; ++s) {
+      int bi = -1;
+      for (int i = 0; i < N; ++i)
+        if (!((taken >> i) & 1u) && (bi < 0 || z[i] > z[bi])) bi = i;
+      taken |= 1u << bi;
+      isel[s] = bi;
+      psel[s] = expf(z[bi] - zmax) / den;
+      ps += psel[s];
+    }
+    for (int s = 0; s < k; ++s) {
+      top_idx[(size_t)tt * k + s] = isel[s];
+      top_w[(size_t)tt * k + s] = renorm ? psel[s] / ps : psel[s];
+      if (hist) atomicAdd(&cnt[isel[s]], 1);
     }
   }
-  float den = 0.0f;
-#pragma unroll
-  for (int e = 0; e < NP; ++e)
-    if (e < N) den += expf(acc[e] - zmax);
-  if (logits) {
-#pragma unroll
-    for (int e = 0; e < NP; ++e)
-      if (e < N) logits[(size_t)t * N + e] = acc[e];
-  }
-  if (probs) {
-#pragma unroll
-    for (int e = 0; e < NP; ++e)
-      if (e < N) probs[(size_t)t * N + e] = expf(acc[e] - zmax) / den;
-  }
-  uint32_t taken = 0;
-  float psel[16];
-  int isel[16];
-  float ps = 0.0f;
-  for (int s = 0; s < k; ++s) {
-    float bz = -FLT_MAX;
-    int bi = -1;
-#pragma unroll
-    for (int e = 0; e < NP; ++e) {
-      if (e < N && !((taken >> e) & 1u) && (bi < 0 || acc[e] > bz)) {
-        bz = acc[e];
-        bi = e;
-      }
-    }
-    taken |= 1u << bi;
-    isel[s] = bi;
-    psel[s] = expf(bz - zmax) / den;
-    ps += psel[s];
-  }
-  for (int s = 0; s < k; ++s) {
-    top_idx[(size_t)t * k + s] = isel[s];
-    top_w[(size_t)t * k + s] = renorm ? psel[s] / ps : psel[s];
+  if (hist) {  // this block's expert counts: the first step of the permutation
+    __syncthreads();
+    for (int i = threadIdx.x; i < N; i += blockDim.x) hist[(size_t)blockIdx.x * N + i] = cnt[i];
   }
 }
 
@@ -314,19 +310,22 @@ void launch_logits(const TU* u, const float* w, const float* bias, float* z, int
 
 size_t route_ws_bytes(const moe_shape& s) { return align_up((size_t)s.T * s.N * 4, 256); }
 
+int route_tokens_per_block(int N) { return kRouteThreads / (N <= 8 ? 8 : 16); }
+
 int launch_route(const moe_shape& s, const void* u, int32_t u_dtype, const float* w_route,
                  const float* bias, int32_t* top_idx, float* top_w, float* probs, float* logits,
-                 void* ws, cudaStream_t st) {
+                 void* ws, cudaStream_t st, int32_t* hist) {
   if (s.T == 0) return MOE_OK;
   if (s.N <= 16) {
-    const int blocks = (s.T + kTokPerBlock - 1) / kTokPerBlock;
+    const int blocks = (s.T + route_tokens_per_block(s.N) - 1) / route_tokens_per_block(s.N);
 #define MOE_FUSED(NP, TU)                                                                     \
   do {                                                                                        \
     MOE_PREFER_SHARED((router_fused_small<NP, TU>));                                          \
-    launch_pdl(router_fused_small<NP, TU>, dim3(blocks), dim3(kTokPerBlock), 0, st, static_cast<const TU*>(u),     \
+    launch_pdl(router_fused_small<NP, TU>, dim3(blocks), dim3(kRouteThreads), 0, st,           \
+               static_cast<const TU*>(u),                                                       \
                                                                 w_route,                        \
                                                       bias, s.T, s.d, s.N, s.k, s.renorm,     \
-                                                      top_idx, top_w, probs, logits);         \
+                                                      top_idx, top_w, probs, logits, hist);   \
   } while (0)
     if (u_dtype == MOE_F32) {
       if (s.N <= 8) MOE_FUSED(8, float); else MOE_FUSED(16, float);
