@@ -563,11 +563,15 @@ def main():
     ap.add_argument("--workload", default="small",
                     choices=["small", "mixtral", "tiny", "decode", "latent"])
     ap.add_argument("--decode-T", type=int, default=32, help="decode batch (1, 8 or 32)")
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="override T (smaller cases for profiling captures)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     wl = W.decode(T=args.decode_T) if args.workload == "decode" else W.ALL[args.workload]()
+    if args.tokens > 0 and args.workload != "decode":
+        wl.T = args.tokens
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -666,13 +670,16 @@ def main():
 
     # roofline of the dominant kernel: the tcgen05 grouped GEMM (gate/up + down launches)
     hbm, tf_burst, tf_sust, peak_src = _peaks()
+    fused = (wl.h % 64 == 0 and wl.h <= 256 and wl.d % 128 == 0
+             and (wl.h // 64 + wl.d // 128) * 64 <= 512)
     kept_timed = [kept[i % n_rep] for i in range(args.steps)]
     gemm_flops = sum(6.0 * wl.d * wl.h * kr for kr in kept_timed)
     gemm_s = sum(ffn_ms) / 1e3
     achieved_tf = gemm_flops / gemm_s / 1e12
     roofline = {"bound": "tensor", "achieved": achieved_tf, "peak": tf_burst, "unit": "TFLOP/s",
                 "frac": achieved_tf / tf_burst, "traffic": None,
-                "kernel": "tc_grouped_gemm (gate/up + down, 2 launches per step, graph replay)",
+                "kernel": ("tc_fused_ffn (gate/up + SwiGLU + down in one launch, H on chip)"
+                           if fused else "tc_grouped_gemm (gate/up + down, 2 launches per step)"),
                 "peak_source": f"{peak_src} bf16_tflops (burst)",
                 "ms_per_launch_pair": gemm_s / args.steps * 1e3}
 
