@@ -277,7 +277,11 @@ typedef struct {
 } moe_q4_layer;
 
 /* Limits: T <= 32, N <= 64, k <= 8, d % 32 == 0, h % 32 == 0, h / 32 a
- * divisor of 32.  Returns 0 for shapes outside them. */
+ * divisor of 32, and the kernel's per-CTA shared-memory plan (token rows,
+ * router rows, one phase-A item, the selected experts' down rows of one
+ * output slice) within 226 KB.  Returns 0 for shapes outside them.  The
+ * workspace holds the hidden vectors, the routing scratch, the chained
+ * activations and the grid-barrier words; one call at a time per workspace. */
 MOE_API size_t moe_decode_workspace_bytes(const moe_shape* shape);
 
 /* One decode layer: u [T][d] fp16 (bit patterns) -> y [T][d] fp16, the
@@ -291,8 +295,11 @@ MOE_API int moe_decode_layer(const moe_shape* shape, const moe_q4_layer* layer, 
 
 /* n_layers chained layers: u_{l+1} = fp16(u_l + y_l), u_out = u_{n_layers}.
  * `layers` is a host array of n_layers structs.  top_idx_all [n_layers][T][k]
- * (nullable) receives every layer's routing.  Same kernels as
- * moe_decode_layer, so a chain equals the layer calls made one by one. */
+ * (nullable) receives every layer's routing.  Up to 32 layers run in one
+ * cooperative launch (one CTA per SM, two grid barriers per layer, every
+ * barrier wait bounded: MOE_ERR_TIMEOUT in the device status word).  Same
+ * kernel and per-layer arithmetic as moe_decode_layer, so a chain equals the
+ * layer calls made one by one.  Capturable in a CUDA graph. */
 MOE_API int moe_decode_step(const moe_shape* shape, int32_t n_layers, const moe_q4_layer* layers,
                             const uint16_t* u0, uint16_t* u_out, int32_t* top_idx_all, void* ws,
                             size_t ws_bytes, void* stream);

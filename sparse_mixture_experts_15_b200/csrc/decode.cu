@@ -7,19 +7,28 @@
 // MoE: how sparse activation saves compute" §3.1-§3.2 fixes the arithmetic.
 // Layers chain as u_{l+1} = fp16(u_l + y_l).
 //
-// Per layer two phases, each one launch:
-//   decode_gateup (grid = experts x 16-row hidden slices): every CTA stages
-//     u and W_route in shared memory and routes all T tokens itself (the
-//     router is tiny: N x d fp32), leaves at once if
-//     no token selected its expert (so unselected weights are never read),
-//     otherwise dequantises its 16 gate + 16 up rows in registers and writes
-//     H[e][t][slice] = SiLU(g) * u for its tokens.
-//   decode_down (grid = 32-row slices of the output): stages the H row of
-//     every (token, slot) in shared memory; for every selected expert,
-//     dequantises its down rows once and forms each (token, slot) dot with
-//     H, then sums the slots in order: y = sum_s a_s W_down H,
-//     u_next = fp16(u + y).
-// Weights are streamed with 16-byte loads and dequantised in registers.
+// At decode sizes a layer moves well under a megabyte, so the step is bound
+// by its chain of dependent phases, not by HBM.  All layers of a call run in
+// ONE persistent cooperative launch (one CTA per SM, all co-resident), with
+// two grid barriers per layer instead of two kernel boundaries:
+//   route   every CTA stages u_l and W_route (fp32) in shared memory and
+//           routes all T tokens itself (identical, deterministic code, so
+//           every CTA holds the same selection); the pairs are grouped by
+//           expert.  (The next layer's router rows are fetched while the
+//           CTA waits at the first barrier.)
+//   phase A items (selected expert, RA hidden rows) are spread over the
+//           CTAs: the item's gate/up q4 rows are staged, dequantised once
+//           into shared fp32, and every (row, token) dot is formed;
+//           H[e][t][rows] = SiLU(g) * v goes to global memory (L2).
+//   barrier
+//   phase B slices of RB output rows: the selected experts' down rows of the
+//           slice were staged before the barrier; every (token, slot) pair
+//           dots its H row with them, the slots are summed in order,
+//           y = sum_s a_s W_down H, u_{l+1} = fp16(u_l + y).
+//   barrier
+// Unselected experts' weights are never read.  Every barrier wait is bounded
+// (2 s of device time); on timeout the kernel records MOE_ERR_TIMEOUT, raises
+// an abort flag that releases every other CTA, and all CTAs return.
 #include <cfloat>
 
 #include "common.cuh"
@@ -27,12 +36,21 @@
 namespace moe {
 namespace {
 
-constexpr int kRowsA = 16;    // hidden rows per gate/up CTA (x2: gate and up)
-constexpr int kRowsB = 32;    // output rows per down CTA
-constexpr int kMaxT = 32;     // decode batch limit
-constexpr int kMaxN = 64;     // expert limit of the decode kernels
+constexpr int kThreads = 256;
+constexpr int kMaxT = 32;            // decode batch limit
+constexpr int kMaxN = 64;            // expert limit (64-bit selection mask)
+constexpr int kLayersPerLaunch = 32; // layer descriptors carried by one launch
+constexpr size_t kSmemLimit = 226 * 1024;  // dynamic; leaves room for static
+constexpr unsigned long long kBarrierBudgetNs = 2000000000ull;
 
 __device__ __forceinline__ float f16f(uint16_t c) { return __half2float(__ushort_as_half(c)); }
+
+// q - 8 as fp32 for the 4 nibbles (each 0..15) held in the bytes of v:
+// the bytes are placed under the exponent of 2^23, so the float is 2^23 + q
+// exactly, and subtracting 2^23 + 8 is exact too (no int-to-float convert).
+__device__ __forceinline__ float nib(uint32_t v, int b) {
+  return __uint_as_float(__byte_perm(v, 0x4B000000u, 0x7540 | b)) - 8388616.0f;
+}
 
 // 32 weights of one q4_0 block: byte j -> element j (low nibble), j+16 (high).
 __device__ __forceinline__ void dequant_block(const uint8_t* qs, uint16_t scale, float* w) {
@@ -41,19 +59,36 @@ __device__ __forceinline__ void dequant_block(const uint8_t* qs, uint16_t scale,
   const uint32_t wd[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
+    const uint32_t lo = wd[i] & 0x0F0F0F0Fu, hi = (wd[i] >> 4) & 0x0F0F0F0Fu;
 #pragma unroll
     for (int b = 0; b < 4; ++b) {
-      const uint32_t byte = (wd[i] >> (8 * b)) & 0xFFu;
-      w[4 * i + b] = (float)((int)(byte & 0xFu) - 8) * s;
-      w[16 + 4 * i + b] = (float)((int)(byte >> 4) - 8) * s;
+      w[4 * i + b] = nib(lo, b) * s;
+      w[16 + 4 * i + b] = nib(hi, b) * s;
     }
   }
 }
 
-// 16-byte global -> shared copies issued without waiting (LDGSTS); one wait
-// afterwards pays a single memory latency for the whole staging.
+// Elements 4c..4c+3 of a q4_0 block (c < 4: low nibbles of bytes 4c..4c+3;
+// c >= 4: high nibbles of bytes 4(c-4)..).  Eight threads with consecutive c
+// write one block's 128 bytes as consecutive 16-byte pieces.
+__device__ __forceinline__ float4 dequant_quad(const uint8_t* qs, uint16_t scale, int c) {
+  const uint32_t word = reinterpret_cast<const uint32_t*>(qs)[c & 3];
+  const uint32_t v = (c < 4 ? word : word >> 4) & 0x0F0F0F0Fu;
+  const float s = f16f(scale);
+  return make_float4(nib(v, 0) * s, nib(v, 1) * s, nib(v, 2) * s, nib(v, 3) * s);
+}
+
+// Asynchronous global -> shared copies (LDGSTS), all issued before one wait.
+// The .cg form reads through L2 only, so data written by other CTAs of this
+// launch before a grid barrier is seen.
 __device__ __forceinline__ void cp16(void* smem, const void* gmem) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
+                   static_cast<uint32_t>(__cvta_generic_to_shared(smem))),
+               "l"(gmem)
+               : "memory");
+}
+__device__ __forceinline__ void cp4(void* smem, const void* gmem) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(
                    static_cast<uint32_t>(__cvta_generic_to_shared(smem))),
                "l"(gmem)
                : "memory");
@@ -62,8 +97,8 @@ __device__ __forceinline__ void cp_wait_all() {
   asm volatile("cp.async.wait_all;" ::: "memory");
 }
 
-// Copies rows x row_bytes (multiple of 16) from gmem (row stride g_stride
-// bytes) to smem rows of s_stride bytes, all threads of the CTA cooperating.
+// rows x row_bytes (multiple of 16) from gmem (row stride g_stride bytes) to
+// shared rows of s_stride bytes; all threads of the CTA cooperate.
 __device__ __forceinline__ void stage_rows(char* smem, int s_stride, const char* gmem,
                                            size_t g_stride, int rows, int row_bytes) {
   const int per_row = row_bytes / 16;
@@ -73,263 +108,613 @@ __device__ __forceinline__ void stage_rows(char* smem, int s_stride, const char*
   }
 }
 
+// A contiguous byte range (both ends 4-byte aligned) to shared memory, in
+// 16-byte copies when both addresses and the size allow it.
+__device__ __forceinline__ void stage_bytes(void* smem, const void* gmem, int nbytes) {
+  char* s = static_cast<char*>(smem);
+  const char* g = static_cast<const char*>(gmem);
+  if (((reinterpret_cast<uintptr_t>(s) | reinterpret_cast<uintptr_t>(g) | (uintptr_t)nbytes) &
+       15u) == 0) {
+    for (int i = threadIdx.x; i < nbytes / 16; i += blockDim.x) cp16(s + 16 * i, g + 16 * i);
+  } else {
+    for (int i = threadIdx.x; i < nbytes / 4; i += blockDim.x) cp4(s + 4 * i, g + 4 * i);
+  }
+}
+
+// Softmax and top-k of one token for N up to 64, logits read from shared
+// memory (the register version above covers N <= 32).
+__device__ __noinline__ void topk_wide(const float* zt, int N, int k, int renorm, int* sel,
+                                       float* aw) {
+  float zmax = -FLT_MAX;
+  for (int i = 0; i < N; ++i) zmax = fmaxf(zmax, zt[i]);
+  float den = 0.0f;
+  for (int i = 0; i < N; ++i) den += expf(zt[i] - zmax);
+  uint64_t taken = 0;
+  float ps = 0.0f;
+  float a[8];
+  for (int s = 0; s < k; ++s) {
+    int bi = -1;
+    for (int i = 0; i < N; ++i)
+      if (!((taken >> i) & 1ull) && (bi < 0 || zt[i] > zt[bi])) bi = i;
+    if (bi < 0) bi = __ffsll((long long)~taken) - 1;  // only NaN logits left
+    taken |= 1ull << bi;
+    sel[s] = bi;
+    a[s] = expf(zt[bi] - zmax) / den;
+    ps += a[s];
+  }
+  for (int s = 0; s < k; ++s) aw[s] = renorm ? a[s] / ps : a[s];
+}
+
 // Routing of all T tokens inside one CTA from u_s [T] rows (fp16, row stride
-// us_ld elements) and w_s [N] rows (fp32, stride ws_ld), both staged in
-// shared memory with a 16-byte pad per row so the threads of a warp
-// (consecutive (t, i) pairs) hit distinct banks.  z is the sequential fp32
-// FMA chain over j (the order the oracle uses); ties go to the lower expert
-// index.  Leaves sel[t][s] and aw[t][s] in shared memory.
+// us_ld elements) and w_s [N] rows (fp32, stride ws_ld), both in shared
+// memory with a 16-byte pad per row so the threads of a warp (consecutive
+// (t, i) pairs) hit distinct banks.  z is the sequential fp32 FMA chain over
+// j (the order the oracle uses); the shared-memory operands of the next 8
+// elements are loaded while the current 8 FMAs run.  Ties go to the lower
+// expert index.  Leaves sel[t][s] and
+// aw[t][s] in shared memory.
+__device__ __forceinline__ void fma8(float& a, const uint4& xu, const float4& w0,
+                                     const float4& w1) {
+  const float2 x0 = __half22float2(*reinterpret_cast<const __half2*>(&xu.x));
+  const float2 x1 = __half22float2(*reinterpret_cast<const __half2*>(&xu.y));
+  const float2 x2 = __half22float2(*reinterpret_cast<const __half2*>(&xu.z));
+  const float2 x3 = __half22float2(*reinterpret_cast<const __half2*>(&xu.w));
+  a = __fmaf_rn(w0.x, x0.x, a);
+  a = __fmaf_rn(w0.y, x0.y, a);
+  a = __fmaf_rn(w0.z, x1.x, a);
+  a = __fmaf_rn(w0.w, x1.y, a);
+  a = __fmaf_rn(w1.x, x2.x, a);
+  a = __fmaf_rn(w1.y, x2.y, a);
+  a = __fmaf_rn(w1.z, x3.x, a);
+  a = __fmaf_rn(w1.w, x3.y, a);
+}
+
+// Softmax, top-k and combine weights of one token from its N logits zt.
+template <int NR>
+__device__ __forceinline__ void topk_token(const float* zt, int N, int k, int renorm, int* sel,
+                                           float* aw) {
+  float zr[NR];
+#pragma unroll
+  for (int i = 0; i < NR; ++i) zr[i] = i < N ? zt[i] : 0.0f;
+  float zmax = -FLT_MAX;
+#pragma unroll
+  for (int i = 0; i < NR; ++i)
+    if (i < N) zmax = fmaxf(zmax, zr[i]);
+  float den = 0.0f;
+#pragma unroll
+  for (int i = 0; i < NR; ++i)
+    if (i < N) den += expf(zr[i] - zmax);
+  uint32_t taken = 0;
+  float ps = 0.0f;
+  float a[8];
+  for (int s = 0; s < k; ++s) {
+    int bi = -1;
+    float bz = 0.0f;
+#pragma unroll
+    for (int i = 0; i < NR; ++i)
+      if (i < N && !((taken >> i) & 1u) && (bi < 0 || zr[i] > bz)) {
+        bi = i;
+        bz = zr[i];
+      }
+    if (bi < 0) {  // only NaN logits left: take the lowest free index
+      bi = __ffs(~taken) - 1;
+      bz = zr[0];
+#pragma unroll
+      for (int i = 0; i < NR; ++i)
+        if (i == bi) bz = zr[i];
+    }
+    taken |= 1u << bi;
+    sel[s] = bi;
+    a[s] = expf(bz - zmax) / den;
+    ps += a[s];
+  }
+  for (int s = 0; s < k; ++s) aw[s] = renorm ? a[s] / ps : a[s];
+}
+
 __device__ void route_in_cta(const __half* u_s, int us_ld, const float* w_s, int ws_ld, int T,
                              int d, int N, int k, int renorm, const float* __restrict__ bias,
                              float* z, int* sel, float* aw) {
-  const int pairs = T * N;
-  for (int p = threadIdx.x; p < pairs; p += blockDim.x) {
-    const int t = p / N, i = p - t * N;
-    const __half2* ut = reinterpret_cast<const __half2*>(u_s + (size_t)t * us_ld);
-    const float2* wi = reinterpret_cast<const float2*>(w_s + (size_t)i * ws_ld);
-    float a = 0.0f;
-#pragma unroll 8
-    for (int j = 0; j < d / 2; ++j) {
-      const float2 x = __half22float2(ut[j]);
-      const float2 v = wi[j];
-      a = __fmaf_rn(v.x, x.x, a);
-      a = __fmaf_rn(v.y, x.y, a);
+  const int steps = d / 8;
+  if (T >= 16) {
+    // a thread forms the chains of two experts (i, i + 1) for one token, so
+    // each activation load feeds both; a warp holds 32 tokens of one expert
+    // pair, whose router rows are shared-memory broadcasts.
+    const int npair = (N + 1) / 2, units = T * npair;
+    for (int uu = threadIdx.x; uu < units; uu += blockDim.x) {
+      const int ip = uu / T, t = uu - ip * T;
+      const int i0 = 2 * ip, i1 = i0 + 1 < N ? i0 + 1 : i0;
+      const uint4* ut = reinterpret_cast<const uint4*>(u_s + (size_t)t * us_ld);
+      const float4* w0r = reinterpret_cast<const float4*>(w_s + (size_t)i0 * ws_ld);
+      const float4* w1r = reinterpret_cast<const float4*>(w_s + (size_t)i1 * ws_ld);
+      float a = 0.0f, b = 0.0f;
+      uint4 xu = ut[0];
+      float4 wa0 = w0r[0], wa1 = w0r[1], wb0 = w1r[0], wb1 = w1r[1];
+      for (int c = 0; c + 1 < steps; ++c) {
+        const uint4 nxu = ut[c + 1];
+        const float4 nwa0 = w0r[2 * c + 2], nwa1 = w0r[2 * c + 3];
+        const float4 nwb0 = w1r[2 * c + 2], nwb1 = w1r[2 * c + 3];
+        fma8(a, xu, wa0, wa1);
+        fma8(b, xu, wb0, wb1);
+        xu = nxu;
+        wa0 = nwa0;
+        wa1 = nwa1;
+        wb0 = nwb0;
+        wb1 = nwb1;
+      }
+      fma8(a, xu, wa0, wa1);
+      fma8(b, xu, wb0, wb1);
+      z[t * N + i0] = bias ? __fadd_rn(a, bias[i0]) : a;
+      if (i1 != i0) z[t * N + i1] = bias ? __fadd_rn(b, bias[i1]) : b;
     }
-    z[p] = bias ? __fadd_rn(a, bias[i]) : a;
+  } else {
+    for (int p = threadIdx.x; p < T * N; p += blockDim.x) {
+      const int t = p / N, i = p - t * N;
+      const uint4* ut = reinterpret_cast<const uint4*>(u_s + (size_t)t * us_ld);
+      const float4* wi = reinterpret_cast<const float4*>(w_s + (size_t)i * ws_ld);
+      float a = 0.0f;
+      uint4 xu = ut[0];
+      float4 w0 = wi[0], w1 = wi[1];
+      for (int c = 0; c + 1 < steps; ++c) {  // next 8 elements loaded under this step's FMAs
+        const uint4 nxu = ut[c + 1];
+        const float4 nw0 = wi[2 * c + 2], nw1 = wi[2 * c + 3];
+        fma8(a, xu, w0, w1);
+        xu = nxu;
+        w0 = nw0;
+        w1 = nw1;
+      }
+      fma8(a, xu, w0, w1);
+      z[p] = bias ? __fadd_rn(a, bias[i]) : a;
+    }
   }
   __syncthreads();
   for (int t = threadIdx.x; t < T; t += blockDim.x) {
-    const float* zt = z + t * N;
-    float zmax = -FLT_MAX;
-    for (int i = 0; i < N; ++i) zmax = fmaxf(zmax, zt[i]);
-    float den = 0.0f;
-    for (int i = 0; i < N; ++i) den += expf(zt[i] - zmax);
-    uint64_t taken = 0;
-    float ps = 0.0f;
-    for (int s = 0; s < k; ++s) {
-      int bi = -1;
-      for (int i = 0; i < N; ++i)
-        if (!((taken >> i) & 1ull) && (bi < 0 || zt[i] > zt[bi])) bi = i;
-      taken |= 1ull << bi;
-      sel[t * k + s] = bi;
-      aw[t * k + s] = expf(zt[bi] - zmax) / den;
-      ps += aw[t * k + s];
-    }
-    if (renorm)
-      for (int s = 0; s < k; ++s) aw[t * k + s] /= ps;
+    if (N <= 8)
+      topk_token<8>(z + t * N, N, k, renorm, sel + t * k, aw + t * k);
+    else if (N <= 32)
+      topk_token<32>(z + t * N, N, k, renorm, sel + t * k, aw + t * k);
+    else
+      topk_wide(z + t * N, N, k, renorm, sel + t * k, aw + t * k);
   }
   __syncthreads();
 }
 
-__global__ void __launch_bounds__(128)
-    decode_gateup(const __half* __restrict__ u, int T, int d, int N, int k, int h, int renorm,
-                  const float* __restrict__ w_route, const float* __restrict__ bias,
-                  const uint8_t* __restrict__ gq, const uint16_t* __restrict__ gs,
-                  const uint8_t* __restrict__ uq, const uint16_t* __restrict__ us,
-                  float* __restrict__ H, int32_t* __restrict__ top_idx, float* __restrict__ top_w) {
-  pdl_wait();
-  pdl_allow_next();
-  extern __shared__ __align__(16) char dyn[];
-  const int us_ld = d + 8, ws_ld = d + 4, nb = d / 32;
-  __half* u_s = reinterpret_cast<__half*>(dyn);                          // [T][d+8]
-  float* w_s = reinterpret_cast<float*>(dyn + (size_t)T * us_ld * 2);     // [N][d+4]
-  uint8_t* q_s = reinterpret_cast<uint8_t*>(w_s + (size_t)N * ws_ld);     // [32][d/2]
-  uint16_t* sc_s = reinterpret_cast<uint16_t*>(q_s + 2 * kRowsA * (d / 2));  // [32][d/32]
-  __shared__ float z[kMaxT * kMaxN];
-  __shared__ int sel[kMaxT * 8];
-  __shared__ float aw[kMaxT * 8];
-  __shared__ int toks[kMaxT];
-  __shared__ int ntok;
-  __shared__ float gu[2 * kRowsA][kMaxT + 1];
-  const int slices = h / kRowsA;
-  const int e = blockIdx.x / slices, slice = blockIdx.x - e * slices;
-  stage_rows(reinterpret_cast<char*>(u_s), us_ld * 2, reinterpret_cast<const char*>(u),
-             (size_t)d * 2, T, d * 2);
-  stage_rows(reinterpret_cast<char*>(w_s), ws_ld * 4, reinterpret_cast<const char*>(w_route),
-             (size_t)d * 4, N, d * 4);
-  cp_wait_all();
+// ------------------------------------------------------------- grid barrier
+__device__ __forceinline__ unsigned ld_acquire(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ unsigned long long global_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Arrival counter bar[0] (zeroed before the launch) and abort flag bar[1].
+// Barrier number n of the launch completes when bar[0] reaches G * (n + 1).
+// grid_arrive: after the CTA's own work (bar.sync), thread 0 publishes it
+// (fence.acq_rel at gpu scope, then a relaxed add).  The CTA may issue
+// independent copies before grid_wait, which polls with acquire loads and
+// returns false (every CTA then returns) on timeout or abort.
+__device__ __forceinline__ void grid_arrive(unsigned* bar) {
   __syncthreads();
-  route_in_cta(u_s, us_ld, w_s, ws_ld, T, d, N, k, renorm, bias, z, sel, aw);
-  if (blockIdx.x == 0) {
-    for (int x = threadIdx.x; x < T * k; x += blockDim.x) {
-      top_idx[x] = sel[x];
-      if (top_w) top_w[x] = aw[x];
-    }
-  }
+  if (threadIdx.x == 0)
+    asm volatile("fence.acq_rel.gpu;\n\tred.relaxed.gpu.global.add.u32 [%0], 1;" ::"l"(bar)
+                 : "memory");
+}
+
+__device__ bool grid_wait(unsigned* bar, unsigned target, int* status) {
+  __shared__ int ok;
   if (threadIdx.x == 0) {
-    int n = 0;
-    for (int t = 0; t < T; ++t) {
-      bool hit = false;
-      for (int s = 0; s < k; ++s) hit |= sel[t * k + s] == e;
-      if (hit) toks[n++] = t;
-    }
-    ntok = n;
-  }
-  __syncthreads();
-  const int n = ntok;
-  if (n == 0) return;  // expert not selected: its weights are never read
-
-  // stage this CTA's 16 gate + 16 up rows (q4 bytes and scales) in one go
-  const size_t row_g = (size_t)e * h + slice * kRowsA;
-  stage_rows(reinterpret_cast<char*>(q_s), d / 2, reinterpret_cast<const char*>(gq + row_g * (d / 2)),
-             d / 2, kRowsA, d / 2);
-  stage_rows(reinterpret_cast<char*>(q_s + kRowsA * (d / 2)), d / 2,
-             reinterpret_cast<const char*>(uq + row_g * (d / 2)), d / 2, kRowsA, d / 2);
-  if (nb * 2 >= 16) {
-    stage_rows(reinterpret_cast<char*>(sc_s), nb * 2,
-               reinterpret_cast<const char*>(gs + row_g * nb), (size_t)nb * 2, kRowsA, nb * 2);
-    stage_rows(reinterpret_cast<char*>(sc_s + kRowsA * nb), nb * 2,
-               reinterpret_cast<const char*>(us + row_g * nb), (size_t)nb * 2, kRowsA, nb * 2);
-  } else {
-    for (int i = threadIdx.x; i < 2 * kRowsA * nb; i += blockDim.x) {
-      const int r = i / nb, c = i - r * nb;
-      sc_s[i] = (r < kRowsA ? gs : us)[(row_g + (r % kRowsA)) * nb + c];
-    }
-  }
-  cp_wait_all();
-  __syncthreads();
-
-  // (row, token) dots: consecutive threads take consecutive tokens of the
-  // same weight row (the row's bytes are a shared-memory broadcast).
-  for (int p = threadIdx.x; p < 2 * kRowsA * n; p += blockDim.x) {
-    const int r = p / n, i = p - r * n;
-    const uint8_t* q = q_s + (size_t)r * (d / 2);
-    const uint16_t* sc = sc_s + (size_t)r * nb;
-    const __half2* ut = reinterpret_cast<const __half2*>(u_s + (size_t)toks[i] * us_ld);
-    float a0 = 0.0f, a1 = 0.0f;
-    for (int bb = 0; bb < nb; ++bb) {
-      float w[32];
-      dequant_block(q + bb * 16, sc[bb], w);
-#pragma unroll
-      for (int c = 0; c < 16; ++c) {
-        const float2 x = __half22float2(ut[bb * 16 + c]);
-        a0 = fmaf(w[2 * c], x.x, a0);
-        a1 = fmaf(w[2 * c + 1], x.y, a1);
-      }
-    }
-    gu[r][i] = a0 + a1;
-  }
-  __syncthreads();
-  for (int x = threadIdx.x; x < n * kRowsA; x += blockDim.x) {
-    const int i = x / kRowsA, r = x - i * kRowsA;
-    H[((size_t)e * T + toks[i]) * h + slice * kRowsA + r] = silu(gu[r][i]) * gu[kRowsA + r][i];
-  }
-}
-
-__global__ void __launch_bounds__(128)
-    decode_down(const __half* __restrict__ u, int T, int d, int N, int k, int h,
-                const int32_t* __restrict__ top_idx, const float* __restrict__ top_w,
-                const uint8_t* __restrict__ dq, const uint16_t* __restrict__ dsc,
-                const float* __restrict__ H, __half* __restrict__ y, __half* __restrict__ u_next,
-                int* status) {
-  pdl_wait();
-  pdl_allow_next();
-  extern __shared__ __align__(16) char dyn[];
-  const int TKmax = T * k, h_ld = h + 4;
-  float* hs = reinterpret_cast<float*>(dyn);  // [T*k][h+4]: H row of each (token, slot)
-  uint8_t* q_s = reinterpret_cast<uint8_t*>(hs + (size_t)TKmax * h_ld);  // [N][32][h/2]
-  uint16_t* sc_s = reinterpret_cast<uint16_t*>(q_s + (size_t)N * kRowsB * (h / 2));
-  __shared__ float yslot[kMaxT * 8][kRowsB + 1];
-  __shared__ int sel[kMaxT * 8];
-  __shared__ int list[kMaxT * 8];  // pairs grouped by expert (counting sort)
-  __shared__ int start[kMaxN + 1];
-  const int nb = h / 32;  // q4 blocks per down row
-  const int row0 = blockIdx.x * kRowsB;
-  const int TK = T * k;
-  if (threadIdx.x == 0) {  // pairs grouped by expert, in (token, slot) order
-    int cnt[kMaxN];
-    for (int e = 0; e < N; ++e) cnt[e] = 0;
-    for (int x = 0; x < TK; ++x) {
-      int e = top_idx[x];
-      if (e < 0 || e >= N) {
-        record_error(status, MOE_ERR_BOUNDS);
-        e = 0;
-      }
-      sel[x] = e;
-      ++cnt[e];
-    }
-    int run = 0;
-    for (int e = 0; e < N; ++e) {
-      start[e] = run;
-      run += cnt[e];
-      cnt[e] = start[e];
-    }
-    start[N] = run;
-    for (int x = 0; x < TK; ++x) list[cnt[sel[x]]++] = x;
-  }
-  __syncthreads();
-  for (int i = threadIdx.x; i < TK * (h / 4); i += blockDim.x) {
-    const int x = i / (h / 4), c = i - x * (h / 4);
-    cp16(hs + (size_t)x * h_ld + c * 4, H + ((size_t)sel[x] * T + x / k) * h + c * 4);
-  }
-  for (int e = 0; e < N; ++e) {  // only the selected experts' rows are read
-    if (start[e + 1] == start[e]) continue;
-    const size_t row = (size_t)e * d + row0;
-    stage_rows(reinterpret_cast<char*>(q_s + (size_t)e * kRowsB * (h / 2)), h / 2,
-               reinterpret_cast<const char*>(dq + row * (h / 2)), h / 2, kRowsB, h / 2);
-    for (int i = threadIdx.x; i < kRowsB * nb; i += blockDim.x)
-      sc_s[(size_t)e * kRowsB * nb + i] = dsc[row * nb + i];
-  }
-  cp_wait_all();
-  __syncthreads();
-  // thread = (row r, quarter q): row r of the selected expert, pairs q, q+4, ...
-  const int r = threadIdx.x & (kRowsB - 1), q = threadIdx.x >> 5;
-  // a token selects an expert at most once, so an expert has <= T <= 32 pairs
-  constexpr int kPer = kMaxT / 4;
-  for (int e = 0; e < N; ++e) {
-    const int ne = start[e + 1] - start[e];
-    const int* le = list + start[e];
-    if (ne == 0) continue;  // unselected expert: nothing read
-    const uint8_t* qrow = q_s + ((size_t)e * kRowsB + r) * (h / 2);
-    const uint16_t* srow = sc_s + ((size_t)e * kRowsB + r) * nb;
-    float acc[kPer];
-#pragma unroll
-    for (int j = 0; j < kPer; ++j) acc[j] = 0.0f;
-    for (int bb = 0; bb < nb; ++bb) {
-      float w[32];
-      dequant_block(qrow + bb * 16, srow[bb], w);
-#pragma unroll
-      for (int j = 0; j < kPer; ++j) {
-        const int li = q + 4 * j;
-        if (li < ne) {
-          const float4* hc = reinterpret_cast<const float4*>(hs + (size_t)le[li] * h_ld + bb * 32);
-          float a = 0.0f;
-#pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            const float4 hh = hc[c];
-            a = fmaf(w[4 * c], hh.x, a);
-            a = fmaf(w[4 * c + 1], hh.y, a);
-            a = fmaf(w[4 * c + 2], hh.z, a);
-            a = fmaf(w[4 * c + 3], hh.w, a);
-          }
-          acc[j] += a;
+    int good = 1;
+    const unsigned long long t0 = global_ns();
+    unsigned polls = 0;
+    while (ld_acquire(bar) < target) {
+      if ((++polls & 15u) == 0) {
+        if (ld_acquire(bar + 1) != 0u) {
+          good = 0;
+          break;
+        }
+        if (global_ns() - t0 > kBarrierBudgetNs) {
+          record_error(status, MOE_ERR_TIMEOUT);
+          atomicExch(bar + 1, 1u);
+          good = 0;
+          break;
         }
       }
     }
-#pragma unroll
-    for (int j = 0; j < kPer; ++j) {
-      const int li = q + 4 * j;
-      if (li < ne) yslot[le[li]][r] = acc[j];
-    }
+    ok = good;
   }
   __syncthreads();
-  for (int x = threadIdx.x; x < T * kRowsB; x += blockDim.x) {
-    const int t = x / kRowsB, rr = x - t * kRowsB;
-    float acc = 0.0f;
-    for (int s2 = 0; s2 < k; ++s2) acc = fmaf(top_w[t * k + s2], yslot[t * k + s2][rr], acc);
-    const size_t o = (size_t)t * d + row0 + rr;
-    y[o] = __float2half_rn(acc);
-    if (u_next) u_next[o] = __float2half_rn(__half2float(u[o]) + acc);
+  return ok != 0;
+}
+
+// ------------------------------------------------------------ launch plan
+struct LayerPtrs {
+  const float* w_route;
+  const float* bias;
+  const uint8_t* gq;
+  const uint16_t* gs;
+  const uint8_t* uq;
+  const uint16_t* us;
+  const uint8_t* dq;
+  const uint16_t* ds;
+};
+
+// Shared-memory layout (byte offsets) and work split of one launch.
+struct Plan {
+  int RA;        // hidden rows per phase-A item (gate and up each)
+  int RB;        // output rows per phase-B slice
+  int nbuf;      // router-weight buffers (2: next layer prefetched)
+  int nsel_max;  // experts a layer can select: min(N, T*k)
+  int part_cap;  // floats of the phase-A partial-sum buffer
+  uint32_t u, wr0, wr1, z, sel, aw, cnt, start, fill, list, esel, epos, misc;
+  uint32_t aq, as, deq, part, bq, bs, zs;
+  uint32_t total;
+};
+
+struct Params {
+  LayerPtrs layer[kLayersPerLaunch];
+  int n_layers;
+  int T, d, N, k, h, renorm;
+  Plan plan;
+  const __half* u_in;   // layer 0 input
+  __half* u_work;       // inputs of layers 1.. (updated in place)
+  __half* u_out;        // last layer's u_next (nullable)
+  __half* y;            // last layer's y (nullable)
+  int32_t* top_idx;     // [n_layers][T][k] (nullable)
+  float* top_w;         // [T][k] of the last layer (nullable)
+  float* H;             // [N][T][h] fp32 scratch
+  unsigned* bar;        // [0] arrivals, [1] abort
+  int* status;
+};
+
+uint32_t take(uint32_t& off, size_t bytes) {
+  const uint32_t o = off;
+  off += (uint32_t)((bytes + 15) / 16 * 16);
+  return o;
+}
+
+bool make_plan(const moe_shape& s, int sms, Plan* out) {
+  const int T = s.T, d = s.d, N = s.N, k = s.k, h = s.h;
+  const int nb = d / 32, nbh = h / 32;
+  int RB = 4;
+  while (RB < 32 && d / RB > sms) RB *= 2;
+  const int nsel_max = N < T * k ? N : T * k;
+  for (int nbuf = 2; nbuf >= 1; --nbuf) {
+    for (int RA = 8; RA >= 2; RA /= 2) {
+      Plan p{};
+      p.RA = RA;
+      p.RB = RB;
+      p.nbuf = nbuf;
+      p.nsel_max = nsel_max;
+      p.part_cap = 2048 + 4 * RA * T;  // >= 2 (g, v) x units x 2 tokens
+      uint32_t off = 0;
+      p.u = take(off, (size_t)T * (d + 8) * 2);
+      p.wr0 = take(off, (size_t)N * (d + 4) * 4);
+      p.wr1 = nbuf == 2 ? take(off, (size_t)N * (d + 4) * 4) : p.wr0;
+      p.z = take(off, (size_t)T * N * 4);
+      p.sel = take(off, (size_t)T * k * 4);
+      p.aw = take(off, (size_t)T * k * 4);
+      p.cnt = take(off, (size_t)N * 4);
+      p.start = take(off, (size_t)(N + 1) * 4);
+      p.fill = take(off, (size_t)N * 4);
+      p.list = take(off, (size_t)T * k * 4);
+      p.esel = take(off, (size_t)N * 4);
+      p.epos = take(off, (size_t)N * 4);
+      p.misc = take(off, 16);
+      p.aq = take(off, (size_t)2 * RA * (d / 2));
+      p.as = take(off, (size_t)2 * RA * nb * 2);
+      p.deq = take(off, (size_t)2 * RA * (d + 4) * 4);
+      p.part = take(off, (size_t)p.part_cap * 4);
+      p.bq = take(off, (size_t)nsel_max * RB * (h / 2));
+      p.bs = take(off, (size_t)nsel_max * RB * nbh * 2);
+      p.zs = take(off, (size_t)T * k * (RB + 1) * 4);
+      p.total = off;
+      if (off <= kSmemLimit) {
+        *out = p;
+        return true;
+      }
+    }
+  }
+  return false;
+}
+
+// ---------------------------------------------------------------- kernel
+__global__ void __launch_bounds__(kThreads, 1) decode_persistent(const __grid_constant__ Params p) {
+  extern __shared__ __align__(16) char sm[];
+  const Plan& P = p.plan;
+  const int T = p.T, d = p.d, N = p.N, k = p.k, h = p.h, Tk = T * k;
+  const int RA = P.RA, RB = P.RB, nb = d / 32, nbh = h / 32;
+  const int us_ld = d + 8, ws_ld = d + 4, dq_ld = d + 4;
+  const int G = gridDim.x, b = blockIdx.x, tid = threadIdx.x;
+  __half* u_s = reinterpret_cast<__half*>(sm + P.u);
+  float* z = reinterpret_cast<float*>(sm + P.z);
+  int* sel = reinterpret_cast<int*>(sm + P.sel);
+  float* aw = reinterpret_cast<float*>(sm + P.aw);
+  int* cnt = reinterpret_cast<int*>(sm + P.cnt);
+  int* start = reinterpret_cast<int*>(sm + P.start);
+  int* fill = reinterpret_cast<int*>(sm + P.fill);
+  int* list = reinterpret_cast<int*>(sm + P.list);
+  int* esel = reinterpret_cast<int*>(sm + P.esel);
+  int* epos = reinterpret_cast<int*>(sm + P.epos);
+  int* nsel_s = reinterpret_cast<int*>(sm + P.misc);
+  uint8_t* aq = reinterpret_cast<uint8_t*>(sm + P.aq);
+  uint16_t* as = reinterpret_cast<uint16_t*>(sm + P.as);
+  float* deq = reinterpret_cast<float*>(sm + P.deq);
+  float* part = reinterpret_cast<float*>(sm + P.part);
+  uint8_t* bq = reinterpret_cast<uint8_t*>(sm + P.bq);
+  uint16_t* bs = reinterpret_cast<uint16_t*>(sm + P.bs);
+  float* zs = reinterpret_cast<float*>(sm + P.zs);
+  const int slicesA = h / RA, nslices = d / RB;
+  unsigned n_bar = 0;
+
+  stage_rows(sm + P.wr0, ws_ld * 4, reinterpret_cast<const char*>(p.layer[0].w_route),
+             (size_t)d * 4, N, d * 4);
+  for (int l = 0; l < p.n_layers; ++l) {
+    const LayerPtrs& L = p.layer[l];
+    const bool last = l == p.n_layers - 1;
+    const __half* u_cur = l == 0 ? p.u_in : p.u_work;
+    __half* u_next = last ? p.u_out : p.u_work;
+    float* wr_s = reinterpret_cast<float*>(sm + ((l & 1) && P.nbuf == 2 ? P.wr1 : P.wr0));
+    if (l > 0 && P.nbuf == 1)
+      stage_rows(reinterpret_cast<char*>(wr_s), ws_ld * 4,
+                 reinterpret_cast<const char*>(L.w_route), (size_t)d * 4, N, d * 4);
+    stage_rows(reinterpret_cast<char*>(u_s), us_ld * 2, reinterpret_cast<const char*>(u_cur),
+               (size_t)d * 2, T, d * 2);
+    for (int e = tid; e < N; e += blockDim.x) cnt[e] = 0;
+    cp_wait_all();
+    __syncthreads();
+
+    // ---- routing (every CTA), then the pairs grouped by expert
+    route_in_cta(u_s, us_ld, wr_s, ws_ld, T, d, N, k, p.renorm, L.bias, z, sel, aw);
+    if (b == 0) {
+      for (int x = tid; x < Tk; x += blockDim.x) {
+        if (p.top_idx) p.top_idx[(size_t)l * Tk + x] = sel[x];
+        if (last && p.top_w) p.top_w[x] = aw[x];
+      }
+    }
+    // counts by shared atomics, starts and the selected-expert list by one
+    // warp (N <= 64: two experts per lane), then each pair's token is placed
+    // in its expert's list.  The order inside a list does not affect any
+    // result (every (row, token) dot is formed the same way).
+    for (int x = tid; x < Tk; x += blockDim.x) atomicAdd(&cnt[sel[x]], 1);
+    __syncthreads();
+    if (tid < 32) {
+      const int lane = tid;
+      const int c0 = lane < N ? cnt[lane] : 0, c1 = lane + 32 < N ? cnt[lane + 32] : 0;
+      int s0 = c0, s1 = c1;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v0 = __shfl_up_sync(0xffffffffu, s0, o), v1 = __shfl_up_sync(0xffffffffu, s1, o);
+        if (lane >= o) {
+          s0 += v0;
+          s1 += v1;
+        }
+      }
+      const int tot0 = __shfl_sync(0xffffffffu, s0, 31);
+      const unsigned f0 = __ballot_sync(0xffffffffu, c0 > 0), f1 = __ballot_sync(0xffffffffu, c1 > 0);
+      const unsigned lt = (1u << lane) - 1u;
+      if (lane < N) {
+        start[lane] = s0 - c0;
+        fill[lane] = s0 - c0;
+        const int r = __popc(f0 & lt);
+        epos[lane] = c0 ? r : -1;
+        if (c0) esel[r] = lane;
+      }
+      if (lane + 32 < N) {
+        start[lane + 32] = tot0 + s1 - c1;
+        fill[lane + 32] = tot0 + s1 - c1;
+        const int r = __popc(f0) + __popc(f1 & lt);
+        epos[lane + 32] = c1 ? r : -1;
+        if (c1) esel[r] = lane + 32;
+      }
+      if (lane == 0) {
+        start[N] = Tk;
+        *nsel_s = __popc(f0) + __popc(f1);
+      }
+    }
+    __syncthreads();
+    for (int x = tid; x < Tk; x += blockDim.x) list[atomicAdd(&fill[sel[x]], 1)] = x / k;
+    const int nsel = *nsel_s;
+
+    // ---- issue this CTA's first phase-A item and the down rows of its first
+    // phase-B slice together, before the first wait.
+    const int nitems = nsel * slicesA;
+    auto stage_item = [&](int it) {
+      const int e = esel[it / slicesA], sl = it % slicesA;
+      const size_t row = (size_t)e * h + (size_t)sl * RA;
+      stage_bytes(aq, L.gq + row * (d / 2), RA * (d / 2));
+      stage_bytes(aq + RA * (d / 2), L.uq + row * (d / 2), RA * (d / 2));
+      stage_bytes(as, L.gs + row * nb, RA * nb * 2);
+      stage_bytes(as + RA * nb, L.us + row * nb, RA * nb * 2);
+    };
+    auto stage_slice = [&](int sl) {
+      for (int j = 0; j < nsel; ++j) {
+        const size_t row = (size_t)esel[j] * d + (size_t)sl * RB;
+        stage_bytes(bq + (size_t)j * RB * (h / 2), L.dq + row * (h / 2), RB * (h / 2));
+        stage_bytes(bs + (size_t)j * RB * nbh, L.ds + row * nbh, RB * nbh * 2);
+      }
+    };
+    __syncthreads();  // list complete before the item loop reads it
+    if (b < nitems) stage_item(b);
+    if (b < nslices) stage_slice(b);
+
+    // ---- phase A: H[e][t][rows] = SiLU(W_gate u) * (W_up u) for the items
+    for (int it = b; it < nitems; it += G) {
+      const int e = esel[it / slicesA], sl = it % slicesA;
+      const int ne = start[e + 1] - start[e];
+      const int* toks = list + start[e];
+      if (it != b) stage_item(it);
+      cp_wait_all();
+      __syncthreads();
+      for (int x = tid; x < 2 * RA * nb * 8; x += blockDim.x) {  // 8 threads per block
+        const int blk = x >> 3, c = x & 7;
+        const int w = blk / nb, bb = blk - w * nb;
+        *reinterpret_cast<float4*>(deq + (size_t)w * dq_ld + bb * 32 + 4 * c) =
+            dequant_quad(aq + (size_t)w * (d / 2) + bb * 16, as[w * nb + bb], c);
+      }
+      __syncthreads();
+      // unit = (token pair, hidden row r, part of d): one thread forms the
+      // gate and the up dot of row r for two tokens, so each weight and
+      // activation it loads feeds two FMAs.  d is split into nparts so that
+      // about a CTA's worth of units run at once.
+      const int npairs = (ne + 1) >> 1;
+      int nparts = 1;
+      while (nparts < nb && npairs * RA * nparts < kThreads) nparts *= 2;
+      const int units = nparts * RA * npairs;
+      for (int uu = tid; uu < units; uu += blockDim.x) {
+        const int ip = uu % npairs, rest = uu / npairs;
+        const int r = rest % RA, pp = rest / RA;
+        const int i0 = 2 * ip, i1 = i0 + 1 < ne ? i0 + 1 : i0;
+        const int b0 = pp * nb / nparts, b1 = (pp + 1) * nb / nparts;
+        const float4* gw = reinterpret_cast<const float4*>(deq + (size_t)r * dq_ld);
+        const float4* vw = reinterpret_cast<const float4*>(deq + (size_t)(RA + r) * dq_ld);
+        const uint4* x0r = reinterpret_cast<const uint4*>(u_s + (size_t)toks[i0] * us_ld);
+        const uint4* x1r = reinterpret_cast<const uint4*>(u_s + (size_t)toks[i1] * us_ld);
+        float g0a = 0.f, g0b = 0.f, v0a = 0.f, v0b = 0.f, g1a = 0.f, g1b = 0.f, v1a = 0.f,
+              v1b = 0.f;
+        for (int c = b0 * 4; c < b1 * 4; ++c) {  // 8 elements per step
+          const float4 ga = gw[2 * c], gb = gw[2 * c + 1], va = vw[2 * c], vb = vw[2 * c + 1];
+          const uint4 xu = x0r[c], yu = x1r[c];
+          float x[8], y[8];
+          const uint32_t xw[4] = {xu.x, xu.y, xu.z, xu.w}, yw[4] = {yu.x, yu.y, yu.z, yu.w};
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const float2 fx = __half22float2(*reinterpret_cast<const __half2*>(&xw[q]));
+            const float2 fy = __half22float2(*reinterpret_cast<const __half2*>(&yw[q]));
+            x[2 * q] = fx.x;
+            x[2 * q + 1] = fx.y;
+            y[2 * q] = fy.x;
+            y[2 * q + 1] = fy.y;
+          }
+          const float gv[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
+          const float vv[8] = {va.x, va.y, va.z, va.w, vb.x, vb.y, vb.z, vb.w};
+#pragma unroll
+          for (int q = 0; q < 8; q += 2) {
+            g0a = fmaf(gv[q], x[q], g0a);
+            g0b = fmaf(gv[q + 1], x[q + 1], g0b);
+            v0a = fmaf(vv[q], x[q], v0a);
+            v0b = fmaf(vv[q + 1], x[q + 1], v0b);
+            g1a = fmaf(gv[q], y[q], g1a);
+            g1b = fmaf(gv[q + 1], y[q + 1], g1b);
+            v1a = fmaf(vv[q], y[q], v1a);
+            v1b = fmaf(vv[q + 1], y[q + 1], v1b);
+          }
+        }
+        float* pr = part + ((size_t)(r * ne + i0) * nparts + pp) * 2;
+        pr[0] = g0a + g0b;
+        pr[1] = v0a + v0b;
+        if (i1 != i0) {
+          float* pq = part + ((size_t)(r * ne + i1) * nparts + pp) * 2;
+          pq[0] = g1a + g1b;
+          pq[1] = v1a + v1b;
+        }
+      }
+      __syncthreads();
+      for (int v = tid; v < RA * ne; v += blockDim.x) {
+        const int i = v / RA, r = v - i * RA;
+        const float* pr = part + (size_t)(r * ne + i) * nparts * 2;
+        float g = 0.f, vu = 0.f;
+#pragma unroll 4
+        for (int pp = 0; pp < nparts; ++pp) {
+          g += pr[2 * pp];
+          vu += pr[2 * pp + 1];
+        }
+        p.H[((size_t)e * T + toks[i]) * h + (size_t)sl * RA + r] = silu(g) * vu;
+      }
+    }
+    grid_arrive(p.bar);
+    if (P.nbuf == 2 && !last)  // next layer's router rows, while the barrier completes
+      stage_rows(sm + ((l & 1) ? P.wr0 : P.wr1), ws_ld * 4,
+                 reinterpret_cast<const char*>(p.layer[l + 1].w_route), (size_t)d * 4, N, d * 4);
+    if (!grid_wait(p.bar, (unsigned)G * ++n_bar, p.status)) {
+      cp_wait_all();
+      return;
+    }
+
+    // ---- phase B: y = sum_s a_s W_down[e_s] H_s, u_next = fp16(u + y)
+    for (int sl = b; sl < nslices; sl += G) {
+      if (sl != b) stage_slice(sl);
+      cp_wait_all();
+      __syncthreads();
+      // unit = (pair x, row group g, q4 block pp), pp fastest so a pair's
+      // nbh partial dots sit in adjacent lanes; the rows of a slice are split
+      // into rgroups groups when there are few pairs, so more threads work.
+      int rgroups = 1;
+      while (rgroups < RB && Tk * nbh * rgroups * 2 <= (int)blockDim.x) rgroups *= 2;
+      const int rper = RB / rgroups;
+      const int units = Tk * nbh * rgroups;
+      for (int base = 0; base < units; base += blockDim.x) {  // uniform per warp
+        const int uu = base + tid;
+        const bool valid = uu < units;
+        const int pp = uu % nbh, rest = uu / nbh;
+        const int g = rest % rgroups, x = valid ? rest / rgroups : 0;
+        const int e = sel[x];
+        const int j = epos[e];
+        float hc[32];
+        if (valid) {
+          const float4* hp =
+              reinterpret_cast<const float4*>(p.H + ((size_t)e * T + x / k) * h + pp * 32);
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            const float4 v = __ldcg(hp + c);
+            hc[4 * c] = v.x;
+            hc[4 * c + 1] = v.y;
+            hc[4 * c + 2] = v.z;
+            hc[4 * c + 3] = v.w;
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < 32; ++c) hc[c] = 0.f;
+        }
+        for (int r = g * rper; r < (g + 1) * rper; ++r) {
+          float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+          if (valid) {
+            float wv[32];
+            dequant_block(bq + ((size_t)j * RB + r) * (h / 2) + pp * 16,
+                          bs[((size_t)j * RB + r) * nbh + pp], wv);
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+              a0 = fmaf(wv[4 * c], hc[4 * c], a0);
+              a1 = fmaf(wv[4 * c + 1], hc[4 * c + 1], a1);
+              a2 = fmaf(wv[4 * c + 2], hc[4 * c + 2], a2);
+              a3 = fmaf(wv[4 * c + 3], hc[4 * c + 3], a3);
+            }
+          }
+          float zz = (a0 + a1) + (a2 + a3);
+          for (int o = nbh / 2; o >= 1; o >>= 1) zz += __shfl_xor_sync(0xffffffffu, zz, o);
+          if (valid && pp == 0) zs[x * (RB + 1) + r] = zz;
+        }
+      }
+      __syncthreads();
+      for (int v = tid; v < T * RB; v += blockDim.x) {
+        const int t = v / RB, r = v - t * RB;
+        float acc = 0.0f;
+        for (int s2 = 0; s2 < k; ++s2)
+          acc = fmaf(aw[t * k + s2], zs[(t * k + s2) * (RB + 1) + r], acc);
+        const int m = sl * RB + r;
+        const size_t o = (size_t)t * d + m;
+        if (last && p.y) p.y[o] = __float2half_rn(acc);
+        if (u_next) u_next[o] = __float2half_rn(__half2float(u_s[(size_t)t * us_ld + m]) + acc);
+      }
+      __syncthreads();
+    }
+    grid_arrive(p.bar);
+    if (!grid_wait(p.bar, (unsigned)G * ++n_bar, p.status)) {
+      cp_wait_all();
+      return;
+    }
   }
 }
 
+// ------------------------------------------------------------------ host
 struct WsLayout {
   float* H;
   int32_t* idx;
   float* w;
-  __half* ping;
-  __half* pong;
-  __half* y;
+  __half* work;
+  unsigned* bar;
   size_t bytes;
 };
 
@@ -339,65 +724,102 @@ WsLayout carve_decode(const moe_shape& s, void* base) {
   L.H = c.take<float>((size_t)s.N * s.T * s.h);
   L.idx = c.take<int32_t>((size_t)s.T * s.k);
   L.w = c.take<float>((size_t)s.T * s.k);
-  L.ping = c.take<__half>((size_t)s.T * s.d);
-  L.pong = c.take<__half>((size_t)s.T * s.d);
-  L.y = c.take<__half>((size_t)s.T * s.d);
+  L.work = c.take<__half>((size_t)s.T * s.d);
+  L.bar = c.take<unsigned>(4);
   L.bytes = c.used();
   return L;
 }
 
-size_t gateup_smem(const moe_shape& s);
-size_t down_smem(const moe_shape& s);
-bool decode_smem_ok(const moe_shape& s);
+struct DeviceInfo {
+  int sms = 0;
+  bool configured = false;
+};
+
+// SM count of the current device; the kernel's shared-memory limit is raised
+// once per device.
+bool device_info(int* sms) {
+  static DeviceInfo info[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+  DeviceInfo& di = info[dev];
+  if (!di.configured) {
+    if (cudaDeviceGetAttribute(&di.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaFuncSetAttribute(decode_persistent, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)kSmemLimit) != cudaSuccess)
+      return false;
+    di.configured = true;
+  }
+  *sms = di.sms;
+  return true;
+}
 
 bool decode_shape_ok(const moe_shape* s) {
-  return shape_ok(s) && s->T <= kMaxT && s->N <= kMaxN && s->k <= 8 && s->d % 32 == 0 &&
-         s->d % kRowsB == 0 && s->h % kRowsA == 0 && s->h % 32 == 0 && 32 % (s->h / 32) == 0 &&
-         (s->h / 32) <= 32 && decode_smem_ok(*s);
+  if (!shape_ok(s) || s->T > kMaxT || s->N > kMaxN || s->k > 8 || s->d % 32 != 0 ||
+      s->h % 32 != 0 || (s->h / 32) > 32 || 32 % (s->h / 32) != 0)
+    return false;
+  Plan p;
+  return make_plan(*s, 148, &p);
 }
+
+bool aligned4(const void* q) { return (reinterpret_cast<uintptr_t>(q) & 3u) == 0; }
 
 bool layer_ok(const moe_q4_layer* L) {
   return L && L->w_route && L->gate_qs && L->gate_scales && L->up_qs && L->up_scales &&
          L->down_qs && L->down_scales && aligned16(L->gate_qs) && aligned16(L->up_qs) &&
-         aligned16(L->down_qs) && aligned16(L->w_route);
+         aligned16(L->down_qs) && aligned16(L->w_route) && aligned4(L->gate_scales) &&
+         aligned4(L->up_scales) && aligned4(L->down_scales) && aligned4(L->bias);
 }
 
-size_t gateup_smem(const moe_shape& s) {
-  return (size_t)s.T * (s.d + 8) * 2 + (size_t)s.N * (s.d + 4) * 4 + 2 * kRowsA * (s.d / 2) +
-         2 * kRowsA * (s.d / 32) * 2 + 16;
-}
-size_t down_smem(const moe_shape& s) {
-  return (size_t)s.T * s.k * (s.h + 4) * 4 + (size_t)s.N * kRowsB * (s.h / 2) +
-         (size_t)s.N * kRowsB * (s.h / 32) * 2 + 16;
+LayerPtrs layer_ptrs(const moe_q4_layer& L) {
+  return LayerPtrs{L.w_route, L.bias, L.gate_qs, L.gate_scales,
+                   L.up_qs,   L.up_scales, L.down_qs, L.down_scales};
 }
 
-bool decode_smem_ok(const moe_shape& s) {
-  return gateup_smem(s) <= 160 * 1024 && down_smem(s) <= 160 * 1024;
-}
-
-int launch_decode_layer(const moe_shape& s, const moe_q4_layer& L, const __half* u, __half* y,
-                        __half* u_next, int32_t* idx, float* w, float* H, cudaStream_t st) {
-  if (s.T == 0) return MOE_OK;
-  static bool configured[64] = {false};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !configured[dev]) {
-    if (cudaFuncSetAttribute(decode_gateup, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             160 * 1024) != cudaSuccess ||
-        cudaFuncSetAttribute(decode_down, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             160 * 1024) != cudaSuccess)
-      return MOE_ERR_CUDA;
-    configured[dev] = true;
-  }
-  MOE_PREFER_SHARED((decode_gateup));
-  launch_pdl(decode_gateup, dim3(s.N * (s.h / kRowsA)), dim3(128), gateup_smem(s), st, 
-      u, s.T, s.d, s.N, s.k, s.h, s.renorm, L.w_route, L.bias, L.gate_qs, L.gate_scales, L.up_qs,
-      L.up_scales, H, idx, w);
-  MOE_PREFER_SHARED((decode_down));
-  launch_pdl(decode_down, dim3(s.d / kRowsB), dim3(128), down_smem(s), st, u, s.T, s.d, s.N, s.k, s.h, idx, w,
-                                                       L.down_qs, L.down_scales, H, y, u_next,
-                                                       status_word());
-  return launch_status();
+// One cooperative launch over layers [0, n) of `layers`.
+int launch_decode(const moe_shape& s, const moe_q4_layer* layers, int n, const __half* u_in,
+                  __half* u_out, __half* y, int32_t* top_idx, float* top_w, const WsLayout& W,
+                  cudaStream_t st) {
+  int sms = 0;
+  if (!device_info(&sms)) return MOE_ERR_CUDA;
+  Params p{};
+  if (!make_plan(s, sms, &p.plan)) return MOE_ERR_UNSUPPORTED;
+  int occ = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, decode_persistent, kThreads,
+                                                    p.plan.total) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (occ < 1) return MOE_ERR_UNSUPPORTED;
+  const int items = p.plan.nsel_max * (s.h / p.plan.RA), slices = s.d / p.plan.RB;
+  int grid = items > slices ? items : slices;
+  if (grid > sms) grid = sms;
+  for (int l = 0; l < n; ++l) p.layer[l] = layer_ptrs(layers[l]);
+  p.n_layers = n;
+  p.T = s.T;
+  p.d = s.d;
+  p.N = s.N;
+  p.k = s.k;
+  p.h = s.h;
+  p.renorm = s.renorm;
+  p.u_in = u_in;
+  p.u_work = W.work;
+  p.u_out = u_out;
+  p.y = y;
+  p.top_idx = top_idx;
+  p.top_w = top_w;
+  p.H = W.H;
+  p.bar = W.bar;
+  p.status = status_word();
+  if (cudaMemsetAsync(W.bar, 0, 4 * sizeof(unsigned), st) != cudaSuccess) return MOE_ERR_CUDA;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = p.plan.total;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, decode_persistent, p) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
 }  // namespace
@@ -418,10 +840,10 @@ extern "C" int moe_decode_layer(const moe_shape* shape, const moe_q4_layer* laye
   if (!aligned16(u) || !aligned16(y) || !aligned16(u_next)) return MOE_ERR_INVALID_ARG;
   WsLayout W = carve_decode(*shape, ws);
   if (!ws || ws_bytes < W.bytes) return MOE_ERR_WORKSPACE;
-  return launch_decode_layer(*shape, *layer, reinterpret_cast<const __half*>(u),
-                             reinterpret_cast<__half*>(y), reinterpret_cast<__half*>(u_next),
-                             top_idx ? top_idx : W.idx, top_w ? top_w : W.w, W.H,
-                             as_stream(stream));
+  if (shape->T == 0) return MOE_OK;
+  return launch_decode(*shape, layer, 1, reinterpret_cast<const __half*>(u),
+                       reinterpret_cast<__half*>(u_next), reinterpret_cast<__half*>(y),
+                       top_idx ? top_idx : W.idx, top_w ? top_w : W.w, W, as_stream(stream));
 }
 
 extern "C" int moe_decode_step(const moe_shape* shape, int32_t n_layers,
@@ -435,16 +857,18 @@ extern "C" int moe_decode_step(const moe_shape* shape, int32_t n_layers,
   if (!aligned16(u0) || !aligned16(u_out)) return MOE_ERR_INVALID_ARG;
   WsLayout W = carve_decode(*shape, ws);
   if (!ws || ws_bytes < W.bytes) return MOE_ERR_WORKSPACE;
+  if (shape->T == 0) return MOE_OK;
   const moe_shape& s = *shape;
   cudaStream_t st = as_stream(stream);
-  const __half* cur = reinterpret_cast<const __half*>(u0);
-  for (int l = 0; l < n_layers; ++l) {
-    __half* next = l == n_layers - 1 ? reinterpret_cast<__half*>(u_out)
-                                     : ((l & 1) ? W.pong : W.ping);
-    int32_t* idx = top_idx_all ? top_idx_all + (size_t)l * s.T * s.k : W.idx;
-    const int rc = launch_decode_layer(s, layers[l], cur, W.y, next, idx, W.w, W.H, st);
+  const size_t Tk = (size_t)s.T * s.k;
+  for (int l0 = 0; l0 < n_layers; l0 += kLayersPerLaunch) {
+    const int n = n_layers - l0 < kLayersPerLaunch ? n_layers - l0 : kLayersPerLaunch;
+    const bool last_chunk = l0 + n == n_layers;
+    const __half* in = l0 == 0 ? reinterpret_cast<const __half*>(u0) : W.work;
+    __half* out = last_chunk ? reinterpret_cast<__half*>(u_out) : W.work;
+    const int rc = launch_decode(s, layers + l0, n, in, out, nullptr,
+                                 top_idx_all ? top_idx_all + l0 * Tk : nullptr, nullptr, W, st);
     if (rc != MOE_OK) return rc;
-    cur = next;
   }
   return MOE_OK;
 }

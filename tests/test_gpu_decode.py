@@ -140,3 +140,64 @@ def test_decode_reads_only_selected_experts():
     moe.moe_decode_layer(s, layer, _f16(u), y2)
     torch.cuda.synchronize()
     assert torch.equal(y1, y2)
+
+
+@pytest.mark.parametrize("T,d,N,k,h", [
+    (32, 512, 64, 8, 128),   # 64 experts top-8: several phase-A items per CTA
+    (32, 1024, 8, 2, 256),   # 8 output rows per phase-B slice, h/32 = 8 parts
+    (5, 64, 4, 2, 32),       # tiny: one q4 block per hidden row, ragged T
+    (3, 96, 4, 3, 64),       # d/32 = 3 blocks: uneven phase-A parts
+])
+def test_decode_layer_other_shapes(T, d, N, k, h):
+    import dataclasses
+    wl = dataclasses.replace(W.decode(T=T, n_layers=1), d=d, N=N, k=k, h=h)
+    L = Layer(wl, 0)
+    u = _u0(wl)
+    s = moe.shape(T, d, N, k, h, 1, 0)
+    assert moe.moe_decode_workspace_bytes(s) > 0
+    y = torch.empty((T, d), dtype=torch.float16, device="cuda")
+    un = torch.empty_like(y)
+    idx = torch.empty((T, k), dtype=torch.int32, device="cuda")
+    moe.moe_decode_layer(s, L.abi, _f16(u), y, un, idx)
+    torch.cuda.synchronize()
+    oidx, otw, oy, oun = O.decode_layer(u, L.w_route_h, L.mats, k)
+    assert np.array_equal(idx.cpu().numpy(), oidx)
+    assert rel_err(y.float().cpu().numpy(), oy) < TOL_Q4
+
+
+def test_decode_step_chunks_and_graph_replay():
+    """40 layers (more than one launch carries) at T=1: the chained call equals
+    the layer calls made one by one, and a CUDA-graph replay of the chained
+    call reproduces it bit for bit."""
+    wl = W.decode(T=1, n_layers=40)
+    layers = [Layer(wl, l) for l in range(wl.n_layers)]
+    s = moe.shape(wl.T, wl.d, wl.N, wl.k, wl.h, 1, 0)
+    u0 = _f16(_u0(wl))
+    out = torch.empty_like(u0)
+    idx_all = torch.empty((wl.n_layers, wl.T, wl.k), dtype=torch.int32, device="cuda")
+    abis = [L.abi for L in layers]
+    moe.moe_decode_step(s, abis, u0, out, idx_all)
+    cur = u0
+    for l, L in enumerate(layers):
+        y = torch.empty_like(cur)
+        nxt = torch.empty_like(cur)
+        idx = torch.empty((wl.T, wl.k), dtype=torch.int32, device="cuda")
+        moe.moe_decode_layer(s, L.abi, cur, y, nxt, idx)
+        assert torch.equal(idx, idx_all[l]), f"layer {l}"
+        cur = nxt
+    torch.cuda.synchronize()
+    assert np.array_equal(_codes(cur), _codes(out))
+    ws = torch.empty(moe.moe_decode_workspace_bytes(s), dtype=torch.uint8, device="cuda")
+    out2 = torch.zeros_like(out)
+    g = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        with torch.cuda.graph(g, stream=side):
+            moe.moe_decode_step(s, abis, u0, out2, ws=ws)
+    torch.cuda.current_stream().wait_stream(side)
+    for _ in range(2):
+        out2.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        assert np.array_equal(_codes(out2), _codes(out))
