@@ -68,6 +68,25 @@ __device__ __forceinline__ void load8(const __half* p, float* o) {
 
 __device__ __forceinline__ float silu(float g) { return g / (1.0f + expf(-g)); }
 
+// Gated activations of the bf16 tensor-core epilogues, whose result is rounded
+// to bf16 (8 significant bits): the hardware exp2/reciprocal/tanh
+// approximations (about 2^-21, 2^-22 and 2^-11 relative error) stay well
+// below that rounding.  ACT is a compile-time constant so a SwiGLU kernel
+// carries no trace of the capped variant.
+__device__ __forceinline__ float tanh_approx(float x) {
+  float y;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+template <int ACT>
+__device__ __forceinline__ float gated_act(float g, float v, float bg, float bu) {
+  if (ACT == MOE_ACT_SITU_GLU) {  // beta * tanh(x / beta) soft caps
+    g = bg * tanh_approx(__fdividef(g, bg));
+    v = bu * tanh_approx(__fdividef(v, bu));
+  }
+  return __fdividef(g, 1.0f + __expf(-g)) * v;
+}
+
 // ------------------------------------------- programmatic dependent launch
 // Every kernel is launched with programmatic stream serialization: its CTAs
 // may be scheduled while the previous kernel on the stream drains, and they

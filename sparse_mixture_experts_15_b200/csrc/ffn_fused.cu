@@ -37,7 +37,6 @@ struct FusedParams {
   CUtensorMap map_d;  // W_down [G*width][h], box 64 x 128
   const int32_t* offsets;
   int G, width, h;
-  int act_kind;
   float beta_g, beta_u;
   float* y_rows;  // [R][width]
   int* status;
@@ -57,14 +56,6 @@ struct FLayout {
   }
 };
 
-__device__ __forceinline__ float f_act(float g, float v, int kind, float bg, float bu) {
-  if (kind == MOE_ACT_SITU_GLU) {
-    g = bg * tanhf(g / bg);
-    v = bu * tanhf(v / bu);
-  }
-  return silu(g) * v;
-}
-
 __device__ __forceinline__ bool all_epi_ok(bool ok) {
   uint32_t r;
   asm volatile(
@@ -78,6 +69,7 @@ __device__ __forceinline__ bool all_epi_ok(bool ok) {
   return r != 0;
 }
 
+template <int ACT>
 __global__ void __launch_bounds__(fThreads, 1) tc_fused_ffn(const __grid_constant__ FusedParams p) {
   using L = FLayout;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -323,12 +315,12 @@ __global__ void __launch_bounds__(fThreads, 1) tc_fused_ffn(const __grid_constan
           uint32_t packed[8];
 #pragma unroll
           for (int i = 0; i < 16; i += 2) {
-            const float h0 = f_act(epi[(q * 16 + i) * fEpiLd + lane],
-                                   epi[(64 + q * 16 + i) * fEpiLd + lane], p.act_kind, p.beta_g,
-                                   p.beta_u);
-            const float h1 = f_act(epi[(q * 16 + i + 1) * fEpiLd + lane],
-                                   epi[(64 + q * 16 + i + 1) * fEpiLd + lane], p.act_kind,
-                                   p.beta_g, p.beta_u);
+            const float h0 = gated_act<ACT>(epi[(q * 16 + i) * fEpiLd + lane],
+                                            epi[(64 + q * 16 + i) * fEpiLd + lane], p.beta_g,
+                                            p.beta_u);
+            const float h1 = gated_act<ACT>(epi[(q * 16 + i + 1) * fEpiLd + lane],
+                                            epi[(64 + q * 16 + i + 1) * fEpiLd + lane], p.beta_g,
+                                            p.beta_u);
             __nv_bfloat162 hv = __floats2bfloat162_rn(h0, h1);
             packed[i >> 1] = *reinterpret_cast<uint32_t*>(&hv);
           }
@@ -422,7 +414,6 @@ int launch_ffn_fused(int G, int64_t R, int width, int h, const __nv_bfloat16* x_
   p.G = G;
   p.width = width;
   p.h = h;
-  p.act_kind = act.kind;
   p.beta_g = act.beta_gate;
   p.beta_u = act.beta_up;
   p.y_rows = y_rows;
@@ -431,7 +422,11 @@ int launch_ffn_fused(int G, int64_t R, int width, int h, const __nv_bfloat16* x_
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !configured[dev]) {
-    if (cudaFuncSetAttribute(tc_fused_ffn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(tc_fused_ffn<MOE_ACT_SWIGLU>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)FLayout::bytes(1024)) != cudaSuccess ||
+        cudaFuncSetAttribute(tc_fused_ffn<MOE_ACT_SITU_GLU>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)FLayout::bytes(1024)) != cudaSuccess)
       return MOE_ERR_CUDA;
     configured[dev] = true;
@@ -440,8 +435,15 @@ int launch_ffn_fused(int G, int64_t R, int width, int h, const __nv_bfloat16* x_
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   int64_t grid = (R + fBN - 1) / fBN + G;  // upper bound on the tiles
   if (grid > sms) grid = sms;
-  MOE_PREFER_SHARED((tc_fused_ffn));
-  launch_pdl(tc_fused_ffn, dim3((unsigned)grid), dim3(fThreads), FLayout::bytes(G), st, p);
+  if (act.kind == MOE_ACT_SITU_GLU) {
+    MOE_PREFER_SHARED((tc_fused_ffn<MOE_ACT_SITU_GLU>));
+    launch_pdl(tc_fused_ffn<MOE_ACT_SITU_GLU>, dim3((unsigned)grid), dim3(fThreads),
+               FLayout::bytes(G), st, p);
+  } else {
+    MOE_PREFER_SHARED((tc_fused_ffn<MOE_ACT_SWIGLU>));
+    launch_pdl(tc_fused_ffn<MOE_ACT_SWIGLU>, dim3((unsigned)grid), dim3(fThreads),
+               FLayout::bytes(G), st, p);
+  }
   return launch_status();
 }
 

@@ -63,14 +63,6 @@ struct TcParams {
   int* status;
 };
 
-__device__ __forceinline__ float epi_act(float g, float v, int kind, float bg, float bu) {
-  if (kind == MOE_ACT_SITU_GLU) {
-    g = bg * tanhf(g / bg);
-    v = bu * tanhf(v / bu);
-  }
-  return silu(g) * v;
-}
-
 __device__ __forceinline__ void named_sync_epi() {
   asm volatile("bar.sync 1, 128;" ::: "memory");
 }
@@ -91,7 +83,7 @@ struct Layout {
   }
 };
 
-template <int BN, int S>
+template <int BN, int S, int ACT>
 __global__ void __launch_bounds__(kThreads, 1) tc_grouped_gemm(const __grid_constant__ TcParams p) {
   using L = Layout<BN, S>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -338,12 +330,12 @@ __global__ void __launch_bounds__(kThreads, 1) tc_grouped_gemm(const __grid_cons
             uint32_t packed[8];
 #pragma unroll
             for (int i = 0; i < 16; i += 2) {
-              const float h0 = epi_act(epi[(q * 16 + i) * kEpiLd + lane],
-                                       epi[(64 + q * 16 + i) * kEpiLd + lane], p.act_kind,
-                                       p.beta_g, p.beta_u);
-              const float h1 = epi_act(epi[(q * 16 + i + 1) * kEpiLd + lane],
-                                       epi[(64 + q * 16 + i + 1) * kEpiLd + lane], p.act_kind,
-                                       p.beta_g, p.beta_u);
+              const float h0 = gated_act<ACT>(epi[(q * 16 + i) * kEpiLd + lane],
+                                              epi[(64 + q * 16 + i) * kEpiLd + lane], p.beta_g,
+                                              p.beta_u);
+              const float h1 = gated_act<ACT>(epi[(q * 16 + i + 1) * kEpiLd + lane],
+                                              epi[(64 + q * 16 + i + 1) * kEpiLd + lane],
+                                              p.beta_g, p.beta_u);
               __nv_bfloat162 hv = __floats2bfloat162_rn(h0, h1);
               packed[i >> 1] = *reinterpret_cast<uint32_t*>(&hv);
             }
@@ -430,14 +422,14 @@ int sm_count() {
   return cached[dev];
 }
 
-template <int BN, int S>
+template <int BN, int S, int ACT>
 int launch_tc(const TcParams& p, int64_t tiles_upper, cudaStream_t st) {
   const size_t smem = Layout<BN, S>::bytes(p.G);
   static bool configured[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !configured[dev]) {
-    if (cudaFuncSetAttribute(tc_grouped_gemm<BN, S>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(tc_grouped_gemm<BN, S, ACT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)Layout<BN, S>::bytes(1024)) != cudaSuccess)
       return MOE_ERR_CUDA;
     configured[dev] = true;
@@ -445,8 +437,8 @@ int launch_tc(const TcParams& p, int64_t tiles_upper, cudaStream_t st) {
   int64_t grid = sm_count();
   if (tiles_upper < grid) grid = tiles_upper;
   if (grid <= 0) return MOE_OK;
-  MOE_PREFER_SHARED((tc_grouped_gemm<BN, S>));
-  launch_pdl(tc_grouped_gemm<BN, S>, dim3((unsigned)grid), dim3(kThreads), smem, st, p);
+  MOE_PREFER_SHARED((tc_grouped_gemm<BN, S, ACT>));
+  launch_pdl(tc_grouped_gemm<BN, S, ACT>, dim3((unsigned)grid), dim3(kThreads), smem, st, p);
   return launch_status();
 }
 
@@ -461,8 +453,12 @@ int pick_bn(int m_tiles, int64_t max_rows, int G) {
 
 int launch_tc_bn(const TcParams& p, int64_t max_rows, int bn, cudaStream_t st) {
   const int64_t upper = (int64_t)p.m_tiles * ((max_rows + bn - 1) / bn + p.G);
-  if (bn == 256) return launch_tc<256, 4>(p, upper, st);
-  return launch_tc<128, 6>(p, upper, st);
+  const bool situ = p.mode == MODE_GATEUP && p.act_kind == MOE_ACT_SITU_GLU;
+  if (bn == 256)
+    return situ ? launch_tc<256, 4, MOE_ACT_SITU_GLU>(p, upper, st)
+                : launch_tc<256, 4, MOE_ACT_SWIGLU>(p, upper, st);
+  return situ ? launch_tc<128, 6, MOE_ACT_SITU_GLU>(p, upper, st)
+              : launch_tc<128, 6, MOE_ACT_SWIGLU>(p, upper, st);
 }
 
 }  // namespace
