@@ -202,6 +202,15 @@ bool dispatch_small_ok(const moe_shape& s);
 int launch_dispatch_small(const moe_shape& s, const int32_t* top_idx, const int32_t* hist,
                           int32_t* counts, int32_t* offsets, int32_t* perm_tok, int32_t* row_of,
                           int32_t* overflow, int32_t* totals, cudaStream_t st);
+// Router + permutation + gather in one cooperative launch (route_dispatch.cu),
+// for few experts when a CTA's token rows and the router rows fit on chip.
+bool route_dispatch_ok(const moe_shape& s, int32_t dtype);
+size_t route_dispatch_ws_bytes(const moe_shape& s);
+int launch_route_dispatch(const moe_shape& s, const void* u, int32_t dtype, const float* w_route,
+                          const float* bias, int32_t* top_idx, float* top_w, float* probs,
+                          float* logits, int32_t* counts, int32_t* offsets, int32_t* perm_tok,
+                          int32_t* row_of, int32_t* overflow, int32_t* totals, void* x_rows,
+                          void* ws, cudaStream_t st);
 size_t aux_stats_ws_bytes(int32_t N);
 int launch_aux_stats(int32_t T, int32_t N, int32_t k, const float* probs, const int32_t* top_idx,
                      float* f, float* P, float* n_sum_fP, int32_t* loads, void* ws,

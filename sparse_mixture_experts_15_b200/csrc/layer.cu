@@ -26,6 +26,7 @@ struct LayerBufs {
   void* ffn_ws;
   float* y_rows;
   void* stats_ws;
+  void* rd_ws;
   size_t bytes;
 };
 
@@ -59,6 +60,7 @@ LayerBufs carve_layer(const moe_shape& s, int32_t act_dtype, void* base) {
   b.ffn_ws = c.take<char>(ffn_ws_bytes(s, s.d, act_dtype));
   b.y_rows = c.take<float>(Tk * s.d);
   b.stats_ws = c.take<char>(aux_stats_ws_bytes(s.N));
+  b.rd_ws = c.take<char>(route_dispatch_ws_bytes(s));
   b.bytes = c.used();
   return b;
 }
@@ -147,27 +149,40 @@ extern "C" int moe_layer_fwd(const moe_shape* shape, const moe_layer_weights* w,
   int32_t* totals = o.totals ? o.totals : b.totals;
   cudaStream_t st = as_stream(stream);
 
-  // Few experts: the router also counts each block's dispatches, and one
-  // kernel then scans and scatters (2 launches instead of 4 before the gather).
-  const bool small = dispatch_small_ok(s);
-  int32_t* hist = small ? static_cast<int32_t*>(b.permute_ws) : nullptr;
-  int rc = launch_route(s, u, act_dtype, w->w_route, w->bias, top_idx, top_w, probs, b.logits,
-                        nullptr, st, hist);
-  if (rc != MOE_OK) return rc;
-  if (want_stats) {
-    rc = launch_aux_stats(s.T, s.N, s.k, probs, top_idx, o.f, o.P, o.n_sum_fP, nullptr, b.stats_ws,
-                          st);
+  int rc;
+  if (route_dispatch_ok(s, act_dtype)) {
+    // Few experts, token rows fit on chip: routing, permutation and gather in
+    // one cooperative launch.
+    rc = launch_route_dispatch(s, u, act_dtype, w->w_route, w->bias, top_idx, top_w, probs,
+                               nullptr, counts, offsets, perm_tok, row_of, overflow, totals,
+                               b.x_rows, b.rd_ws, st);
+    if (rc == MOE_OK && want_stats)
+      rc = launch_aux_stats(s.T, s.N, s.k, probs, top_idx, o.f, o.P, o.n_sum_fP, nullptr,
+                            b.stats_ws, st);
+    if (rc != MOE_OK) return rc;
+  } else {
+    // Few experts: the router also counts each block's dispatches, and one
+    // kernel then scans and scatters (2 launches instead of 4 before the gather).
+    const bool small = dispatch_small_ok(s);
+    int32_t* hist = small ? static_cast<int32_t*>(b.permute_ws) : nullptr;
+    rc = launch_route(s, u, act_dtype, w->w_route, w->bias, top_idx, top_w, probs, b.logits,
+                      nullptr, st, hist);
+    if (rc != MOE_OK) return rc;
+    if (want_stats) {
+      rc = launch_aux_stats(s.T, s.N, s.k, probs, top_idx, o.f, o.P, o.n_sum_fP, nullptr,
+                            b.stats_ws, st);
+      if (rc != MOE_OK) return rc;
+    }
+    if (small) {
+      rc = launch_dispatch_small(s, top_idx, hist, counts, offsets, perm_tok, row_of, overflow,
+                                 totals, st);
+    } else {
+      rc = launch_permute(s, top_idx, counts, offsets, perm_tok, row_of, overflow, totals,
+                          b.permute_ws, st);
+    }
+    if (rc == MOE_OK) rc = launch_gather(s, s.d, u, act_dtype, perm_tok, offsets, b.x_rows, st);
     if (rc != MOE_OK) return rc;
   }
-  if (small) {
-    rc = launch_dispatch_small(s, top_idx, hist, counts, offsets, perm_tok, row_of, overflow,
-                               totals, st);
-  } else {
-    rc = launch_permute(s, top_idx, counts, offsets, perm_tok, row_of, overflow, totals,
-                        b.permute_ws, st);
-  }
-  if (rc == MOE_OK) rc = launch_gather(s, s.d, u, act_dtype, perm_tok, offsets, b.x_rows, st);
-  if (rc != MOE_OK) return rc;
   rc = run_ffn(s, s.d, b.x_rows, act_dtype, offsets, w->w_gate, w->w_up, w->w_down, w->act,
                b.y_rows, b.ffn_ws, st);
   if (rc != MOE_OK) return rc;

@@ -188,3 +188,21 @@ def test_layer_mixtral_full_size_sampled():
                        round_h=1)
     got = y[torch.from_numpy(tokens).long().cuda()].float().cpu().numpy()
     assert rel_err(got, ref) < TOL_BF16
+
+
+@pytest.mark.parametrize("case", ["capacity_zipf", "n16_top4"])
+def test_layer_fused_routing_paths(case):
+    """The one-launch routing + permutation + gather of the layer path (few
+    experts, token rows on chip): capacity drops with skewed loads, and the
+    16-expert variant, bit-exact routing and permutation on every token."""
+    import dataclasses
+    if case == "capacity_zipf":
+        wl = dataclasses.replace(W.small(T=1024), capacity_factor=1.0, zipf_s=1.2)
+    else:
+        wl = dataclasses.replace(W.small(T=600), N=16, k=4)
+    y, outs = _layer_gpu(wl)
+    ref, idx, tw, perm = _layer_oracle(wl, np.arange(wl.T, dtype=np.int32))
+    _check_routing(outs, idx, tw, perm)
+    if case == "capacity_zipf":
+        assert int(perm["totals"][1]) > 0, "the skewed loads should overflow the capacity"
+    assert rel_err(y.float().cpu().numpy(), ref) < TOL_BF16
