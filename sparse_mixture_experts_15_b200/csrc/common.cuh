@@ -234,7 +234,7 @@ int launch_ffn_tc(const moe_shape& s, int32_t width, const __nv_bfloat16* x_rows
                   cudaStream_t st);
 
 // Fused single-launch expert FFN for small hidden widths (ffn_fused.cu).
-bool ffn_fused_ok(int width, int h);
+bool ffn_fused_ok(int width, int h, int G);
 int launch_ffn_fused(int G, int64_t R, int width, int h, const __nv_bfloat16* x_rows,
                      const int32_t* offsets, const __nv_bfloat16* w_gate,
                      const __nv_bfloat16* w_up, const __nv_bfloat16* w_down, const moe_act& act,

@@ -26,7 +26,7 @@
 namespace moe {
 namespace {
 
-constexpr int fBM = 128, fBK = 64, fBN = 64, fS = 6, fThreads = 192, fEpiLd = 33;
+constexpr int fBM = 128, fBK = 64, fBN = 64, fS = 7, fThreads = 192, fEpiLd = 33;
 constexpr int fHMax = 256;
 constexpr long long fWaitBudget = 4000000000LL;
 
@@ -394,9 +394,11 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, ui
 
 }  // namespace
 
-bool ffn_fused_ok(int width, int h) {
+constexpr size_t fSmemLimit = 227 * 1024;
+
+bool ffn_fused_ok(int width, int h, int G) {
   return h % 64 == 0 && h <= fHMax && width % fBM == 0 && width >= fBM &&
-         (h / 64 + width / fBM) * fBN <= 512;
+         (h / 64 + width / fBM) * fBN <= 512 && FLayout::bytes(G) <= fSmemLimit;
 }
 
 int launch_ffn_fused(int G, int64_t R, int width, int h, const __nv_bfloat16* x_rows,
@@ -424,10 +426,10 @@ int launch_ffn_fused(int G, int64_t R, int width, int h, const __nv_bfloat16* x_
   if (dev >= 0 && dev < 64 && !configured[dev]) {
     if (cudaFuncSetAttribute(tc_fused_ffn<MOE_ACT_SWIGLU>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)FLayout::bytes(1024)) != cudaSuccess ||
+                             (int)fSmemLimit) != cudaSuccess ||
         cudaFuncSetAttribute(tc_fused_ffn<MOE_ACT_SITU_GLU>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)FLayout::bytes(1024)) != cudaSuccess)
+                             (int)fSmemLimit) != cudaSuccess)
       return MOE_ERR_CUDA;
     configured[dev] = true;
   }

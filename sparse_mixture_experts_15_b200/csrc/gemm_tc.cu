@@ -473,7 +473,7 @@ int launch_ffn_tc(const moe_shape& s, int32_t width, const __nv_bfloat16* x_rows
                   cudaStream_t st) {
   const int64_t R = (int64_t)s.T * s.k;
   if (R == 0) return MOE_OK;
-  if (ffn_fused_ok(width, s.h))  // small h: both GEMMs in one launch, H stays on chip
+  if (ffn_fused_ok(width, s.h, s.N))  // small h: both GEMMs in one launch, H stays on chip
     return launch_ffn_fused(s.N, R, width, s.h, x_rows, offsets, w_gate, w_up, w_down, act,
                             y_rows, st);
   __nv_bfloat16* H = static_cast<__nv_bfloat16*>(ws);

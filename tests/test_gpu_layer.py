@@ -203,6 +203,14 @@ def test_layer_fused_routing_paths(case):
     y, outs = _layer_gpu(wl)
     ref, idx, tw, perm = _layer_oracle(wl, np.arange(wl.T, dtype=np.int32))
     _check_routing(outs, idx, tw, perm)
+    got = y.float().cpu().numpy()
     if case == "capacity_zipf":
         assert int(perm["totals"][1]) > 0, "the skewed loads should overflow the capacity"
-    assert rel_err(y.float().cpu().numpy(), ref) < TOL_BF16
+        # Hundreds of tokens lose both slots: their rows are exactly zero, and
+        # the tolerance applies to the rows the layer computes (with the zero
+        # rows in rms(y), max|y|/rms(y) ~ 11 and one bf16 ulp of the largest
+        # output alone would exceed it).
+        gone = (perm["row_of"] < 0).all(1)
+        assert gone.sum() > 0 and np.all(got[gone] == 0.0)
+        got, ref = got[~gone], ref[~gone]
+    assert rel_err(got, ref) < TOL_BF16
