@@ -696,6 +696,7 @@ bool device_info(int* sms) {
         cudaFuncSetAttribute(decode_persistent, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)kSmemLimit) != cudaSuccess)
       return false;
+    MOE_PREFER_SHARED((decode_persistent));
     di.configured = true;
   }
   *sms = di.sms;

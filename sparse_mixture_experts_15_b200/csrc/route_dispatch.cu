@@ -324,6 +324,10 @@ int launch_route_dispatch(const moe_shape& s, const void* u, int32_t dtype, cons
   if (!make_rd_plan(s, dtype, sms, &p.plan)) return MOE_ERR_UNSUPPORTED;
   if (dev >= 0 && dev < 64 && !configured[dev]) {
     const int lim = (int)kRDSmemLimit;
+    MOE_PREFER_SHARED((route_dispatch<8, float>));
+    MOE_PREFER_SHARED((route_dispatch<16, float>));
+    MOE_PREFER_SHARED((route_dispatch<8, __nv_bfloat16>));
+    MOE_PREFER_SHARED((route_dispatch<16, __nv_bfloat16>));
     if (cudaFuncSetAttribute(route_dispatch<8, float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              lim) != cudaSuccess ||
         cudaFuncSetAttribute(route_dispatch<16, float>,

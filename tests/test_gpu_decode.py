@@ -201,3 +201,15 @@ def test_decode_step_chunks_and_graph_replay():
         g.replay()
         torch.cuda.synchronize()
         assert np.array_equal(_codes(out2), _codes(out))
+
+
+def test_decode_empty_batch():
+    """T = 0: both decode entry points succeed and launch nothing."""
+    wl = W.decode(T=1, n_layers=2)
+    layers = [Layer(wl, l) for l in range(2)]
+    s = moe.shape(0, wl.d, wl.N, wl.k, wl.h, 1, 0)
+    u = torch.empty((0, wl.d), dtype=torch.float16, device="cuda")
+    y = torch.empty_like(u)
+    moe.moe_decode_layer(s, layers[0].abi, u, y)
+    moe.moe_decode_step(s, [L.abi for L in layers], u, y)
+    torch.cuda.synchronize()

@@ -214,3 +214,40 @@ def test_layer_fused_routing_paths(case):
         assert gone.sum() > 0 and np.all(got[gone] == 0.0)
         got, ref = got[~gone], ref[~gone]
     assert rel_err(got, ref) < TOL_BF16
+
+
+@pytest.mark.parametrize("case", ["top1_no_renorm", "n17_top3", "n32_top4"])
+def test_layer_edge_routing_configurations(case):
+    """Top-1 with a = p (the Switch multiplier of §3.2), an odd expert count
+    above 16 and a 32-expert top-4 layer (the general router, permutation and
+    gather kernels): routing bit-exact, outputs within the bf16 bound."""
+    import dataclasses
+    if case == "top1_no_renorm":
+        wl = dataclasses.replace(W.small(T=300), k=1, renorm=0)
+    elif case == "n17_top3":
+        wl = dataclasses.replace(W.small(T=333), N=17, k=3)
+    else:
+        wl = dataclasses.replace(W.small(T=500), N=32, k=4)
+    y, outs = _layer_gpu(wl)
+    ref, idx, tw, perm = _layer_oracle(wl, np.arange(wl.T, dtype=np.int32))
+    _check_routing(outs, idx, tw, perm)
+    if case == "top1_no_renorm":
+        assert np.all(outs["top_w"] < 1.0)  # p of the top expert, not renormalised to 1
+    assert rel_err(y.float().cpu().numpy(), ref) < TOL_BF16
+
+
+def test_layer_empty_batch():
+    """T = 0: the call succeeds, every expert count and offset is zero."""
+    wl = W.small(T=1)
+    s = moe.shape(0, wl.d, wl.N, wl.k, wl.h, 1, 0)
+    w, b = dev_router(wl)
+    wg, wu, wd = dev_experts(wl)
+    u = torch.empty((0, wl.d), dtype=torch.bfloat16, device="cuda")
+    y = torch.empty((0, wl.d), dtype=torch.bfloat16, device="cuda")
+    i32 = dict(dtype=torch.int32, device="cuda")
+    outs = dict(counts=torch.full((wl.N,), -1, **i32), offsets=torch.full((wl.N + 1,), -1, **i32),
+                totals=torch.full((3,), -1, **i32))
+    moe.moe_layer_fwd(s, w, wg, wu, wd, u, y, bias=b, outputs=outs)
+    torch.cuda.synchronize()
+    for key, t in outs.items():
+        assert torch.all(t == 0), key
