@@ -91,6 +91,94 @@ __global__ void __launch_bounds__((BT / TM) * (BN / TN))
   }
 }
 
+// Many experts (N > 16): a 128 x 128 (tokens x experts) block tile, 8 x 8
+// logits per thread, K walked in steps of 16 through double-buffered shared
+// tiles (the next step's global loads are held in registers while the
+// current step computes).  Each logit is still one thread's FMA chain over j
+// in ascending order, so the result equals the other router kernels bit for
+// bit.  A thread's rows are {4 ty + i, 64 + 4 ty + i} and its experts
+// {4 tx + j, 64 + 4 tx + j}, so the 16-byte shared reads of a warp are
+// broadcasts or consecutive.
+constexpr int kBigBT = 128, kBigBN = 128, kBigBK = 16, kBigThreads = 256;
+
+template <typename TU>
+__global__ void __launch_bounds__(kBigThreads)
+    router_logits_big(const TU* __restrict__ u, const float* __restrict__ w,
+                      const float* __restrict__ bias, float* __restrict__ z, int T, int d, int N) {
+  pdl_wait();
+  pdl_allow_next();
+  __shared__ __align__(16) float us[2][kBigBK][kBigBT];
+  __shared__ __align__(16) float wsm[2][kBigBK][kBigBN];
+  const int t0 = blockIdx.x * kBigBT, n0 = blockIdx.y * kBigBN;
+  const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
+  // this thread's share of a K step: row lr (token / expert), 8 columns at lc
+  const int lr = tid >> 1, lc = (tid & 1) * 8;
+  float acc[8][8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[i][j] = 0.0f;
+  float ru[8], rw[8];
+  auto fetch = [&](int k0) {
+    const int kw = min(kBigBK, d - k0);  // multiple of 8
+    if (t0 + lr < T && lc < kw) {
+      load8(u + (size_t)(t0 + lr) * d + k0 + lc, ru);
+    } else {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) ru[j] = 0.0f;
+    }
+    if (n0 + lr < N && lc < kw) {
+      load8(w + (size_t)(n0 + lr) * d + k0 + lc, rw);
+    } else {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) rw[j] = 0.0f;
+    }
+  };
+  auto put = [&](int buf) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      us[buf][lc + j][lr] = ru[j];
+      wsm[buf][lc + j][lr] = rw[j];
+    }
+  };
+  fetch(0);
+  put(0);
+  __syncthreads();
+  int buf = 0;
+  for (int k0 = 0; k0 < d; k0 += kBigBK) {
+    const bool more = k0 + kBigBK < d;
+    if (more) fetch(k0 + kBigBK);
+    const int kw = min(kBigBK, d - k0);
+    for (int kk = 0; kk < kw; ++kk) {
+      const float4 a0 = *reinterpret_cast<const float4*>(&us[buf][kk][4 * ty]);
+      const float4 a1 = *reinterpret_cast<const float4*>(&us[buf][kk][64 + 4 * ty]);
+      const float4 b0 = *reinterpret_cast<const float4*>(&wsm[buf][kk][4 * tx]);
+      const float4 b1 = *reinterpret_cast<const float4*>(&wsm[buf][kk][64 + 4 * tx]);
+      const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+      const float b[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[i][j] = __fmaf_rn(b[j], a[i], acc[i][j]);
+    }
+    if (more) {
+      put(buf ^ 1);
+      __syncthreads();
+      buf ^= 1;
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int t = t0 + (i < 4 ? 4 * ty + i : 64 + 4 * ty + i - 4);
+    if (t >= T) continue;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int n = n0 + (j < 4 ? 4 * tx + j : 64 + 4 * tx + j - 4);
+      if (n < N) z[(size_t)t * N + n] = bias ? __fadd_rn(acc[i][j], bias[n]) : acc[i][j];
+    }
+  }
+}
+
 // (z, index) ordering of the top-k: larger z first, equal z -> lower index.
 __device__ __forceinline__ bool better(float za, int ia, float zb, int ib) {
   return za > zb || (za == zb && ia < ib);
@@ -300,9 +388,9 @@ void launch_logits(const TU* u, const float* w, const float* bias, float* z, int
     MOE_PREFER_SHARED((router_logits_kernel<64, 16, 4, 4, TU>));
     launch_pdl(router_logits_kernel<64, 16, 4, 4, TU>, dim3(grid), dim3(64), 0, st, u, w, bias, z, T, d, N);
   } else {
-    dim3 grid((T + 63) / 64, (N + 63) / 64);
-    MOE_PREFER_SHARED((router_logits_kernel<64, 64, 4, 4, TU>));
-    launch_pdl(router_logits_kernel<64, 64, 4, 4, TU>, dim3(grid), dim3(256), 0, st, u, w, bias, z, T, d, N);
+    dim3 grid((T + kBigBT - 1) / kBigBT, (N + kBigBN - 1) / kBigBN);
+    MOE_PREFER_SHARED((router_logits_big<TU>));
+    launch_pdl(router_logits_big<TU>, grid, dim3(kBigThreads), 0, st, u, w, bias, z, T, d, N);
   }
 }
 
