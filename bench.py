@@ -166,6 +166,34 @@ class Replica:
         return sum(t.numel() * t.element_size() for t in [self.u, self.w_route, *self.w])
 
 
+def layer_launches(wl: W.Workload, sms: int = 148) -> int:
+    """Kernels moe_layer_fwd launches for this workload (the library's own
+    path choices restated): routing, permutation and row copies in one
+    cooperative launch when a CTA's token rows and the router rows fit on chip,
+    else router (+counts) / permutation / gather; the expert FFN in one fused
+    launch for small h, else gate/up + down; then the combine."""
+    T, d, N, k, h = wl.T, wl.d, wl.N, wl.k, wl.h
+    el = 4 if wl.act_dtype == S.DT_F32 else 2
+    r16 = lambda b: -(-b // 16) * 16
+    grid = min(T, sms)
+    tpc = -(-T // grid) if T else 0
+    smem = (r16(tpc * (d * el + 16)) + r16(N * (d + 4) * 4) + r16(tpc * N * 4) + 2 * r16(tpc * k * 4)
+            + 3 * 64 + 80 + 8 * 16 * 4 + r16(-(-T // tpc) * N * 4 if tpc else 0))
+    one_launch_routing = (T > 0 and N <= 16 and k <= N and tpc * k <= 256
+                          and smem <= 200 * 1024 and wl.act_dtype in (S.DT_F32, S.DT_BF16))
+    if one_launch_routing:
+        routing = 1
+    elif N <= 16 and k <= 16 and (-(-T // (16 if N <= 8 else 8))) * N <= 8192:
+        routing = 3  # router with counts, dispatch, gather
+    else:
+        routing = 6  # logits, top-k, histogram, scan, scatter, gather
+    if wl.act_dtype == S.DT_F32:
+        ffn = 2
+    else:
+        ffn = 1 if (h % 64 == 0 and h <= 256 and d % 128 == 0 and (h // 64 + d // 128) * 64 <= 512) else 2
+    return routing + ffn + 1
+
+
 class Step:
     """The layer step through the C ABI, split at the expert FFN so that the
     tcgen05 GEMM launches can be timed on their own stream position."""
@@ -198,11 +226,7 @@ class Step:
         self.lws = torch.empty(moe.moe_layer_workspace_bytes(self.s, wl.act_dtype),
                                dtype=torch.uint8, device="cuda")
         self.outs = {"top_idx": self.top_idx, "top_w": self.top_w, "totals": self.totals}
-        tpb = 16 if N <= 8 else 8  # tokens per router block
-        small = N <= 16 and k <= 16 and ((T + tpb - 1) // tpb) * N <= 8192
-        # moe_layer_fwd: route (+counts), dispatch, gather, 2 GEMMs, combine for few
-        # experts; route (2), permute (3), gather, 2 GEMMs, combine otherwise
-        self.launches_per_step = 6 if small else 9
+        self.launches_per_step = layer_launches(wl)
 
     def layer(self, r: Replica):
         """The product entry point: the whole layer in one C-ABI call."""
