@@ -3,7 +3,7 @@
 // (equations z, p, a); the router runs in fp32 as its code's softmax of
 // logits.float() does.
 //
-// Logits are a register-tiled SIMT GEMM: each thread owns TM tokens x TN
+// Logits are a register-tiled SIMT GEMM: each thread owns 8 tokens x 8
 // experts and walks the input dimension in ascending order with one fused
 // multiply-add per step, so every logit is the same sequential fp32 chain
 // whatever the tiling (the reproducible order the routing decision needs).
@@ -16,80 +16,6 @@
 
 namespace moe {
 namespace {
-
-constexpr int kBK = 32;
-
-template <int BT, int BN, int TM, int TN, typename TU>
-__global__ void __launch_bounds__((BT / TM) * (BN / TN))
-    router_logits_kernel(const TU* __restrict__ u, const float* __restrict__ w,
-                         const float* __restrict__ bias, float* __restrict__ z, int T, int d,
-                         int N) {
-  pdl_wait();
-  pdl_allow_next();
-  constexpr int NT = (BT / TM) * (BN / TN);
-  __shared__ __align__(16) float us[kBK][BT];
-  __shared__ __align__(16) float wsm[kBK][BN];
-  const int t0 = blockIdx.x * BT, n0 = blockIdx.y * BN;
-  const int tid = threadIdx.x;
-  const int tx = tid % (BN / TN);
-  const int ty = tid / (BN / TN);
-  float acc[TM][TN];
-#pragma unroll
-  for (int i = 0; i < TM; ++i)
-#pragma unroll
-    for (int j = 0; j < TN; ++j) acc[i][j] = 0.0f;
-
-  for (int k0 = 0; k0 < d; k0 += kBK) {
-    const int kw = min(kBK, d - k0);  // multiple of 8
-    for (int v = tid; v < BT * (kBK / 8); v += NT) {
-      const int r = v / (kBK / 8), c8 = (v % (kBK / 8)) * 8;
-      float tmp[8];
-      if (t0 + r < T && c8 < kw) {
-        load8(u + (size_t)(t0 + r) * d + k0 + c8, tmp);
-      } else {
-#pragma unroll
-        for (int j = 0; j < 8; ++j) tmp[j] = 0.0f;
-      }
-#pragma unroll
-      for (int j = 0; j < 8; ++j) us[c8 + j][r] = tmp[j];
-    }
-    for (int v = tid; v < BN * (kBK / 8); v += NT) {
-      const int r = v / (kBK / 8), c8 = (v % (kBK / 8)) * 8;
-      float tmp[8];
-      if (n0 + r < N && c8 < kw) {
-        load8(w + (size_t)(n0 + r) * d + k0 + c8, tmp);
-      } else {
-#pragma unroll
-        for (int j = 0; j < 8; ++j) tmp[j] = 0.0f;
-      }
-#pragma unroll
-      for (int j = 0; j < 8; ++j) wsm[c8 + j][r] = tmp[j];
-    }
-    __syncthreads();
-    for (int kk = 0; kk < kw; ++kk) {
-      float a[TM], b[TN];
-#pragma unroll
-      for (int i = 0; i < TM; ++i) a[i] = us[kk][ty * TM + i];
-#pragma unroll
-      for (int j = 0; j < TN; ++j) b[j] = wsm[kk][tx * TN + j];
-#pragma unroll
-      for (int i = 0; i < TM; ++i)
-#pragma unroll
-        for (int j = 0; j < TN; ++j) acc[i][j] = __fmaf_rn(b[j], a[i], acc[i][j]);
-    }
-    __syncthreads();
-  }
-#pragma unroll
-  for (int i = 0; i < TM; ++i) {
-    const int t = t0 + ty * TM + i;
-    if (t >= T) continue;
-#pragma unroll
-    for (int j = 0; j < TN; ++j) {
-      const int n = n0 + tx * TN + j;
-      if (n < N) z[(size_t)t * N + n] = bias ? __fadd_rn(acc[i][j], bias[n]) : acc[i][j];
-    }
-  }
-}
 
 // Many experts (N > 16): a 128 x 128 (tokens x experts) block tile, 8 x 8
 // logits per thread, K walked in steps of 16 through double-buffered shared
@@ -379,19 +305,9 @@ __global__ void __launch_bounds__(kRouteThreads)
 template <typename TU>
 void launch_logits(const TU* u, const float* w, const float* bias, float* z, int T, int d, int N,
                    cudaStream_t st) {
-  if (N <= 8) {
-    dim3 grid((T + 63) / 64, 1);
-    MOE_PREFER_SHARED((router_logits_kernel<64, 8, 2, 4, TU>));
-    launch_pdl(router_logits_kernel<64, 8, 2, 4, TU>, dim3(grid), dim3(64), 0, st, u, w, bias, z, T, d, N);
-  } else if (N <= 16) {
-    dim3 grid((T + 63) / 64, 1);
-    MOE_PREFER_SHARED((router_logits_kernel<64, 16, 4, 4, TU>));
-    launch_pdl(router_logits_kernel<64, 16, 4, 4, TU>, dim3(grid), dim3(64), 0, st, u, w, bias, z, T, d, N);
-  } else {
-    dim3 grid((T + kBigBT - 1) / kBigBT, (N + kBigBN - 1) / kBigBN);
-    MOE_PREFER_SHARED((router_logits_big<TU>));
-    launch_pdl(router_logits_big<TU>, grid, dim3(kBigThreads), 0, st, u, w, bias, z, T, d, N);
-  }
+  dim3 grid((T + kBigBT - 1) / kBigBT, (N + kBigBN - 1) / kBigBN);
+  MOE_PREFER_SHARED((router_logits_big<TU>));
+  launch_pdl(router_logits_big<TU>, grid, dim3(kBigThreads), 0, st, u, w, bias, z, T, d, N);
 }
 
 }  // namespace
