@@ -73,9 +73,13 @@ def lib():
         L.or_ledger.argtypes = [i64, i64, i64, i64, vp, vp, vp, vp]
         L.or_bandwidth_gain.argtypes = [i64, i64, i64]
         L.or_bandwidth_gain.restype = dbl
+        L.or_qb_cutoffs.argtypes = [i64, i64, i64, vp, vp, vp]
+        L.or_qb_exact.argtypes = [i64, i64, vp, vp, i64, vp, vp]
+        L.or_qb_hist.argtypes = [i64, i64, vp, vp, i64, i64, vp]
         for f in (L.or_mat_decode, L.or_route, L.or_route_from_logits, L.or_aux_stats,
                   L.or_permute, L.or_matvec, L.or_expert, L.or_moe_tokens, L.or_moe_dense,
-                  L.or_rmsnorm, L.or_ledger, L.or_combine):
+                  L.or_rmsnorm, L.or_ledger, L.or_combine, L.or_qb_cutoffs, L.or_qb_exact,
+                  L.or_qb_hist):
             f.restype = None
         _lib = L
     return _lib
@@ -330,3 +334,36 @@ def ledger(d, h, N, k):
 
 def bandwidth_gain(ffn, top_k, ffn_e):
     return float(lib().or_bandwidth_gain(ffn, top_k, ffn_e))
+
+
+# ------------------------------------------------------- quantile balancing
+def qb_cutoffs(scores, k, bias=None):
+    """a_i: the k-th largest s_ij + b_j of each token (Stable LatentMoE demo
+    document, Quantile Balancing), fp32."""
+    s = _c(scores, np.float32)
+    T, N = s.shape
+    b = None if bias is None else _c(bias, np.float32)
+    a = np.empty(T, np.float32)
+    lib().or_qb_cutoffs(T, N, k, s.ctypes.data, _p(b), a.ctypes.data)
+    return a
+
+
+def qb_exact(scores, cutoffs, q):
+    """(b, loads): b_j = the q-th smallest required_ij = a_i - s_ij; loads_j =
+    #{i : required_ij <= b_j}."""
+    s, a = _c(scores, np.float32), _c(cutoffs, np.float32)
+    T, N = s.shape
+    b = np.empty(N, np.float32)
+    loads = np.empty(N, np.int32)
+    lib().or_qb_exact(T, N, s.ctypes.data, a.ctypes.data, q, b.ctypes.data, loads.ctypes.data)
+    return b, loads
+
+
+def qb_hist(scores, cutoffs, q, bins):
+    """The histogram estimate of the same quantile (bins equal bins over the
+    range of required_j, the upper edge of the bin where the count reaches q)."""
+    s, a = _c(scores, np.float32), _c(cutoffs, np.float32)
+    T, N = s.shape
+    b = np.empty(N, np.float32)
+    lib().or_qb_hist(T, N, s.ctypes.data, a.ctypes.data, q, bins, b.ctypes.data)
+    return b

@@ -420,3 +420,102 @@ void or_ledger(int64_t d, int64_t h, int64_t N, int64_t k, int64_t* one, int64_t
 double or_bandwidth_gain(int64_t ffn, int64_t top_k, int64_t ffn_e) {
   return (double)ffn / (double)(top_k * ffn_e);
 }
+
+/* ------------------------------------------------------- quantile balancing */
+/* [LatentMoE] Quantile Balancing.  With every token's top-k cutoff a_i held
+ * fixed, expert j takes token i iff s_ij + b_j >= a_i, i.e. iff
+ * b_j >= required_ij = a_i - s_ij; the bias that gives expert j exactly q
+ * tokens is the q-th smallest required_ij, found in one step instead of a
+ * fixed-step update.  The arithmetic is the router's fp32: the selection
+ * score s_ij + b_j and required_ij = a_i - s_ij each round once. */
+
+static int or_cmp_float_desc(const void* x, const void* y) {
+  const float a = *(const float*)x, b = *(const float*)y;
+  return (a < b) - (a > b);
+}
+static int or_cmp_float_asc(const void* x, const void* y) {
+  const float a = *(const float*)x, b = *(const float*)y;
+  return (a > b) - (a < b);
+}
+
+/* a_i = the k-th largest selection score s_ij + b_j (b nullable = 0). */
+void or_qb_cutoffs(int64_t T, int64_t N, int64_t k, const float* s, const float* b, float* a) {
+  float* row = (float*)malloc((size_t)N * sizeof(float));
+  for (int64_t t = 0; t < T; ++t) {
+    for (int64_t j = 0; j < N; ++j) {
+      const float v = s[t * N + j];
+      row[j] = b ? v + b[j] : v;
+    }
+    qsort(row, (size_t)N, sizeof(float), or_cmp_float_desc);
+    a[t] = row[k - 1];
+  }
+  free(row);
+}
+
+/* b_j = the q-th smallest (1-based) required_ij over the T tokens, a zero
+ * returned as +0; loads_j = #{i : required_ij <= b_j} (q when the values are
+ * distinct). */
+void or_qb_exact(int64_t T, int64_t N, const float* s, const float* a, int64_t q, float* b_out,
+                 int32_t* loads) {
+  float* req = (float*)malloc((size_t)T * sizeof(float));
+  float* srt = (float*)malloc((size_t)T * sizeof(float));
+  for (int64_t j = 0; j < N; ++j) {
+    for (int64_t i = 0; i < T; ++i) req[i] = a[i] - s[i * N + j];
+    memcpy(srt, req, (size_t)T * sizeof(float));
+    qsort(srt, (size_t)T, sizeof(float), or_cmp_float_asc);
+    float v = srt[q - 1];
+    if (v == 0.0f) v = 0.0f;
+    b_out[j] = v;
+    if (loads) {
+      int32_t c = 0;
+      for (int64_t i = 0; i < T; ++i) c += req[i] <= v;
+      loads[j] = c;
+    }
+  }
+  free(req);
+  free(srt);
+}
+
+/* Histogram estimate of the same quantile: B equal bins over [lo, hi], the
+ * smallest and largest required_ij of expert j; the bin of v is
+ * min(B - 1, trunc((v - lo) * scale)) with scale = B / (hi - lo); the
+ * estimate is the upper edge lo + (c + 1) * w of the first bin c at which the
+ * running count reaches q, w = (hi - lo) / B.  Every step is one fp32
+ * operation; hi == lo gives lo. */
+void or_qb_hist(int64_t T, int64_t N, const float* s, const float* a, int64_t q, int64_t B,
+                float* b_out) {
+  float* req = (float*)malloc((size_t)T * sizeof(float));
+  int64_t* cnt = (int64_t*)malloc((size_t)B * sizeof(int64_t));
+  for (int64_t j = 0; j < N; ++j) {
+    float lo = 0.0f, hi = 0.0f;
+    for (int64_t i = 0; i < T; ++i) {
+      req[i] = a[i] - s[i * N + j];
+      if (i == 0 || req[i] < lo) lo = req[i];
+      if (i == 0 || req[i] > hi) hi = req[i];
+    }
+    if (!(hi > lo)) {
+      b_out[j] = lo;
+      continue;
+    }
+    const float range = hi - lo;
+    const float scale = (float)B / range;
+    const float w = range / (float)B;
+    for (int64_t c = 0; c < B; ++c) cnt[c] = 0;
+    for (int64_t i = 0; i < T; ++i) {
+      const float x = (req[i] - lo) * scale;
+      int64_t c = (int64_t)x;
+      if (c > B - 1) c = B - 1;
+      ++cnt[c];
+    }
+    int64_t c = 0, cum = 0;
+    for (; c < B; ++c) {
+      cum += cnt[c];
+      if (cum >= q) break;
+    }
+    if (c > B - 1) c = B - 1;
+    const float edge = (float)(c + 1) * w;
+    b_out[j] = lo + edge;
+  }
+  free(req);
+  free(cnt);
+}

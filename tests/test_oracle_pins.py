@@ -510,3 +510,59 @@ def test_latent_single_expert_closed_form():
         m = d @ bf16(_silu(G) * U)
         mh = bf16(m / np.sqrt(np.mean(m * m) + 1e-6))
         assert np.allclose(y[t], W_upp.decode() @ mh, rtol=1e-11, atol=1e-12)
+
+
+# ------------------------------------------------------- quantile balancing
+# Stable LatentMoE demo document, Quantile Balancing: with every token's top-k
+# cutoff a_i fixed, the bias that gives expert j exactly q tokens is the q-th
+# smallest required_ij = a_i - s_ij.
+def test_qb_hand_example():
+    # k = 1: a_i = max_j s_ij = [3, 2, 5, 1.5].
+    # expert 0: required = a - s_0 = [0, 2, 0, 0.5] -> sorted [0, 0, 0.5, 2]
+    # expert 1: required = a - s_1 = [2, 0, 1, 0]   -> sorted [0, 0, 1, 2]
+    s = np.array([[3, 1], [0, 2], [5, 4], [1, 1.5]], np.float32)
+    a = O.qb_cutoffs(s, 1)
+    assert a.tolist() == [3.0, 2.0, 5.0, 1.5]
+    b, loads = O.qb_exact(s, a, 2)
+    assert b.tolist() == [0.0, 0.0] and loads.tolist() == [2, 2]
+    b, loads = O.qb_exact(s, a, 3)
+    assert b.tolist() == [0.5, 1.0] and loads.tolist() == [3, 3]
+    # 4 bins over [0, 2] (width 0.5): expert 0 counts [2, 1, 0, 1] reach 3 in
+    # bin 1 -> edge 1.0; expert 1 counts [2, 0, 1, 1] reach 3 in bin 2 -> 1.5
+    assert O.qb_hist(s, a, 3, 4).tolist() == [1.0, 1.5]
+
+
+def test_qb_matches_numpy_sort_and_balances():
+    rng = np.random.default_rng(11)
+    T, N, k, q = 300, 13, 3, 47
+    s = rng.standard_normal((T, N)).astype(np.float32)
+    bias = (0.1 * rng.standard_normal(N)).astype(np.float32)
+    a = O.qb_cutoffs(s, k, bias)
+    sel = (s + bias[None, :]).astype(np.float32)  # one fp32 add per score
+    assert np.array_equal(a, np.sort(sel, axis=1)[:, N - k])
+    req = (a[:, None] - s).astype(np.float32)
+    b, loads = O.qb_exact(s, a, q)
+    ref = np.sort(req, axis=0)[q - 1]
+    assert np.array_equal(b, ref + np.float32(0.0))
+    # the q-th order statistic: fewer than q tokens lie strictly below it and
+    # at least q clear it (more only through ties, e.g. required = 0 for the
+    # tokens whose k-th expert is j itself)
+    assert np.all((req < b[None, :]).sum(0) <= q - 1)
+    assert np.all(loads >= q)
+    assert np.array_equal(loads, (req <= b[None, :]).sum(0))
+    ties = (req == b[None, :]).sum(0)
+    assert np.all(loads - ties <= q - 1)
+
+
+def test_qb_histogram_estimate_brackets_the_exact_quantile():
+    rng = np.random.default_rng(5)
+    T, N, k, q, B = 1000, 7, 2, 250, 64
+    s = rng.standard_normal((T, N)).astype(np.float32)
+    a = O.qb_cutoffs(s, k)
+    exact, _ = O.qb_exact(s, a, q)
+    est = O.qb_hist(s, a, q, B)
+    req = (a[:, None] - s).astype(np.float32)
+    w = (req.max(0) - req.min(0)) / B
+    slack = 4 * np.spacing(np.abs(req).max(0))
+    assert np.all(est >= exact - slack)
+    assert np.all(est - exact <= w + slack)
