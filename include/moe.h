@@ -304,6 +304,29 @@ MOE_API int moe_decode_step(const moe_shape* shape, int32_t n_layers, const moe_
                             const uint16_t* u0, uint16_t* u_out, int32_t* top_idx_all, void* ws,
                             size_t ws_bytes, void* stream);
 
+/* ---------------------------------------------------- quantile balancing */
+/* Quantile balancing of the expert biases ("Stable LatentMoE interactive demo
+ * document", Quantile Balancing).  scores [T][N] fp32 are the router logits,
+ * bias [N] fp32 (nullable = 0) the current balancing bias.  With every
+ * token's cutoff a_i = the k-th largest s_ij + b_j held fixed, expert j takes
+ * token i iff b_j >= required_ij = a_i - s_ij, so the bias giving expert j q
+ * tokens is the q-th smallest required_ij:
+ *   cutoff [T]      (nullable: kept in the workspace) a_i;
+ *   bias_exact [N]  the q-th smallest required_ij (a zero as +0);
+ *   bias_hist [N]   (nullable, needs bins >= 1) the histogram estimate: bins
+ *                   equal bins over the [min, max] of required_j, the upper
+ *                   edge of the first bin whose running count reaches q;
+ *   loads [N]       (nullable) #{i : required_ij <= bias_exact_j} (q, or more
+ *                   through ties).
+ * Every step is one fp32 operation in a fixed order (bit-reproducible).
+ * Limits: 1 <= T <= 32768, 1 <= N <= 1024, 1 <= k <= min(N, 32),
+ * 1 <= q <= T, 0 <= bins <= 4096.  Device pointers, caller-owned. */
+MOE_API size_t moe_quantile_balance_workspace_bytes(int32_t T, int32_t N);
+MOE_API int moe_quantile_balance(int32_t T, int32_t N, int32_t k, const float* scores,
+                                 const float* bias, int32_t q, int32_t bins, float* cutoff,
+                                 float* bias_exact, float* bias_hist, int32_t* loads, void* ws,
+                                 size_t ws_bytes, void* stream);
+
 /* ----------------------------------------------------------- diagnostics */
 /* Human-readable name of a status code (static string). */
 MOE_API const char* moe_status_string(int32_t status);

@@ -494,7 +494,7 @@ void or_qb_hist(int64_t T, int64_t N, const float* s, const float* a, int64_t q,
       if (i == 0 || req[i] > hi) hi = req[i];
     }
     if (!(hi > lo)) {
-      b_out[j] = lo;
+      b_out[j] = lo == 0.0f ? 0.0f : lo;
       continue;
     }
     const float range = hi - lo;

@@ -83,6 +83,9 @@ _PROTOS = {
                                 _vp, _sz, _vp]),
     "moe_decode_step": (_i32, [_P_SHAPE, _i32, ctypes.POINTER(MoeQ4Layer), _vp, _vp, _vp, _vp,
                                _sz, _vp]),
+    "moe_quantile_balance_workspace_bytes": (_sz, [_i32, _i32]),
+    "moe_quantile_balance": (_i32, [_i32, _i32, _i32, _vp, _vp, _i32, _i32, _vp, _vp, _vp, _vp,
+                                    _vp, _sz, _vp]),
     "moe_status_string": (ctypes.c_char_p, [_i32]),
     "moe_device_status": (_i32, [_vp, ctypes.POINTER(_i32)]),
     "moe_reset_device_status": (_i32, [_vp]),
@@ -270,6 +273,20 @@ def moe_decode_step(s: MoeShape, layers, u0, u_out, top_idx_all=None, ws=None, s
     _check(_lib.moe_decode_step(ctypes.byref(s), len(layers), arr, _ptr(u0), _ptr(u_out),
                                 _ptr(top_idx_all), _ptr(wbuf), wlen, _stream(stream)),
            "moe_decode_step")
+
+
+def moe_quantile_balance_workspace_bytes(T: int, N: int) -> int:
+    return int(_lib.moe_quantile_balance_workspace_bytes(T, N))
+
+
+def moe_quantile_balance(scores, k: int, q: int, bias_exact, bias=None, bins: int = 0,
+                         cutoff=None, bias_hist=None, loads=None, ws=None, stream=None):
+    """scores [T][N] fp32 device tensor; outputs are device tensors (see moe.h)."""
+    T, N = scores.shape
+    wbuf, wlen = _ws(moe_quantile_balance_workspace_bytes(T, N), scores.device, ws)
+    _check(_lib.moe_quantile_balance(T, N, k, _ptr(scores), _ptr(bias), q, bins, _ptr(cutoff),
+                                     _ptr(bias_exact), _ptr(bias_hist), _ptr(loads), _ptr(wbuf),
+                                     wlen, _stream(stream)), "moe_quantile_balance")
 
 
 def moe_device_status(stream=None) -> int:

@@ -109,3 +109,27 @@ def test_workspace_queries_are_host_only_and_monotone():
               lambda s: lib.moe_layer_workspace_bytes(ctypes.byref(s), 1),
               lambda s: lib.moe_expert_ffn_workspace_bytes(ctypes.byref(s), 512, 1)):
         assert 0 < q(small) <= q(big)
+
+
+def test_quantile_balance_rejects_bad_arguments_on_the_host():
+    lib = moe._lib
+    p = 4096  # any non-null address: the checks run before any device work
+    bad = [(0, 8, 2, 1, 0),        # T = 0
+           (100, 0, 1, 1, 0),      # N = 0
+           (100, 2000, 2, 1, 0),   # N > 1024
+           (100, 8, 9, 1, 0),      # k > N
+           (100, 64, 33, 1, 0),    # k > 32
+           (100, 8, 2, 0, 0),      # q = 0
+           (100, 8, 2, 101, 0),    # q > T
+           (100, 8, 2, 10, 5000),  # bins > 4096
+           (40000, 8, 2, 10, 0)]   # T > 32768
+    for T, N, k, q, bins in bad:
+        assert lib.moe_quantile_balance(T, N, k, p, None, q, bins, p, p, None, None, p, 1 << 20,
+                                        None) == -1
+    # a histogram output needs bins >= 1
+    assert lib.moe_quantile_balance(100, 8, 2, 10, None, 10, 0, p, p, p, None, p, 1 << 20,
+                                    None) == -1
+    # no cutoff output and no workspace
+    assert lib.moe_quantile_balance(100, 8, 2, p, None, 10, 0, None, p, None, None, None, 0,
+                                    None) == -6
+    assert lib.moe_quantile_balance_workspace_bytes(100, 8) >= 400
