@@ -219,7 +219,11 @@ typedef struct {
  * weighted combine, plus the aux statistics when out->f/P/n_sum_fP are set.
  * u and y are [T][d] in act_dtype (MOE_F32 or MOE_BF16).  y excludes the
  * residual: a dropped dispatch contributes zero (tutorial §3.5: the
- * residual path carries it).  ws: moe_layer_workspace_bytes. */
+ * residual path carries it).  ws: moe_layer_workspace_bytes.  For few
+ * experts whose token rows fit on chip, routing, permutation and gather run
+ * as one cooperative launch whose grid-barrier words live in ws (zeroed by
+ * the call), so a workspace serves one call at a time; results are the same
+ * bit for bit on either path.  Capturable in a CUDA graph. */
 MOE_API size_t moe_layer_workspace_bytes(const moe_shape* shape, int32_t act_dtype);
 MOE_API int moe_layer_fwd(const moe_shape* shape, const moe_layer_weights* w, const void* u,
                   int32_t act_dtype, void* y, const moe_layer_outputs* out, void* ws,
