@@ -76,10 +76,11 @@ def lib():
         L.or_qb_cutoffs.argtypes = [i64, i64, i64, vp, vp, vp]
         L.or_qb_exact.argtypes = [i64, i64, vp, vp, i64, vp, vp]
         L.or_qb_hist.argtypes = [i64, i64, vp, vp, i64, i64, vp]
+        L.or_aux_grad.argtypes = [i64, i64, dbl, vp, vp, vp]
         for f in (L.or_mat_decode, L.or_route, L.or_route_from_logits, L.or_aux_stats,
                   L.or_permute, L.or_matvec, L.or_expert, L.or_moe_tokens, L.or_moe_dense,
                   L.or_rmsnorm, L.or_ledger, L.or_combine, L.or_qb_cutoffs, L.or_qb_exact,
-                  L.or_qb_hist):
+                  L.or_qb_hist, L.or_aux_grad):
             f.restype = None
         _lib = L
     return _lib
@@ -367,3 +368,12 @@ def qb_hist(scores, cutoffs, q, bins):
     b = np.empty(N, np.float32)
     lib().or_qb_hist(T, N, s.ctypes.data, a.ctypes.data, q, bins, b.ctypes.data)
     return b
+
+
+def aux_grad(probs, f, alpha=1.0):
+    """dL_aux/dz [T][N] with the loads f held constant (tutorial §3.7)."""
+    p, f = _c(probs, np.float64), _c(f, np.float64)
+    T, N = p.shape
+    dz = np.empty((T, N), np.float64)
+    lib().or_aux_grad(T, N, alpha, p.ctypes.data, f.ctypes.data, dz.ctypes.data)
+    return dz

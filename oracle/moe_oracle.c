@@ -519,3 +519,16 @@ void or_qb_hist(int64_t T, int64_t N, const float* s, const float* a, int64_t q,
   free(req);
   free(cnt);
 }
+
+/* ------------------------------------------------------ aux-loss gradient */
+/* [MoE tutorial] §3.7: with the batch loads f held constant,
+ * dL_aux/dz_tj = (alpha N / T) p_tj (f_j - sum_i f_i p_ti), in double. */
+void or_aux_grad(int64_t T, int64_t N, double alpha, const double* p, const double* f,
+                 double* dz) {
+  const double c = alpha * (double)N / (double)T;
+  for (int64_t t = 0; t < T; ++t) {
+    double fbar = 0.0;
+    for (int64_t i = 0; i < N; ++i) fbar += f[i] * p[t * N + i];
+    for (int64_t j = 0; j < N; ++j) dz[t * N + j] = c * p[t * N + j] * (f[j] - fbar);
+  }
+}

@@ -566,3 +566,47 @@ def test_qb_histogram_estimate_brackets_the_exact_quantile():
     slack = 4 * np.spacing(np.abs(req).max(0))
     assert np.all(est >= exact - slack)
     assert np.all(est - exact <= w + slack)
+
+
+# ------------------------------------------------------- aux-loss gradient
+def _aux_loss(z, f, alpha):
+    """alpha N sum_i f_i P_i with P the batch mean of softmax(z) (tutorial §3.4)."""
+    e = np.exp(z - z.max(1, keepdims=True))
+    p = e / e.sum(1, keepdims=True)
+    return alpha * z.shape[1] * float((f * p.mean(0)).sum())
+
+
+def test_aux_grad_matches_central_differences():
+    """Tutorial §3.7 closed form vs a numerical derivative of §3.4's L_aux with
+    the loads f held constant."""
+    rng = np.random.default_rng(8)
+    T, N, alpha = 6, 5, 0.01
+    z = rng.standard_normal((T, N))
+    f = rng.dirichlet(np.ones(N))
+    e = np.exp(z - z.max(1, keepdims=True))
+    p = e / e.sum(1, keepdims=True)
+    dz = O.aux_grad(p, f, alpha)
+    h = 1e-6
+    num = np.empty_like(z)
+    for t in range(T):
+        for j in range(N):
+            zp, zm = z.copy(), z.copy()
+            zp[t, j] += h
+            zm[t, j] -= h
+            num[t, j] = (_aux_loss(zp, f, alpha) - _aux_loss(zm, f, alpha)) / (2 * h)
+    assert np.allclose(dz, num, rtol=1e-6, atol=1e-11)
+
+
+def test_aux_grad_invariants():
+    rng = np.random.default_rng(9)
+    T, N = 50, 8
+    p = rng.dirichlet(np.ones(N), size=T)
+    f = rng.dirichlet(np.ones(N))
+    dz = O.aux_grad(p, f, 1.0)
+    assert np.allclose(dz.sum(1), 0.0, atol=1e-15)  # softmax gradients sum to zero per token
+    # perfectly balanced loads push no logit
+    assert np.allclose(O.aux_grad(p, np.full(N, 1.0 / N), 1.0), 0.0, atol=1e-16)
+    # the over-loaded expert of a token with p = f is pushed down (positive gradient)
+    f2 = np.array([0.7, 0.1, 0.1, 0.1])
+    g = O.aux_grad(np.array([[0.25, 0.25, 0.25, 0.25]]), f2, 1.0)
+    assert g[0, 0] > 0 and np.all(g[0, 1:] < 0)
