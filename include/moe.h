@@ -123,6 +123,15 @@ MOE_API int moe_aux_stats(int32_t T, int32_t N, int32_t k, const float* probs, c
                   float* f, float* P, float* n_sum_fP, int32_t* loads, void* ws, size_t ws_bytes,
                   void* stream);
 
+/* Gradient of the aux loss with respect to the router logits, with the
+ * batch loads held constant (tutorial §3.7):
+ *   dz[t][j] = (alpha N / T) p[t][j] (f[j] - sum_i f[i] p[t][i]).
+ * probs [T][N] fp32 (moe_route's probs), f [N] fp32 (moe_aux_stats' f),
+ * dz [T][N] fp32 out.  fp32 arithmetic (max|error| about 1e-6 of max|dz|).
+ * T = 0 is a no-op. */
+MOE_API int moe_aux_grad(int32_t T, int32_t N, float alpha, const float* probs, const float* f,
+                         float* dz, void* stream);
+
 /* --------------------------------------------------------------- permute */
 /* Group the T*k dispatches by expert (tutorial §3.5, §3.6, §3.8).
  * Dispatch (t, s) -> expert top_idx[t][s]; its rank = dispatches to the same

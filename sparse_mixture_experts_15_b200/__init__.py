@@ -83,6 +83,7 @@ _PROTOS = {
                                 _vp, _sz, _vp]),
     "moe_decode_step": (_i32, [_P_SHAPE, _i32, ctypes.POINTER(MoeQ4Layer), _vp, _vp, _vp, _vp,
                                _sz, _vp]),
+    "moe_aux_grad": (_i32, [_i32, _i32, _f32, _vp, _vp, _vp, _vp]),
     "moe_quantile_balance_workspace_bytes": (_sz, [_i32, _i32]),
     "moe_quantile_balance": (_i32, [_i32, _i32, _i32, _vp, _vp, _i32, _i32, _vp, _vp, _vp, _vp,
                                     _vp, _sz, _vp]),
@@ -273,6 +274,13 @@ def moe_decode_step(s: MoeShape, layers, u0, u_out, top_idx_all=None, ws=None, s
     _check(_lib.moe_decode_step(ctypes.byref(s), len(layers), arr, _ptr(u0), _ptr(u_out),
                                 _ptr(top_idx_all), _ptr(wbuf), wlen, _stream(stream)),
            "moe_decode_step")
+
+
+def moe_aux_grad(probs, f, dz, alpha: float = 1.0, stream=None):
+    """dL_aux/dz [T][N] (fp32 device tensors) with the loads f held constant."""
+    T, N = probs.shape
+    _check(_lib.moe_aux_grad(T, N, alpha, _ptr(probs), _ptr(f), _ptr(dz), _stream(stream)),
+           "moe_aux_grad")
 
 
 def moe_quantile_balance_workspace_bytes(T: int, N: int) -> int:

@@ -80,6 +80,28 @@ __global__ void stats_finish(const int32_t* __restrict__ argmax_cnt,
   }
 }
 
+// Tutorial §3.7: with the batch loads f held constant,
+// dL_aux/dz_tj = c p_tj (f_j - sum_i f_i p_ti), c = alpha N / T.  One warp
+// per token: lane l sums f_i p_ti over i = l, l + 32, ... in order, a
+// butterfly adds the 32 partial sums, then each lane writes its experts.
+__global__ void __launch_bounds__(256)
+    aux_grad_kernel(const float* __restrict__ probs, const float* __restrict__ f, int T, int N,
+                    float c, float* __restrict__ dz) {
+  pdl_wait();
+  pdl_allow_next();
+  const int lane = threadIdx.x & 31;
+  for (int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; t < T;
+       t += (gridDim.x * blockDim.x) >> 5) {
+    const float* pt = probs + (size_t)t * N;
+    float part = 0.0f;
+    for (int i = lane; i < N; i += 32) part = __fmaf_rn(f[i], pt[i], part);
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) part = __fadd_rn(part, __shfl_xor_sync(0xffffffffu, part, o));
+    for (int j = lane; j < N; j += 32)
+      dz[(size_t)t * N + j] = __fmul_rn(__fmul_rn(c, pt[j]), __fsub_rn(f[j], part));
+  }
+}
+
 }  // namespace
 
 size_t aux_stats_ws_bytes(int32_t N) { return align_up((size_t)N * 12, 256); }
@@ -119,4 +141,18 @@ extern "C" int moe_aux_stats(int32_t T, int32_t N, int32_t k, const float* probs
   if (T > 0 && !top_idx) return MOE_ERR_INVALID_ARG;
   if (!ws || ws_bytes < aux_stats_ws_bytes(N)) return MOE_ERR_WORKSPACE;
   return launch_aux_stats(T, N, k, probs, top_idx, f, P, n_sum_fP, loads, ws, as_stream(stream));
+}
+
+extern "C" int moe_aux_grad(int32_t T, int32_t N, float alpha, const float* probs, const float* f,
+                            float* dz, void* stream) {
+  using namespace moe;
+  if (T < 0 || N <= 0 || N > 1024) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (!probs || !f || !dz) return MOE_ERR_INVALID_ARG;
+  const float c = (float)((double)alpha * (double)N / (double)T);
+  int blocks = (T + 7) / 8;
+  if (blocks > 148 * 16) blocks = 148 * 16;
+  MOE_PREFER_SHARED((aux_grad_kernel));
+  launch_pdl(aux_grad_kernel, dim3(blocks), dim3(256), 0, as_stream(stream), probs, f, T, N, c, dz);
+  return launch_status();
 }

@@ -133,3 +133,11 @@ def test_quantile_balance_rejects_bad_arguments_on_the_host():
     assert lib.moe_quantile_balance(100, 8, 2, p, None, 10, 0, None, p, None, None, None, 0,
                                     None) == -6
     assert lib.moe_quantile_balance_workspace_bytes(100, 8) >= 400
+
+
+def test_aux_grad_host_checks():
+    lib = moe._lib
+    assert lib.moe_aux_grad(-1, 8, 1.0, 4096, 4096, 4096, None) == -1
+    assert lib.moe_aux_grad(10, 0, 1.0, 4096, 4096, 4096, None) == -1
+    assert lib.moe_aux_grad(10, 8, 1.0, None, 4096, 4096, None) == -1
+    assert lib.moe_aux_grad(0, 8, 1.0, None, None, None, None) == 0  # empty batch: no-op

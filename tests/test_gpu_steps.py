@@ -145,6 +145,29 @@ def test_aux_stats_vs_oracle(name, T):
     assert loads.cpu().numpy().sum() == wl.k * T  # §3.6 conservation
 
 
+@pytest.mark.parametrize("name,T", [("small", 4096), ("latent", 512)])
+def test_aux_grad_vs_oracle(name, T):
+    """Tutorial §3.7: dL_aux/dz from the GPU's own probabilities and loads,
+    against the oracle's closed form on the same values."""
+    wl = W.ALL[name](T=T)
+    z, pr, idx, tw = _route_gpu(wl)
+    N, alpha = wl.N, 0.01
+    f = torch.empty(N, device="cuda")
+    P = torch.empty(N, device="cuda")
+    ns = torch.empty(1, device="cuda")
+    probs = torch.from_numpy(pr).cuda()
+    moe.moe_aux_stats(probs, torch.from_numpy(idx).cuda(), f, P, ns)
+    dz = torch.empty((T, N), device="cuda")
+    moe.moe_aux_grad(probs, f, dz, alpha)
+    torch.cuda.synchronize()
+    got = dz.cpu().numpy().astype(np.float64)
+    ref = O.aux_grad(pr.astype(np.float64), f.cpu().numpy().astype(np.float64), alpha)
+    scale = np.abs(ref).max()
+    assert scale > 0
+    assert np.abs(got - ref).max() <= 1e-5 * scale
+    assert np.abs(got.sum(1)).max() <= 1e-5 * scale  # the gradients of a token sum to zero
+
+
 # ----------------------------------------------------------------- permute
 def _permute_gpu(idx_np, N, C):
     T, k = idx_np.shape
