@@ -1,4 +1,4 @@
-"""CPU oracle for the sparse-MoE SwiGLU layer forward (ctypes over moe_oracle.c).
+"""CPU oracle for the sparse-MoE SwiGLU layer forward and its backward (ctypes over moe_oracle.c).
 
 TEST INFRASTRUCTURE ONLY: imported by tests/, by the smoke check and by the
 CPU-baseline leg of bench.py.  The GPU product path never imports it.
@@ -18,7 +18,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 SO = os.path.join(_HERE, "_moe_oracle.so")
 SRC = os.path.join(_HERE, "moe_oracle.c")
 
-F32, BF16, F16, Q4_0 = 0, 1, 2, 3
+F32, BF16, F16, Q4_0, F64 = 0, 1, 2, 3, 4
 
 
 def build(force: bool = False) -> str:
@@ -77,6 +77,13 @@ def lib():
         L.or_qb_exact.argtypes = [i64, i64, vp, vp, i64, vp, vp]
         L.or_qb_hist.argtypes = [i64, i64, vp, vp, i64, i64, vp]
         L.or_aux_grad.argtypes = [i64, i64, dbl, vp, vp, vp]
+        L.or_layer_loss.argtypes = [i64, i64, i64, ctypes.c_int, vp, vp, vp, ctypes.c_int, dbl,
+                                    dbl, vp, vp, vp, i64, vp, vp, vp, dbl, vp, vp]
+        L.or_layer_loss.restype = dbl
+        L.or_layer_backward.argtypes = [i64, i64, i64, ctypes.c_int, vp, vp, vp, ctypes.c_int,
+                                        dbl, dbl, vp, vp, vp, i64, vp, vp, vp, dbl, vp, vp, vp,
+                                        vp, vp, vp, vp]
+        L.or_layer_backward.restype = None
         for f in (L.or_mat_decode, L.or_route, L.or_route_from_logits, L.or_aux_stats,
                   L.or_permute, L.or_matvec, L.or_expert, L.or_moe_tokens, L.or_moe_dense,
                   L.or_rmsnorm, L.or_ledger, L.or_combine, L.or_qb_cutoffs, L.or_qb_exact,
@@ -102,6 +109,8 @@ class Mat:
         self.dtype, self.rows, self.cols = dtype, rows, cols
         if dtype == F32:
             self.data = _c(data, np.float32)
+        elif dtype == F64:
+            self.data = _c(data, np.float64)
         elif dtype in (BF16, F16):
             self.data = _c(data, np.uint16)
         else:
@@ -377,3 +386,53 @@ def aux_grad(probs, f, alpha=1.0):
     dz = np.empty((T, N), np.float64)
     lib().or_aux_grad(T, N, alpha, p.ctypes.data, f.ctypes.data, dz.ctypes.data)
     return dz
+
+
+# ----------------------------------------------------------- layer backward
+def _layer_args(Wg, Wu, Wd, u, top_idx, row_of, dy, Wr, z, f):
+    u = _c(u, np.float64)
+    T, d_in = u.shape
+    idx = _c(top_idx, np.int32)
+    k = idx.shape[1]
+    N = len(Wg)
+    d_out = Wd[0].rows
+    dy = _c(dy, np.float64).reshape(T, d_out)
+    Wr = None if Wr is None else _c(Wr, np.float64)
+    z = None if z is None else _c(z, np.float64)
+    if Wr is None and z is None:
+        raise ValueError("give the router weights or the logits")
+    row_of = None if row_of is None else _c(row_of, np.int32)
+    f = None if f is None else _c(f, np.float64)
+    return u, T, d_in, idx, k, N, d_out, dy, Wr, z, row_of, f
+
+
+def layer_loss(Wg, Wu, Wd, u, top_idx, dy, Wr=None, z=None, row_of=None, renorm=1, act=0,
+               beta_g=0.0, beta_u=0.0, alpha=0.0, f=None):
+    """(L, y): L = sum dy . y (+ alpha N sum f_i P_i when f is given) with the
+    selected sets top_idx and the dropped dispatches (row_of < 0) held fixed,
+    everything in double.  z = u Wr^T when Wr is given, else the given logits."""
+    u, T, d_in, idx, k, N, d_out, dy, Wr, z, row_of, f = _layer_args(
+        Wg, Wu, Wd, u, top_idx, row_of, dy, Wr, z, f)
+    y = np.empty((T, d_out), np.float64)
+    L = lib().or_layer_loss(T, N, k, renorm, mat_array(Wg), mat_array(Wu), mat_array(Wd), act,
+                            beta_g, beta_u, _p(Wr), _p(z), u.ctypes.data, d_in, idx.ctypes.data,
+                            _p(row_of), dy.ctypes.data, alpha, _p(f), y.ctypes.data)
+    return float(L), y
+
+
+def layer_backward(Wg, Wu, Wd, u, top_idx, dy, Wr=None, z=None, row_of=None, renorm=1, act=0,
+                   beta_g=0.0, beta_u=0.0, alpha=0.0, f=None):
+    """Gradients of layer_loss: dict of dz [T][N], du [T][d_in], dWr [N][d_in]
+    (None without Wr), dWg, dWu [N][h][d_in], dWd [N][d_out][h]."""
+    u, T, d_in, idx, k, N, d_out, dy, Wr, z, row_of, f = _layer_args(
+        Wg, Wu, Wd, u, top_idx, row_of, dy, Wr, z, f)
+    h = Wg[0].rows
+    out = dict(dz=np.empty((T, N)), du=np.empty((T, d_in)),
+               dWr=None if Wr is None else np.empty((N, d_in)),
+               dWg=np.empty((N, h, d_in)), dWu=np.empty((N, h, d_in)), dWd=np.empty((N, d_out, h)))
+    lib().or_layer_backward(T, N, k, renorm, mat_array(Wg), mat_array(Wu), mat_array(Wd), act,
+                            beta_g, beta_u, _p(Wr), _p(z), u.ctypes.data, d_in, idx.ctypes.data,
+                            _p(row_of), dy.ctypes.data, alpha, _p(f), out["dz"].ctypes.data,
+                            out["du"].ctypes.data, _p(out["dWr"]), out["dWg"].ctypes.data,
+                            out["dWu"].ctypes.data, out["dWd"].ctypes.data)
+    return out

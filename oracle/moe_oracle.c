@@ -1,5 +1,6 @@
 /*
- * CPU oracle for the sparse Mixture-of-Experts SwiGLU layer forward.
+ * CPU oracle for the sparse Mixture-of-Experts SwiGLU layer forward and its
+ * backward.
  *
  * TEST INFRASTRUCTURE ONLY.  Only the tests, the smoke check and the CPU
  * baseline leg of the benchmark may load this library.  The GPU product path
@@ -21,11 +22,13 @@
  * in fp32 (§3.2 and its code: softmax of logits.float()); the logits decide
  * the discrete top-k, so they are formed in fp32 in one fixed summation order
  * (or_router_logit below) which any implementation can reproduce bit for bit.
+ * The layer backward at the end of the file forms the logits in double too:
+ * it is the exact-arithmetic gradient, not a replay of the routing decision.
  * Compiled with -ffp-contract=off so each operation rounds on its own.
  *
  * Parity pins: every function is checked against worked numbers printed on
  * the pages, closed forms, brute force or textbook identities in
- * tests/test_oracle_pins.py.  The softmax/SiLU/tanh transcendental values
+ * tests/test_oracle_pins.py and, for the backward, tests/test_oracle_backward.py.  The softmax/SiLU/tanh transcendental values
  * themselves have no printed example beyond the tutorial's aux-loss figures.
  */
 #include <math.h>
@@ -63,7 +66,7 @@ double or_f16_to_f64(uint16_t h) {
 }
 
 /* Storage of an activation or weight tensor. */
-enum { OR_F32 = 0, OR_BF16 = 1, OR_F16 = 2, OR_Q4_0 = 3 };
+enum { OR_F32 = 0, OR_BF16 = 1, OR_F16 = 2, OR_Q4_0 = 3, OR_F64 = 4 };
 
 /* One [rows][cols] matrix in any storage type.  q4_0 (format named in
  * [MCU #13] §4): blocks of 32 consecutive values along a row, one fp16 scale
@@ -73,7 +76,7 @@ enum { OR_F32 = 0, OR_BF16 = 1, OR_F16 = 2, OR_Q4_0 = 3 };
 typedef struct {
   int dtype;
   int64_t rows, cols;
-  const void* data;       /* f32 / bf16 / f16 */
+  const void* data;       /* f32 / bf16 / f16 / f64 */
   const uint8_t* qs;      /* q4_0: [rows][cols/2] */
   const uint16_t* scales; /* q4_0: [rows][cols/32] fp16 codes */
 } or_mat;
@@ -83,6 +86,7 @@ static inline double mat_get(const or_mat* m, int64_t r, int64_t c) {
     case OR_F32: return (double)((const float*)m->data)[r * m->cols + c];
     case OR_BF16: return or_bf16_to_f64(((const uint16_t*)m->data)[r * m->cols + c]);
     case OR_F16: return or_f16_to_f64(((const uint16_t*)m->data)[r * m->cols + c]);
+    case OR_F64: return ((const double*)m->data)[r * m->cols + c];
     default: {
       int64_t b = c / 32, j = c % 32;
       uint8_t byte = m->qs[r * (m->cols / 2) + b * 16 + (j & 15)];
@@ -531,4 +535,241 @@ void or_aux_grad(int64_t T, int64_t N, double alpha, const double* p, const doub
     for (int64_t i = 0; i < N; ++i) fbar += f[i] * p[t * N + i];
     for (int64_t j = 0; j < N; ++j) dz[t * N + j] = c * p[t * N + j] * (f[j] - fbar);
   }
+}
+
+/* ------------------------------------------------------- layer backward */
+/* The loss whose gradient the backward pass forms:
+ *   L = sum_t dy_t . y_t  +  alpha N sum_i f_i P_i      (second term when f != NULL)
+ * y_t = sum over kept slots s of a_{t,s} F_{e_{t,s}}(u_t)   [MoE tutorial] §3.1, §3.2
+ * p_t = softmax(z_t), z_t = W_route u_t (or the given z_t when W_route is NULL)
+ * a_{t,s} = p_{t,e_{t,s}} / sum_r p_{t,e_{t,r}}  (renorm = 1; over all k slots,
+ *           kept or dropped, as in the forward), or p_{t,e_{t,s}} (renorm = 0)
+ * P_i = (1/T) sum_t p_{t,i}                               [MoE tutorial] §3.4
+ * dy is the upstream gradient dL/dy.  The selected sets (top_idx) and the
+ * dropped dispatches (row_of < 0) are inputs and are held fixed: top-k and the
+ * capacity cut are piecewise constant in the parameters, so they contribute
+ * no derivative; the loads f are held fixed as [MoE tutorial] §3.7 states.
+ * Every quantity, the logits included, is in double: this is the exact-
+ * arithmetic gradient, not a replay of the fp32 routing decision.  Only the
+ * selected experts of kept dispatches receive weight gradient, the property
+ * the [LatentMoE] demo tests ("only selected experts receive gradient"). */
+
+/* Softmax of one row in double, max subtracted (as or_route_from_logits). */
+static void or_softmax_row(int64_t N, const double* z, double* p) {
+  double zmax = -INFINITY, den = 0.0;
+  for (int64_t i = 0; i < N; ++i) zmax = fmax(zmax, z[i]);
+  for (int64_t i = 0; i < N; ++i) den += exp(z[i] - zmax);
+  for (int64_t i = 0; i < N; ++i) p[i] = exp(z[i] - zmax) / den;
+}
+
+/* z_t (W_route given: W_route u_t in double; else the given row), p_t, and
+ * the combine weights a_t of the k slots. */
+static void or_token_weights(int64_t N, int64_t d_in, int64_t k, int renorm, const double* Wr,
+                             const double* z_in, const double* u, const int32_t* sel, double* z,
+                             double* p, double* a) {
+  for (int64_t j = 0; j < N; ++j) {
+    if (Wr) {
+      double acc = 0.0;
+      for (int64_t c = 0; c < d_in; ++c) acc += Wr[j * d_in + c] * u[c];
+      z[j] = acc;
+    } else {
+      z[j] = z_in[j];
+    }
+  }
+  or_softmax_row(N, z, p);
+  double ssum = 0.0;
+  for (int64_t s = 0; s < k; ++s) ssum += p[sel[s]];
+  for (int64_t s = 0; s < k; ++s) a[s] = renorm ? p[sel[s]] / ssum : p[sel[s]];
+}
+
+/* L above; y (nullable) receives y_t [T][d_out].  Wr [N][d_in] or NULL (then
+ * z [T][N] is used); f [N] or NULL (no balancing term). */
+double or_layer_loss(int64_t T, int64_t N, int64_t k, int renorm, const or_mat* Wg,
+                     const or_mat* Wu, const or_mat* Wd, int act, double beta_g, double beta_u,
+                     const double* Wr, const double* z, const double* u, int64_t d_in,
+                     const int32_t* top_idx, const int32_t* row_of, const double* dy,
+                     double alpha, const double* f, double* y) {
+  int64_t d_out = Wd[0].rows;
+  double* zt = (double*)malloc(sizeof(double) * (size_t)N);
+  double* pt = (double*)malloc(sizeof(double) * (size_t)N);
+  double* at = (double*)malloc(sizeof(double) * (size_t)k);
+  double* F = (double*)malloc(sizeof(double) * (size_t)d_out);
+  double* yt = (double*)malloc(sizeof(double) * (size_t)d_out);
+  double* P = (double*)calloc((size_t)N, sizeof(double));
+  double L = 0.0;
+  for (int64_t t = 0; t < T; ++t) {
+    or_token_weights(N, d_in, k, renorm, Wr, z ? z + t * N : NULL, u + t * d_in, top_idx + t * k,
+                     zt, pt, at);
+    for (int64_t i = 0; i < N; ++i) P[i] += pt[i];
+    for (int64_t m = 0; m < d_out; ++m) yt[m] = 0.0;
+    for (int64_t s = 0; s < k; ++s) {
+      if (row_of && row_of[t * k + s] < 0) continue;
+      int32_t e = top_idx[t * k + s];
+      or_expert(&Wg[e], &Wu[e], &Wd[e], u + t * d_in, act, beta_g, beta_u, 0, F);
+      for (int64_t m = 0; m < d_out; ++m) yt[m] += at[s] * F[m];
+    }
+    for (int64_t m = 0; m < d_out; ++m) L += dy[t * d_out + m] * yt[m];
+    if (y)
+      for (int64_t m = 0; m < d_out; ++m) y[t * d_out + m] = yt[m];
+  }
+  if (f) {
+    double acc = 0.0;
+    for (int64_t i = 0; i < N; ++i) acc += f[i] * (P[i] / (double)T);
+    L += alpha * (double)N * acc;
+  }
+  free(zt);
+  free(pt);
+  free(at);
+  free(F);
+  free(yt);
+  free(P);
+  return L;
+}
+
+static inline double sigmoid(double x) { return 1.0 / (1.0 + exp(-x)); }
+
+/* Backward of one expert evaluation F(u) = W_down (SiLU(g') (*) v'),
+ * g = W_gate u, v = W_up u, g' = g and v' = v (act = 0) or the soft caps
+ * beta tanh(x / beta) of [LatentMoE] (act = 1).  Given dF = dL/dF [d_out]:
+ *   dH = W_down^T dF,            dW_down += dF H^T
+ *   dg' = dH (*) v' (*) SiLU'(g'), SiLU'(x) = s(x) (1 + x (1 - s(x))), s = sigmoid
+ *   dv' = dH (*) SiLU(g')
+ *   dg = dg' (1 - tanh^2(g / beta_g)) under the cap, else dg'; the same for v
+ *   dW_gate += dg u^T, dW_up += dv u^T, du += W_gate^T dg + W_up^T dv.
+ * F(u) is returned in out.  Accumulators: dWg, dWu [h][d_in], dWd [d_out][h],
+ * du [d_in]. */
+static void or_expert_backward(const or_mat* Wg, const or_mat* Wu, const or_mat* Wd,
+                               const double* u, int act, double beta_g, double beta_u,
+                               const double* dF, double* out, double* dWg, double* dWu,
+                               double* dWd, double* du) {
+  int64_t h = Wg->rows, d_in = Wg->cols, d_out = Wd->rows;
+  double* g = (double*)malloc(sizeof(double) * (size_t)h);
+  double* v = (double*)malloc(sizeof(double) * (size_t)h);
+  double* H = (double*)malloc(sizeof(double) * (size_t)h);
+  double* dH = (double*)malloc(sizeof(double) * (size_t)h);
+  or_matvec(Wg, u, g);
+  or_matvec(Wu, u, v);
+  for (int64_t i = 0; i < h; ++i) {
+    double gc = act == 1 ? beta_g * tanh(g[i] / beta_g) : g[i];
+    double vc = act == 1 ? beta_u * tanh(v[i] / beta_u) : v[i];
+    H[i] = silu(gc) * vc;
+  }
+  or_matvec(Wd, H, out);
+  for (int64_t i = 0; i < h; ++i) {
+    double acc = 0.0;
+    for (int64_t m = 0; m < d_out; ++m) acc += mat_get(Wd, m, i) * dF[m];
+    dH[i] = acc;
+  }
+  for (int64_t m = 0; m < d_out; ++m)
+    for (int64_t i = 0; i < h; ++i) dWd[m * h + i] += dF[m] * H[i];
+  for (int64_t i = 0; i < h; ++i) {
+    double gc = g[i], vc = v[i], jg = 1.0, jv = 1.0;
+    if (act == 1) {
+      double tg = tanh(g[i] / beta_g), tv = tanh(v[i] / beta_u);
+      gc = beta_g * tg;
+      vc = beta_u * tv;
+      jg = 1.0 - tg * tg;
+      jv = 1.0 - tv * tv;
+    }
+    double sg = sigmoid(gc);
+    double dg = dH[i] * vc * (sg * (1.0 + gc * (1.0 - sg))) * jg;
+    double dv = dH[i] * silu(gc) * jv;
+    for (int64_t c = 0; c < d_in; ++c) {
+      dWg[i * d_in + c] += dg * u[c];
+      dWu[i * d_in + c] += dv * u[c];
+      du[c] += mat_get(Wg, i, c) * dg + mat_get(Wu, i, c) * dv;
+    }
+  }
+  free(g);
+  free(v);
+  free(H);
+  free(dH);
+}
+
+/* dL/d(everything) for L of or_layer_loss, with the same inputs.
+ * Per token t (a_s, p from or_token_weights):
+ *   kept slot s, expert e:  da_s = dy_t . F_e(u_t); the expert backward with
+ *                           dF = a_s dy_t adds to dW*_e and du_t
+ *   dropped slot:           da_s = 0 (it contributes nothing to y_t)
+ *   renorm:                 dp_{e_s} = (da_s - sum_r a_r da_r) / sum_r p_{e_r}
+ *   no renorm:              dp_{e_s} = da_s;  dp_i = 0 outside the selected set
+ *   softmax:                dz_j = p_j (dp_j - sum_i p_i dp_i)
+ *   balancing term:         dz_j += (alpha N / T) p_j (f_j - sum_i f_i p_i)  (§3.7)
+ *   router (Wr given):      dWr_j += dz_j u_t,  du_t += sum_j dz_j Wr_j
+ * Outputs (fully overwritten): dz [T][N], du [T][d_in], dWr [N][d_in] (only
+ * when Wr is given; may be NULL), dWg, dWu [N][h][d_in], dWd [N][d_out][h]. */
+void or_layer_backward(int64_t T, int64_t N, int64_t k, int renorm, const or_mat* Wg,
+                       const or_mat* Wu, const or_mat* Wd, int act, double beta_g,
+                       double beta_u, const double* Wr, const double* z, const double* u,
+                       int64_t d_in, const int32_t* top_idx, const int32_t* row_of,
+                       const double* dy, double alpha, const double* f, double* dz, double* du,
+                       double* dWr, double* dWg, double* dWu, double* dWd) {
+  int64_t h = Wg[0].rows, d_out = Wd[0].rows;
+  memset(du, 0, sizeof(double) * (size_t)(T * d_in));
+  memset(dWg, 0, sizeof(double) * (size_t)(N * h * d_in));
+  memset(dWu, 0, sizeof(double) * (size_t)(N * h * d_in));
+  memset(dWd, 0, sizeof(double) * (size_t)(N * d_out * h));
+  if (Wr && dWr) memset(dWr, 0, sizeof(double) * (size_t)(N * d_in));
+  double* zt = (double*)malloc(sizeof(double) * (size_t)N);
+  double* pt = (double*)malloc(sizeof(double) * (size_t)N);
+  double* dp = (double*)malloc(sizeof(double) * (size_t)N);
+  double* at = (double*)malloc(sizeof(double) * (size_t)k);
+  double* da = (double*)malloc(sizeof(double) * (size_t)k);
+  double* dF = (double*)malloc(sizeof(double) * (size_t)d_out);
+  double* F = (double*)malloc(sizeof(double) * (size_t)d_out);
+  for (int64_t t = 0; t < T; ++t) {
+    const double* ut = u + t * d_in;
+    const double* dyt = dy + t * d_out;
+    const int32_t* sel = top_idx + t * k;
+    double* dut = du + t * d_in;
+    double* dzt = dz + t * N;
+    or_token_weights(N, d_in, k, renorm, Wr, z ? z + t * N : NULL, ut, sel, zt, pt, at);
+    for (int64_t s = 0; s < k; ++s) {
+      da[s] = 0.0;
+      if (row_of && row_of[t * k + s] < 0) continue;
+      int32_t e = sel[s];
+      for (int64_t m = 0; m < d_out; ++m) dF[m] = at[s] * dyt[m];
+      or_expert_backward(&Wg[e], &Wu[e], &Wd[e], ut, act, beta_g, beta_u, dF, F,
+                         dWg + (int64_t)e * h * d_in, dWu + (int64_t)e * h * d_in,
+                         dWd + (int64_t)e * d_out * h, dut);
+      double acc = 0.0;
+      for (int64_t m = 0; m < d_out; ++m) acc += dyt[m] * F[m];
+      da[s] = acc;
+    }
+    for (int64_t i = 0; i < N; ++i) dp[i] = 0.0;
+    if (renorm) {
+      double ssum = 0.0, ada = 0.0;
+      for (int64_t s = 0; s < k; ++s) {
+        ssum += pt[sel[s]];
+        ada += at[s] * da[s];
+      }
+      for (int64_t s = 0; s < k; ++s) dp[sel[s]] = (da[s] - ada) / ssum;
+    } else {
+      for (int64_t s = 0; s < k; ++s) dp[sel[s]] = da[s];
+    }
+    double pdp = 0.0;
+    for (int64_t i = 0; i < N; ++i) pdp += pt[i] * dp[i];
+    for (int64_t j = 0; j < N; ++j) dzt[j] = pt[j] * (dp[j] - pdp);
+    if (f) {
+      const double c = alpha * (double)N / (double)T;
+      double fbar = 0.0;
+      for (int64_t i = 0; i < N; ++i) fbar += f[i] * pt[i];
+      for (int64_t j = 0; j < N; ++j) dzt[j] += c * pt[j] * (f[j] - fbar);
+    }
+    if (Wr) {
+      for (int64_t j = 0; j < N; ++j) {
+        for (int64_t c = 0; c < d_in; ++c) {
+          if (dWr) dWr[j * d_in + c] += dzt[j] * ut[c];
+          dut[c] += dzt[j] * Wr[j * d_in + c];
+        }
+      }
+    }
+  }
+  free(zt);
+  free(pt);
+  free(dp);
+  free(at);
+  free(da);
+  free(dF);
+  free(F);
 }
