@@ -244,14 +244,14 @@ extern "C" int moe_quantile_balance(int32_t T, int32_t N, int32_t k, const float
   else MOE_QB_CUT(32);
 #undef MOE_QB_CUT
   const size_t smem = select_smem(T, bias_hist ? bins : 0);
-  static bool configured[64] = {false};
+  static std::atomic<bool> configured[kMaxDevices];
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !configured[dev]) {
+  if (needs_setup(configured, dev)) {
     if (cudaFuncSetAttribute(qb_select, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)select_smem(kQBMaxT, kQBMaxBins)) != cudaSuccess)
       return MOE_ERR_CUDA;
-    configured[dev] = true;
+    mark_setup(configured, dev);
   }
   MOE_PREFER_SHARED((qb_select));
   launch_pdl(qb_select, dim3((unsigned)N), dim3(kQBThreads), smem, st, scores,

@@ -8,9 +8,28 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "../../include/moe.h"
 
 namespace moe {
+
+// ------------------------------------------------------- per-device caches
+// Host-side values set up lazily once per device index (kernel attributes, SM
+// counts, symbol addresses) live in static arrays of atomics, so host threads
+// that make their first calls at the same time do not race.  Every such setup
+// is idempotent, so two threads doing it once each is harmless.
+constexpr int kMaxDevices = 64;
+
+inline bool device_slot(int dev) { return dev >= 0 && dev < kMaxDevices; }
+
+// True while the once-per-device setup guarded by `done` has not run on dev.
+inline bool needs_setup(const std::atomic<bool>* done, int dev) {
+  return device_slot(dev) && !done[dev].load(std::memory_order_acquire);
+}
+inline void mark_setup(std::atomic<bool>* done, int dev) {
+  done[dev].store(true, std::memory_order_release);
+}
 
 // ------------------------------------------------------------- device status
 // The sticky status word lives in status.cu; kernels receive its address as an
@@ -142,13 +161,12 @@ inline int launch_status() {
 // call site.
 #define MOE_PREFER_SHARED(kernel)                                                      \
   do {                                                                                 \
-    static bool moe_done_[64] = {false};                                               \
+    static std::atomic<bool> moe_done_[::moe::kMaxDevices];                            \
     int moe_dev_ = 0;                                                                  \
-    if (cudaGetDevice(&moe_dev_) == cudaSuccess && moe_dev_ >= 0 && moe_dev_ < 64 &&   \
-        !moe_done_[moe_dev_]) {                                                        \
+    if (cudaGetDevice(&moe_dev_) == cudaSuccess && ::moe::needs_setup(moe_done_, moe_dev_)) { \
       cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,     \
                            (int)cudaSharedmemCarveoutMaxShared);                       \
-      moe_done_[moe_dev_] = true;                                                      \
+      ::moe::mark_setup(moe_done_, moe_dev_);                                          \
     }                                                                                  \
   } while (0)
 

@@ -679,27 +679,24 @@ WsLayout carve_decode(const moe_shape& s, void* base) {
   return L;
 }
 
-struct DeviceInfo {
-  int sms = 0;
-  bool configured = false;
-};
-
 // SM count of the current device; the kernel's shared-memory limit is raised
 // once per device.
 bool device_info(int* sms) {
-  static DeviceInfo info[64];
+  static std::atomic<int> sm_count[kMaxDevices];
+  static std::atomic<bool> configured[kMaxDevices];
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
-  DeviceInfo& di = info[dev];
-  if (!di.configured) {
-    if (cudaDeviceGetAttribute(&di.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+  if (cudaGetDevice(&dev) != cudaSuccess || !device_slot(dev)) return false;
+  if (needs_setup(configured, dev)) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
         cudaFuncSetAttribute(decode_persistent, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)kSmemLimit) != cudaSuccess)
       return false;
     MOE_PREFER_SHARED((decode_persistent));
-    di.configured = true;
+    sm_count[dev].store(n, std::memory_order_relaxed);
+    mark_setup(configured, dev);
   }
-  *sms = di.sms;
+  *sms = sm_count[dev].load(std::memory_order_relaxed);
   return true;
 }
 

@@ -410,29 +410,30 @@ bool make_tmap(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, u
 }
 
 int sm_count() {
-  static int cached[64] = {0};
+  static std::atomic<int> cached[kMaxDevices];
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev < 0 || dev >= 64) return 148;
-  if (!cached[dev]) {
-    int n = 0;
+  if (!device_slot(dev)) return 148;
+  int n = cached[dev].load(std::memory_order_relaxed);
+  if (!n) {
     cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    cached[dev] = n > 0 ? n : 148;
+    if (n <= 0) n = 148;
+    cached[dev].store(n, std::memory_order_relaxed);
   }
-  return cached[dev];
+  return n;
 }
 
 template <int BN, int S, int ACT>
 int launch_tc(const TcParams& p, int64_t tiles_upper, cudaStream_t st) {
   const size_t smem = Layout<BN, S>::bytes(p.G);
-  static bool configured[64] = {false};
+  static std::atomic<bool> configured[kMaxDevices];
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !configured[dev]) {
+  if (needs_setup(configured, dev)) {
     if (cudaFuncSetAttribute(tc_grouped_gemm<BN, S, ACT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)Layout<BN, S>::bytes(1024)) != cudaSuccess)
       return MOE_ERR_CUDA;
-    configured[dev] = true;
+    mark_setup(configured, dev);
   }
   int64_t grid = sm_count();
   if (tiles_upper < grid) grid = tiles_upper;

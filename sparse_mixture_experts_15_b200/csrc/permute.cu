@@ -353,15 +353,17 @@ namespace {
 // per device with that device current (in host code the array's name is only a
 // host-side stand-in and must not be handed to a kernel).
 int32_t* noalloc_scratch() {
-  static int32_t* addr[64] = {nullptr};
+  static std::atomic<int32_t*> addr[kMaxDevices];
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-  if (!addr[dev]) {
+  if (cudaGetDevice(&dev) != cudaSuccess || !device_slot(dev)) return nullptr;
+  int32_t* a = addr[dev].load(std::memory_order_acquire);
+  if (!a) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_permute_noalloc_scratch) != cudaSuccess) return nullptr;
-    addr[dev] = static_cast<int32_t*>(p);
+    a = static_cast<int32_t*>(p);
+    addr[dev].store(a, std::memory_order_release);
   }
-  return addr[dev];
+  return a;
 }
 
 }  // namespace

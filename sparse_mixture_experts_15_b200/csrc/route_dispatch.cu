@@ -315,14 +315,14 @@ int launch_route_dispatch(const moe_shape& s, const void* u, int32_t dtype, cons
                           float* logits, int32_t* counts, int32_t* offsets, int32_t* perm_tok,
                           int32_t* row_of, int32_t* overflow, int32_t* totals, void* x_rows,
                           void* ws, cudaStream_t st) {
-  static bool configured[64] = {false};
+  static std::atomic<bool> configured[kMaxDevices];
   int dev = 0, sms = 0;
   if (cudaGetDevice(&dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
     return MOE_ERR_CUDA;
   RDParams p{};
   if (!make_rd_plan(s, dtype, sms, &p.plan)) return MOE_ERR_UNSUPPORTED;
-  if (dev >= 0 && dev < 64 && !configured[dev]) {
+  if (needs_setup(configured, dev)) {
     const int lim = (int)kRDSmemLimit;
     MOE_PREFER_SHARED((route_dispatch<8, float>));
     MOE_PREFER_SHARED((route_dispatch<16, float>));
@@ -337,7 +337,7 @@ int launch_route_dispatch(const moe_shape& s, const void* u, int32_t dtype, cons
         cudaFuncSetAttribute(route_dispatch<16, __nv_bfloat16>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, lim) != cudaSuccess)
       return MOE_ERR_CUDA;
-    configured[dev] = true;
+    mark_setup(configured, dev);
   }
   p.u = u;
   p.w_route = w_route;

@@ -9,15 +9,17 @@ __device__ int g_status_word = 0;
 
 int* status_word() {
   // One address per device, looked up once with that device current.
-  static int* addr[64] = {nullptr};
+  static std::atomic<int*> addr[kMaxDevices];
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-  if (!addr[dev]) {
+  if (cudaGetDevice(&dev) != cudaSuccess || !device_slot(dev)) return nullptr;
+  int* a = addr[dev].load(std::memory_order_acquire);
+  if (!a) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess) return nullptr;
-    addr[dev] = static_cast<int*>(p);
+    a = static_cast<int*>(p);
+    addr[dev].store(a, std::memory_order_release);
   }
-  return addr[dev];
+  return a;
 }
 
 }  // namespace moe
