@@ -420,10 +420,10 @@ int launch_ffn_fused(int G, int64_t R, int width, int h, const __nv_bfloat16* x_
   p.beta_u = act.beta_up;
   p.y_rows = y_rows;
   p.status = status_word();
-  static std::atomic<bool> configured[kMaxDevices];
+  static bool configured[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
-  if (needs_setup(configured, dev)) {
+  if (dev >= 0 && dev < 64 && !configured[dev]) {
     if (cudaFuncSetAttribute(tc_fused_ffn<MOE_ACT_SWIGLU>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)fSmemLimit) != cudaSuccess ||
@@ -431,7 +431,7 @@ int launch_ffn_fused(int G, int64_t R, int width, int h, const __nv_bfloat16* x_
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)fSmemLimit) != cudaSuccess)
       return MOE_ERR_CUDA;
-    mark_setup(configured, dev);
+    configured[dev] = true;
   }
   int sms = 0;
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
