@@ -18,7 +18,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 SO = os.path.join(_HERE, "_moe_oracle.so")
 SRC = os.path.join(_HERE, "moe_oracle.c")
 
-F32, BF16, F16, Q4_0, F64 = 0, 1, 2, 3, 4
+F32, BF16, F16, Q4_0, F64, E4M3 = 0, 1, 2, 3, 4, 5
 
 
 def build(force: bool = False) -> str:
@@ -31,7 +31,8 @@ def build(force: bool = False) -> str:
 
 class OrMat(ctypes.Structure):
     _fields_ = [("dtype", ctypes.c_int), ("rows", ctypes.c_int64), ("cols", ctypes.c_int64),
-                ("data", ctypes.c_void_p), ("qs", ctypes.c_void_p), ("scales", ctypes.c_void_p)]
+                ("data", ctypes.c_void_p), ("qs", ctypes.c_void_p), ("scales", ctypes.c_void_p),
+                ("row_scale", ctypes.c_void_p)]
 
 
 _lib = None
@@ -77,6 +78,12 @@ def lib():
         L.or_qb_exact.argtypes = [i64, i64, vp, vp, i64, vp, vp]
         L.or_qb_hist.argtypes = [i64, i64, vp, vp, i64, i64, vp]
         L.or_aux_grad.argtypes = [i64, i64, dbl, vp, vp, vp]
+        L.or_e4m3_to_f64.argtypes = [ctypes.c_uint8]
+        L.or_e4m3_to_f64.restype = dbl
+        L.or_round_e4m3.argtypes = [dbl]
+        L.or_round_e4m3.restype = ctypes.c_uint8
+        L.or_quant_e4m3_rows.argtypes = [i64, i64, vp, vp, vp]
+        L.or_quant_e4m3_rows.restype = None
         L.or_layer_loss.argtypes = [i64, i64, i64, ctypes.c_int, vp, vp, vp, ctypes.c_int, dbl,
                                     dbl, vp, vp, vp, i64, vp, vp, vp, dbl, vp, vp]
         L.or_layer_loss.restype = dbl
@@ -107,17 +114,21 @@ class Mat:
 
     def __init__(self, dtype, rows, cols, data=None, qs=None, scales=None):
         self.dtype, self.rows, self.cols = dtype, rows, cols
+        self.row_scale = None
         if dtype == F32:
             self.data = _c(data, np.float32)
         elif dtype == F64:
             self.data = _c(data, np.float64)
         elif dtype in (BF16, F16):
             self.data = _c(data, np.uint16)
+        elif dtype == E4M3:  # data: uint8 codes [rows][cols]; scales: fp32 per row
+            self.data, self.row_scale = _c(data, np.uint8), _c(scales, np.float32)
         else:
             self.qs, self.scales, self.data = _c(qs, np.uint8), _c(scales, np.uint16), None
         self.s = OrMat(dtype, rows, cols, _p(self.data),
                        _p(getattr(self, "qs", None)) if dtype == Q4_0 else None,
-                       _p(getattr(self, "scales", None)) if dtype == Q4_0 else None)
+                       _p(getattr(self, "scales", None)) if dtype == Q4_0 else None,
+                       _p(self.row_scale))
 
     def decode(self):
         out = np.empty((self.rows, self.cols), dtype=np.float64)
@@ -150,29 +161,64 @@ def round_bf16_array(x) -> np.ndarray:
 
 
 def latent_tokens(x_codes, w_route, k, W_dp, get_expert, W_upp, shared, beta_g, beta_u, eps,
-                  renorm=1, bias=None):
+                  renorm=1, bias=None, fp8=False):
     """LatentMoE forward for the given token rows (Stable LatentMoE demo document:
     width separation, RMSNorm before the up-projection, SiTU-GLU soft caps):
       routing on the full-width x; x_l = bf16(W_dp x); m = sum_s a_s E_s(x_l) with
       the soft-capped routed experts (hidden stored as bf16);
       m^ = bf16(m / sqrt(mean m^2 + eps)); y = W_upp m^ + sum_j S_j(x) (plain SwiGLU).
     get_expert(e) returns the (gate, up, down) matrices of routed expert e.
+    fp8=True is the FP8 form of the routed experts: their matrices are E4M3
+    with a scale per row, x_l is quantised to E4M3 with a scale per token
+    (quant_e4m3_rows) and H is rounded to E4M3 with no scale.
     Returns (top_idx, top_w, y in float64)."""
     x = decode(BF16, x_codes)
     _, _, idx, tw = route(x.astype(np.float32), w_route, k, renorm, bias)
     y = np.zeros((x.shape[0], W_upp.rows))
     for t in range(x.shape[0]):
         xl = round_bf16_array(matvec(W_dp, x[t]))
+        if fp8:
+            xc, xs = quant_e4m3_rows(xl)
+            xl = e4m3_mat(xc, xs).decode()[0]
         m = np.zeros(W_dp.rows)
         for s_ in range(k):
             g, u, d = get_expert(int(idx[t, s_]))
-            m += tw[t, s_] * expert(g, u, d, xl, act=1, beta_g=beta_g, beta_u=beta_u, round_h=1)
+            m += tw[t, s_] * expert(g, u, d, xl, act=1, beta_g=beta_g, beta_u=beta_u,
+                                    round_h=2 if fp8 else 1)
         mh = round_bf16_array(rmsnorm(m, eps))
         yt = matvec(W_upp, mh)
         for (g, u, d) in shared:
             yt = yt + expert(g, u, d, x[t], act=0, round_h=1)
         y[t] = yt
     return idx, tw, y
+
+
+def e4m3_to_f64(code: int) -> float:
+    return lib().or_e4m3_to_f64(int(code))
+
+
+def round_e4m3(x) -> np.ndarray:
+    """Nearest FP8 E4M3 codes (uint8) of float64 values, ties to even, saturating at 448."""
+    x = np.asarray(x, np.float64)
+    out = np.array([lib().or_round_e4m3(float(v)) for v in x.ravel()], np.uint8)
+    return out.reshape(x.shape)
+
+
+def quant_e4m3_rows(x):
+    """(codes uint8 [rows][cols], scales fp32 [rows]): per row s = amax / 448,
+    codes = nearest E4M3 of the fp32 quotient x / s."""
+    x = _c(np.atleast_2d(x), np.float32)
+    rows, cols = x.shape
+    codes = np.empty((rows, cols), np.uint8)
+    scales = np.empty(rows, np.float32)
+    lib().or_quant_e4m3_rows(rows, cols, x.ctypes.data, codes.ctypes.data, scales.ctypes.data)
+    return codes, scales
+
+
+def e4m3_mat(codes, scales):
+    """An E4M3 matrix with one fp32 scale per row."""
+    codes = np.atleast_2d(codes)
+    return Mat(E4M3, codes.shape[0], codes.shape[1], data=codes, scales=scales)
 
 
 def round_f16(x) -> np.ndarray:

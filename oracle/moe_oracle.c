@@ -66,7 +66,61 @@ double or_f16_to_f64(uint16_t h) {
 }
 
 /* Storage of an activation or weight tensor. */
-enum { OR_F32 = 0, OR_BF16 = 1, OR_F16 = 2, OR_Q4_0 = 3, OR_F64 = 4 };
+enum { OR_F32 = 0, OR_BF16 = 1, OR_F16 = 2, OR_Q4_0 = 3, OR_F64 = 4, OR_E4M3 = 5 };
+
+/* FP8 E4M3 code -> exact double.  The OCP "e4m3fn" layout: sign, 4 exponent
+ * bits (bias 7), 3 mantissa bits; exponent field 0 holds the subnormals
+ * m * 2^-9; S.1111.111 is NaN; there is no infinity and the largest finite
+ * value is 1.75 * 2^8 = 448, the limit [LatentMoE] compares the SiTU-GLU
+ * product bound with. */
+double or_e4m3_to_f64(uint8_t c) {
+  int sign = c >> 7, ex = (c >> 3) & 0xF, man = c & 7;
+  double v;
+  if (ex == 15 && man == 7) return NAN;
+  if (ex == 0) {
+    v = ldexp((double)man, -9);
+  } else {
+    v = ldexp((double)(8 + man), ex - 10);
+  }
+  return sign ? -v : v;
+}
+
+/* Nearest E4M3 code to x, ties to the even code (even mantissa), by search
+ * over the 127 finite magnitudes; magnitudes above 448 give 448 (saturation,
+ * the "satfinite" conversion), NaN gives the NaN code, the sign of x (also
+ * of a zero result) is kept. */
+uint8_t or_round_e4m3(double x) {
+  if (isnan(x)) return 0x7F;
+  uint8_t sign = signbit(x) ? 0x80 : 0x00;
+  double a = fabs(x), bd = INFINITY;
+  int best = 0;
+  for (int c = 0; c <= 0x7E; ++c) {
+    double dist = fabs(or_e4m3_to_f64((uint8_t)c) - a);
+    if (dist < bd || (dist == bd && (c & 1) == 0)) {
+      bd = dist;
+      best = c;
+    }
+  }
+  return (uint8_t)(sign | best);
+}
+
+/* Row-wise E4M3 quantisation of an fp32 [rows][cols] matrix: per row
+ * s = amax / 448 (one fp32 division; s = 1 for an all-zero row) and
+ * code = nearest E4M3 of the fp32 quotient x / s, so that s * e4m3(code)
+ * approximates x and the row's largest magnitude maps to +-448. */
+void or_quant_e4m3_rows(int64_t rows, int64_t cols, const float* x, uint8_t* codes,
+                        float* scales) {
+  for (int64_t r = 0; r < rows; ++r) {
+    float amax = 0.0f;
+    for (int64_t c = 0; c < cols; ++c) amax = fmaxf(amax, fabsf(x[r * cols + c]));
+    const float s = amax > 0.0f ? amax / 448.0f : 1.0f;
+    scales[r] = s;
+    for (int64_t c = 0; c < cols; ++c) {
+      const float q = x[r * cols + c] / s;
+      codes[r * cols + c] = or_round_e4m3((double)q);
+    }
+  }
+}
 
 /* One [rows][cols] matrix in any storage type.  q4_0 (format named in
  * [MCU #13] §4): blocks of 32 consecutive values along a row, one fp16 scale
@@ -79,6 +133,7 @@ typedef struct {
   const void* data;       /* f32 / bf16 / f16 / f64 */
   const uint8_t* qs;      /* q4_0: [rows][cols/2] */
   const uint16_t* scales; /* q4_0: [rows][cols/32] fp16 codes */
+  const float* row_scale; /* e4m3: [rows] fp32, value = row_scale[r] * e4m3(data[r][c]) */
 } or_mat;
 
 static inline double mat_get(const or_mat* m, int64_t r, int64_t c) {
@@ -87,6 +142,8 @@ static inline double mat_get(const or_mat* m, int64_t r, int64_t c) {
     case OR_BF16: return or_bf16_to_f64(((const uint16_t*)m->data)[r * m->cols + c]);
     case OR_F16: return or_f16_to_f64(((const uint16_t*)m->data)[r * m->cols + c]);
     case OR_F64: return ((const double*)m->data)[r * m->cols + c];
+    case OR_E4M3:
+      return (double)m->row_scale[r] * or_e4m3_to_f64(((const uint8_t*)m->data)[r * m->cols + c]);
     default: {
       int64_t b = c / 32, j = c % 32;
       uint8_t byte = m->qs[r * (m->cols / 2) + b * 16 + (j & 15)];
@@ -310,7 +367,9 @@ static inline double silu(double g) { return g / (1.0 + exp(-g)); }
  * act = 1 applies the SiTU-GLU soft caps of [LatentMoE]: the gate and up
  * pre-activations become beta_g tanh(g / beta_g) and beta_u tanh(u / beta_u)
  * before SiLU and the product.  round_h = 1 rounds the hidden vector to bf16
- * (the storage of the intermediate in the bf16 layers).  W_gate, W_up:
+ * (the storage of the intermediate in the bf16 layers), round_h = 2 to FP8
+ * E4M3 with no scale (the FP8 experts: the soft caps keep |H| below
+ * beta_g * beta_u = 100 < 448, so H needs no per-row scale).  W_gate, W_up:
  * [h][d_in]; W_down: [d_out][h]. */
 void or_expert(const or_mat* Wg, const or_mat* Wu, const or_mat* Wd, const double* u, int act,
                double beta_g, double beta_u, int round_h, double* out) {
@@ -326,7 +385,9 @@ void or_expert(const or_mat* Wg, const or_mat* Wu, const or_mat* Wd, const doubl
       ui = beta_u * tanh(ui / beta_u);
     }
     double hi = silu(gi) * ui;
-    g[i] = round_h ? or_round_bf16(hi) : hi;
+    g[i] = round_h == 1 ? or_round_bf16(hi)
+           : round_h == 2 ? or_e4m3_to_f64(or_round_e4m3(hi))
+                          : hi;
   }
   or_matvec(Wd, g, out);
   free(g);
