@@ -111,7 +111,17 @@ def _check(rc: int, where: str):
 
 
 def _ptr(t):
-    return None if t is None else t.data_ptr()
+    """Device address of a tensor the library reads or writes (None -> NULL).
+    The kernels take every tensor as a dense row-major array in device
+    memory, so a host tensor or a strided view is refused here, before any
+    call: its address would point the kernels at the wrong memory."""
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError(f"expected a CUDA tensor, got a tensor on {t.device}")
+    if not t.is_contiguous():
+        raise ValueError(f"expected a contiguous tensor, got strides {tuple(t.stride())}")
+    return t.data_ptr()
 
 
 def _stream(stream):

@@ -141,3 +141,18 @@ def test_aux_grad_host_checks():
     assert lib.moe_aux_grad(10, 0, 1.0, 4096, 4096, 4096, None) == -1
     assert lib.moe_aux_grad(10, 8, 1.0, None, 4096, 4096, None) == -1
     assert lib.moe_aux_grad(0, 8, 1.0, None, None, None, None) == 0  # empty batch: no-op
+
+
+def test_binding_refuses_host_tensors_before_the_call():
+    """A host tensor's address handed to a kernel would be read as device
+    memory; the binding refuses it before calling into the library."""
+    import torch
+    s = moe.shape(16, 64, 4, 2, 128)
+    u = torch.zeros((16, 64), dtype=torch.bfloat16)
+    perm = torch.zeros(32, dtype=torch.int32)
+    offsets = torch.zeros(5, dtype=torch.int32)
+    x_rows = torch.zeros((32, 64), dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        moe.moe_gather(s, 64, u, perm, offsets, x_rows)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        moe.q4_layer(torch.zeros((4, 64)), *[torch.zeros(8, dtype=torch.uint8)] * 6)
