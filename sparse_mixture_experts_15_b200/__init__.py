@@ -124,6 +124,25 @@ def _ptr(t):
     return t.data_ptr()
 
 
+def _need(what, t, n):
+    """Refuse a tensor with fewer than n elements where the call touches n.
+    The library sees only the address, so a short tensor would be read or
+    written past its end on the device."""
+    if t is not None and t.numel() < n:
+        raise ValueError(f"{what}: {t.numel()} elements, the call needs at least {n}")
+
+
+def _outputs(s: MoeShape, outputs):
+    """moe_layer_outputs from a dict of tensors, each checked against its
+    documented size."""
+    Tk, TN, N = s.T * s.k, s.T * s.N, s.N
+    sizes = dict(top_idx=Tk, top_w=Tk, probs=TN, counts=N, offsets=N + 1, perm_tok=Tk,
+                 row_of=Tk, overflow=N, totals=3, f=N, P=N, n_sum_fP=1)
+    for key, t in (outputs or {}).items():
+        _need(key, t, sizes[key])
+    return MoeLayerOutputs(**{key: _ptr(t) for key, t in (outputs or {}).items()})
+
+
 def _stream(stream):
     if stream is None:
         import torch
@@ -163,6 +182,10 @@ def moe_capacity(T: int, N: int, k: int, factor: float) -> int:
 
 def moe_route(s: MoeShape, u, w_route, top_idx, top_w, bias=None, probs=None, logits=None,
               ws=None, stream=None):
+    for what, t, n in (("u", u, s.T * s.d), ("w_route", w_route, s.N * s.d), ("bias", bias, s.N),
+                       ("top_idx", top_idx, s.T * s.k), ("top_w", top_w, s.T * s.k),
+                       ("probs", probs, s.T * s.N), ("logits", logits, s.T * s.N)):
+        _need(what, t, n)
     nb = _lib.moe_route_workspace_bytes(ctypes.byref(s))
     wbuf, wlen = (None, 0) if logits is not None else _ws(nb, u.device, ws)
     _check(_lib.moe_route(ctypes.byref(s), _ptr(u), _dtype_code(u), _ptr(w_route), _ptr(bias),
@@ -174,14 +197,26 @@ def moe_aux_stats(probs, top_idx, f=None, P=None, n_sum_fP=None, loads=None, ws=
                   stream=None):
     T, k = top_idx.shape
     N = f.shape[0] if f is not None else (P.shape[0] if P is not None else loads.shape[0])
+    for what, t, n in (("probs", probs, T * N), ("f", f, N), ("P", P, N), ("n_sum_fP", n_sum_fP, 1),
+                       ("loads", loads, N)):
+        _need(what, t, n)
     wbuf, wlen = _ws(_lib.moe_aux_stats_workspace_bytes(N), top_idx.device, ws)
     _check(_lib.moe_aux_stats(T, N, k, _ptr(probs), _ptr(top_idx), _ptr(f), _ptr(P),
                               _ptr(n_sum_fP), _ptr(loads), _ptr(wbuf), wlen, _stream(stream)),
            "moe_aux_stats")
 
 
+def _permute_sizes(s, top_idx, counts, offsets, perm_tok, row_of, overflow, totals):
+    Tk = s.T * s.k
+    for what, t, n in (("top_idx", top_idx, Tk), ("counts", counts, s.N),
+                       ("offsets", offsets, s.N + 1), ("perm_tok", perm_tok, Tk),
+                       ("row_of", row_of, Tk), ("overflow", overflow, s.N), ("totals", totals, 3)):
+        _need(what, t, n)
+
+
 def moe_permute(s: MoeShape, top_idx, counts, offsets, perm_tok, row_of, overflow, totals,
                 ws=None, stream=None):
+    _permute_sizes(s, top_idx, counts, offsets, perm_tok, row_of, overflow, totals)
     wbuf, wlen = _ws(_lib.moe_permute_workspace_bytes(ctypes.byref(s)), top_idx.device, ws)
     _check(_lib.moe_permute(ctypes.byref(s), _ptr(top_idx), _ptr(counts), _ptr(offsets),
                             _ptr(perm_tok), _ptr(row_of), _ptr(overflow), _ptr(totals), _ptr(wbuf),
@@ -191,12 +226,18 @@ def moe_permute(s: MoeShape, top_idx, counts, offsets, perm_tok, row_of, overflo
 def moe_permute_noalloc(s: MoeShape, top_idx, counts, offsets, perm_tok, row_of, overflow,
                         totals, stream=None):
     """moe_permute without a workspace (the library's fixed 1 MiB scratch)."""
+    _permute_sizes(s, top_idx, counts, offsets, perm_tok, row_of, overflow, totals)
     _check(_lib.moe_permute_noalloc(ctypes.byref(s), _ptr(top_idx), _ptr(counts), _ptr(offsets),
                                     _ptr(perm_tok), _ptr(row_of), _ptr(overflow), _ptr(totals),
                                     _stream(stream)), "moe_permute_noalloc")
 
 
 def moe_gather(s: MoeShape, width: int, u, perm_tok, offsets, x_rows, stream=None):
+    """perm_tok is read for the offsets[N] grouped rows only, a count the
+    device holds, so its size is not checked here."""
+    _need("u", u, s.T * width)
+    _need("offsets", offsets, s.N + 1)
+    _need("x_rows", x_rows, s.T * s.k * width)
     _check(_lib.moe_gather(ctypes.byref(s), width, _ptr(u), _dtype_code(u), _ptr(perm_tok),
                            _ptr(offsets), _ptr(x_rows), _stream(stream)), "moe_gather")
 
@@ -204,6 +245,11 @@ def moe_gather(s: MoeShape, width: int, u, perm_tok, offsets, x_rows, stream=Non
 def moe_expert_ffn(s: MoeShape, width: int, x_rows, offsets, w_gate, w_up, w_down, y_rows,
                    a: MoeAct | None = None, ws=None, stream=None):
     a = a or act()
+    rows = s.T * s.k
+    for what, t, n in (("x_rows", x_rows, rows * width), ("offsets", offsets, s.N + 1),
+                       ("w_gate", w_gate, s.N * s.h * width), ("w_up", w_up, s.N * s.h * width),
+                       ("w_down", w_down, s.N * width * s.h), ("y_rows", y_rows, rows * width)):
+        _need(what, t, n)
     dt = _dtype_code(x_rows)
     nb = _lib.moe_expert_ffn_workspace_bytes(ctypes.byref(s), width, dt)
     wbuf, wlen = _ws(nb, x_rows.device, ws)
@@ -214,6 +260,10 @@ def moe_expert_ffn(s: MoeShape, width: int, x_rows, offsets, w_gate, w_up, w_dow
 
 
 def moe_combine(s: MoeShape, width: int, y_rows, row_of, top_w, y, stream=None):
+    """y_rows is read at the rows row_of names, so its size is not checked here."""
+    for what, t, n in (("row_of", row_of, s.T * s.k), ("top_w", top_w, s.T * s.k),
+                       ("y", y, s.T * width)):
+        _need(what, t, n)
     _check(_lib.moe_combine(ctypes.byref(s), width, _ptr(y_rows), _ptr(row_of), _ptr(top_w),
                             _ptr(y), _dtype_code(y), _stream(stream)), "moe_combine")
 
@@ -227,9 +277,13 @@ def moe_layer_fwd(s: MoeShape, w_route, w_gate, w_up, w_down, u, y, bias=None, a
     """The whole layer.  `outputs` maps moe_layer_outputs field names to tensors."""
     a = a or act()
     dt = _dtype_code(u)
+    for what, t, n in (("u", u, s.T * s.d), ("y", y, s.T * s.d), ("w_route", w_route, s.N * s.d),
+                       ("bias", bias, s.N), ("w_gate", w_gate, s.N * s.h * s.d),
+                       ("w_up", w_up, s.N * s.h * s.d), ("w_down", w_down, s.N * s.d * s.h)):
+        _need(what, t, n)
+    O = _outputs(s, outputs)
     W = MoeLayerWeights(_ptr(w_route), _ptr(bias), _ptr(w_gate), _ptr(w_up), _ptr(w_down),
                         _dtype_code(w_gate), a)
-    O = MoeLayerOutputs(**{k: _ptr(v) for k, v in (outputs or {}).items()})
     wbuf, wlen = _ws(moe_layer_workspace_bytes(s, dt), u.device, ws)
     _check(_lib.moe_layer_fwd(ctypes.byref(s), ctypes.byref(W), _ptr(u), dt, _ptr(y),
                               ctypes.byref(O), _ptr(wbuf), wlen, _stream(stream)), "moe_layer_fwd")
@@ -249,9 +303,14 @@ def moe_latent_fwd(s: MoeShape, w_route, w_gate, w_up, w_down, lw: MoeLatentWeig
                    bias=None, a=None, outputs: dict | None = None, ws=None, stream=None):
     """The LatentMoE layer; x, y bf16 [T][d]; routed experts at latent width."""
     a = a or act()
+    l = lw.latent
+    for what, t, n in (("x", x, s.T * s.d), ("y", y, s.T * s.d), ("w_route", w_route, s.N * s.d),
+                       ("bias", bias, s.N), ("w_gate", w_gate, s.N * s.h * l),
+                       ("w_up", w_up, s.N * s.h * l), ("w_down", w_down, s.N * l * s.h)):
+        _need(what, t, n)
+    O = _outputs(s, outputs)
     W = MoeLayerWeights(_ptr(w_route), _ptr(bias), _ptr(w_gate), _ptr(w_up), _ptr(w_down), BF16,
                         a)
-    O = MoeLayerOutputs(**{k: _ptr(v) for k, v in (outputs or {}).items()})
     wbuf, wlen = _ws(moe_latent_workspace_bytes(s, lw), x.device, ws)
     _check(_lib.moe_latent_fwd(ctypes.byref(s), ctypes.byref(W), ctypes.byref(lw), _ptr(x),
                                _ptr(y), ctypes.byref(O), _ptr(wbuf), wlen, _stream(stream)),
@@ -271,6 +330,9 @@ def moe_decode_workspace_bytes(s: MoeShape) -> int:
 def moe_decode_layer(s: MoeShape, layer: MoeQ4Layer, u, y, u_next=None, top_idx=None,
                      top_w=None, ws=None, stream=None):
     """u, y, u_next: fp16 tensors [T][d]."""
+    for what, t, n in (("u", u, s.T * s.d), ("y", y, s.T * s.d), ("u_next", u_next, s.T * s.d),
+                       ("top_idx", top_idx, s.T * s.k), ("top_w", top_w, s.T * s.k)):
+        _need(what, t, n)
     wbuf, wlen = _ws(moe_decode_workspace_bytes(s), u.device, ws)
     _check(_lib.moe_decode_layer(ctypes.byref(s), ctypes.byref(layer), _ptr(u), _ptr(y),
                                  _ptr(u_next), _ptr(top_idx), _ptr(top_w), _ptr(wbuf), wlen,
@@ -279,6 +341,9 @@ def moe_decode_layer(s: MoeShape, layer: MoeQ4Layer, u, y, u_next=None, top_idx=
 
 def moe_decode_step(s: MoeShape, layers, u0, u_out, top_idx_all=None, ws=None, stream=None):
     """`layers`: a sequence of MoeQ4Layer (host structs of device pointers)."""
+    for what, t, n in (("u0", u0, s.T * s.d), ("u_out", u_out, s.T * s.d),
+                       ("top_idx_all", top_idx_all, len(layers) * s.T * s.k)):
+        _need(what, t, n)
     arr = (MoeQ4Layer * len(layers))(*layers)
     wbuf, wlen = _ws(moe_decode_workspace_bytes(s), u0.device, ws)
     _check(_lib.moe_decode_step(ctypes.byref(s), len(layers), arr, _ptr(u0), _ptr(u_out),
@@ -289,6 +354,8 @@ def moe_decode_step(s: MoeShape, layers, u0, u_out, top_idx_all=None, ws=None, s
 def moe_aux_grad(probs, f, dz, alpha: float = 1.0, stream=None):
     """dL_aux/dz [T][N] (fp32 device tensors) with the loads f held constant."""
     T, N = probs.shape
+    _need("f", f, N)
+    _need("dz", dz, T * N)
     _check(_lib.moe_aux_grad(T, N, alpha, _ptr(probs), _ptr(f), _ptr(dz), _stream(stream)),
            "moe_aux_grad")
 
@@ -301,6 +368,9 @@ def moe_quantile_balance(scores, k: int, q: int, bias_exact, bias=None, bins: in
                          cutoff=None, bias_hist=None, loads=None, ws=None, stream=None):
     """scores [T][N] fp32 device tensor; outputs are device tensors (see moe.h)."""
     T, N = scores.shape
+    for what, t, n in (("bias_exact", bias_exact, N), ("bias", bias, N), ("cutoff", cutoff, T),
+                       ("bias_hist", bias_hist, N), ("loads", loads, N)):
+        _need(what, t, n)
     wbuf, wlen = _ws(moe_quantile_balance_workspace_bytes(T, N), scores.device, ws)
     _check(_lib.moe_quantile_balance(T, N, k, _ptr(scores), _ptr(bias), q, bins, _ptr(cutoff),
                                      _ptr(bias_exact), _ptr(bias_hist), _ptr(loads), _ptr(wbuf),

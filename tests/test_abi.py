@@ -156,3 +156,29 @@ def test_binding_refuses_host_tensors_before_the_call():
         moe.moe_gather(s, 64, u, perm, offsets, x_rows)
     with pytest.raises(ValueError, match="CUDA tensor"):
         moe.q4_layer(torch.zeros((4, 64)), *[torch.zeros(8, dtype=torch.uint8)] * 6)
+
+
+def test_binding_refuses_short_tensors_before_the_call():
+    """The library sees only addresses; the binding checks each tensor against
+    the size the header documents, so a short one never reaches a kernel."""
+    import torch
+    s = moe.shape(16, 64, 4, 2, 128)
+    i32 = dict(dtype=torch.int32)
+    with pytest.raises(ValueError, match="x_rows: .* at least 2048"):
+        moe.moe_gather(s, 64, torch.zeros((16, 64)), torch.zeros(32, **i32),
+                       torch.zeros(5, **i32), torch.zeros((31, 64)))
+    with pytest.raises(ValueError, match="offsets"):
+        moe.moe_permute(s, torch.zeros((16, 2), **i32), torch.zeros(4, **i32),
+                        torch.zeros(4, **i32), torch.zeros(32, **i32), torch.zeros((16, 2), **i32),
+                        torch.zeros(4, **i32), torch.zeros(3, **i32))
+    with pytest.raises(ValueError, match="w_down"):
+        moe.moe_layer_fwd(s, torch.zeros((4, 64)), torch.zeros((4, 128, 64)),
+                          torch.zeros((4, 128, 64)), torch.zeros((4, 64, 127)),
+                          torch.zeros((16, 64)), torch.zeros((16, 64)))
+    with pytest.raises(ValueError, match="row_of"):
+        moe.moe_layer_fwd(s, torch.zeros((4, 64)), torch.zeros((4, 128, 64)),
+                          torch.zeros((4, 128, 64)), torch.zeros((4, 64, 128)),
+                          torch.zeros((16, 64)), torch.zeros((16, 64)),
+                          outputs={"row_of": torch.zeros(31, **i32)})
+    with pytest.raises(ValueError, match="dz"):
+        moe.moe_aux_grad(torch.zeros((16, 4)), torch.zeros(4), torch.zeros(63))
