@@ -124,22 +124,37 @@ def _ptr(t):
     return t.data_ptr()
 
 
-def _need(what, t, n):
-    """Refuse a tensor with fewer than n elements where the call touches n.
-    The library sees only the address, so a short tensor would be read or
-    written past its end on the device."""
-    if t is not None and t.numel() < n:
+_F32, _I32, _F16, _BF16, _U8 = "float32", "int32", "float16", "bfloat16", "uint8"
+_ACT = (_F32, _BF16, _F16)  # activation storage types
+_Q4_SCALES = ("int16", "uint16")  # fp16 scale codes, any 16-bit integer view
+
+
+def _need(what, t, n, dtypes=None):
+    """Refuse a tensor with fewer than n elements where the call touches n, or
+    of another element type than the library reads or writes there.  The
+    library sees only the address, so a short or narrower tensor would be read
+    or written past its end on the device."""
+    if t is None:
+        return
+    if t.numel() < n:
         raise ValueError(f"{what}: {t.numel()} elements, the call needs at least {n}")
+    if dtypes is not None:
+        allowed = (dtypes,) if isinstance(dtypes, str) else tuple(dtypes)
+        name = str(t.dtype).replace("torch.", "")
+        if name not in allowed:
+            raise ValueError(f"{what}: dtype {name}, the call needs {' or '.join(allowed)}")
 
 
 def _outputs(s: MoeShape, outputs):
     """moe_layer_outputs from a dict of tensors, each checked against its
     documented size."""
     Tk, TN, N = s.T * s.k, s.T * s.N, s.N
-    sizes = dict(top_idx=Tk, top_w=Tk, probs=TN, counts=N, offsets=N + 1, perm_tok=Tk,
-                 row_of=Tk, overflow=N, totals=3, f=N, P=N, n_sum_fP=1)
+    sizes = dict(top_idx=(Tk, _I32), top_w=(Tk, _F32), probs=(TN, _F32), counts=(N, _I32),
+                 offsets=(N + 1, _I32), perm_tok=(Tk, _I32), row_of=(Tk, _I32),
+                 overflow=(N, _I32), totals=(3, _I32), f=(N, _F32), P=(N, _F32),
+                 n_sum_fP=(1, _F32))
     for key, t in (outputs or {}).items():
-        _need(key, t, sizes[key])
+        _need(key, t, *sizes[key])
     return MoeLayerOutputs(**{key: _ptr(t) for key, t in (outputs or {}).items()})
 
 
@@ -182,10 +197,11 @@ def moe_capacity(T: int, N: int, k: int, factor: float) -> int:
 
 def moe_route(s: MoeShape, u, w_route, top_idx, top_w, bias=None, probs=None, logits=None,
               ws=None, stream=None):
-    for what, t, n in (("u", u, s.T * s.d), ("w_route", w_route, s.N * s.d), ("bias", bias, s.N),
-                       ("top_idx", top_idx, s.T * s.k), ("top_w", top_w, s.T * s.k),
-                       ("probs", probs, s.T * s.N), ("logits", logits, s.T * s.N)):
-        _need(what, t, n)
+    for args in (("u", u, s.T * s.d, _ACT), ("w_route", w_route, s.N * s.d, _F32),
+                 ("bias", bias, s.N, _F32), ("top_idx", top_idx, s.T * s.k, _I32),
+                 ("top_w", top_w, s.T * s.k, _F32), ("probs", probs, s.T * s.N, _F32),
+                 ("logits", logits, s.T * s.N, _F32)):
+        _need(*args)
     nb = _lib.moe_route_workspace_bytes(ctypes.byref(s))
     wbuf, wlen = (None, 0) if logits is not None else _ws(nb, u.device, ws)
     _check(_lib.moe_route(ctypes.byref(s), _ptr(u), _dtype_code(u), _ptr(w_route), _ptr(bias),
@@ -197,9 +213,10 @@ def moe_aux_stats(probs, top_idx, f=None, P=None, n_sum_fP=None, loads=None, ws=
                   stream=None):
     T, k = top_idx.shape
     N = f.shape[0] if f is not None else (P.shape[0] if P is not None else loads.shape[0])
-    for what, t, n in (("probs", probs, T * N), ("f", f, N), ("P", P, N), ("n_sum_fP", n_sum_fP, 1),
-                       ("loads", loads, N)):
-        _need(what, t, n)
+    for args in (("probs", probs, T * N, _F32), ("top_idx", top_idx, T * k, _I32),
+                 ("f", f, N, _F32), ("P", P, N, _F32), ("n_sum_fP", n_sum_fP, 1, _F32),
+                 ("loads", loads, N, _I32)):
+        _need(*args)
     wbuf, wlen = _ws(_lib.moe_aux_stats_workspace_bytes(N), top_idx.device, ws)
     _check(_lib.moe_aux_stats(T, N, k, _ptr(probs), _ptr(top_idx), _ptr(f), _ptr(P),
                               _ptr(n_sum_fP), _ptr(loads), _ptr(wbuf), wlen, _stream(stream)),
@@ -211,7 +228,7 @@ def _permute_sizes(s, top_idx, counts, offsets, perm_tok, row_of, overflow, tota
     for what, t, n in (("top_idx", top_idx, Tk), ("counts", counts, s.N),
                        ("offsets", offsets, s.N + 1), ("perm_tok", perm_tok, Tk),
                        ("row_of", row_of, Tk), ("overflow", overflow, s.N), ("totals", totals, 3)):
-        _need(what, t, n)
+        _need(what, t, n, _I32)
 
 
 def moe_permute(s: MoeShape, top_idx, counts, offsets, perm_tok, row_of, overflow, totals,
@@ -235,9 +252,10 @@ def moe_permute_noalloc(s: MoeShape, top_idx, counts, offsets, perm_tok, row_of,
 def moe_gather(s: MoeShape, width: int, u, perm_tok, offsets, x_rows, stream=None):
     """perm_tok is read for the offsets[N] grouped rows only, a count the
     device holds, so its size is not checked here."""
-    _need("u", u, s.T * width)
-    _need("offsets", offsets, s.N + 1)
-    _need("x_rows", x_rows, s.T * s.k * width)
+    _need("u", u, s.T * width, _ACT)
+    _need("perm_tok", perm_tok, 0, _I32)
+    _need("offsets", offsets, s.N + 1, _I32)
+    _need("x_rows", x_rows, s.T * s.k * width, str(u.dtype).replace("torch.", ""))
     _check(_lib.moe_gather(ctypes.byref(s), width, _ptr(u), _dtype_code(u), _ptr(perm_tok),
                            _ptr(offsets), _ptr(x_rows), _stream(stream)), "moe_gather")
 
@@ -246,10 +264,13 @@ def moe_expert_ffn(s: MoeShape, width: int, x_rows, offsets, w_gate, w_up, w_dow
                    a: MoeAct | None = None, ws=None, stream=None):
     a = a or act()
     rows = s.T * s.k
-    for what, t, n in (("x_rows", x_rows, rows * width), ("offsets", offsets, s.N + 1),
-                       ("w_gate", w_gate, s.N * s.h * width), ("w_up", w_up, s.N * s.h * width),
-                       ("w_down", w_down, s.N * width * s.h), ("y_rows", y_rows, rows * width)):
-        _need(what, t, n)
+    x_dt = str(x_rows.dtype).replace("torch.", "")
+    for args in (("x_rows", x_rows, rows * width, (_F32, _BF16)),
+                 ("offsets", offsets, s.N + 1, _I32),
+                 ("w_gate", w_gate, s.N * s.h * width, x_dt), ("w_up", w_up, s.N * s.h * width, x_dt),
+                 ("w_down", w_down, s.N * width * s.h, x_dt),
+                 ("y_rows", y_rows, rows * width, _F32)):
+        _need(*args)
     dt = _dtype_code(x_rows)
     nb = _lib.moe_expert_ffn_workspace_bytes(ctypes.byref(s), width, dt)
     wbuf, wlen = _ws(nb, x_rows.device, ws)
@@ -261,9 +282,9 @@ def moe_expert_ffn(s: MoeShape, width: int, x_rows, offsets, w_gate, w_up, w_dow
 
 def moe_combine(s: MoeShape, width: int, y_rows, row_of, top_w, y, stream=None):
     """y_rows is read at the rows row_of names, so its size is not checked here."""
-    for what, t, n in (("row_of", row_of, s.T * s.k), ("top_w", top_w, s.T * s.k),
-                       ("y", y, s.T * width)):
-        _need(what, t, n)
+    for args in (("y_rows", y_rows, 0, _F32), ("row_of", row_of, s.T * s.k, _I32),
+                 ("top_w", top_w, s.T * s.k, _F32), ("y", y, s.T * width, _ACT)):
+        _need(*args)
     _check(_lib.moe_combine(ctypes.byref(s), width, _ptr(y_rows), _ptr(row_of), _ptr(top_w),
                             _ptr(y), _dtype_code(y), _stream(stream)), "moe_combine")
 
@@ -277,10 +298,12 @@ def moe_layer_fwd(s: MoeShape, w_route, w_gate, w_up, w_down, u, y, bias=None, a
     """The whole layer.  `outputs` maps moe_layer_outputs field names to tensors."""
     a = a or act()
     dt = _dtype_code(u)
-    for what, t, n in (("u", u, s.T * s.d), ("y", y, s.T * s.d), ("w_route", w_route, s.N * s.d),
-                       ("bias", bias, s.N), ("w_gate", w_gate, s.N * s.h * s.d),
-                       ("w_up", w_up, s.N * s.h * s.d), ("w_down", w_down, s.N * s.d * s.h)):
-        _need(what, t, n)
+    u_dt = str(u.dtype).replace("torch.", "")
+    for args in (("u", u, s.T * s.d, (_F32, _BF16)), ("y", y, s.T * s.d, u_dt),
+                 ("w_route", w_route, s.N * s.d, _F32), ("bias", bias, s.N, _F32),
+                 ("w_gate", w_gate, s.N * s.h * s.d, u_dt), ("w_up", w_up, s.N * s.h * s.d, u_dt),
+                 ("w_down", w_down, s.N * s.d * s.h, u_dt)):
+        _need(*args)
     O = _outputs(s, outputs)
     W = MoeLayerWeights(_ptr(w_route), _ptr(bias), _ptr(w_gate), _ptr(w_up), _ptr(w_down),
                         _dtype_code(w_gate), a)
@@ -304,10 +327,11 @@ def moe_latent_fwd(s: MoeShape, w_route, w_gate, w_up, w_down, lw: MoeLatentWeig
     """The LatentMoE layer; x, y bf16 [T][d]; routed experts at latent width."""
     a = a or act()
     l = lw.latent
-    for what, t, n in (("x", x, s.T * s.d), ("y", y, s.T * s.d), ("w_route", w_route, s.N * s.d),
-                       ("bias", bias, s.N), ("w_gate", w_gate, s.N * s.h * l),
-                       ("w_up", w_up, s.N * s.h * l), ("w_down", w_down, s.N * l * s.h)):
-        _need(what, t, n)
+    for args in (("x", x, s.T * s.d, _BF16), ("y", y, s.T * s.d, _BF16),
+                 ("w_route", w_route, s.N * s.d, _F32), ("bias", bias, s.N, _F32),
+                 ("w_gate", w_gate, s.N * s.h * l, _BF16), ("w_up", w_up, s.N * s.h * l, _BF16),
+                 ("w_down", w_down, s.N * l * s.h, _BF16)):
+        _need(*args)
     O = _outputs(s, outputs)
     W = MoeLayerWeights(_ptr(w_route), _ptr(bias), _ptr(w_gate), _ptr(w_up), _ptr(w_down), BF16,
                         a)
@@ -319,6 +343,14 @@ def moe_latent_fwd(s: MoeShape, w_route, w_gate, w_up, w_down, lw: MoeLatentWeig
 
 def q4_layer(w_route, gate_qs, gate_scales, up_qs, up_scales, down_qs, down_scales,
              bias=None) -> MoeQ4Layer:
+    """One q4_0 layer's device pointers (sizes follow the shape of the call
+    that uses it, so only the element types are checked here)."""
+    for args in (("w_route", w_route, 0, _F32), ("bias", bias, 0, _F32),
+                 ("gate_qs", gate_qs, 0, _U8), ("up_qs", up_qs, 0, _U8),
+                 ("down_qs", down_qs, 0, _U8), ("gate_scales", gate_scales, 0, _Q4_SCALES),
+                 ("up_scales", up_scales, 0, _Q4_SCALES),
+                 ("down_scales", down_scales, 0, _Q4_SCALES)):
+        _need(*args)
     return MoeQ4Layer(_ptr(w_route), _ptr(bias), _ptr(gate_qs), _ptr(gate_scales), _ptr(up_qs),
                       _ptr(up_scales), _ptr(down_qs), _ptr(down_scales))
 
@@ -330,9 +362,10 @@ def moe_decode_workspace_bytes(s: MoeShape) -> int:
 def moe_decode_layer(s: MoeShape, layer: MoeQ4Layer, u, y, u_next=None, top_idx=None,
                      top_w=None, ws=None, stream=None):
     """u, y, u_next: fp16 tensors [T][d]."""
-    for what, t, n in (("u", u, s.T * s.d), ("y", y, s.T * s.d), ("u_next", u_next, s.T * s.d),
-                       ("top_idx", top_idx, s.T * s.k), ("top_w", top_w, s.T * s.k)):
-        _need(what, t, n)
+    for args in (("u", u, s.T * s.d, _F16), ("y", y, s.T * s.d, _F16),
+                 ("u_next", u_next, s.T * s.d, _F16), ("top_idx", top_idx, s.T * s.k, _I32),
+                 ("top_w", top_w, s.T * s.k, _F32)):
+        _need(*args)
     wbuf, wlen = _ws(moe_decode_workspace_bytes(s), u.device, ws)
     _check(_lib.moe_decode_layer(ctypes.byref(s), ctypes.byref(layer), _ptr(u), _ptr(y),
                                  _ptr(u_next), _ptr(top_idx), _ptr(top_w), _ptr(wbuf), wlen,
@@ -341,9 +374,9 @@ def moe_decode_layer(s: MoeShape, layer: MoeQ4Layer, u, y, u_next=None, top_idx=
 
 def moe_decode_step(s: MoeShape, layers, u0, u_out, top_idx_all=None, ws=None, stream=None):
     """`layers`: a sequence of MoeQ4Layer (host structs of device pointers)."""
-    for what, t, n in (("u0", u0, s.T * s.d), ("u_out", u_out, s.T * s.d),
-                       ("top_idx_all", top_idx_all, len(layers) * s.T * s.k)):
-        _need(what, t, n)
+    for args in (("u0", u0, s.T * s.d, _F16), ("u_out", u_out, s.T * s.d, _F16),
+                 ("top_idx_all", top_idx_all, len(layers) * s.T * s.k, _I32)):
+        _need(*args)
     arr = (MoeQ4Layer * len(layers))(*layers)
     wbuf, wlen = _ws(moe_decode_workspace_bytes(s), u0.device, ws)
     _check(_lib.moe_decode_step(ctypes.byref(s), len(layers), arr, _ptr(u0), _ptr(u_out),
@@ -354,8 +387,9 @@ def moe_decode_step(s: MoeShape, layers, u0, u_out, top_idx_all=None, ws=None, s
 def moe_aux_grad(probs, f, dz, alpha: float = 1.0, stream=None):
     """dL_aux/dz [T][N] (fp32 device tensors) with the loads f held constant."""
     T, N = probs.shape
-    _need("f", f, N)
-    _need("dz", dz, T * N)
+    _need("probs", probs, T * N, _F32)
+    _need("f", f, N, _F32)
+    _need("dz", dz, T * N, _F32)
     _check(_lib.moe_aux_grad(T, N, alpha, _ptr(probs), _ptr(f), _ptr(dz), _stream(stream)),
            "moe_aux_grad")
 
@@ -368,9 +402,10 @@ def moe_quantile_balance(scores, k: int, q: int, bias_exact, bias=None, bins: in
                          cutoff=None, bias_hist=None, loads=None, ws=None, stream=None):
     """scores [T][N] fp32 device tensor; outputs are device tensors (see moe.h)."""
     T, N = scores.shape
-    for what, t, n in (("bias_exact", bias_exact, N), ("bias", bias, N), ("cutoff", cutoff, T),
-                       ("bias_hist", bias_hist, N), ("loads", loads, N)):
-        _need(what, t, n)
+    for args in (("scores", scores, T * N, _F32), ("bias_exact", bias_exact, N, _F32),
+                 ("bias", bias, N, _F32), ("cutoff", cutoff, T, _F32),
+                 ("bias_hist", bias_hist, N, _F32), ("loads", loads, N, _I32)):
+        _need(*args)
     wbuf, wlen = _ws(moe_quantile_balance_workspace_bytes(T, N), scores.device, ws)
     _check(_lib.moe_quantile_balance(T, N, k, _ptr(scores), _ptr(bias), q, bins, _ptr(cutoff),
                                      _ptr(bias_exact), _ptr(bias_hist), _ptr(loads), _ptr(wbuf),

@@ -155,7 +155,8 @@ def test_binding_refuses_host_tensors_before_the_call():
     with pytest.raises(ValueError, match="CUDA tensor"):
         moe.moe_gather(s, 64, u, perm, offsets, x_rows)
     with pytest.raises(ValueError, match="CUDA tensor"):
-        moe.q4_layer(torch.zeros((4, 64)), *[torch.zeros(8, dtype=torch.uint8)] * 6)
+        qs, sc = torch.zeros(8, dtype=torch.uint8), torch.zeros(8, dtype=torch.int16)
+        moe.q4_layer(torch.zeros((4, 64)), qs, sc, qs, sc, qs, sc)
 
 
 def test_binding_refuses_short_tensors_before_the_call():
@@ -182,3 +183,21 @@ def test_binding_refuses_short_tensors_before_the_call():
                           outputs={"row_of": torch.zeros(31, **i32)})
     with pytest.raises(ValueError, match="dz"):
         moe.moe_aux_grad(torch.zeros((16, 4)), torch.zeros(4), torch.zeros(63))
+
+
+def test_binding_refuses_other_element_types():
+    """A narrower element type would let the kernels write past the end."""
+    import torch
+    s = moe.shape(16, 64, 4, 2, 128)
+    with pytest.raises(ValueError, match="top_w: dtype bfloat16"):
+        moe.moe_route(s, torch.zeros((16, 64)), torch.zeros((4, 64)),
+                      torch.zeros((16, 2), dtype=torch.int32),
+                      torch.zeros((16, 2), dtype=torch.bfloat16))
+    with pytest.raises(ValueError, match="w_up: dtype float32"):
+        bf = dict(dtype=torch.bfloat16)
+        moe.moe_layer_fwd(s, torch.zeros((4, 64)), torch.zeros((4, 128, 64), **bf),
+                          torch.zeros((4, 128, 64)), torch.zeros((4, 64, 128), **bf),
+                          torch.zeros((16, 64), **bf), torch.zeros((16, 64), **bf))
+    with pytest.raises(ValueError, match="top_idx: dtype int64"):
+        moe.moe_permute(s, torch.zeros((16, 2), dtype=torch.int64),
+                        *[torch.zeros(64, dtype=torch.int32)] * 6)
