@@ -84,6 +84,12 @@ def lib():
         L.or_round_e4m3.restype = ctypes.c_uint8
         L.or_quant_e4m3_rows.argtypes = [i64, i64, vp, vp, vp]
         L.or_quant_e4m3_rows.restype = None
+        L.or_latent_loss.argtypes = [i64, i64, i64, ctypes.c_int, vp, vp, vp, dbl, dbl, vp, vp,
+                                     vp, i64, vp, vp, vp, dbl, vp, i64, vp, vp, vp]
+        L.or_latent_loss.restype = dbl
+        L.or_latent_backward.argtypes = [i64, i64, i64, ctypes.c_int, vp, vp, vp, dbl, dbl, vp,
+                                         vp, vp, i64, vp, vp, vp, dbl, vp, i64, vp, vp] + [vp] * 11
+        L.or_latent_backward.restype = None
         L.or_layer_loss.argtypes = [i64, i64, i64, ctypes.c_int, vp, vp, vp, ctypes.c_int, dbl,
                                     dbl, vp, vp, vp, i64, vp, vp, vp, dbl, vp, vp]
         L.or_layer_loss.restype = dbl
@@ -481,4 +487,55 @@ def layer_backward(Wg, Wu, Wd, u, top_idx, dy, Wr=None, z=None, row_of=None, ren
                             _p(row_of), dy.ctypes.data, alpha, _p(f), out["dz"].ctypes.data,
                             out["du"].ctypes.data, _p(out["dWr"]), out["dWg"].ctypes.data,
                             out["dWu"].ctypes.data, out["dWd"].ctypes.data)
+    return out
+
+
+def _latent_args(routed, Wr, W_dp, W_upp, shared, x, top_idx, dy):
+    Wg, Wu, Wd = routed
+    x = _c(x, np.float64)
+    T, d = x.shape
+    idx = _c(top_idx, np.int32)
+    sg = [m[0] for m in shared]
+    su = [m[1] for m in shared]
+    sd = [m[2] for m in shared]
+    sh_arrays = (mat_array(sg), mat_array(su), mat_array(sd)) if shared else (None, None, None)
+    return (Wg, Wu, Wd, _c(Wr, np.float64), x, T, d, idx, idx.shape[1], len(Wg),
+            _c(dy, np.float64).reshape(T, d), sh_arrays)
+
+
+def latent_loss(routed, Wr, W_dp, W_upp, shared, x, top_idx, dy, beta_g, beta_u, eps=1e-6,
+                renorm=1):
+    """(L, y) of the LatentMoE layer in double (no intermediate rounding) with
+    the selected sets top_idx held fixed; routed = (gates, ups, downs) lists of
+    Mats at the latent width, shared = [(gate, up, down)] at full width."""
+    Wg, Wu, Wd, Wr, x, T, d, idx, k, N, dy, sh = _latent_args(routed, Wr, W_dp, W_upp, shared,
+                                                              x, top_idx, dy)
+    y = np.empty((T, d), np.float64)
+    L = lib().or_latent_loss(T, N, k, renorm, mat_array(Wg), mat_array(Wu), mat_array(Wd), beta_g,
+                             beta_u, Wr.ctypes.data, ctypes.byref(W_dp.s), ctypes.byref(W_upp.s),
+                             len(shared), *sh, eps, x.ctypes.data, d, idx.ctypes.data,
+                             dy.ctypes.data, y.ctypes.data)
+    return float(L), y
+
+
+def latent_backward(routed, Wr, W_dp, W_upp, shared, x, top_idx, dy, beta_g, beta_u, eps=1e-6,
+                    renorm=1):
+    """Gradients of latent_loss: dict of dz, dx, dWr, dWdp, dWupp, dWg, dWu,
+    dWd, dSg, dSu, dSd (the shared ones None without shared experts)."""
+    Wg, Wu, Wd, Wr, x, T, d, idx, k, N, dy, sh = _latent_args(routed, Wr, W_dp, W_upp, shared,
+                                                              x, top_idx, dy)
+    l, h = W_dp.rows, Wg[0].rows
+    n = len(shared)
+    s_h = shared[0][0].rows if n else 0
+    out = dict(dz=np.empty((T, N)), dx=np.empty((T, d)), dWr=np.empty((N, d)),
+               dWdp=np.empty((l, d)), dWupp=np.empty((d, l)), dWg=np.empty((N, h, l)),
+               dWu=np.empty((N, h, l)), dWd=np.empty((N, l, h)),
+               dSg=np.empty((n, s_h, d)) if n else None, dSu=np.empty((n, s_h, d)) if n else None,
+               dSd=np.empty((n, d, s_h)) if n else None)
+    lib().or_latent_backward(T, N, k, renorm, mat_array(Wg), mat_array(Wu), mat_array(Wd),
+                             beta_g, beta_u, Wr.ctypes.data, ctypes.byref(W_dp.s),
+                             ctypes.byref(W_upp.s), n, *sh, eps, x.ctypes.data, d,
+                             idx.ctypes.data, dy.ctypes.data,
+                             *[_p(out[key]) for key in ("dz", "dx", "dWr", "dWdp", "dWupp", "dWg",
+                                                        "dWu", "dWd", "dSg", "dSu", "dSd")])
     return out

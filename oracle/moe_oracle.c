@@ -834,3 +834,206 @@ void or_layer_backward(int64_t T, int64_t N, int64_t k, int renorm, const or_mat
   free(dF);
   free(F);
 }
+
+/* ------------------------------------------------ LatentMoE layer backward */
+/* The LatentMoE layer of [LatentMoE] (width separation, RMSNorm before the
+ * up-projection, SiTU-GLU routed experts, plain SwiGLU shared experts), in
+ * double with no intermediate rounding, for one token x (width d):
+ *   z = W_route x,  p = softmax(z),  a over the selected set (renorm or not)
+ *   x_l = W_dp x                                  (width l)
+ *   m = sum_s a_s E_{e_s}(x_l)                    (SiTU-GLU experts, width l)
+ *   r = sqrt(mean(m^2) + eps),  m^ = m / r
+ *   y = W_upp m^ + sum_j S_j(x)                   (width d)
+ * and L = sum_t dy_t . y_t.  The selected sets are inputs held fixed. */
+static void or_latent_token(int64_t N, int64_t k, int renorm, const or_mat* Wg,
+                            const or_mat* Wu, const or_mat* Wd, double beta_g, double beta_u,
+                            const double* Wr, const or_mat* Wdp, const or_mat* Wupp,
+                            int64_t n_shared, const or_mat* Sg, const or_mat* Su,
+                            const or_mat* Sd, double eps, const double* x, int64_t d,
+                            const int32_t* sel, double* z, double* p, double* a, double* xl,
+                            double* m, double* mh, double* r_out, double* y) {
+  int64_t l = Wdp->rows;
+  double* F = (double*)malloc(sizeof(double) * (size_t)(l > d ? l : d));
+  or_token_weights(N, d, k, renorm, Wr, NULL, x, sel, z, p, a);
+  or_matvec(Wdp, x, xl);
+  for (int64_t i = 0; i < l; ++i) m[i] = 0.0;
+  for (int64_t s = 0; s < k; ++s) {
+    int32_t e = sel[s];
+    or_expert(&Wg[e], &Wu[e], &Wd[e], xl, 1, beta_g, beta_u, 0, F);
+    for (int64_t i = 0; i < l; ++i) m[i] += a[s] * F[i];
+  }
+  double ss = 0.0;
+  for (int64_t i = 0; i < l; ++i) ss += m[i] * m[i];
+  double r = sqrt(ss / (double)l + eps);
+  for (int64_t i = 0; i < l; ++i) mh[i] = m[i] / r;
+  *r_out = r;
+  or_matvec(Wupp, mh, y);
+  for (int64_t j = 0; j < n_shared; ++j) {
+    or_expert(&Sg[j], &Su[j], &Sd[j], x, 0, 0.0, 0.0, 0, F);
+    for (int64_t c = 0; c < d; ++c) y[c] += F[c];
+  }
+  free(F);
+}
+
+/* L = sum_t dy_t . y_t of the LatentMoE layer above; y (nullable) [T][d].
+ * Routed experts: W_gate, W_up [h][l], W_down [l][h]; W_dp [l][d];
+ * W_upp [d][l]; shared experts [sh][d], [d][sh]; W_route [N][d] double. */
+double or_latent_loss(int64_t T, int64_t N, int64_t k, int renorm, const or_mat* Wg,
+                      const or_mat* Wu, const or_mat* Wd, double beta_g, double beta_u,
+                      const double* Wr, const or_mat* Wdp, const or_mat* Wupp, int64_t n_shared,
+                      const or_mat* Sg, const or_mat* Su, const or_mat* Sd, double eps,
+                      const double* x, int64_t d, const int32_t* top_idx, const double* dy,
+                      double* y) {
+  int64_t l = Wdp->rows;
+  double* z = (double*)malloc(sizeof(double) * (size_t)N);
+  double* p = (double*)malloc(sizeof(double) * (size_t)N);
+  double* a = (double*)malloc(sizeof(double) * (size_t)k);
+  double* xl = (double*)malloc(sizeof(double) * (size_t)l);
+  double* m = (double*)malloc(sizeof(double) * (size_t)l);
+  double* mh = (double*)malloc(sizeof(double) * (size_t)l);
+  double* yt = (double*)malloc(sizeof(double) * (size_t)d);
+  double L = 0.0, r;
+  for (int64_t t = 0; t < T; ++t) {
+    or_latent_token(N, k, renorm, Wg, Wu, Wd, beta_g, beta_u, Wr, Wdp, Wupp, n_shared, Sg, Su,
+                    Sd, eps, x + t * d, d, top_idx + t * k, z, p, a, xl, m, mh, &r, yt);
+    for (int64_t c = 0; c < d; ++c) L += dy[t * d + c] * yt[c];
+    if (y)
+      for (int64_t c = 0; c < d; ++c) y[t * d + c] = yt[c];
+  }
+  free(z);
+  free(p);
+  free(a);
+  free(xl);
+  free(m);
+  free(mh);
+  free(yt);
+  return L;
+}
+
+/* Gradients of or_latent_loss.  Per token:
+ *   dW_upp += dy m^T,  dm^ = W_upp^T dy
+ *   RMSNorm:  dm = dm^ / r - m (sum_i dm^_i m_i) / (l r^3)
+ *   routed slot s (expert e):  da_s = dm . E_e(x_l); the expert backward
+ *       (soft caps included) with dF = a_s dm adds to dW*_e and dx_l
+ *   renorm / softmax / router as in or_layer_backward: dz, dW_route += dz x^T,
+ *       dx += W_route^T dz
+ *   dW_dp += dx_l x^T,  dx += W_dp^T dx_l
+ *   shared expert j: the SwiGLU backward with dF = dy adds to dS*_j and dx.
+ * Outputs, all overwritten: dz [T][N], dx [T][d], dWr [N][d], dWdp [l][d],
+ * dWupp [d][l], dWg, dWu [N][h][l], dWd [N][l][h], dSg, dSu [n][sh][d],
+ * dSd [n][d][sh] (the shared ones may be NULL when n_shared = 0). */
+void or_latent_backward(int64_t T, int64_t N, int64_t k, int renorm, const or_mat* Wg,
+                        const or_mat* Wu, const or_mat* Wd, double beta_g, double beta_u,
+                        const double* Wr, const or_mat* Wdp, const or_mat* Wupp,
+                        int64_t n_shared, const or_mat* Sg, const or_mat* Su, const or_mat* Sd,
+                        double eps, const double* x, int64_t d, const int32_t* top_idx,
+                        const double* dy, double* dz, double* dx, double* dWr, double* dWdp,
+                        double* dWupp, double* dWg, double* dWu, double* dWd, double* dSg,
+                        double* dSu, double* dSd) {
+  int64_t l = Wdp->rows, h = Wg[0].rows, sh = n_shared > 0 ? Sg[0].rows : 0;
+  memset(dx, 0, sizeof(double) * (size_t)(T * d));
+  memset(dWr, 0, sizeof(double) * (size_t)(N * d));
+  memset(dWdp, 0, sizeof(double) * (size_t)(l * d));
+  memset(dWupp, 0, sizeof(double) * (size_t)(d * l));
+  memset(dWg, 0, sizeof(double) * (size_t)(N * h * l));
+  memset(dWu, 0, sizeof(double) * (size_t)(N * h * l));
+  memset(dWd, 0, sizeof(double) * (size_t)(N * l * h));
+  if (n_shared > 0) {
+    memset(dSg, 0, sizeof(double) * (size_t)(n_shared * sh * d));
+    memset(dSu, 0, sizeof(double) * (size_t)(n_shared * sh * d));
+    memset(dSd, 0, sizeof(double) * (size_t)(n_shared * d * sh));
+  }
+  double* z = (double*)malloc(sizeof(double) * (size_t)N);
+  double* p = (double*)malloc(sizeof(double) * (size_t)N);
+  double* dp = (double*)malloc(sizeof(double) * (size_t)N);
+  double* a = (double*)malloc(sizeof(double) * (size_t)k);
+  double* da = (double*)malloc(sizeof(double) * (size_t)k);
+  double* xl = (double*)malloc(sizeof(double) * (size_t)l);
+  double* dxl = (double*)malloc(sizeof(double) * (size_t)l);
+  double* m = (double*)malloc(sizeof(double) * (size_t)l);
+  double* mh = (double*)malloc(sizeof(double) * (size_t)l);
+  double* dmh = (double*)malloc(sizeof(double) * (size_t)l);
+  double* dm = (double*)malloc(sizeof(double) * (size_t)l);
+  double* dF = (double*)malloc(sizeof(double) * (size_t)(l > d ? l : d));
+  double* F = (double*)malloc(sizeof(double) * (size_t)(l > d ? l : d));
+  double* yt = (double*)malloc(sizeof(double) * (size_t)d);
+  for (int64_t t = 0; t < T; ++t) {
+    const double* xt = x + t * d;
+    const double* dyt = dy + t * d;
+    const int32_t* sel = top_idx + t * k;
+    double* dxt = dx + t * d;
+    double* dzt = dz + t * N;
+    double r;
+    or_latent_token(N, k, renorm, Wg, Wu, Wd, beta_g, beta_u, Wr, Wdp, Wupp, n_shared, Sg, Su,
+                    Sd, eps, xt, d, sel, z, p, a, xl, m, mh, &r, yt);
+    /* up-projection and RMSNorm */
+    for (int64_t i = 0; i < l; ++i) {
+      double acc = 0.0;
+      for (int64_t c = 0; c < d; ++c) acc += mat_get(Wupp, c, i) * dyt[c];
+      dmh[i] = acc;
+    }
+    for (int64_t c = 0; c < d; ++c)
+      for (int64_t i = 0; i < l; ++i) dWupp[c * l + i] += dyt[c] * mh[i];
+    double dot = 0.0;
+    for (int64_t i = 0; i < l; ++i) dot += dmh[i] * m[i];
+    for (int64_t i = 0; i < l; ++i) dm[i] = dmh[i] / r - m[i] * dot / ((double)l * r * r * r);
+    /* routed experts */
+    for (int64_t i = 0; i < l; ++i) dxl[i] = 0.0;
+    for (int64_t s = 0; s < k; ++s) {
+      int32_t e = sel[s];
+      for (int64_t i = 0; i < l; ++i) dF[i] = a[s] * dm[i];
+      or_expert_backward(&Wg[e], &Wu[e], &Wd[e], xl, 1, beta_g, beta_u, dF, F,
+                         dWg + (int64_t)e * h * l, dWu + (int64_t)e * h * l,
+                         dWd + (int64_t)e * l * h, dxl);
+      double acc = 0.0;
+      for (int64_t i = 0; i < l; ++i) acc += dm[i] * F[i];
+      da[s] = acc;
+    }
+    /* combine weights, softmax, router */
+    for (int64_t j = 0; j < N; ++j) dp[j] = 0.0;
+    if (renorm) {
+      double ssum = 0.0, ada = 0.0;
+      for (int64_t s = 0; s < k; ++s) {
+        ssum += p[sel[s]];
+        ada += a[s] * da[s];
+      }
+      for (int64_t s = 0; s < k; ++s) dp[sel[s]] = (da[s] - ada) / ssum;
+    } else {
+      for (int64_t s = 0; s < k; ++s) dp[sel[s]] = da[s];
+    }
+    double pdp = 0.0;
+    for (int64_t j = 0; j < N; ++j) pdp += p[j] * dp[j];
+    for (int64_t j = 0; j < N; ++j) dzt[j] = p[j] * (dp[j] - pdp);
+    for (int64_t j = 0; j < N; ++j) {
+      for (int64_t c = 0; c < d; ++c) {
+        dWr[j * d + c] += dzt[j] * xt[c];
+        dxt[c] += dzt[j] * Wr[j * d + c];
+      }
+    }
+    /* down-projection into the latent width */
+    for (int64_t i = 0; i < l; ++i) {
+      for (int64_t c = 0; c < d; ++c) {
+        dWdp[i * d + c] += dxl[i] * xt[c];
+        dxt[c] += mat_get(Wdp, i, c) * dxl[i];
+      }
+    }
+    /* shared experts at full width */
+    for (int64_t j = 0; j < n_shared; ++j)
+      or_expert_backward(&Sg[j], &Su[j], &Sd[j], xt, 0, 0.0, 0.0, dyt, F,
+                         dSg + j * sh * d, dSu + j * sh * d, dSd + j * d * sh, dxt);
+  }
+  free(z);
+  free(p);
+  free(dp);
+  free(a);
+  free(da);
+  free(xl);
+  free(dxl);
+  free(m);
+  free(mh);
+  free(dmh);
+  free(dm);
+  free(dF);
+  free(F);
+  free(yt);
+}

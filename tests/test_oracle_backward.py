@@ -225,3 +225,145 @@ def test_zero_upstream_gradient():
     _close(g["dz"], oracle.aux_grad(probs, c["f"], 0.1), rel=1e-13)
     _close(g["du"], g["dz"] @ c["Wr"], rel=1e-13)
     _close(g["dWr"], g["dz"].T @ c["u"], rel=1e-13)
+
+
+# ----------------------------------------------------------- LatentMoE layer
+LD, LL, LH, LN, LK, LSH, NSH = 12, 8, 10, 6, 2, 14, 2
+
+
+def _latent_case(seed, renorm=1):
+    rng = np.random.default_rng(seed)
+    c = dict(Wg=rng.normal(0, 0.5, (LN, LH, LL)), Wu=rng.normal(0, 0.5, (LN, LH, LL)),
+             Wd=rng.normal(0, 0.5, (LN, LL, LH)), Wr=rng.normal(0, 0.6, (LN, LD)),
+             Wdp=rng.normal(0, 0.4, (LL, LD)), Wupp=rng.normal(0, 0.4, (LD, LL)),
+             Sg=rng.normal(0, 0.3, (NSH, LSH, LD)), Su=rng.normal(0, 0.3, (NSH, LSH, LD)),
+             Sd=rng.normal(0, 0.3, (NSH, LD, LSH)), x=rng.normal(0, 1.0, (7, LD)),
+             dy=rng.normal(0, 1.0, (7, LD)), renorm=renorm)
+    z = c["x"] @ c["Wr"].T
+    c["idx"] = np.argsort(-z, axis=1, kind="stable")[:, :LK].astype(np.int32)
+    return c
+
+
+def _m64(a):
+    return oracle.Mat(oracle.F64, a.shape[0], a.shape[1], data=a)
+
+
+def _latent(c, eps, fn):
+    routed = (_mats(c["Wg"]), _mats(c["Wu"]), _mats(c["Wd"]))
+    shared = [(_m64(c["Sg"][j]), _m64(c["Su"][j]), _m64(c["Sd"][j])) for j in range(NSH)]
+    return fn(routed, c["Wr"], _m64(c["Wdp"]), _m64(c["Wupp"]), shared, c["x"], c["idx"],
+              c["dy"], BG, BU, eps=eps, renorm=c["renorm"])
+
+
+def _latent_torch(c, eps):
+    t = {n: torch.tensor(c[n], dtype=torch.float64, requires_grad=True)
+         for n in ("Wg", "Wu", "Wd", "Wr", "Wdp", "Wupp", "Sg", "Su", "Sd", "x")}
+    idx = torch.tensor(c["idx"], dtype=torch.long)
+    x = t["x"]
+    z = x @ t["Wr"].T
+    z.retain_grad()
+    p = torch.softmax(z, dim=1)
+    ps = torch.gather(p, 1, idx)
+    a = ps / ps.sum(1, keepdim=True) if c["renorm"] else ps
+    xl = x @ t["Wdp"].T
+    g = BG * torch.tanh(torch.einsum("tkhl,tl->tkh", t["Wg"][idx], xl) / BG)
+    v = BU * torch.tanh(torch.einsum("tkhl,tl->tkh", t["Wu"][idx], xl) / BU)
+    F = torch.einsum("tkmh,tkh->tkm", t["Wd"][idx], torch.nn.functional.silu(g) * v)
+    m = (a.unsqueeze(-1) * F).sum(1)
+    mh = m / torch.sqrt((m * m).mean(1, keepdim=True) + eps)
+    y = mh @ t["Wupp"].T
+    for j in range(NSH):
+        hs = torch.nn.functional.silu(x @ t["Sg"][j].T) * (x @ t["Su"][j].T)
+        y = y + hs @ t["Sd"][j].T
+    L = (torch.tensor(c["dy"]) * y).sum()
+    L.backward()
+    out = {n: t[n].grad.numpy() for n in t}
+    out["z"] = z.grad.numpy()
+    return float(L.detach()), y.detach().numpy(), out
+
+
+@pytest.mark.parametrize("renorm", [1, 0])
+@pytest.mark.parametrize("eps", [1e-6, 0.3])
+def test_latent_backward_matches_autograd(renorm, eps):
+    c = _latent_case(61 + renorm, renorm)
+    L, y = _latent(c, eps, oracle.latent_loss)
+    g = _latent(c, eps, oracle.latent_backward)
+    tL, ty, tg = _latent_torch(c, eps)
+    assert abs(L - tL) <= 1e-12 * max(1.0, abs(tL))
+    _close(y, ty)
+    for ours, theirs in (("dz", "z"), ("dx", "x"), ("dWr", "Wr"), ("dWdp", "Wdp"),
+                         ("dWupp", "Wupp"), ("dWg", "Wg"), ("dWu", "Wu"), ("dWd", "Wd"),
+                         ("dSg", "Sg"), ("dSu", "Su"), ("dSd", "Sd")):
+        _close(g[ours], tg[theirs])
+
+
+def test_latent_loss_forward_is_the_pinned_pieces():
+    """The loss's forward composed from the pinned oracle pieces: the matvec,
+    the SiTU-GLU expert, RMSNorm and numpy's softmax."""
+    c = _latent_case(71)
+    eps = 1e-6
+    _, y = _latent(c, eps, oracle.latent_loss)
+    for t in range(c["x"].shape[0]):
+        z = c["Wr"] @ c["x"][t]
+        p = np.exp(z - z.max())
+        p /= p.sum()
+        sel = c["idx"][t]
+        a = p[sel] / p[sel].sum()
+        xl = oracle.matvec(_m64(c["Wdp"]), c["x"][t])
+        m = sum(a[s] * oracle.expert(_m64(c["Wg"][e]), _m64(c["Wu"][e]), _m64(c["Wd"][e]), xl,
+                                     act=1, beta_g=BG, beta_u=BU) for s, e in enumerate(sel))
+        yt = oracle.matvec(_m64(c["Wupp"]), oracle.rmsnorm(m, eps))
+        for j in range(NSH):
+            yt = yt + oracle.expert(_m64(c["Sg"][j]), _m64(c["Su"][j]), _m64(c["Sd"][j]), c["x"][t])
+        _close(y[t], yt, rel=1e-13)
+
+
+def test_latent_backward_central_differences():
+    c = _latent_case(81)
+    eps = 1e-6
+    g = _latent(c, eps, oracle.latent_backward)
+    rng = np.random.default_rng(4)
+    h = 1e-5
+    for name, gname in (("Wg", "dWg"), ("Wd", "dWd"), ("Wr", "dWr"), ("Wdp", "dWdp"),
+                        ("Wupp", "dWupp"), ("Sd", "dSd"), ("x", "dx")):
+        G = g[gname]
+        nz = np.argwhere(np.abs(G) > 1e-3 * np.abs(G).max())
+        for pos in map(tuple, nz[rng.choice(len(nz), size=min(8, len(nz)), replace=False)]):
+            cp, cm = dict(c), dict(c)
+            cp[name], cm[name] = c[name].copy(), c[name].copy()
+            cp[name][pos] += h
+            cm[name][pos] -= h
+            fd = (_latent(cp, eps, oracle.latent_loss)[0] -
+                  _latent(cm, eps, oracle.latent_loss)[0]) / (2 * h)
+            assert abs(fd - G[pos]) <= 1e-6 * np.abs(G).max(), (name, pos, fd, G[pos])
+
+
+def test_latent_only_selected_experts_receive_gradient():
+    """Stable LatentMoE demo document, forward-contract tab: only the selected
+    routed experts receive gradient."""
+    c = _latent_case(91)
+    c["idx"][:, 0] = 0
+    c["idx"][:, 1] = np.where(np.arange(7) % 2 == 0, 1, 2)
+    g = _latent(c, 1e-6, oracle.latent_backward)
+    for e in range(LN):
+        used = e in (0, 1, 2)
+        for n in ("dWg", "dWu", "dWd"):
+            assert bool(np.abs(g[n][e]).max() > 0) == used, (n, e)
+
+
+def test_latent_rmsnorm_makes_the_routed_scale_a_null_direction():
+    """Stable LatentMoE demo document, RMSNorm tab: with RMSNorm before the
+    up-projection the output does not depend on the routed experts' scale.
+    With eps = 0, y(c W_down) = y(W_down) for every c > 0, so the derivative
+    along W_down itself, sum(dW_down * W_down), is zero; W_upp and the shared
+    W_down enter linearly, so their Euler sums add up to the loss."""
+    c = _latent_case(101)
+    L, _ = _latent(c, 0.0, oracle.latent_loss)
+    g = _latent(c, 0.0, oracle.latent_backward)
+    scale = np.abs(g["dWd"]).max() * np.abs(c["Wd"]).max() * c["Wd"].size
+    assert abs(np.sum(g["dWd"] * c["Wd"])) <= 1e-12 * scale
+    euler = np.sum(g["dWupp"] * c["Wupp"]) + np.sum(g["dSd"] * c["Sd"])
+    assert abs(euler - L) <= 1e-12 * max(1.0, abs(L))
+    # with a positive eps the scale is no longer a null direction
+    g2 = _latent(c, 0.3, oracle.latent_backward)
+    assert abs(np.sum(g2["dWd"] * c["Wd"])) > 1e-6
