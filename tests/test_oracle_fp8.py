@@ -132,3 +132,31 @@ def test_fp8_expert_error_matches_the_e4m3_estimate(seed):
     fp8 = oracle.expert(q8(Wg), q8(Wu), q8(Wd), x8, act=1, beta_g=4.0, beta_u=25.0, round_h=2)
     rel = np.sqrt(np.mean((fp8 - exact) ** 2)) / np.sqrt(np.mean(exact ** 2))
     assert 0.03 < rel < 0.10, rel
+
+
+def test_fp8_latent_layer_routes_the_same_and_stays_within_e4m3_error():
+    """The FP8 form of the LatentMoE layer: routing (fp32, on x) is unchanged,
+    and the output stays within a few percent of the bf16 layer's rms.  The
+    routed branch's E4M3 error (about 6.5% of its rms) is divided by RMSNorm's
+    scale and added to the unchanged shared experts."""
+    rng = np.random.default_rng(5)
+    N, d, l, h, sh, T, k = 6, 64, 32, 48, 40, 6, 2
+
+    def bf(rows, cols, sig=0.2):
+        v = (rng.standard_normal((rows, cols)) * sig).astype(np.float32)
+        return oracle.Mat(oracle.BF16, rows, cols, data=v.view(np.uint32) >> 16)
+
+    experts = [(bf(h, l), bf(h, l), bf(l, h)) for _ in range(N)]
+    q8 = lambda m: oracle.e4m3_mat(*oracle.quant_e4m3_rows(m.decode().astype(np.float32)))  # noqa
+    experts8 = [tuple(q8(m) for m in trip) for trip in experts]
+    shared = [(bf(sh, d), bf(sh, d), bf(d, sh)) for _ in range(2)]
+    W_dp, W_upp = bf(l, d), bf(d, l)
+    w_route = rng.standard_normal((N, d)).astype(np.float32)
+    x = (rng.standard_normal((T, d)).astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
+    i16, w16, y16 = oracle.latent_tokens(x, w_route, k, W_dp, lambda e: experts[e], W_upp,
+                                         shared, 4.0, 25.0, 1e-6)
+    i8, w8, y8 = oracle.latent_tokens(x, w_route, k, W_dp, lambda e: experts8[e], W_upp, shared,
+                                      4.0, 25.0, 1e-6, fp8=True)
+    assert np.array_equal(i16, i8) and np.array_equal(w16, w8)
+    rel = np.sqrt(np.mean((y8 - y16) ** 2)) / np.sqrt(np.mean(y16 ** 2))
+    assert 1e-3 < rel < 0.1, rel
