@@ -316,6 +316,68 @@ def run_cpu_baseline(wl: W.Workload, host, budget_s: float = 12.0):
     return done / el, el, n
 
 
+def decode_cpu_baseline(wl: W.Workload, budget_s: float = 12.0):
+    """The oracle on the host cores for the decode workload: every layer of a
+    step for random samples of the batch's tokens (the tokens of a decode
+    batch are independent of one another).  Returns (tokens/s, seconds, sample)."""
+    import oracle as O
+    N, d, h = wl.N, wl.d, wl.h
+    layers = []
+    for layer in range(wl.n_layers):
+        wr = S.normal(wl.seed, W.tid(W.TID_WROUTE, layer), (N, d), W.SIGMA_W, S.DT_F32)
+        planes = []
+        for base, rows, cols in ((W.TID_WGATE, h, d), (W.TID_WUP, h, d), (W.TID_WDOWN, d, h)):
+            hq, hs = S.q4(wl.seed, W.tid(base, layer), N * rows, cols)
+            planes.append([O.Mat(O.Q4_0, rows, cols, qs=hq[e * rows:(e + 1) * rows],
+                                 scales=hs[e * rows:(e + 1) * rows]) for e in range(N)])
+        layers.append((wr, list(zip(*planes))))
+    u0 = S.normal(wl.seed, W.TID_U, (wl.T, d), 1.0, S.DT_F16)
+    n = min(wl.T, 4)
+    rng = np.random.default_rng(0)
+    done, t0 = 0, time.perf_counter()
+    while True:
+        u = u0[np.sort(rng.choice(wl.T, n, replace=False))]
+        for wr, mats in layers:
+            u = O.decode_layer(u, wr, mats, wl.k)[3]
+        done += n
+        el = time.perf_counter() - t0
+        if el >= budget_s:
+            return done / el, el, n
+
+
+def latent_cpu_baseline(wl: W.Workload, budget_s: float = 12.0):
+    """The oracle on the host cores for the LatentMoE workload, one random
+    token per sample.  The sampled token's 16 routed experts are generated
+    before its timed pass (generation is not oracle work)."""
+    import oracle as O
+    from inputs import host_latent_dense, host_latent_expert
+    W_dp, W_upp, shared = host_latent_dense(wl)
+    w_route = S.normal(wl.seed, W.TID_WROUTE, (wl.N, wl.d), W.SIGMA_W, S.DT_F32)
+    x_all = S.rmsnorm_rows(wl.seed, W.TID_U, wl.T, wl.d, S.DT_BF16)
+    rng = np.random.default_rng(0)
+    done, timed = 0, 0.0
+    while timed < budget_s:
+        x = x_all[[int(rng.integers(wl.T))]]
+        _, _, idx, _ = O.route(O.as_f32(O.BF16, x), w_route, wl.k)
+        experts = {int(e): host_latent_expert(wl, int(e)) for e in idx[0]}
+        t0 = time.perf_counter()
+        O.latent_tokens(x, w_route, wl.k, W_dp, experts.__getitem__, W_upp, shared,
+                        wl.beta_gate, wl.beta_up, 1e-6)
+        timed += time.perf_counter() - t0
+        done += 1
+    return done / timed, timed, 1
+
+
+def latent_launches(wl: W.Workload) -> int:
+    """Kernels moe_latent_fwd launches for a LatentMoE workload with more than
+    16 routed experts (the library's path restated): router logits and top-k,
+    the three permutation kernels, x_l = W_dp x, the gather, routed gate/up,
+    routed down, the combine, RMSNorm, the shared experts' gate/up when there
+    are shared experts, and the output GEMM."""
+    assert wl.N > 16
+    return 2 + 3 + 1 + 1 + 1 + 1 + 1 + 1 + (1 if wl.n_shared > 0 else 0) + 1
+
+
 def reference_arm(args, wl):
     """--impl reference: the CPU oracle timed on this machine's host cores."""
     host = oracle_host_inputs(wl)
@@ -457,6 +519,12 @@ def decode_main(args, wl, torch, moe, rank, world, dist):
     eb.record(stream)
     torch.cuda.synchronize()
     e_ms = max_over_ranks(ea.elapsed_time(eb), dist, "cuda")
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, el_s, n = decode_cpu_baseline(wl)
+        cpu = {"value": v, "unit": "tokens/s", "cores": os.cpu_count(), "kind": "oracle",
+               "sample": f"random samples of {n} tokens through all {wl.n_layers} layers, "
+                         f"{el_s:.1f} s of CPU work"}
     if rank == 0:
         line = {"metric": METRIC, "value": whole_job_rate(wl.T, args.steps, world, ms),
                 "unit": "tokens/s",
@@ -475,7 +543,7 @@ def decode_main(args, wl, torch, moe, rank, world, dist):
                                        "cooperative launch",
                              "bytes_per_step": bytes_timed / args.steps,
                              "peak_source": f"{src} hbm_gbs"},
-                "cpu_baseline": None,
+                "cpu_baseline": cpu,
                 "e2e": {"value": tokens / (e_ms / 1e3), "unit": "tokens/s",
                         "h2d_bytes_per_step": wl.T * wl.d * 2,
                         "d2h_bytes_per_step": wl.T * wl.d * 2},
@@ -578,6 +646,12 @@ def latent_main(args, wl, torch, moe, rank, world, dist):
     torch.cuda.synchronize()
     e_ms = max_over_ranks(ea.elapsed_time(eb), dist, "cuda")
     tokens = wl.T * args.steps * world
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, el_s, n = latent_cpu_baseline(wl)
+        cpu = {"value": v, "unit": "tokens/s", "cores": os.cpu_count(), "kind": "oracle",
+               "sample": f"random single tokens of the latent batch, {el_s:.1f} s of "
+                         "oracle work (their routed experts generated untimed)"}
     if rank == 0:
         line = {"metric": METRIC, "value": whole_job_rate(wl.T, args.steps, world, ms),
                 "unit": "tokens/s",
@@ -596,10 +670,10 @@ def latent_main(args, wl, torch, moe, rank, world, dist):
                              "bytes_per_step": step_bytes,
                              "tflops": flops / per_step_s / 1e12,
                              "peak_source": f"{src} hbm_gbs"},
-                "cpu_baseline": None,
+                "cpu_baseline": cpu,
                 "e2e": {"value": tokens / (e_ms / 1e3), "unit": "tokens/s",
                         "h2d_bytes_per_step": wl.T * d * 2, "d2h_bytes_per_step": wl.T * d * 2},
-                "gpu_launches": None, "clocks": clocks}
+                "gpu_launches": latent_launches(wl) * args.steps, "clocks": clocks}
         print(json.dumps(line), flush=True)
 
 
