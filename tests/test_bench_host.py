@@ -1,0 +1,31 @@
+"""Host-side pieces of bench.py that need no GPU: the oracle CPU baselines of
+the decode and LatentMoE workloads (on shrunken shapes) and the LatentMoE
+launch count."""
+import dataclasses
+import os
+import sys
+
+from conftest import ROOT
+
+sys.path.insert(0, os.path.join(ROOT, "tests"))
+
+import bench  # noqa: E402
+from synthetic import workloads as W  # noqa: E402
+
+
+def test_decode_cpu_baseline_runs_a_bounded_sample():
+    wl = W.decode(T=8, n_layers=2)
+    rate, seconds, n = bench.decode_cpu_baseline(wl, budget_s=0.2)
+    assert rate > 0 and seconds >= 0.2 and n == 4
+
+
+def test_latent_cpu_baseline_runs_a_bounded_sample():
+    wl = dataclasses.replace(W.latent(T=64), N=32, d=256, latent=128, h=128, shared_hidden=128)
+    rate, seconds, n = bench.latent_cpu_baseline(wl, budget_s=0.2)
+    assert rate > 0 and seconds >= 0.2 and n == 1
+
+
+def test_latent_launch_count_matches_the_profiled_list():
+    # 13 kernels per step in the committed LatentMoE launch list
+    assert bench.latent_launches(W.latent()) == 13
+    assert bench.latent_launches(dataclasses.replace(W.latent(), n_shared=0)) == 12
