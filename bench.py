@@ -302,6 +302,23 @@ def cpu_sample_tokens(wl: W.Workload) -> int:
     return int(max(16, min(wl.T, 2.0e10 / per_token)))
 
 
+def cpu_model() -> str:
+    """The host CPU's model name, for the baseline line."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.startswith("model name"):
+                    return ln.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def oracle_threads() -> int:
+    import oracle as O
+    return O.threads()
+
+
 def run_cpu_baseline(wl: W.Workload, host, budget_s: float = 12.0):
     n = cpu_sample_tokens(wl)
     rng = np.random.default_rng(0)
@@ -392,7 +409,7 @@ def reference_arm(args, wl):
         oracle_pass(wl, host, samples[args.warmup + i])
     el = time.perf_counter() - t0
     value = n * args.steps / el
-    cores = os.cpu_count()
+    cores = oracle_threads()
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": el / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
@@ -522,7 +539,8 @@ def decode_main(args, wl, torch, moe, rank, world, dist):
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, el_s, n = decode_cpu_baseline(wl)
-        cpu = {"value": v, "unit": "tokens/s", "cores": os.cpu_count(), "kind": "oracle",
+        cpu = {"value": v, "unit": "tokens/s", "cores": min(n, oracle_threads()), "kind": "oracle",
+               "cpu": cpu_model(),
                "sample": f"random samples of {n} tokens through all {wl.n_layers} layers, "
                          f"{el_s:.1f} s of CPU work"}
     if rank == 0:
@@ -649,7 +667,7 @@ def latent_main(args, wl, torch, moe, rank, world, dist):
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, el_s, n = latent_cpu_baseline(wl)
-        cpu = {"value": v, "unit": "tokens/s", "cores": os.cpu_count(), "kind": "oracle",
+        cpu = {"value": v, "unit": "tokens/s", "cores": 1, "kind": "oracle", "cpu": cpu_model(),
                "sample": f"random single tokens of the latent batch, {el_s:.1f} s of "
                          "oracle work (their routed experts generated untimed)"}
     if rank == 0:
@@ -843,7 +861,13 @@ def main():
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         host = oracle_host_inputs(wl)
         v, el_s, n = run_cpu_baseline(wl, host)
-        cpu = {"value": v, "unit": "tokens/s", "cores": os.cpu_count(), "kind": "oracle",
+        import oracle as O
+        threads = O.threads()
+        O.set_threads(1)
+        v1, _, _ = run_cpu_baseline(wl, host, budget_s=6.0)
+        O.set_threads(threads)
+        cpu = {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+               "one_thread_value": v1, "cpu": cpu_model(),
                "sample": f"random samples of {n} tokens of the {wl.name} batch, "
                          f"{el_s:.1f} s of CPU work"}
 

@@ -78,6 +78,10 @@ def lib():
         L.or_qb_exact.argtypes = [i64, i64, vp, vp, i64, vp, vp]
         L.or_qb_hist.argtypes = [i64, i64, vp, vp, i64, i64, vp]
         L.or_aux_grad.argtypes = [i64, i64, dbl, vp, vp, vp]
+        L.or_threads.argtypes = []
+        L.or_threads.restype = ctypes.c_int
+        L.or_set_threads.argtypes = [ctypes.c_int]
+        L.or_set_threads.restype = None
         L.or_e4m3_to_f64.argtypes = [ctypes.c_uint8]
         L.or_e4m3_to_f64.restype = dbl
         L.or_round_e4m3.argtypes = [dbl]
@@ -539,3 +543,12 @@ def latent_backward(routed, Wr, W_dp, W_upp, shared, x, top_idx, dy, beta_g, bet
                              *[_p(out[key]) for key in ("dz", "dx", "dWr", "dWdp", "dWupp", "dWg",
                                                         "dWu", "dWd", "dSg", "dSu", "dSd")])
     return out
+
+
+def threads() -> int:
+    """Threads the oracle's OpenMP loops use."""
+    return int(lib().or_threads())
+
+
+def set_threads(n: int):
+    lib().or_set_threads(int(n))

@@ -29,3 +29,16 @@ def test_latent_launch_count_matches_the_profiled_list():
     # 13 kernels per step in the committed LatentMoE launch list
     assert bench.latent_launches(W.latent()) == 13
     assert bench.latent_launches(dataclasses.replace(W.latent(), n_shared=0)) == 12
+
+
+def test_oracle_thread_count_is_reported_and_settable():
+    import oracle as O
+    n = O.threads()
+    assert n >= 1 and bench.oracle_threads() == n
+    O.set_threads(1)
+    try:
+        assert O.threads() == 1
+    finally:
+        O.set_threads(n)
+    assert O.threads() == n
+    assert isinstance(bench.cpu_model(), str)
