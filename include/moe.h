@@ -265,7 +265,10 @@ typedef struct {
 MOE_API size_t moe_latent_workspace_bytes(const moe_shape* shape, const moe_latent_weights* lw);
 /* shape: T tokens, d model width, N routed experts, k, h routed hidden width.
  * w: router [N][d] fp32 (+bias) and the routed experts (bf16, latent width),
- * w->w_dtype == MOE_BF16.  x, y [T][d] bf16.  out: as for moe_layer_fwd. */
+ * w->w_dtype == MOE_BF16.  x, y [T][d] bf16.  out: as for moe_layer_fwd.
+ * Returns MOE_ERR_INVALID_ARG for unsupported widths, NULL or misaligned
+ * pointers or non-positive SiTU-GLU caps, MOE_ERR_UNSUPPORTED for non-bf16
+ * experts, MOE_ERR_WORKSPACE for a short workspace. */
 MOE_API int moe_latent_fwd(const moe_shape* shape, const moe_layer_weights* w,
                            const moe_latent_weights* lw, const void* x, void* y,
                            const moe_layer_outputs* out, void* ws, size_t ws_bytes, void* stream);
@@ -294,7 +297,10 @@ typedef struct {
  * router rows, one phase-A item, the selected experts' down rows of one
  * output slice) within 226 KB.  Returns 0 for shapes outside them.  The
  * workspace holds the hidden vectors, the routing scratch, the chained
- * activations and the grid-barrier words; one call at a time per workspace. */
+ * activations and the grid-barrier words; one call at a time per workspace.
+ * The two decode calls return MOE_ERR_INVALID_ARG for a shape outside these
+ * limits, a NULL weight pointer or a NULL / misaligned activation pointer,
+ * MOE_ERR_WORKSPACE for a short workspace, and MOE_OK at once for T = 0. */
 MOE_API size_t moe_decode_workspace_bytes(const moe_shape* shape);
 
 /* One decode layer: u [T][d] fp16 (bit patterns) -> y [T][d] fp16, the
@@ -333,7 +339,10 @@ MOE_API int moe_decode_step(const moe_shape* shape, int32_t n_layers, const moe_
  *                   through ties).
  * Every step is one fp32 operation in a fixed order (bit-reproducible).
  * Limits: 1 <= T <= 32768, 1 <= N <= 1024, 1 <= k <= min(N, 32),
- * 1 <= q <= T, 0 <= bins <= 4096.  Device pointers, caller-owned. */
+ * 1 <= q <= T, 0 <= bins <= 4096.  Device pointers, caller-owned.
+ * Returns MOE_ERR_INVALID_ARG outside the limits or for NULL scores or
+ * bias_exact, MOE_ERR_WORKSPACE when cutoff is NULL and ws is shorter than
+ * moe_quantile_balance_workspace_bytes(T, N). */
 MOE_API size_t moe_quantile_balance_workspace_bytes(int32_t T, int32_t N);
 MOE_API int moe_quantile_balance(int32_t T, int32_t N, int32_t k, const float* scores,
                                  const float* bias, int32_t q, int32_t bins, float* cutoff,
