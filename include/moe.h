@@ -299,7 +299,8 @@ typedef struct {
  * workspace holds the hidden vectors, the routing scratch, the chained
  * activations and the grid-barrier words; one call at a time per workspace.
  * The two decode calls return MOE_ERR_INVALID_ARG for a shape outside these
- * limits, a NULL weight pointer or a NULL / misaligned activation pointer,
+ * limits, a NULL or misaligned weight or activation pointer (q4 planes and
+ * the router 16-byte aligned, scales and bias 4-byte aligned),
  * MOE_ERR_WORKSPACE for a short workspace, and MOE_OK at once for T = 0. */
 MOE_API size_t moe_decode_workspace_bytes(const moe_shape* shape);
 
