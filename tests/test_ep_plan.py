@@ -211,3 +211,41 @@ def test_gloo_ranks_reproduce_the_single_gpu_layer(world):
         T = batches[r][0].shape[0]
         assert np.array_equal(got[r], ref[t0:t0 + T]), f"rank {r}"
         t0 += T
+
+
+def test_plan_invariants_on_random_counts():
+    """For random per-rank counts and capacities: every owner's receive
+    buffer is tiled exactly by the sources' kept rows, send and receive sizes
+    agree pairwise, each expert keeps min(C, all dispatches) rows (all of them
+    for C = 0), and a rank keeps rows for an expert only while the ranks
+    before it left room."""
+    from hypothesis import given, settings, strategies as st
+
+    @settings(max_examples=200, deadline=None)
+    @given(st.integers(1, 4), st.integers(1, 4), st.integers(0, 12), st.data())
+    def check(R, E, C, data):
+        N = R * E
+        counts = np.array(data.draw(st.lists(st.lists(st.integers(0, 9), min_size=N, max_size=N),
+                                             min_size=R, max_size=R)))
+        plans = [ep.plan(counts, C, r) for r in range(R)]
+        kept = np.stack([p.kept for p in plans])
+        tot = counts.sum(0)
+        assert np.array_equal(kept.sum(0), np.minimum(tot, C) if C else tot)
+        assert np.array_equal(plans[0].overflow, tot - kept.sum(0))
+        for r in range(1, R):  # a later rank keeps rows only if the earlier ranks kept all theirs
+            later = kept[r] > 0
+            assert np.array_equal(kept[:r, later], counts[:r, later])
+        for a in range(R):
+            for b in range(R):
+                assert plans[a].send_counts[b] == plans[b].recv_counts[a]
+        for o in range(R):
+            cover = []
+            for r in range(R):
+                for e in range(o * E, (o + 1) * E):
+                    cover += list(range(plans[r].send_base[e], plans[r].send_base[e] + kept[r, e]))
+                    el = e - o * E
+                    assert plans[o].recv_src_base[el, r] == plans[r].send_base[e]
+            assert sorted(cover) == list(range(plans[o].recv_rows))
+            assert plans[o].recv_rows == int(plans[o].recv_counts.sum())
+
+    check()
