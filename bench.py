@@ -333,55 +333,104 @@ def run_cpu_baseline(wl: W.Workload, host, budget_s: float = 12.0):
     return done / el, el, n
 
 
+def workload_label(wl: W.Workload) -> str:
+    """The workload as both bench arms name it in config.workload."""
+    if wl.name == "decode":
+        return (f"decode: T={wl.T} d={wl.d} N={wl.N} h={wl.h} top-{wl.k}, "
+                f"{wl.n_layers} layers per step")
+    if wl.name == "latent":
+        return (f"latent: T={wl.T} d={wl.d} l={wl.latent} E={wl.N} H={wl.h} top-{wl.k}, "
+                f"{wl.n_shared} shared of hidden {wl.shared_hidden}, "
+                f"caps {wl.beta_gate:g}/{wl.beta_up:g}")
+    return f"{wl.name}: T={wl.T} d={wl.d} N={wl.N} h={wl.h} top-{wl.k}"
+
+
+class DecodeOracle:
+    """The decode workload's host weights (every layer, q4_0) and one oracle
+    sample: random tokens of the batch through all layers (the tokens of a
+    decode batch are independent of one another)."""
+
+    def __init__(self, wl: W.Workload):
+        import oracle as O
+        self.O, self.wl = O, wl
+        N, d, h = wl.N, wl.d, wl.h
+        self.layers = []
+        for layer in range(wl.n_layers):
+            wr = S.normal(wl.seed, W.tid(W.TID_WROUTE, layer), (N, d), W.SIGMA_W, S.DT_F32)
+            planes = []
+            for base, rows, cols in ((W.TID_WGATE, h, d), (W.TID_WUP, h, d), (W.TID_WDOWN, d, h)):
+                hq, hs = S.q4(wl.seed, W.tid(base, layer), N * rows, cols)
+                planes.append([O.Mat(O.Q4_0, rows, cols, qs=hq[e * rows:(e + 1) * rows],
+                                     scales=hs[e * rows:(e + 1) * rows]) for e in range(N)])
+            self.layers.append((wr, list(zip(*planes))))
+        self.u0 = S.normal(wl.seed, W.TID_U, (wl.T, d), 1.0, S.DT_F16)
+        self.n = min(wl.T, 4)
+
+    def sample(self, rng) -> int:
+        u = self.u0[np.sort(rng.choice(self.wl.T, self.n, replace=False))]
+        for wr, mats in self.layers:
+            u = self.O.decode_layer(u, wr, mats, self.wl.k)[3]
+        return self.n
+
+
+def _tests_on_path():
+    """The host-side input helpers shared with the tests live in tests/."""
+    path = os.path.join(ROOT, "tests")
+    if path not in sys.path:
+        sys.path.insert(0, path)
+
+
+class LatentOracle:
+    """The LatentMoE workload's dense host weights; one oracle sample is one
+    random token, whose 16 routed experts prepare() generates untimed
+    (generation is not oracle work; 59 GB of experts never sit on the host)."""
+
+    def __init__(self, wl: W.Workload):
+        import oracle as O
+        _tests_on_path()
+        from inputs import host_latent_dense
+        self.O, self.wl = O, wl
+        self.W_dp, self.W_upp, self.shared = host_latent_dense(wl)
+        self.w_route = S.normal(wl.seed, W.TID_WROUTE, (wl.N, wl.d), W.SIGMA_W, S.DT_F32)
+        self.x_all = S.rmsnorm_rows(wl.seed, W.TID_U, wl.T, wl.d, S.DT_BF16)
+
+    def prepare(self, rng):
+        from inputs import host_latent_expert
+        x = self.x_all[[int(rng.integers(self.wl.T))]]
+        _, _, idx, _ = self.O.route(self.O.as_f32(self.O.BF16, x), self.w_route, self.wl.k)
+        return x, {int(e): host_latent_expert(self.wl, int(e)) for e in idx[0]}
+
+    def run(self, prepared) -> int:
+        x, experts = prepared
+        self.O.latent_tokens(x, self.w_route, self.wl.k, self.W_dp, experts.__getitem__,
+                             self.W_upp, self.shared, self.wl.beta_gate, self.wl.beta_up, 1e-6)
+        return 1
+
+
 def decode_cpu_baseline(wl: W.Workload, budget_s: float = 12.0):
-    """The oracle on the host cores for the decode workload: every layer of a
-    step for random samples of the batch's tokens (the tokens of a decode
-    batch are independent of one another).  Returns (tokens/s, seconds, sample)."""
-    import oracle as O
-    N, d, h = wl.N, wl.d, wl.h
-    layers = []
-    for layer in range(wl.n_layers):
-        wr = S.normal(wl.seed, W.tid(W.TID_WROUTE, layer), (N, d), W.SIGMA_W, S.DT_F32)
-        planes = []
-        for base, rows, cols in ((W.TID_WGATE, h, d), (W.TID_WUP, h, d), (W.TID_WDOWN, d, h)):
-            hq, hs = S.q4(wl.seed, W.tid(base, layer), N * rows, cols)
-            planes.append([O.Mat(O.Q4_0, rows, cols, qs=hq[e * rows:(e + 1) * rows],
-                                 scales=hs[e * rows:(e + 1) * rows]) for e in range(N)])
-        layers.append((wr, list(zip(*planes))))
-    u0 = S.normal(wl.seed, W.TID_U, (wl.T, d), 1.0, S.DT_F16)
-    n = min(wl.T, 4)
+    """The oracle on the host cores for the decode workload, DecodeOracle
+    samples until the budget is spent.  Returns (tokens/s, seconds, sample)."""
+    ora = DecodeOracle(wl)
     rng = np.random.default_rng(0)
     done, t0 = 0, time.perf_counter()
     while True:
-        u = u0[np.sort(rng.choice(wl.T, n, replace=False))]
-        for wr, mats in layers:
-            u = O.decode_layer(u, wr, mats, wl.k)[3]
-        done += n
+        done += ora.sample(rng)
         el = time.perf_counter() - t0
         if el >= budget_s:
-            return done / el, el, n
+            return done / el, el, ora.n
 
 
 def latent_cpu_baseline(wl: W.Workload, budget_s: float = 12.0):
-    """The oracle on the host cores for the LatentMoE workload, one random
-    token per sample.  The sampled token's 16 routed experts are generated
-    before its timed pass (generation is not oracle work)."""
-    import oracle as O
-    from inputs import host_latent_dense, host_latent_expert
-    W_dp, W_upp, shared = host_latent_dense(wl)
-    w_route = S.normal(wl.seed, W.TID_WROUTE, (wl.N, wl.d), W.SIGMA_W, S.DT_F32)
-    x_all = S.rmsnorm_rows(wl.seed, W.TID_U, wl.T, wl.d, S.DT_BF16)
+    """The oracle on the host cores for the LatentMoE workload, one timed
+    token per sample (its experts generated before the timed pass)."""
+    ora = LatentOracle(wl)
     rng = np.random.default_rng(0)
     done, timed = 0, 0.0
     while timed < budget_s:
-        x = x_all[[int(rng.integers(wl.T))]]
-        _, _, idx, _ = O.route(O.as_f32(O.BF16, x), w_route, wl.k)
-        experts = {int(e): host_latent_expert(wl, int(e)) for e in idx[0]}
+        prepared = ora.prepare(rng)
         t0 = time.perf_counter()
-        O.latent_tokens(x, w_route, wl.k, W_dp, experts.__getitem__, W_upp, shared,
-                        wl.beta_gate, wl.beta_up, 1e-6)
+        done += ora.run(prepared)
         timed += time.perf_counter() - t0
-        done += 1
     return done / timed, timed, 1
 
 
@@ -396,29 +445,52 @@ def latent_launches(wl: W.Workload) -> int:
 
 
 def reference_arm(args, wl):
-    """--impl reference: the CPU oracle timed on this machine's host cores."""
-    host = oracle_host_inputs(wl)
-    n = cpu_sample_tokens(wl) // 4 or 1
-    rng = np.random.default_rng(1)
-    samples = [np.sort(rng.choice(wl.T, n, replace=False)).astype(np.int32)
-               for _ in range(args.warmup + args.steps)]
-    for i in range(args.warmup):
-        oracle_pass(wl, host, samples[i])
-    t0 = time.perf_counter()
-    for i in range(args.steps):
-        oracle_pass(wl, host, samples[args.warmup + i])
-    el = time.perf_counter() - t0
-    value = n * args.steps / el
+    """--impl reference: the CPU oracle timed on this machine's host cores, each
+    step a bounded sample of the workload (W untimed steps first)."""
     cores = oracle_threads()
+    rng = np.random.default_rng(1)
+    if wl.name == "decode":
+        ora = DecodeOracle(wl)
+        for _ in range(args.warmup):
+            ora.sample(rng)
+        t0 = time.perf_counter()
+        n = sum(ora.sample(rng) for _ in range(args.steps))
+        el = time.perf_counter() - t0
+        cores = min(ora.n, cores)
+        sample = f"{ora.n} random tokens through all {wl.n_layers} layers per step"
+    elif wl.name == "latent":
+        ora = LatentOracle(wl)
+        for _ in range(args.warmup):
+            ora.run(ora.prepare(rng))
+        n, el = 0, 0.0
+        for _ in range(args.steps):
+            prepared = ora.prepare(rng)
+            t0 = time.perf_counter()
+            n += ora.run(prepared)
+            el += time.perf_counter() - t0
+        cores = 1
+        sample = "one random token per step (its 16 routed experts generated untimed)"
+    else:
+        host = oracle_host_inputs(wl)
+        m = cpu_sample_tokens(wl) // 4 or 1
+        samples = [np.sort(rng.choice(wl.T, m, replace=False)).astype(np.int32)
+                   for _ in range(args.warmup + args.steps)]
+        for i in range(args.warmup):
+            oracle_pass(wl, host, samples[i])
+        t0 = time.perf_counter()
+        for i in range(args.steps):
+            oracle_pass(wl, host, samples[args.warmup + i])
+        el = time.perf_counter() - t0
+        n = m * args.steps
+        sample = f"{m} random tokens of the {wl.name} batch per step"
+    value = n / el
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": el / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": wl.name, "T": wl.T, "d": wl.d, "N": wl.N, "k": wl.k,
-                       "h": wl.h},
+            "config": {"workload": workload_label(wl)},
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores,
-                             "kind": "oracle",
-                             "sample": f"{n} random tokens of the {wl.name} batch per step"},
+                             "kind": "oracle", "cpu": cpu_model(), "sample": sample},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -550,8 +622,7 @@ def decode_main(args, wl, torch, moe, rank, world, dist):
                 "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "q4_0 weights, fp16 activations, fp32 math",
                 "data": "synthetic",
-                "config": {"workload": f"decode: T={wl.T} d={wl.d} N={wl.N} h={wl.h} "
-                                       f"top-{wl.k}, {wl.n_layers} layers per step",
+                "config": {"workload": workload_label(wl),
                            "global_batch": wl.T * world, "parallelism": f"replicas x{world}",
                            "l2": f"weights rotate over {n_rep} replicas "
                                  f"({n_rep * one.nbytes() / 2**20:.0f} MiB > L2)"},
@@ -572,7 +643,7 @@ def decode_main(args, wl, torch, moe, rank, world, dist):
 
 # ----------------------------------------------------------- latent workload
 def latent_main(args, wl, torch, moe, rank, world, dist):
-    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    _tests_on_path()
     stream = torch.cuda.current_stream()
     st = stream.cuda_stream
     E, d, l, h, n, sh = wl.N, wl.d, wl.latent, wl.h, wl.n_shared, wl.shared_hidden
@@ -676,8 +747,7 @@ def latent_main(args, wl, torch, moe, rank, world, dist):
                 "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
                 "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-                "config": {"workload": f"latent: T={wl.T} d={d} l={l} E={E} H={h} top-{wl.k}, "
-                                       f"{n} shared of hidden {sh}, caps 4/25",
+                "config": {"workload": workload_label(wl),
                            "global_batch": wl.T * world, "parallelism": f"replicas x{world}",
                            "l2": "routed expert weights 59 GB > L2",
                            "experts_touched": used},
@@ -876,8 +946,7 @@ def main():
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
                 "dtype": "bf16" if wl.act_dtype == S.DT_BF16 else "f32", "data": "synthetic",
-                "config": {"workload": f"{wl.name}: T={wl.T} d={wl.d} N={wl.N} h={wl.h} "
-                                       f"top-{wl.k}", "global_batch": wl.T * world,
+                "config": {"workload": workload_label(wl), "global_batch": wl.T * world,
                            "parallelism": f"replicas x{world}",
                            "l2": f"inputs rotate over {n_rep} replicas "
                                  f"({n_rep * one.nbytes() / 2**20:.0f} MiB > L2)",
