@@ -42,3 +42,25 @@ def test_oracle_thread_count_is_reported_and_settable():
         O.set_threads(n)
     assert O.threads() == n
     assert isinstance(bench.cpu_model(), str)
+
+
+def _reference_line(capsys, workload, **kw):
+    import argparse
+    import json
+    wl = W.decode(T=8, n_layers=2) if workload == "decode" else W.ALL[workload](**kw)
+    args = argparse.Namespace(gpus=1, steps=1, warmup=3)
+    bench.reference_arm(args, wl)
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    return wl, line
+
+
+def test_reference_arm_line(capsys):
+    """--impl reference prints the contract's line: the oracle's rate on the
+    same workload label as the GPU arm, with its cpu_baseline and e2e."""
+    for workload, kw in (("decode", {}), ("small", {"T": 512})):
+        wl, line = _reference_line(capsys, workload, **kw)
+        assert line["impl"] == "reference" and line["value"] > 0
+        assert line["config"]["workload"] == bench.workload_label(wl)
+        assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
+        assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["value"] == line["value"]
+        assert line["unit"] == "tokens/s" and line["higher_is_better"] is True
