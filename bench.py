@@ -319,8 +319,8 @@ def oracle_threads() -> int:
     return O.threads()
 
 
-def run_cpu_baseline(wl: W.Workload, host, budget_s: float = 12.0):
-    n = cpu_sample_tokens(wl)
+def run_cpu_baseline(wl: W.Workload, host, budget_s: float = 12.0, n: int = 0):
+    n = n or cpu_sample_tokens(wl)
     rng = np.random.default_rng(0)
     done, t0 = 0, time.perf_counter()
     while True:
@@ -934,7 +934,8 @@ def main():
         import oracle as O
         threads = O.threads()
         O.set_threads(1)
-        v1, _, _ = run_cpu_baseline(wl, host, budget_s=6.0)
+        v1, _, _ = run_cpu_baseline(wl, host, budget_s=6.0,
+                                    n=max(1, cpu_sample_tokens(wl) // threads))
         O.set_threads(threads)
         cpu = {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle",
                "one_thread_value": v1, "cpu": cpu_model(),
