@@ -113,6 +113,7 @@ double or_e4m3_to_f64(uint8_t c) {
 uint8_t or_round_e4m3(double x) {
   if (isnan(x)) return 0x7F;
   uint8_t sign = signbit(x) ? 0x80 : 0x00;
+  if (isinf(x)) return (uint8_t)(sign | 0x7E); /* saturates like any magnitude above 448 */
   double a = fabs(x), bd = INFINITY;
   int best = 0;
   for (int c = 0; c <= 0x7E; ++c) {

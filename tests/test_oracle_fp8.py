@@ -61,8 +61,9 @@ def test_encode_saturates_above_448():
     """Above 448 the oracle saturates (a 'satfinite' conversion); torch agrees
     up to the tie at 464 and returns NaN beyond it, which the quantiser never
     reaches (its quotients stay within 448 times one fp32 rounding)."""
-    x = np.array([448.0, 449.0, 463.9, 464.0, 465.0, 1e6, -1e6])
-    assert list(oracle.round_e4m3(x)) == [0x7E] * 6 + [0xFE]
+    x = np.array([448.0, 449.0, 463.9, 464.0, 465.0, 1e6, -1e6, np.inf, -np.inf])
+    assert list(oracle.round_e4m3(x)) == [0x7E] * 6 + [0xFE, 0x7E, 0xFE]
+    assert oracle.round_e4m3([np.nan])[0] == 0x7F
     assert np.array_equal(oracle.round_e4m3(x[:4]), _torch_encode(x[:4]))
 
 
