@@ -65,3 +65,17 @@ def test_irwin_hall_moments():
     x = S.normal(3, 9, (200000,), 1.0, S.DT_F32).astype(np.float64)
     assert abs(x.mean()) < 0.01 and abs(x.var() - 1.0) < 0.01
     assert np.abs(x).max() <= 6.0
+
+
+def test_q4_scale_classes():
+    """q4_0 test scales: 1/64 zero, 7/64 subnormal (the fp16 subnormal-decode
+    case of the deployment notes), the rest normal in [2^-9, 2^-7), both signs."""
+    _, scales = S.q4(1002, 3, 4096, 512)
+    c = scales.ravel()
+    ex, man = (c >> 10) & 0x1F, c & 0x3FF
+    zero = (c & 0x7FFF) == 0
+    sub = (ex == 0) & (man != 0)
+    normal = (ex == 6) | (ex == 7)
+    assert np.all(zero | sub | normal)
+    assert abs(zero.mean() - 1 / 64) < 0.005 and abs(sub.mean() - 7 / 64) < 0.01
+    assert 0.45 < ((c >> 15) == 1)[normal].mean() < 0.55
