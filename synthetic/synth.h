@@ -63,8 +63,8 @@ SYNTH_HD uint16_t synth_f32_to_bf16_bits(uint32_t u) {
 }
 
 /* q4_0 block scale code (fp16 bit pattern) for global block index gi.
- * One block in eight gets a subnormal scale, one in 64 a zero scale, the rest
- * a normal scale in [2^-9, 2^-7) with a random sign. */
+ * One block in 64 gets a zero scale, 7 in 64 a subnormal scale, the rest a
+ * normal scale in [2^-9, 2^-7) with a random sign. */
 SYNTH_HD uint16_t synth_q4_scale_code(uint64_t key, uint64_t gi) {
   uint64_t h = synth_splitmix64(key ^ 0x5CA1E5ull) ;
   h = synth_splitmix64(h + gi);
