@@ -55,6 +55,10 @@ def profiled_traffic(workload: str):
         return None
     return rec["bytes"]
 L2_BYTES = 126 * 1024 * 1024
+# Nominal B200 figures (dense bf16 tensor cores, HBM3e), the second
+# denominator next to the measured peaks.
+SPEC_BF16_TFLOPS = 2250.0
+SPEC_HBM_GBS = 8000.0
 
 
 def _peaks():
@@ -631,7 +635,8 @@ def decode_main(args, wl, torch, moe, rank, world, dist):
                              "kernel": "decode_persistent: all layers of the step in one "
                                        "cooperative launch",
                              "bytes_per_step": bytes_timed / args.steps,
-                             "peak_source": f"{src} hbm_gbs"},
+                             "peak_source": f"{src} hbm_gbs",
+                             "frac_of_spec": achieved / SPEC_HBM_GBS},
                 "cpu_baseline": cpu,
                 "e2e": {"value": tokens / (e_ms / 1e3), "unit": "tokens/s",
                         "h2d_bytes_per_step": wl.T * wl.d * 2,
@@ -757,7 +762,8 @@ def latent_main(args, wl, torch, moe, rank, world, dist):
                                        "touched expert once)",
                              "bytes_per_step": step_bytes,
                              "tflops": flops / per_step_s / 1e12,
-                             "peak_source": f"{src} hbm_gbs"},
+                             "peak_source": f"{src} hbm_gbs",
+                             "frac_of_spec": achieved / SPEC_HBM_GBS},
                 "cpu_baseline": cpu,
                 "e2e": {"value": tokens / (e_ms / 1e3), "unit": "tokens/s",
                         "h2d_bytes_per_step": wl.T * d * 2, "d2h_bytes_per_step": wl.T * d * 2},
@@ -893,6 +899,7 @@ def main():
                 "kernel": ("tc_fused_ffn (gate/up + SwiGLU + down in one launch, H on chip)"
                            if fused else "tc_grouped_gemm (gate/up + down, 2 launches per step)"),
                 "peak_source": f"{peak_src} bf16_tflops (burst)",
+                "frac_of_spec": achieved_tf / SPEC_BF16_TFLOPS,
                 "ms_per_launch_pair": gemm_s / args.steps * 1e3}
 
     # end to end: pinned host input -> device -> layer -> pinned host output
