@@ -506,6 +506,14 @@ DECODE_LAYERS_PER_LAUNCH = 32  # layer descriptors one decode launch carries
 Q4_EXPERT_BYTES = lambda wl: 3 * wl.h * wl.d // 2 + 3 * wl.h * wl.d // 32 * 2  # qs + fp16 scales
 
 
+def decode_step_bytes(wl: W.Workload, sel) -> int:
+    """Algorithmic HBM bytes of one decode step: per layer the fp32 router,
+    the q4_0 weights of the union of the experts the batch selected (each
+    read once), and the fp16 activations in and out.  sel: [layers][T][k]."""
+    return sum(wl.N * wl.d * 4 + len(np.unique(sel[layer])) * Q4_EXPERT_BYTES(wl)
+               + 2 * wl.T * wl.d * 2 for layer in range(wl.n_layers))
+
+
 class DecodeReplica:
     """24 layers of q4_0 experts (all N experts resident; only selected ones read)."""
 
@@ -564,15 +572,8 @@ def decode_main(args, wl, torch, moe, rank, world, dist):
     for i in range(args.warmup):
         graphs[i % n_rep].replay()
     torch.cuda.synchronize()
-    # algorithmic bytes: router + the union of selected experts + u in/out, per layer
     sel = idx_all.cpu().numpy()
-    ebytes = Q4_EXPERT_BYTES(wl)
-    step_bytes = []
-    for i in range(n_rep):
-        b = 0
-        for l in range(wl.n_layers):
-            b += wl.N * wl.d * 4 + len(np.unique(sel[i, l])) * ebytes + 2 * wl.T * wl.d * 2
-        step_bytes.append(b)
+    step_bytes = [decode_step_bytes(wl, sel[i]) for i in range(n_rep)]
     sampler = ClockSampler(int(os.environ.get("LOCAL_RANK", "0"))) if rank == 0 else None
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if dist:

@@ -64,3 +64,27 @@ def test_reference_arm_line(capsys):
         assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
         assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["value"] == line["value"]
         assert line["unit"] == "tokens/s" and line["higher_is_better"] is True
+
+
+def test_decode_step_bytes_match_the_algorithmic_figures():
+    """Decode roofline bytes per step: 24 layers x (router 16,384 B + 110,592 B
+    per selected q4_0 expert + fp16 activations in and out), so 5.75 MB at one
+    token (two experts per layer) and about 23.2 MB at 32 tokens, where the
+    batch's union covers all 8 experts in every layer (the oracle's routing of
+    the decode batch through each layer's router)."""
+    import numpy as np
+    import oracle as O
+    import synthetic as S
+    assert bench.Q4_EXPERT_BYTES(W.decode(T=1)) == 110592
+    wl1 = W.decode(T=1)
+    sel1 = np.array([[[0, 5]]] * wl1.n_layers)
+    assert bench.decode_step_bytes(wl1, sel1) == 24 * (16384 + 2 * 110592 + 2048) == 5750784
+    wl = W.decode(T=32)
+    sel = []
+    u = S.normal(wl.seed, W.TID_U, (wl.T, wl.d), 1.0, S.DT_F16)
+    for layer in range(wl.n_layers):
+        wr = S.normal(wl.seed, W.tid(W.TID_WROUTE, layer), (wl.N, wl.d), W.SIGMA_W, S.DT_F32)
+        sel.append(O.route(O.as_f32(O.F16, u), wr, wl.k)[2])
+    sel = np.array(sel)
+    assert all(len(np.unique(sel[layer])) == 8 for layer in range(wl.n_layers))
+    assert bench.decode_step_bytes(wl, sel) == 24 * (16384 + 8 * 110592 + 65536) == 23199744
