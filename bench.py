@@ -252,14 +252,10 @@ class Step:
         m.moe_combine(self.s, self.wl.d, self.y_rows, self.row_of, self.top_w, self.y)
 
 
-def _algorithmic(wl: W.Workload, kept_rows: int):
-    """Algorithmic FLOPs and HBM bytes of one step (bf16 weights and activations)."""
-    el = 2 if wl.act_dtype != S.DT_F32 else 4
-    flops_router = 2.0 * wl.T * wl.N * wl.d
-    flops_experts = 6.0 * wl.d * wl.h * kept_rows
-    w_bytes = 3.0 * wl.N * wl.d * wl.h * el
-    act_bytes = 2.0 * wl.T * wl.d * el + wl.N * wl.d * 4
-    return flops_router, flops_experts, w_bytes, act_bytes
+def expert_flops(wl: W.Workload, kept_rows: int) -> float:
+    """FLOPs of the expert GEMMs for kept_rows grouped rows: gate, up and down
+    are three products of 2 d h FLOPs each per row."""
+    return 6.0 * wl.d * wl.h * kept_rows
 
 
 # --------------------------------------------------------------- oracle legs
@@ -891,7 +887,7 @@ def main():
     fused = (wl.h % 64 == 0 and wl.h <= 256 and wl.d % 128 == 0
              and (wl.h // 64 + wl.d // 128) * 64 <= 512)
     kept_timed = [kept[i % n_rep] for i in range(args.steps)]
-    gemm_flops = sum(6.0 * wl.d * wl.h * kr for kr in kept_timed)
+    gemm_flops = sum(expert_flops(wl, kr) for kr in kept_timed)
     gemm_s = sum(ffn_ms) / 1e3
     achieved_tf = gemm_flops / gemm_s / 1e12
     roofline = {"bound": "tensor", "achieved": achieved_tf, "peak": tf_burst, "unit": "TFLOP/s",

@@ -88,3 +88,13 @@ def test_decode_step_bytes_match_the_algorithmic_figures():
     sel = np.array(sel)
     assert all(len(np.unique(sel[layer])) == 8 for layer in range(wl.n_layers))
     assert bench.decode_step_bytes(wl, sel) == 24 * (16384 + 8 * 110592 + 65536) == 23199744
+
+
+def test_small_layer_algorithmic_work():
+    """The small layer's work per step: T (2 N d + k 6 d h) = 3.25 GFLOP with
+    every dispatch kept (no capacity); the roofline counts the expert part."""
+    wl = W.small()
+    experts = bench.expert_flops(wl, wl.T * wl.k)
+    assert experts == 6 * 512 * 128 * 8192
+    router = 2 * wl.T * wl.N * wl.d
+    assert abs((router + experts) / 1e9 - 3.25) < 0.01
