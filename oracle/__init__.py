@@ -151,10 +151,6 @@ def mat_array(mats):
     return arr
 
 
-def bf16_to_f64(code: int) -> float:
-    return lib().or_bf16_to_f64(int(code))
-
-
 def f16_to_f64(code: int) -> float:
     return lib().or_f16_to_f64(int(code))
 

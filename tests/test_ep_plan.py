@@ -75,6 +75,7 @@ def test_plan_matches_global_permutation(R, N, k, C):
             for s in range(k):
                 e = int(idxs[r][t, s])
                 o = p.owner(e)
+                assert o == ep.owner_of(e, N, R)
                 g = int(glob["row_of"][t0 + t, s])
                 if j[t, s] < p.kept[e]:
                     pos = int(p.send_base[e] + j[t, s])
