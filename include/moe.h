@@ -21,6 +21,11 @@
  *     W_down [N][d][h] (the expert-grouped storage of the deployment notes,
  *     "Kestrel-MCU notes 13", §2).
  *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default).
+ *   - Host threads: any entry point may be called from several host threads
+ *     at once (the library's per-device setup is done once, atomically).  Two
+ *     calls whose device work may overlap must not share a workspace, and
+ *     moe_permute_noalloc calls must not overlap at all (one shared scratch).
+ *     The device status word is per device, shared by all streams.
  *   - Return value: MOE_OK (0) or a negative MOE_ERR_*.  Argument errors are
  *     detected on the host, synchronously, before anything is launched.
  *     Errors found by a kernel (an index out of range, a bounded wait that
