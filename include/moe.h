@@ -22,7 +22,8 @@
  *     "Kestrel-MCU notes 13", §2).
  *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default).
  *   - Host threads: any entry point may be called from several host threads
- *     at once (the library's per-device setup is done once, atomically).  Two
+ *     at once (the lazy per-device setup only repeats idempotent attribute
+ *     calls when first calls race).  Two
  *     calls whose device work may overlap must not share a workspace, and
  *     moe_permute_noalloc calls must not overlap at all (one shared scratch).
  *     The device status word is per device, shared by all streams.
