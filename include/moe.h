@@ -23,10 +23,10 @@
  *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default).
  *   - Host threads: any entry point may be called from several host threads
  *     at once (the lazy per-device setup only repeats idempotent attribute
- *     calls when first calls race).  Two
- *     calls whose device work may overlap must not share a workspace, and
- *     moe_permute_noalloc calls must not overlap at all (one shared scratch).
- *     The device status word is per device, shared by all streams.
+ *     calls when first calls race).  Two calls whose device work may overlap
+ *     must not share a workspace, and moe_permute_noalloc calls must not
+ *     overlap at all (one shared scratch).  The device status word is per
+ *     device, shared by all streams.
  *   - Return value: MOE_OK (0) or a negative MOE_ERR_*.  Argument errors are
  *     detected on the host, synchronously, before anything is launched.
  *     Errors found by a kernel (an index out of range, a bounded wait that
