@@ -356,6 +356,36 @@ MOE_API int moe_quantile_balance(int32_t T, int32_t N, int32_t k, const float* s
                                  float* bias_exact, float* bias_hist, int32_t* loads, void* ws,
                                  size_t ws_bytes, void* stream);
 
+/* -------------------------------------------------- expert parallelism */
+/* Exchange plan of expert parallelism, host only (no device work).  world
+ * ranks, N experts, expert e held by rank e / (N / world).  An expert's
+ * capacity counts the dispatches of all ranks in one global order (rank 0's
+ * tokens first, then rank 1's, each in token order), so the expert-parallel
+ * layer equals the single-device layer (tutorial §3.5, §3.6, §3.8) on the
+ * ranks' batches laid end to end.  Input, host:
+ *   counts_all [world][N]  every rank's dispatches per expert, before capacity
+ *                          (each rank's moe_permute counts with capacity 0)
+ * Outputs for `rank`, host, all overwritten (E = N / world):
+ *   kept [N]            my dispatches to e that fit: the first kept[e] of my
+ *                       run of dispatches to e in token order
+ *   local_offsets [N+1] my grouped layout of kept rows (exclusive prefix)
+ *   send_base [N]       row of the owner's receive buffer where my kept rows
+ *                       for e start; my j-th kept dispatch to e lands there + j
+ *   send_counts [world] rows I send to each rank (its experts, in order)
+ *   recv_offsets [E+1]  my receive buffer grouped by my local experts, then by
+ *                       source rank, then by the source's token order
+ *   recv_src_base [E][world]  row where source r's rows for local expert el
+ *                       start (results go back from there)
+ *   recv_counts [world] rows I receive from each rank
+ *   overflow [N]        (nullable) dropped dispatches of all ranks per expert
+ * Returns MOE_ERR_INVALID_ARG when N % world != 0, rank or capacity is out
+ * of range, a count is negative, a pointer is NULL, or a row count exceeds
+ * 2^31 - 1. */
+MOE_API int moe_ep_plan(int32_t world, int32_t rank, int32_t N, int32_t capacity,
+                        const int32_t* counts_all, int32_t* kept, int32_t* local_offsets,
+                        int32_t* send_base, int32_t* send_counts, int32_t* recv_offsets,
+                        int32_t* recv_src_base, int32_t* recv_counts, int32_t* overflow);
+
 /* ----------------------------------------------------------- diagnostics */
 /* Human-readable name of a status code (static string). */
 MOE_API const char* moe_status_string(int32_t status);

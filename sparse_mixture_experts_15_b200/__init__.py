@@ -87,6 +87,7 @@ _PROTOS = {
     "moe_quantile_balance_workspace_bytes": (_sz, [_i32, _i32]),
     "moe_quantile_balance": (_i32, [_i32, _i32, _i32, _vp, _vp, _i32, _i32, _vp, _vp, _vp, _vp,
                                     _vp, _sz, _vp]),
+    "moe_ep_plan": (_i32, [_i32, _i32, _i32, _i32] + [_vp] * 9),
     "moe_status_string": (ctypes.c_char_p, [_i32]),
     "moe_device_status": (_i32, [_vp, ctypes.POINTER(_i32)]),
     "moe_reset_device_status": (_i32, [_vp]),
@@ -410,6 +411,29 @@ def moe_quantile_balance(scores, k: int, q: int, bias_exact, bias=None, bins: in
     _check(_lib.moe_quantile_balance(T, N, k, _ptr(scores), _ptr(bias), q, bins, _ptr(cutoff),
                                      _ptr(bias_exact), _ptr(bias_hist), _ptr(loads), _ptr(wbuf),
                                      wlen, _stream(stream)), "moe_quantile_balance")
+
+
+def moe_ep_plan(counts_all, capacity: int, rank: int) -> dict:
+    """Host-only exchange plan of expert parallelism: counts_all [world][N]
+    (every rank's dispatches per expert) -> this rank's plan arrays (numpy
+    int32): kept, local_offsets, send_base, send_counts, recv_offsets,
+    recv_src_base [E][world], recv_counts, overflow."""
+    import numpy as np
+    c = np.ascontiguousarray(counts_all, dtype=np.int32)
+    if c.ndim != 2:
+        raise ValueError("counts_all must be [world][N]")
+    world, N = c.shape
+    E = N // world if world else 0
+    out = dict(kept=np.empty(N, np.int32), local_offsets=np.empty(N + 1, np.int32),
+               send_base=np.empty(N, np.int32), send_counts=np.empty(world, np.int32),
+               recv_offsets=np.empty(E + 1, np.int32),
+               recv_src_base=np.empty((E, world), np.int32),
+               recv_counts=np.empty(world, np.int32), overflow=np.empty(N, np.int32))
+    order = ("kept", "local_offsets", "send_base", "send_counts", "recv_offsets",
+             "recv_src_base", "recv_counts", "overflow")
+    _check(_lib.moe_ep_plan(world, rank, N, capacity, c.ctypes.data,
+                            *[out[key].ctypes.data for key in order]), "moe_ep_plan")
+    return out
 
 
 def moe_device_status(stream=None) -> int:

@@ -44,7 +44,7 @@ class EpPlan:
     rank: int
     world: int
     experts_per_rank: int
-    kept: np.ndarray           # [N] int64
+    kept: np.ndarray           # [N] int32
     local_offsets: np.ndarray  # [N + 1]
     send_base: np.ndarray      # [N]
     send_counts: np.ndarray    # [R]
@@ -69,41 +69,21 @@ def owner_of(e: int, N: int, world: int) -> int:
 def plan(counts_all, capacity: int, rank: int) -> EpPlan:
     """The exchange plan of `rank` from every rank's per-expert dispatch
     counts counts_all [R][N] (before capacity) and the per-expert capacity C
-    (0 = unlimited).  Pure integer arithmetic; every rank derives the same
-    global picture from the same counts."""
-    c = np.asarray(counts_all, dtype=np.int64)
+    (0 = unlimited), computed by the library's host-only moe_ep_plan.  Every
+    rank derives the same global picture from the same counts."""
+    from . import moe_ep_plan
+    c = np.asarray(counts_all)
     if c.ndim != 2:
         raise ValueError("counts_all must be [world][N]")
     R, N = c.shape
     if R < 1 or N % R != 0 or not 0 <= rank < R:
-        raise ValueError(f"{N} experts do not split over {R} ranks")
+        raise ValueError(f"{N} experts do not split over {R} ranks, or rank {rank} is out of range")
     if capacity < 0 or (c < 0).any():
         raise ValueError("negative capacity or count")
-    E = N // R
-    # global order per expert: rank 0's dispatches first, then rank 1's, ...
-    before = np.cumsum(c, axis=0) - c                    # [R][N] dispatches of lower ranks
-    if capacity > 0:
-        kept_all = np.clip(capacity - before, 0, c)      # [R][N]
-    else:
-        kept_all = c.copy()
-    kept_before = np.cumsum(kept_all, axis=0) - kept_all  # [R][N] kept rows of lower ranks
-    kept_tot = kept_all.sum(axis=0)                      # [N]
-    # each owner's receive buffer: its experts in order, each all sources
-    expert_base = np.zeros(N, np.int64)                  # first row of expert e at its owner
-    for o in range(R):
-        seg = kept_tot[o * E:(o + 1) * E]
-        expert_base[o * E:(o + 1) * E] = np.cumsum(seg) - seg
-    kept = kept_all[rank]
-    local_offsets = np.concatenate([[0], np.cumsum(kept)]).astype(np.int64)
-    send_base = expert_base + kept_before[rank]
-    send_counts = kept.reshape(R, E).sum(axis=1)
-    mine = slice(rank * E, (rank + 1) * E)
-    recv_offsets = np.concatenate([[0], np.cumsum(kept_tot[mine])]).astype(np.int64)
-    recv_src_base = (expert_base[mine][:, None] + kept_before[:, mine].T)  # [E][R]
-    recv_counts = kept_all[:, mine].sum(axis=1)
-    overflow = c.sum(axis=0) - kept_tot
-    return EpPlan(rank, R, E, kept, local_offsets, send_base, send_counts, recv_offsets,
-                  recv_src_base, recv_counts, overflow)
+    p = moe_ep_plan(c, capacity, rank)
+    return EpPlan(rank, R, N // R, p["kept"], p["local_offsets"], p["send_base"],
+                  p["send_counts"], p["recv_offsets"], p["recv_src_base"], p["recv_counts"],
+                  p["overflow"])
 
 
 def exchange_counts(counts_local, group=None):

@@ -201,3 +201,21 @@ def test_binding_refuses_other_element_types():
     with pytest.raises(ValueError, match="top_idx: dtype int64"):
         moe.moe_permute(s, torch.zeros((16, 2), dtype=torch.int64),
                         *[torch.zeros(64, dtype=torch.int32)] * 6)
+
+
+def test_ep_plan_host_checks():
+    """moe_ep_plan is host only: bad arguments return MOE_ERR_INVALID_ARG."""
+    import numpy as np
+    lib = moe._lib
+    c = np.array([[3, 0, 2, 1], [1, 4, 0, 2]], np.int32)
+    bufs = [np.zeros(64, np.int32) for _ in range(8)]
+    ptrs = [b.ctypes.data for b in bufs]
+    assert lib.moe_ep_plan(2, 0, 4, 3, c.ctypes.data, *ptrs) == 0
+    assert lib.moe_ep_plan(3, 0, 4, 3, c.ctypes.data, *ptrs) == -1   # 4 experts over 3 ranks
+    assert lib.moe_ep_plan(2, 2, 4, 3, c.ctypes.data, *ptrs) == -1   # rank out of range
+    assert lib.moe_ep_plan(2, 0, 4, -1, c.ctypes.data, *ptrs) == -1  # negative capacity
+    assert lib.moe_ep_plan(2, 0, 4, 3, None, *ptrs) == -1
+    neg = c.copy()
+    neg[1, 2] = -1
+    assert lib.moe_ep_plan(2, 0, 4, 3, neg.ctypes.data, *ptrs) == -1
+    assert lib.moe_ep_plan(2, 0, 4, 3, c.ctypes.data, *ptrs[:7], None) == 0  # overflow optional
