@@ -57,6 +57,15 @@ int main(void) {
   if (moe_permute_workspace_bytes(&s) == 0) return 15;
   if (moe_quantile_balance(0, 8, 2, NULL, NULL, 1, 0, NULL, NULL, NULL, NULL, NULL, 0, NULL)
       != MOE_ERR_INVALID_ARG) return 16;
+  /* the expert-parallel exchange plan is host only */
+  const int32_t counts[2][4] = {{3, 0, 2, 1}, {1, 4, 0, 2}};
+  int32_t kept[4], loff[5], sbase[4], scnt[2], roff[3], rsrc[2][2], rcnt[2], ovf[4];
+  if (moe_ep_plan(2, 1, 4, 3, &counts[0][0], kept, loff, sbase, scnt, roff, &rsrc[0][0], rcnt,
+                  ovf) != MOE_OK)
+    return 17;
+  if (kept[1] != 3 || kept[3] != 2 || sbase[0] != 3 || roff[2] != 5 || rsrc[1][1] != 3 ||
+      ovf[0] != 1)
+    return 18;
   printf("ok\n");
   return 0;
 }
