@@ -260,6 +260,27 @@ def test_permute_brute_force(T, N, k, C):
     assert int(out["totals"][2]) == (np.maximum(C - L, 0).sum() if C else 0)
 
 
+def test_permute_brute_force_random_shapes():
+    """The same comparison over random shapes, capacities and expert sets
+    (distinct experts per token, any order), including empty experts."""
+    from hypothesis import given, settings, strategies as st
+
+    @settings(max_examples=150, deadline=None)
+    @given(st.integers(1, 60), st.integers(1, 10), st.data())
+    def check(T, N, data):
+        k = data.draw(st.integers(1, N))
+        C = data.draw(st.integers(0, 2 * T))
+        seed = data.draw(st.integers(0, 2**31 - 1))
+        rng = np.random.default_rng(seed)
+        idx = np.stack([rng.permutation(N)[:k] for _ in range(T)]).astype(np.int32)
+        out = O.permute(idx, N, C)
+        rows, row_of = _permute_brute(idx, N, C)
+        assert np.array_equal(out["perm_tok"], rows)
+        assert np.array_equal(out["row_of"], row_of)
+
+    check()
+
+
 # ---------------------------------------------------------------- experts
 def _rand_mat(rows, cols, scale=0.3):
     return O.Mat(O.F32, rows, cols, data=(RNG.standard_normal((rows, cols)) * scale)
