@@ -29,8 +29,9 @@
  * Parity pins: every function is checked against worked numbers printed on
  * the pages, closed forms, brute force or textbook identities in
  * tests/test_oracle_pins.py, tests/test_oracle_backward.py (the backward) and
- * tests/test_oracle_fp8.py (the E4M3 pieces).  The softmax/SiLU/tanh transcendental values
- * themselves have no printed example beyond the tutorial's aux-loss figures.
+ * tests/test_oracle_fp8.py (the E4M3 pieces).  The softmax/SiLU/tanh
+ * transcendental values themselves have no printed example beyond the
+ * tutorial's aux-loss figures.
  */
 #include <math.h>
 #include <stdint.h>
