@@ -98,3 +98,14 @@ def test_small_layer_algorithmic_work():
     assert experts == 6 * 512 * 128 * 8192
     router = 2 * wl.T * wl.N * wl.d
     assert abs((router + experts) / 1e9 - 3.25) < 0.01
+
+
+def test_layer_launch_counts():
+    """Kernels per moe_layer_fwd step that bench.py claims: 3 for the small
+    layer (one-launch routing, fused FFN, combine: the committed launch list),
+    6 for the Mixtral-shaped layer (router with counts, dispatch, gather,
+    gate/up GEMM, down GEMM, combine) and 4 for the fp32 layer (one-launch
+    routing, two SIMT expert kernels, combine)."""
+    assert bench.layer_launches(W.small()) == 3
+    assert bench.layer_launches(W.mixtral()) == 6
+    assert bench.layer_launches(W.tiny()) == 4
