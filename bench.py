@@ -2,9 +2,15 @@
 
 One step = one full pass of the layer (router -> permutation -> gather ->
 grouped tcgen05 SwiGLU experts -> weighted combine) over one batch of seeded
-synthetic tokens already resident in HBM.  Default workload: the small-model
-layer (T=4096, d=512, N=8 experts, h=128, top-2, bf16).  Other workloads:
---workload mixtral | tiny.
+synthetic tokens already resident in HBM.  Default workload: the
+Mixtral-shaped layer (T=8192, d=4096, N=8 experts, h=14336, top-2, router
+bias b_i = -1.2 ln(i+1), capacity factor 1.25, bf16).  Other workloads:
+--workload small | latent | decode | tiny.
+
+Timing: one pass is exactly --steps steps between two CUDA events, bracketed
+by a barrier and a device synchronize.  Passes repeat until about one second
+of device time has been timed, so that the clock sampler sees the timed
+kernels; the reported time is the median pass (max over ranks per pass).
 
 Prints ONE JSON line (rank 0).  With torchrun (N > 1) every rank runs its own
 replica of the workload (the layer needs no collective: "replicas only",
@@ -79,6 +85,40 @@ def max_over_ranks(value: float, dist, device) -> float:
     t = torch.tensor([value], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+MIN_TIMED_MS = 1000.0  # device time covered by the timed passes together
+MAX_PASSES = 200
+
+
+def timed_passes(run_pass, dist, device, min_total_ms: float = MIN_TIMED_MS):
+    """Times passes of exactly `steps` steps until min_total_ms of device time.
+
+    run_pass() launches one pass and returns its two recorded CUDA events.
+    Every pass is bracketed by a barrier (N > 1) and a device synchronize, its
+    time is the max over ranks, and the number of passes follows from the
+    first pass's max-over-ranks time, so that every rank takes the same
+    collective steps.  Returns (median pass ms, list of pass ms)."""
+    import torch
+
+    def one():
+        if dist:
+            dist.barrier()
+        torch.cuda.synchronize()
+        a, b = run_pass()
+        torch.cuda.synchronize()
+        return max_over_ranks(a.elapsed_time(b), dist, device)
+
+    first = one()
+    n = int(min(MAX_PASSES, max(3, -(-min_total_ms // max(first, 1e-3)))))
+    passes = [first] + [one() for _ in range(n - 1)]
+    return statistics.median(passes), passes
+
+
+def pass_summary(passes, steps: int) -> str:
+    """How the timed passes went, for config.timing."""
+    return (f"{len(passes)} passes of {steps} steps (median reported; "
+            f"min {min(passes):.3f} ms, max {max(passes):.3f} ms per pass)")
 
 
 def whole_job_rate(tokens_per_rank_step: int, steps: int, world: int, ms: float) -> float:
@@ -571,22 +611,22 @@ def decode_main(args, wl, torch, moe, rank, world, dist):
     sel = idx_all.cpu().numpy()
     step_bytes = [decode_step_bytes(wl, sel[i]) for i in range(n_rep)]
     sampler = ClockSampler(int(os.environ.get("LOCAL_RANK", "0"))) if rank == 0 else None
-    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    if dist:
-        dist.barrier()
-    torch.cuda.synchronize()
+
+    def run_pass():
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for i in range(args.steps):
+            graphs[i % n_rep].replay()
+        b.record(stream)
+        return a, b
+
     if sampler:
         sampler.start()
         time.sleep(0.3)
     torch.cuda.nvtx.range_push("timed")
-    a.record(stream)
-    for i in range(args.steps):
-        graphs[i % n_rep].replay()
-    b.record(stream)
+    ms, passes = timed_passes(run_pass, dist, "cuda")
     torch.cuda.nvtx.range_pop()
-    torch.cuda.synchronize()
     clocks = sampler.stop() if sampler else None
-    ms = max_over_ranks(a.elapsed_time(b), dist, "cuda")
     hbm, _, _, src = _peaks()
     bytes_timed = sum(step_bytes[i % n_rep] for i in range(args.steps))
     achieved = bytes_timed / (ms / 1e3) / 1e9
@@ -625,6 +665,7 @@ def decode_main(args, wl, torch, moe, rank, world, dist):
                 "data": "synthetic",
                 "config": {"workload": workload_label(wl),
                            "global_batch": wl.T * world, "parallelism": f"replicas x{world}",
+                           "timing": pass_summary(passes, args.steps),
                            "l2": f"weights rotate over {n_rep} replicas "
                                  f"({n_rep * one.nbytes() / 2**20:.0f} MiB > L2)"},
                 "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
@@ -704,22 +745,22 @@ def latent_main(args, wl, torch, moe, rank, world, dist):
     flops = (2.0 * wl.T * E * d + 2.0 * wl.T * l * d + 6.0 * l * h * wl.T * wl.k
              + 2.0 * wl.T * d * l + n * 6.0 * wl.T * d * sh)
     sampler = ClockSampler(int(os.environ.get("LOCAL_RANK", "0"))) if rank == 0 else None
-    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    if dist:
-        dist.barrier()
-    torch.cuda.synchronize()
+
+    def run_pass():
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.steps):
+            g.replay()
+        b.record(stream)
+        return a, b
+
     if sampler:
         sampler.start()
         time.sleep(0.3)
     torch.cuda.nvtx.range_push("timed")
-    a.record(stream)
-    for _ in range(args.steps):
-        g.replay()
-    b.record(stream)
+    ms, passes = timed_passes(run_pass, dist, "cuda")
     torch.cuda.nvtx.range_pop()
-    torch.cuda.synchronize()
     clocks = sampler.stop() if sampler else None
-    ms = max_over_ranks(a.elapsed_time(b), dist, "cuda")
     hbm, tf, _, src = _peaks()
     per_step_s = ms / args.steps / 1e3
     achieved = step_bytes / per_step_s / 1e9
@@ -751,6 +792,7 @@ def latent_main(args, wl, torch, moe, rank, world, dist):
                 "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
                 "config": {"workload": workload_label(wl),
                            "global_batch": wl.T * world, "parallelism": f"replicas x{world}",
+                           "timing": pass_summary(passes, args.steps),
                            "l2": "routed expert weights 59 GB > L2",
                            "experts_touched": used},
                 "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
@@ -774,7 +816,7 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="small",
+    ap.add_argument("--workload", default="mixtral",
                     choices=["small", "mixtral", "tiny", "decode", "latent"])
     ap.add_argument("--decode-T", type=int, default=32, help="decode batch (1, 8 or 32)")
     ap.add_argument("--tokens", type=int, default=0,
@@ -852,33 +894,29 @@ def main():
         full_g[i % n_rep].replay()
     torch.cuda.synchronize()
 
-    t_start, t_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     sampler = ClockSampler(local) if rank == 0 else None
-    if dist:
-        dist.barrier()
-    torch.cuda.synchronize()
+
+    def graph_pass(graphs):
+        def run():
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for i in range(args.steps):
+                graphs[i % n_rep].replay()
+            b.record(stream)
+            return a, b
+        return run
+
     if sampler:
         sampler.start()
         time.sleep(0.3)
     torch.cuda.nvtx.range_push("timed")
-    t_start.record(stream)
-    for i in range(args.steps):
-        full_g[i % n_rep].replay()
-    t_stop.record(stream)
+    ms, passes = timed_passes(graph_pass(full_g), dist, "cuda")
     torch.cuda.nvtx.range_pop()
-    torch.cuda.synchronize()
-    if dist:
-        dist.barrier()
     clocks = sampler.stop() if sampler else None
-    ms = max_over_ranks(t_start.elapsed_time(t_stop), dist, "cuda")
-    # the dominant kernel alone: the two tcgen05 GEMM launches of each step
-    f_start, f_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    f_start.record(stream)
-    for i in range(args.steps):
-        ffn_g[i % n_rep].replay()
-    f_stop.record(stream)
-    torch.cuda.synchronize()
-    ffn_ms = [f_start.elapsed_time(f_stop) / args.steps] * args.steps
+    # the dominant kernel alone: the expert FFN launches of each step, timed
+    # the same way (median pass)
+    f_ms, _ = timed_passes(graph_pass(ffn_g), dist, "cuda", min_total_ms=MIN_TIMED_MS / 2)
+    ffn_ms = [f_ms / args.steps] * args.steps
     tokens = wl.T * args.steps * world
     value = whole_job_rate(wl.T, args.steps, world, ms)
 
@@ -1007,6 +1045,7 @@ def main():
                 "dtype": "bf16" if wl.act_dtype == S.DT_BF16 else "f32", "data": "synthetic",
                 "config": {"workload": workload_label(wl), "global_batch": wl.T * world,
                            "parallelism": f"replicas x{world}",
+                           "timing": pass_summary(passes, args.steps),
                            "l2": f"inputs rotate over {n_rep} replicas "
                                  f"({n_rep * one.nbytes() / 2**20:.0f} MiB > L2)",
                            "capacity": wl.capacity()},

@@ -176,7 +176,10 @@ MOE_API int moe_permute_noalloc(const moe_shape* shape, const int32_t* top_idx, 
 /* ---------------------------------------------------------------- gather */
 /* x_rows[r] = u[perm_tok[r]] for r < offsets[N] (tutorial §3.6: expert i
  * receives its [L_i, d] rows).  u [T][width] in dtype; x_rows has room for
- * T*k rows of width elements.  Rows >= offsets[N] are left untouched. */
+ * T*k rows of width elements.  Rows >= offsets[N] are left untouched.  An
+ * offsets[N] outside [0, T*k] or a perm_tok entry outside [0, T) records
+ * MOE_ERR_BOUNDS in the device status word; no row beyond T*k is written
+ * and a row with a bad token id is skipped. */
 MOE_API int moe_gather(const moe_shape* shape, int32_t width, const void* u, int32_t dtype,
                const int32_t* perm_tok, const int32_t* offsets, void* x_rows, void* stream);
 
@@ -198,7 +201,9 @@ MOE_API int moe_expert_ffn(const moe_shape* shape, int32_t width, const void* x_
 /* y[t] = sum over kept slots s (row_of[t][s] >= 0, ascending s) of
  * top_w[t][s] * y_rows[row_of[t][s]]  (tutorial §3.2 eq. y); dropped slots
  * add nothing and the weights are not renormalised.  y [T][width] in y_dtype
- * (MOE_F32, MOE_BF16 or MOE_F16), fully overwritten. */
+ * (MOE_F32, MOE_BF16 or MOE_F16), fully overwritten.  A row_of entry at or
+ * above T*k (y_rows holds T*k rows) records MOE_ERR_BOUNDS in the device
+ * status word and that slot adds nothing. */
 MOE_API int moe_combine(const moe_shape* shape, int32_t width, const float* y_rows,
                 const int32_t* row_of, const float* top_w, void* y, int32_t y_dtype,
                 void* stream);
@@ -394,6 +399,24 @@ MOE_API const char* moe_status_string(int32_t status);
 MOE_API int moe_device_status(void* stream, int32_t* status);
 /* Clears the device status word (asynchronous on stream). */
 MOE_API int moe_reset_device_status(void* stream);
+
+/* Failure-detection check of the bounded device waits (no counterpart on the
+ * pages; it tests this library's own error path).  Launches one small kernel
+ * that runs the named wait on a condition nothing satisfies:
+ *   MOE_WAIT_GRID_BARRIER  the grid barrier of the cooperative kernels (two
+ *                          co-resident CTAs wait for one arrival too many),
+ *   MOE_WAIT_MBARRIER      the mbarrier wait of the tcgen05 kernels (a fresh
+ *                          barrier whose first phase never completes).
+ * The wait gives up after about budget_ns nanoseconds (1e3 .. 2e9), records
+ * MOE_ERR_TIMEOUT in the status word and the kernel returns, so the context
+ * stays usable: moe_device_status then reads MOE_ERR_TIMEOUT until
+ * moe_reset_device_status.  Asynchronous on stream.  Returns
+ * MOE_ERR_INVALID_ARG for an unknown kind or a budget out of range.  The
+ * grid-barrier check keeps its counter in a fixed device array shared by
+ * all calls, so calls that overlap on the GPU race. */
+#define MOE_WAIT_GRID_BARRIER 0
+#define MOE_WAIT_MBARRIER 1
+MOE_API int moe_wait_check(int32_t kind, int64_t budget_ns, void* stream);
 
 #ifdef __cplusplus
 }

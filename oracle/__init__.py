@@ -199,6 +199,54 @@ def latent_tokens(x_codes, w_route, k, W_dp, get_expert, W_upp, shared, beta_g, 
     return idx, tw, y
 
 
+def latent_tokens_expert_major(x_codes, w_route, k, W_dp, get_expert, W_upp, shared, beta_g,
+                               beta_u, eps, renorm=1, bias=None, threads=8):
+    """The same LatentMoE forward as latent_tokens, with the routed experts
+    visited in ascending expert order, each fetched once through get_expert(e)
+    (so that a sample of tokens covering all 896 experts never holds more than
+    a few experts' weights).  Every expert output of a (token, slot) pair is
+    the same or_expert call as in latent_tokens, and m sums them in slot order,
+    so the result is bit-identical; only the loop nest differs.  Expert
+    evaluations run on `threads` Python threads (ctypes releases the GIL)."""
+    import concurrent.futures as cf
+
+    x = decode(BF16, x_codes)
+    _, _, idx, tw = route(x.astype(np.float32), w_route, k, renorm, bias)
+    T = x.shape[0]
+    xl = np.stack([round_bf16_array(matvec(W_dp, x[t])) for t in range(T)]) if T else \
+        np.zeros((0, W_dp.rows))
+    outs = np.zeros((T, k, W_dp.rows))
+    pairs = {}
+    for t in range(T):
+        for s_ in range(k):
+            pairs.setdefault(int(idx[t, s_]), []).append((t, s_))
+
+    def run(e, mats):
+        g, u, d = mats
+        for t, s_ in pairs[e]:
+            outs[t, s_] = expert(g, u, d, xl[t], act=1, beta_g=beta_g, beta_u=beta_u, round_h=1)
+
+    with cf.ThreadPoolExecutor(max_workers=threads) as ex:
+        futs = []
+        for e in sorted(pairs):
+            futs.append(ex.submit(run, e, get_expert(e)))
+            if len(futs) >= 2 * threads:  # bound the experts held at once
+                futs.pop(0).result()
+        for f in futs:
+            f.result()
+    y = np.zeros((T, W_upp.rows))
+    for t in range(T):
+        m = np.zeros(W_dp.rows)
+        for s_ in range(k):
+            m += tw[t, s_] * outs[t, s_]
+        mh = round_bf16_array(rmsnorm(m, eps))
+        yt = matvec(W_upp, mh)
+        for (g, u, d) in shared:
+            yt = yt + expert(g, u, d, x[t], act=0, round_h=1)
+        y[t] = yt
+    return idx, tw, y
+
+
 def e4m3_to_f64(code: int) -> float:
     return lib().or_e4m3_to_f64(int(code))
 

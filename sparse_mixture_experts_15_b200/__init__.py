@@ -91,6 +91,7 @@ _PROTOS = {
     "moe_status_string": (ctypes.c_char_p, [_i32]),
     "moe_device_status": (_i32, [_vp, ctypes.POINTER(_i32)]),
     "moe_reset_device_status": (_i32, [_vp]),
+    "moe_wait_check": (_i32, [_i32, _i64, _vp]),
 }
 for _name, (_res, _args) in _PROTOS.items():
     _fn = getattr(_lib, _name)
@@ -444,6 +445,15 @@ def moe_device_status(stream=None) -> int:
 
 def moe_reset_device_status(stream=None):
     _check(_lib.moe_reset_device_status(_stream(stream)), "moe_reset_device_status")
+
+
+WAIT_GRID_BARRIER, WAIT_MBARRIER = 0, 1
+
+
+def moe_wait_check(kind: int, budget_ns: int, stream=None):
+    """Runs one bounded device wait on a condition nothing satisfies (see
+    include/moe.h): the wait records MOE_ERR_TIMEOUT and the kernel returns."""
+    _check(_lib.moe_wait_check(kind, budget_ns, _stream(stream)), "moe_wait_check")
 
 
 def status_string(code: int) -> str:

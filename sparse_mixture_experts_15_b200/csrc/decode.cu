@@ -704,8 +704,13 @@ bool decode_shape_ok(const moe_shape* s) {
   if (!shape_ok(s) || s->T > kMaxT || s->N > kMaxN || s->k > 8 || s->d % 32 != 0 ||
       s->h % 32 != 0 || (s->h / 32) > 32 || 32 % (s->h / 32) != 0)
     return false;
+  // Plan with the current device's SM count, as launch_decode does (fewer
+  // SMs take more rows per CTA and more shared memory); 148 (B200) when no
+  // device is visible, where nothing can be launched anyway.
+  int sms = 0;
+  if (!device_info(&sms) || sms <= 0) sms = 148;
   Plan p;
-  return make_plan(*s, 148, &p);
+  return make_plan(*s, sms, &p);
 }
 
 bool aligned4(const void* q) { return (reinterpret_cast<uintptr_t>(q) & 3u) == 0; }

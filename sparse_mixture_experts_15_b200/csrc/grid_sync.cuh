@@ -32,7 +32,8 @@ __device__ __forceinline__ void grid_arrive(unsigned* bar) {
                  : "memory");
 }
 
-static __device__ bool grid_wait(unsigned* bar, unsigned target, int* status) {
+static __device__ bool grid_wait(unsigned* bar, unsigned target, int* status,
+                                 unsigned long long budget_ns = kBarrierBudgetNs) {
   __shared__ int ok;
   if (threadIdx.x == 0) {
     int good = 1;
@@ -44,7 +45,7 @@ static __device__ bool grid_wait(unsigned* bar, unsigned target, int* status) {
           good = 0;
           break;
         }
-        if (global_ns() - t0 > kBarrierBudgetNs) {
+        if (global_ns() - t0 > budget_ns) {
           record_error(status, MOE_ERR_TIMEOUT);
           atomicExch(bar + 1, 1u);
           good = 0;

@@ -11,11 +11,15 @@ namespace {
 // One warp per grouped row, 16-byte vectors (row bytes are a multiple of 16).
 __global__ void __launch_bounds__(256)
     gather_rows(const uint4* __restrict__ u, int vec_per_row, const int32_t* __restrict__ perm_tok,
-                const int32_t* __restrict__ offsets, int N, int T, uint4* __restrict__ x_rows,
-                int* status) {
+                const int32_t* __restrict__ offsets, int N, int T, int max_rows,
+                uint4* __restrict__ x_rows, int* status) {
   pdl_wait();
   pdl_allow_next();
-  const int rows = offsets[N];
+  int rows = offsets[N];
+  if (rows < 0 || rows > max_rows) {  // x_rows and perm_tok hold T*k rows
+    if (blockIdx.x == 0 && threadIdx.x == 0) record_error(status, MOE_ERR_BOUNDS);
+    rows = rows < 0 ? 0 : max_rows;
+  }
   const int lane = threadIdx.x & 31;
   for (int r = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; r < rows;
        r += (gridDim.x * blockDim.x) >> 5) {
@@ -57,7 +61,8 @@ __device__ __forceinline__ void store4<__half>(__half* y, float4 v) {
 template <typename TY>
 __global__ void __launch_bounds__(256)
     combine_rows(const float4* __restrict__ y_rows, int width4, const int32_t* __restrict__ row_of,
-                 const float* __restrict__ top_w, int T, int k, TY* __restrict__ y) {
+                 const float* __restrict__ top_w, int T, int k, TY* __restrict__ y,
+                 int* status) {
   pdl_wait();
   pdl_allow_next();
   const int lane = threadIdx.x & 31;
@@ -68,6 +73,10 @@ __global__ void __launch_bounds__(256)
       for (int s = 0; s < k; ++s) {
         const int r = row_of[(size_t)t * k + s];
         if (r < 0) continue;
+        if (r >= T * k) {  // y_rows holds T*k rows
+          record_error(status, MOE_ERR_BOUNDS);
+          continue;
+        }
         const float a = top_w[(size_t)t * k + s];
         const float4 v = y_rows[(size_t)r * width4 + c];
         acc.x = __fmaf_rn(a, v.x, acc.x);
@@ -95,8 +104,7 @@ int launch_gather(const moe_shape& s, int32_t width, const void* u, int32_t dtyp
   if (max_rows == 0) return MOE_OK;
   MOE_PREFER_SHARED((gather_rows));
   launch_pdl(gather_rows, dim3(grid_cap(max_rows)), dim3(256), 0, st, static_cast<const uint4*>(u), vec, perm_tok,
-                                                  offsets, s.N, s.T,
-                                                  static_cast<uint4*>(x_rows), status_word());
+             offsets, s.N, s.T, (int)max_rows, static_cast<uint4*>(x_rows), status_word());
   return launch_status();
 }
 
@@ -109,15 +117,15 @@ int launch_combine(const moe_shape& s, int32_t width, const float* y_rows, const
   if (y_dtype == MOE_F32) {
     MOE_PREFER_SHARED((combine_rows<float>));
     launch_pdl(combine_rows<float>, dim3(grid), dim3(256), 0, st, yr, w4, row_of, top_w, s.T, s.k,
-                                              static_cast<float*>(y));
+               static_cast<float*>(y), status_word());
   } else if (y_dtype == MOE_BF16) {
     MOE_PREFER_SHARED((combine_rows<__nv_bfloat16>));
-    launch_pdl(combine_rows<__nv_bfloat16>, dim3(grid), dim3(256), 0, st, yr, w4, row_of, top_w, s.T, s.k,
-                                                      static_cast<__nv_bfloat16*>(y));
+    launch_pdl(combine_rows<__nv_bfloat16>, dim3(grid), dim3(256), 0, st, yr, w4, row_of, top_w,
+               s.T, s.k, static_cast<__nv_bfloat16*>(y), status_word());
   } else {
     MOE_PREFER_SHARED((combine_rows<__half>));
     launch_pdl(combine_rows<__half>, dim3(grid), dim3(256), 0, st, yr, w4, row_of, top_w, s.T, s.k,
-                                               static_cast<__half*>(y));
+               static_cast<__half*>(y), status_word());
   }
   return launch_status();
 }

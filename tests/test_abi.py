@@ -219,3 +219,13 @@ def test_ep_plan_host_checks():
     neg[1, 2] = -1
     assert lib.moe_ep_plan(2, 0, 4, 3, neg.ctypes.data, *ptrs) == -1
     assert lib.moe_ep_plan(2, 0, 4, 3, c.ctypes.data, *ptrs[:7], None) == 0  # overflow optional
+
+
+def test_wait_check_rejects_bad_arguments_on_the_host():
+    """moe_wait_check refuses an unknown wait kind or a budget out of range
+    before touching the device."""
+    lib = moe._lib
+    assert lib.moe_wait_check(2, 1_000_000, None) == -1
+    assert lib.moe_wait_check(-1, 1_000_000, None) == -1
+    assert lib.moe_wait_check(0, 999, None) == -1
+    assert lib.moe_wait_check(1, 2_000_000_001, None) == -1

@@ -102,15 +102,44 @@ def test_latent_bottleneck_is_where_routed_experts_live():
     assert rel_err(y_full.float().cpu().numpy(), ref) > 0.05  # the routed branch mattered
 
 
-def test_latent_full_size_sampled():
+def expert_cover_tokens(idx, N, seed=5):
+    """A few tokens whose top-k sets together contain every expert routed to at
+    all: greedy set cover (each step takes the token that adds the most experts
+    not yet covered; ties to the lower token index after a seeded shuffle)."""
+    rng = np.random.default_rng(seed)
+    order = rng.permutation(idx.shape[0])
+    sets = [set(idx[t].tolist()) for t in range(idx.shape[0])]
+    need = set(idx.ravel().tolist())
+    chosen = []
+    while need:
+        best = max(order, key=lambda t: (len(sets[t] & need), -t))
+        chosen.append(int(best))
+        need -= sets[best]
+    return np.sort(np.array(chosen, dtype=np.int64))
+
+
+def test_latent_full_size_routing_all_tokens_and_expert_cover():
     """The LatentMoE-shaped layer at full size: T=4096, d=4096, l=3584, 896
-    routed experts of hidden 3072, top-16, 2 shared experts; outputs on
-    sampled tokens, routing bit-exact on those tokens."""
+    routed experts of hidden 3072, top-16, 2 shared experts.  Routing indices,
+    combine weights and per-expert counts against the oracle on all 4096
+    tokens; outputs on a set of tokens whose routed experts cover every expert
+    that any token selected (each expert generated once on the host)."""
     wl = W.latent()
     y, outs = _run_gpu(wl)
+    x_all = host_u(wl)
+    w_route = S.normal(wl.seed, W.TID_WROUTE, (wl.N, wl.d), W.SIGMA_W, S.DT_F32)
+    _, _, idx, tw = O.route(O.as_f32(O.BF16, x_all), w_route, wl.k)
+    assert np.array_equal(outs["top_idx"], idx)
+    assert np.allclose(outs["top_w"], tw, rtol=2e-6, atol=1e-7)
+    perm = O.permute(idx, wl.N, 0)
+    assert np.array_equal(outs["counts"], perm["counts"])
     assert outs["counts"].sum() == wl.k * wl.T
-    tokens = np.sort(np.random.default_rng(5).choice(wl.T, 6, replace=False))
-    idx, tw, ref = _oracle(wl, tokens)
-    assert np.array_equal(outs["top_idx"][tokens], idx)
+    tokens = expert_cover_tokens(idx, wl.N)
+    assert set(idx[tokens].ravel().tolist()) == set(np.nonzero(perm["counts"])[0].tolist())
+    W_dp, W_upp, shared = host_latent_dense(wl)
+    idx_s, _, ref = O.latent_tokens_expert_major(
+        x_all[tokens], w_route, wl.k, W_dp, lambda e: host_latent_expert(wl, e), W_upp, shared,
+        wl.beta_gate, wl.beta_up, 1e-6, threads=max(1, min(16, O.threads())))
+    assert np.array_equal(idx_s, idx[tokens])
     got = y[torch.from_numpy(tokens).long().cuda()].float().cpu().numpy()
     assert rel_err(got, ref) < TOL_BF16

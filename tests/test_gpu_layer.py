@@ -163,10 +163,32 @@ def test_layer_small_bf16_ragged_T():
     assert rel_err(y.float().cpu().numpy(), ref) < TOL_BF16
 
 
+def tile_cover_tokens(perm, N, tile=128, seed=3, n_dropped=4):
+    """Tokens whose outputs together touch every (expert, `tile`-row token tile)
+    of the grouped layout, each expert's last (ragged) row among them, plus a
+    few tokens with a dropped slot: one random row per tile, mapped back to its
+    token through perm_tok."""
+    rng = np.random.default_rng(seed)
+    off, perm_tok = perm["offsets"], perm["perm_tok"]
+    rows = []
+    for e in range(N):
+        beg, end = int(off[e]), int(off[e + 1])
+        for t0 in range(beg, end, tile):
+            rows.append(int(rng.integers(t0, min(t0 + tile, end))))
+        if end > beg:
+            rows.append(end - 1)
+    tokens = [int(perm_tok[r]) for r in rows]
+    dropped = np.where((perm["row_of"] < 0).any(1))[0]
+    if len(dropped):
+        tokens += rng.choice(dropped, min(n_dropped, len(dropped)), replace=False).tolist()
+    return np.unique(np.array(tokens, dtype=np.int32))
+
+
 def test_layer_mixtral_full_size_sampled():
     """Mixtral-shaped layer at full size with Zipf-skewed loads and capacity
-    1.25: routing, overflow and totals bit-exact on all 8192 tokens, outputs on
-    sampled tokens (including tokens with a dropped slot)."""
+    1.25: routing, overflow and totals bit-exact on all 8192 tokens; outputs on
+    tokens that cover every (expert, 128-row token tile) of the grouped rows,
+    each expert's ragged last tile, and tokens with a dropped slot."""
     wl = W.mixtral()
     y, outs = _layer_gpu(wl)
     u_codes = host_u(wl)
@@ -176,16 +198,17 @@ def test_layer_mixtral_full_size_sampled():
     perm = O.permute(idx, wl.N, wl.capacity())
     _check_routing(outs, idx, tw, perm)
     assert int(perm["totals"][1]) > 0, "the skewed loads should overflow the capacity"
-    rng = np.random.default_rng(3)
-    dropped = np.where((perm["row_of"] < 0).any(1))[0]
-    tokens = np.sort(np.concatenate([rng.choice(wl.T, 12, replace=False),
-                                     rng.choice(dropped, min(4, len(dropped)), replace=False)]))
-    tokens = np.unique(tokens).astype(np.int32)
+    tokens = tile_cover_tokens(perm, wl.N)
+    kept = perm["row_of"][tokens]
+    for e in range(wl.N):  # every tile of every expert is touched
+        beg, end = int(perm["offsets"][e]), int(perm["offsets"][e + 1])
+        hit = {(r - beg) // 128 for r in kept.ravel() if beg <= r < end}
+        assert hit == set(range(-(-(end - beg) // 128))), e
+    assert (kept < 0).any(), "a token with a dropped slot is among those checked"
     mats = [host_expert(wl, e) for e in range(wl.N)]
     ref = O.moe_tokens([m[0] for m in mats], [m[1] for m in mats], [m[2] for m in mats],
                        O.decode(od, u_codes[tokens]), idx[tokens], tw[tokens],
-                       row_of=perm["row_of"][tokens], tokens=np.arange(len(tokens), dtype=np.int32),
-                       round_h=1)
+                       row_of=kept, tokens=np.arange(len(tokens), dtype=np.int32), round_h=1)
     got = y[torch.from_numpy(tokens).long().cuda()].float().cpu().numpy()
     assert rel_err(got, ref) < TOL_BF16
 

@@ -330,6 +330,35 @@ def test_situ_glu_soft_caps():
     assert np.allclose(big, plain, rtol=1e-9, atol=1e-12)
 
 
+def test_situ_glu_gate_and_up_caps_are_not_interchangeable():
+    """LatentMoE document, SiTU-GLU: the caps multiply to beta_g * beta_u, given
+    as 4 x 25 = 100 (gate cap first, up cap second).  With one hidden unit and
+    an identity down projection the hidden value is exposed:
+      gate saturated (g -> +inf): H = SiLU(4) * 25 tanh(v / 25);
+      up saturated   (v -> +inf): H = SiLU(4 tanh(g / 4)) * 25;
+      both saturated:             H = SiLU(4) * 25 = 98.2..., below 100,
+    where exchanged caps would give SiLU(25) * 4 = 99.99...  The workload
+    constants carry the same assignment."""
+    from synthetic import workloads as W
+    one = O.Mat(O.F32, 1, 1, data=np.ones((1, 1), np.float32))
+
+    def hidden(g, v):
+        Wg = O.Mat(O.F32, 1, 1, data=np.array([[g]], np.float32))
+        Wu = O.Mat(O.F32, 1, 1, data=np.array([[v]], np.float32))
+        return float(O.expert(Wg, Wu, one, np.ones(1), act=1, beta_g=4.0, beta_u=25.0)[0])
+
+    silu4 = 4.0 / (1.0 + math.exp(-4.0))
+    assert math.isclose(hidden(1e4, 5.0), silu4 * 25.0 * math.tanh(5.0 / 25.0), rel_tol=1e-14)
+    g = 3.0
+    gc = 4.0 * math.tanh(g / 4.0)
+    assert math.isclose(hidden(g, 1e4), gc / (1.0 + math.exp(-gc)) * 25.0, rel_tol=1e-14)
+    both = hidden(1e4, 1e4)
+    assert math.isclose(both, silu4 * 25.0, rel_tol=1e-14) and both < 100.0
+    assert abs(both - 25.0 / (1.0 + math.exp(-25.0)) * 4.0) > 1.5
+    wl = W.latent()
+    assert (wl.beta_gate, wl.beta_up) == (4.0, 25.0)
+
+
 def test_round_h_rounds_hidden_to_bf16():
     d, h = 16, 32
     Wg, Wu = _rand_mat(h, d), _rand_mat(h, d)
@@ -531,6 +560,23 @@ def test_latent_single_expert_closed_form():
         m = d @ bf16(_silu(G) * U)
         mh = bf16(m / np.sqrt(np.mean(m * m) + 1e-6))
         assert np.allclose(y[t], W_upp.decode() @ mh, rtol=1e-11, atol=1e-12)
+
+
+def test_latent_expert_major_order_is_bit_identical():
+    """The expert-major loop nest (each routed expert fetched once, used by the
+    full-size GPU parity test) returns exactly the per-token forward."""
+    x, wr, W_dp, ex, W_upp, sh = _latent_case(N=9, T=11)
+    fetched = []
+
+    def get(e):
+        fetched.append(e)
+        return ex[e]
+
+    i1, w1, y1 = O.latent_tokens(x, wr, 3, W_dp, lambda e: ex[e], W_upp, sh, 4.0, 25.0, 1e-6)
+    i2, w2, y2 = O.latent_tokens_expert_major(x, wr, 3, W_dp, get, W_upp, sh, 4.0, 25.0, 1e-6,
+                                              threads=4)
+    assert np.array_equal(i1, i2) and np.array_equal(w1, w2) and np.array_equal(y1, y2)
+    assert fetched == sorted(set(i1.ravel().tolist()))  # every routed expert once, in order
 
 
 # ------------------------------------------------------- quantile balancing

@@ -66,3 +66,39 @@ def test_noalloc_permute_rejects_oversize():
     rc = lib.moe_permute_noalloc(ctypes.byref(s), p, p, p, p, p, p, p,
                                  torch.cuda.current_stream().cuda_stream)
     assert rc == -6 and moe.status_string(rc).startswith("MOE_ERR_WORKSPACE")
+
+
+def _one_case_on(stream, T=3000, N=64, k=4, C=0):
+    """Both entry points on `stream` (a torch stream of the current device)."""
+    lib = moe._lib
+    rng = np.random.default_rng(11)
+    z = rng.standard_normal((T, N)) + np.linspace(1.0, 0.0, N)[None, :]
+    with torch.cuda.stream(stream):
+        idx = torch.from_numpy(np.argsort(-z, axis=1)[:, :k].astype(np.int32)).cuda()
+        s = moe.shape(T, 64, N, k, 64, 1, C)
+        ref, got = _buffers(T, N, k), _buffers(T, N, k)
+        nb = lib.moe_permute_workspace_bytes(ctypes.byref(s))
+        ws = torch.empty(nb, dtype=torch.uint8, device="cuda")
+        assert _call(lib.moe_permute, s, idx, ref, ws.data_ptr(), nb) == 0
+        assert _call(lib.moe_permute_noalloc, s, idx, got) == 0
+    stream.synchronize()
+    rows = int(ref["offsets"][N].item())
+    for key in ("counts", "offsets", "row_of", "overflow", "totals"):
+        assert torch.equal(got[key], ref[key]), key
+    assert torch.equal(got["perm_tok"][:rows], ref["perm_tok"][:rows])
+
+
+def test_noalloc_permute_on_a_side_stream():
+    """The entry point runs on whatever stream the caller passes."""
+    _one_case_on(torch.cuda.Stream(), C=30)
+    assert moe.moe_device_status() == 0
+
+
+@pytest.mark.skipif(not torch.cuda.is_available() or torch.cuda.device_count() < 2,
+                    reason="needs a second visible GPU")
+def test_noalloc_permute_on_a_second_device():
+    """The fixed array exists once per device; its address is looked up per
+    device, so a call on device 1 uses device 1's copy."""
+    with torch.cuda.device(1):
+        _one_case_on(torch.cuda.current_stream(), C=30)
+        assert moe.moe_device_status() == 0
