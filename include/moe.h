@@ -64,6 +64,7 @@ extern "C" {
 #define MOE_BF16 1
 #define MOE_F16 2
 #define MOE_Q4_0 3
+#define MOE_E4M3 4 /* OCP FP8 E4M3 codes (1 byte) with one fp32 scale per row */
 
 /* Expert activation.  MOE_ACT_SWIGLU: H = SiLU(g) * v.  MOE_ACT_SITU_GLU:
  * H = SiLU(beta_gate tanh(g / beta_gate)) * beta_up tanh(v / beta_up), the
@@ -283,6 +284,42 @@ MOE_API size_t moe_latent_workspace_bytes(const moe_shape* shape, const moe_late
 MOE_API int moe_latent_fwd(const moe_shape* shape, const moe_layer_weights* w,
                            const moe_latent_weights* lw, const void* x, void* y,
                            const moe_layer_outputs* out, void* ws, size_t ws_bytes, void* stream);
+
+/* FP8 routed experts (Stable LatentMoE demo document, SiTU-GLU: the soft caps
+ * bound the hidden product by beta_g * beta_u = 100, under E4M3's largest
+ * finite value 448, which is what FP8 experts need).  Values are
+ * scale[row] * e4m3(code[row][col]) (OCP E4M3: bias 7, no infinity, 448 the
+ * largest finite value); moe_quantize_e4m3_rows makes them from bf16 or fp32
+ * rows: s = amax(row) / 448 (1 for a zero row), code = e4m3(x / s) rounded to
+ * nearest even and saturated at 448, each division one fp32 operation. */
+typedef struct {
+  const float* gate_scale; /* [N * h] row scales of w_gate's codes */
+  const float* up_scale;   /* [N * h] row scales of w_up's codes */
+  const float* down_scale; /* [N * l] row scales of w_down's codes */
+} moe_e4m3_scales;
+
+/* x: [rows][cols] in x_dtype (MOE_BF16 or MOE_F32), cols a multiple of 16;
+ * codes [rows][cols] bytes and scales [rows] fp32 (device, caller-owned).
+ * Asynchronous on stream.  MOE_ERR_INVALID_ARG for a bad size, NULL or
+ * misaligned pointer (x and codes 16-B aligned, scales 4-B aligned),
+ * MOE_ERR_UNSUPPORTED for another x_dtype. */
+MOE_API int moe_quantize_e4m3_rows(int64_t rows, int32_t cols, const void* x, int32_t x_dtype,
+                                   uint8_t* codes, float* scales, void* stream);
+
+/* The LatentMoE layer of moe_latent_fwd with E4M3 routed experts: w->w_dtype
+ * == MOE_E4M3 and w->w_gate, w_up, w_down hold codes (gate, up [N][h][l],
+ * down [N][l][h] bytes) with the row scales in *scales.  x_l = W_dp x (bf16)
+ * is quantised per token the same way as the weights; the gate/up and down
+ * GEMMs run on the FP8 tensor cores (E4M3 x E4M3, fp32 accumulate) with the
+ * scales applied to the fp32 results; H is stored as E4M3 codes with no
+ * scale.  The router, W_dp, W_upp and the shared experts stay bf16 / fp32.
+ * Requires l and h multiples of 128.  Workspace: moe_latent_workspace_bytes.
+ * Errors as moe_latent_fwd; MOE_ERR_INVALID_ARG when scales or one of its
+ * pointers is NULL. */
+MOE_API int moe_latent_fwd_e4m3(const moe_shape* shape, const moe_layer_weights* w,
+                                const moe_e4m3_scales* scales, const moe_latent_weights* lw,
+                                const void* x, void* y, const moe_layer_outputs* out, void* ws,
+                                size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------- q4_0 decode */
 /* Small-batch decode with q4_0 experts (deployment notes "Kestrel-MCU notes

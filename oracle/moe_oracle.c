@@ -108,23 +108,31 @@ double or_e4m3_to_f64(uint8_t c) {
   return sign ? -v : v;
 }
 
-/* Nearest E4M3 code to x, ties to the even code (even mantissa), by search
- * over the 127 finite magnitudes; magnitudes above 448 give 448 (saturation,
- * the "satfinite" conversion), NaN gives the NaN code, the sign of x (also
- * of a zero result) is kept. */
+/* Nearest E4M3 code to x, ties to the even code (even mantissa), among the
+ * 127 finite magnitudes (codes 0x00..0x7E, increasing with the code);
+ * magnitudes above 448 give 448 (saturation, the "satfinite" conversion),
+ * NaN gives the NaN code, the sign of x (also of a zero result) is kept.
+ * The search is a bisection for the largest magnitude not above |x| in the
+ * table of decoded magnitudes, then the nearer of it and the next one. */
+static double e4m3_mag[127];
+
+__attribute__((constructor)) static void e4m3_mag_fill(void) { /* at library load */
+  for (int c = 0; c <= 0x7E; ++c) e4m3_mag[c] = or_e4m3_to_f64((uint8_t)c);
+}
+
 uint8_t or_round_e4m3(double x) {
   if (isnan(x)) return 0x7F;
   uint8_t sign = signbit(x) ? 0x80 : 0x00;
   if (isinf(x)) return (uint8_t)(sign | 0x7E); /* saturates like any magnitude above 448 */
-  double a = fabs(x), bd = INFINITY;
-  int best = 0;
-  for (int c = 0; c <= 0x7E; ++c) {
-    double dist = fabs(or_e4m3_to_f64((uint8_t)c) - a);
-    if (dist < bd || (dist == bd && (c & 1) == 0)) {
-      bd = dist;
-      best = c;
-    }
+  double a = fabs(x);
+  if (a >= e4m3_mag[0x7E]) return (uint8_t)(sign | 0x7E);
+  int lo = 0, hi = 0x7E; /* e4m3_mag[lo] <= a < e4m3_mag[hi] */
+  while (hi - lo > 1) {
+    int mid = (lo + hi) / 2;
+    if (e4m3_mag[mid] <= a) lo = mid; else hi = mid;
   }
+  double dlo = a - e4m3_mag[lo], dhi = e4m3_mag[hi] - a;
+  int best = dlo < dhi ? lo : dhi < dlo ? hi : ((lo & 1) == 0 ? lo : hi);
   return (uint8_t)(sign | best);
 }
 
@@ -134,6 +142,7 @@ uint8_t or_round_e4m3(double x) {
  * approximates x and the row's largest magnitude maps to +-448. */
 void or_quant_e4m3_rows(int64_t rows, int64_t cols, const float* x, uint8_t* codes,
                         float* scales) {
+#pragma omp parallel for schedule(static)
   for (int64_t r = 0; r < rows; ++r) {
     float amax = 0.0f;
     for (int64_t c = 0; c < cols; ++c) amax = fmaxf(amax, fabsf(x[r * cols + c]));

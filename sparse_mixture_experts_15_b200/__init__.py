@@ -14,7 +14,7 @@ import os
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libmoe.so")
 
-F32, BF16, F16, Q4_0 = 0, 1, 2, 3
+F32, BF16, F16, Q4_0, E4M3 = 0, 1, 2, 3, 4
 ACT_SWIGLU, ACT_SITU_GLU = 0, 1
 
 if not os.path.exists(LIB_PATH):
@@ -56,6 +56,10 @@ class MoeLatentWeights(ctypes.Structure):
                 ("shared_up", _vp), ("shared_down", _vp), ("rms_eps", _f32)]
 
 
+class MoeE4M3Scales(ctypes.Structure):
+    _fields_ = [(n, _vp) for n in ("gate_scale", "up_scale", "down_scale")]
+
+
 _P_SHAPE = ctypes.POINTER(MoeShape)
 _PROTOS = {
     "moe_capacity": (_i32, [_i64, _i32, _i32, _f64, ctypes.POINTER(_i32)]),
@@ -78,6 +82,11 @@ _PROTOS = {
     "moe_latent_fwd": (_i32, [_P_SHAPE, ctypes.POINTER(MoeLayerWeights),
                               ctypes.POINTER(MoeLatentWeights), _vp, _vp,
                               ctypes.POINTER(MoeLayerOutputs), _vp, _sz, _vp]),
+    "moe_quantize_e4m3_rows": (_i32, [_i64, _i32, _vp, _i32, _vp, _vp, _vp]),
+    "moe_latent_fwd_e4m3": (_i32, [_P_SHAPE, ctypes.POINTER(MoeLayerWeights),
+                                   ctypes.POINTER(MoeE4M3Scales),
+                                   ctypes.POINTER(MoeLatentWeights), _vp, _vp,
+                                   ctypes.POINTER(MoeLayerOutputs), _vp, _sz, _vp]),
     "moe_decode_workspace_bytes": (_sz, [_P_SHAPE]),
     "moe_decode_layer": (_i32, [_P_SHAPE, ctypes.POINTER(MoeQ4Layer), _vp, _vp, _vp, _vp, _vp,
                                 _vp, _sz, _vp]),
@@ -341,6 +350,44 @@ def moe_latent_fwd(s: MoeShape, w_route, w_gate, w_up, w_down, lw: MoeLatentWeig
     _check(_lib.moe_latent_fwd(ctypes.byref(s), ctypes.byref(W), ctypes.byref(lw), _ptr(x),
                                _ptr(y), ctypes.byref(O), _ptr(wbuf), wlen, _stream(stream)),
            "moe_latent_fwd")
+
+
+_CODES = (_U8, "float8_e4m3fn")
+
+
+def moe_quantize_e4m3_rows(x, codes, scales, stream=None):
+    """Row-wise E4M3 quantisation (include/moe.h): x [rows][cols] bf16 or fp32
+    -> codes [rows][cols] (uint8 or float8_e4m3fn), scales [rows] fp32."""
+    rows, cols = x.shape[0], x.numel() // max(x.shape[0], 1)
+    _need("x", x, rows * cols, (_BF16, _F32))
+    _need("codes", codes, rows * cols, _CODES)
+    _need("scales", scales, rows, _F32)
+    _check(_lib.moe_quantize_e4m3_rows(rows, cols, _ptr(x), _dtype_code(x), _ptr(codes),
+                                       _ptr(scales), _stream(stream)), "moe_quantize_e4m3_rows")
+
+
+def moe_latent_fwd_e4m3(s: MoeShape, w_route, w_gate, w_up, w_down, gate_scale, up_scale,
+                        down_scale, lw: MoeLatentWeights, x, y, bias=None, a=None,
+                        outputs: dict | None = None, ws=None, stream=None):
+    """The LatentMoE layer with E4M3 routed experts (codes + fp32 row scales)."""
+    a = a or act()
+    l = lw.latent
+    for args in (("x", x, s.T * s.d, _BF16), ("y", y, s.T * s.d, _BF16),
+                 ("w_route", w_route, s.N * s.d, _F32), ("bias", bias, s.N, _F32),
+                 ("w_gate", w_gate, s.N * s.h * l, _CODES), ("w_up", w_up, s.N * s.h * l, _CODES),
+                 ("w_down", w_down, s.N * l * s.h, _CODES),
+                 ("gate_scale", gate_scale, s.N * s.h, _F32),
+                 ("up_scale", up_scale, s.N * s.h, _F32),
+                 ("down_scale", down_scale, s.N * l, _F32)):
+        _need(*args)
+    O = _outputs(s, outputs)
+    W = MoeLayerWeights(_ptr(w_route), _ptr(bias), _ptr(w_gate), _ptr(w_up), _ptr(w_down), E4M3,
+                        a)
+    sc = MoeE4M3Scales(_ptr(gate_scale), _ptr(up_scale), _ptr(down_scale))
+    wbuf, wlen = _ws(moe_latent_workspace_bytes(s, lw), x.device, ws)
+    _check(_lib.moe_latent_fwd_e4m3(ctypes.byref(s), ctypes.byref(W), ctypes.byref(sc),
+                                    ctypes.byref(lw), _ptr(x), _ptr(y), ctypes.byref(O),
+                                    _ptr(wbuf), wlen, _stream(stream)), "moe_latent_fwd_e4m3")
 
 
 def q4_layer(w_route, gate_qs, gate_scales, up_qs, up_scales, down_qs, down_scales,

@@ -4,6 +4,7 @@
 
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -104,6 +105,14 @@ __device__ __forceinline__ float gated_act(float g, float v, float bg, float bu)
     v = bu * tanh_approx(__fdividef(v, bu));
   }
   return __fdividef(g, 1.0f + __expf(-g)) * v;
+}
+
+// Four fp32 values to four OCP E4M3 codes (round to nearest even, magnitudes
+// above 448 saturate to 448), v[0] in the lowest byte.
+__device__ __forceinline__ uint32_t e4m3x4_rn(const float* v) {
+  const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(v[0], v[1]), __NV_SATFINITE, __NV_E4M3);
+  const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(v[2], v[3]), __NV_SATFINITE, __NV_E4M3);
+  return (lo & 0xFFFFu) | (hi << 16);
 }
 
 // ------------------------------------------- programmatic dependent launch
@@ -251,6 +260,12 @@ int launch_ffn_tc(const moe_shape& s, int32_t width, const __nv_bfloat16* x_rows
                   const __nv_bfloat16* w_down, const moe_act& act, float* y_rows, void* ws,
                   cudaStream_t st);
 
+// Gather of the expert path fused with per-token E4M3 quantisation (fp8.cu):
+// codes[r] = e4m3 codes of x[perm_tok[r]] / scales[r], rows r < offsets[N].
+int launch_quant_gather_e4m3(const moe_shape& s, int cols, const __nv_bfloat16* x,
+                             const int32_t* perm_tok, const int32_t* offsets, uint8_t* codes,
+                             float* scales, cudaStream_t st);
+
 // Fused single-launch expert FFN for small hidden widths (ffn_fused.cu).
 bool ffn_fused_ok(int width, int h, int G);
 int launch_ffn_fused(int G, int64_t R, int width, int h, const __nv_bfloat16* x_rows,
@@ -273,16 +288,25 @@ struct TcSeg {
   int bcol;           // column offset into B
 };
 
+// E4M3 operands of a grouped GEMM: codes in the operand arrays, fp32 scales
+// per row of A (gate/up: gate rows, up rows) and per row of B (nullable: 1).
+struct TcF8 {
+  const float* a_scale[2];
+  const float* b_scale;
+};
+
 // Gate/up GEMM with the fused activation: for group g and its rows of X,
-// out[row][g * out_col_group + j] = act(X W_gate[g]^T, X W_up[g]^T)[j] as bf16.
+// out[row][g * out_col_group + j] = act(X W_gate[g]^T, X W_up[g]^T)[j] as bf16
+// (f8 == nullptr: bf16 X and weights), or as E4M3 codes with no scale (f8:
+// E4M3 X and weights with their row scales; K a multiple of 128).
 // offsets == nullptr: every group uses rows [0, T) of X.
-int tc_gateup(const int32_t* offsets, int T, int G, const __nv_bfloat16* X, int64_t x_rows,
-              int K, const __nv_bfloat16* w_gate, const __nv_bfloat16* w_up, int hidden,
-              const moe_act& act, __nv_bfloat16* out, int out_ld, int out_col_group,
-              cudaStream_t st);
+int tc_gateup(const int32_t* offsets, int T, int G, const void* X, int64_t x_rows, int K,
+              const void* w_gate, const void* w_up, int hidden, const moe_act& act, void* out,
+              int out_ld, int out_col_group, cudaStream_t st, const TcF8* f8 = nullptr);
 // Store-mode GEMM over 1..3 K-segments accumulated into one fp32 tile:
 // out[row][g * m_rows + m] = sum_s A_s[g * a_rows + arow_s + m] . B_s[row][bcol_s ...].
+// f8: one segment of E4M3 operands, fp32 output scaled by the row scales.
 int tc_store(const int32_t* offsets, int T, int G, int m_rows, const TcSeg* segs, int nseg,
-             void* out, int mode, int out_ld, cudaStream_t st);
+             void* out, int mode, int out_ld, cudaStream_t st, const TcF8* f8 = nullptr);
 
 }  // namespace moe

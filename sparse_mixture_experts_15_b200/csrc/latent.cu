@@ -60,8 +60,9 @@ struct LatentBufs {
   int32_t* totals;
   void* permute_ws;
   __nv_bfloat16* x_l;
-  __nv_bfloat16* x_rows;
-  __nv_bfloat16* H;
+  __nv_bfloat16* x_rows;  // E4M3 experts: the gathered codes of x_l (1 byte each)
+  float* x_scale;         // E4M3 experts: one scale per gathered row
+  __nv_bfloat16* H;       // E4M3 experts: H as codes
   float* y_rows;
   float* m;
   __nv_bfloat16* m_hat;
@@ -87,6 +88,7 @@ LatentBufs carve_latent(const moe_shape& s, const moe_latent_weights& lw, void* 
   b.permute_ws = c.take<char>(permute_ws_bytes(s));
   b.x_l = c.take<__nv_bfloat16>((size_t)s.T * l);
   b.x_rows = c.take<__nv_bfloat16>(Tk * l);
+  b.x_scale = c.take<float>(Tk);
   b.H = c.take<__nv_bfloat16>(Tk * s.h);
   b.y_rows = c.take<float>(Tk * l);
   b.m = c.take<float>((size_t)s.T * l);
@@ -117,13 +119,19 @@ extern "C" size_t moe_latent_workspace_bytes(const moe_shape* shape,
   return moe::carve_latent(*shape, *lw, nullptr).bytes;
 }
 
-extern "C" int moe_latent_fwd(const moe_shape* shape, const moe_layer_weights* w,
-                              const moe_latent_weights* lw, const void* x, void* y,
-                              const moe_layer_outputs* out, void* ws, size_t ws_bytes,
-                              void* stream) {
-  using namespace moe;
+namespace moe {
+namespace {
+
+// The layer with bf16 routed experts (e4m3 == nullptr) or E4M3 ones.
+int latent_forward(const moe_shape* shape, const moe_layer_weights* w,
+                   const moe_e4m3_scales* e4m3, const moe_latent_weights* lw, const void* x,
+                   void* y, const moe_layer_outputs* out, void* ws, size_t ws_bytes,
+                   void* stream) {
   if (!latent_ok(shape, lw) || !w) return MOE_ERR_INVALID_ARG;
-  if (w->w_dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+  if (w->w_dtype != (e4m3 ? MOE_E4M3 : MOE_BF16)) return MOE_ERR_UNSUPPORTED;
+  if (e4m3 && (!e4m3->gate_scale || !e4m3->up_scale || !e4m3->down_scale))
+    return MOE_ERR_INVALID_ARG;
+  if (e4m3 && (lw->latent % 128 != 0 || shape->h % 128 != 0)) return MOE_ERR_UNSUPPORTED;
   if (w->act.kind != MOE_ACT_SWIGLU &&
       !(w->act.kind == MOE_ACT_SITU_GLU && w->act.beta_gate > 0.0f && w->act.beta_up > 0.0f))
     return MOE_ERR_INVALID_ARG;
@@ -172,12 +180,26 @@ extern "C" int moe_latent_fwd(const moe_shape* shape, const moe_layer_weights* w
     rc = tc_store(nullptr, s.T, 1, l, &seg, 1, b.x_l, MODE_STORE_BF16, l, st);
     if (rc != MOE_OK) return rc;
   }
-  rc = launch_gather(s, l, b.x_l, MOE_BF16, perm_tok, offsets, b.x_rows, st);
-  if (rc != MOE_OK) return rc;
-  rc = tc_gateup(offsets, Tk, s.N, b.x_rows, Tk, l, static_cast<const __nv_bfloat16*>(w->w_gate),
-                 static_cast<const __nv_bfloat16*>(w->w_up), s.h, w->act, b.H, s.h, 0, st);
-  if (rc != MOE_OK) return rc;
-  {
+  if (e4m3) {
+    // E4M3 experts: x_l quantised per token while it is gathered; gate/up
+    // with the row scales, H stored as E4M3 codes; down with its row scales
+    TcF8 gu{{e4m3->gate_scale, e4m3->up_scale}, b.x_scale};
+    TcF8 dn{{e4m3->down_scale, nullptr}, nullptr};
+    rc = launch_quant_gather_e4m3(s, l, b.x_l, perm_tok, offsets,
+                                  reinterpret_cast<uint8_t*>(b.x_rows), b.x_scale, st);
+    if (rc == MOE_OK)
+      rc = tc_gateup(offsets, Tk, s.N, b.x_rows, Tk, l, w->w_gate, w->w_up, s.h, w->act, b.H, s.h,
+                     0, st, &gu);
+    if (rc != MOE_OK) return rc;
+    TcSeg seg{w->w_down, (int64_t)s.N * l, s.h, 0, b.H, Tk, s.h, 0};
+    rc = tc_store(offsets, Tk, s.N, l, &seg, 1, b.y_rows, MODE_STORE_F32, l, st, &dn);
+    if (rc != MOE_OK) return rc;
+  } else {
+    rc = launch_gather(s, l, b.x_l, MOE_BF16, perm_tok, offsets, b.x_rows, st);
+    if (rc != MOE_OK) return rc;
+    rc = tc_gateup(offsets, Tk, s.N, b.x_rows, Tk, l, w->w_gate, w->w_up, s.h, w->act, b.H, s.h,
+                   0, st);
+    if (rc != MOE_OK) return rc;
     TcSeg seg{w->w_down, (int64_t)s.N * l, s.h, 0, b.H, Tk, s.h, 0};
     rc = tc_store(offsets, Tk, s.N, l, &seg, 1, b.y_rows, MODE_STORE_F32, l, st);
     if (rc != MOE_OK) return rc;
@@ -208,4 +230,22 @@ extern "C" int moe_latent_fwd(const moe_shape* shape, const moe_layer_weights* w
     segs[1 + j] = TcSeg{lw->shared_down, (int64_t)nsh * s.d, sh, j * s.d, b.H_sh, s.T, nsh * sh,
                         j * sh};
   return tc_store(nullptr, s.T, 1, s.d, segs, 1 + nsh, y, MODE_STORE_BF16, s.d, st);
+}
+
+}  // namespace
+}  // namespace moe
+
+extern "C" int moe_latent_fwd(const moe_shape* shape, const moe_layer_weights* w,
+                              const moe_latent_weights* lw, const void* x, void* y,
+                              const moe_layer_outputs* out, void* ws, size_t ws_bytes,
+                              void* stream) {
+  return moe::latent_forward(shape, w, nullptr, lw, x, y, out, ws, ws_bytes, stream);
+}
+
+extern "C" int moe_latent_fwd_e4m3(const moe_shape* shape, const moe_layer_weights* w,
+                                   const moe_e4m3_scales* scales, const moe_latent_weights* lw,
+                                   const void* x, void* y, const moe_layer_outputs* out, void* ws,
+                                   size_t ws_bytes, void* stream) {
+  if (!scales) return MOE_ERR_INVALID_ARG;
+  return moe::latent_forward(shape, w, scales, lw, x, y, out, ws, ws_bytes, stream);
 }

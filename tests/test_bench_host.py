@@ -25,6 +25,12 @@ def test_latent_cpu_baseline_runs_a_bounded_sample():
     assert rate > 0 and seconds >= 0.2 and n == 1
 
 
+def test_latent_fp8_cpu_baseline_runs_a_bounded_sample():
+    wl = dataclasses.replace(W.latent(T=64), N=32, d=256, latent=128, h=128, shared_hidden=128)
+    rate, seconds, n = bench.latent_cpu_baseline(wl, budget_s=0.2, fp8=True)
+    assert rate > 0 and seconds >= 0.2 and n == 1
+
+
 def test_latent_launch_count_matches_the_profiled_list():
     # 13 kernels per step in the committed LatentMoE launch list
     assert bench.latent_launches(W.latent()) == 13

@@ -1,0 +1,173 @@
+"""GPU parity of the FP8 E4M3 routed experts of the LatentMoE layer (Stable
+LatentMoE demo document, SiTU-GLU: the soft caps bound the hidden product by
+beta_g * beta_u = 100 < 448, the E4M3 maximum) against the CPU oracle's FP8
+form, through the C ABI.
+
+The row quantiser must match the oracle's bit for bit (its decisions are taken
+on the same fp32 quotients).  The layer output is compared within the bf16
+bound, 2e-2 of rms(y): the GPU forms H with approximate transcendentals, so an
+element of H near a rounding boundary can take the neighbouring E4M3 code."""
+import numpy as np
+import pytest
+
+import oracle as O
+import synthetic as S
+from synthetic import workloads as W
+
+from inputs import dev_latent, dev_u, host_latent_dense, host_u, rel_err
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+TOL = 2e-2
+
+if torch.cuda.is_available():
+    import sparse_mixture_experts_15_b200 as moe
+
+
+@pytest.fixture(autouse=True)
+def _clean_status():
+    moe.moe_reset_device_status()
+    yield
+    assert moe.moe_device_status() == 0
+
+
+def _quant_dev(x):
+    codes = torch.empty(x.shape, dtype=torch.uint8, device="cuda")
+    scales = torch.empty(x.shape[0], dtype=torch.float32, device="cuda")
+    moe.moe_quantize_e4m3_rows(x, codes, scales)
+    return codes, scales
+
+
+@pytest.mark.parametrize("dtype", ["bfloat16", "float32"])
+def test_quantize_rows_bit_exact(dtype):
+    """Rows of very different magnitudes (subnormal E4M3 codes included), an
+    all-zero row and a row with one outlier: codes and scales bit-exact."""
+    rng = np.random.default_rng(4)
+    rows, cols = 67, 1040
+    x = rng.standard_normal((rows, cols)).astype(np.float32)
+    x *= (10.0 ** rng.uniform(-6, 4, rows)).astype(np.float32)[:, None]
+    x[5] = 0.0
+    x[9, 17] = 3.0e4
+    xt = torch.from_numpy(x).to(getattr(torch, dtype))
+    codes, scales = _quant_dev(xt.cuda())
+    torch.cuda.synchronize()
+    oc, os_ = O.quant_e4m3_rows(xt.float().numpy())
+    assert np.array_equal(scales.cpu().numpy().view(np.uint32), os_.view(np.uint32))
+    assert np.array_equal(codes.cpu().numpy(), oc)
+    assert scales[5].item() == 1.0 and int(codes[5].abs().sum()) == 0
+    assert int(codes[9, 17]) == 0x7E  # the outlier maps to +448
+
+
+def small_latent(T=200):
+    return W.Workload("latent_small", T=T, d=256, N=32, k=4, h=128, seed=1005,
+                      act_dtype=S.DT_BF16, w_dtype="bf16", rms_inputs=True, latent=128,
+                      n_shared=2, shared_hidden=128, beta_gate=4.0, beta_up=25.0)
+
+
+def _dev_fp8(wl, dw):
+    """Device E4M3 routed experts from the bf16 ones, by the library's quantiser."""
+    out = {}
+    for name in ("w_gate", "w_up", "w_down"):
+        w = dw[name]
+        c, s = _quant_dev(w.reshape(-1, w.shape[-1]))
+        out[name] = c.reshape(w.shape)
+        out[name + "_scale"] = s
+    return out
+
+
+def _host_expert_fp8(wl, e):
+    """Oracle-side E4M3 expert e: host bf16 weights, the oracle's quantiser."""
+    l, h = wl.latent, wl.h
+    mats = []
+    for tid, rows, cols in ((W.TID_WGATE, h, l), (W.TID_WUP, h, l), (W.TID_WDOWN, l, h)):
+        codes = S.normal(wl.seed, tid, (rows, cols), W.SIGMA_W, S.DT_BF16, offset=e * rows * cols)
+        c, s = O.quant_e4m3_rows(O.decode(O.BF16, codes).astype(np.float32))
+        mats.append(O.e4m3_mat(c, s))
+    return tuple(mats)
+
+
+def _run_fp8(wl, dw, f8):
+    s = moe.shape(wl.T, wl.d, wl.N, wl.k, wl.h, 1, 0)
+    lw = moe.latent_weights(wl.latent, dw["w_dp"], dw["w_upp"], dw["shared_gate"],
+                            dw["shared_up"], dw["shared_down"], wl.n_shared, wl.shared_hidden,
+                            1e-6)
+    x = dev_u(wl)
+    y = torch.empty((wl.T, wl.d), dtype=torch.bfloat16, device="cuda")
+    i32 = dict(dtype=torch.int32, device="cuda")
+    outs = dict(top_idx=torch.empty((wl.T, wl.k), **i32), counts=torch.empty(wl.N, **i32))
+    moe.moe_latent_fwd_e4m3(s, dw["w_route"], f8["w_gate"], f8["w_up"], f8["w_down"],
+                            f8["w_gate_scale"], f8["w_up_scale"], f8["w_down_scale"], lw, x, y,
+                            a=moe.act(moe.ACT_SITU_GLU, wl.beta_gate, wl.beta_up), outputs=outs)
+    torch.cuda.synchronize()
+    return y, {k: v.cpu().numpy() for k, v in outs.items()}
+
+
+def _oracle_fp8(wl, tokens, experts):
+    x = host_u(wl)[tokens]
+    w_route = S.normal(wl.seed, W.TID_WROUTE, (wl.N, wl.d), W.SIGMA_W, S.DT_F32)
+    W_dp, W_upp, shared = host_latent_dense(wl)
+    return O.latent_tokens(x, w_route, wl.k, W_dp, experts, W_upp, shared, wl.beta_gate,
+                           wl.beta_up, 1e-6, fp8=True)
+
+
+def test_latent_fp8_small_all_tokens():
+    """Small LatentMoE layer with E4M3 routed experts, every token: the device
+    quantiser reproduces the oracle's expert codes, routing is unchanged, and
+    y matches the oracle's FP8 form."""
+    wl = small_latent()
+    dw = dev_latent(wl)
+    f8 = _dev_fp8(wl, dw)
+    cache = {e: _host_expert_fp8(wl, e) for e in range(wl.N)}
+    for e in (0, 7, wl.N - 1):  # device codes = oracle codes, scales bit-exact
+        g, u, d = cache[e]
+        assert np.array_equal(f8["w_gate"][e].cpu().numpy(), g.data)
+        assert np.array_equal(f8["w_down"][e].cpu().numpy(), d.data)
+        assert np.array_equal(f8["w_up_scale"][e * wl.h:(e + 1) * wl.h].cpu().numpy(),
+                              u.row_scale)
+    y, outs = _run_fp8(wl, dw, f8)
+    idx, _, ref = _oracle_fp8(wl, np.arange(wl.T), cache.__getitem__)
+    assert np.array_equal(outs["top_idx"], idx)
+    assert outs["counts"].sum() == wl.k * wl.T
+    got = y.float().cpu().numpy()
+    assert np.all(np.isfinite(got))
+    assert rel_err(got, ref) < TOL
+    # the FP8 layer differs from the bf16 one by the quantisation error only
+    _, _, ref_bf16 = O.latent_tokens(host_u(wl), S.normal(wl.seed, W.TID_WROUTE,
+                                                          (wl.N, wl.d), W.SIGMA_W, S.DT_F32),
+                                     wl.k, *_dense_and_bf16_experts(wl))
+    assert 1e-3 < rel_err(got, ref_bf16) < 0.2
+
+
+def _dense_and_bf16_experts(wl):
+    from inputs import host_latent_expert
+    W_dp, W_upp, shared = host_latent_dense(wl)
+    return (W_dp, lambda e: host_latent_expert(wl, e), W_upp, shared, wl.beta_gate, wl.beta_up,
+            1e-6)
+
+
+def test_latent_fp8_full_size_sampled():
+    """The LatentMoE-shaped layer at full size with E4M3 routed experts:
+    routing of every token unchanged against the bf16 oracle routing, outputs
+    on sampled tokens against the oracle's FP8 form (their 16 experts each
+    quantised on the host by the oracle)."""
+    wl = W.latent()
+    dw = dev_latent(wl)
+    f8 = _dev_fp8(wl, dw)
+    for name in ("w_gate", "w_up", "w_down"):
+        del dw[name]  # the bf16 routed experts are no longer needed
+    torch.cuda.empty_cache()
+    y, outs = _run_fp8(wl, dw, f8)
+    assert outs["counts"].sum() == wl.k * wl.T
+    tokens = np.sort(np.random.default_rng(9).choice(wl.T, 4, replace=False))
+    cache = {}
+
+    def get(e):
+        if e not in cache:
+            cache[e] = _host_expert_fp8(wl, e)
+        return cache[e]
+
+    idx, _, ref = _oracle_fp8(wl, tokens, get)
+    assert np.array_equal(outs["top_idx"][tokens], idx)
+    got = y[torch.from_numpy(tokens).long().cuda()].float().cpu().numpy()
+    assert rel_err(got, ref) < TOL

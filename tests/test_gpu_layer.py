@@ -75,7 +75,10 @@ def test_expert_ffn_f32_simt():
     ([16], 128, 64),                                   # one tile, smallest shapes
     ([0, 5, 130, 257, 16, 1, 300, 64], 512, 256),      # ragged tails, empty expert
     ([1024] * 8, 512, 128),                            # the small-model layer's shape
-    ([700, 333, 1500, 410], 512, 1024),                # 256-token tiles
+    ([700, 333, 1500, 410], 512, 1024),                # CTA pairs, 128-token tiles
+    ([1100, 257, 1500, 143], 1024, 2048),              # CTA pairs, 256-token tiles, ragged
+    ([100, 37, 260, 5], 512, 512),                     # CTA pairs, few rows per expert
+    ([300, 0, 77, 513], 384, 320),                     # single-CTA tiles (h % 128 != 0)
 ])
 def test_expert_ffn_bf16_tensor_cores(counts, width, h):
     got, ref = _ffn_case(counts, width, h, S.DT_BF16, sample=600)
