@@ -250,6 +250,46 @@ MOE_API int moe_layer_fwd(const moe_shape* shape, const moe_layer_weights* w, co
                   int32_t act_dtype, void* y, const moe_layer_outputs* out, void* ws,
                   size_t ws_bytes, void* stream);
 
+/* ---------------------------------------------------------- layer backward */
+/* Gradients of L = sum_t dy_t . y_t + alpha N sum_i f_i P_i for the bf16 layer
+ * of moe_layer_fwd (tutorial §3.1, §3.2; §3.4 P_i = mean_t p_ti; §3.7 the
+ * balancing term's gradient with the loads f held fixed), with the forward's
+ * selected sets and capacity drops held fixed (top-k and the capacity cut
+ * are piecewise constant): a dropped dispatch gets no gradient, and only the
+ * selected experts of kept dispatches get weight gradient.
+ *   dz [T][N]         dL/dz (router logits): renormalisation and softmax
+ *                     backward of da_s = dy_t . F_{e_s}(u_t), plus the term
+ *                     (alpha N / T) p_tj (f_j - sum_i f_i p_ti) when f != NULL
+ *   du [T][d]         dL/du: the experts' input gradients of the kept slots
+ *                     plus sum_j dz_tj W_route[j]
+ *   dw_route [N][d]   sum_t dz_t u_t^T (nullable: not formed)
+ *   dw_gate, dw_up [N][h][d], dw_down [N][d][h]   every expert's matrix,
+ *                     zero for an expert with no kept dispatch
+ * All fp32, device, caller-owned, fully overwritten. */
+typedef struct {
+  float* du;
+  float* dz;
+  float* dw_route;
+  float* dw_gate;
+  float* dw_up;
+  float* dw_down;
+} moe_layer_grads;
+
+MOE_API size_t moe_layer_bwd_workspace_bytes(const moe_shape* shape);
+/* shape, w, u as for moe_layer_fwd (bf16 experts; h and d multiples of 128);
+ * dy [T][d] bf16; fwd: the forward's top_idx, top_w, probs, offsets,
+ * perm_tok and row_of (moe_layer_fwd fills them when they are requested in
+ * its outputs).  The expert GEMMs run on the tensor cores (bf16 operands,
+ * fp32 accumulate, the weights and token rows read in their stored layout);
+ * every reduction has a fixed order, so the result is reproducible.
+ * Returns MOE_ERR_INVALID_ARG for NULL or misaligned pointers or unsupported
+ * widths, MOE_ERR_UNSUPPORTED for non-bf16 experts, MOE_ERR_WORKSPACE for a
+ * short workspace. */
+MOE_API int moe_layer_bwd(const moe_shape* shape, const moe_layer_weights* w, const void* u,
+                          const void* dy, const moe_layer_outputs* fwd, float alpha,
+                          const float* f, const moe_layer_grads* grads, void* ws,
+                          size_t ws_bytes, void* stream);
+
 /* -------------------------------------------------------------- LatentMoE */
 /* Latent-space MoE layer (Stable LatentMoE demo document: width separation,
  * RMSNorm before the up-projection, SiTU-GLU soft caps).  The routed experts
@@ -427,6 +467,68 @@ MOE_API int moe_ep_plan(int32_t world, int32_t rank, int32_t N, int32_t capacity
                         const int32_t* counts_all, int32_t* kept, int32_t* local_offsets,
                         int32_t* send_base, int32_t* send_counts, int32_t* recv_offsets,
                         int32_t* recv_src_base, int32_t* recv_counts, int32_t* overflow);
+
+/* Expert parallelism, device side: the dispatch and combine all-to-alls the
+ * tutorial names as the multi-device cost of experts split over devices,
+ * each fused with its neighbouring step (the gather, the weighted combine).
+ * Rank r owns experts [r E, (r+1) E), E = N / world.  Every rank holds, in
+ * its own device memory, the buffers below; the peer_* arrays (device
+ * memory, [world] entries) hold every rank's buffers as addresses this
+ * device can load and store (peer memory over NVLink after
+ * cudaDeviceEnablePeerAccess or an IPC / symmetric-memory mapping; plain
+ * device addresses when the ranks share one device).  No TMA and no
+ * multicast touch peer memory: plain loads and stores only. */
+typedef struct {
+  int32_t world, rank;
+  int32_t recv_capacity;       /* rows of recv_rows / out_rows on every rank */
+  void* recv_rows;             /* this rank: received token rows, bf16 [recv_capacity][d] */
+  float* recv_w;               /* this rank: their combine weights [recv_capacity] */
+  void* out_rows;              /* this rank: weighted expert outputs a * F(u), bf16 */
+  uint32_t* arrive;            /* this rank: arrival flags [world], one per source */
+  uint32_t* done;              /* this rank: one flag, experts finished */
+  void* const* peer_recv_rows; /* [world] every rank's recv_rows */
+  float* const* peer_recv_w;   /* [world] every rank's recv_w */
+  void* const* peer_out_rows;  /* [world] every rank's out_rows */
+  uint32_t* const* peer_arrive;/* [world] every rank's arrive */
+  uint32_t* const* peer_done;  /* [world] every rank's done */
+} moe_ep_buffers;
+
+/* One step, per rank, on its stream, in this order (epoch = the step number,
+ * starting at 1; flags are never reset, a later epoch supersedes):
+ *   moe_route, moe_permute with capacity 0 (counts, offsets, perm_tok, row_of
+ *   of this rank's dispatches), an all-gather of the counts (NCCL), then
+ *   moe_ep_plan on the host and a copy of kept / send_base to the device;
+ *   moe_ep_dispatch: every kept dispatch's row of u (bf16 [T][d]) and its
+ *     combine weight top_w are stored into the owner's recv buffers at the
+ *     plan's row; the last CTA raises arrive[rank] on every rank (release,
+ *     system scope) -- also when this rank sends nothing;
+ *   moe_ep_expert_ffn: waits until every source's arrival flag reached epoch,
+ *     runs this rank's E experts (moe_expert_ffn's kernels; expert_shape:
+ *     T = recv_capacity, k = 1, N = E, d, h) on the received rows grouped by
+ *     recv_offsets [E+1] (the plan's), stores bf16 rows a * F(u) into
+ *     out_rows and raises done;
+ *   moe_ep_combine: waits until every rank's done flag reached epoch, then
+ *     y_t = sum over kept slots (ascending s) of the owners' out_rows rows,
+ *     loaded from their memory; y bf16 [T][d], fully overwritten.
+ * With the plan's global order (rank 0's rows of an expert first), y equals
+ * the single-device layer on the ranks' batches laid end to end.  A rank
+ * reuses its buffers next step only after its own combine, which follows
+ * every owner's done flag, so the flags order every overwrite.  Every wait
+ * is bounded (about 2 s) and records MOE_ERR_TIMEOUT in the status word; a
+ * destination row beyond recv_capacity records MOE_ERR_BOUNDS and is not
+ * stored.  ws: moe_ep_workspace_bytes(expert_shape), separate per rank. */
+MOE_API size_t moe_ep_workspace_bytes(const moe_shape* expert_shape);
+MOE_API int moe_ep_dispatch(const moe_shape* shape, const moe_ep_buffers* bufs, uint32_t epoch,
+                            const void* u, const int32_t* perm_tok, const int32_t* offsets,
+                            const int32_t* row_of, const float* top_w, const int32_t* kept,
+                            const int32_t* send_base, void* ws, size_t ws_bytes, void* stream);
+MOE_API int moe_ep_expert_ffn(const moe_shape* expert_shape, const moe_ep_buffers* bufs,
+                              uint32_t epoch, const int32_t* recv_offsets, const void* w_gate,
+                              const void* w_up, const void* w_down, const moe_act* act, void* ws,
+                              size_t ws_bytes, void* stream);
+MOE_API int moe_ep_combine(const moe_shape* shape, const moe_ep_buffers* bufs, uint32_t epoch,
+                           const int32_t* top_idx, const int32_t* row_of, const int32_t* offsets,
+                           const int32_t* kept, const int32_t* send_base, void* y, void* stream);
 
 /* ----------------------------------------------------------- diagnostics */
 /* Human-readable name of a status code (static string). */

@@ -56,8 +56,18 @@ class MoeLatentWeights(ctypes.Structure):
                 ("shared_up", _vp), ("shared_down", _vp), ("rms_eps", _f32)]
 
 
+class MoeLayerGrads(ctypes.Structure):
+    _fields_ = [(n, _vp) for n in ("du", "dz", "dw_route", "dw_gate", "dw_up", "dw_down")]
+
+
 class MoeE4M3Scales(ctypes.Structure):
     _fields_ = [(n, _vp) for n in ("gate_scale", "up_scale", "down_scale")]
+
+
+class MoeEpBuffers(ctypes.Structure):
+    _fields_ = [("world", _i32), ("rank", _i32), ("recv_capacity", _i32)] + [
+        (n, _vp) for n in ("recv_rows", "recv_w", "out_rows", "arrive", "done", "peer_recv_rows",
+                           "peer_recv_w", "peer_out_rows", "peer_arrive", "peer_done")]
 
 
 _P_SHAPE = ctypes.POINTER(MoeShape)
@@ -78,6 +88,10 @@ _PROTOS = {
     "moe_layer_workspace_bytes": (_sz, [_P_SHAPE, _i32]),
     "moe_layer_fwd": (_i32, [_P_SHAPE, ctypes.POINTER(MoeLayerWeights), _vp, _i32, _vp,
                              ctypes.POINTER(MoeLayerOutputs), _vp, _sz, _vp]),
+    "moe_layer_bwd_workspace_bytes": (_sz, [_P_SHAPE]),
+    "moe_layer_bwd": (_i32, [_P_SHAPE, ctypes.POINTER(MoeLayerWeights), _vp, _vp,
+                             ctypes.POINTER(MoeLayerOutputs), _f32, _vp,
+                             ctypes.POINTER(MoeLayerGrads), _vp, _sz, _vp]),
     "moe_latent_workspace_bytes": (_sz, [_P_SHAPE, ctypes.POINTER(MoeLatentWeights)]),
     "moe_latent_fwd": (_i32, [_P_SHAPE, ctypes.POINTER(MoeLayerWeights),
                               ctypes.POINTER(MoeLatentWeights), _vp, _vp,
@@ -97,6 +111,13 @@ _PROTOS = {
     "moe_quantile_balance": (_i32, [_i32, _i32, _i32, _vp, _vp, _i32, _i32, _vp, _vp, _vp, _vp,
                                     _vp, _sz, _vp]),
     "moe_ep_plan": (_i32, [_i32, _i32, _i32, _i32] + [_vp] * 9),
+    "moe_ep_workspace_bytes": (_sz, [_P_SHAPE]),
+    "moe_ep_dispatch": (_i32, [_P_SHAPE, ctypes.POINTER(MoeEpBuffers), ctypes.c_uint32] +
+                        [_vp] * 7 + [_vp, _sz, _vp]),
+    "moe_ep_expert_ffn": (_i32, [_P_SHAPE, ctypes.POINTER(MoeEpBuffers), ctypes.c_uint32, _vp,
+                                 _vp, _vp, _vp, ctypes.POINTER(MoeAct), _vp, _sz, _vp]),
+    "moe_ep_combine": (_i32, [_P_SHAPE, ctypes.POINTER(MoeEpBuffers), ctypes.c_uint32] +
+                       [_vp] * 6 + [_vp]),
     "moe_status_string": (ctypes.c_char_p, [_i32]),
     "moe_device_status": (_i32, [_vp, ctypes.POINTER(_i32)]),
     "moe_reset_device_status": (_i32, [_vp]),
@@ -323,6 +344,42 @@ def moe_layer_fwd(s: MoeShape, w_route, w_gate, w_up, w_down, u, y, bias=None, a
                               ctypes.byref(O), _ptr(wbuf), wlen, _stream(stream)), "moe_layer_fwd")
 
 
+def moe_layer_bwd_workspace_bytes(s: MoeShape) -> int:
+    return int(_lib.moe_layer_bwd_workspace_bytes(ctypes.byref(s)))
+
+
+def moe_layer_bwd(s: MoeShape, w_route, w_gate, w_up, w_down, u, dy, fwd: dict, grads: dict,
+                  bias=None, a=None, alpha: float = 0.0, f=None, ws=None, stream=None):
+    """Layer backward (include/moe.h): fwd holds the forward's top_idx, top_w,
+    probs, offsets, perm_tok, row_of; grads the fp32 outputs du, dz, dw_route
+    (optional), dw_gate, dw_up, dw_down; f (optional) the loads of the
+    balancing term."""
+    a = a or act()
+    Tk = s.T * s.k
+    for args in (("u", u, s.T * s.d, _BF16), ("dy", dy, s.T * s.d, _BF16),
+                 ("w_route", w_route, s.N * s.d, _F32), ("bias", bias, s.N, _F32),
+                 ("w_gate", w_gate, s.N * s.h * s.d, _BF16), ("w_up", w_up, s.N * s.h * s.d, _BF16),
+                 ("w_down", w_down, s.N * s.d * s.h, _BF16), ("f", f, s.N, _F32),
+                 ("top_idx", fwd.get("top_idx"), Tk, _I32), ("top_w", fwd.get("top_w"), Tk, _F32),
+                 ("probs", fwd.get("probs"), s.T * s.N, _F32),
+                 ("offsets", fwd.get("offsets"), s.N + 1, _I32),
+                 ("perm_tok", fwd.get("perm_tok"), 0, _I32), ("row_of", fwd.get("row_of"), Tk, _I32),
+                 ("du", grads.get("du"), s.T * s.d, _F32), ("dz", grads.get("dz"), s.T * s.N, _F32),
+                 ("dw_route", grads.get("dw_route"), s.N * s.d, _F32),
+                 ("dw_gate", grads.get("dw_gate"), s.N * s.h * s.d, _F32),
+                 ("dw_up", grads.get("dw_up"), s.N * s.h * s.d, _F32),
+                 ("dw_down", grads.get("dw_down"), s.N * s.d * s.h, _F32)):
+        _need(*args)
+    W = MoeLayerWeights(_ptr(w_route), _ptr(bias), _ptr(w_gate), _ptr(w_up), _ptr(w_down), BF16, a)
+    O = _outputs(s, fwd)
+    G = MoeLayerGrads(*(_ptr(grads.get(n)) for n in ("du", "dz", "dw_route", "dw_gate", "dw_up",
+                                                     "dw_down")))
+    wbuf, wlen = _ws(moe_layer_bwd_workspace_bytes(s), u.device, ws)
+    _check(_lib.moe_layer_bwd(ctypes.byref(s), ctypes.byref(W), _ptr(u), _ptr(dy),
+                              ctypes.byref(O), alpha, _ptr(f), ctypes.byref(G), _ptr(wbuf), wlen,
+                              _stream(stream)), "moe_layer_bwd")
+
+
 def latent_weights(latent, w_down_proj, w_up_proj, shared_gate=None, shared_up=None,
                    shared_down=None, n_shared=0, shared_hidden=0, rms_eps=1e-6):
     return MoeLatentWeights(latent, n_shared, shared_hidden, _ptr(w_down_proj), _ptr(w_up_proj),
@@ -482,6 +539,61 @@ def moe_ep_plan(counts_all, capacity: int, rank: int) -> dict:
     _check(_lib.moe_ep_plan(world, rank, N, capacity, c.ctypes.data,
                             *[out[key].ctypes.data for key in order]), "moe_ep_plan")
     return out
+
+
+def ep_buffers(world: int, rank: int, recv_capacity: int, mine: dict, peers: dict):
+    """moe_ep_buffers of `rank`: mine holds this rank's tensors (recv_rows,
+    recv_w, out_rows, arrive, done); peers holds, per name, an int64 device
+    tensor [world] of every rank's addresses of that buffer as this device
+    sees them."""
+    return MoeEpBuffers(world, rank, recv_capacity, *(_ptr(mine[n]) for n in (
+        "recv_rows", "recv_w", "out_rows", "arrive", "done")), *(_ptr(peers[n]) for n in (
+            "recv_rows", "recv_w", "out_rows", "arrive", "done")))
+
+
+def moe_ep_workspace_bytes(expert_shape: MoeShape) -> int:
+    return int(_lib.moe_ep_workspace_bytes(ctypes.byref(expert_shape)))
+
+
+def moe_ep_dispatch(s: MoeShape, bufs: MoeEpBuffers, epoch: int, u, perm_tok, offsets, row_of,
+                    top_w, kept, send_base, ws, stream=None):
+    """Stores this rank's kept dispatch rows (and combine weights) into their
+    owners' receive buffers and raises its arrival flag on every rank."""
+    for args in (("u", u, s.T * s.d, _BF16), ("perm_tok", perm_tok, 0, _I32),
+                 ("offsets", offsets, s.N + 1, _I32), ("row_of", row_of, s.T * s.k, _I32),
+                 ("top_w", top_w, s.T * s.k, _F32), ("kept", kept, s.N, _I32),
+                 ("send_base", send_base, s.N, _I32)):
+        _need(*args)
+    _check(_lib.moe_ep_dispatch(ctypes.byref(s), ctypes.byref(bufs), epoch, _ptr(u),
+                                _ptr(perm_tok), _ptr(offsets), _ptr(row_of), _ptr(top_w),
+                                _ptr(kept), _ptr(send_base), _ptr(ws), ws.numel(),
+                                _stream(stream)), "moe_ep_dispatch")
+
+
+def moe_ep_expert_ffn(expert_shape: MoeShape, bufs: MoeEpBuffers, epoch: int, recv_offsets,
+                      w_gate, w_up, w_down, ws, a=None, stream=None):
+    """Waits for every source, runs this rank's experts on the received rows
+    and raises its done flag."""
+    s, a = expert_shape, a or act()
+    for args in (("recv_offsets", recv_offsets, s.N + 1, _I32),
+                 ("w_gate", w_gate, s.N * s.h * s.d, _BF16), ("w_up", w_up, s.N * s.h * s.d, _BF16),
+                 ("w_down", w_down, s.N * s.d * s.h, _BF16)):
+        _need(*args)
+    _check(_lib.moe_ep_expert_ffn(ctypes.byref(s), ctypes.byref(bufs), epoch, _ptr(recv_offsets),
+                                  _ptr(w_gate), _ptr(w_up), _ptr(w_down), ctypes.byref(a),
+                                  _ptr(ws), ws.numel(), _stream(stream)), "moe_ep_expert_ffn")
+
+
+def moe_ep_combine(s: MoeShape, bufs: MoeEpBuffers, epoch: int, top_idx, row_of, offsets, kept,
+                   send_base, y, stream=None):
+    """Waits for every owner, then y_t = sum of its kept slots' output rows."""
+    for args in (("top_idx", top_idx, s.T * s.k, _I32), ("row_of", row_of, s.T * s.k, _I32),
+                 ("offsets", offsets, s.N + 1, _I32), ("kept", kept, s.N, _I32),
+                 ("send_base", send_base, s.N, _I32), ("y", y, s.T * s.d, _BF16)):
+        _need(*args)
+    _check(_lib.moe_ep_combine(ctypes.byref(s), ctypes.byref(bufs), epoch, _ptr(top_idx),
+                               _ptr(row_of), _ptr(offsets), _ptr(kept), _ptr(send_base), _ptr(y),
+                               _stream(stream)), "moe_ep_combine")
 
 
 def moe_device_status(stream=None) -> int:

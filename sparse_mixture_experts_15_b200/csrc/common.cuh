@@ -226,9 +226,13 @@ int route_tokens_per_block(int N);
 // Permutation in one launch from the router's per-block counts (few experts;
 // dispatch_small_ok says when): see dispatch_small in permute.cu.
 bool dispatch_small_ok(const moe_shape& s);
+// row_w (nullable): row_w[r] = top_w of the dispatch that owns grouped row r,
+// for the down GEMM's weighted epilogue (also for launch_permute and
+// launch_route_dispatch).
 int launch_dispatch_small(const moe_shape& s, const int32_t* top_idx, const int32_t* hist,
                           int32_t* counts, int32_t* offsets, int32_t* perm_tok, int32_t* row_of,
-                          int32_t* overflow, int32_t* totals, cudaStream_t st);
+                          int32_t* overflow, int32_t* totals, cudaStream_t st,
+                          const float* top_w = nullptr, float* row_w = nullptr);
 // Router + permutation + gather in one cooperative launch (route_dispatch.cu),
 // for few experts when a CTA's token rows and the router rows fit on chip.
 bool route_dispatch_ok(const moe_shape& s, int32_t dtype);
@@ -237,7 +241,7 @@ int launch_route_dispatch(const moe_shape& s, const void* u, int32_t dtype, cons
                           const float* bias, int32_t* top_idx, float* top_w, float* probs,
                           float* logits, int32_t* counts, int32_t* offsets, int32_t* perm_tok,
                           int32_t* row_of, int32_t* overflow, int32_t* totals, void* x_rows,
-                          void* ws, cudaStream_t st);
+                          void* ws, cudaStream_t st, float* row_w = nullptr);
 size_t aux_stats_ws_bytes(int32_t N);
 int launch_aux_stats(int32_t T, int32_t N, int32_t k, const float* probs, const int32_t* top_idx,
                      float* f, float* P, float* n_sum_fP, int32_t* loads, void* ws,
@@ -245,20 +249,27 @@ int launch_aux_stats(int32_t T, int32_t N, int32_t k, const float* probs, const 
 size_t permute_ws_bytes(const moe_shape& s);
 int launch_permute(const moe_shape& s, const int32_t* top_idx, int32_t* counts, int32_t* offsets,
                    int32_t* perm_tok, int32_t* row_of, int32_t* overflow, int32_t* totals,
-                   void* ws, cudaStream_t st);
+                   void* ws, cudaStream_t st, const float* top_w = nullptr,
+                   float* row_w = nullptr);
 int launch_gather(const moe_shape& s, int32_t width, const void* u, int32_t dtype,
                   const int32_t* perm_tok, const int32_t* offsets, void* x_rows, cudaStream_t st);
 int launch_combine(const moe_shape& s, int32_t width, const float* y_rows, const int32_t* row_of,
                    const float* top_w, void* y, int32_t y_dtype, cudaStream_t st);
+// y[t] = sum over kept slots s (ascending) of rows[row_of[t][s]], bf16 rows
+// already weighted by their combine weights; fp32 sum, one rounding to y_dtype.
+int launch_combine_weighted(const moe_shape& s, int32_t width, const __nv_bfloat16* rows,
+                            const int32_t* row_of, void* y, int32_t y_dtype, cudaStream_t st);
 size_t ffn_simt_ws_bytes(const moe_shape& s);
 int launch_ffn_simt(const moe_shape& s, int32_t width, const float* x_rows, const int32_t* offsets,
                     const float* w_gate, const float* w_up, const float* w_down,
                     const moe_act& act, float* y_rows, void* ws, cudaStream_t st);
 size_t ffn_tc_ws_bytes(const moe_shape& s, int32_t width);
+// y_rows: fp32 expert outputs F(u) per grouped row, or (row_w != nullptr) bf16
+// rows already weighted, row_w[r] * F(u) (the combine then only adds them).
 int launch_ffn_tc(const moe_shape& s, int32_t width, const __nv_bfloat16* x_rows,
                   const int32_t* offsets, const __nv_bfloat16* w_gate, const __nv_bfloat16* w_up,
-                  const __nv_bfloat16* w_down, const moe_act& act, float* y_rows, void* ws,
-                  cudaStream_t st);
+                  const __nv_bfloat16* w_down, const moe_act& act, void* y_rows, void* ws,
+                  cudaStream_t st, const float* row_w = nullptr);
 
 // Gather of the expert path fused with per-token E4M3 quantisation (fp8.cu):
 // codes[r] = e4m3 codes of x[perm_tok[r]] / scales[r], rows r < offsets[N].
@@ -271,7 +282,7 @@ bool ffn_fused_ok(int width, int h, int G);
 int launch_ffn_fused(int G, int64_t R, int width, int h, const __nv_bfloat16* x_rows,
                      const int32_t* offsets, const __nv_bfloat16* w_gate,
                      const __nv_bfloat16* w_up, const __nv_bfloat16* w_down, const moe_act& act,
-                     float* y_rows, cudaStream_t st);
+                     void* y_rows, cudaStream_t st, const float* row_w = nullptr);
 
 // Grouped tcgen05 GEMM helpers (gemm_tc.cu).
 enum TcMode { MODE_GATEUP = 0, MODE_STORE_F32 = 1, MODE_STORE_BF16 = 2 };
@@ -306,7 +317,11 @@ int tc_gateup(const int32_t* offsets, int T, int G, const void* X, int64_t x_row
 // Store-mode GEMM over 1..3 K-segments accumulated into one fp32 tile:
 // out[row][g * m_rows + m] = sum_s A_s[g * a_rows + arow_s + m] . B_s[row][bcol_s ...].
 // f8: one segment of E4M3 operands, fp32 output scaled by the row scales.
+// b_row_scale (nullable): a factor per token row, applied to the fp32 result
+// before the store (the combine weights of the grouped rows); with f8, its
+// b_scale plays this part.
 int tc_store(const int32_t* offsets, int T, int G, int m_rows, const TcSeg* segs, int nseg,
-             void* out, int mode, int out_ld, cudaStream_t st, const TcF8* f8 = nullptr);
+             void* out, int mode, int out_ld, cudaStream_t st, const TcF8* f8 = nullptr,
+             const float* b_row_scale = nullptr);
 
 }  // namespace moe

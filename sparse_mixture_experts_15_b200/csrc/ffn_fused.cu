@@ -38,7 +38,8 @@ struct FusedParams {
   const int32_t* offsets;
   int G, width, h;
   float beta_g, beta_u;
-  float* y_rows;  // [R][width]
+  void* y_rows;         // [R][width] fp32, or bf16 weighted rows when row_w is set
+  const float* row_w;   // nullable: combine weight of each grouped row
   int* status;
 };
 
@@ -349,9 +350,19 @@ __global__ void __launch_bounds__(fThreads, 1) tc_fused_ffn(const __grid_constan
           float v[32];
           tc::tmem_ld_32x32b_x32(
               tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)((mA + m2) * fBN + c), v);
+          if (p.row_w) {  // a * F(u) as bf16: the combine only adds the rows
+            __nv_bfloat16* yb = static_cast<__nv_bfloat16*>(p.y_rows);
 #pragma unroll
-          for (int j = 0; j < 32; ++j)
-            if (c + j < n_valid) p.y_rows[(size_t)(tok0 + c + j) * p.width + col] = v[j];
+            for (int j = 0; j < 32; ++j)
+              if (c + j < n_valid)
+                yb[(size_t)(tok0 + c + j) * p.width + col] =
+                    __float2bfloat16_rn(v[j] * p.row_w[tok0 + c + j]);
+          } else {
+            float* yf = static_cast<float*>(p.y_rows);
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (c + j < n_valid) yf[(size_t)(tok0 + c + j) * p.width + col] = v[j];
+          }
         }
       }
       tc::tc_fence_before();
@@ -404,7 +415,7 @@ bool ffn_fused_ok(int width, int h, int G) {
 int launch_ffn_fused(int G, int64_t R, int width, int h, const __nv_bfloat16* x_rows,
                      const int32_t* offsets, const __nv_bfloat16* w_gate,
                      const __nv_bfloat16* w_up, const __nv_bfloat16* w_down, const moe_act& act,
-                     float* y_rows, cudaStream_t st) {
+                     void* y_rows, cudaStream_t st, const float* row_w) {
   if (R == 0) return MOE_OK;
   FusedParams p{};
   if (!make_map(&p.map_g, w_gate, (uint64_t)G * h, width, 64) ||
@@ -419,6 +430,7 @@ int launch_ffn_fused(int G, int64_t R, int width, int h, const __nv_bfloat16* x_
   p.beta_g = act.beta_gate;
   p.beta_u = act.beta_up;
   p.y_rows = y_rows;
+  p.row_w = row_w;
   p.status = status_word();
   static bool configured[64] = {false};
   int dev = 0;

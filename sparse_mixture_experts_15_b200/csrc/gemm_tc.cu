@@ -72,8 +72,10 @@ struct TcParams {
   int out_col_group;      // output column offset per group (groups sharing tokens)
   int* status;
   // E4M3 operands only: fp32 scale per row of A (gate/up mode: gate rows in
-  // a_scale[0], up rows in a_scale[1]) and per row of B (nullable: scale 1);
-  // the operand value is scale * e4m3(code).
+  // a_scale[0], up rows in a_scale[1]); the operand value is
+  // scale * e4m3(code).  b_scale (nullable): a factor per row of B, the
+  // token rows (E4M3 token scales, or the combine weight a of each grouped
+  // row, so the down GEMM stores a * F(u)).
   const float* a_scale[2];
   const float* b_scale;
 };
@@ -415,7 +417,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_grouped_gemm(const __grid_cons
       for (int c = 0; c < n_valid; c += 32) {
         float v[32];
         tc::tmem_ld_32x32b_x32(t_row + (uint32_t)c, v);
-        if (F8) {
+        if (F8 || p.b_scale) {  // row scales of A (E4M3) and of B (E4M3, or combine weights)
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
             const float bs = p.b_scale && c + j < n_valid ? p.b_scale[tok0 + c + j] : 1.0f;
@@ -660,19 +662,20 @@ size_t ffn_tc_ws_bytes(const moe_shape& s, int32_t /*width*/) {
 
 int launch_ffn_tc(const moe_shape& s, int32_t width, const __nv_bfloat16* x_rows,
                   const int32_t* offsets, const __nv_bfloat16* w_gate, const __nv_bfloat16* w_up,
-                  const __nv_bfloat16* w_down, const moe_act& act, float* y_rows, void* ws,
-                  cudaStream_t st) {
+                  const __nv_bfloat16* w_down, const moe_act& act, void* y_rows, void* ws,
+                  cudaStream_t st, const float* row_w) {
   const int64_t R = (int64_t)s.T * s.k;
   if (R == 0) return MOE_OK;
   if (ffn_fused_ok(width, s.h, s.N))  // small h: both GEMMs in one launch, H stays on chip
     return launch_ffn_fused(s.N, R, width, s.h, x_rows, offsets, w_gate, w_up, w_down, act,
-                            y_rows, st);
+                            y_rows, st, row_w);
   __nv_bfloat16* H = static_cast<__nv_bfloat16*>(ws);
   int rc = tc_gateup(offsets, (int)R, s.N, x_rows, R, width, w_gate, w_up, s.h, act, H, s.h, 0,
                      st);
   if (rc != MOE_OK) return rc;
   TcSeg seg{w_down, (int64_t)s.N * width, s.h, 0, H, R, s.h, 0};
-  return tc_store(offsets, (int)R, s.N, width, &seg, 1, y_rows, MODE_STORE_F32, width, st);
+  return tc_store(offsets, (int)R, s.N, width, &seg, 1, y_rows,
+                  row_w ? MODE_STORE_BF16 : MODE_STORE_F32, width, st, nullptr, row_w);
 }
 
 // Gate/up GEMM with the fused activation: for group g and its rows of X,
@@ -720,10 +723,10 @@ int tc_gateup(const int32_t* offsets, int T, int G, const void* X, int64_t x_row
 // Plain GEMM over 1..3 K-segments accumulated into one output:
 // out[row][g * m_rows + m] = sum_s (A_s[g * a_rows_s + arow_s + m] . B_s[row][bcol_s + ...]).
 int tc_store(const int32_t* offsets, int T, int G, int m_rows, const TcSeg* segs, int nseg,
-             void* out, int mode, int out_ld, cudaStream_t st, const TcF8* f8) {
+             void* out, int mode, int out_ld, cudaStream_t st, const TcF8* f8,
+             const float* b_row_scale) {
   if (nseg < 1 || nseg > kMaxSeg) return MOE_ERR_INVALID_ARG;
-  if (f8 && (nseg != 1 || mode != MODE_STORE_F32 || segs[0].K % (2 * kBK) != 0))
-    return MOE_ERR_UNSUPPORTED;
+  if (f8 && (nseg != 1 || segs[0].K % (2 * kBK) != 0)) return MOE_ERR_UNSUPPORTED;
   const bool u8 = f8 != nullptr;
   const int ke = u8 ? 2 * kBK : kBK;
   TcParams p{};
@@ -773,6 +776,7 @@ int tc_store(const int32_t* offsets, int T, int G, int m_rows, const TcSeg* segs
   p.out_ld = out_ld;
   p.out_col_group = 0;
   p.status = status_word();
+  p.b_scale = b_row_scale;
   if (f8) {
     p.a_scale[0] = f8->a_scale[0];
     p.b_scale = f8->b_scale;

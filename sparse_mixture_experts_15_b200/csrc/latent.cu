@@ -63,7 +63,8 @@ struct LatentBufs {
   __nv_bfloat16* x_rows;  // E4M3 experts: the gathered codes of x_l (1 byte each)
   float* x_scale;         // E4M3 experts: one scale per gathered row
   __nv_bfloat16* H;       // E4M3 experts: H as codes
-  float* y_rows;
+  float* y_rows;  // bf16 rows a * E(x_l) (half the room used)
+  float* row_w;   // combine weight of each grouped row
   float* m;
   __nv_bfloat16* m_hat;
   __nv_bfloat16* H_sh;
@@ -91,6 +92,7 @@ LatentBufs carve_latent(const moe_shape& s, const moe_latent_weights& lw, void* 
   b.x_scale = c.take<float>(Tk);
   b.H = c.take<__nv_bfloat16>(Tk * s.h);
   b.y_rows = c.take<float>(Tk * l);
+  b.row_w = c.take<float>(Tk);
   b.m = c.take<float>((size_t)s.T * l);
   b.m_hat = c.take<__nv_bfloat16>((size_t)s.T * l);
   b.H_sh = c.take<__nv_bfloat16>((size_t)s.T * (lw.n_shared > 0 ? lw.n_shared : 1) *
@@ -172,7 +174,7 @@ int latent_forward(const moe_shape* shape, const moe_layer_weights* w,
                           b.stats_ws, st);
   if (rc == MOE_OK)
     rc = launch_permute(s, top_idx, counts, offsets, perm_tok, row_of, overflow, totals,
-                        b.permute_ws, st);
+                        b.permute_ws, st, top_w, b.row_w);
   if (rc != MOE_OK) return rc;
   // x_l = W_dp x (width separation: routed experts work in l < d)
   {
@@ -184,7 +186,7 @@ int latent_forward(const moe_shape* shape, const moe_layer_weights* w,
     // E4M3 experts: x_l quantised per token while it is gathered; gate/up
     // with the row scales, H stored as E4M3 codes; down with its row scales
     TcF8 gu{{e4m3->gate_scale, e4m3->up_scale}, b.x_scale};
-    TcF8 dn{{e4m3->down_scale, nullptr}, nullptr};
+    TcF8 dn{{e4m3->down_scale, nullptr}, b.row_w};
     rc = launch_quant_gather_e4m3(s, l, b.x_l, perm_tok, offsets,
                                   reinterpret_cast<uint8_t*>(b.x_rows), b.x_scale, st);
     if (rc == MOE_OK)
@@ -192,7 +194,7 @@ int latent_forward(const moe_shape* shape, const moe_layer_weights* w,
                      0, st, &gu);
     if (rc != MOE_OK) return rc;
     TcSeg seg{w->w_down, (int64_t)s.N * l, s.h, 0, b.H, Tk, s.h, 0};
-    rc = tc_store(offsets, Tk, s.N, l, &seg, 1, b.y_rows, MODE_STORE_F32, l, st, &dn);
+    rc = tc_store(offsets, Tk, s.N, l, &seg, 1, b.y_rows, MODE_STORE_BF16, l, st, &dn);
     if (rc != MOE_OK) return rc;
   } else {
     rc = launch_gather(s, l, b.x_l, MOE_BF16, perm_tok, offsets, b.x_rows, st);
@@ -201,10 +203,13 @@ int latent_forward(const moe_shape* shape, const moe_layer_weights* w,
                    0, st);
     if (rc != MOE_OK) return rc;
     TcSeg seg{w->w_down, (int64_t)s.N * l, s.h, 0, b.H, Tk, s.h, 0};
-    rc = tc_store(offsets, Tk, s.N, l, &seg, 1, b.y_rows, MODE_STORE_F32, l, st);
+    rc = tc_store(offsets, Tk, s.N, l, &seg, 1, b.y_rows, MODE_STORE_BF16, l, st, nullptr,
+                  b.row_w);
     if (rc != MOE_OK) return rc;
   }
-  rc = launch_combine(s, l, b.y_rows, row_of, top_w, b.m, MOE_F32, st);
+  // the down GEMMs stored bf16 rows a * E(x_l): the combine adds them
+  rc = launch_combine_weighted(s, l, reinterpret_cast<const __nv_bfloat16*>(b.y_rows), row_of,
+                               b.m, MOE_F32, st);
   if (rc != MOE_OK) return rc;
   {
     int blocks = (s.T + 7) / 8;

@@ -24,7 +24,8 @@ struct LayerBufs {
   void* permute_ws;
   void* x_rows;
   void* ffn_ws;
-  float* y_rows;
+  float* y_rows;  // bf16 layers: bf16 rows a * F(u) (half the room used)
+  float* row_w;   // combine weight of each grouped row
   void* stats_ws;
   void* rd_ws;
   size_t bytes;
@@ -59,15 +60,19 @@ LayerBufs carve_layer(const moe_shape& s, int32_t act_dtype, void* base) {
   b.x_rows = c.take<char>(Tk * s.d * dtype_bytes(act_dtype));
   b.ffn_ws = c.take<char>(ffn_ws_bytes(s, s.d, act_dtype));
   b.y_rows = c.take<float>(Tk * s.d);
+  b.row_w = c.take<float>(Tk);
   b.stats_ws = c.take<char>(aux_stats_ws_bytes(s.N));
   b.rd_ws = c.take<char>(route_dispatch_ws_bytes(s));
   b.bytes = c.used();
   return b;
 }
 
+// row_w (bf16 only, nullable): store bf16 rows row_w[r] * F(u) into y_rows
+// instead of fp32 F(u).
 int run_ffn(const moe_shape& s, int32_t width, const void* x_rows, int32_t dtype,
             const int32_t* offsets, const void* w_gate, const void* w_up, const void* w_down,
-            const moe_act& act, float* y_rows, void* ws, cudaStream_t st) {
+            const moe_act& act, float* y_rows, void* ws, cudaStream_t st,
+            const float* row_w = nullptr) {
   if (dtype == MOE_F32) {
     return launch_ffn_simt(s, width, static_cast<const float*>(x_rows), offsets,
                            static_cast<const float*>(w_gate), static_cast<const float*>(w_up),
@@ -76,7 +81,7 @@ int run_ffn(const moe_shape& s, int32_t width, const void* x_rows, int32_t dtype
   return launch_ffn_tc(s, width, static_cast<const __nv_bfloat16*>(x_rows), offsets,
                        static_cast<const __nv_bfloat16*>(w_gate),
                        static_cast<const __nv_bfloat16*>(w_up),
-                       static_cast<const __nv_bfloat16*>(w_down), act, y_rows, ws, st);
+                       static_cast<const __nv_bfloat16*>(w_down), act, y_rows, ws, st, row_w);
 }
 
 bool act_ok(const moe_act* a) {
@@ -148,6 +153,10 @@ extern "C" int moe_layer_fwd(const moe_shape* shape, const moe_layer_weights* w,
   int32_t* overflow = o.overflow ? o.overflow : b.overflow;
   int32_t* totals = o.totals ? o.totals : b.totals;
   cudaStream_t st = as_stream(stream);
+  // bf16 layers: the permutation records each grouped row's combine weight,
+  // the down GEMM stores bf16 rows a * F(u), and the combine adds them (the
+  // down projection carries the multiply of the weighted combine y = sum a F)
+  float* row_w = act_dtype == MOE_BF16 ? b.row_w : nullptr;
 
   int rc;
   if (route_dispatch_ok(s, act_dtype)) {
@@ -155,7 +164,7 @@ extern "C" int moe_layer_fwd(const moe_shape* shape, const moe_layer_weights* w,
     // one cooperative launch.
     rc = launch_route_dispatch(s, u, act_dtype, w->w_route, w->bias, top_idx, top_w, probs,
                                nullptr, counts, offsets, perm_tok, row_of, overflow, totals,
-                               b.x_rows, b.rd_ws, st);
+                               b.x_rows, b.rd_ws, st, row_w);
     if (rc == MOE_OK && want_stats)
       rc = launch_aux_stats(s.T, s.N, s.k, probs, top_idx, o.f, o.P, o.n_sum_fP, nullptr,
                             b.stats_ws, st);
@@ -175,16 +184,19 @@ extern "C" int moe_layer_fwd(const moe_shape* shape, const moe_layer_weights* w,
     }
     if (small) {
       rc = launch_dispatch_small(s, top_idx, hist, counts, offsets, perm_tok, row_of, overflow,
-                                 totals, st);
+                                 totals, st, top_w, row_w);
     } else {
       rc = launch_permute(s, top_idx, counts, offsets, perm_tok, row_of, overflow, totals,
-                          b.permute_ws, st);
+                          b.permute_ws, st, top_w, row_w);
     }
     if (rc == MOE_OK) rc = launch_gather(s, s.d, u, act_dtype, perm_tok, offsets, b.x_rows, st);
     if (rc != MOE_OK) return rc;
   }
   rc = run_ffn(s, s.d, b.x_rows, act_dtype, offsets, w->w_gate, w->w_up, w->w_down, w->act,
-               b.y_rows, b.ffn_ws, st);
+               b.y_rows, b.ffn_ws, st, row_w);
   if (rc != MOE_OK) return rc;
+  if (row_w)
+    return launch_combine_weighted(s, s.d, reinterpret_cast<const __nv_bfloat16*>(b.y_rows),
+                                   row_of, y, act_dtype, st);
   return launch_combine(s, s.d, b.y_rows, row_of, top_w, y, act_dtype, st);
 }

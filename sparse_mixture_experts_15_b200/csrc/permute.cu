@@ -122,7 +122,8 @@ __global__ void __launch_bounds__(1024)
 __global__ void __launch_bounds__(kChunk)
     permute_scatter(const int32_t* __restrict__ idx, int64_t total, int k, int N, int C,
                     const int32_t* __restrict__ base, const int32_t* __restrict__ offsets,
-                    int32_t* __restrict__ perm_tok, int32_t* __restrict__ row_of) {
+                    int32_t* __restrict__ perm_tok, int32_t* __restrict__ row_of,
+                    const float* __restrict__ top_w, float* __restrict__ row_w) {
   pdl_wait();
   pdl_allow_next();
   extern __shared__ int32_t wcnt[];  // [8][N]
@@ -153,6 +154,7 @@ __global__ void __launch_bounds__(kChunk)
     const int r = offsets[e] + rank;
     row_of[x] = r;
     perm_tok[r] = (int32_t)(x / k);
+    if (row_w) row_w[r] = top_w[x];  // the combine weight of grouped row r
   }
 }
 
@@ -172,7 +174,8 @@ __global__ void __launch_bounds__(512)
                    int32_t* __restrict__ counts,
                    int32_t* __restrict__ offsets, int32_t* __restrict__ overflow,
                    int32_t* __restrict__ totals, int32_t* __restrict__ perm_tok,
-                   int32_t* __restrict__ row_of, int* status) {
+                   int32_t* __restrict__ row_of, const float* __restrict__ top_w,
+                   float* __restrict__ row_w, int* status) {
   pdl_wait();
   pdl_allow_next();
   __shared__ int hist_s[kDispatchMaxHist];
@@ -252,6 +255,7 @@ __global__ void __launch_bounds__(512)
     if (!(C > 0 && rank >= C)) {
       row = off_s[e] + rank;
       perm_tok[row] = (int32_t)(x / k);
+      if (row_w) row_w[row] = top_w[x];
     }
   }
   row_of[x] = row;
@@ -267,7 +271,7 @@ size_t permute_ws_bytes(const moe_shape& s) {
 
 int launch_permute(const moe_shape& s, const int32_t* top_idx, int32_t* counts, int32_t* offsets,
                    int32_t* perm_tok, int32_t* row_of, int32_t* overflow, int32_t* totals,
-                   void* ws, cudaStream_t st) {
+                   void* ws, cudaStream_t st, const float* top_w, float* row_w) {
   const int64_t total = (int64_t)s.T * s.k;
   const int nblk = (int)((total + kChunk - 1) / kChunk);
   int32_t* hist = static_cast<int32_t*>(ws);
@@ -279,9 +283,8 @@ int launch_permute(const moe_shape& s, const int32_t* top_idx, int32_t* counts, 
   launch_pdl(permute_scan, dim3(1), dim3(1024), 0, st, hist, nblk, s.N, s.capacity, counts, offsets, overflow, totals);
   if (nblk > 0) {
     MOE_PREFER_SHARED((permute_scatter));
-    launch_pdl(permute_scatter, dim3(nblk), dim3(kChunk), (size_t)s.N * 8 * 4, st, top_idx, total, s.k, s.N,
-                                                               s.capacity, hist, offsets,
-                                                               perm_tok, row_of);
+    launch_pdl(permute_scatter, dim3(nblk), dim3(kChunk), (size_t)s.N * 8 * 4, st, top_idx,
+               total, s.k, s.N, s.capacity, hist, offsets, perm_tok, row_of, top_w, row_w);
   }
   return launch_status();
 }
@@ -294,7 +297,8 @@ bool dispatch_small_ok(const moe_shape& s) {
 
 int launch_dispatch_small(const moe_shape& s, const int32_t* top_idx, const int32_t* hist,
                           int32_t* counts, int32_t* offsets, int32_t* perm_tok, int32_t* row_of,
-                          int32_t* overflow, int32_t* totals, cudaStream_t st) {
+                          int32_t* overflow, int32_t* totals, cudaStream_t st,
+                          const float* top_w, float* row_w) {
   const int tpb = route_tokens_per_block(s.N);
   const int nblk = (s.T + tpb - 1) / tpb;
   const int per = tpb * s.k;  // dispatches of one router block
@@ -312,7 +316,7 @@ int launch_dispatch_small(const moe_shape& s, const int32_t* top_idx, const int3
   MOE_PREFER_SHARED((dispatch_small));
   launch_pdl(dispatch_small, dim3(blocks > 0 ? blocks : 1), dim3(threads), 0, st, top_idx, total,
              s.k, s.N, s.capacity, hist, nblk, rpb, counts, offsets, overflow, totals, perm_tok,
-             row_of, status_word());
+             row_of, top_w, row_w, status_word());
   return launch_status();
 }
 

@@ -56,6 +56,7 @@ struct RDParams {
   int32_t* overflow;
   int32_t* totals;
   void* x_rows;
+  float* row_w;   // nullable: combine weight of each grouped row
   int32_t* hist;  // [grid][N] scratch
   unsigned* bar;  // [0] arrivals, [1] abort
   int* status;
@@ -279,6 +280,7 @@ __global__ void __launch_bounds__(kRDThreads, 1) route_dispatch(const __grid_con
     const int x = tb * k + tid;
     p.row_of[x] = row;
     if (row >= 0) p.perm_tok[row] = tb + tid / k;
+    if (row >= 0 && p.row_w) p.row_w[row] = aw[tid];
   }
   __syncthreads();
   // row copies: dispatch i's row into the grouped rows (one warp per dispatch)
@@ -314,7 +316,7 @@ int launch_route_dispatch(const moe_shape& s, const void* u, int32_t dtype, cons
                           const float* bias, int32_t* top_idx, float* top_w, float* probs,
                           float* logits, int32_t* counts, int32_t* offsets, int32_t* perm_tok,
                           int32_t* row_of, int32_t* overflow, int32_t* totals, void* x_rows,
-                          void* ws, cudaStream_t st) {
+                          void* ws, cudaStream_t st, float* row_w) {
   static std::atomic<bool> configured[kMaxDevices];
   int dev = 0, sms = 0;
   if (cudaGetDevice(&dev) != cudaSuccess ||
@@ -350,6 +352,7 @@ int launch_route_dispatch(const moe_shape& s, const void* u, int32_t dtype, cons
   p.C = s.capacity;
   p.top_idx = top_idx;
   p.top_w = top_w;
+  p.row_w = row_w;
   p.probs = probs;
   p.logits = logits;
   p.counts = counts;

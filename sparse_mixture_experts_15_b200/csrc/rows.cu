@@ -89,6 +89,39 @@ __global__ void __launch_bounds__(256)
   }
 }
 
+// One warp per token; rows already carry their weights (bf16 a * F(u)), the
+// kept slots are added in ascending s in fp32 and rounded once.
+template <typename TY>
+__global__ void __launch_bounds__(256)
+    combine_weighted(const uint4* __restrict__ rows, int width8,
+                     const int32_t* __restrict__ row_of, int T, int k, TY* __restrict__ y,
+                     int* status) {
+  pdl_wait();
+  pdl_allow_next();
+  const int lane = threadIdx.x & 31;
+  for (int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; t < T;
+       t += (gridDim.x * blockDim.x) >> 5) {
+    for (int c = lane; c < width8; c += 32) {
+      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      for (int s = 0; s < k; ++s) {
+        const int r = row_of[(size_t)t * k + s];
+        if (r < 0) continue;
+        if (r >= T * k) {  // rows holds T*k rows
+          record_error(status, MOE_ERR_BOUNDS);
+          continue;
+        }
+        float v[8];
+        load8(reinterpret_cast<const __nv_bfloat16*>(rows + (size_t)r * width8 + c), v);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] += v[i];
+      }
+      TY* o = y + ((size_t)t * width8 + c) * 8;
+      store4<TY>(o, make_float4(acc[0], acc[1], acc[2], acc[3]));
+      store4<TY>(o + 4, make_float4(acc[4], acc[5], acc[6], acc[7]));
+    }
+  }
+}
+
 int grid_cap(int64_t warps) {
   int64_t b = (warps + 7) / 8;
   if (b > 148 * 16) b = 148 * 16;
@@ -125,6 +158,28 @@ int launch_combine(const moe_shape& s, int32_t width, const float* y_rows, const
   } else {
     MOE_PREFER_SHARED((combine_rows<__half>));
     launch_pdl(combine_rows<__half>, dim3(grid), dim3(256), 0, st, yr, w4, row_of, top_w, s.T, s.k,
+               static_cast<__half*>(y), status_word());
+  }
+  return launch_status();
+}
+
+int launch_combine_weighted(const moe_shape& s, int32_t width, const __nv_bfloat16* rows,
+                            const int32_t* row_of, void* y, int32_t y_dtype, cudaStream_t st) {
+  if (s.T == 0) return MOE_OK;
+  const int w8 = width / 8;
+  const int grid = grid_cap(s.T);
+  const uint4* r = reinterpret_cast<const uint4*>(rows);
+  if (y_dtype == MOE_F32) {
+    MOE_PREFER_SHARED((combine_weighted<float>));
+    launch_pdl(combine_weighted<float>, dim3(grid), dim3(256), 0, st, r, w8, row_of, s.T, s.k,
+               static_cast<float*>(y), status_word());
+  } else if (y_dtype == MOE_BF16) {
+    MOE_PREFER_SHARED((combine_weighted<__nv_bfloat16>));
+    launch_pdl(combine_weighted<__nv_bfloat16>, dim3(grid), dim3(256), 0, st, r, w8, row_of,
+               s.T, s.k, static_cast<__nv_bfloat16*>(y), status_word());
+  } else {
+    MOE_PREFER_SHARED((combine_weighted<__half>));
+    launch_pdl(combine_weighted<__half>, dim3(grid), dim3(256), 0, st, r, w8, row_of, s.T, s.k,
                static_cast<__half*>(y), status_word());
   }
   return launch_status();

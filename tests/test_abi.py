@@ -229,3 +229,30 @@ def test_wait_check_rejects_bad_arguments_on_the_host():
     assert lib.moe_wait_check(-1, 1_000_000, None) == -1
     assert lib.moe_wait_check(0, 999, None) == -1
     assert lib.moe_wait_check(1, 2_000_000_001, None) == -1
+
+
+def test_new_entry_points_reject_bad_arguments_on_the_host():
+    """The FP8, expert-parallel and backward entry points refuse NULL or
+    ill-sized arguments before touching the device."""
+    lib = moe._lib
+    s = moe.shape(64, 256, 8, 2, 256)
+    # E4M3 quantiser: columns must be a multiple of 16, pointers non-NULL
+    assert lib.moe_quantize_e4m3_rows(4, 24, None, moe.BF16, None, None, None) == -1
+    assert lib.moe_quantize_e4m3_rows(4, 32, None, moe.BF16, None, None, None) == -1
+    assert lib.moe_quantize_e4m3_rows(4, 32, None, 7, None, None, None) == -2
+    assert lib.moe_quantize_e4m3_rows(0, 32, None, moe.BF16, None, None, None) == 0
+    # FP8 LatentMoE layer: NULL scales
+    assert lib.moe_latent_fwd_e4m3(ctypes.byref(s), None, None, None, None, None, None, None, 0,
+                                   None) == -1
+    # expert parallelism: NULL buffers
+    assert lib.moe_ep_dispatch(ctypes.byref(s), None, 1, *([None] * 7), None, 0, None) == -1
+    assert lib.moe_ep_combine(ctypes.byref(s), None, 1, *([None] * 6), None) == -1
+    es = moe.shape(128, 256, 4, 1, 256)
+    assert lib.moe_ep_expert_ffn(ctypes.byref(es), None, 1, None, None, None, None, None, None, 0,
+                                 None) == -1
+    assert lib.moe_ep_workspace_bytes(ctypes.byref(es)) >= 256
+    # layer backward: widths must be multiples of 128; NULL pointers
+    assert lib.moe_layer_bwd_workspace_bytes(ctypes.byref(moe.shape(64, 200, 8, 2, 256))) == 0
+    assert lib.moe_layer_bwd_workspace_bytes(ctypes.byref(s)) > 0
+    assert lib.moe_layer_bwd(ctypes.byref(s), None, None, None, None, 0.0, None, None, None, 0,
+                             None) == -1
