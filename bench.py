@@ -285,8 +285,17 @@ class Step:
                                outputs=self.outs, ws=self.lws)
 
     def ffn(self, r: Replica):
-        self.moe.moe_expert_ffn(self.s, self.wl.d, self.x_rows, self.offsets, *r.w, self.y_rows,
+        """The expert FFN alone on replica r's own grouped rows (filled by
+        split(r)), so consecutive replays read rows and weights that are not
+        L2-resident."""
+        self.moe.moe_expert_ffn(self.s, self.wl.d, r.x_rows, r.offsets, *r.w, self.y_rows,
                                 self.act, ws=self.ws_ffn)
+
+    def split(self, r: Replica):
+        """The step split at the expert FFN; keeps r's grouped rows and offsets."""
+        self(r)
+        r.x_rows = self.x_rows.clone()
+        r.offsets = self.offsets.clone()
 
     def __call__(self, r: Replica):
         m = self.moe
@@ -917,7 +926,8 @@ def main():
 
     for i in range(args.warmup):
         step.layer(reps[i % n_rep])
-    step(reps[0])  # the step split at the expert FFN: fills x_rows / offsets for the GEMM replay
+    for r in reps:  # each replica's grouped rows and offsets for the GEMM-only replays
+        step.split(r)
     torch.cuda.synchronize()
     kept = [0] * n_rep
     for i in range(n_rep):

@@ -96,6 +96,12 @@ __device__ __forceinline__ void cp4(void* smem, const void* gmem) {
 __device__ __forceinline__ void cp_wait_all() {
   asm volatile("cp.async.wait_all;" ::: "memory");
 }
+// Bulk prefetch into L2; skipped unless the address is 16-byte aligned and
+// the size a multiple of 16 (the instruction's requirements).
+__device__ __forceinline__ void prefetch_l2(const void* gmem, uint32_t bytes) {
+  if (((reinterpret_cast<uintptr_t>(gmem) | bytes) & 15u) != 0 || bytes == 0) return;
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(gmem), "r"(bytes) : "memory");
+}
 
 // rows x row_bytes (multiple of 16) from gmem (row stride g_stride bytes) to
 // shared rows of s_stride bytes; all threads of the CTA cooperate.
@@ -488,6 +494,29 @@ __global__ void __launch_bounds__(kThreads, 1) decode_persistent(const __grid_co
     __syncthreads();  // list complete before the item loop reads it
     if (b < nitems) stage_item(b);
     if (b < nslices) stage_slice(b);
+    // When the batch dispatches at least as many pairs as there are experts
+    // (nearly every expert selected), the next layer's rows go to L2 now, so
+    // that its staging after routing reads L2 instead of DRAM: CTA b takes
+    // phase-A item (expert b / slicesA, slice b % slicesA) -- the item CTA b
+    // stages when every expert is selected, and every (expert, slice) is some
+    // CTA's -- and the down rows of its phase-B slice for every expert.
+    // Smaller batches keep reading the selected experts only.
+    if (!last && Tk >= N && tid == 0) {
+      const LayerPtrs& Ln = p.layer[l + 1];
+      if (b < N * slicesA) {
+        const size_t row = (size_t)(b / slicesA) * h + (size_t)(b % slicesA) * RA;
+        prefetch_l2(Ln.gq + row * (d / 2), RA * (d / 2));
+        prefetch_l2(Ln.uq + row * (d / 2), RA * (d / 2));
+        prefetch_l2(Ln.gs + row * nb, RA * nb * 2);
+        prefetch_l2(Ln.us + row * nb, RA * nb * 2);
+      }
+      if (b < nslices)
+        for (int e = 0; e < N; ++e) {
+          const size_t row = (size_t)e * d + (size_t)b * RB;
+          prefetch_l2(Ln.dq + row * (h / 2), RB * (h / 2));
+          prefetch_l2(Ln.ds + row * nbh, RB * nbh * 2);
+        }
+    }
 
     // ---- phase A: H[e][t][rows] = SiLU(W_gate u) * (W_up u) for the items
     for (int it = b; it < nitems; it += G) {
