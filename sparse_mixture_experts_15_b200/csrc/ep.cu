@@ -146,6 +146,7 @@ __global__ void __launch_bounds__(256) ep_dispatch(const __grid_constant__ Dispa
 
 struct CombineParams {
   int T, k, N, E, world, w8;  // w8: 16-byte vectors (8 bf16) per row
+  int recv_capacity;          // rows of every output buffer
   const int32_t* top_idx;
   const int32_t* row_of;     // local capacity-0 permutation
   const int32_t* offsets;
@@ -177,7 +178,12 @@ __global__ void __launch_bounds__(256) ep_combine(const __grid_constant__ Combin
         if (r < 0 || e < 0 || e >= p.N) continue;
         const int j = r - p.offsets[e];
         if (j < 0 || j >= p.kept[e]) continue;  // dropped by the capacity
-        const uint4 v4 = p.out_rows[e / p.E][(size_t)(p.send_base[e] + j) * p.w8 + c];
+        const int row = p.send_base[e] + j;
+        if (row < 0 || row >= p.recv_capacity) {  // a plan that does not fit the buffers
+          record_error(p.status, MOE_ERR_BOUNDS);
+          continue;
+        }
+        const uint4 v4 = p.out_rows[e / p.E][(size_t)row * p.w8 + c];
         float v[8];
         load8(reinterpret_cast<const __nv_bfloat16*>(&v4), v);
 #pragma unroll
@@ -320,6 +326,7 @@ extern "C" int moe_ep_combine(const moe_shape* shape, const moe_ep_buffers* bufs
   p.E = s.N / bufs->world;
   p.world = bufs->world;
   p.w8 = s.d / 8;
+  p.recv_capacity = bufs->recv_capacity;
   p.top_idx = top_idx;
   p.row_of = row_of;
   p.offsets = offsets;
