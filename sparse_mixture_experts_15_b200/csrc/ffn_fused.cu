@@ -36,6 +36,7 @@ struct FusedParams {
   CUtensorMap map_x;  // x_rows [R][width],   box 64 x fBN
   CUtensorMap map_d;  // W_down [G*width][h], box 64 x 128
   const int32_t* offsets;
+  int R;  // rows of x_rows and y_rows
   int G, width, h;
   float beta_g, beta_u;
   void* y_rows;         // [R][width] fp32, or bf16 weighted rows when row_w is set
@@ -126,7 +127,7 @@ __global__ void __launch_bounds__(fThreads, 1) tc_fused_ffn(const __grid_constan
       if (g < p.G) {
         beg = p.offsets[g];
         cnt = p.offsets[g + 1] - beg;
-        if (cnt < 0 || beg < 0) {
+        if (cnt < 0 || beg < 0 || beg > p.R || cnt > p.R - beg) {  // rows outside the buffers
           record_error(p.status, MOE_ERR_BOUNDS);
           cnt = 0;
         }
@@ -424,6 +425,7 @@ int launch_ffn_fused(int G, int64_t R, int width, int h, const __nv_bfloat16* x_
       !make_map(&p.map_d, w_down, (uint64_t)G * width, h, fBM))
     return MOE_ERR_CUDA;
   p.offsets = offsets;
+  p.R = (int)R;
   p.G = G;
   p.width = width;
   p.h = h;

@@ -34,6 +34,7 @@ constexpr long long wWaitBudget = 4000000000LL;
 struct BwdParams {
   CUtensorMap maps[4];
   const int32_t* offsets;  // [G+1] padded row ranges (multiples of 64)
+  int rows;                // rows of the token-row operands and outputs
   int G;
   int nseg;
   int seg_end[2];          // cumulative k-blocks (dgrad)
@@ -149,9 +150,9 @@ __global__ void __launch_bounds__(wThreads, 1) tc_bwd_gemm(const __grid_constant
       if (g < p.G) {
         beg = p.offsets[g];
         cnt = p.offsets[g + 1] - beg;
-        if (cnt < 0 || beg < 0 || (cnt & 63) != 0) {
+        if (cnt < 0 || beg < 0 || (cnt & 63) != 0 || beg > p.rows || cnt > p.rows - beg) {
           record_error(p.status, MOE_ERR_BOUNDS);
-          cnt = cnt < 0 ? 0 : cnt & ~63;
+          cnt = (cnt < 0 || beg < 0 || beg > p.rows || cnt > p.rows - beg) ? 0 : cnt & ~63;
         }
       }
       int t = 0;
@@ -469,6 +470,7 @@ int bwd_dgrad_act(const int32_t* offsets, int G, int64_t rows, int width, int h,
     return MOE_ERR_CUDA;
   p.maps[2] = p.maps[3] = p.maps[0];
   p.offsets = offsets;
+  p.rows = (int)rows;
   p.G = G;
   p.nseg = 1;
   p.seg_end[0] = width / wBK;
@@ -505,6 +507,7 @@ int bwd_dgrad_x(const int32_t* offsets, int G, int64_t rows, int width, int h,
       !make_bmap(&p.maps[2], dG, rows, h, wBN) || !make_bmap(&p.maps[3], dV, rows, h, wBN))
     return MOE_ERR_CUDA;
   p.offsets = offsets;
+  p.rows = (int)rows;
   p.G = G;
   p.nseg = 2;
   p.seg_end[0] = h / wBK;
@@ -533,6 +536,7 @@ int bwd_wgrad(const int32_t* offsets, int G, int64_t rows, const __nv_bfloat16* 
     return MOE_ERR_CUDA;
   p.maps[2] = p.maps[3] = p.maps[0];
   p.offsets = offsets;
+  p.rows = (int)rows;
   p.G = G;
   p.nseg = 1;
   p.m_tiles = M / wBM;

@@ -56,7 +56,7 @@ constexpr int kMaxSeg = 3;
 struct TcParams {
   CUtensorMap maps[4];
   const int32_t* offsets;  // [G+1] token row ranges; nullptr: every group uses rows [0, T)
-  int T;
+  int T;                   // with offsets: rows of B and of the output
   int G;
   int nseg;
   int seg_end[kMaxSeg];   // cumulative 64-wide k-blocks at the end of each segment
@@ -179,7 +179,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_grouped_gemm(const __grid_cons
         if (p.offsets) {
           beg = p.offsets[g];
           cnt = p.offsets[g + 1] - beg;
-          if (cnt < 0 || beg < 0) {
+          if (cnt < 0 || beg < 0 || beg > p.T || cnt > p.T - beg) {  // rows outside the buffers
             record_error(p.status, MOE_ERR_BOUNDS);
             cnt = 0;
           }
