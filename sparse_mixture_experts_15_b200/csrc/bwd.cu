@@ -25,20 +25,9 @@
 // bit run to run.
 #include <algorithm>
 
-#include "common.cuh"
+#include "bwd.cuh"
 
 namespace moe {
-
-int bwd_dgrad_act(const int32_t* offsets, int G, int64_t rows, int width, int h,
-                  const __nv_bfloat16* dy_rows, const __nv_bfloat16* w_down,
-                  const __nv_bfloat16* g_pre, const __nv_bfloat16* v_pre, const float* row_w,
-                  const moe_act& act, __nv_bfloat16* dG, __nv_bfloat16* dV, float* da_part,
-                  cudaStream_t st);
-int bwd_dgrad_x(const int32_t* offsets, int G, int64_t rows, int width, int h,
-                const __nv_bfloat16* dG, const __nv_bfloat16* dV, const __nv_bfloat16* w_gate,
-                const __nv_bfloat16* w_up, float* dX, cudaStream_t st);
-int bwd_wgrad(const int32_t* offsets, int G, int64_t rows, const __nv_bfloat16* A, int M,
-              const __nv_bfloat16* B, int Ncols, float* dW, cudaStream_t st);
 
 namespace {
 
@@ -250,10 +239,11 @@ struct DuParams {
   const int32_t* row_of;
   const int32_t* offsets;
   const int32_t* pad;
-  const float* dX;        // [rows][d]
+  const float* dX;        // [rows][d], nullable: no expert rows
   const float* dz;        // [T][N]
-  const float* w_route;   // [N][d]
+  const float* w_route;   // [N][d], nullable: no router term
   float* du;              // [T][d]
+  int add;                // accumulate into du instead of overwriting it
 };
 
 // One warp per token: the kept slots' dX rows in slot order, then the router
@@ -266,8 +256,9 @@ __global__ void __launch_bounds__(256) bwd_du(const __grid_constant__ DuParams p
        t += (gridDim.x * blockDim.x) >> 5) {
     const size_t x0 = (size_t)t * p.k;
     for (int c = lane * 4; c < p.d; c += 128) {
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int s = 0; s < p.k; ++s) {
+      float4 acc = p.add ? *reinterpret_cast<const float4*>(p.du + (size_t)t * p.d + c)
+                         : make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int s = 0; p.dX && s < p.k; ++s) {
         const int r = padded_row(p.row_of, p.top_idx, p.offsets, p.pad, p.N, x0 + s);
         if (r < 0) continue;
         const float4 v = *reinterpret_cast<const float4*>(p.dX + (size_t)r * p.d + c);
@@ -276,7 +267,7 @@ __global__ void __launch_bounds__(256) bwd_du(const __grid_constant__ DuParams p
         acc.z += v.z;
         acc.w += v.w;
       }
-      for (int j = 0; j < p.N; ++j) {
+      for (int j = 0; p.w_route && j < p.N; ++j) {
         const float z = p.dz[(size_t)t * p.N + j];
         const float4 w = *reinterpret_cast<const float4*>(p.w_route + (size_t)j * p.d + c);
         acc.x = fmaf(z, w.x, acc.x);
@@ -305,41 +296,6 @@ __global__ void __launch_bounds__(256)
   dw[i] = acc;
 }
 
-struct BwdBufs {
-  int32_t* pad;
-  __nv_bfloat16 *x, *dyr, *dyw, *g, *v, *H, *dG, *dV;
-  float *a, *da_part, *dX;
-  int64_t rows;
-  size_t bytes;
-};
-
-int64_t padded_rows(const moe_shape& s) { return (int64_t)s.T * s.k + 64LL * s.N; }
-
-BwdBufs carve_bwd(const moe_shape& s, void* base) {
-  Carver c(base);
-  BwdBufs b;
-  const int64_t R = padded_rows(s);
-  b.rows = R;
-  b.pad = c.take<int32_t>(s.N + 1);
-  b.x = c.take<__nv_bfloat16>((size_t)R * s.d);
-  b.dyr = c.take<__nv_bfloat16>((size_t)R * s.d);
-  b.dyw = c.take<__nv_bfloat16>((size_t)R * s.d);
-  b.g = c.take<__nv_bfloat16>((size_t)R * s.h);
-  b.v = c.take<__nv_bfloat16>((size_t)R * s.h);
-  b.H = c.take<__nv_bfloat16>((size_t)R * s.h);
-  b.dG = c.take<__nv_bfloat16>((size_t)R * s.h);
-  b.dV = c.take<__nv_bfloat16>((size_t)R * s.h);
-  b.a = c.take<float>(R);
-  b.da_part = c.take<float>((size_t)R * (s.h / 128 > 0 ? s.h / 128 : 1));
-  b.dX = c.take<float>((size_t)R * s.d);
-  b.bytes = c.used();
-  return b;
-}
-
-bool bwd_shape_ok(const moe_shape* s) {
-  return shape_ok(s) && s->h > 0 && s->h % 128 == 0 && s->d % 128 == 0;
-}
-
 int grid_warps(int64_t warps) {
   int64_t b = (warps + 7) / 8;
   if (b > 148 * 16) b = 148 * 16;
@@ -347,62 +303,55 @@ int grid_warps(int64_t warps) {
 }
 
 }  // namespace
-}  // namespace moe
 
-extern "C" size_t moe_layer_bwd_workspace_bytes(const moe_shape* shape) {
-  if (!moe::bwd_shape_ok(shape)) return 0;
-  return moe::carve_bwd(*shape, nullptr).bytes;
+// ------------------------------------------------- pieces shared by layers
+int64_t bwd_padded_rows(const moe_shape& s) { return (int64_t)s.T * s.k + 64LL * s.N; }
+
+BwdBufs carve_bwd(const moe_shape& s, int width, void* base) {
+  Carver c(base);
+  BwdBufs b;
+  const int64_t R = bwd_padded_rows(s);
+  b.rows = R;
+  b.pad = c.take<int32_t>(s.N + 1);
+  b.x = c.take<__nv_bfloat16>((size_t)R * width);
+  b.dyr = c.take<__nv_bfloat16>((size_t)R * width);
+  b.dyw = c.take<__nv_bfloat16>((size_t)R * width);
+  b.g = c.take<__nv_bfloat16>((size_t)R * s.h);
+  b.v = c.take<__nv_bfloat16>((size_t)R * s.h);
+  b.H = c.take<__nv_bfloat16>((size_t)R * s.h);
+  b.dG = c.take<__nv_bfloat16>((size_t)R * s.h);
+  b.dV = c.take<__nv_bfloat16>((size_t)R * s.h);
+  b.a = c.take<float>(R);
+  b.da_part = c.take<float>((size_t)R * (s.h / 128 > 0 ? s.h / 128 : 1));
+  b.dX = c.take<float>((size_t)R * width);
+  b.bytes = c.used();
+  return b;
 }
 
-extern "C" int moe_layer_bwd(const moe_shape* shape, const moe_layer_weights* w, const void* u,
-                             const void* dy, const moe_layer_outputs* fwd, float alpha,
-                             const float* f, const moe_layer_grads* grads, void* ws,
-                             size_t ws_bytes, void* stream) {
-  using namespace moe;
-  if (!bwd_shape_ok(shape) || !w || !fwd || !grads) return MOE_ERR_INVALID_ARG;
-  const moe_shape& s = *shape;
-  if (w->w_dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
-  if (w->act.kind != MOE_ACT_SWIGLU &&
-      !(w->act.kind == MOE_ACT_SITU_GLU && w->act.beta_gate > 0.0f && w->act.beta_up > 0.0f))
-    return MOE_ERR_INVALID_ARG;
-  if (!w->w_route || !w->w_gate || !w->w_up || !w->w_down) return MOE_ERR_INVALID_ARG;
-  if (!fwd->top_idx || !fwd->top_w || !fwd->probs || !fwd->row_of || !fwd->offsets ||
-      !fwd->perm_tok)
-    return MOE_ERR_INVALID_ARG;
-  if (!grads->du || !grads->dz || !grads->dw_gate || !grads->dw_up || !grads->dw_down)
-    return MOE_ERR_INVALID_ARG;
-  if (s.T > 0 && (!u || !dy)) return MOE_ERR_INVALID_ARG;
-  const void* al[] = {u, dy, w->w_route, w->w_gate, w->w_up, w->w_down, grads->du,
-                      grads->dw_gate, grads->dw_up, grads->dw_down, grads->dw_route};
-  for (const void* q : al)
-    if (!aligned16(q)) return MOE_ERR_INVALID_ARG;
-  BwdBufs b = carve_bwd(s, ws);
-  if (!ws || ws_bytes < b.bytes) return MOE_ERR_WORKSPACE;
-  cudaStream_t st = as_stream(stream);
-  const auto* U = static_cast<const __nv_bfloat16*>(u);
-  const auto* Wg = static_cast<const __nv_bfloat16*>(w->w_gate);
-  const auto* Wu = static_cast<const __nv_bfloat16*>(w->w_up);
-  const auto* Wd = static_cast<const __nv_bfloat16*>(w->w_down);
-  const int N = s.N, d = s.d, h = s.h;
+int experts_backward(const moe_shape& s, int width, const __nv_bfloat16* u,
+                     const __nv_bfloat16* dy, const __nv_bfloat16* Wg, const __nv_bfloat16* Wu,
+                     const __nv_bfloat16* Wd, const moe_act& act, const moe_layer_outputs& fwd,
+                     const BwdBufs& b, float* dw_gate, float* dw_up, float* dw_down,
+                     cudaStream_t st) {
+  const int N = s.N, h = s.h;
   const int64_t R = b.rows;
-
   MOE_PREFER_SHARED((pad_offsets));
-  launch_pdl(pad_offsets, dim3(1), dim3(32), 0, st, fwd->offsets, N, b.pad);
+  launch_pdl(pad_offsets, dim3(1), dim3(32), 0, st, fwd.offsets, N, b.pad);
   int rc = launch_status();
   if (rc != MOE_OK) return rc;
   {
     GatherParams p{};
-    p.u = static_cast<const uint4*>(u);
-    p.dy = static_cast<const uint4*>(dy);
-    p.vec = d / 8;
+    p.u = reinterpret_cast<const uint4*>(u);
+    p.dy = reinterpret_cast<const uint4*>(dy);
+    p.vec = width / 8;
     p.T = s.T;
     p.k = s.k;
     p.N = N;
-    p.offsets = fwd->offsets;
+    p.offsets = fwd.offsets;
     p.pad = b.pad;
-    p.perm_tok = fwd->perm_tok;
-    p.row_of = fwd->row_of;
-    p.top_w = fwd->top_w;
+    p.perm_tok = fwd.perm_tok;
+    p.row_of = fwd.row_of;
+    p.top_w = fwd.top_w;
     p.max_rows = (int)R;
     p.x = reinterpret_cast<uint4*>(b.x);
     p.dyr = reinterpret_cast<uint4*>(b.dyr);
@@ -415,82 +364,143 @@ extern "C" int moe_layer_bwd(const moe_shape* shape, const moe_layer_weights* w,
   }
   // the forward's pre-activations on the padded rows: G = X Wg^T, V = X Wu^T
   {
-    TcSeg sg{Wg, (int64_t)N * h, d, 0, b.x, R, d, 0};
+    TcSeg sg{Wg, (int64_t)N * h, width, 0, b.x, R, width, 0};
     rc = tc_store(b.pad, (int)R, N, h, &sg, 1, b.g, MODE_STORE_BF16, h, st);
     if (rc != MOE_OK) return rc;
-    TcSeg su{Wu, (int64_t)N * h, d, 0, b.x, R, d, 0};
+    TcSeg su{Wu, (int64_t)N * h, width, 0, b.x, R, width, 0};
     rc = tc_store(b.pad, (int)R, N, h, &su, 1, b.v, MODE_STORE_BF16, h, st);
     if (rc != MOE_OK) return rc;
   }
   {
     const int64_t n8 = R * h / 8;
     const int blocks = (int)std::min<int64_t>((n8 + 255) / 256, 148 * 8);
-    if (w->act.kind == MOE_ACT_SITU_GLU) {
+    if (act.kind == MOE_ACT_SITU_GLU) {
       MOE_PREFER_SHARED((bwd_hidden<MOE_ACT_SITU_GLU>));
       launch_pdl(bwd_hidden<MOE_ACT_SITU_GLU>, dim3(blocks), dim3(256), 0, st, b.g, b.v, n8,
-                 w->act.beta_gate, w->act.beta_up, b.H);
+                 act.beta_gate, act.beta_up, b.H);
     } else {
       MOE_PREFER_SHARED((bwd_hidden<MOE_ACT_SWIGLU>));
-      launch_pdl(bwd_hidden<MOE_ACT_SWIGLU>, dim3(blocks), dim3(256), 0, st, b.g, b.v, n8,
-                 0.0f, 0.0f, b.H);
+      launch_pdl(bwd_hidden<MOE_ACT_SWIGLU>, dim3(blocks), dim3(256), 0, st, b.g, b.v, n8, 0.0f,
+                 0.0f, b.H);
     }
     if ((rc = launch_status()) != MOE_OK) return rc;
   }
-  rc = bwd_dgrad_act(b.pad, N, R, d, h, b.dyr, Wd, b.g, b.v, b.a, w->act, b.dG, b.dV, b.da_part,
+  rc = bwd_dgrad_act(b.pad, N, R, width, h, b.dyr, Wd, b.g, b.v, b.a, act, b.dG, b.dV, b.da_part,
                      st);
   if (rc != MOE_OK) return rc;
-  rc = bwd_dgrad_x(b.pad, N, R, d, h, b.dG, b.dV, Wg, Wu, b.dX, st);
+  rc = bwd_dgrad_x(b.pad, N, R, width, h, b.dG, b.dV, Wg, Wu, b.dX, st);
   if (rc != MOE_OK) return rc;
-  rc = bwd_wgrad(b.pad, N, R, b.dG, h, b.x, d, grads->dw_gate, st);
-  if (rc == MOE_OK) rc = bwd_wgrad(b.pad, N, R, b.dV, h, b.x, d, grads->dw_up, st);
-  if (rc == MOE_OK) rc = bwd_wgrad(b.pad, N, R, b.dyw, d, b.H, h, grads->dw_down, st);
-  if (rc != MOE_OK) return rc;
+  rc = bwd_wgrad(b.pad, N, R, b.dG, h, b.x, width, dw_gate, st);
+  if (rc == MOE_OK) rc = bwd_wgrad(b.pad, N, R, b.dV, h, b.x, width, dw_up, st);
+  if (rc == MOE_OK) rc = bwd_wgrad(b.pad, N, R, b.dyw, width, b.H, h, dw_down, st);
+  return rc;
+}
+
+int bwd_router_dz(const moe_shape& s, const moe_layer_outputs& fwd, const BwdBufs& b, float alpha,
+                  const float* f, float* dz, cudaStream_t st) {
   if (s.T == 0) return MOE_OK;
-  {
-    DzParams p{};
-    p.T = s.T;
-    p.N = N;
-    p.k = s.k;
-    p.renorm = s.renorm;
-    p.m_tiles = h / 128;
-    p.top_idx = fwd->top_idx;
-    p.top_w = fwd->top_w;
-    p.probs = fwd->probs;
-    p.row_of = fwd->row_of;
-    p.offsets = fwd->offsets;
-    p.pad = b.pad;
-    p.da_part = b.da_part;
-    p.f = f;
-    p.alpha = alpha;
-    p.dz = grads->dz;
-    MOE_PREFER_SHARED((bwd_dz));
-    launch_pdl(bwd_dz, dim3((s.T + 7) / 8), dim3(256), 0, st, p);
-    if ((rc = launch_status()) != MOE_OK) return rc;
-  }
-  {
-    DuParams p{};
-    p.T = s.T;
-    p.N = N;
-    p.k = s.k;
-    p.d = d;
-    p.top_idx = fwd->top_idx;
-    p.row_of = fwd->row_of;
-    p.offsets = fwd->offsets;
-    p.pad = b.pad;
-    p.dX = b.dX;
-    p.dz = grads->dz;
-    p.w_route = w->w_route;
-    p.du = grads->du;
-    MOE_PREFER_SHARED((bwd_du));
-    launch_pdl(bwd_du, dim3(grid_warps(s.T)), dim3(256), 0, st, p);
-    if ((rc = launch_status()) != MOE_OK) return rc;
-  }
-  if (grads->dw_route) {
-    const int64_t n = (int64_t)N * d;
-    MOE_PREFER_SHARED((bwd_dw_route));
-    launch_pdl(bwd_dw_route, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, st, grads->dz, U,
-               s.T, N, d, grads->dw_route);
-    rc = launch_status();
-  }
+  DzParams p{};
+  p.T = s.T;
+  p.N = s.N;
+  p.k = s.k;
+  p.renorm = s.renorm;
+  p.m_tiles = s.h / 128;
+  p.top_idx = fwd.top_idx;
+  p.top_w = fwd.top_w;
+  p.probs = fwd.probs;
+  p.row_of = fwd.row_of;
+  p.offsets = fwd.offsets;
+  p.pad = b.pad;
+  p.da_part = b.da_part;
+  p.f = f;
+  p.alpha = alpha;
+  p.dz = dz;
+  MOE_PREFER_SHARED((bwd_dz));
+  launch_pdl(bwd_dz, dim3((s.T + 7) / 8), dim3(256), 0, st, p);
+  return launch_status();
+}
+
+int bwd_token_sum(const moe_shape& s, int width, const moe_layer_outputs& fwd, const BwdBufs* b,
+                  const float* dz, const float* w_route, float* out, bool add, cudaStream_t st) {
+  if (s.T == 0) return MOE_OK;
+  DuParams p{};
+  p.T = s.T;
+  p.N = s.N;
+  p.k = s.k;
+  p.d = width;
+  p.top_idx = fwd.top_idx;
+  p.row_of = fwd.row_of;
+  p.offsets = fwd.offsets;
+  p.pad = b ? b->pad : nullptr;
+  p.dX = b ? b->dX : nullptr;
+  p.dz = dz;
+  p.w_route = w_route;
+  p.du = out;
+  p.add = add ? 1 : 0;
+  MOE_PREFER_SHARED((bwd_du));
+  launch_pdl(bwd_du, dim3(grid_warps(s.T)), dim3(256), 0, st, p);
+  return launch_status();
+}
+
+int bwd_router_wgrad(const float* dz, const __nv_bfloat16* u, int T, int N, int d, float* dw,
+                     cudaStream_t st) {
+  const int64_t n = (int64_t)N * d;
+  if (n == 0) return MOE_OK;
+  MOE_PREFER_SHARED((bwd_dw_route));
+  launch_pdl(bwd_dw_route, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, st, dz, u, T, N, d,
+             dw);
+  return launch_status();
+}
+
+bool bwd_act_ok(const moe_act& a) {
+  return a.kind == MOE_ACT_SWIGLU ||
+         (a.kind == MOE_ACT_SITU_GLU && a.beta_gate > 0.0f && a.beta_up > 0.0f);
+}
+
+}  // namespace moe
+
+extern "C" size_t moe_layer_bwd_workspace_bytes(const moe_shape* shape) {
+  using namespace moe;
+  if (!shape_ok(shape) || shape->h <= 0 || shape->h % 128 != 0 || shape->d % 128 != 0) return 0;
+  return carve_bwd(*shape, shape->d, nullptr).bytes;
+}
+
+extern "C" int moe_layer_bwd(const moe_shape* shape, const moe_layer_weights* w, const void* u,
+                             const void* dy, const moe_layer_outputs* fwd, float alpha,
+                             const float* f, const moe_layer_grads* grads, void* ws,
+                             size_t ws_bytes, void* stream) {
+  using namespace moe;
+  if (!shape_ok(shape) || shape->h <= 0 || shape->h % 128 != 0 || shape->d % 128 != 0 || !w ||
+      !fwd || !grads)
+    return MOE_ERR_INVALID_ARG;
+  const moe_shape& s = *shape;
+  if (w->w_dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+  if (!bwd_act_ok(w->act)) return MOE_ERR_INVALID_ARG;
+  if (!w->w_route || !w->w_gate || !w->w_up || !w->w_down) return MOE_ERR_INVALID_ARG;
+  if (!fwd->top_idx || !fwd->top_w || !fwd->probs || !fwd->row_of || !fwd->offsets ||
+      !fwd->perm_tok)
+    return MOE_ERR_INVALID_ARG;
+  if (!grads->du || !grads->dz || !grads->dw_gate || !grads->dw_up || !grads->dw_down)
+    return MOE_ERR_INVALID_ARG;
+  if (s.T > 0 && (!u || !dy)) return MOE_ERR_INVALID_ARG;
+  const void* al[] = {u, dy, w->w_route, w->w_gate, w->w_up, w->w_down, grads->du,
+                      grads->dw_gate, grads->dw_up, grads->dw_down, grads->dw_route};
+  for (const void* q : al)
+    if (!aligned16(q)) return MOE_ERR_INVALID_ARG;
+  BwdBufs b = carve_bwd(s, s.d, ws);
+  if (!ws || ws_bytes < b.bytes) return MOE_ERR_WORKSPACE;
+  cudaStream_t st = as_stream(stream);
+  const auto* U = static_cast<const __nv_bfloat16*>(u);
+  int rc = experts_backward(s, s.d, U, static_cast<const __nv_bfloat16*>(dy),
+                            static_cast<const __nv_bfloat16*>(w->w_gate),
+                            static_cast<const __nv_bfloat16*>(w->w_up),
+                            static_cast<const __nv_bfloat16*>(w->w_down), w->act, *fwd, b,
+                            grads->dw_gate, grads->dw_up, grads->dw_down, st);
+  if (rc == MOE_OK) rc = bwd_router_dz(s, *fwd, b, alpha, f, grads->dz, st);
+  // du = the kept slots' expert input gradients + sum_j dz_j W_route[j]
+  if (rc == MOE_OK)
+    rc = bwd_token_sum(s, s.d, *fwd, &b, grads->dz, w->w_route, grads->du, false, st);
+  if (rc == MOE_OK && grads->dw_route)
+    rc = bwd_router_wgrad(grads->dz, U, s.T, s.N, s.d, grads->dw_route, st);
   return rc;
 }

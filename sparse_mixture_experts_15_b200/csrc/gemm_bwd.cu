@@ -526,6 +526,34 @@ int bwd_dgrad_x(const int32_t* offsets, int G, int64_t rows, int width, int h,
   return launch_bwd<MOE_ACT_SWIGLU, false>(p, upper, st);
 }
 
+// out [rows][M] fp32 = B [rows][K] A_g, A [G*K][M] read MN-major: one K-segment
+// of the dgrad GEMM with the plain fp32 epilogue (dense layers use G = 1).
+int bwd_dgrad_plain(const int32_t* offsets, int G, int64_t rows, int K, int M,
+                    const __nv_bfloat16* B, const __nv_bfloat16* A, float* out,
+                    cudaStream_t st) {
+  if (K % wBK != 0 || M % wBM != 0) return MOE_ERR_UNSUPPORTED;
+  BwdParams p{};
+  if (!make_bmap(&p.maps[0], A, (uint64_t)G * K, M, 64) ||
+      !make_bmap(&p.maps[1], B, rows, K, wBN))
+    return MOE_ERR_CUDA;
+  p.maps[2] = p.maps[3] = p.maps[0];
+  p.offsets = offsets;
+  p.rows = (int)rows;
+  p.G = G;
+  p.nseg = 1;
+  p.seg_end[0] = K / wBK;
+  p.amap[0] = 0;
+  p.bmap[0] = 1;
+  p.a_k_per_group = K;
+  p.m_tiles = M / wBM;
+  p.mode = BMODE_DGRAD_F32;
+  p.out = out;
+  p.out_ld = M;
+  p.status = status_word();
+  const int64_t upper = (int64_t)p.m_tiles * ((rows + wBN - 1) / wBN + G);
+  return launch_bwd<MOE_ACT_SWIGLU, false>(p, upper, st);
+}
+
 // dW[g] = A_g^T B_g over group g's rows: A [rows][M] and B [rows][Ncols]
 // read MN-major; dW fp32 [G][M][Ncols].
 int bwd_wgrad(const int32_t* offsets, int G, int64_t rows, const __nv_bfloat16* A, int M,
