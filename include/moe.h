@@ -361,6 +361,42 @@ MOE_API int moe_latent_fwd_e4m3(const moe_shape* shape, const moe_layer_weights*
                                 const void* x, void* y, const moe_layer_outputs* out, void* ws,
                                 size_t ws_bytes, void* stream);
 
+/* Gradients of L = sum_t dy_t . y_t for the LatentMoE layer of
+ * moe_latent_fwd (bf16 routed experts), with the forward's selected sets held
+ * fixed (the reading of the layer backward above): through y = W_upp m^ +
+ * sum_j S_j(x), the RMSNorm m^ = m / sqrt(mean(m^2) + eps), the routed
+ * experts on x_l = W_dp x and the router on x.  All fp32, device,
+ * caller-owned, fully overwritten:
+ *   dx [T][d], dz [T][N], dw_route [N][d] (nullable), dw_gate, dw_up
+ *   [N][h][l], dw_down [N][l][h], dw_dp [l][d], dw_upp [d][l], dsh_gate,
+ *   dsh_up [n_shared][sh][d], dsh_down [n_shared][d][sh] (with shared
+ *   experts). */
+typedef struct {
+  float* dx;
+  float* dz;
+  float* dw_route;
+  float* dw_gate;
+  float* dw_up;
+  float* dw_down;
+  float* dw_dp;
+  float* dw_upp;
+  float* dsh_gate;
+  float* dsh_up;
+  float* dsh_down;
+} moe_latent_grads;
+
+MOE_API size_t moe_latent_bwd_workspace_bytes(const moe_shape* shape,
+                                              const moe_latent_weights* lw);
+/* w, lw, x as for moe_latent_fwd (d, l, h and sh multiples of 128); dy
+ * [T][d] bf16; fwd: that forward's top_idx, top_w, probs, offsets, perm_tok
+ * and row_of.  The GEMMs run on the tensor cores (bf16 operands, fp32
+ * accumulate); every reduction has a fixed order.  Errors as
+ * moe_layer_bwd. */
+MOE_API int moe_latent_bwd(const moe_shape* shape, const moe_layer_weights* w,
+                           const moe_latent_weights* lw, const void* x, const void* dy,
+                           const moe_layer_outputs* fwd, const moe_latent_grads* grads, void* ws,
+                           size_t ws_bytes, void* stream);
+
 /* ---------------------------------------------------------- q4_0 decode */
 /* Small-batch decode with q4_0 experts (deployment notes "Kestrel-MCU notes
  * 13", §2 lookup loading of the selected experts only, §4 q4_0 experts with an

@@ -60,6 +60,11 @@ class MoeLayerGrads(ctypes.Structure):
     _fields_ = [(n, _vp) for n in ("du", "dz", "dw_route", "dw_gate", "dw_up", "dw_down")]
 
 
+class MoeLatentGrads(ctypes.Structure):
+    _fields_ = [(n, _vp) for n in ("dx", "dz", "dw_route", "dw_gate", "dw_up", "dw_down", "dw_dp",
+                                   "dw_upp", "dsh_gate", "dsh_up", "dsh_down")]
+
+
 class MoeE4M3Scales(ctypes.Structure):
     _fields_ = [(n, _vp) for n in ("gate_scale", "up_scale", "down_scale")]
 
@@ -97,6 +102,11 @@ _PROTOS = {
                               ctypes.POINTER(MoeLatentWeights), _vp, _vp,
                               ctypes.POINTER(MoeLayerOutputs), _vp, _sz, _vp]),
     "moe_quantize_e4m3_rows": (_i32, [_i64, _i32, _vp, _i32, _vp, _vp, _vp]),
+    "moe_latent_bwd_workspace_bytes": (_sz, [_P_SHAPE, ctypes.POINTER(MoeLatentWeights)]),
+    "moe_latent_bwd": (_i32, [_P_SHAPE, ctypes.POINTER(MoeLayerWeights),
+                              ctypes.POINTER(MoeLatentWeights), _vp, _vp,
+                              ctypes.POINTER(MoeLayerOutputs), ctypes.POINTER(MoeLatentGrads), _vp,
+                              _sz, _vp]),
     "moe_latent_fwd_e4m3": (_i32, [_P_SHAPE, ctypes.POINTER(MoeLayerWeights),
                                    ctypes.POINTER(MoeE4M3Scales),
                                    ctypes.POINTER(MoeLatentWeights), _vp, _vp,
@@ -407,6 +417,32 @@ def moe_latent_fwd(s: MoeShape, w_route, w_gate, w_up, w_down, lw: MoeLatentWeig
     _check(_lib.moe_latent_fwd(ctypes.byref(s), ctypes.byref(W), ctypes.byref(lw), _ptr(x),
                                _ptr(y), ctypes.byref(O), _ptr(wbuf), wlen, _stream(stream)),
            "moe_latent_fwd")
+
+
+def moe_latent_bwd(s: MoeShape, w_route, w_gate, w_up, w_down, lw: MoeLatentWeights, x, dy,
+                   fwd: dict, grads: dict, bias=None, a=None, ws=None, stream=None):
+    """LatentMoE backward (include/moe.h): fwd holds the forward's top_idx,
+    top_w, probs, offsets, perm_tok, row_of; grads the fp32 outputs."""
+    a = a or act()
+    l, n, sh = lw.latent, lw.n_shared, lw.shared_hidden
+    sizes = dict(dx=s.T * s.d, dz=s.T * s.N, dw_route=s.N * s.d, dw_gate=s.N * s.h * l,
+                 dw_up=s.N * s.h * l, dw_down=s.N * l * s.h, dw_dp=l * s.d, dw_upp=s.d * l,
+                 dsh_gate=n * sh * s.d, dsh_up=n * sh * s.d, dsh_down=n * s.d * sh)
+    for key, t in grads.items():
+        _need(key, t, sizes[key], _F32)
+    for args in (("x", x, s.T * s.d, _BF16), ("dy", dy, s.T * s.d, _BF16),
+                 ("w_route", w_route, s.N * s.d, _F32), ("bias", bias, s.N, _F32),
+                 ("w_gate", w_gate, s.N * s.h * l, _BF16), ("w_up", w_up, s.N * s.h * l, _BF16),
+                 ("w_down", w_down, s.N * l * s.h, _BF16)):
+        _need(*args)
+    W = MoeLayerWeights(_ptr(w_route), _ptr(bias), _ptr(w_gate), _ptr(w_up), _ptr(w_down), BF16, a)
+    O = _outputs(s, fwd)
+    G = MoeLatentGrads(*(_ptr(grads.get(k)) for k in sizes))
+    wbuf, wlen = _ws(int(_lib.moe_latent_bwd_workspace_bytes(ctypes.byref(s), ctypes.byref(lw))),
+                     x.device, ws)
+    _check(_lib.moe_latent_bwd(ctypes.byref(s), ctypes.byref(W), ctypes.byref(lw), _ptr(x),
+                               _ptr(dy), ctypes.byref(O), ctypes.byref(G), _ptr(wbuf), wlen,
+                               _stream(stream)), "moe_latent_bwd")
 
 
 _CODES = (_U8, "float8_e4m3fn")

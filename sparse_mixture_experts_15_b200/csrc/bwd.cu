@@ -56,8 +56,8 @@ __global__ void pad_offsets(const int32_t* __restrict__ offsets, int N, int32_t*
 }
 
 struct GatherParams {
-  const uint4* u;           // [T][d] bf16
-  const uint4* dy;          // [T][d] bf16
+  const uint4* u;           // [T][d] bf16, nullable: x rows and a not written
+  const uint4* dy;          // [T][d] bf16, nullable: dy rows not written
   int vec, T, k, N;
   const int32_t* offsets;   // [N+1] forward grouped layout
   const int32_t* pad;       // [N+1]
@@ -103,28 +103,33 @@ __global__ void __launch_bounds__(256) bwd_gather(const __grid_constant__ Gather
           if (p.row_of[(size_t)t * p.k + s] == src) a = p.top_w[(size_t)t * p.k + s];
       }
     }
-    uint4* xo = p.x + (size_t)r * p.vec;
-    uint4* d1 = p.dyr + (size_t)r * p.vec;
-    uint4* d2 = p.dyw + (size_t)r * p.vec;
-    for (int v = lane; v < p.vec; v += 32) {
-      if (t < 0) {
-        xo[v] = d1[v] = d2[v] = make_uint4(0, 0, 0, 0);
-        continue;
-      }
-      xo[v] = p.u[(size_t)t * p.vec + v];
-      const uint4 g = p.dy[(size_t)t * p.vec + v];
-      d1[v] = g;
-      float f[8];
-      load8(reinterpret_cast<const __nv_bfloat16*>(&g), f);
-      uint32_t w[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        __nv_bfloat162 b2 = __floats2bfloat162_rn(a * f[2 * i], a * f[2 * i + 1]);
-        w[i] = *reinterpret_cast<uint32_t*>(&b2);
-      }
-      d2[v] = make_uint4(w[0], w[1], w[2], w[3]);
+    if (p.u) {
+      uint4* xo = p.x + (size_t)r * p.vec;
+      for (int v = lane; v < p.vec; v += 32)
+        xo[v] = t < 0 ? make_uint4(0, 0, 0, 0) : p.u[(size_t)t * p.vec + v];
+      if (lane == 0) p.a[r] = a;
     }
-    if (lane == 0) p.a[r] = a;
+    if (p.dy) {
+      uint4* d1 = p.dyr + (size_t)r * p.vec;
+      uint4* d2 = p.dyw + (size_t)r * p.vec;
+      for (int v = lane; v < p.vec; v += 32) {
+        if (t < 0) {
+          d1[v] = d2[v] = make_uint4(0, 0, 0, 0);
+          continue;
+        }
+        const uint4 g = p.dy[(size_t)t * p.vec + v];
+        d1[v] = g;
+        float f[8];
+        load8(reinterpret_cast<const __nv_bfloat16*>(&g), f);
+        uint32_t w[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          __nv_bfloat162 b2 = __floats2bfloat162_rn(a * f[2 * i], a * f[2 * i + 1]);
+          w[i] = *reinterpret_cast<uint32_t*>(&b2);
+        }
+        d2[v] = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+    }
   }
 }
 
@@ -328,63 +333,64 @@ BwdBufs carve_bwd(const moe_shape& s, int width, void* base) {
   return b;
 }
 
-int experts_backward(const moe_shape& s, int width, const __nv_bfloat16* u,
-                     const __nv_bfloat16* dy, const __nv_bfloat16* Wg, const __nv_bfloat16* Wu,
-                     const __nv_bfloat16* Wd, const moe_act& act, const moe_layer_outputs& fwd,
-                     const BwdBufs& b, float* dw_gate, float* dw_up, float* dw_down,
-                     cudaStream_t st) {
+namespace {
+
+int launch_gather(const moe_shape& s, int width, const __nv_bfloat16* u, const __nv_bfloat16* dy,
+                  const moe_layer_outputs& fwd, const BwdBufs& b, cudaStream_t st) {
+  GatherParams p{};
+  p.u = reinterpret_cast<const uint4*>(u);
+  p.dy = reinterpret_cast<const uint4*>(dy);
+  p.vec = width / 8;
+  p.T = s.T;
+  p.k = s.k;
+  p.N = s.N;
+  p.offsets = fwd.offsets;
+  p.pad = b.pad;
+  p.perm_tok = fwd.perm_tok;
+  p.row_of = fwd.row_of;
+  p.top_w = fwd.top_w;
+  p.max_rows = (int)b.rows;
+  p.x = reinterpret_cast<uint4*>(b.x);
+  p.dyr = reinterpret_cast<uint4*>(b.dyr);
+  p.dyw = reinterpret_cast<uint4*>(b.dyw);
+  p.a = b.a;
+  p.status = status_word();
+  MOE_PREFER_SHARED((bwd_gather));
+  launch_pdl(bwd_gather, dim3(grid_warps(b.rows)), dim3(256), 0, st, p);
+  return launch_status();
+}
+
+}  // namespace
+
+int experts_forward_rows(const moe_shape& s, int width, const __nv_bfloat16* u,
+                         const __nv_bfloat16* Wg, const __nv_bfloat16* Wu, const moe_act& act,
+                         const moe_layer_outputs& fwd, const BwdBufs& b, cudaStream_t st) {
   const int N = s.N, h = s.h;
   const int64_t R = b.rows;
   MOE_PREFER_SHARED((pad_offsets));
   launch_pdl(pad_offsets, dim3(1), dim3(32), 0, st, fwd.offsets, N, b.pad);
   int rc = launch_status();
+  if (rc == MOE_OK) rc = launch_gather(s, width, u, nullptr, fwd, b, st);
   if (rc != MOE_OK) return rc;
-  {
-    GatherParams p{};
-    p.u = reinterpret_cast<const uint4*>(u);
-    p.dy = reinterpret_cast<const uint4*>(dy);
-    p.vec = width / 8;
-    p.T = s.T;
-    p.k = s.k;
-    p.N = N;
-    p.offsets = fwd.offsets;
-    p.pad = b.pad;
-    p.perm_tok = fwd.perm_tok;
-    p.row_of = fwd.row_of;
-    p.top_w = fwd.top_w;
-    p.max_rows = (int)R;
-    p.x = reinterpret_cast<uint4*>(b.x);
-    p.dyr = reinterpret_cast<uint4*>(b.dyr);
-    p.dyw = reinterpret_cast<uint4*>(b.dyw);
-    p.a = b.a;
-    p.status = status_word();
-    MOE_PREFER_SHARED((bwd_gather));
-    launch_pdl(bwd_gather, dim3(grid_warps(R)), dim3(256), 0, st, p);
-    if ((rc = launch_status()) != MOE_OK) return rc;
-  }
   // the forward's pre-activations on the padded rows: G = X Wg^T, V = X Wu^T
-  {
-    TcSeg sg{Wg, (int64_t)N * h, width, 0, b.x, R, width, 0};
-    rc = tc_store(b.pad, (int)R, N, h, &sg, 1, b.g, MODE_STORE_BF16, h, st);
-    if (rc != MOE_OK) return rc;
-    TcSeg su{Wu, (int64_t)N * h, width, 0, b.x, R, width, 0};
-    rc = tc_store(b.pad, (int)R, N, h, &su, 1, b.v, MODE_STORE_BF16, h, st);
-    if (rc != MOE_OK) return rc;
-  }
-  {
-    const int64_t n8 = R * h / 8;
-    const int blocks = (int)std::min<int64_t>((n8 + 255) / 256, 148 * 8);
-    if (act.kind == MOE_ACT_SITU_GLU) {
-      MOE_PREFER_SHARED((bwd_hidden<MOE_ACT_SITU_GLU>));
-      launch_pdl(bwd_hidden<MOE_ACT_SITU_GLU>, dim3(blocks), dim3(256), 0, st, b.g, b.v, n8,
-                 act.beta_gate, act.beta_up, b.H);
-    } else {
-      MOE_PREFER_SHARED((bwd_hidden<MOE_ACT_SWIGLU>));
-      launch_pdl(bwd_hidden<MOE_ACT_SWIGLU>, dim3(blocks), dim3(256), 0, st, b.g, b.v, n8, 0.0f,
-                 0.0f, b.H);
-    }
-    if ((rc = launch_status()) != MOE_OK) return rc;
-  }
+  TcSeg sg{Wg, (int64_t)N * h, width, 0, b.x, R, width, 0};
+  rc = tc_store(b.pad, (int)R, N, h, &sg, 1, b.g, MODE_STORE_BF16, h, st);
+  if (rc != MOE_OK) return rc;
+  TcSeg su{Wu, (int64_t)N * h, width, 0, b.x, R, width, 0};
+  rc = tc_store(b.pad, (int)R, N, h, &su, 1, b.v, MODE_STORE_BF16, h, st);
+  if (rc != MOE_OK) return rc;
+  return bwd_hidden_rows(b.g, b.v, R * h, act, b.H, st);
+}
+
+int experts_backward_rows(const moe_shape& s, int width, const __nv_bfloat16* dy,
+                          const __nv_bfloat16* Wg, const __nv_bfloat16* Wu,
+                          const __nv_bfloat16* Wd, const moe_act& act,
+                          const moe_layer_outputs& fwd, const BwdBufs& b, float* dw_gate,
+                          float* dw_up, float* dw_down, cudaStream_t st) {
+  const int N = s.N, h = s.h;
+  const int64_t R = b.rows;
+  int rc = launch_gather(s, width, nullptr, dy, fwd, b, st);
+  if (rc != MOE_OK) return rc;
   rc = bwd_dgrad_act(b.pad, N, R, width, h, b.dyr, Wd, b.g, b.v, b.a, act, b.dG, b.dV, b.da_part,
                      st);
   if (rc != MOE_OK) return rc;
@@ -394,6 +400,33 @@ int experts_backward(const moe_shape& s, int width, const __nv_bfloat16* u,
   if (rc == MOE_OK) rc = bwd_wgrad(b.pad, N, R, b.dV, h, b.x, width, dw_up, st);
   if (rc == MOE_OK) rc = bwd_wgrad(b.pad, N, R, b.dyw, width, b.H, h, dw_down, st);
   return rc;
+}
+
+int experts_backward(const moe_shape& s, int width, const __nv_bfloat16* u,
+                     const __nv_bfloat16* dy, const __nv_bfloat16* Wg, const __nv_bfloat16* Wu,
+                     const __nv_bfloat16* Wd, const moe_act& act, const moe_layer_outputs& fwd,
+                     const BwdBufs& b, float* dw_gate, float* dw_up, float* dw_down,
+                     cudaStream_t st) {
+  int rc = experts_forward_rows(s, width, u, Wg, Wu, act, fwd, b, st);
+  if (rc != MOE_OK) return rc;
+  return experts_backward_rows(s, width, dy, Wg, Wu, Wd, act, fwd, b, dw_gate, dw_up, dw_down, st);
+}
+
+int bwd_hidden_rows(const __nv_bfloat16* g, const __nv_bfloat16* v, int64_t n,
+                    const moe_act& act, __nv_bfloat16* H, cudaStream_t st) {
+  const int64_t n8 = n / 8;
+  if (n8 == 0) return MOE_OK;
+  const int blocks = (int)std::min<int64_t>((n8 + 255) / 256, 148 * 8);
+  if (act.kind == MOE_ACT_SITU_GLU) {
+    MOE_PREFER_SHARED((bwd_hidden<MOE_ACT_SITU_GLU>));
+    launch_pdl(bwd_hidden<MOE_ACT_SITU_GLU>, dim3(blocks), dim3(256), 0, st, g, v, n8,
+               act.beta_gate, act.beta_up, H);
+  } else {
+    MOE_PREFER_SHARED((bwd_hidden<MOE_ACT_SWIGLU>));
+    launch_pdl(bwd_hidden<MOE_ACT_SWIGLU>, dim3(blocks), dim3(256), 0, st, g, v, n8, 0.0f, 0.0f,
+               H);
+  }
+  return launch_status();
 }
 
 int bwd_router_dz(const moe_shape& s, const moe_layer_outputs& fwd, const BwdBufs& b, float alpha,

@@ -20,6 +20,19 @@ struct BwdBufs {
 
 BwdBufs carve_bwd(const moe_shape& s, int width, void* base);
 
+// The two halves of experts_backward: the forward rows (padded offsets, the
+// gathered inputs b.x and weights b.a, the pre-activations b.g, b.v and
+// b.H), then the backward rows (the gathered dy, dG, dV, da partials, b.dX
+// and the weight gradients).
+int experts_forward_rows(const moe_shape& s, int width, const __nv_bfloat16* u,
+                         const __nv_bfloat16* Wg, const __nv_bfloat16* Wu, const moe_act& act,
+                         const moe_layer_outputs& fwd, const BwdBufs& b, cudaStream_t st);
+int experts_backward_rows(const moe_shape& s, int width, const __nv_bfloat16* dy,
+                          const __nv_bfloat16* Wg, const __nv_bfloat16* Wu,
+                          const __nv_bfloat16* Wd, const moe_act& act,
+                          const moe_layer_outputs& fwd, const BwdBufs& b, float* dw_gate,
+                          float* dw_up, float* dw_down, cudaStream_t st);
+
 // The grouped experts' backward for inputs u [T][width] and upstream dy
 // [T][width] (both bf16), routed as fwd says: recomputes the pre-activations
 // and H on the padded rows, then dG, dV and the da partial sums, the input
@@ -46,6 +59,10 @@ int bwd_router_wgrad(const float* dz, const __nv_bfloat16* u, int T, int N, int 
                      cudaStream_t st);
 
 bool bwd_act_ok(const moe_act& a);
+
+// H = bf16(act(g, v)) over n elements (a multiple of 8), g and v bf16.
+int bwd_hidden_rows(const __nv_bfloat16* g, const __nv_bfloat16* v, int64_t n,
+                    const moe_act& act, __nv_bfloat16* H, cudaStream_t st);
 
 // tcgen05 backward GEMMs (gemm_bwd.cu); rows: padded row count, offsets: the
 // padded group ranges.

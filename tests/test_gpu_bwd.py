@@ -105,3 +105,63 @@ def test_layer_backward_vs_oracle(case):
         assert (kept == 0).any(), "the case should leave an expert without rows"
     if case == "capacity_drops":
         assert perm["totals"][1] > 0
+
+
+def test_latent_backward_vs_oracle():
+    """The LatentMoE layer's backward (RMSNorm, W_dp, W_upp, SiTU-GLU routed
+    experts in the latent width, SwiGLU shared experts, the router on x)
+    against or_latent_backward on every token of a small layer; experts
+    nobody selected get exactly zero gradient."""
+    from inputs import dev_latent, host_latent_dense, host_latent_expert
+    wl = W.Workload("latent_small", T=200, d=256, N=32, k=4, h=128, seed=1005,
+                    act_dtype=S.DT_BF16, w_dtype="bf16", rms_inputs=True, latent=128,
+                    n_shared=2, shared_hidden=128, beta_gate=4.0, beta_up=25.0)
+    T, d, N, k, h, l, n, sh = wl.T, wl.d, wl.N, wl.k, wl.h, wl.latent, wl.n_shared, \
+        wl.shared_hidden
+    dw = dev_latent(wl)
+    s = moe.shape(T, d, N, k, h, 1, 0)
+    lw = moe.latent_weights(l, dw["w_dp"], dw["w_upp"], dw["shared_gate"], dw["shared_up"],
+                            dw["shared_down"], n, sh, 1e-6)
+    x = dev_u(wl)
+    a = moe.act(moe.ACT_SITU_GLU, wl.beta_gate, wl.beta_up)
+    i32 = dict(dtype=torch.int32, device="cuda")
+    fwd = dict(top_idx=torch.empty((T, k), **i32),
+               top_w=torch.empty((T, k), dtype=torch.float32, device="cuda"),
+               probs=torch.empty((T, N), dtype=torch.float32, device="cuda"),
+               offsets=torch.empty(N + 1, **i32), perm_tok=torch.empty(T * k, **i32),
+               row_of=torch.empty((T, k), **i32))
+    y = torch.empty((T, d), dtype=torch.bfloat16, device="cuda")
+    moe.moe_latent_fwd(s, dw["w_route"], dw["w_gate"], dw["w_up"], dw["w_down"], lw, x, y, a=a,
+                       outputs=fwd)
+    dy = dev_normal(wl.seed, TID_DY, (T, d), 1.0, S.DT_BF16)
+    f32 = dict(dtype=torch.float32, device="cuda")
+    grads = dict(dx=torch.empty((T, d), **f32), dz=torch.empty((T, N), **f32),
+                 dw_route=torch.empty((N, d), **f32), dw_gate=torch.empty((N, h, l), **f32),
+                 dw_up=torch.empty((N, h, l), **f32), dw_down=torch.empty((N, l, h), **f32),
+                 dw_dp=torch.empty((l, d), **f32), dw_upp=torch.empty((d, l), **f32),
+                 dsh_gate=torch.empty((n, sh, d), **f32), dsh_up=torch.empty((n, sh, d), **f32),
+                 dsh_down=torch.empty((n, d, sh), **f32))
+    moe.moe_latent_bwd(s, dw["w_route"], dw["w_gate"], dw["w_up"], dw["w_down"], lw, x, dy, fwd,
+                       grads, a=a)
+    torch.cuda.synchronize()
+    got = {key: t.cpu().numpy() for key, t in grads.items()}
+
+    idx = fwd["top_idx"].cpu().numpy()
+    W_dp, W_upp, shared = host_latent_dense(wl)
+    mats = [host_latent_expert(wl, e) for e in range(N)]
+    wr = S.normal(wl.seed, W.TID_WROUTE, (N, d), W.SIGMA_W, S.DT_F32)
+    ref = O.latent_backward(([m[0] for m in mats], [m[1] for m in mats], [m[2] for m in mats]),
+                            wr.astype(np.float64), W_dp, W_upp, shared,
+                            O.decode(O.BF16, host_u(wl)), idx,
+                            O.decode(O.BF16, S.normal(wl.seed, TID_DY, (T, d), 1.0, S.DT_BF16)),
+                            wl.beta_gate, wl.beta_up, 1e-6)
+    pairs = (("dx", "dx"), ("dz", "dz"), ("dw_route", "dWr"), ("dw_gate", "dWg"),
+             ("dw_up", "dWu"), ("dw_down", "dWd"), ("dw_dp", "dWdp"), ("dw_upp", "dWupp"),
+             ("dsh_gate", "dSg"), ("dsh_up", "dSu"), ("dsh_down", "dSd"))
+    errs = {gk: rel_err(got[gk], ref[rk]) for gk, rk in pairs}
+    assert all(np.isfinite(v) for v in errs.values()), errs
+    assert max(errs.values()) < TOL, errs
+    unused = np.setdiff1d(np.arange(N), idx.ravel())
+    for e in unused:
+        for gk in ("dw_gate", "dw_up", "dw_down"):
+            assert not np.any(got[gk][e]), (gk, e)
