@@ -346,6 +346,21 @@ typedef struct {
 MOE_API int moe_quantize_e4m3_rows(int64_t rows, int32_t cols, const void* x, int32_t x_dtype,
                                    uint8_t* codes, float* scales, void* stream);
 
+/* The grouped expert FFN of moe_expert_ffn with E4M3 operands: x_rows
+ * [T*k][width] codes with x_scale [T*k] (one scale per row, e.g. from
+ * moe_quantize_e4m3_rows), the experts' E4M3 codes (gate, up [N][h][width],
+ * down [N][width][h]) with their row scales, SiTU-GLU or SwiGLU; H is stored
+ * as E4M3 codes with no scale in ws; y_rows [T*k][width] fp32, F(u) of each
+ * grouped row (not weighted).  width a multiple of 256, h of 128.
+ * ws: moe_expert_ffn_e4m3_workspace_bytes.  Errors as moe_expert_ffn. */
+MOE_API size_t moe_expert_ffn_e4m3_workspace_bytes(const moe_shape* shape);
+MOE_API int moe_expert_ffn_e4m3(const moe_shape* shape, int32_t width, const uint8_t* x_rows,
+                                const float* x_scale, const int32_t* offsets,
+                                const uint8_t* w_gate, const uint8_t* w_up,
+                                const uint8_t* w_down, const moe_e4m3_scales* scales,
+                                const moe_act* act, float* y_rows, void* ws, size_t ws_bytes,
+                                void* stream);
+
 /* The LatentMoE layer of moe_latent_fwd with E4M3 routed experts: w->w_dtype
  * == MOE_E4M3 and w->w_gate, w_up, w_down hold codes (gate, up [N][h][l],
  * down [N][l][h] bytes) with the row scales in *scales.  x_l = W_dp x (bf16)
@@ -519,7 +534,7 @@ typedef struct {
   int32_t recv_capacity;       /* rows of recv_rows / out_rows on every rank */
   void* recv_rows;             /* this rank: received token rows, bf16 [recv_capacity][d] */
   float* recv_w;               /* this rank: their combine weights [recv_capacity] */
-  void* out_rows;              /* this rank: weighted expert outputs a * F(u), bf16 */
+  void* out_rows;              /* this rank: weighted expert outputs a * F(u), fp32 [recv_capacity][d] */
   uint32_t* arrive;            /* this rank: arrival flags [world], one per source */
   uint32_t* done;              /* this rank: one flag, experts finished */
   void* const* peer_recv_rows; /* [world] every rank's recv_rows */
@@ -541,7 +556,7 @@ typedef struct {
  *   moe_ep_expert_ffn: waits until every source's arrival flag reached epoch,
  *     runs this rank's E experts (moe_expert_ffn's kernels; expert_shape:
  *     T = recv_capacity, k = 1, N = E, d, h) on the received rows grouped by
- *     recv_offsets [E+1] (the plan's), stores bf16 rows a * F(u) into
+ *     recv_offsets [E+1] (the plan's), stores fp32 rows a * F(u) into
  *     out_rows and raises done;
  *   moe_ep_combine: waits until every rank's done flag reached epoch, then
  *     y_t = sum over kept slots (ascending s) of the owners' out_rows rows,

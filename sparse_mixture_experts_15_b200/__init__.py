@@ -102,6 +102,10 @@ _PROTOS = {
                               ctypes.POINTER(MoeLatentWeights), _vp, _vp,
                               ctypes.POINTER(MoeLayerOutputs), _vp, _sz, _vp]),
     "moe_quantize_e4m3_rows": (_i32, [_i64, _i32, _vp, _i32, _vp, _vp, _vp]),
+    "moe_expert_ffn_e4m3_workspace_bytes": (_sz, [_P_SHAPE]),
+    "moe_expert_ffn_e4m3": (_i32, [_P_SHAPE, _i32, _vp, _vp, _vp, _vp, _vp, _vp,
+                                   ctypes.POINTER(MoeE4M3Scales), ctypes.POINTER(MoeAct), _vp,
+                                   _vp, _sz, _vp]),
     "moe_latent_bwd_workspace_bytes": (_sz, [_P_SHAPE, ctypes.POINTER(MoeLatentWeights)]),
     "moe_latent_bwd": (_i32, [_P_SHAPE, ctypes.POINTER(MoeLayerWeights),
                               ctypes.POINTER(MoeLatentWeights), _vp, _vp,
@@ -457,6 +461,29 @@ def moe_quantize_e4m3_rows(x, codes, scales, stream=None):
     _need("scales", scales, rows, _F32)
     _check(_lib.moe_quantize_e4m3_rows(rows, cols, _ptr(x), _dtype_code(x), _ptr(codes),
                                        _ptr(scales), _stream(stream)), "moe_quantize_e4m3_rows")
+
+
+def moe_expert_ffn_e4m3(s: MoeShape, width: int, x_rows, x_scale, offsets, w_gate, w_up,
+                        w_down, gate_scale, up_scale, down_scale, y_rows, a=None, ws=None,
+                        stream=None):
+    """Grouped expert FFN with E4M3 operands (include/moe.h); y_rows fp32."""
+    a = a or act()
+    R = s.T * s.k
+    for args in (("x_rows", x_rows, R * width, _CODES), ("x_scale", x_scale, R, _F32),
+                 ("offsets", offsets, s.N + 1, _I32),
+                 ("w_gate", w_gate, s.N * s.h * width, _CODES),
+                 ("w_up", w_up, s.N * s.h * width, _CODES),
+                 ("w_down", w_down, s.N * width * s.h, _CODES),
+                 ("gate_scale", gate_scale, s.N * s.h, _F32), ("up_scale", up_scale, s.N * s.h, _F32),
+                 ("down_scale", down_scale, s.N * width, _F32), ("y_rows", y_rows, R * width, _F32)):
+        _need(*args)
+    sc = MoeE4M3Scales(_ptr(gate_scale), _ptr(up_scale), _ptr(down_scale))
+    wbuf, wlen = _ws(int(_lib.moe_expert_ffn_e4m3_workspace_bytes(ctypes.byref(s))),
+                     x_rows.device, ws)
+    _check(_lib.moe_expert_ffn_e4m3(ctypes.byref(s), width, _ptr(x_rows), _ptr(x_scale),
+                                    _ptr(offsets), _ptr(w_gate), _ptr(w_up), _ptr(w_down),
+                                    ctypes.byref(sc), ctypes.byref(a), _ptr(y_rows), _ptr(wbuf),
+                                    wlen, _stream(stream)), "moe_expert_ffn_e4m3")
 
 
 def moe_latent_fwd_e4m3(s: MoeShape, w_route, w_gate, w_up, w_down, gate_scale, up_scale,

@@ -255,16 +255,16 @@ int launch_gather(const moe_shape& s, int32_t width, const void* u, int32_t dtyp
                   const int32_t* perm_tok, const int32_t* offsets, void* x_rows, cudaStream_t st);
 int launch_combine(const moe_shape& s, int32_t width, const float* y_rows, const int32_t* row_of,
                    const float* top_w, void* y, int32_t y_dtype, cudaStream_t st);
-// y[t] = sum over kept slots s (ascending) of rows[row_of[t][s]], bf16 rows
+// y[t] = sum over kept slots s (ascending) of rows[row_of[t][s]], fp32 rows
 // already weighted by their combine weights; fp32 sum, one rounding to y_dtype.
-int launch_combine_weighted(const moe_shape& s, int32_t width, const __nv_bfloat16* rows,
+int launch_combine_weighted(const moe_shape& s, int32_t width, const float* rows,
                             const int32_t* row_of, void* y, int32_t y_dtype, cudaStream_t st);
 size_t ffn_simt_ws_bytes(const moe_shape& s);
 int launch_ffn_simt(const moe_shape& s, int32_t width, const float* x_rows, const int32_t* offsets,
                     const float* w_gate, const float* w_up, const float* w_down,
                     const moe_act& act, float* y_rows, void* ws, cudaStream_t st);
 size_t ffn_tc_ws_bytes(const moe_shape& s, int32_t width);
-// y_rows: fp32 expert outputs F(u) per grouped row, or (row_w != nullptr) bf16
+// y_rows: fp32 expert outputs F(u) per grouped row, or (row_w != nullptr) the
 // rows already weighted, row_w[r] * F(u) (the combine then only adds them).
 int launch_ffn_tc(const moe_shape& s, int32_t width, const __nv_bfloat16* x_rows,
                   const int32_t* offsets, const __nv_bfloat16* w_gate, const __nv_bfloat16* w_up,

@@ -5,7 +5,7 @@
 //
 // R ranks, expert e on rank e / (N / R).  Each rank holds, in its own memory,
 // a receive buffer of bf16 rows (with one combine weight per row), an output
-// buffer of bf16 rows, R arrival flags and one done flag; every rank can
+// buffer of fp32 rows, R arrival flags and one done flag; every rank can
 // address every rank's buffers (peer memory over NVLink, or one device).
 // One step, with the exchange plan of moe_ep_plan (rows of one expert from
 // rank 0 first, then rank 1, ..., each in token order, capacity in that
@@ -17,7 +17,7 @@
 //                       owner (release, system scope)
 //   expert FFN (owner)  waits until every source has arrived, runs the
 //                       grouped SwiGLU experts on its receive buffer and
-//                       stores bf16 rows a * F(u) into its output buffer,
+//                       stores fp32 rows a * F(u) into its output buffer,
 //                       then raises its done flag
 //   combine   (source)  waits for every owner's done flag and forms
 //                       y_t = sum over kept slots of the owners' output rows,
@@ -145,14 +145,14 @@ __global__ void __launch_bounds__(256) ep_dispatch(const __grid_constant__ Dispa
 }
 
 struct CombineParams {
-  int T, k, N, E, world, w8;  // w8: 16-byte vectors (8 bf16) per row
+  int T, k, N, E, world, w4;  // w4: float4 vectors per row
   int recv_capacity;          // rows of every output buffer
   const int32_t* top_idx;
   const int32_t* row_of;     // local capacity-0 permutation
   const int32_t* offsets;
   const int32_t* kept;
   const int32_t* send_base;
-  const uint4* const* out_rows;  // [world] owners' weighted output rows
+  const float4* const* out_rows;  // [world] owners' weighted output rows (fp32)
   const unsigned* const* done;   // [world] owners' done flags
   unsigned epoch;
   __nv_bfloat16* y;
@@ -170,8 +170,8 @@ __global__ void __launch_bounds__(256) ep_combine(const __grid_constant__ Combin
   const int lane = threadIdx.x & 31;
   for (int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; t < p.T;
        t += (gridDim.x * blockDim.x) >> 5) {
-    for (int c = lane; c < p.w8; c += 32) {
-      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    for (int c = lane; c < p.w4; c += 32) {
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
       for (int s = 0; s < p.k; ++s) {
         const int r = p.row_of[(size_t)t * p.k + s];
         const int e = p.top_idx[(size_t)t * p.k + s];
@@ -183,20 +183,17 @@ __global__ void __launch_bounds__(256) ep_combine(const __grid_constant__ Combin
           record_error(p.status, MOE_ERR_BOUNDS);
           continue;
         }
-        const uint4 v4 = p.out_rows[e / p.E][(size_t)row * p.w8 + c];
-        float v[8];
-        load8(reinterpret_cast<const __nv_bfloat16*>(&v4), v);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) acc[i] += v[i];
+        const float4 v = p.out_rows[e / p.E][(size_t)row * p.w4 + c];
+        acc.x += v.x;
+        acc.y += v.y;
+        acc.z += v.z;
+        acc.w += v.w;
       }
-      uint4 o;
-      uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        __nv_bfloat162 b2 = __floats2bfloat162_rn(acc[2 * i], acc[2 * i + 1]);
-        ow[i] = *reinterpret_cast<uint32_t*>(&b2);
-      }
-      reinterpret_cast<uint4*>(p.y + (size_t)t * p.w8 * 8)[c] = o;
+      __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y), hi = __floats2bfloat162_rn(acc.z, acc.w);
+      uint2 o;
+      o.x = *reinterpret_cast<uint32_t*>(&lo);
+      o.y = *reinterpret_cast<uint32_t*>(&hi);
+      reinterpret_cast<uint2*>(p.y + (size_t)t * p.w4 * 4)[c] = o;
     }
   }
   pdl_allow_next();
@@ -325,14 +322,14 @@ extern "C" int moe_ep_combine(const moe_shape* shape, const moe_ep_buffers* bufs
   p.N = s.N;
   p.E = s.N / bufs->world;
   p.world = bufs->world;
-  p.w8 = s.d / 8;
+  p.w4 = s.d / 4;
   p.recv_capacity = bufs->recv_capacity;
   p.top_idx = top_idx;
   p.row_of = row_of;
   p.offsets = offsets;
   p.kept = kept;
   p.send_base = send_base;
-  p.out_rows = reinterpret_cast<const uint4* const*>(bufs->peer_out_rows);
+  p.out_rows = reinterpret_cast<const float4* const*>(bufs->peer_out_rows);
   p.done = reinterpret_cast<const unsigned* const*>(bufs->peer_done);
   p.epoch = epoch;
   p.y = static_cast<__nv_bfloat16*>(y);

@@ -39,7 +39,7 @@ struct FusedParams {
   int R;  // rows of x_rows and y_rows
   int G, width, h;
   float beta_g, beta_u;
-  void* y_rows;         // [R][width] fp32, or bf16 weighted rows when row_w is set
+  void* y_rows;         // [R][width] fp32 (weighted by row_w when it is set)
   const float* row_w;   // nullable: combine weight of each grouped row
   int* status;
 };
@@ -351,19 +351,13 @@ __global__ void __launch_bounds__(fThreads, 1) tc_fused_ffn(const __grid_constan
           float v[32];
           tc::tmem_ld_32x32b_x32(
               tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)((mA + m2) * fBN + c), v);
-          if (p.row_w) {  // a * F(u) as bf16: the combine only adds the rows
-            __nv_bfloat16* yb = static_cast<__nv_bfloat16*>(p.y_rows);
+          // F(u), or a * F(u) when row_w is set (the combine then only adds rows)
+          float* yf = static_cast<float*>(p.y_rows);
 #pragma unroll
-            for (int j = 0; j < 32; ++j)
-              if (c + j < n_valid)
-                yb[(size_t)(tok0 + c + j) * p.width + col] =
-                    __float2bfloat16_rn(v[j] * p.row_w[tok0 + c + j]);
-          } else {
-            float* yf = static_cast<float*>(p.y_rows);
-#pragma unroll
-            for (int j = 0; j < 32; ++j)
-              if (c + j < n_valid) yf[(size_t)(tok0 + c + j) * p.width + col] = v[j];
-          }
+          for (int j = 0; j < 32; ++j)
+            if (c + j < n_valid)
+              yf[(size_t)(tok0 + c + j) * p.width + col] =
+                  p.row_w ? v[j] * p.row_w[tok0 + c + j] : v[j];
         }
       }
       tc::tc_fence_before();

@@ -135,3 +135,40 @@ extern "C" int moe_quantize_e4m3_rows(int64_t rows, int32_t cols, const void* x,
   }
   return launch_status();
 }
+
+extern "C" size_t moe_expert_ffn_e4m3_workspace_bytes(const moe_shape* shape) {
+  if (!moe::shape_ok(shape) || shape->h <= 0) return 0;
+  return moe::align_up((size_t)shape->T * shape->k * shape->h, 256);  // H as E4M3 codes
+}
+
+extern "C" int moe_expert_ffn_e4m3(const moe_shape* shape, int32_t width, const uint8_t* x_rows,
+                                   const float* x_scale, const int32_t* offsets,
+                                   const uint8_t* w_gate, const uint8_t* w_up,
+                                   const uint8_t* w_down, const moe_e4m3_scales* scales,
+                                   const moe_act* act, float* y_rows, void* ws, size_t ws_bytes,
+                                   void* stream) {
+  using namespace moe;
+  if (!shape_ok(shape) || !act || !scales || !offsets || !w_gate || !w_up || !w_down)
+    return MOE_ERR_INVALID_ARG;
+  const moe_shape& s = *shape;
+  if (width <= 0 || width % 256 != 0 || s.h <= 0 || s.h % 128 != 0) return MOE_ERR_UNSUPPORTED;
+  if (act->kind != MOE_ACT_SWIGLU &&
+      !(act->kind == MOE_ACT_SITU_GLU && act->beta_gate > 0.0f && act->beta_up > 0.0f))
+    return MOE_ERR_INVALID_ARG;
+  if (!scales->gate_scale || !scales->up_scale || !scales->down_scale) return MOE_ERR_INVALID_ARG;
+  if (s.T > 0 && (!x_rows || !x_scale || !y_rows)) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x_rows) || !aligned16(w_gate) || !aligned16(w_up) || !aligned16(w_down) ||
+      !aligned16(y_rows))
+    return MOE_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < moe_expert_ffn_e4m3_workspace_bytes(shape)) return MOE_ERR_WORKSPACE;
+  const int64_t R = (int64_t)s.T * s.k;
+  if (R == 0) return MOE_OK;
+  cudaStream_t st = as_stream(stream);
+  TcF8 gu{{scales->gate_scale, scales->up_scale}, x_scale};
+  int rc = tc_gateup(offsets, (int)R, s.N, x_rows, R, width, w_gate, w_up, s.h, *act, ws, s.h, 0,
+                     st, &gu);
+  if (rc != MOE_OK) return rc;
+  TcF8 dn{{scales->down_scale, nullptr}, nullptr};
+  TcSeg seg{w_down, (int64_t)s.N * width, s.h, 0, ws, R, s.h, 0};
+  return tc_store(offsets, (int)R, s.N, width, &seg, 1, y_rows, MODE_STORE_F32, width, st, &dn);
+}

@@ -675,7 +675,7 @@ int launch_ffn_tc(const moe_shape& s, int32_t width, const __nv_bfloat16* x_rows
   if (rc != MOE_OK) return rc;
   TcSeg seg{w_down, (int64_t)s.N * width, s.h, 0, H, R, s.h, 0};
   return tc_store(offsets, (int)R, s.N, width, &seg, 1, y_rows,
-                  row_w ? MODE_STORE_BF16 : MODE_STORE_F32, width, st, nullptr, row_w);
+                  MODE_STORE_F32, width, st, nullptr, row_w);
 }
 
 // Gate/up GEMM with the fused activation: for group g and its rows of X,

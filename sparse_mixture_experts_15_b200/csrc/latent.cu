@@ -63,7 +63,7 @@ struct LatentBufs {
   __nv_bfloat16* x_rows;  // E4M3 experts: the gathered codes of x_l (1 byte each)
   float* x_scale;         // E4M3 experts: one scale per gathered row
   __nv_bfloat16* H;       // E4M3 experts: H as codes
-  float* y_rows;  // bf16 rows a * E(x_l) (half the room used)
+  float* y_rows;  // fp32 rows a * E(x_l)
   float* row_w;   // combine weight of each grouped row
   float* m;
   __nv_bfloat16* m_hat;
@@ -194,7 +194,7 @@ int latent_forward(const moe_shape* shape, const moe_layer_weights* w,
                      0, st, &gu);
     if (rc != MOE_OK) return rc;
     TcSeg seg{w->w_down, (int64_t)s.N * l, s.h, 0, b.H, Tk, s.h, 0};
-    rc = tc_store(offsets, Tk, s.N, l, &seg, 1, b.y_rows, MODE_STORE_BF16, l, st, &dn);
+    rc = tc_store(offsets, Tk, s.N, l, &seg, 1, b.y_rows, MODE_STORE_F32, l, st, &dn);
     if (rc != MOE_OK) return rc;
   } else {
     rc = launch_gather(s, l, b.x_l, MOE_BF16, perm_tok, offsets, b.x_rows, st);
@@ -203,13 +203,12 @@ int latent_forward(const moe_shape* shape, const moe_layer_weights* w,
                    0, st);
     if (rc != MOE_OK) return rc;
     TcSeg seg{w->w_down, (int64_t)s.N * l, s.h, 0, b.H, Tk, s.h, 0};
-    rc = tc_store(offsets, Tk, s.N, l, &seg, 1, b.y_rows, MODE_STORE_BF16, l, st, nullptr,
+    rc = tc_store(offsets, Tk, s.N, l, &seg, 1, b.y_rows, MODE_STORE_F32, l, st, nullptr,
                   b.row_w);
     if (rc != MOE_OK) return rc;
   }
-  // the down GEMMs stored bf16 rows a * E(x_l): the combine adds them
-  rc = launch_combine_weighted(s, l, reinterpret_cast<const __nv_bfloat16*>(b.y_rows), row_of,
-                               b.m, MOE_F32, st);
+  // the down GEMMs stored rows a * E(x_l): the combine adds them
+  rc = launch_combine_weighted(s, l, b.y_rows, row_of, b.m, MOE_F32, st);
   if (rc != MOE_OK) return rc;
   {
     int blocks = (s.T + 7) / 8;

@@ -24,7 +24,7 @@ struct LayerBufs {
   void* permute_ws;
   void* x_rows;
   void* ffn_ws;
-  float* y_rows;  // bf16 layers: bf16 rows a * F(u) (half the room used)
+  float* y_rows;  // bf16 layers: fp32 rows a * F(u)
   float* row_w;   // combine weight of each grouped row
   void* stats_ws;
   void* rd_ws;
@@ -67,8 +67,8 @@ LayerBufs carve_layer(const moe_shape& s, int32_t act_dtype, void* base) {
   return b;
 }
 
-// row_w (bf16 only, nullable): store bf16 rows row_w[r] * F(u) into y_rows
-// instead of fp32 F(u).
+// row_w (bf16 only, nullable): store rows row_w[r] * F(u) into y_rows instead
+// of F(u).
 int run_ffn(const moe_shape& s, int32_t width, const void* x_rows, int32_t dtype,
             const int32_t* offsets, const void* w_gate, const void* w_up, const void* w_down,
             const moe_act& act, float* y_rows, void* ws, cudaStream_t st,
@@ -154,8 +154,8 @@ extern "C" int moe_layer_fwd(const moe_shape* shape, const moe_layer_weights* w,
   int32_t* totals = o.totals ? o.totals : b.totals;
   cudaStream_t st = as_stream(stream);
   // bf16 layers: the permutation records each grouped row's combine weight,
-  // the down GEMM stores bf16 rows a * F(u), and the combine adds them (the
-  // down projection carries the multiply of the weighted combine y = sum a F)
+  // the down GEMM stores rows a * F(u), and the combine adds them (the down
+  // projection carries the multiply of the weighted combine y = sum a F)
   float* row_w = act_dtype == MOE_BF16 ? b.row_w : nullptr;
 
   int rc;
@@ -195,8 +195,6 @@ extern "C" int moe_layer_fwd(const moe_shape* shape, const moe_layer_weights* w,
   rc = run_ffn(s, s.d, b.x_rows, act_dtype, offsets, w->w_gate, w->w_up, w->w_down, w->act,
                b.y_rows, b.ffn_ws, st, row_w);
   if (rc != MOE_OK) return rc;
-  if (row_w)
-    return launch_combine_weighted(s, s.d, reinterpret_cast<const __nv_bfloat16*>(b.y_rows),
-                                   row_of, y, act_dtype, st);
+  if (row_w) return launch_combine_weighted(s, s.d, b.y_rows, row_of, y, act_dtype, st);
   return launch_combine(s, s.d, b.y_rows, row_of, top_w, y, act_dtype, st);
 }

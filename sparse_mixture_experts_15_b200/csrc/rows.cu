@@ -89,11 +89,11 @@ __global__ void __launch_bounds__(256)
   }
 }
 
-// One warp per token; rows already carry their weights (bf16 a * F(u)), the
+// One warp per token; rows already carry their weights (fp32 a * F(u)), the
 // kept slots are added in ascending s in fp32 and rounded once.
 template <typename TY>
 __global__ void __launch_bounds__(256)
-    combine_weighted(const uint4* __restrict__ rows, int width8,
+    combine_weighted(const float4* __restrict__ rows, int width4,
                      const int32_t* __restrict__ row_of, int T, int k, TY* __restrict__ y,
                      int* status) {
   pdl_wait();
@@ -101,8 +101,8 @@ __global__ void __launch_bounds__(256)
   const int lane = threadIdx.x & 31;
   for (int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; t < T;
        t += (gridDim.x * blockDim.x) >> 5) {
-    for (int c = lane; c < width8; c += 32) {
-      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    for (int c = lane; c < width4; c += 32) {
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
       for (int s = 0; s < k; ++s) {
         const int r = row_of[(size_t)t * k + s];
         if (r < 0) continue;
@@ -110,14 +110,13 @@ __global__ void __launch_bounds__(256)
           record_error(status, MOE_ERR_BOUNDS);
           continue;
         }
-        float v[8];
-        load8(reinterpret_cast<const __nv_bfloat16*>(rows + (size_t)r * width8 + c), v);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) acc[i] += v[i];
+        const float4 v = rows[(size_t)r * width4 + c];
+        acc.x += v.x;
+        acc.y += v.y;
+        acc.z += v.z;
+        acc.w += v.w;
       }
-      TY* o = y + ((size_t)t * width8 + c) * 8;
-      store4<TY>(o, make_float4(acc[0], acc[1], acc[2], acc[3]));
-      store4<TY>(o + 4, make_float4(acc[4], acc[5], acc[6], acc[7]));
+      store4<TY>(y + ((size_t)t * width4 + c) * 4, acc);
     }
   }
 }
@@ -163,23 +162,23 @@ int launch_combine(const moe_shape& s, int32_t width, const float* y_rows, const
   return launch_status();
 }
 
-int launch_combine_weighted(const moe_shape& s, int32_t width, const __nv_bfloat16* rows,
+int launch_combine_weighted(const moe_shape& s, int32_t width, const float* rows,
                             const int32_t* row_of, void* y, int32_t y_dtype, cudaStream_t st) {
   if (s.T == 0) return MOE_OK;
-  const int w8 = width / 8;
+  const int w4 = width / 4;
   const int grid = grid_cap(s.T);
-  const uint4* r = reinterpret_cast<const uint4*>(rows);
+  const float4* r = reinterpret_cast<const float4*>(rows);
   if (y_dtype == MOE_F32) {
     MOE_PREFER_SHARED((combine_weighted<float>));
-    launch_pdl(combine_weighted<float>, dim3(grid), dim3(256), 0, st, r, w8, row_of, s.T, s.k,
+    launch_pdl(combine_weighted<float>, dim3(grid), dim3(256), 0, st, r, w4, row_of, s.T, s.k,
                static_cast<float*>(y), status_word());
   } else if (y_dtype == MOE_BF16) {
     MOE_PREFER_SHARED((combine_weighted<__nv_bfloat16>));
-    launch_pdl(combine_weighted<__nv_bfloat16>, dim3(grid), dim3(256), 0, st, r, w8, row_of,
+    launch_pdl(combine_weighted<__nv_bfloat16>, dim3(grid), dim3(256), 0, st, r, w4, row_of,
                s.T, s.k, static_cast<__nv_bfloat16*>(y), status_word());
   } else {
     MOE_PREFER_SHARED((combine_weighted<__half>));
-    launch_pdl(combine_weighted<__half>, dim3(grid), dim3(256), 0, st, r, w8, row_of, s.T, s.k,
+    launch_pdl(combine_weighted<__half>, dim3(grid), dim3(256), 0, st, r, w4, row_of, s.T, s.k,
                static_cast<__half*>(y), status_word());
   }
   return launch_status();

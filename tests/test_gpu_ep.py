@@ -66,7 +66,7 @@ def _ep_layer(wl, splits, u_all, w, b, wg, wu, wd, epochs=1):
     cap = max(16, max(p.recv_rows for p in plans))
     bufs = [dict(recv_rows=torch.zeros((cap, d), dtype=torch.bfloat16, device="cuda"),
                  recv_w=torch.zeros(cap, dtype=torch.float32, device="cuda"),
-                 out_rows=torch.zeros((cap, d), dtype=torch.bfloat16, device="cuda"),
+                 out_rows=torch.zeros((cap, d), dtype=torch.float32, device="cuda"),
                  arrive=torch.zeros(R, **i32), done=torch.zeros(4, **i32)) for _ in range(R)]
     peers = {n: _ptrs([bf[n] for bf in bufs]) for n in bufs[0]}
     es = moe.shape(cap, d, E, 1, h, 1, 0)
@@ -148,7 +148,7 @@ def test_ep_wait_runs_out_without_arrivals():
     cap = 64
     bufs = [dict(recv_rows=torch.zeros((cap, wl.d), dtype=torch.bfloat16, device="cuda"),
                  recv_w=torch.zeros(cap, dtype=torch.float32, device="cuda"),
-                 out_rows=torch.zeros((cap, wl.d), dtype=torch.bfloat16, device="cuda"),
+                 out_rows=torch.zeros((cap, wl.d), dtype=torch.float32, device="cuda"),
                  arrive=torch.zeros(R, **i32), done=torch.zeros(4, **i32)) for _ in range(R)]
     peers = {n: _ptrs([bf[n] for bf in bufs]) for n in bufs[0]}
     es = moe.shape(cap, wl.d, E, 1, wl.h, 1, 0)
