@@ -351,7 +351,7 @@ MOE_API int moe_quantize_e4m3_rows(int64_t rows, int32_t cols, const void* x, in
  * moe_quantize_e4m3_rows), the experts' E4M3 codes (gate, up [N][h][width],
  * down [N][width][h]) with their row scales, SiTU-GLU or SwiGLU; H is stored
  * as E4M3 codes with no scale in ws; y_rows [T*k][width] fp32, F(u) of each
- * grouped row (not weighted).  width a multiple of 256, h of 128.
+ * grouped row (not weighted).  width and h multiples of 128.
  * ws: moe_expert_ffn_e4m3_workspace_bytes.  Errors as moe_expert_ffn. */
 MOE_API size_t moe_expert_ffn_e4m3_workspace_bytes(const moe_shape* shape);
 MOE_API int moe_expert_ffn_e4m3(const moe_shape* shape, int32_t width, const uint8_t* x_rows,

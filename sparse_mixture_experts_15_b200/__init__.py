@@ -463,6 +463,10 @@ def moe_quantize_e4m3_rows(x, codes, scales, stream=None):
                                        _ptr(scales), _stream(stream)), "moe_quantize_e4m3_rows")
 
 
+def moe_expert_ffn_e4m3_workspace_bytes(s: MoeShape) -> int:
+    return int(_lib.moe_expert_ffn_e4m3_workspace_bytes(ctypes.byref(s)))
+
+
 def moe_expert_ffn_e4m3(s: MoeShape, width: int, x_rows, x_scale, offsets, w_gate, w_up,
                         w_down, gate_scale, up_scale, down_scale, y_rows, a=None, ws=None,
                         stream=None):

@@ -151,7 +151,7 @@ extern "C" int moe_expert_ffn_e4m3(const moe_shape* shape, int32_t width, const 
   if (!shape_ok(shape) || !act || !scales || !offsets || !w_gate || !w_up || !w_down)
     return MOE_ERR_INVALID_ARG;
   const moe_shape& s = *shape;
-  if (width <= 0 || width % 256 != 0 || s.h <= 0 || s.h % 128 != 0) return MOE_ERR_UNSUPPORTED;
+  if (width <= 0 || width % 128 != 0 || s.h <= 0 || s.h % 128 != 0) return MOE_ERR_UNSUPPORTED;
   if (act->kind != MOE_ACT_SWIGLU &&
       !(act->kind == MOE_ACT_SITU_GLU && act->beta_gate > 0.0f && act->beta_up > 0.0f))
     return MOE_ERR_INVALID_ARG;

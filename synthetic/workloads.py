@@ -57,6 +57,7 @@ class Workload:
     shared_hidden: int = 0
     beta_gate: float = 0.0
     beta_up: float = 0.0
+    expert_sigma: float = 0.0      # sigma of the routed experts' weights (0: SIGMA_W)
     extra: dict = field(default_factory=dict)
 
     def router_bias(self):
@@ -71,6 +72,10 @@ class Workload:
             return 0
         T = self.T if T is None else T
         return int(math.ceil(self.capacity_factor * self.k * T / self.N))
+
+    @property
+    def w_sigma(self) -> float:
+        return self.expert_sigma if self.expert_sigma > 0.0 else SIGMA_W
 
     @property
     def expert_in(self) -> int:

@@ -96,6 +96,14 @@ def rel_err(got, ref):
     return float(np.max(np.abs(got - ref))) / (rms if rms > 0 else 1.0)
 
 
+def fro_err(got, ref):
+    """||got - ref|| / ||ref|| (Frobenius), the gradients' tolerance measure."""
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    n = float(np.linalg.norm(ref))
+    return float(np.linalg.norm(got - ref)) / (n if n > 0 else 1.0)
+
+
 # ------------------------------------------------------------- LatentMoE
 def dev_latent(wl: W.Workload, device="cuda"):
     """Device weights of a LatentMoE workload (bf16; router fp32)."""
@@ -104,9 +112,9 @@ def dev_latent(wl: W.Workload, device="cuda"):
     st = torch.cuda.current_stream().cuda_stream
     out = dict(
         w_route=dev_normal(wl.seed, W.TID_WROUTE, (E, d), W.SIGMA_W, S.DT_F32, device),
-        w_gate=dev_normal(wl.seed, W.TID_WGATE, (E, h, l), W.SIGMA_W, S.DT_BF16, device),
-        w_up=dev_normal(wl.seed, W.TID_WUP, (E, h, l), W.SIGMA_W, S.DT_BF16, device),
-        w_down=dev_normal(wl.seed, W.TID_WDOWN, (E, l, h), W.SIGMA_W, S.DT_BF16, device),
+        w_gate=dev_normal(wl.seed, W.TID_WGATE, (E, h, l), wl.w_sigma, S.DT_BF16, device),
+        w_up=dev_normal(wl.seed, W.TID_WUP, (E, h, l), wl.w_sigma, S.DT_BF16, device),
+        w_down=dev_normal(wl.seed, W.TID_WDOWN, (E, l, h), wl.w_sigma, S.DT_BF16, device),
         w_dp=dev_normal(wl.seed, W.TID_WDP, (l, d), W.SIGMA_W, S.DT_BF16, device),
         w_upp=dev_normal(wl.seed, W.TID_WUPP, (d, l), W.SIGMA_W, S.DT_BF16, device))
     sg = torch.empty((max(n, 1), sh, d), dtype=torch.bfloat16, device=device)
@@ -123,9 +131,9 @@ def dev_latent(wl: W.Workload, device="cuda"):
 
 def host_latent_expert(wl: W.Workload, e: int):
     l, h = wl.latent, wl.h
-    g = S.normal(wl.seed, W.TID_WGATE, (h, l), W.SIGMA_W, S.DT_BF16, offset=e * h * l)
-    u = S.normal(wl.seed, W.TID_WUP, (h, l), W.SIGMA_W, S.DT_BF16, offset=e * h * l)
-    d = S.normal(wl.seed, W.TID_WDOWN, (l, h), W.SIGMA_W, S.DT_BF16, offset=e * l * h)
+    g = S.normal(wl.seed, W.TID_WGATE, (h, l), wl.w_sigma, S.DT_BF16, offset=e * h * l)
+    u = S.normal(wl.seed, W.TID_WUP, (h, l), wl.w_sigma, S.DT_BF16, offset=e * h * l)
+    d = S.normal(wl.seed, W.TID_WDOWN, (l, h), wl.w_sigma, S.DT_BF16, offset=e * l * h)
     return O.Mat(O.BF16, h, l, data=g), O.Mat(O.BF16, h, l, data=u), O.Mat(O.BF16, l, h, data=d)
 
 

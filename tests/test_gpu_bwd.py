@@ -5,9 +5,15 @@ The oracle differentiates L = sum dy . y + alpha N sum f_i P_i in double with
 the selected sets and the capacity drops held fixed (the reading of the
 tutorial's §3.7 and of the Stable LatentMoE demo's "only selected experts
 receive gradient").  The GPU keeps the expert operands in bf16 (the forward's
-storage) with fp32 accumulation, so every gradient is compared within the
-bf16 bound of the forward, max|d|/rms <= 2e-2; an expert with no kept
-dispatch must get exactly zero weight gradient."""
+storage) with fp32 accumulation.  Each gradient element passes through at
+most four bf16 roundings (the gathered input, g / v / H, a * dy and dG / dV),
+each an error of at most 2^-9 of the value and about 2^-9 / sqrt(3) rms, so
+the relative Frobenius error ||got - ref|| / ||ref|| of every gradient is
+expected near 2.3e-3; it is bounded by 1e-2.  A max-over-elements measure
+would not do here: a weight gradient of an expert with one or two rows is an
+outer product of heavy-tailed vectors whose largest element is 20-50 times its
+rms, so one element's 2^-9 rounding reads as several 1e-2 of rms.  An expert
+with no kept dispatch must get exactly zero weight gradient."""
 import dataclasses
 
 import numpy as np
@@ -17,13 +23,13 @@ import oracle as O
 import synthetic as S
 from synthetic import workloads as W
 
-from inputs import (dev_experts, dev_normal, dev_router, dev_u, host_expert, host_router, host_u,
-                    rel_err)
+from inputs import (dev_experts, dev_normal, dev_router, dev_u, fro_err, host_expert, host_router,
+                    host_u)
 
 torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
 
-TOL = 2e-2
+TOL = 1e-2
 TID_DY = 60
 
 if torch.cuda.is_available():
@@ -93,7 +99,7 @@ def test_layer_backward_vs_oracle(case):
                            f=f_loads.astype(np.float64))
     pairs = (("dz", "dz"), ("du", "du"), ("dw_route", "dWr"), ("dw_gate", "dWg"),
              ("dw_up", "dWu"), ("dw_down", "dWd"))
-    errs = {g: rel_err(got[g], ref[r]) for g, r in pairs}
+    errs = {g: fro_err(got[g], ref[r]) for g, r in pairs}
     assert all(np.isfinite(v) for v in errs.values()), errs
     assert max(errs.values()) < TOL, errs
     # only the selected experts of kept dispatches receive weight gradient
@@ -158,7 +164,7 @@ def test_latent_backward_vs_oracle():
     pairs = (("dx", "dx"), ("dz", "dz"), ("dw_route", "dWr"), ("dw_gate", "dWg"),
              ("dw_up", "dWu"), ("dw_down", "dWd"), ("dw_dp", "dWdp"), ("dw_upp", "dWupp"),
              ("dsh_gate", "dSg"), ("dsh_up", "dSu"), ("dsh_down", "dSd"))
-    errs = {gk: rel_err(got[gk], ref[rk]) for gk, rk in pairs}
+    errs = {gk: fro_err(got[gk], ref[rk]) for gk, rk in pairs}
     assert all(np.isfinite(v) for v in errs.values()), errs
     assert max(errs.values()) < TOL, errs
     unused = np.setdiff1d(np.arange(N), idx.ravel())
