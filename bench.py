@@ -288,8 +288,11 @@ class Step:
         """The expert FFN alone on replica r's own grouped rows (filled by
         split(r)), so consecutive replays read rows and weights that are not
         L2-resident."""
-        self.moe.moe_expert_ffn(self.s, self.wl.d, r.x_rows, r.offsets, *r.w, self.y_rows,
-                                self.act, ws=self.ws_ffn)
+        self._ffn(r, r.x_rows, r.offsets)
+
+    def _ffn(self, r: Replica, x_rows, offsets):
+        self.moe.moe_expert_ffn(self.s, self.wl.d, x_rows, offsets, *r.w, self.y_rows, self.act,
+                                ws=self.ws_ffn)
 
     def split(self, r: Replica):
         """The step split at the expert FFN; keeps r's grouped rows and offsets."""
@@ -304,7 +307,7 @@ class Step:
         m.moe_permute(self.s, self.top_idx, self.counts, self.offsets, self.perm, self.row_of,
                       self.overflow, self.totals, ws=self.ws_perm)
         m.moe_gather(self.s, self.wl.d, r.u, self.perm, self.offsets, self.x_rows)
-        self.ffn(r)
+        self._ffn(r, self.x_rows, self.offsets)
         m.moe_combine(self.s, self.wl.d, self.y_rows, self.row_of, self.top_w, self.y)
 
 
