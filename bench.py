@@ -880,6 +880,9 @@ def main():
     ap.add_argument("--decode-T", type=int, default=32, help="decode batch (1, 8 or 32)")
     ap.add_argument("--tokens", type=int, default=0,
                     help="override T (smaller cases for profiling captures)")
+    ap.add_argument("--experts", type=int, default=0,
+                    help="latent workload: override the routed expert count (profiling captures "
+                         "of a few GB with the full-size per-expert shape)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--fp8", action="store_true",
@@ -892,6 +895,10 @@ def main():
     wl = W.decode(T=args.decode_T) if args.workload == "decode" else W.ALL[args.workload]()
     if args.tokens > 0 and args.workload != "decode":
         wl.T = args.tokens
+    if args.experts > 0:
+        if args.workload != "latent":
+            ap.error("--experts applies to the latent workload")
+        wl.N = args.experts
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

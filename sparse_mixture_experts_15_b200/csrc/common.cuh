@@ -24,6 +24,9 @@ constexpr int kMaxDevices = 64;
 
 inline bool device_slot(int dev) { return dev >= 0 && dev < kMaxDevices; }
 
+// SM count of the current device (cached per device; 148 if unknown).
+int sm_count();
+
 // True while the once-per-device setup guarded by `done` has not run on dev.
 inline bool needs_setup(const std::atomic<bool>* done, int dev) {
   return device_slot(dev) && !done[dev].load(std::memory_order_acquire);

@@ -37,6 +37,22 @@
 #include "tc_primitives.cuh"
 
 namespace moe {
+
+// SM count of the current device, looked up once per device.
+int sm_count() {
+  static std::atomic<int> cached[kMaxDevices];
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (!device_slot(dev)) return 148;
+  int n = cached[dev].load(std::memory_order_relaxed);
+  if (!n) {
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+    cached[dev].store(n, std::memory_order_relaxed);
+  }
+  return n;
+}
+
 namespace {
 
 constexpr int kBM = 128;
@@ -533,20 +549,6 @@ bool make_tmap(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, u
              const_cast<void*>(base), dims, strides, box,
              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-int sm_count() {
-  static std::atomic<int> cached[kMaxDevices];
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (!device_slot(dev)) return 148;
-  int n = cached[dev].load(std::memory_order_relaxed);
-  if (!n) {
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    if (n <= 0) n = 148;
-    cached[dev].store(n, std::memory_order_relaxed);
-  }
-  return n;
 }
 
 // Clusters of two CTAs that can be resident at once for a pair kernel (a GPC

@@ -17,54 +17,71 @@
 namespace moe {
 namespace {
 
-// Many experts (N > 16): a 128 x 128 (tokens x experts) block tile, 8 x 8
-// logits per thread, K walked in steps of 16 through double-buffered shared
-// tiles (the next step's global loads are held in registers while the
-// current step computes).  Each logit is still one thread's FMA chain over j
-// in ascending order, so the result equals the other router kernels bit for
-// bit.  A thread's rows are {4 ty + i, 64 + 4 ty + i} and its experts
-// {4 tx + j, 64 + 4 tx + j}, so the 16-byte shared reads of a warp are
-// broadcasts or consecutive.
-constexpr int kBigBT = 128, kBigBN = 128, kBigBK = 16, kBigThreads = 256;
+// Many experts (N > 16): a block tile of 8 TG tokens x 128 experts with
+// 16 TG threads, 8 x 8 logits per thread, K walked in steps of 16 through
+// double-buffered shared tiles (the next step's global loads are held in
+// registers while the current step computes).  Each logit is still one
+// thread's FMA chain over j in ascending order, so the result equals the
+// other router kernels bit for bit.  A thread's tokens are {4 ty + i,
+// 4 TG + 4 ty + i} and its experts {4 tx + j, 64 + 4 tx + j}, so the 16-byte
+// shared reads of a warp are broadcasts or consecutive.  TG (8..16) is picked
+// per launch so that the tiles fill whole waves of SMs (see pick_tg).
+constexpr int kBigBN = 128, kBigBK = 16;
 
-template <typename TU>
-__global__ void __launch_bounds__(kBigThreads)
+template <typename TU, int TG>
+__global__ void __launch_bounds__(16 * TG)
     router_logits_big(const TU* __restrict__ u, const float* __restrict__ w,
                       const float* __restrict__ bias, float* __restrict__ z, int T, int d, int N) {
+  constexpr int BT = 8 * TG, HALF = 4 * TG, NT = 16 * TG;
+  constexpr int WU = (2 * kBigBN + NT - 1) / NT;  // weight-row loads per thread (1 or 2)
   pdl_wait();
   pdl_allow_next();
-  __shared__ __align__(16) float us[2][kBigBK][kBigBT];
+  __shared__ __align__(16) float us[2][kBigBK][BT];
   __shared__ __align__(16) float wsm[2][kBigBK][kBigBN];
-  const int t0 = blockIdx.x * kBigBT, n0 = blockIdx.y * kBigBN;
+  const int t0 = blockIdx.x * BT, n0 = blockIdx.y * kBigBN;
   const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
-  // this thread's share of a K step: row lr (token / expert), 8 columns at lc
-  const int lr = tid >> 1, lc = (tid & 1) * 8;
   float acc[8][8];
 #pragma unroll
   for (int i = 0; i < 8; ++i)
 #pragma unroll
     for (int j = 0; j < 8; ++j) acc[i][j] = 0.0f;
-  float ru[8], rw[8];
+  // a K step's loads: token row tid >> 1 (8 columns at (tid & 1) * 8), and
+  // expert rows (tid + q NT) >> 1 for q < WU
+  float ru[8], rw[WU][8];
   auto fetch = [&](int k0) {
     const int kw = min(kBigBK, d - k0);  // multiple of 8
-    if (t0 + lr < T && lc < kw) {
-      load8(u + (size_t)(t0 + lr) * d + k0 + lc, ru);
-    } else {
+    {
+      const int lr = tid >> 1, lc = (tid & 1) * 8;
+      if (t0 + lr < T && lc < kw) {
+        load8(u + (size_t)(t0 + lr) * d + k0 + lc, ru);
+      } else {
 #pragma unroll
-      for (int j = 0; j < 8; ++j) ru[j] = 0.0f;
+        for (int j = 0; j < 8; ++j) ru[j] = 0.0f;
+      }
     }
-    if (n0 + lr < N && lc < kw) {
-      load8(w + (size_t)(n0 + lr) * d + k0 + lc, rw);
-    } else {
 #pragma unroll
-      for (int j = 0; j < 8; ++j) rw[j] = 0.0f;
+    for (int q = 0; q < WU; ++q) {
+      const int x = tid + q * NT, lr = x >> 1, lc = (x & 1) * 8;
+      if (lr < kBigBN && n0 + lr < N && lc < kw) {
+        load8(w + (size_t)(n0 + lr) * d + k0 + lc, rw[q]);
+      } else {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) rw[q][j] = 0.0f;
+      }
     }
   };
   auto put = [&](int buf) {
+    {
+      const int lr = tid >> 1, lc = (tid & 1) * 8;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      us[buf][lc + j][lr] = ru[j];
-      wsm[buf][lc + j][lr] = rw[j];
+      for (int j = 0; j < 8; ++j) us[buf][lc + j][lr] = ru[j];
+    }
+#pragma unroll
+    for (int q = 0; q < WU; ++q) {
+      const int x = tid + q * NT, lr = x >> 1, lc = (x & 1) * 8;
+      if (lr < kBigBN)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) wsm[buf][lc + j][lr] = rw[q][j];
     }
   };
   fetch(0);
@@ -77,7 +94,7 @@ __global__ void __launch_bounds__(kBigThreads)
     const int kw = min(kBigBK, d - k0);
     for (int kk = 0; kk < kw; ++kk) {
       const float4 a0 = *reinterpret_cast<const float4*>(&us[buf][kk][4 * ty]);
-      const float4 a1 = *reinterpret_cast<const float4*>(&us[buf][kk][64 + 4 * ty]);
+      const float4 a1 = *reinterpret_cast<const float4*>(&us[buf][kk][HALF + 4 * ty]);
       const float4 b0 = *reinterpret_cast<const float4*>(&wsm[buf][kk][4 * tx]);
       const float4 b1 = *reinterpret_cast<const float4*>(&wsm[buf][kk][64 + 4 * tx]);
       const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
@@ -95,7 +112,7 @@ __global__ void __launch_bounds__(kBigThreads)
   }
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    const int t = t0 + (i < 4 ? 4 * ty + i : 64 + 4 * ty + i - 4);
+    const int t = t0 + (i < 4 ? 4 * ty + i : HALF + 4 * ty + i - 4);
     if (t >= T) continue;
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
@@ -103,6 +120,27 @@ __global__ void __launch_bounds__(kBigThreads)
       if (n < N) z[(size_t)t * N + n] = bias ? __fadd_rn(acc[i][j], bias[n]) : acc[i][j];
     }
   }
+}
+
+// Token-tile width 8 TG for the large router: one CTA's tile takes about the
+// same time whatever TG (FMA-bound per SM), so the step lasts about
+// ceil(tiles / SMs) tiles of 8 TG tokens; the TG with the least
+// ceil(tiles / SMs) * TG wins (larger TG on ties).  4096 tokens x 896
+// experts on 148 SMs: TG = 13 (280 tiles, 2 per SM) against TG = 16's 224
+// tiles, also 2 per SM but 128 tokens each.
+int pick_tg(int T, int N, int sms) {
+  const int64_t nt = (N + kBigBN - 1) / kBigBN;
+  int best = 16;
+  int64_t best_cost = INT64_MAX;
+  for (int tg = 16; tg >= 8; --tg) {
+    const int64_t tiles = nt * ((T + 8 * tg - 1) / (8 * tg));
+    const int64_t cost = (tiles + sms - 1) / sms * tg;
+    if (cost < best_cost) {
+      best_cost = cost;
+      best = tg;
+    }
+  }
+  return best;
 }
 
 // (z, index) ordering of the top-k: larger z first, equal z -> lower index.
@@ -302,12 +340,28 @@ __global__ void __launch_bounds__(kRouteThreads)
   }
 }
 
+template <typename TU, int TG>
+void launch_logits_tg(const TU* u, const float* w, const float* bias, float* z, int T, int d,
+                      int N, cudaStream_t st) {
+  dim3 grid((T + 8 * TG - 1) / (8 * TG), (N + kBigBN - 1) / kBigBN);
+  MOE_PREFER_SHARED((router_logits_big<TU, TG>));
+  launch_pdl(router_logits_big<TU, TG>, grid, dim3(16 * TG), 0, st, u, w, bias, z, T, d, N);
+}
+
 template <typename TU>
 void launch_logits(const TU* u, const float* w, const float* bias, float* z, int T, int d, int N,
                    cudaStream_t st) {
-  dim3 grid((T + kBigBT - 1) / kBigBT, (N + kBigBN - 1) / kBigBN);
-  MOE_PREFER_SHARED((router_logits_big<TU>));
-  launch_pdl(router_logits_big<TU>, grid, dim3(kBigThreads), 0, st, u, w, bias, z, T, d, N);
+  switch (pick_tg(T, N, sm_count())) {
+    case 8: return launch_logits_tg<TU, 8>(u, w, bias, z, T, d, N, st);
+    case 9: return launch_logits_tg<TU, 9>(u, w, bias, z, T, d, N, st);
+    case 10: return launch_logits_tg<TU, 10>(u, w, bias, z, T, d, N, st);
+    case 11: return launch_logits_tg<TU, 11>(u, w, bias, z, T, d, N, st);
+    case 12: return launch_logits_tg<TU, 12>(u, w, bias, z, T, d, N, st);
+    case 13: return launch_logits_tg<TU, 13>(u, w, bias, z, T, d, N, st);
+    case 14: return launch_logits_tg<TU, 14>(u, w, bias, z, T, d, N, st);
+    case 15: return launch_logits_tg<TU, 15>(u, w, bias, z, T, d, N, st);
+    default: return launch_logits_tg<TU, 16>(u, w, bias, z, T, d, N, st);
+  }
 }
 
 }  // namespace

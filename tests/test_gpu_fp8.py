@@ -4,11 +4,13 @@ beta_g * beta_u = 100 < 448, the E4M3 maximum) against the CPU oracle's FP8
 form, through the C ABI.
 
 The row quantiser must match the oracle's bit for bit (its decisions are taken
-on the same fp32 quotients).  The E4M3 tensor-core MMA accumulates with less
-than fp32 precision, so an element of H near a rounding midpoint can take the
-neighbouring E4M3 code: outputs are compared by relative Frobenius error
-within 2e-2, with a guard of 0.1 on max|d|/rms, and the grouped FFN test
-checks that every differing code is such a near-midpoint neighbour."""
+on the same fp32 quotients).  The grouped E4M3 FFN is compared within the
+bf16 bound, max|d|/rms <= 2e-2, and its H codes one by one (a code may differ
+only where H lies at a rounding midpoint).  The layer's x_l = bf16(W_dp x)
+comes from an fp32 tensor-core GEMM, so a last-place bf16 difference from the
+oracle's x_l can move a token's E4M3 scale (its amax) and with it every code
+of that token: the layer outputs are compared by relative Frobenius error
+within 2e-2, with a guard of 0.1 on max|d|/rms."""
 import numpy as np
 import pytest
 
@@ -94,19 +96,18 @@ def _ffn_inputs(width, h, counts, seed):
 def test_expert_ffn_e4m3_vs_oracle(case):
     """Grouped rows against the oracle's expert with E4M3 matrices and H
     rounded to E4M3 (the hidden vector is the oracle's expert with an identity
-    down projection).
+    down projection, taken before rounding).
 
-    The FP8 tensor-core MMA does not accumulate in full fp32 (on the B200 its
-    pre-activations differ from the exact sums by about 1e-4 relative, with
-    bf16 operands the same GEMMs agree to fp32 rounding), so the E4M3 code of
-    H, a rounding decision taken on that value, can land on the neighbouring
-    code where the exact H lies near the midpoint of two codes.  Checked:
-    differing codes are few (<= 2%), each is the neighbour of the oracle's
-    code, and the exact H lies within 2^-9 of the midpoint between them
-    (relative to |H|, or to rms(H) where H is smaller); the fp32 rows equal W_down times the kernel's own H codes within
-    the accumulation error (max|d|/rms <= 2e-3); and the rows match the
-    oracle within a relative Frobenius error of 2e-2 (a 0.5% share of H
-    elements one code step off moves y by about 0.6%)."""
+    The code of H is a rounding decision the kernel takes on an fp32 value
+    formed with approximate SiLU / tanh, so where the exact H lies at a
+    midpoint of two codes the kernel may take the neighbour; and a tiny H
+    whose sign differs rounds to the other zero.  Checked: H values (decoded,
+    so +0 = -0) differ in at most 0.1% of elements, each differing code is the
+    neighbour of the oracle's and the exact H lies within 2^-9 (of |H|, or of
+    rms(H) where H is smaller) of the midpoint between them; the fp32 rows
+    equal W_down times the kernel's own H codes within 1e-5 of rms (the E4M3
+    MMA accumulates in fp32); and the rows match the oracle within the bf16
+    bound, max|d|/rms <= 2e-2."""
     width, h, counts, kind = FFN_CASES[case]
     N, R = len(counts), int(sum(counts))
     (xc, xs), mats = _ffn_inputs(width, h, counts, seed=77 + width + h)
@@ -162,8 +163,8 @@ def _check_e4m3_ffn(act_kind, width, h, offs, xc, xs, mats, got_y, got_h):
                                   round_h=0)
             chk_y[i] = dn_val @ e4[got_h[i]]
     ref_codes = O.round_e4m3(exact_h)
-    diff = got_h != ref_codes
-    assert diff.mean() <= 0.02, f"{int(diff.sum())} of {diff.size} H codes differ"
+    diff = e4[got_h] != e4[ref_codes]  # values: the two zeros are equal
+    assert diff.mean() <= 1e-3, f"{int(diff.sum())} of {diff.size} H values differ"
     if diff.any():
         gd, rd, hx = got_h[diff], ref_codes[diff], exact_h[diff]
         step = np.abs((gd & 0x7F).astype(int) - (rd & 0x7F).astype(int))
@@ -173,11 +174,11 @@ def _check_e4m3_ffn(act_kind, width, h, offs, xc, xs, mats, got_y, got_h):
         # scales with the terms of the sum, not with a small (cancelled) result
         off = np.abs(hx - mid) / np.maximum(np.abs(hx), np.sqrt(np.mean(exact_h ** 2)))
         assert off.max() <= 2.0 ** -9, f"a differing code {off.max():.2e} away from a midpoint"
-    down_err, fro = rel_err(got_y, chk_y), fro_err(got_y, ref_y)
-    print(f"H codes differing {diff.mean():.4%}, down GEMM vs own H {down_err:.2e}, "
-          f"rows vs oracle {fro:.2e} (Frobenius)")
-    assert down_err <= 2e-3, "down GEMM against the kernel's own H codes"
-    assert fro <= TOL
+    down_err, err = rel_err(got_y, chk_y), rel_err(got_y, ref_y)
+    print(f"H values differing {diff.mean():.4%}, down GEMM vs own H {down_err:.2e}, "
+          f"rows vs oracle {err:.2e} (max|d|/rms)")
+    assert down_err <= 1e-5, "down GEMM against the kernel's own H codes"
+    assert err <= TOL
 
 
 def small_latent(T=200):
@@ -259,6 +260,8 @@ def test_latent_fp8_small_all_tokens():
     assert outs["counts"].sum() == wl.k * wl.T
     got = y.float().cpu().numpy()
     assert np.all(np.isfinite(got))
+    print(f"layer vs oracle: {fro_err(got, ref):.2e} (Frobenius), {rel_err(got, ref):.2e} "
+          f"(max|d|/rms)")
     assert fro_err(got, ref) < TOL
     assert rel_err(got, ref) < 0.1
     # the FP8 layer differs from the bf16 one by the quantisation error only
@@ -303,5 +306,7 @@ def test_latent_fp8_full_size_sampled():
     # E4M3 H codes may sit one step off where H is near a rounding midpoint
     # (test_expert_ffn_e4m3_vs_oracle): relative Frobenius error, and a
     # looser guard on the largest element
+    print(f"layer vs oracle: {fro_err(got, ref):.2e} (Frobenius), {rel_err(got, ref):.2e} "
+          f"(max|d|/rms)")
     assert fro_err(got, ref) < TOL
     assert rel_err(got, ref) < 0.1
