@@ -351,13 +351,16 @@ __global__ void __launch_bounds__(fThreads, 1) tc_fused_ffn(const __grid_constan
           float v[32];
           tc::tmem_ld_32x32b_x32(
               tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)((mA + m2) * fBN + c), v);
-          // F(u), or a * F(u) when row_w is set (the combine then only adds rows)
+          // F(u), or a * F(u) when row_w is set (the combine then only adds
+          // rows).  Lane j loads token c + j's weight once; the stores take it
+          // by shuffle, so no load waits behind a store it might alias.
           float* yf = static_cast<float*>(p.y_rows);
+          const float wl = p.row_w && c + lane < n_valid ? p.row_w[tok0 + c + lane] : 1.0f;
 #pragma unroll
-          for (int j = 0; j < 32; ++j)
-            if (c + j < n_valid)
-              yf[(size_t)(tok0 + c + j) * p.width + col] =
-                  p.row_w ? v[j] * p.row_w[tok0 + c + j] : v[j];
+          for (int j = 0; j < 32; ++j) {
+            const float a = __shfl_sync(0xffffffffu, wl, j);
+            if (c + j < n_valid) yf[(size_t)(tok0 + c + j) * p.width + col] = v[j] * a;
+          }
         }
       }
       tc::tc_fence_before();

@@ -434,11 +434,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_grouped_gemm(const __grid_cons
         float v[32];
         tc::tmem_ld_32x32b_x32(t_row + (uint32_t)c, v);
         if (F8 || p.b_scale) {  // row scales of A (E4M3) and of B (E4M3, or combine weights)
+          // lane j loads token c + j's factor once; the others take it by shuffle
+          const float bl = p.b_scale && c + lane < n_valid ? p.b_scale[tok0 + c + lane] : 1.0f;
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const float bs = p.b_scale && c + j < n_valid ? p.b_scale[tok0 + c + j] : 1.0f;
-            v[j] = v[j] * w_scale * bs;
-          }
+          for (int j = 0; j < 32; ++j) v[j] = v[j] * w_scale * __shfl_sync(0xffffffffu, bl, j);
         }
         if (p.mode == MODE_GATEUP) {
 #pragma unroll

@@ -101,7 +101,8 @@ __global__ void __launch_bounds__(256)
   const int lane = threadIdx.x & 31;
   for (int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; t < T;
        t += (gridDim.x * blockDim.x) >> 5) {
-    for (int c = lane; c < width4; c += 32) {
+#pragma unroll 4
+    for (int c = lane; c < width4; c += 32) {  // unrolled: the row loads of 4 steps in flight
       float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
       for (int s = 0; s < k; ++s) {
         const int r = row_of[(size_t)t * k + s];
