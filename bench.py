@@ -603,6 +603,25 @@ class DecodeReplica:
         return sum(t.numel() * t.element_size() for t in self.keep)
 
 
+DECODE_PHASES = ("stage u", "route", "group pairs", "gate/up", "barrier 1", "down",
+                 "barrier 2")
+
+
+def decode_phases(wl, moe, s, rep, out, ws, torch, sm_mhz: float):
+    """Per-layer phase durations (us, median over layers 1..) of one traced
+    decode step: SM-cycle stamps of block 0 converted at the sampled clock."""
+    stamps = torch.zeros((wl.n_layers, 8), dtype=torch.int64, device="cuda")
+    for _ in range(2):  # the second call is warm
+        moe.moe_decode_step_trace(s, rep.layers, rep.u, out, stamps, ws=ws)
+    torch.cuda.synchronize()
+    st = stamps.cpu().numpy().astype(np.float64)
+    cyc = np.diff(st, axis=1)[1:] if wl.n_layers > 1 else np.diff(st, axis=1)
+    per = np.median(cyc, axis=0) / sm_mhz
+    layer = np.median(st[1:, 7] - st[1:, 0] if wl.n_layers > 1 else st[:, 7] - st[:, 0]) / sm_mhz
+    return {"layer_us": float(layer), "sm_mhz": sm_mhz,
+            **{name: float(v) for name, v in zip(DECODE_PHASES, per)}}
+
+
 def decode_main(args, wl, torch, moe, rank, world, dist):
     stream = torch.cuda.current_stream()
     one = DecodeReplica(wl, rank_seed(wl.seed, rank, world), torch, moe)
@@ -675,6 +694,8 @@ def decode_main(args, wl, torch, moe, rank, world, dist):
     eb.record(stream)
     torch.cuda.synchronize()
     e_ms = max_over_ranks(ea.elapsed_time(eb), dist, "cuda")
+    phases = decode_phases(wl, moe, s, reps[0], out, ws, torch,
+                           (clocks or {}).get("sm_mhz") or 1965.0)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, el_s, n = decode_cpu_baseline(wl)
@@ -698,6 +719,7 @@ def decode_main(args, wl, torch, moe, rank, world, dist):
                              "frac": achieved / hbm, "traffic": None,
                              "kernel": "decode_persistent: all layers of the step in one "
                                        "cooperative launch",
+                             "phases_us": phases,
                              "bytes_per_step": bytes_timed / args.steps,
                              "peak_source": f"{src} hbm_gbs",
                              "frac_of_spec": achieved / SPEC_HBM_GBS},

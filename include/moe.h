@@ -463,6 +463,18 @@ MOE_API int moe_decode_step(const moe_shape* shape, int32_t n_layers, const moe_
                             const uint16_t* u0, uint16_t* u_out, int32_t* top_idx_all, void* ws,
                             size_t ws_bytes, void* stream);
 
+/* moe_decode_step that also records, for each layer, eight SM-cycle stamps
+ * (clock64 of block 0, thread 0) into stamps [n_layers][8] (device memory,
+ * 8-byte aligned; caller-owned): layer start, input rows staged, routed,
+ * dispatch pairs grouped by expert, gate/up phase done, first grid barrier
+ * passed, down phase done, second grid barrier passed.  Differences are
+ * cycles of that SM's clock; results are identical to moe_decode_step.
+ * MOE_ERR_INVALID_ARG for a null or misaligned stamps pointer. */
+MOE_API int moe_decode_step_trace(const moe_shape* shape, int32_t n_layers,
+                                  const moe_q4_layer* layers, const uint16_t* u0, uint16_t* u_out,
+                                  int32_t* top_idx_all, void* ws, size_t ws_bytes,
+                                  uint64_t* stamps, void* stream);
+
 /* ---------------------------------------------------- quantile balancing */
 /* Quantile balancing of the expert biases ("Stable LatentMoE interactive demo
  * document", Quantile Balancing).  scores [T][N] fp32 are the router logits,

@@ -120,6 +120,8 @@ _PROTOS = {
                                 _vp, _sz, _vp]),
     "moe_decode_step": (_i32, [_P_SHAPE, _i32, ctypes.POINTER(MoeQ4Layer), _vp, _vp, _vp, _vp,
                                _sz, _vp]),
+    "moe_decode_step_trace": (_i32, [_P_SHAPE, _i32, ctypes.POINTER(MoeQ4Layer), _vp, _vp, _vp,
+                                     _vp, _sz, _vp, _vp]),
     "moe_aux_grad": (_i32, [_i32, _i32, _f32, _vp, _vp, _vp, _vp]),
     "moe_quantile_balance_workspace_bytes": (_sz, [_i32, _i32]),
     "moe_quantile_balance": (_i32, [_i32, _i32, _i32, _vp, _vp, _i32, _i32, _vp, _vp, _vp, _vp,
@@ -555,6 +557,21 @@ def moe_decode_step(s: MoeShape, layers, u0, u_out, top_idx_all=None, ws=None, s
     _check(_lib.moe_decode_step(ctypes.byref(s), len(layers), arr, _ptr(u0), _ptr(u_out),
                                 _ptr(top_idx_all), _ptr(wbuf), wlen, _stream(stream)),
            "moe_decode_step")
+
+
+def moe_decode_step_trace(s: MoeShape, layers, u0, u_out, stamps, top_idx_all=None, ws=None,
+                          stream=None):
+    """moe_decode_step plus per-layer phase stamps: stamps is an int64 device
+    tensor of at least 8 * len(layers) elements (SM cycles, see moe.h)."""
+    for args in (("u0", u0, s.T * s.d, _F16), ("u_out", u_out, s.T * s.d, _F16),
+                 ("top_idx_all", top_idx_all, len(layers) * s.T * s.k, _I32),
+                 ("stamps", stamps, 8 * len(layers), "int64")):
+        _need(*args)
+    arr = (MoeQ4Layer * len(layers))(*layers)
+    wbuf, wlen = _ws(moe_decode_workspace_bytes(s), u0.device, ws)
+    _check(_lib.moe_decode_step_trace(ctypes.byref(s), len(layers), arr, _ptr(u0), _ptr(u_out),
+                                      _ptr(top_idx_all), _ptr(wbuf), wlen, _ptr(stamps),
+                                      _stream(stream)), "moe_decode_step_trace")
 
 
 def moe_aux_grad(probs, f, dz, alpha: float = 1.0, stream=None):

@@ -322,7 +322,18 @@ struct Params {
   float* H;             // [N][T][h] fp32 scratch
   unsigned* bar;        // [0] arrivals, [1] abort
   int* status;
+  unsigned long long* stamps;  // nullable: [n_layers][kStamps] SM cycle stamps of CTA 0
 };
+
+// Phase boundaries stamped per layer when a trace buffer is given: layer
+// start, input staged, routed, pairs grouped, phase A done, first barrier
+// passed, phase B done, second barrier passed.
+constexpr int kStamps = 8;
+
+__device__ __forceinline__ void stamp(const Params& p, int l, int i) {
+  if (p.stamps && blockIdx.x == 0 && threadIdx.x == 0)
+    p.stamps[(size_t)l * kStamps + i] = clock64();
+}
 
 uint32_t take(uint32_t& off, size_t bytes) {
   const uint32_t o = off;
@@ -411,6 +422,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_persistent(const __grid_co
     const bool last = l == p.n_layers - 1;
     const __half* u_cur = l == 0 ? p.u_in : p.u_work;
     __half* u_next = last ? p.u_out : p.u_work;
+    stamp(p, l, 0);
     float* wr_s = reinterpret_cast<float*>(sm + ((l & 1) && P.nbuf == 2 ? P.wr1 : P.wr0));
     if (l > 0 && P.nbuf == 1)
       stage_rows(reinterpret_cast<char*>(wr_s), ws_ld * 4,
@@ -420,9 +432,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_persistent(const __grid_co
     for (int e = tid; e < N; e += blockDim.x) cnt[e] = 0;
     cp_wait_all();
     __syncthreads();
+    stamp(p, l, 1);
 
     // ---- routing (every CTA), then the pairs grouped by expert
     route_in_cta(u_s, us_ld, wr_s, ws_ld, T, d, N, k, p.renorm, L.bias, z, sel, aw);
+    stamp(p, l, 2);
     if (b == 0) {
       for (int x = tid; x < Tk; x += blockDim.x) {
         if (p.top_idx) p.top_idx[(size_t)l * Tk + x] = sel[x];
@@ -492,6 +506,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_persistent(const __grid_co
       }
     };
     __syncthreads();  // list complete before the item loop reads it
+    stamp(p, l, 3);
     if (b < nitems) stage_item(b);
     if (b < nslices) stage_slice(b);
     // When the batch dispatches at least as many pairs as there are experts
@@ -602,6 +617,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_persistent(const __grid_co
         p.H[((size_t)e * T + toks[i]) * h + (size_t)sl * RA + r] = silu(g) * vu;
       }
     }
+    stamp(p, l, 4);
     grid_arrive(p.bar);
     if (P.nbuf == 2 && !last)  // next layer's router rows, while the barrier completes
       stage_rows(sm + ((l & 1) ? P.wr0 : P.wr1), ws_ld * 4,
@@ -610,6 +626,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_persistent(const __grid_co
       cp_wait_all();
       return;
     }
+    stamp(p, l, 5);
 
     // ---- phase B: y = sum_s a_s W_down[e_s] H_s, u_next = fp16(u + y)
     for (int sl = b; sl < nslices; sl += G) {
@@ -678,11 +695,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_persistent(const __grid_co
       }
       __syncthreads();
     }
+    stamp(p, l, 6);
     grid_arrive(p.bar);
     if (!grid_wait(p.bar, (unsigned)G * ++n_bar, p.status)) {
       cp_wait_all();
       return;
     }
+    stamp(p, l, 7);
   }
 }
 
@@ -759,7 +778,7 @@ LayerPtrs layer_ptrs(const moe_q4_layer& L) {
 // One cooperative launch over layers [0, n) of `layers`.
 int launch_decode(const moe_shape& s, const moe_q4_layer* layers, int n, const __half* u_in,
                   __half* u_out, __half* y, int32_t* top_idx, float* top_w, const WsLayout& W,
-                  cudaStream_t st) {
+                  cudaStream_t st, unsigned long long* stamps = nullptr) {
   int sms = 0;
   if (!device_info(&sms)) return MOE_ERR_CUDA;
   Params p{};
@@ -789,6 +808,7 @@ int launch_decode(const moe_shape& s, const moe_q4_layer* layers, int n, const _
   p.H = W.H;
   p.bar = W.bar;
   p.status = status_word();
+  p.stamps = stamps;
   if (cudaMemsetAsync(W.bar, 0, 4 * sizeof(unsigned), st) != cudaSuccess) return MOE_ERR_CUDA;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
@@ -827,9 +847,10 @@ extern "C" int moe_decode_layer(const moe_shape* shape, const moe_q4_layer* laye
                        top_idx ? top_idx : W.idx, top_w ? top_w : W.w, W, as_stream(stream));
 }
 
-extern "C" int moe_decode_step(const moe_shape* shape, int32_t n_layers,
-                               const moe_q4_layer* layers, const uint16_t* u0, uint16_t* u_out,
-                               int32_t* top_idx_all, void* ws, size_t ws_bytes, void* stream) {
+namespace {
+int decode_step(const moe_shape* shape, int32_t n_layers, const moe_q4_layer* layers,
+                const uint16_t* u0, uint16_t* u_out, int32_t* top_idx_all, void* ws,
+                size_t ws_bytes, void* stream, uint64_t* stamps) {
   using namespace moe;
   if (!decode_shape_ok(shape) || n_layers <= 0 || !layers) return MOE_ERR_INVALID_ARG;
   for (int l = 0; l < n_layers; ++l)
@@ -847,9 +868,28 @@ extern "C" int moe_decode_step(const moe_shape* shape, int32_t n_layers,
     const bool last_chunk = l0 + n == n_layers;
     const __half* in = l0 == 0 ? reinterpret_cast<const __half*>(u0) : W.work;
     __half* out = last_chunk ? reinterpret_cast<__half*>(u_out) : W.work;
-    const int rc = launch_decode(s, layers + l0, n, in, out, nullptr,
-                                 top_idx_all ? top_idx_all + l0 * Tk : nullptr, nullptr, W, st);
+    const int rc = launch_decode(
+        s, layers + l0, n, in, out, nullptr, top_idx_all ? top_idx_all + l0 * Tk : nullptr,
+        nullptr, W, st,
+        stamps ? reinterpret_cast<unsigned long long*>(stamps) + (size_t)l0 * kStamps : nullptr);
     if (rc != MOE_OK) return rc;
   }
   return MOE_OK;
+}
+}  // namespace
+
+extern "C" int moe_decode_step(const moe_shape* shape, int32_t n_layers,
+                               const moe_q4_layer* layers, const uint16_t* u0, uint16_t* u_out,
+                               int32_t* top_idx_all, void* ws, size_t ws_bytes, void* stream) {
+  return decode_step(shape, n_layers, layers, u0, u_out, top_idx_all, ws, ws_bytes, stream,
+                     nullptr);
+}
+
+extern "C" int moe_decode_step_trace(const moe_shape* shape, int32_t n_layers,
+                                     const moe_q4_layer* layers, const uint16_t* u0,
+                                     uint16_t* u_out, int32_t* top_idx_all, void* ws,
+                                     size_t ws_bytes, uint64_t* stamps, void* stream) {
+  if (!stamps || (reinterpret_cast<uintptr_t>(stamps) & 7u)) return MOE_ERR_INVALID_ARG;
+  return decode_step(shape, n_layers, layers, u0, u_out, top_idx_all, ws, ws_bytes, stream,
+                     stamps);
 }

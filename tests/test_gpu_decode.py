@@ -203,6 +203,32 @@ def test_decode_step_chunks_and_graph_replay():
         assert np.array_equal(_codes(out2), _codes(out))
 
 
+def test_decode_step_trace_matches_and_stamps_phases():
+    """The traced step (40 layers, two launches) gives the same output and
+    routing as moe_decode_step, and each layer's eight phase stamps are
+    non-decreasing SM cycle counts (block 0 stays on one SM)."""
+    wl = W.decode(T=8, n_layers=40)
+    layers = [Layer(wl, l) for l in range(wl.n_layers)]
+    s = moe.shape(wl.T, wl.d, wl.N, wl.k, wl.h, 1, 0)
+    u0 = _f16(_u0(wl))
+    abis = [L.abi for L in layers]
+    out, out_t = torch.empty_like(u0), torch.empty_like(u0)
+    idx, idx_t = (torch.empty((wl.n_layers, wl.T, wl.k), dtype=torch.int32, device="cuda")
+                  for _ in range(2))
+    moe.moe_decode_step(s, abis, u0, out, idx)
+    stamps = torch.zeros((wl.n_layers, 8), dtype=torch.int64, device="cuda")
+    moe.moe_decode_step_trace(s, abis, u0, out_t, stamps, idx_t)
+    torch.cuda.synchronize()
+    assert np.array_equal(_codes(out), _codes(out_t))
+    assert torch.equal(idx, idx_t)
+    st = stamps.cpu().numpy()
+    assert np.all(st > 0)
+    assert np.all(np.diff(st, axis=1) >= 0)
+    assert np.all(st[1:32, 0] >= st[:31, 7])  # layers of one launch follow each other
+    with pytest.raises(ValueError):
+        moe.moe_decode_step_trace(s, abis, u0, out_t, stamps[:4], idx_t)
+
+
 def test_decode_empty_batch():
     """T = 0: both decode entry points succeed and launch nothing."""
     wl = W.decode(T=1, n_layers=2)
