@@ -4,9 +4,9 @@ beta_g * beta_u = 100 < 448, the E4M3 maximum) against the CPU oracle's FP8
 form, through the C ABI.
 
 The row quantiser must match the oracle's bit for bit (its decisions are taken
-on the same fp32 quotients).  The grouped E4M3 FFN is compared within the
-bf16 bound, max|d|/rms <= 2e-2, and its H codes one by one (a code may differ
-only where H lies at a rounding midpoint).  The layer's x_l = bf16(W_dp x)
+on the same fp32 quotients).  The grouped E4M3 FFN's H codes are compared
+one by one (a code may differ only where H lies at a rounding midpoint), its
+rows with matching codes within the bf16 bound, max|d|/rms <= 2e-2.  The layer's x_l = bf16(W_dp x)
 comes from an fp32 tensor-core GEMM, so a last-place bf16 difference from the
 oracle's x_l can move a token's E4M3 scale (its amax) and with it every code
 of that token: the layer outputs are compared by relative Frobenius error
@@ -106,8 +106,11 @@ def test_expert_ffn_e4m3_vs_oracle(case):
     neighbour of the oracle's and the exact H lies within 2^-9 (of |H|, or of
     rms(H) where H is smaller) of the midpoint between them; the fp32 rows
     equal W_down times the kernel's own H codes within 1e-5 of rms (the E4M3
-    MMA accumulates in fp32); and the rows match the oracle within the bf16
-    bound, max|d|/rms <= 2e-2."""
+    MMA accumulates in fp32); and the rows whose H codes all equal the
+    oracle's match the oracle's rows within the bf16 bound, max|d|/rms <=
+    2e-2.  (One neighbouring code of a large H element in a 128-wide expert
+    moves its row by up to ~0.1 of rms, so rows with a flip are held to the
+    two checks before instead.)"""
     width, h, counts, kind = FFN_CASES[case]
     N, R = len(counts), int(sum(counts))
     (xc, xs), mats = _ffn_inputs(width, h, counts, seed=77 + width + h)
@@ -174,9 +177,15 @@ def _check_e4m3_ffn(act_kind, width, h, offs, xc, xs, mats, got_y, got_h):
         # scales with the terms of the sum, not with a small (cancelled) result
         off = np.abs(hx - mid) / np.maximum(np.abs(hx), np.sqrt(np.mean(exact_h ** 2)))
         assert off.max() <= 2.0 ** -9, f"a differing code {off.max():.2e} away from a midpoint"
-    down_err, err = rel_err(got_y, chk_y), rel_err(got_y, ref_y)
-    print(f"H values differing {diff.mean():.4%}, down GEMM vs own H {down_err:.2e}, "
-          f"rows vs oracle {err:.2e} (max|d|/rms)")
+    # rows whose H codes all equal the oracle's: the bf16 bound against the
+    # oracle; a row with a (validated) neighbouring code is fixed by the
+    # check against W_down times the kernel's own codes
+    clean = ~diff.any(axis=1)
+    rms = float(np.sqrt(np.mean(ref_y ** 2)))
+    down_err = rel_err(got_y, chk_y)
+    err = float(np.max(np.abs(got_y[clean] - ref_y[clean]), initial=0.0)) / rms
+    print(f"H values differing {diff.mean():.4%} ({int((~clean).sum())} of {len(clean)} rows), "
+          f"down GEMM vs own H {down_err:.2e}, clean rows vs oracle {err:.2e} (max|d|/rms)")
     assert down_err <= 1e-5, "down GEMM against the kernel's own H codes"
     assert err <= TOL
 
