@@ -28,6 +28,9 @@ namespace {
 
 constexpr int fBM = 128, fBK = 64, fBN = 64, fS = 7, fThreads = 192, fEpiLd = 33;
 constexpr int fHMax = 256;
+// mbarriers after the stage ring: a_done per hidden slice (h / 64 <= 4),
+// h_ready, b_done per output slice (width / 128 <= 8), b_free, drain
+constexpr int kMaxA = fHMax / 64, kMaxB = 8, kBars = kMaxA + 1 + kMaxB + 2;
 constexpr long long fWaitBudget = 4000000000LL;
 
 struct FusedParams {
@@ -49,11 +52,11 @@ struct FLayout {
   static constexpr int X_BYTES = fBN * fBK * 2;  // 8 KB
   static constexpr int STAGE = A_BYTES + X_BYTES;
   static constexpr int H_BYTES = fBN * fHMax * 2;  // 32 KB
-  static constexpr int EPI_BYTES = fBM * fEpiLd * 4;
+  static constexpr int EPI_BYTES = fBM * fEpiLd * 4 + fBN * 4;  // exchange tile + row weights
   static size_t bytes(int G) {
     size_t b = 1024 + (size_t)fS * STAGE + H_BYTES + EPI_BYTES + (size_t)3 * (G + 1) * 4;
     b = align_up(b, 8);
-    b += (size_t)(2 * fS + 5) * 8 + 16;
+    b += (size_t)(2 * fS + kBars) * 8 + 16;
     return b;
   }
 };
@@ -80,19 +83,20 @@ __global__ void __launch_bounds__(fThreads, 1) tc_fused_ffn(const __grid_constan
   uint8_t* stages = smem;
   uint8_t* hs = smem + fS * L::STAGE;  // H tile, 1024-aligned (fS * STAGE is)
   float* epi = reinterpret_cast<float*>(hs + L::H_BYTES);
-  int* grp_beg = reinterpret_cast<int*>(epi + fBM * fEpiLd);
+  float* fac = epi + fBM * fEpiLd;  // [fBN] the tile's combine weights
+  int* grp_beg = reinterpret_cast<int*>(fac + fBN);
   int* grp_cnt = grp_beg + (p.G + 1);
   int* grp_pre = grp_cnt + (p.G + 1);
   uint64_t* bars = reinterpret_cast<uint64_t*>(
       (reinterpret_cast<uintptr_t>(grp_pre + p.G + 1) + 7) & ~static_cast<uintptr_t>(7));
   uint64_t* full = bars;
   uint64_t* empty = bars + fS;
-  uint64_t* a_done = bars + 2 * fS;
-  uint64_t* h_ready = a_done + 1;
-  uint64_t* b_done = a_done + 2;
-  uint64_t* b_free = a_done + 3;
-  uint64_t* drain = a_done + 4;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * fS + 5);
+  uint64_t* a_done = bars + 2 * fS;  // [kMaxA]: slice m's gate/up accumulators ready
+  uint64_t* h_ready = a_done + kMaxA;
+  uint64_t* b_done = h_ready + 1;    // [kMaxB]: output slice m2's accumulator ready
+  uint64_t* b_free = b_done + kMaxB;
+  uint64_t* drain = b_free + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * fS + kBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -102,9 +106,9 @@ __global__ void __launch_bounds__(fThreads, 1) tc_fused_ffn(const __grid_constan
       tc::mbar_init(tc::smem_u32(&full[s]), 1);
       tc::mbar_init(tc::smem_u32(&empty[s]), 1);
     }
-    tc::mbar_init(tc::smem_u32(a_done), 1);
+    for (int i = 0; i < kMaxA; ++i) tc::mbar_init(tc::smem_u32(&a_done[i]), 1);
     tc::mbar_init(tc::smem_u32(h_ready), 128);
-    tc::mbar_init(tc::smem_u32(b_done), 1);
+    for (int i = 0; i < kMaxB; ++i) tc::mbar_init(tc::smem_u32(&b_done[i]), 1);
     tc::mbar_init(tc::smem_u32(b_free), 128);
     tc::mbar_init(tc::smem_u32(drain), 1);
     tc::fence_barrier_init();
@@ -247,9 +251,10 @@ __global__ void __launch_bounds__(fThreads, 1) tc_fused_ffn(const __grid_constan
               phase ^= 1u;
             }
           }
+          // slice m's accumulator: its epilogue overlaps the next slice's MMAs
+          if (ok) tc::mma_commit(tc::smem_u32(&a_done[m]));
         }
         if (!ok) break;
-        tc::mma_commit(tc::smem_u32(a_done));
         if (!tc::mbar_wait(tc::smem_u32(h_ready), par, abort_flag, fWaitBudget) ||
             !tc::mbar_wait(tc::smem_u32(b_free), par ^ 1u, abort_flag, fWaitBudget)) {
           ok = false;
@@ -276,9 +281,9 @@ __global__ void __launch_bounds__(fThreads, 1) tc_fused_ffn(const __grid_constan
               phase ^= 1u;
             }
           }
+          if (ok) tc::mma_commit(tc::smem_u32(&b_done[m2]));
         }
         if (!ok) break;
-        tc::mma_commit(tc::smem_u32(b_done));
       }
       if (!ok) {
         record_error(p.status, MOE_ERR_TIMEOUT);
@@ -298,14 +303,21 @@ __global__ void __launch_bounds__(fThreads, 1) tc_fused_ffn(const __grid_constan
       const int n_valid = min(fBN, grp_cnt[g] - n * fBN);
       const int tok0 = grp_beg[g] + n * fBN;
       const uint32_t par = (uint32_t)(it & 1);
-      if (!all_epi_ok(tc::mbar_wait(tc::smem_u32(a_done), par, abort_flag, fWaitBudget))) {
-        record_error(p.status, MOE_ERR_TIMEOUT);
-        *abort_flag = 1;
-        break;
+      bool ok = true;
+      // the tile's combine weights, fetched while phase A runs, once every
+      // epilogue warp is done with the previous tile's (the named barriers
+      // of epilogue A publish them before epilogue B reads them)
+      if (p.row_w) {
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        for (int i = row; i < fBN; i += 128) fac[i] = i < n_valid ? p.row_w[tok0 + i] : 1.0f;
       }
-      tc::tc_fence_after();
       // H = act(gate, up) -> bf16 into the swizzled K-major tile (k-block m)
-      for (int m = 0; m < mA; ++m) {
+      for (int m = 0; m < mA && ok; ++m) {
+        if (!all_epi_ok(tc::mbar_wait(tc::smem_u32(&a_done[m]), par, abort_flag, fWaitBudget))) {
+          ok = false;
+          break;
+        }
+        tc::tc_fence_after();
         for (int c = 0; c < fBN; c += 32) {
           float v[32];
           tc::tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(m * fBN + c),
@@ -335,33 +347,40 @@ __global__ void __launch_bounds__(fThreads, 1) tc_fused_ffn(const __grid_constan
           asm volatile("bar.sync 1, 128;" ::: "memory");
         }
       }
-      // make the generic-proxy stores visible to the tensor core, then hand over
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      tc::tc_fence_before();
-      tc::mbar_arrive(tc::smem_u32(h_ready));
-      if (!all_epi_ok(tc::mbar_wait(tc::smem_u32(b_done), par, abort_flag, fWaitBudget))) {
+      if (!ok) {
         record_error(p.status, MOE_ERR_TIMEOUT);
         *abort_flag = 1;
         break;
       }
-      tc::tc_fence_after();
+      // make the generic-proxy stores visible to the tensor core, then hand over
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      tc::tc_fence_before();
+      tc::mbar_arrive(tc::smem_u32(h_ready));
       for (int m2 = 0; m2 < mB; ++m2) {
+        // output slice m2's accumulator: stored while later slices' MMAs run
+        if (!all_epi_ok(tc::mbar_wait(tc::smem_u32(&b_done[m2]), par, abort_flag, fWaitBudget))) {
+          ok = false;
+          break;
+        }
+        tc::tc_fence_after();
         const int col = m2 * fBM + row;
         for (int c = 0; c < n_valid; c += 32) {
           float v[32];
           tc::tmem_ld_32x32b_x32(
               tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)((mA + m2) * fBN + c), v);
           // F(u), or a * F(u) when row_w is set (the combine then only adds
-          // rows).  Lane j loads token c + j's weight once; the stores take it
-          // by shuffle, so no load waits behind a store it might alias.
+          // rows); the weights were staged in shared memory at the tile start
           float* yf = static_cast<float*>(p.y_rows);
-          const float wl = p.row_w && c + lane < n_valid ? p.row_w[tok0 + c + lane] : 1.0f;
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const float a = __shfl_sync(0xffffffffu, wl, j);
-            if (c + j < n_valid) yf[(size_t)(tok0 + c + j) * p.width + col] = v[j] * a;
-          }
+          for (int j = 0; j < 32; ++j)
+            if (c + j < n_valid)
+              yf[(size_t)(tok0 + c + j) * p.width + col] = p.row_w ? v[j] * fac[c + j] : v[j];
         }
+      }
+      if (!ok) {
+        record_error(p.status, MOE_ERR_TIMEOUT);
+        *abort_flag = 1;
+        break;
       }
       tc::tc_fence_before();
       tc::mbar_arrive(tc::smem_u32(b_free));

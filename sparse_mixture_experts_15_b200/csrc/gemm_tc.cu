@@ -105,7 +105,7 @@ struct Layout {
   static constexpr int A_BYTES = kBM * kBK * 2;
   static constexpr int B_BYTES = BN / CG * kBK * 2;  // this CTA's token rows
   static constexpr int STAGE = A_BYTES + B_BYTES;
-  static constexpr int EPI_BYTES = kBM * kEpiLd * 4;
+  static constexpr int EPI_BYTES = kBM * kEpiLd * 4 + BN * 4;  // exchange tile + token factors
   static size_t bytes(int G) {
     size_t b = 1024;  // alignment slack of the dynamic smem base
     b += (size_t)S * STAGE + EPI_BYTES;
@@ -134,7 +134,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_grouped_gemm(const __grid_cons
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* stages = smem;
   float* epi = reinterpret_cast<float*>(smem + S * L::STAGE);
-  int* grp_beg = reinterpret_cast<int*>(epi + kBM * kEpiLd);
+  float* fac = epi + kBM * kEpiLd;  // [BN] the tile's token-row factors (b_scale)
+  int* grp_beg = reinterpret_cast<int*>(fac + BN);
   int* grp_cnt = grp_beg + (p.G + 1);
   int* grp_pre = grp_cnt + (p.G + 1);
   uint64_t* bars = reinterpret_cast<uint64_t*>(
@@ -400,8 +401,14 @@ __global__ void __launch_bounds__(kThreads, 1) tc_grouped_gemm(const __grid_cons
       const int tok0 = grp_beg[g] + n * BN;
       const int b = it & 1;
       const uint32_t use = (uint32_t)(it >> 1);
+      // the tile's token-row factors, fetched while the accumulator is being
+      // computed, once every epilogue warp is done with the previous tile's
+      if (p.b_scale) {
+        named_sync_epi();
+        for (int i = row; i < BN; i += 128) fac[i] = i < n_valid ? p.b_scale[tok0 + i] : 1.0f;
+      }
       // The four epilogue warps share named barriers, so they take the
-      // give-up decision together.
+      // give-up decision together (the barrier also publishes fac).
       const bool got = tc::mbar_wait(tc::smem_u32(&tfull[b]), use & 1u, abort_flag, kWaitBudget);
       uint32_t all_ok;
       asm volatile(
@@ -434,10 +441,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_grouped_gemm(const __grid_cons
         float v[32];
         tc::tmem_ld_32x32b_x32(t_row + (uint32_t)c, v);
         if (F8 || p.b_scale) {  // row scales of A (E4M3) and of B (E4M3, or combine weights)
-          // lane j loads token c + j's factor once; the others take it by shuffle
-          const float bl = p.b_scale && c + lane < n_valid ? p.b_scale[tok0 + c + lane] : 1.0f;
 #pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] = v[j] * w_scale * __shfl_sync(0xffffffffu, bl, j);
+          for (int j = 0; j < 32; ++j) v[j] = v[j] * w_scale * (p.b_scale ? fac[c + j] : 1.0f);
         }
         if (p.mode == MODE_GATEUP) {
 #pragma unroll
