@@ -603,21 +603,22 @@ class DecodeReplica:
         return sum(t.numel() * t.element_size() for t in self.keep)
 
 
-DECODE_PHASES = ("stage u", "route", "group pairs", "gate/up", "barrier 1", "down",
-                 "barrier 2")
+DECODE_PHASES = ("stage u", "route", "group pairs", "stage gate/up rows", "dequantise",
+                 "gate/up dots", "H store", "barrier 1", "down rows ready", "down dots",
+                 "combine + u_next", "barrier 2")
 
 
 def decode_phases(wl, moe, s, rep, out, ws, torch, sm_mhz: float):
     """Per-layer phase durations (us, median over layers 1..) of one traced
     decode step: SM-cycle stamps of block 0 converted at the sampled clock."""
-    stamps = torch.zeros((wl.n_layers, 8), dtype=torch.int64, device="cuda")
+    stamps = torch.zeros((wl.n_layers, moe.DECODE_STAMPS), dtype=torch.int64, device="cuda")
     for _ in range(2):  # the second call is warm
         moe.moe_decode_step_trace(s, rep.layers, rep.u, out, stamps, ws=ws)
     torch.cuda.synchronize()
     st = stamps.cpu().numpy().astype(np.float64)
     cyc = np.diff(st, axis=1)[1:] if wl.n_layers > 1 else np.diff(st, axis=1)
     per = np.median(cyc, axis=0) / sm_mhz
-    layer = np.median(st[1:, 7] - st[1:, 0] if wl.n_layers > 1 else st[:, 7] - st[:, 0]) / sm_mhz
+    layer = np.median(st[1:, -1] - st[1:, 0] if wl.n_layers > 1 else st[:, -1] - st[:, 0]) / sm_mhz
     return {"layer_us": float(layer), "sm_mhz": sm_mhz,
             **{name: float(v) for name, v in zip(DECODE_PHASES, per)}}
 

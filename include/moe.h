@@ -463,12 +463,16 @@ MOE_API int moe_decode_step(const moe_shape* shape, int32_t n_layers, const moe_
                             const uint16_t* u0, uint16_t* u_out, int32_t* top_idx_all, void* ws,
                             size_t ws_bytes, void* stream);
 
-/* moe_decode_step that also records, for each layer, eight SM-cycle stamps
- * (clock64 of block 0, thread 0) into stamps [n_layers][8] (device memory,
- * 8-byte aligned; caller-owned): layer start, input rows staged, routed,
- * dispatch pairs grouped by expert, gate/up phase done, first grid barrier
- * passed, down phase done, second grid barrier passed.  Differences are
- * cycles of that SM's clock; results are identical to moe_decode_step.
+/* moe_decode_step that also records, for each layer, 13 SM-cycle stamps
+ * (clock64 of block 0, thread 0) into stamps [n_layers][13] (device memory,
+ * 8-byte aligned; caller-owned): 0 layer start, 1 input rows staged,
+ * 2 routed, 3 dispatch pairs grouped by expert, 4 gate/up q4 rows staged,
+ * 5 dequantised, 6 gate/up dots formed, 7 gate/up phase done (H stored),
+ * 8 first grid barrier passed, 9 down rows ready, 10 down dots formed,
+ * 11 down phase done (u_next stored), 12 second grid barrier passed.
+ * Stamps 4-6 and 9-10 time block 0's first item and slice (equal to 7 and 11
+ * when it has none).  Differences are cycles of that SM's clock; results are
+ * identical to moe_decode_step.
  * MOE_ERR_INVALID_ARG for a null or misaligned stamps pointer. */
 MOE_API int moe_decode_step_trace(const moe_shape* shape, int32_t n_layers,
                                   const moe_q4_layer* layers, const uint16_t* u0, uint16_t* u_out,

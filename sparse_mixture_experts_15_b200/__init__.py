@@ -559,13 +559,17 @@ def moe_decode_step(s: MoeShape, layers, u0, u_out, top_idx_all=None, ws=None, s
            "moe_decode_step")
 
 
+DECODE_STAMPS = 13  # phase stamps per layer of moe_decode_step_trace
+
+
 def moe_decode_step_trace(s: MoeShape, layers, u0, u_out, stamps, top_idx_all=None, ws=None,
                           stream=None):
     """moe_decode_step plus per-layer phase stamps: stamps is an int64 device
-    tensor of at least 8 * len(layers) elements (SM cycles, see moe.h)."""
+    tensor of at least DECODE_STAMPS * len(layers) elements (SM cycles, see
+    moe.h)."""
     for args in (("u0", u0, s.T * s.d, _F16), ("u_out", u_out, s.T * s.d, _F16),
                  ("top_idx_all", top_idx_all, len(layers) * s.T * s.k, _I32),
-                 ("stamps", stamps, 8 * len(layers), "int64")):
+                 ("stamps", stamps, DECODE_STAMPS * len(layers), "int64")):
         _need(*args)
     arr = (MoeQ4Layer * len(layers))(*layers)
     wbuf, wlen = _ws(moe_decode_workspace_bytes(s), u0.device, ws)

@@ -325,10 +325,13 @@ struct Params {
   unsigned long long* stamps;  // nullable: [n_layers][kStamps] SM cycle stamps of CTA 0
 };
 
-// Phase boundaries stamped per layer when a trace buffer is given: layer
-// start, input staged, routed, pairs grouped, phase A done, first barrier
-// passed, phase B done, second barrier passed.
-constexpr int kStamps = 8;
+// Phase boundaries stamped per layer when a trace buffer is given: 0 layer
+// start, 1 input staged, 2 routed, 3 pairs grouped, 4 gate/up rows staged,
+// 5 dequantised, 6 dots formed, 7 phase A done (H stored), 8 first barrier
+// passed, 9 down rows ready, 10 down dots formed, 11 phase B done (u_next
+// stored), 12 second barrier passed.  Stamps 4-6 and 9-10 are block 0's
+// first item / slice (taken at 7 and 11 when it has none).
+constexpr int kStamps = 13;
 
 __device__ __forceinline__ void stamp(const Params& p, int l, int i) {
   if (p.stamps && blockIdx.x == 0 && threadIdx.x == 0)
@@ -541,6 +544,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_persistent(const __grid_co
       if (it != b) stage_item(it);
       cp_wait_all();
       __syncthreads();
+      if (it == b) stamp(p, l, 4);
       for (int x = tid; x < 2 * RA * nb * 8; x += blockDim.x) {  // 8 threads per block
         const int blk = x >> 3, c = x & 7;
         const int w = blk / nb, bb = blk - w * nb;
@@ -548,6 +552,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_persistent(const __grid_co
             dequant_quad(aq + (size_t)w * (d / 2) + bb * 16, as[w * nb + bb], c);
       }
       __syncthreads();
+      if (it == b) stamp(p, l, 5);
       // unit = (token pair, hidden row r, part of d): one thread forms the
       // gate and the up dot of row r for two tokens, so each weight and
       // activation it loads feeds two FMAs.  d is split into nparts so that
@@ -605,6 +610,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_persistent(const __grid_co
         }
       }
       __syncthreads();
+      if (it == b) stamp(p, l, 6);
       for (int v = tid; v < RA * ne; v += blockDim.x) {
         const int i = v / RA, r = v - i * RA;
         const float* pr = part + (size_t)(r * ne + i) * nparts * 2;
@@ -617,7 +623,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_persistent(const __grid_co
         p.H[((size_t)e * T + toks[i]) * h + (size_t)sl * RA + r] = silu(g) * vu;
       }
     }
-    stamp(p, l, 4);
+    if (b >= nitems)
+      for (int i = 4; i < 7; ++i) stamp(p, l, i);
+    stamp(p, l, 7);
     grid_arrive(p.bar);
     if (P.nbuf == 2 && !last)  // next layer's router rows, while the barrier completes
       stage_rows(sm + ((l & 1) ? P.wr0 : P.wr1), ws_ld * 4,
@@ -626,13 +634,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_persistent(const __grid_co
       cp_wait_all();
       return;
     }
-    stamp(p, l, 5);
+    stamp(p, l, 8);
 
     // ---- phase B: y = sum_s a_s W_down[e_s] H_s, u_next = fp16(u + y)
     for (int sl = b; sl < nslices; sl += G) {
       if (sl != b) stage_slice(sl);
       cp_wait_all();
       __syncthreads();
+      if (sl == b) stamp(p, l, 9);
       // unit = (pair x, row group g, q4 block pp), pp fastest so a pair's
       // nbh partial dots sit in adjacent lanes; the rows of a slice are split
       // into rgroups groups when there are few pairs, so more threads work.
@@ -683,6 +692,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_persistent(const __grid_co
         }
       }
       __syncthreads();
+      if (sl == b) stamp(p, l, 10);
       for (int v = tid; v < T * RB; v += blockDim.x) {
         const int t = v / RB, r = v - t * RB;
         float acc = 0.0f;
@@ -695,13 +705,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_persistent(const __grid_co
       }
       __syncthreads();
     }
-    stamp(p, l, 6);
+    if (b >= nslices)
+      for (int i = 9; i < 11; ++i) stamp(p, l, i);
+    stamp(p, l, 11);
     grid_arrive(p.bar);
     if (!grid_wait(p.bar, (unsigned)G * ++n_bar, p.status)) {
       cp_wait_all();
       return;
     }
-    stamp(p, l, 7);
+    stamp(p, l, 12);
   }
 }
 
