@@ -369,12 +369,18 @@ __global__ void __launch_bounds__(fThreads, 1) tc_fused_ffn(const __grid_constan
           tc::tmem_ld_32x32b_x32(
               tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)((mA + m2) * fBN + c), v);
           // F(u), or a * F(u) when row_w is set (the combine then only adds
-          // rows); the weights were staged in shared memory at the tile start
+          // rows); the weights were staged in shared memory at the tile start.
+          // All 32 weights are read before the chunk's first store: a read
+          // between stores through generic pointers would wait out its
+          // shared-memory latency once per store.
+          if (p.row_w) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] *= fac[c + j];
+          }
           float* yf = static_cast<float*>(p.y_rows);
 #pragma unroll
           for (int j = 0; j < 32; ++j)
-            if (c + j < n_valid)
-              yf[(size_t)(tok0 + c + j) * p.width + col] = p.row_w ? v[j] * fac[c + j] : v[j];
+            if (c + j < n_valid) yf[(size_t)(tok0 + c + j) * p.width + col] = v[j];
         }
       }
       if (!ok) {
