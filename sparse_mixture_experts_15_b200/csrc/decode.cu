@@ -96,11 +96,12 @@ __device__ __forceinline__ void cp4(void* smem, const void* gmem) {
 __device__ __forceinline__ void cp_wait_all() {
   asm volatile("cp.async.wait_all;" ::: "memory");
 }
-// Bulk prefetch into L2; skipped unless the address is 16-byte aligned and
-// the size a multiple of 16 (the instruction's requirements).
-__device__ __forceinline__ void prefetch_l2(const void* gmem, uint32_t bytes) {
-  if (((reinterpret_cast<uintptr_t>(gmem) | bytes) & 15u) != 0 || bytes == 0) return;
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(gmem), "r"(bytes) : "memory");
+// cp.async groups: the copies issued since the last commit form one group;
+// wait_group<n> returns once at most n of this thread's groups are pending.
+__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_wait_group() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
 // rows x row_bytes (multiple of 16) from gmem (row stride g_stride bytes) to
@@ -510,39 +511,24 @@ __global__ void __launch_bounds__(kThreads, 1) decode_persistent(const __grid_co
     };
     __syncthreads();  // list complete before the item loop reads it
     stamp(p, l, 3);
+    // Separate cp.async groups: phase A waits for its gate/up rows only, not
+    // for the down rows of the slice (needed after the barrier).
     if (b < nitems) stage_item(b);
+    cp_commit();
     if (b < nslices) stage_slice(b);
-    // When the batch dispatches at least as many pairs as there are experts
-    // (nearly every expert selected), the next layer's rows go to L2 now, so
-    // that its staging after routing reads L2 instead of DRAM: CTA b takes
-    // phase-A item (expert b / slicesA, slice b % slicesA) -- the item CTA b
-    // stages when every expert is selected, and every (expert, slice) is some
-    // CTA's -- and the down rows of its phase-B slice for every expert.
-    // Smaller batches keep reading the selected experts only.
-    if (!last && Tk >= N && tid == 0) {
-      const LayerPtrs& Ln = p.layer[l + 1];
-      if (b < N * slicesA) {
-        const size_t row = (size_t)(b / slicesA) * h + (size_t)(b % slicesA) * RA;
-        prefetch_l2(Ln.gq + row * (d / 2), RA * (d / 2));
-        prefetch_l2(Ln.uq + row * (d / 2), RA * (d / 2));
-        prefetch_l2(Ln.gs + row * nb, RA * nb * 2);
-        prefetch_l2(Ln.us + row * nb, RA * nb * 2);
-      }
-      if (b < nslices)
-        for (int e = 0; e < N; ++e) {
-          const size_t row = (size_t)e * d + (size_t)b * RB;
-          prefetch_l2(Ln.dq + row * (h / 2), RB * (h / 2));
-          prefetch_l2(Ln.ds + row * nbh, RB * nbh * 2);
-        }
-    }
-
+    cp_commit();
     // ---- phase A: H[e][t][rows] = SiLU(W_gate u) * (W_up u) for the items
     for (int it = b; it < nitems; it += G) {
       const int e = esel[it / slicesA], sl = it % slicesA;
       const int ne = start[e + 1] - start[e];
       const int* toks = list + start[e];
-      if (it != b) stage_item(it);
-      cp_wait_all();
+      if (it != b) {
+        stage_item(it);
+        cp_commit();
+        cp_wait_group<0>();
+      } else {
+        cp_wait_group<1>();  // this item's group; the slice's may still be in flight
+      }
       __syncthreads();
       if (it == b) stamp(p, l, 4);
       for (int x = tid; x < 2 * RA * nb * 8; x += blockDim.x) {  // 8 threads per block
@@ -630,6 +616,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_persistent(const __grid_co
     if (P.nbuf == 2 && !last)  // next layer's router rows, while the barrier completes
       stage_rows(sm + ((l & 1) ? P.wr0 : P.wr1), ws_ld * 4,
                  reinterpret_cast<const char*>(p.layer[l + 1].w_route), (size_t)d * 4, N, d * 4);
+    cp_commit();  // the router rows' own group: phase B does not wait for it
     if (!grid_wait(p.bar, (unsigned)G * ++n_bar, p.status)) {
       cp_wait_all();
       return;
@@ -638,8 +625,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_persistent(const __grid_co
 
     // ---- phase B: y = sum_s a_s W_down[e_s] H_s, u_next = fp16(u + y)
     for (int sl = b; sl < nslices; sl += G) {
-      if (sl != b) stage_slice(sl);
-      cp_wait_all();
+      if (sl != b) {
+        stage_slice(sl);
+        cp_commit();
+        cp_wait_group<0>();
+      } else {
+        cp_wait_group<1>();  // this slice's rows; the next router rows may still be in flight
+      }
       __syncthreads();
       if (sl == b) stamp(p, l, 9);
       // unit = (pair x, row group g, q4 block pp), pp fastest so a pair's
