@@ -21,10 +21,13 @@
 //           into shared fp32, and every (row, token) dot is formed;
 //           H[e][t][rows] = SiLU(g) * v goes to global memory (L2).
 //   barrier
-//   phase B slices of RB output rows: the selected experts' down rows of the
-//           slice were staged before the barrier; every (token, slot) pair
-//           dots its H row with them, the slots are summed in order,
-//           y = sum_s a_s W_down H, u_{l+1} = fp16(u_l + y).
+//   phase B units of (one token, RB output rows), T * d / RB of them: the
+//           token's k selected experts' down rows of the unit were staged
+//           before the barrier; each slot's H row (read from L2) is dotted
+//           with them, the slots are summed in order,
+//           y = sum_s a_s W_down H, u_{l+1} = fp16(u_l + y).  A unit reads
+//           only its token's k rows of H, so an H row is read by d / RB CTAs
+//           rather than by every CTA.
 //   barrier
 // Unselected experts' weights are never read.  Every barrier wait is bounded
 // (2 s of device time); on timeout the kernel records MOE_ERR_TIMEOUT, raises
@@ -300,7 +303,7 @@ struct LayerPtrs {
 // Shared-memory layout (byte offsets) and work split of one launch.
 struct Plan {
   int RA;        // hidden rows per phase-A item (gate and up each)
-  int RB;        // output rows per phase-B slice
+  int RB;        // output rows per phase-B unit (one token x RB rows)
   int nbuf;      // router-weight buffers (2: next layer prefetched)
   int nsel_max;  // experts a layer can select: min(N, T*k)
   int part_cap;  // floats of the phase-A partial-sum buffer
@@ -348,9 +351,14 @@ uint32_t take(uint32_t& off, size_t bytes) {
 bool make_plan(const moe_shape& s, int sms, Plan* out) {
   const int T = s.T, d = s.d, N = s.N, k = s.k, h = s.h;
   const int nb = d / 32, nbh = h / 32;
-  int RB = 4;
-  while (RB < 32 && d / RB > sms) RB *= 2;
+  // phase-B units are (token, RB output rows): ideally the T * d / RB units
+  // fill at most one wave of CTAs, and each unit reads only its token's k
+  // rows of H; RB divides d.  Smaller RB (more units per CTA), then a single
+  // router buffer, then fewer hidden rows per item when shared memory is short.
+  int RB_max = 4;
+  while (RB_max < d && d % (2 * RB_max) == 0 && (int64_t)T * (d / RB_max) > sms) RB_max *= 2;
   const int nsel_max = N < T * k ? N : T * k;
+  for (int RB = RB_max; RB >= 4; RB /= 2)
   for (int nbuf = 2; nbuf >= 1; --nbuf) {
     for (int RA = 8; RA >= 2; RA /= 2) {
       Plan p{};
@@ -377,9 +385,9 @@ bool make_plan(const moe_shape& s, int sms, Plan* out) {
       p.as = take(off, (size_t)2 * RA * nb * 2);
       p.deq = take(off, (size_t)2 * RA * (d + 4) * 4);
       p.part = take(off, (size_t)p.part_cap * 4);
-      p.bq = take(off, (size_t)nsel_max * RB * (h / 2));
-      p.bs = take(off, (size_t)nsel_max * RB * nbh * 2);
-      p.zs = take(off, (size_t)T * k * (RB + 1) * 4);
+      p.bq = take(off, (size_t)k * RB * (h / 2));
+      p.bs = take(off, (size_t)k * RB * nbh * 2);
+      p.zs = take(off, (size_t)k * (RB + 1) * 4);
       p.total = off;
       if (off <= kSmemLimit) {
         *out = p;
@@ -416,7 +424,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_persistent(const __grid_co
   uint8_t* bq = reinterpret_cast<uint8_t*>(sm + P.bq);
   uint16_t* bs = reinterpret_cast<uint16_t*>(sm + P.bs);
   float* zs = reinterpret_cast<float*>(sm + P.zs);
-  const int slicesA = h / RA, nslices = d / RB;
+  const int slicesA = h / RA, nsl = d / RB, nunits = T * nsl;
   unsigned n_bar = 0;
 
   stage_rows(sm + P.wr0, ws_ld * 4, reinterpret_cast<const char*>(p.layer[0].w_route),
@@ -502,20 +510,23 @@ __global__ void __launch_bounds__(kThreads, 1) decode_persistent(const __grid_co
       stage_bytes(as, L.gs + row * nb, RA * nb * 2);
       stage_bytes(as + RA * nb, L.us + row * nb, RA * nb * 2);
     };
-    auto stage_slice = [&](int sl) {
-      for (int j = 0; j < nsel; ++j) {
-        const size_t row = (size_t)esel[j] * d + (size_t)sl * RB;
-        stage_bytes(bq + (size_t)j * RB * (h / 2), L.dq + row * (h / 2), RB * (h / 2));
-        stage_bytes(bs + (size_t)j * RB * nbh, L.ds + row * nbh, RB * nbh * 2);
+    // the down rows of phase-B unit un (token un / nsl, rows (un % nsl) RB..)
+    // of the token's k selected experts, slot s at bq + s RB h/2
+    auto stage_unit = [&](int un) {
+      const int t = un / nsl, sl = un - t * nsl;
+      for (int s2 = 0; s2 < k; ++s2) {
+        const size_t row = (size_t)sel[t * k + s2] * d + (size_t)sl * RB;
+        stage_bytes(bq + (size_t)s2 * RB * (h / 2), L.dq + row * (h / 2), RB * (h / 2));
+        stage_bytes(bs + (size_t)s2 * RB * nbh, L.ds + row * nbh, RB * nbh * 2);
       }
     };
     __syncthreads();  // list complete before the item loop reads it
     stamp(p, l, 3);
     // Separate cp.async groups: phase A waits for its gate/up rows only, not
-    // for the down rows of the slice (needed after the barrier).
+    // for the down rows of the phase-B unit (needed after the barrier).
     if (b < nitems) stage_item(b);
     cp_commit();
-    if (b < nslices) stage_slice(b);
+    if (b < nunits) stage_unit(b);
     cp_commit();
     // ---- phase A: H[e][t][rows] = SiLU(W_gate u) * (W_up u) for the items
     for (int it = b; it < nitems; it += G) {
@@ -623,35 +634,36 @@ __global__ void __launch_bounds__(kThreads, 1) decode_persistent(const __grid_co
     }
     stamp(p, l, 8);
 
-    // ---- phase B: y = sum_s a_s W_down[e_s] H_s, u_next = fp16(u + y)
-    for (int sl = b; sl < nslices; sl += G) {
-      if (sl != b) {
-        stage_slice(sl);
+    // ---- phase B: y = sum_s a_s W_down[e_s] H_s, u_next = fp16(u + y), one
+    // (token, RB output rows) unit at a time
+    for (int un = b; un < nunits; un += G) {
+      const int t = un / nsl, sl = un - t * nsl;
+      if (un != b) {
+        stage_unit(un);
         cp_commit();
         cp_wait_group<0>();
       } else {
-        cp_wait_group<1>();  // this slice's rows; the next router rows may still be in flight
+        cp_wait_group<1>();  // this unit's rows; the next router rows may still be in flight
       }
       __syncthreads();
-      if (sl == b) stamp(p, l, 9);
-      // unit = (pair x, row group g, q4 block pp), pp fastest so a pair's
-      // nbh partial dots sit in adjacent lanes; the rows of a slice are split
-      // into rgroups groups when there are few pairs, so more threads work.
+      if (un == b) stamp(p, l, 9);
+      // thread = (slot s, row group g, q4 block pp), pp fastest so a slot's
+      // nbh partial dots sit in adjacent lanes; the RB rows are split into
+      // rgroups groups so that about a CTA's worth of threads work
       int rgroups = 1;
-      while (rgroups < RB && Tk * nbh * rgroups * 2 <= (int)blockDim.x) rgroups *= 2;
+      while (rgroups < RB && k * nbh * rgroups * 2 <= (int)blockDim.x) rgroups *= 2;
       const int rper = RB / rgroups;
-      const int units = Tk * nbh * rgroups;
-      for (int base = 0; base < units; base += blockDim.x) {  // uniform per warp
+      const int nthr = k * nbh * rgroups;
+      for (int base = 0; base < nthr; base += blockDim.x) {  // uniform per warp
         const int uu = base + tid;
-        const bool valid = uu < units;
+        const bool valid = uu < nthr;
         const int pp = uu % nbh, rest = uu / nbh;
-        const int g = rest % rgroups, x = valid ? rest / rgroups : 0;
-        const int e = sel[x];
-        const int j = epos[e];
+        const int g = rest % rgroups, s2 = valid ? rest / rgroups : 0;
+        const int e = sel[t * k + s2];
         float hc[32];
         if (valid) {
           const float4* hp =
-              reinterpret_cast<const float4*>(p.H + ((size_t)e * T + x / k) * h + pp * 32);
+              reinterpret_cast<const float4*>(p.H + ((size_t)e * T + t) * h + pp * 32);
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
             const float4 v = __ldcg(hp + c);
@@ -668,8 +680,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_persistent(const __grid_co
           float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
           if (valid) {
             float wv[32];
-            dequant_block(bq + ((size_t)j * RB + r) * (h / 2) + pp * 16,
-                          bs[((size_t)j * RB + r) * nbh + pp], wv);
+            dequant_block(bq + ((size_t)s2 * RB + r) * (h / 2) + pp * 16,
+                          bs[((size_t)s2 * RB + r) * nbh + pp], wv);
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
               a0 = fmaf(wv[4 * c], hc[4 * c], a0);
@@ -680,16 +692,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_persistent(const __grid_co
           }
           float zz = (a0 + a1) + (a2 + a3);
           for (int o = nbh / 2; o >= 1; o >>= 1) zz += __shfl_xor_sync(0xffffffffu, zz, o);
-          if (valid && pp == 0) zs[x * (RB + 1) + r] = zz;
+          if (valid && pp == 0) zs[s2 * (RB + 1) + r] = zz;
         }
       }
       __syncthreads();
-      if (sl == b) stamp(p, l, 10);
-      for (int v = tid; v < T * RB; v += blockDim.x) {
-        const int t = v / RB, r = v - t * RB;
+      if (un == b) stamp(p, l, 10);
+      for (int r = tid; r < RB; r += blockDim.x) {
         float acc = 0.0f;
-        for (int s2 = 0; s2 < k; ++s2)
-          acc = fmaf(aw[t * k + s2], zs[(t * k + s2) * (RB + 1) + r], acc);
+        for (int q = 0; q < k; ++q) acc = fmaf(aw[t * k + q], zs[q * (RB + 1) + r], acc);
         const int m = sl * RB + r;
         const size_t o = (size_t)t * d + m;
         if (last && p.y) p.y[o] = __float2half_rn(acc);
@@ -697,7 +707,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_persistent(const __grid_co
       }
       __syncthreads();
     }
-    if (b >= nslices)
+    if (b >= nunits)
       for (int i = 9; i < 11; ++i) stamp(p, l, i);
     stamp(p, l, 11);
     grid_arrive(p.bar);
@@ -792,7 +802,7 @@ int launch_decode(const moe_shape& s, const moe_q4_layer* layers, int n, const _
                                                     p.plan.total) != cudaSuccess)
     return MOE_ERR_CUDA;
   if (occ < 1) return MOE_ERR_UNSUPPORTED;
-  const int items = p.plan.nsel_max * (s.h / p.plan.RA), slices = s.d / p.plan.RB;
+  const int items = p.plan.nsel_max * (s.h / p.plan.RA), slices = s.T * (s.d / p.plan.RB);
   int grid = items > slices ? items : slices;
   if (grid > sms) grid = sms;
   for (int l = 0; l < n; ++l) p.layer[l] = layer_ptrs(layers[l]);
