@@ -401,423 +401,6 @@ __global__ void __launch_bounds__(fThreads, 1) tc_fused_ffn(const __grid_constan
   }
 }
 
-// ------------------------------------------------------------- CTA pairs
-// The same FFN on clusters of two CTAs sharing each tcgen05.mma
-// (cta_group::2, M = 256) over 128-token tiles, for h % 128 == 0 and
-// width % 256 == 0.  Phase A: one MMA covers two 64-unit hidden slices (the
-// even CTA stages slice 2p's 64 gate + 64 up rows, the odd CTA slice 2p+1's)
-// and each CTA stages its half of the tokens, so per k-block a CTA moves 16 KB
-// of weights and 8 KB of tokens for 128 tokens (the single-CTA kernel moves
-// 16 + 8 KB for 64 tokens).  Each CTA's accumulator holds its hidden slice for
-// all 128 tokens, while phase B's MMA wants each CTA's half of the tokens for
-// all hidden units: epilogue A writes its own half of the tokens into the H
-// tile and the peer's half into an exchange buffer, each CTA then copies the
-// peer's buffer into its H tile (shared::cluster loads after an mbarrier
-// handshake at cluster scope).  Phase B: the even CTA stages 128 of each 256
-// output rows, the odd CTA the other 128.
-constexpr int pBN = 128;  // tokens per pair tile
-constexpr int pMaxA = fHMax / 128, pMaxB = 4;
-
-struct PLayout {
-  static constexpr int A_BYTES = 128 * fBK * 2;         // this CTA's 128 weight rows
-  static constexpr int X_BYTES = (pBN / 2) * fBK * 2;   // this CTA's 64 token rows
-  static constexpr int STAGE = A_BYTES + X_BYTES;
-  static constexpr int KB_BYTES = (pBN / 2) * 128;      // one 64-unit k-block of H, 64 rows
-  static constexpr int EPI_BYTES = fBM * fEpiLd * 4 + pBN * 4;
-  // stage ring, H tile (h / 64 k-blocks), exchange buffer (h / 128
-  // k-blocks), epilogue exchange + row weights, group tables, barriers
-  __host__ __device__ static int stages(int h) {
-    const int fixed = 1024 + (h / 64) * KB_BYTES + (h / 128) * KB_BYTES + EPI_BYTES + 4096;
-    const int s = (227 * 1024 - fixed) / STAGE;
-    return s > 7 ? 7 : s;
-  }
-  static constexpr int kBars = pMaxA + pMaxB + 5;  // a_done, b_done, h_ready, b_free, x_ready, x_free, drain
-  __host__ __device__ static size_t bytes(int G, int h) {
-    const int S = stages(h);
-    size_t b = 1024 + (size_t)S * STAGE + (size_t)(h / 64) * KB_BYTES +
-               (size_t)(h / 128) * KB_BYTES + EPI_BYTES + (size_t)3 * (G + 1) * 4;
-    b = (b + 7) & ~(size_t)7;
-    b += (size_t)(2 * S + kBars) * 8 + 16;
-    return b;
-  }
-};
-
-template <int ACT>
-__global__ void __launch_bounds__(fThreads, 1)
-    tc_fused_ffn_pair(const __grid_constant__ FusedParams p) {
-  using L = PLayout;
-  extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  const int S = L::stages(p.h);
-  const int kbh = p.h / 64;                      // k-blocks of H
-  uint8_t* stages = smem;
-  uint8_t* hs = smem + S * L::STAGE;             // H tile: kbh k-blocks x 64 rows x 128 B
-  uint8_t* xb = hs + kbh * L::KB_BYTES;          // the peer's token half of this CTA's slices
-  float* epi = reinterpret_cast<float*>(xb + (kbh / 2) * L::KB_BYTES);
-  float* fac = epi + fBM * fEpiLd;               // [pBN] the tile's combine weights
-  int* grp_beg = reinterpret_cast<int*>(fac + pBN);
-  int* grp_cnt = grp_beg + (p.G + 1);
-  int* grp_pre = grp_cnt + (p.G + 1);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(
-      (reinterpret_cast<uintptr_t>(grp_pre + p.G + 1) + 7) & ~static_cast<uintptr_t>(7));
-  uint64_t* full = bars;
-  uint64_t* empty = bars + S;
-  uint64_t* a_done = bars + 2 * S;   // [pMaxA] pair-slice p's accumulator (both CTAs)
-  uint64_t* b_done = a_done + pMaxA; // [pMaxB] output pair-slice m2's accumulator
-  uint64_t* h_ready = b_done + pMaxB;  // even CTA: both H tiles complete (2 arrivals)
-  uint64_t* b_free = h_ready + 1;      // even CTA: both epilogues B done (2 arrivals)
-  uint64_t* x_ready = b_free + 1;      // the peer's exchange buffer is written
-  uint64_t* x_free = x_ready + 1;      // the peer has read this CTA's exchange buffer
-  uint64_t* drain = x_free + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + L::kBars);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-
-  const uint32_t rank = tc::cluster_rank(), peer = rank ^ 1u;
-  const bool leader = rank == 0;
-  const int unit = (int)(blockIdx.x >> 1), n_units = (int)(gridDim.x >> 1);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (warp == 0 && lane == 0) {
-    *abort_flag = 0;
-    for (int i = 0; i < S; ++i) {
-      tc::mbar_init(tc::smem_u32(&full[i]), 1);
-      tc::mbar_init(tc::smem_u32(&empty[i]), 1);
-    }
-    for (int i = 0; i < pMaxA; ++i) tc::mbar_init(tc::smem_u32(&a_done[i]), 1);
-    for (int i = 0; i < pMaxB; ++i) tc::mbar_init(tc::smem_u32(&b_done[i]), 1);
-    tc::mbar_init(tc::smem_u32(h_ready), 2);
-    tc::mbar_init(tc::smem_u32(b_free), 2);
-    tc::mbar_init(tc::smem_u32(x_ready), 1);
-    tc::mbar_init(tc::smem_u32(x_free), 1);
-    tc::mbar_init(tc::smem_u32(drain), 1);
-    tc::fence_barrier_init();
-    tc::tma_prefetch_desc(&p.map_g);
-    tc::tma_prefetch_desc(&p.map_u);
-    tc::tma_prefetch_desc(&p.map_x);
-    tc::tma_prefetch_desc(&p.map_d);
-  }
-  if (warp == 1) {
-    tc::tmem_alloc_pair(tc::smem_u32(tmem_slot), 512);
-    tc::tmem_relinquish_pair();
-  }
-  // both CTAs' barriers exist before either signals the other's
-  tc::tc_fence_before();
-  tc::cluster_sync();
-  pdl_wait();
-  pdl_allow_next();
-  if (warp == 0) {  // group table: one pair tile = (expert, 128 tokens)
-    int carry = 0;
-    for (int base = 0; base < p.G; base += 32) {
-      const int g = base + lane;
-      int beg = 0, cnt = 0;
-      if (g < p.G) {
-        beg = p.offsets[g];
-        cnt = p.offsets[g + 1] - beg;
-        if (cnt < 0 || beg < 0 || beg > p.R || cnt > p.R - beg) {  // rows outside the buffers
-          record_error(p.status, MOE_ERR_BOUNDS);
-          cnt = 0;
-        }
-      }
-      const int t = g < p.G ? (cnt + pBN - 1) / pBN : 0;
-      int incl = t;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int n = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += n;
-      }
-      if (g < p.G) {
-        grp_beg[g] = beg;
-        grp_cnt[g] = cnt;
-        grp_pre[g] = carry + incl - t;
-      }
-      carry += __shfl_sync(0xffffffffu, incl, 31);
-    }
-    if (lane == 0) grp_pre[p.G] = carry;
-  }
-  tc::tc_fence_before();
-  __syncthreads();
-  tc::tc_fence_after();
-  const uint32_t tmem_base = *tmem_slot;
-  const int total_tiles = grp_pre[p.G];
-  const int mA = p.h / 128, mB = p.width / 256, kA = p.width / fBK, kB = p.h / fBK;
-
-  auto decode = [&](int tile, int& g, int& n) {
-    int lo = 0, hi = p.G;
-    while (hi - lo > 1) {
-      const int mid = (lo + hi) >> 1;
-      if (grp_pre[mid] <= tile) lo = mid; else hi = mid;
-    }
-    g = lo;
-    n = tile - grp_pre[g];
-  };
-
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
-      bool ok = true;
-      for (int tile = unit; tile < total_tiles && ok; tile += n_units) {
-        int g, n;
-        decode(tile, g, n);
-        const int n_valid = min(pBN, grp_cnt[g] - n * pBN);
-        const int half = ((n_valid + 15) & ~15) / 2;
-        const int x_row = grp_beg[g] + n * pBN + (int)rank * half;
-        for (int j = 0; j < mA * kA + mB * kB && ok; ++j) {
-          if (!tc::mbar_wait(tc::smem_u32(&empty[stage]), phase ^ 1u, abort_flag, fWaitBudget)) {
-            ok = false;
-            break;
-          }
-          // both CTAs' bytes complete on the even CTA's full barrier
-          const uint32_t fb = tc::mapa_shared(tc::smem_u32(&full[stage]), 0u);
-          const uint32_t sa = tc::smem_u32(stages + stage * L::STAGE);
-          if (j < mA * kA) {  // gate + up rows of hidden block 2 m + rank, token half
-            const int m = j / kA, kb = j - m * kA;
-            const int wrow = g * p.h + (2 * m + (int)rank) * 64;
-            if (leader) tc::mbar_arrive_expect_tx(tc::smem_u32(&full[stage]), 2 * L::STAGE);
-            tc::tma_load_2d_pair(sa, &p.map_g, fb, kb * fBK, wrow);
-            tc::tma_load_2d_pair(sa + L::A_BYTES / 2, &p.map_u, fb, kb * fBK, wrow);
-            tc::tma_load_2d_pair(sa + L::A_BYTES, &p.map_x, fb, kb * fBK, x_row);
-          } else {  // 128 of the 256 down rows of output pair-slice m2
-            const int jj = j - mA * kA, m2 = jj / kB, kb = jj - m2 * kB;
-            if (leader) tc::mbar_arrive_expect_tx(tc::smem_u32(&full[stage]), 2 * L::A_BYTES);
-            tc::tma_load_2d_pair(sa, &p.map_d, fb, kb * fBK,
-                                 g * p.width + m2 * 256 + (int)rank * 128);
-          }
-          if (++stage == S) {
-            stage = 0;
-            phase ^= 1u;
-          }
-        }
-      }
-      if (!ok) {
-        record_error(p.status, MOE_ERR_TIMEOUT);
-        *abort_flag = 1;
-      }
-      // Drain: the even CTA waits for its full barriers (both CTAs' bytes),
-      // the odd CTA until the MMAs released its last stages.
-      for (int i = 0; i < S; ++i) {
-        if (--stage < 0) {
-          stage = S - 1;
-          phase ^= 1u;
-        }
-        if (leader)
-          tc::mbar_wait(tc::smem_u32(&full[stage]), phase, nullptr, fWaitBudget / 8);
-        else
-          tc::mbar_wait(tc::smem_u32(&empty[stage]), phase, nullptr, fWaitBudget / 8);
-      }
-    }
-    __syncwarp();
-  } else if (warp == 1) {
-    // ------------------------------------------------------ MMA (even CTA)
-    if (lane == 0 && leader) {
-      int stage = 0;
-      uint32_t phase = 0;
-      bool ok = true;
-      int it = 0;
-      const uint32_t hs_addr = tc::smem_u32(hs);
-      for (int tile = unit; tile < total_tiles && ok; tile += n_units, ++it) {
-        int g, n;
-        decode(tile, g, n);
-        const int n_valid = min(pBN, grp_cnt[g] - n * pBN);
-        const uint32_t idesc = tc::idesc_bf16_f32(256, (uint32_t)((n_valid + 15) & ~15));
-        const uint32_t par = (uint32_t)(it & 1);
-        // phase A (its TMEM columns were read by the previous tile's
-        // epilogues A, which finished before that tile's h_ready)
-        for (int m = 0; m < mA && ok; ++m) {
-          for (int kb = 0; kb < kA; ++kb) {
-            if (!tc::mbar_wait(tc::smem_u32(&full[stage]), phase, abort_flag, fWaitBudget)) {
-              ok = false;
-              break;
-            }
-            tc::tc_fence_after();
-            const uint32_t sa = tc::smem_u32(stages + stage * L::STAGE);
-#pragma unroll
-            for (int k = 0; k < fBK / 16; ++k)
-              tc::mma_bf16_pair(tmem_base + (uint32_t)(m * pBN), tc::smem_desc_sw128(sa + k * 32),
-                                tc::smem_desc_sw128(sa + L::A_BYTES + k * 32), idesc,
-                                (kb | k) != 0 ? 1u : 0u);
-            tc::mma_commit_pair(tc::smem_u32(&empty[stage]), 0x3);
-            if (++stage == S) {
-              stage = 0;
-              phase ^= 1u;
-            }
-          }
-          if (ok) tc::mma_commit_pair(tc::smem_u32(&a_done[m]), 0x3);
-        }
-        if (!ok) break;
-        if (!tc::mbar_wait_cluster(tc::smem_u32(h_ready), par, abort_flag, fWaitBudget) ||
-            !tc::mbar_wait_cluster(tc::smem_u32(b_free), par ^ 1u, abort_flag, fWaitBudget)) {
-          ok = false;
-          break;
-        }
-        tc::tc_fence_after();
-        for (int m2 = 0; m2 < mB && ok; ++m2) {
-          for (int kb = 0; kb < kB; ++kb) {
-            if (!tc::mbar_wait(tc::smem_u32(&full[stage]), phase, abort_flag, fWaitBudget)) {
-              ok = false;
-              break;
-            }
-            tc::tc_fence_after();
-            const uint32_t sa = tc::smem_u32(stages + stage * L::STAGE);
-            const uint32_t hb = hs_addr + (uint32_t)(kb * L::KB_BYTES);
-#pragma unroll
-            for (int k = 0; k < fBK / 16; ++k)
-              tc::mma_bf16_pair(tmem_base + (uint32_t)((mA + m2) * pBN),
-                                tc::smem_desc_sw128(sa + k * 32), tc::smem_desc_sw128(hb + k * 32),
-                                idesc, (kb | k) != 0 ? 1u : 0u);
-            tc::mma_commit_pair(tc::smem_u32(&empty[stage]), 0x3);
-            if (++stage == S) {
-              stage = 0;
-              phase ^= 1u;
-            }
-          }
-          if (ok) tc::mma_commit_pair(tc::smem_u32(&b_done[m2]), 0x3);
-        }
-        if (!ok) break;
-      }
-      if (!ok) {
-        record_error(p.status, MOE_ERR_TIMEOUT);
-        *abort_flag = 1;
-        // every MMA issued so far finishes before TMEM is released
-        tc::mma_commit_pair(tc::smem_u32(drain), 0x1);
-        tc::mbar_wait(tc::smem_u32(drain), 0, nullptr, fWaitBudget / 8);
-      }
-    }
-    __syncwarp();
-  } else {
-    // ------------------------------------------------- epilogue (both CTAs)
-    const int q = warp & 3, row = q * 32 + lane;
-    const uint32_t h_ready_0 = tc::mapa_shared(tc::smem_u32(h_ready), 0u);
-    const uint32_t b_free_0 = tc::mapa_shared(tc::smem_u32(b_free), 0u);
-    const uint32_t x_ready_peer = tc::mapa_shared(tc::smem_u32(x_ready), peer);
-    const uint32_t x_free_peer = tc::mapa_shared(tc::smem_u32(x_free), peer);
-    const uint32_t xb_peer = tc::mapa_shared(tc::smem_u32(xb), peer);
-    int it = 0;
-    for (int tile = unit; tile < total_tiles; tile += n_units, ++it) {
-      int g, n;
-      decode(tile, g, n);
-      const int n_valid = min(pBN, grp_cnt[g] - n * pBN);
-      const int n_mma = (n_valid + 15) & ~15, half = n_mma / 2;
-      const int tok0 = grp_beg[g] + n * pBN;
-      const uint32_t par = (uint32_t)(it & 1);
-      bool ok = true;
-      if (p.row_w) {  // the tile's combine weights, once every warp is done with the previous
-        asm volatile("bar.sync 1, 128;" ::: "memory");
-        for (int i = row; i < pBN; i += 128) fac[i] = i < n_valid ? p.row_w[tok0 + i] : 1.0f;
-      }
-      // this CTA's exchange buffer may be rewritten once the peer has read it
-      if (!all_epi_ok(tc::mbar_wait_cluster(tc::smem_u32(x_free), par ^ 1u, abort_flag,
-                                            fWaitBudget)))
-        ok = false;
-      // H = act(gate, up) of hidden block 2 m + rank for all tokens: this CTA's
-      // token half into its H tile, the peer's half into the exchange buffer
-      for (int m = 0; m < mA && ok; ++m) {
-        if (!all_epi_ok(tc::mbar_wait(tc::smem_u32(&a_done[m]), par, abort_flag, fWaitBudget))) {
-          ok = false;
-          break;
-        }
-        tc::tc_fence_after();
-        const int hb = 2 * m + (int)rank;
-        for (int c = 0; c < n_mma; c += 32) {
-          float v[32];
-          tc::tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(m * pBN + c),
-                                 v);
-#pragma unroll
-          for (int j = 0; j < 32; ++j) epi[row * fEpiLd + j] = v[j];
-          asm volatile("bar.sync 1, 128;" ::: "memory");
-          const int tok = c + lane;
-          uint32_t packed[8];
-#pragma unroll
-          for (int i = 0; i < 16; i += 2) {
-            const float h0 = gated_act<ACT>(epi[(q * 16 + i) * fEpiLd + lane],
-                                            epi[(64 + q * 16 + i) * fEpiLd + lane], p.beta_g,
-                                            p.beta_u);
-            const float h1 = gated_act<ACT>(epi[(q * 16 + i + 1) * fEpiLd + lane],
-                                            epi[(64 + q * 16 + i + 1) * fEpiLd + lane], p.beta_g,
-                                            p.beta_u);
-            __nv_bfloat162 hv = __floats2bfloat162_rn(h0, h1);
-            packed[i >> 1] = *reinterpret_cast<uint32_t*>(&hv);
-          }
-          if (tok < n_mma) {
-            const int dh = tok < half ? 0 : 1, lr = tok - dh * half;
-            // 16-byte chunks 2q and 2q+1 of row lr, swizzled by (lr mod 8)
-            uint8_t* rowp = (dh == (int)rank ? hs + hb * L::KB_BYTES : xb + m * L::KB_BYTES) +
-                            lr * 128;
-            *reinterpret_cast<uint4*>(rowp + (((2 * q) ^ (lr & 7)) << 4)) =
-                make_uint4(packed[0], packed[1], packed[2], packed[3]);
-            *reinterpret_cast<uint4*>(rowp + (((2 * q + 1) ^ (lr & 7)) << 4)) =
-                make_uint4(packed[4], packed[5], packed[6], packed[7]);
-          }
-          asm volatile("bar.sync 1, 128;" ::: "memory");
-        }
-      }
-      if (ok) {
-        // hand this CTA's exchange buffer to the peer, take the peer's
-        if (threadIdx.x == 64) tc::mbar_arrive_cluster(x_ready_peer);
-        if (!all_epi_ok(tc::mbar_wait_cluster(tc::smem_u32(x_ready), par, abort_flag,
-                                              fWaitBudget)))
-          ok = false;
-      }
-      if (ok) {
-        for (int m = 0; m < mA; ++m) {
-          // the peer's hidden block 2 m + peer for this CTA's token half
-          uint8_t* dst = hs + (2 * m + (int)peer) * L::KB_BYTES;
-          const uint32_t src = xb_peer + (uint32_t)(m * L::KB_BYTES);
-          for (int i = row; i < half * 8; i += 128)
-            *reinterpret_cast<uint4*>(dst + i * 16) = tc::ld_shared_cluster_v4(src + i * 16);
-        }
-        asm volatile("bar.sync 1, 128;" ::: "memory");
-        if (threadIdx.x == 64) tc::mbar_arrive_cluster(x_free_peer);
-        // the generic-proxy writes of the H tile before the tensor core reads it
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        tc::tc_fence_before();
-        asm volatile("bar.sync 1, 128;" ::: "memory");
-        if (threadIdx.x == 64) tc::mbar_arrive_cluster(h_ready_0);
-      }
-      for (int m2 = 0; m2 < mB && ok; ++m2) {
-        if (!all_epi_ok(tc::mbar_wait(tc::smem_u32(&b_done[m2]), par, abort_flag, fWaitBudget))) {
-          ok = false;
-          break;
-        }
-        tc::tc_fence_after();
-        const int col = m2 * 256 + (int)rank * 128 + row;
-        for (int c = 0; c < n_valid; c += 32) {
-          float v[32];
-          tc::tmem_ld_32x32b_x32(
-              tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)((mA + m2) * pBN + c), v);
-          if (p.row_w) {  // all 32 weights read before the chunk's first store
-#pragma unroll
-            for (int j = 0; j < 32; ++j) v[j] *= fac[c + j];
-          }
-          float* yf = static_cast<float*>(p.y_rows);
-#pragma unroll
-          for (int j = 0; j < 32; ++j)
-            if (c + j < n_valid) yf[(size_t)(tok0 + c + j) * p.width + col] = v[j];
-        }
-      }
-      if (!ok) {
-        record_error(p.status, MOE_ERR_TIMEOUT);
-        *abort_flag = 1;
-        break;
-      }
-      tc::tc_fence_before();
-      asm volatile("bar.sync 1, 128;" ::: "memory");
-      if (threadIdx.x == 64) tc::mbar_arrive_cluster(b_free_0);
-    }
-  }
-
-  tc::tc_fence_before();
-  __syncthreads();
-  // TMEM is freed only when neither CTA's roles touch the other any more
-  // (remote arrivals, exchange-buffer reads, MMAs writing both CTAs' TMEM)
-  tc::cluster_sync();
-  if (warp == 1) {
-    tc::tc_fence_after();
-    tc::tmem_dealloc_pair(tmem_base, 512);
-  }
-}
-
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                    const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
                                    const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
@@ -846,14 +429,6 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, ui
 }  // namespace
 
 constexpr size_t fSmemLimit = 227 * 1024;
-
-// The CTA-pair variant: two 64-unit hidden slices per MMA (h % 128 == 0), 256
-// output rows per MMA (width % 256 == 0), all accumulators in 512 TMEM
-// columns.
-bool ffn_fused_pair_ok(int width, int h, int G) {
-  return h % 128 == 0 && h <= fHMax && width % 256 == 0 && width >= 256 &&
-         (h / 128 + width / 256) * pBN <= 512 && PLayout::bytes(G, h) <= fSmemLimit;
-}
 
 bool ffn_fused_ok(int width, int h, int G) {
   return h % 64 == 0 && h <= fHMax && width % fBM == 0 && width >= fBM &&
@@ -890,56 +465,9 @@ int launch_ffn_fused(int G, int64_t R, int width, int h, const __nv_bfloat16* x_
                              (int)fSmemLimit) != cudaSuccess ||
         cudaFuncSetAttribute(tc_fused_ffn<MOE_ACT_SITU_GLU>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)fSmemLimit) != cudaSuccess ||
-        cudaFuncSetAttribute(tc_fused_ffn_pair<MOE_ACT_SWIGLU>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)fSmemLimit) != cudaSuccess ||
-        cudaFuncSetAttribute(tc_fused_ffn_pair<MOE_ACT_SITU_GLU>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)fSmemLimit) != cudaSuccess)
       return MOE_ERR_CUDA;
     configured[dev] = true;
-  }
-  if (ffn_fused_pair_ok(width, h, G)) {
-    // CTA pairs: the grid is the number of clusters of two that can be
-    // resident at once (persistent: no cluster waits for another)
-    static std::atomic<int> resident[kMaxDevices];
-    int np = device_slot(dev) ? resident[dev].load(std::memory_order_relaxed) : 0;
-    const size_t smem = PLayout::bytes(G, h);
-    auto kernel = act.kind == MOE_ACT_SITU_GLU ? tc_fused_ffn_pair<MOE_ACT_SITU_GLU>
-                                               : tc_fused_ffn_pair<MOE_ACT_SWIGLU>;
-    cudaLaunchAttribute attr[2];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[1].val.programmaticStreamSerializationAllowed = 1;
-    cudaLaunchConfig_t cfg = {};
-    cfg.blockDim = dim3(fThreads);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = st;
-    cfg.attrs = attr;
-    if (np <= 0) {
-      int sms = 0;
-      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-      cfg.gridDim = dim3(2 * (unsigned)sms);
-      cfg.numAttrs = 1;
-      if (cudaOccupancyMaxActiveClusters(&np, kernel, &cfg) != cudaSuccess || np <= 0) {
-        cudaGetLastError();
-        return MOE_ERR_CUDA;
-      }
-      if (device_slot(dev)) resident[dev].store(np, std::memory_order_relaxed);
-    }
-    int64_t pairs = (R + pBN - 1) / pBN + G;  // upper bound on the pair tiles
-    if (pairs > np) pairs = np;
-    cfg.gridDim = dim3((unsigned)(2 * pairs));
-    cfg.numAttrs = 2;
-    MOE_PREFER_SHARED((tc_fused_ffn_pair<MOE_ACT_SWIGLU>));
-    MOE_PREFER_SHARED((tc_fused_ffn_pair<MOE_ACT_SITU_GLU>));
-    const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, p);
-    if (e != cudaSuccess) pdl_launch_error() = e;
-    return launch_status();
   }
   int sms = 0;
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);

@@ -43,21 +43,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
-// The same with acquire at cluster scope: for phases completed by arrivals
-// (release at cluster scope) from the peer CTA, whose shared-memory writes
-// the waiting thread then reads.
-__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity), "r"(kTryWaitSuspendNs)
-      : "memory");
-  return ok != 0;
-}
-
 // Bounded wait: gives up after ~budget cycles or when *abort (if not null) is
 // raised by another role of the same CTA.  Returns false on give-up.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort,
@@ -66,17 +51,6 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
   const long long t0 = clock64();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (abort && *abort) return false;
-    if (clock64() - t0 > budget) return false;
-  }
-}
-
-__device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity,
-                                                  volatile int* abort, long long budget) {
-  if (mbar_try_wait_cluster(bar, parity)) return true;
-  const long long t0 = clock64();
-  while (true) {
-    if (mbar_try_wait_cluster(bar, parity)) return true;
     if (abort && *abort) return false;
     if (clock64() - t0 > budget) return false;
   }
@@ -171,16 +145,6 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
   uint32_t r;
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
   return r;
-}
-// 16-byte load from the shared memory of a CTA of the cluster (an address
-// from mapa_shared).
-__device__ __forceinline__ uint4 ld_shared_cluster_v4(uint32_t cluster_addr) {
-  uint4 v;
-  asm volatile("ld.shared::cluster.v4.u32 {%0, %1, %2, %3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "r"(cluster_addr)
-               : "memory");
-  return v;
 }
 // Arrive (release at cluster scope) on an mbarrier given by its
 // shared::cluster address, possibly in the peer CTA.

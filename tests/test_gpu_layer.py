@@ -73,9 +73,9 @@ def test_expert_ffn_f32_simt():
 
 @pytest.mark.parametrize("counts,width,h", [
     ([16], 128, 64),                                   # one tile, smallest shapes
-    ([0, 5, 130, 257, 16, 1, 300, 64], 512, 256),      # fused, CTA pairs: two hidden pair-slices
-    ([1024] * 8, 512, 128),                            # the small-model layer's shape (fused pairs)
-    ([300, 0, 77, 130], 384, 128),                     # fused single-CTA (width % 256 != 0)
+    ([0, 5, 130, 257, 16, 1, 300, 64], 512, 256),      # fused: ragged tails, empty expert
+    ([1024] * 8, 512, 128),                            # the small-model layer's shape (fused)
+    ([300, 0, 77, 130], 384, 128),                     # fused, three output slices
     ([700, 333, 1500, 410], 512, 1024),                # CTA pairs, 128-token tiles
     ([1100, 257, 1500, 143], 1024, 2048),              # CTA pairs, 256-token tiles, ragged
     ([100, 37, 260, 5], 512, 512),                     # CTA pairs, few rows per expert
@@ -88,8 +88,8 @@ def test_expert_ffn_bf16_tensor_cores(counts, width, h):
 
 
 @pytest.mark.parametrize("counts,width,h", [
-    ([100, 37, 260], 256, 192),   # fused single-CTA
-    ([100, 37, 260], 256, 128),   # fused CTA pairs
+    ([100, 37, 260], 256, 192),   # fused, three hidden slices
+    ([100, 37, 260], 256, 128),   # fused, two hidden slices
 ])
 def test_expert_ffn_bf16_situ_glu_soft_caps(counts, width, h):
     """SiTU-GLU epilogue with inputs large enough for the caps to bind."""
