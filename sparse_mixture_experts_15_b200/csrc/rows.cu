@@ -90,7 +90,9 @@ __global__ void __launch_bounds__(256)
 }
 
 // One warp per token; rows already carry their weights (fp32 a * F(u)), the
-// kept slots are added in ascending s in fp32 and rounded once.
+// kept slots are added in ascending s in fp32 and rounded once.  The token's
+// k (<= 32) slot rows are read once into shared memory; the row loads of four
+// slots are issued before their adds, so a warp has several loads in flight.
 template <typename TY>
 __global__ void __launch_bounds__(256)
     combine_weighted(const float4* __restrict__ rows, int width4,
@@ -98,27 +100,39 @@ __global__ void __launch_bounds__(256)
                      int* status) {
   pdl_wait();
   pdl_allow_next();
-  const int lane = threadIdx.x & 31;
+  __shared__ int srow[256 / 32][32];
+  const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
   for (int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; t < T;
        t += (gridDim.x * blockDim.x) >> 5) {
-#pragma unroll 4
-    for (int c = lane; c < width4; c += 32) {  // unrolled: the row loads of 4 steps in flight
+    int r = lane < k ? row_of[(size_t)t * k + lane] : -1;
+    if (r >= T * k) {  // rows holds T*k rows
+      record_error(status, MOE_ERR_BOUNDS);
+      r = -1;
+    }
+    srow[wib][lane] = r;
+    __syncwarp();
+    for (int c = lane; c < width4; c += 32) {
       float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int s = 0; s < k; ++s) {
-        const int r = row_of[(size_t)t * k + s];
-        if (r < 0) continue;
-        if (r >= T * k) {  // rows holds T*k rows
-          record_error(status, MOE_ERR_BOUNDS);
-          continue;
+      for (int s0 = 0; s0 < k; s0 += 4) {
+        float4 v[4];
+        int rs[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          rs[j] = s0 + j < k ? srow[wib][s0 + j] : -1;
+          if (rs[j] >= 0) v[j] = rows[(size_t)rs[j] * width4 + c];
         }
-        const float4 v = rows[(size_t)r * width4 + c];
-        acc.x += v.x;
-        acc.y += v.y;
-        acc.z += v.z;
-        acc.w += v.w;
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          if (rs[j] >= 0) {
+            acc.x += v[j].x;
+            acc.y += v[j].y;
+            acc.z += v[j].z;
+            acc.w += v[j].w;
+          }
       }
       store4<TY>(y + ((size_t)t * width4 + c) * 4, acc);
     }
+    __syncwarp();  // srow is rewritten for the warp's next token
   }
 }
 
