@@ -28,6 +28,20 @@ namespace {
 // per launch so that the tiles fill whole waves of SMs (see pick_tg).
 constexpr int kBigBN = 128, kBigBK = 16;
 
+// (c0, c1) = (b0 * a + c0, b1 * a + c1), each a single-rounding fp32 fma:
+// the packed instruction gives the same results as two __fmaf_rn with half
+// the instructions to issue.
+__device__ __forceinline__ void fma2_rn(float& c0, float& c1, float b0, float b1, float a) {
+  asm("{\n\t.reg .b64 ra, rb, rc;\n\t"
+      "mov.b64 ra, {%2, %2};\n\t"
+      "mov.b64 rb, {%3, %4};\n\t"
+      "mov.b64 rc, {%0, %1};\n\t"
+      "fma.rn.f32x2 rc, rb, ra, rc;\n\t"
+      "mov.b64 {%0, %1}, rc;\n\t}"
+      : "+f"(c0), "+f"(c1)
+      : "f"(a), "f"(b0), "f"(b1));
+}
+
 template <typename TU, int TG>
 __global__ void __launch_bounds__(16 * TG)
     router_logits_big(const TU* __restrict__ u, const float* __restrict__ w,
@@ -102,7 +116,7 @@ __global__ void __launch_bounds__(16 * TG)
 #pragma unroll
       for (int i = 0; i < 8; ++i)
 #pragma unroll
-        for (int j = 0; j < 8; ++j) acc[i][j] = __fmaf_rn(b[j], a[i], acc[i][j]);
+        for (int j = 0; j < 8; j += 2) fma2_rn(acc[i][j], acc[i][j + 1], b[j], b[j + 1], a[i]);
     }
     if (more) {
       put(buf ^ 1);
