@@ -45,6 +45,10 @@ METRIC = "MoE-layer fwd tokens/s on 1 B200"
 PROFILED_TRAFFIC = {
     "small": {"bytes": 11571200 + 0, "src": "sparse_mixture_experts_15_b200/csrc/ffn_fused.cu",
               "sha1": "f01aa212595dfc284b7bf4a906467bdd015125b8", "profile": "profiles/tc_fused_ffn_small.md"},
+    # gate/up + down launches of one Mixtral-shaped step (read + write)
+    "mixtral": {"bytes": (3195234048 + 350338816) + (2617828096 + 188471808),
+                "src": "sparse_mixture_experts_15_b200/csrc/gemm_tc.cu",
+                "sha1": "014eb6f5782a25d799d999bb7701d50385021395", "profile": "profiles/tc_grouped_gemm_mixtral.md"},
 }
 
 
@@ -1032,7 +1036,7 @@ def main():
     tf_peak = tf_sust if long_loop else tf_burst
     roofline = {"bound": "tensor", "achieved": achieved_tf, "peak": tf_peak, "unit": "TFLOP/s",
                 "frac": achieved_tf / tf_peak, "frac_of_burst": achieved_tf / tf_burst,
-                "traffic": profiled_traffic(wl.name) if fused else None,
+                "traffic": profiled_traffic(wl.name),
                 "kernel": ("tc_fused_ffn (gate/up + SwiGLU + down in one launch, H on chip)"
                            if fused else "tc_grouped_gemm (gate/up + down, 2 launches per step)"),
                 "peak_source": (f"{peak_src} bf16_tflops_sustained (GEMM loop of "
