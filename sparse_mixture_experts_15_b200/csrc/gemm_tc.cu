@@ -4,6 +4,8 @@
 // §3.1 equation F and §3.6 (expert i works on its own [L_i, d] rows):
 //   gate/up:  H = act(X_e W_gate,e^T, X_e W_up,e^T)   -> bf16 [rows][h]
 //   down:     Y = H_e W_down,e^T                       -> fp32 [rows][width]
+//             (each row times its token's combine weight a in the layer path,
+//             so the combine only adds rows)
 //
 // Orientation: the expert WEIGHTS are the MMA's M operand (128 rows per tile)
 // and the expert's TOKENS are its N operand (up to BN per tile, rounded up to
