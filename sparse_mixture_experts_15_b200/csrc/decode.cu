@@ -429,6 +429,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_persistent(const __grid_co
 
   stage_rows(sm + P.wr0, ws_ld * 4, reinterpret_cast<const char*>(p.layer[0].w_route),
              (size_t)d * 4, N, d * 4);
+  // Block b's phase-A item of the next layer is staged during the first
+  // barrier when every expert is likely to be selected (T k >= N): with all
+  // N experts selected, block b's item is expert b / slicesA, slice
+  // b % slicesA.  `spec` says that aq / as hold that item for layer l.
+  bool spec = false;
   for (int l = 0; l < p.n_layers; ++l) {
     const LayerPtrs& L = p.layer[l];
     const bool last = l == p.n_layers - 1;
@@ -502,14 +507,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_persistent(const __grid_co
     // ---- issue this CTA's first phase-A item and the down rows of its first
     // phase-B slice together, before the first wait.
     const int nitems = nsel * slicesA;
-    auto stage_item = [&](int it) {
-      const int e = esel[it / slicesA], sl = it % slicesA;
+    auto stage_rows_of = [&](const LayerPtrs& Lx, int e, int sl) {
       const size_t row = (size_t)e * h + (size_t)sl * RA;
-      stage_bytes(aq, L.gq + row * (d / 2), RA * (d / 2));
-      stage_bytes(aq + RA * (d / 2), L.uq + row * (d / 2), RA * (d / 2));
-      stage_bytes(as, L.gs + row * nb, RA * nb * 2);
-      stage_bytes(as + RA * nb, L.us + row * nb, RA * nb * 2);
+      stage_bytes(aq, Lx.gq + row * (d / 2), RA * (d / 2));
+      stage_bytes(aq + RA * (d / 2), Lx.uq + row * (d / 2), RA * (d / 2));
+      stage_bytes(as, Lx.gs + row * nb, RA * nb * 2);
+      stage_bytes(as + RA * nb, Lx.us + row * nb, RA * nb * 2);
     };
+    auto stage_item = [&](int it) { stage_rows_of(L, esel[it / slicesA], it % slicesA); };
     // the down rows of phase-B unit un (token un / nsl, rows (un % nsl) RB..)
     // of the token's k selected experts, slot s at bq + s RB h/2
     auto stage_unit = [&](int un) {
@@ -524,7 +529,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_persistent(const __grid_co
     stamp(p, l, 3);
     // Separate cp.async groups: phase A waits for its gate/up rows only, not
     // for the down rows of the phase-B unit (needed after the barrier).
-    if (b < nitems) stage_item(b);
+    // (the speculative rows are already there when block b's item is the
+    // predicted one: experts 0 .. b / slicesA all selected)
+    if (b < nitems && !(spec && esel[b / slicesA] == b / slicesA)) stage_item(b);
     cp_commit();
     if (b < nunits) stage_unit(b);
     cp_commit();
@@ -628,6 +635,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_persistent(const __grid_co
       stage_rows(sm + ((l & 1) ? P.wr0 : P.wr1), ws_ld * 4,
                  reinterpret_cast<const char*>(p.layer[l + 1].w_route), (size_t)d * 4, N, d * 4);
     cp_commit();  // the router rows' own group: phase B does not wait for it
+    // aq / as are free until the next layer's phase A: stage block b's likely
+    // item of the next layer now (its own group, waited for at the next
+    // layer's start, not by phase B)
+    spec = !last && Tk >= N && b < N * slicesA;
+    if (spec) stage_rows_of(p.layer[l + 1], b / slicesA, b % slicesA);
+    cp_commit();
     if (!grid_wait(p.bar, (unsigned)G * ++n_bar, p.status)) {
       cp_wait_all();
       return;
@@ -643,7 +656,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_persistent(const __grid_co
         cp_commit();
         cp_wait_group<0>();
       } else {
-        cp_wait_group<1>();  // this unit's rows; the next router rows may still be in flight
+        cp_wait_group<2>();  // this unit's rows; the next router rows and item may be in flight
       }
       __syncthreads();
       if (un == b) stamp(p, l, 9);
