@@ -114,7 +114,21 @@ __global__ void __launch_bounds__(kQBThreads)
   __shared__ float s_red[2][kQBThreads / 32];
   int* bin_cnt = reinterpret_cast<int*>(keys + T);  // [bins]
   const int j = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  for (int i = tid; i < T; i += blockDim.x) keys[i] = fkey(__fsub_rn(a[i], s[(size_t)i * N + j]));
+  // required biases a_i - s_ij of column j: eight strided loads in flight per thread
+  for (int i0 = tid; i0 < T; i0 += 8 * blockDim.x) {
+    float sv[8], av[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int i = i0 + u * (int)blockDim.x;
+      sv[u] = i < T ? s[(size_t)i * N + j] : 0.0f;
+      av[u] = i < T ? a[i] : 0.0f;
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int i = i0 + u * (int)blockDim.x;
+      if (i < T) keys[i] = fkey(__fsub_rn(av[u], sv[u]));
+    }
+  }
   if (tid == 0) {
     s_prefix = 0;
     s_rem = q;
@@ -129,14 +143,34 @@ __global__ void __launch_bounds__(kQBThreads)
     __syncthreads();
     digit_counts(keys, T, s_prefix, mask, shift, hist);
     __syncthreads();
-    if (tid == 0) {
-      int rem = s_rem, dgt = 0;
-      for (; dgt < 255; ++dgt) {
-        if (hist[dgt] >= rem) break;
-        rem -= hist[dgt];
+    if (warp == 0) {
+      // the first digit whose cumulative count reaches rem (255 at most),
+      // and rem less the counts before it: lane l scans digits 8l .. 8l+7,
+      // a warp prefix sum finds the lane, that lane finds the digit
+      int v[8], sum = 0;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        v[i] = hist[lane * 8 + i];
+        sum += v[i];
       }
-      s_rem = rem;
-      s_prefix |= (uint32_t)dgt << shift;
+      int incl = sum;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int nb = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += nb;
+      }
+      const int rem = s_rem;
+      const unsigned hit = __ballot_sync(0xffffffffu, incl >= rem);
+      const int L = hit ? __ffs(hit) - 1 : 31;
+      if (lane == L) {
+        int r = rem - (incl - sum), dgt = lane * 8;
+        for (int i = 0; i < 8; ++i, ++dgt) {
+          if (dgt == 255 || v[i] >= r) break;
+          r -= v[i];
+        }
+        s_rem = r;
+        s_prefix |= (uint32_t)dgt << shift;
+      }
     }
     __syncthreads();
   }
@@ -193,14 +227,26 @@ __global__ void __launch_bounds__(kQBThreads)
     atomicAdd(&bin_cnt[cb], 1);
   }
   __syncthreads();
-  if (tid == 0) {
-    int cb = 0, cum = 0;
-    for (; cb < bins; ++cb) {
-      cum += bin_cnt[cb];
-      if (cum >= q) break;
+  if (warp == 0) {
+    // the first bin whose cumulative count reaches q (the last bin at most):
+    // 32 bins per step, a warp prefix sum with the running total carried
+    int cb = bins - 1, carry = 0;
+    for (int base = 0; base < bins; base += 32) {
+      const int c = base + lane < bins ? bin_cnt[base + lane] : 0;
+      int incl = c;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int nb = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += nb;
+      }
+      const unsigned hit = __ballot_sync(0xffffffffu, base + lane < bins && carry + incl >= q);
+      if (hit) {
+        cb = base + __ffs(hit) - 1;
+        break;
+      }
+      carry += __shfl_sync(0xffffffffu, incl, 31);
     }
-    if (cb > bins - 1) cb = bins - 1;
-    b_hist[j] = __fadd_rn(lo, __fmul_rn((float)(cb + 1), width));
+    if (lane == 0) b_hist[j] = __fadd_rn(lo, __fmul_rn((float)(cb + 1), width));
   }
 }
 
