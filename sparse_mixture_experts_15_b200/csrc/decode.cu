@@ -17,8 +17,8 @@
 //           expert.  (The next layer's router rows are fetched while the
 //           CTA waits at the first barrier.)
 //   phase A items (selected expert, RA hidden rows) are spread over the
-//           CTAs: the item's gate/up q4 rows are staged, dequantised once
-//           into shared fp32, and every (row, token) dot is formed;
+//           CTAs: the item's gate/up q4 rows are staged in shared memory
+//           and dequantised in registers inside the (row, token) dots;
 //           H[e][t][rows] = SiLU(g) * v goes to global memory (L2).
 //   barrier
 //   phase B units of (one token, RB output rows), T * d / RB of them: the
@@ -71,15 +71,6 @@ __device__ __forceinline__ void dequant_block(const uint8_t* qs, uint16_t scale,
   }
 }
 
-// Elements 4c..4c+3 of a q4_0 block (c < 4: low nibbles of bytes 4c..4c+3;
-// c >= 4: high nibbles of bytes 4(c-4)..).  Eight threads with consecutive c
-// write one block's 128 bytes as consecutive 16-byte pieces.
-__device__ __forceinline__ float4 dequant_quad(const uint8_t* qs, uint16_t scale, int c) {
-  const uint32_t word = reinterpret_cast<const uint32_t*>(qs)[c & 3];
-  const uint32_t v = (c < 4 ? word : word >> 4) & 0x0F0F0F0Fu;
-  const float s = f16f(scale);
-  return make_float4(nib(v, 0) * s, nib(v, 1) * s, nib(v, 2) * s, nib(v, 3) * s);
-}
 
 // Asynchronous global -> shared copies (LDGSTS), all issued before one wait.
 // The .cg form reads through L2 only, so data written by other CTAs of this
@@ -308,7 +299,7 @@ struct Plan {
   int nsel_max;  // experts a layer can select: min(N, T*k)
   int part_cap;  // floats of the phase-A partial-sum buffer
   uint32_t u, wr0, wr1, z, sel, aw, cnt, start, fill, list, esel, epos, misc;
-  uint32_t aq, as, deq, part, bq, bs, zs;
+  uint32_t aq, as, part, bq, bs, zs;
   uint32_t total;
 };
 
@@ -383,7 +374,6 @@ bool make_plan(const moe_shape& s, int sms, Plan* out) {
       p.misc = take(off, 16);
       p.aq = take(off, (size_t)2 * RA * (d / 2));
       p.as = take(off, (size_t)2 * RA * nb * 2);
-      p.deq = take(off, (size_t)2 * RA * (d + 4) * 4);
       p.part = take(off, (size_t)p.part_cap * 4);
       p.bq = take(off, (size_t)k * RB * (h / 2));
       p.bs = take(off, (size_t)k * RB * nbh * 2);
@@ -404,7 +394,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_persistent(const __grid_co
   const Plan& P = p.plan;
   const int T = p.T, d = p.d, N = p.N, k = p.k, h = p.h, Tk = T * k;
   const int RA = P.RA, RB = P.RB, nb = d / 32, nbh = h / 32;
-  const int us_ld = d + 8, ws_ld = d + 4, dq_ld = d + 4;
+  const int us_ld = d + 8, ws_ld = d + 4;
   const int G = gridDim.x, b = blockIdx.x, tid = threadIdx.x;
   __half* u_s = reinterpret_cast<__half*>(sm + P.u);
   float* z = reinterpret_cast<float*>(sm + P.z);
@@ -419,7 +409,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_persistent(const __grid_co
   int* nsel_s = reinterpret_cast<int*>(sm + P.misc);
   uint8_t* aq = reinterpret_cast<uint8_t*>(sm + P.aq);
   uint16_t* as = reinterpret_cast<uint16_t*>(sm + P.as);
-  float* deq = reinterpret_cast<float*>(sm + P.deq);
   float* part = reinterpret_cast<float*>(sm + P.part);
   uint8_t* bq = reinterpret_cast<uint8_t*>(sm + P.bq);
   uint16_t* bs = reinterpret_cast<uint16_t*>(sm + P.bs);
@@ -548,15 +537,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_persistent(const __grid_co
         cp_wait_group<1>();  // this item's group; the slice's may still be in flight
       }
       __syncthreads();
-      if (it == b) stamp(p, l, 4);
-      for (int x = tid; x < 2 * RA * nb * 8; x += blockDim.x) {  // 8 threads per block
-        const int blk = x >> 3, c = x & 7;
-        const int w = blk / nb, bb = blk - w * nb;
-        *reinterpret_cast<float4*>(deq + (size_t)w * dq_ld + bb * 32 + 4 * c) =
-            dequant_quad(aq + (size_t)w * (d / 2) + bb * 16, as[w * nb + bb], c);
+      if (it == b) {  // (the weights are dequantised in registers inside the dots)
+        stamp(p, l, 4);
+        stamp(p, l, 5);
       }
-      __syncthreads();
-      if (it == b) stamp(p, l, 5);
       // unit = (token pair, hidden row r, part of d): one thread forms the
       // gate and the up dot of row r for two tokens, so each weight and
       // activation it loads feeds two FMAs.  d is split into nparts so that
@@ -570,14 +554,28 @@ __global__ void __launch_bounds__(kThreads, 1) decode_persistent(const __grid_co
         const int r = rest % RA, pp = rest / RA;
         const int i0 = 2 * ip, i1 = i0 + 1 < ne ? i0 + 1 : i0;
         const int b0 = pp * nb / nparts, b1 = (pp + 1) * nb / nparts;
-        const float4* gw = reinterpret_cast<const float4*>(deq + (size_t)r * dq_ld);
-        const float4* vw = reinterpret_cast<const float4*>(deq + (size_t)(RA + r) * dq_ld);
+        // q4_0 rows r of gate and up: nibbles and block scales staged in
+        // shared memory, dequantised in registers 8 elements at a time
+        const uint8_t* gq_r = aq + (size_t)r * (d / 2);
+        const uint8_t* vq_r = aq + (size_t)(RA + r) * (d / 2);
+        const uint16_t* gs_r = as + (size_t)r * nb;
+        const uint16_t* vs_r = as + (size_t)(RA + r) * nb;
         const uint4* x0r = reinterpret_cast<const uint4*>(u_s + (size_t)toks[i0] * us_ld);
         const uint4* x1r = reinterpret_cast<const uint4*>(u_s + (size_t)toks[i1] * us_ld);
         float g0a = 0.f, g0b = 0.f, v0a = 0.f, v0b = 0.f, g1a = 0.f, g1b = 0.f, v1a = 0.f,
               v1b = 0.f;
         for (int c = b0 * 4; c < b1 * 4; ++c) {  // 8 elements per step
-          const float4 ga = gw[2 * c], gb = gw[2 * c + 1], va = vw[2 * c], vb = vw[2 * c + 1];
+          // elements 8c .. 8c+7: block c / 4, offset o = 8 (c % 4) in the
+          // block; byte j of a block holds element j (low nibble) and j + 16
+          // (high nibble)
+          const int blk = c >> 2, o = (c & 3) * 8;
+          const int byte0 = blk * 16 + (o & 15);
+          const uint2 gwd = *reinterpret_cast<const uint2*>(gq_r + byte0);
+          const uint2 vwd = *reinterpret_cast<const uint2*>(vq_r + byte0);
+          const float gsc = f16f(gs_r[blk]), vsc = f16f(vs_r[blk]);
+          const int sh = o >= 16 ? 4 : 0;
+          const uint32_t g_lo = (gwd.x >> sh) & 0x0F0F0F0Fu, g_hi = (gwd.y >> sh) & 0x0F0F0F0Fu;
+          const uint32_t v_lo = (vwd.x >> sh) & 0x0F0F0F0Fu, v_hi = (vwd.y >> sh) & 0x0F0F0F0Fu;
           const uint4 xu = x0r[c], yu = x1r[c];
           float x[8], y[8];
           const uint32_t xw[4] = {xu.x, xu.y, xu.z, xu.w}, yw[4] = {yu.x, yu.y, yu.z, yu.w};
@@ -590,8 +588,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_persistent(const __grid_co
             y[2 * q] = fy.x;
             y[2 * q + 1] = fy.y;
           }
-          const float gv[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
-          const float vv[8] = {va.x, va.y, va.z, va.w, vb.x, vb.y, vb.z, vb.w};
+          float gv[8], vv[8];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {  // (q - 8) s, exact in fp32
+            gv[q] = nib(g_lo, q) * gsc;
+            gv[4 + q] = nib(g_hi, q) * gsc;
+            vv[q] = nib(v_lo, q) * vsc;
+            vv[4 + q] = nib(v_hi, q) * vsc;
+          }
 #pragma unroll
           for (int q = 0; q < 8; q += 2) {
             g0a = fmaf(gv[q], x[q], g0a);
