@@ -256,3 +256,25 @@ def test_new_entry_points_reject_bad_arguments_on_the_host():
     assert lib.moe_layer_bwd_workspace_bytes(ctypes.byref(s)) > 0
     assert lib.moe_layer_bwd(ctypes.byref(s), None, None, None, None, 0.0, None, None, None, 0,
                              None) == -1
+
+
+@pytest.mark.parametrize("T,d,N,k,h,ok", [
+    (32, 512, 64, 8, 128, True),    # the decode GPU tests' shapes
+    (32, 1024, 8, 2, 256, True),
+    (5, 64, 4, 2, 32, True),
+    (3, 96, 4, 3, 64, True),
+    (1, 512, 8, 2, 128, True),
+    (32, 512, 8, 2, 1024, True),    # h / 32 = 32 parts
+    (33, 512, 8, 2, 128, False),    # T > 32
+    (32, 512, 65, 2, 128, False),   # N > 64
+    (32, 512, 64, 9, 128, False),   # k > 8
+    (32, 500, 8, 2, 128, False),    # d not a multiple of 32
+    (32, 512, 8, 2, 96, False),     # h / 32 = 3 does not divide 32
+    (32, 512, 8, 2, 2048, False),   # h / 32 = 64 parts
+    (32, 4096, 8, 2, 128, False),   # token rows alone exceed shared memory
+])
+def test_decode_shape_support_query(T, d, N, k, h, ok):
+    """The decode workspace query is the shape-support check: nonzero exactly
+    for the shapes the persistent kernel's shared-memory plan can hold."""
+    n = moe.moe_decode_workspace_bytes(moe.shape(T, d, N, k, h, 1, 0))
+    assert (n > 0) == ok
