@@ -221,13 +221,24 @@ uint16_t or_round_f16(double x) {
 /* ------------------------------------------------------------------- router */
 
 /* Router logit z = (W_route u)_i  [MoE tutorial] §3.2, formed in fp32.
- * The page fixes fp32 but not the summation order; the order used is the
- * plainest one: a single sequential chain of fused multiply-adds (one
- * rounding each) over j = 0 .. d-1 in ascending order, starting from +0. */
+ * The page fixes fp32 but not the summation order.  The order used is a
+ * blocked sum: the input index is cut into blocks of OR_ROUTER_BLOCK = 128
+ * consecutive elements (the last block may be shorter); each block's partial
+ * sum P_m is a chain of fused multiply-adds (one rounding each) over its
+ * elements in ascending order, starting from +0; z is then +0 plus P_0, plus
+ * P_1, ... in ascending block order, each addition rounded in fp32.  For
+ * d <= 128 this is the plain ascending chain. */
+enum { OR_ROUTER_BLOCK = 128 };
+
 float or_router_logit(const float* w, const float* u, int64_t d) {
-  float acc = 0.0f;
-  for (int64_t j = 0; j < d; ++j) acc = fmaf(w[j], u[j], acc);
-  return acc;
+  float z = 0.0f;
+  for (int64_t j0 = 0; j0 < d; j0 += OR_ROUTER_BLOCK) {
+    const int64_t j1 = j0 + OR_ROUTER_BLOCK < d ? j0 + OR_ROUTER_BLOCK : d;
+    float part = 0.0f;
+    for (int64_t j = j0; j < j1; ++j) part = fmaf(w[j], u[j], part);
+    z = z + part;
+  }
+  return z;
 }
 
 /* Routing of T tokens  [MoE tutorial] §3.2:

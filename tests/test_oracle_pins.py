@@ -68,14 +68,17 @@ def _exact_dot(w, u):
 
 
 def test_router_logit_within_fp32_bound():
-    """Sequential fp32 summation error bound: |z - exact| <= d * u * sum|w u| (u = 2^-24)."""
+    """Summation error bound of any order of d fp32 terms: |z - exact| <= d u sum|w u|
+    (u = 2^-24); the blocked order of 128-element chains meets the tighter
+    (128 + d / 128) u sum|w u|."""
     for d in (8, 64, 512, 4096):
         w = RNG.standard_normal(d).astype(np.float32)
         u = RNG.standard_normal(d).astype(np.float32)
         z = O.router_logit(w, u)
         exact = _exact_dot(w, u)
-        bound = (d + 1) * 2.0 ** -24 * float(np.sum(np.abs(w.astype(np.float64) * u)))
-        assert abs(z - exact) <= bound
+        mass = float(np.sum(np.abs(w.astype(np.float64) * u)))
+        assert abs(z - exact) <= (d + 1) * 2.0 ** -24 * mass
+        assert abs(z - exact) <= (min(d, 128) + (d + 127) // 128 + 1) * 2.0 ** -24 * mass
 
 
 def test_router_logit_integer_inputs_exact():
@@ -85,22 +88,38 @@ def test_router_logit_integer_inputs_exact():
 
 
 def test_router_logit_documented_order():
-    """Hand-worked values that only an ascending sequential sum produces.
+    """Hand-worked values that only the documented blocked order produces
+    (blocks of 128 elements, each an ascending chain from +0, block sums added
+    in ascending order).
 
-    [2^25, -2^25, 1]: ascending gives (2^25 - 2^25) + 1 = 1; descending gives
-    (1 - 2^25) -> -2^25 (ulp 4) then + 2^25 = 0.
-    [2^25, 1, -2^25] spread over the positions 0, 8, 128 of d = 256: ascending
-    gives 2^25 + 1 -> 2^25 then 0; a pairwise tree over 8-element chunks
-    would cancel the two big terms first and give 1.
+    Within one block the order is the ascending chain: [2^25, -2^25, 1] gives
+    (2^25 - 2^25) + 1 = 1; descending would give (1 - 2^25) -> -2^25 (ulp 4),
+    then + 2^25 = 0.
+    Across blocks (d = 256, block 0 = positions 0..127, block 1 = 128..255):
+    - 2^25 at 0, -2^25 at 128, 1 at 129: P_0 = 2^25, P_1 = -2^25 + 1 -> -2^25,
+      z = 0; one ascending chain over all 256 would give 1;
+    - 1 at 0, 2^25 at 128, -2^25 at 129: P_0 = 1, P_1 = 0, z = 1; one chain
+      would give (1 + 2^25 -> 2^25) - 2^25 = 0;
+    - 2^25 at 0, 1 at 8, -2^25 at 128: P_0 = 2^25 + 1 -> 2^25, z = 0; a
+      pairwise tree over 8-element chunks would cancel the big terms first
+      and give 1.
     """
     w = np.ones(3, np.float32)
     assert O.router_logit(w, np.array([2.0 ** 25, -(2.0 ** 25), 1.0], np.float32)) == 1.0
     assert O.router_logit(w, np.array([1.0, -(2.0 ** 25), 2.0 ** 25], np.float32)) == 1.0 - 1.0
     d = 256
     w = np.ones(d, np.float32)
-    u = np.zeros(d, np.float32)
-    u[0], u[8], u[128] = 2.0 ** 25, 1.0, -(2.0 ** 25)
-    assert O.router_logit(w, u) == 0.0
+    for pos, want in (({0: 2.0 ** 25, 128: -(2.0 ** 25), 129: 1.0}, 0.0),
+                      ({0: 1.0, 128: 2.0 ** 25, 129: -(2.0 ** 25)}, 1.0),
+                      ({0: 2.0 ** 25, 8: 1.0, 128: -(2.0 ** 25)}, 0.0)):
+        u = np.zeros(d, np.float32)
+        for j, v in pos.items():
+            u[j] = v
+        assert O.router_logit(w, u) == want
+    # a shorter last block: d = 200 = 128 + 72
+    u = np.zeros(200, np.float32)
+    u[127], u[128], u[199] = 1.0, 2.0 ** 25, -(2.0 ** 25)
+    assert O.router_logit(np.ones(200, np.float32), u) == 1.0
 
 
 def test_router_logit_uses_fused_multiply_add():
