@@ -109,8 +109,10 @@ MOE_API int moe_capacity(int64_t T, int32_t N, int32_t k, double factor, int32_t
  *   top_w    [T][k] fp32 out: a (renormalised when shape->renorm)
  *   probs    [T][N] fp32 out or NULL: softmax p
  *   logits   [T][N] fp32 out or NULL: z
- * z is a sequential fp32 fused-multiply-add chain over j = 0..d-1 (then + b),
- * so routing decisions are reproducible bit for bit.
+ * z is formed in one fixed fp32 order, so routing decisions are reproducible
+ * bit for bit: j = 0..d-1 is cut into blocks of 128 (the last may be
+ * shorter), each block sum is an ascending fused-multiply-add chain from +0,
+ * and z = +0 plus the block sums in ascending order (then + b).
  * Needs ws of moe_route_workspace_bytes(shape) bytes (may be 0 -> ws NULL). */
 MOE_API size_t moe_route_workspace_bytes(const moe_shape* shape);
 MOE_API int moe_route(const moe_shape* shape, const void* u, int32_t u_dtype, const float* w_route,

@@ -61,6 +61,26 @@ __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
 template <>
 __device__ __forceinline__ __half from_f32<__half>(float x) { return __float2half_rn(x); }
 
+// Router logits follow one fixed fp32 order: the input index is cut into
+// blocks of kRouteBlock consecutive elements; each block's partial sum is an
+// ascending chain of fused multiply-adds from +0, and the logit is +0 plus
+// the block sums in ascending block order (then + bias).
+constexpr int kRouteBlock = 128;
+
+// (c0, c1) = (b0 * a + c0, b1 * a + c1), each a single-rounding fp32 fma:
+// the packed instruction gives the same results as two __fmaf_rn with half
+// the instructions to issue.
+__device__ __forceinline__ void fma2_rn(float& c0, float& c1, float b0, float b1, float a) {
+  asm("{\n\t.reg .b64 ra, rb, rc;\n\t"
+      "mov.b64 ra, {%2, %2};\n\t"
+      "mov.b64 rb, {%3, %4};\n\t"
+      "mov.b64 rc, {%0, %1};\n\t"
+      "fma.rn.f32x2 rc, rb, ra, rc;\n\t"
+      "mov.b64 {%0, %1}, rc;\n\t}"
+      : "+f"(c0), "+f"(c1)
+      : "f"(a), "f"(b0), "f"(b1));
+}
+
 // Load 8 consecutive elements (16 B for 16-bit types, 32 B for fp32) as fp32.
 __device__ __forceinline__ void load8(const float* p, float* o) {
   float4 a = *reinterpret_cast<const float4*>(p);

@@ -146,130 +146,209 @@ __device__ __noinline__ void topk_wide(const float* zt, int N, int k, int renorm
   for (int s = 0; s < k; ++s) aw[s] = renorm ? a[s] / ps : a[s];
 }
 
-// Routing of all T tokens inside one CTA from u_s [T] rows (fp16, row stride
-// us_ld elements) and w_s [N] rows (fp32, stride ws_ld), both in shared
-// memory with a 16-byte pad per row so the threads of a warp (consecutive
-// (t, i) pairs) hit distinct banks.  z is the sequential fp32 FMA chain over
-// j (the order the oracle uses); the shared-memory operands of the next 8
-// elements are loaded while the current 8 FMAs run.  Ties go to the lower
-// expert index.  Leaves sel[t][s] and
-// aw[t][s] in shared memory.
-__device__ __forceinline__ void fma8(float& a, const uint4& xu, const float4& w0,
-                                     const float4& w1) {
-  const float2 x0 = __half22float2(*reinterpret_cast<const __half2*>(&xu.x));
-  const float2 x1 = __half22float2(*reinterpret_cast<const __half2*>(&xu.y));
-  const float2 x2 = __half22float2(*reinterpret_cast<const __half2*>(&xu.z));
-  const float2 x3 = __half22float2(*reinterpret_cast<const __half2*>(&xu.w));
-  a = __fmaf_rn(w0.x, x0.x, a);
-  a = __fmaf_rn(w0.y, x0.y, a);
-  a = __fmaf_rn(w0.z, x1.x, a);
-  a = __fmaf_rn(w0.w, x1.y, a);
-  a = __fmaf_rn(w1.x, x2.x, a);
-  a = __fmaf_rn(w1.y, x2.y, a);
-  a = __fmaf_rn(w1.z, x3.x, a);
-  a = __fmaf_rn(w1.w, x3.y, a);
-}
-
-// Softmax, top-k and combine weights of one token from its N logits zt.
+// Softmax, top-k and combine weights of one token from its N logits zt
+// (N <= NR).  The k largest logits in descending order, ties to the lower
+// index (the selection loop of the other router kernels).  With z_0 the
+// first selected logit (the largest) and e_i = exp(z_i - z_0): renormalised
+// weights a_s = e_s / sum of the selected e (e_0 = 1), otherwise a_s = e_s /
+// sum of all N e_i.  One reciprocal replaces the per-slot divisions, and the
+// slot loop is unrolled so the slots stay in registers: this code runs once
+// per layer on the critical path, where a dependent division costs about 90
+// cycles and a loop branch about 20.
 template <int NR>
 __device__ __forceinline__ void topk_token(const float* zt, int N, int k, int renorm, int* sel,
                                            float* aw) {
   float zr[NR];
 #pragma unroll
   for (int i = 0; i < NR; ++i) zr[i] = i < N ? zt[i] : 0.0f;
-  float zmax = -FLT_MAX;
-#pragma unroll
-  for (int i = 0; i < NR; ++i)
-    if (i < N) zmax = fmaxf(zmax, zr[i]);
-  float den = 0.0f;
-#pragma unroll
-  for (int i = 0; i < NR; ++i)
-    if (i < N) den += expf(zr[i] - zmax);
   uint32_t taken = 0;
-  float ps = 0.0f;
-  float a[8];
-  for (int s = 0; s < k; ++s) {
-    int bi = -1;
-    float bz = 0.0f;
+  int si[8];
+  float zs[8];
 #pragma unroll
-    for (int i = 0; i < NR; ++i)
-      if (i < N && !((taken >> i) & 1u) && (bi < 0 || zr[i] > bz)) {
-        bi = i;
-        bz = zr[i];
-      }
-    if (bi < 0) {  // only NaN logits left: take the lowest free index
-      bi = __ffs(~taken) - 1;
-      bz = zr[0];
+  for (int s = 0; s < 8; ++s) {
+    if (s < k) {
+      int bi = -1;
+      float bz = 0.0f;
 #pragma unroll
       for (int i = 0; i < NR; ++i)
-        if (i == bi) bz = zr[i];
+        if (i < N && !((taken >> i) & 1u) && (bi < 0 || zr[i] > bz)) {
+          bi = i;
+          bz = zr[i];
+        }
+      if (bi < 0) {  // only NaN logits left: take the lowest free index
+        bi = __ffs(~taken) - 1;
+#pragma unroll
+        for (int i = 0; i < NR; ++i)
+          if (i == bi) bz = zr[i];
+      }
+      taken |= 1u << bi;
+      si[s] = bi;
+      zs[s] = bz;
     }
-    taken |= 1u << bi;
-    sel[s] = bi;
-    a[s] = expf(bz - zmax) / den;
-    ps += a[s];
   }
-  for (int s = 0; s < k; ++s) aw[s] = renorm ? a[s] / ps : a[s];
+  const float z0 = zs[0];
+  float e[8], S = 0.0f;
+#pragma unroll
+  for (int s = 0; s < 8; ++s)
+    if (s < k) {
+      e[s] = expf(zs[s] - z0);
+      S += e[s];
+    }
+  if (!renorm) {
+    S = 0.0f;
+#pragma unroll
+    for (int i = 0; i < NR; ++i)
+      if (i < N) S += expf(zr[i] - z0);
+  }
+  const float r = 1.0f / S;
+#pragma unroll
+  for (int s = 0; s < 8; ++s)
+    if (s < k) {
+      sel[s] = si[s];
+      aw[s] = e[s] * r;
+    }
 }
 
+// The same selection and weights for N = 8 experts, top-2 (the common decode
+// shape), with the logits in registers: one pass keeps the best two in the
+// order of the selection loop (larger z first, ties to the lower index, and
+// a NaN held only where that loop would hold it).
+__device__ __forceinline__ void topk8_k2(const float* zt, int renorm, int* sel, float* aw) {
+  const float4 za = *reinterpret_cast<const float4*>(zt);
+  const float4 zb = *reinterpret_cast<const float4*>(zt + 4);
+  const float zr[8] = {za.x, za.y, za.z, za.w, zb.x, zb.y, zb.z, zb.w};
+  int b0 = 0, b1 = -1;
+  float z0 = zr[0], z1 = 0.0f;
+#pragma unroll
+  for (int i = 1; i < 8; ++i) {
+    if (zr[i] > z0) {
+      b1 = b0;
+      z1 = z0;
+      b0 = i;
+      z0 = zr[i];
+    } else if (b1 < 0 || zr[i] > z1) {
+      b1 = i;
+      z1 = zr[i];
+    }
+  }
+  const float e1 = expf(z1 - z0);
+  float S = 1.0f + e1;
+  if (!renorm) {
+    S = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) S += expf(zr[i] - z0);
+  }
+  const float r = 1.0f / S;
+  sel[0] = b0;
+  sel[1] = b1;
+  aw[0] = expf(z0 - z0) * r;
+  aw[1] = e1 * r;
+}
+
+// Block sums of the router logits: unit (token t, block m, expert group g of
+// E) runs the group's E chains over the block's kRouteBlock inputs, with the
+// next 8 inputs' shared-memory operands loaded while the current 8 FMAs of
+// each chain run.  The units of a warp are consecutive tokens of one (m, g),
+// so router-row reads are broadcasts and activation reads (rows padded 16 B
+// past a multiple of 128 B) hit distinct banks.  Results go to zp [m][N][T].
+template <int E>
+__device__ __forceinline__ void route_chains(const __half* u_s, int us_ld, const float* w_s,
+                                             int ws_ld, int T, int d, int N, float* zp) {
+  const int nblk = (d + kRouteBlock - 1) / kRouteBlock, ng = (N + E - 1) / E;
+  const int units = T * ng * nblk;
+  for (int uu = threadIdx.x; uu < units; uu += blockDim.x) {
+    const int t = uu % T, r = uu / T, g = r % ng, m = r / ng;
+    const int j0 = m * kRouteBlock, steps = min(kRouteBlock, d - j0) / 8;
+    const int e0 = E * g, nv = min(E, N - e0);
+    const uint4* ut = reinterpret_cast<const uint4*>(u_s + (size_t)t * us_ld + j0);
+    const float4* wr[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e)
+      wr[e] = reinterpret_cast<const float4*>(w_s + (size_t)(e0 + min(e, nv - 1)) * ws_ld + j0);
+    float c[E];
+    float4 wa[E], wb[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      c[e] = 0.0f;
+      wa[e] = wr[e][0];
+      wb[e] = wr[e][1];
+    }
+    uint4 xu = ut[0];
+    for (int st = 0; st < steps; ++st) {
+      const int sn = st + 1 < steps ? st + 1 : st;  // the next step (a repeat at the end)
+      const uint4 nxu = ut[sn];
+      float4 na[E], nb[E];
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        na[e] = wr[e][2 * sn];
+        nb[e] = wr[e][2 * sn + 1];
+      }
+      const uint32_t xw[4] = {xu.x, xu.y, xu.z, xu.w};
+      float x[8];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&xw[q]));
+        x[2 * q] = f.x;
+        x[2 * q + 1] = f.y;
+      }
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        c[e] = __fmaf_rn(wa[e].x, x[0], c[e]);
+        c[e] = __fmaf_rn(wa[e].y, x[1], c[e]);
+        c[e] = __fmaf_rn(wa[e].z, x[2], c[e]);
+        c[e] = __fmaf_rn(wa[e].w, x[3], c[e]);
+        c[e] = __fmaf_rn(wb[e].x, x[4], c[e]);
+        c[e] = __fmaf_rn(wb[e].y, x[5], c[e]);
+        c[e] = __fmaf_rn(wb[e].z, x[6], c[e]);
+        c[e] = __fmaf_rn(wb[e].w, x[7], c[e]);
+        wa[e] = na[e];
+        wb[e] = nb[e];
+      }
+      xu = nxu;
+    }
+#pragma unroll
+    for (int e = 0; e < E; ++e)
+      if (e < nv) zp[((size_t)m * N + e0 + e) * T + t] = c[e];
+  }
+}
+
+// Routing of all T tokens inside one CTA from u_s [T] rows (fp16, row stride
+// us_ld elements) and w_s [N] rows (fp32, stride ws_ld), both in shared
+// memory.  The logits follow the blocked order of kRouteBlock-element
+// chains: the block sums come from route_chains, with the smallest expert
+// group E that still gives every thread at most one unit (fewer chains per
+// thread, shorter dependent work), then each logit adds its blocks in
+// ascending order.  When zb_g is given, the block sums were already formed
+// by the previous layer's phase B (global [nblk][N][T], read through L2) and
+// neither u_s nor w_s is read.  Ties go to the lower expert index.  Leaves
+// sel[t][s] and aw[t][s] in shared memory.
 __device__ void route_in_cta(const __half* u_s, int us_ld, const float* w_s, int ws_ld, int T,
                              int d, int N, int k, int renorm, const float* __restrict__ bias,
-                             float* z, int* sel, float* aw) {
-  const int steps = d / 8;
-  if (T >= 16) {
-    // a thread forms the chains of two experts (i, i + 1) for one token, so
-    // each activation load feeds both; a warp holds 32 tokens of one expert
-    // pair, whose router rows are shared-memory broadcasts.
-    const int npair = (N + 1) / 2, units = T * npair;
-    for (int uu = threadIdx.x; uu < units; uu += blockDim.x) {
-      const int ip = uu / T, t = uu - ip * T;
-      const int i0 = 2 * ip, i1 = i0 + 1 < N ? i0 + 1 : i0;
-      const uint4* ut = reinterpret_cast<const uint4*>(u_s + (size_t)t * us_ld);
-      const float4* w0r = reinterpret_cast<const float4*>(w_s + (size_t)i0 * ws_ld);
-      const float4* w1r = reinterpret_cast<const float4*>(w_s + (size_t)i1 * ws_ld);
-      float a = 0.0f, b = 0.0f;
-      uint4 xu = ut[0];
-      float4 wa0 = w0r[0], wa1 = w0r[1], wb0 = w1r[0], wb1 = w1r[1];
-      for (int c = 0; c + 1 < steps; ++c) {
-        const uint4 nxu = ut[c + 1];
-        const float4 nwa0 = w0r[2 * c + 2], nwa1 = w0r[2 * c + 3];
-        const float4 nwb0 = w1r[2 * c + 2], nwb1 = w1r[2 * c + 3];
-        fma8(a, xu, wa0, wa1);
-        fma8(b, xu, wb0, wb1);
-        xu = nxu;
-        wa0 = nwa0;
-        wa1 = nwa1;
-        wb0 = nwb0;
-        wb1 = nwb1;
-      }
-      fma8(a, xu, wa0, wa1);
-      fma8(b, xu, wb0, wb1);
-      z[t * N + i0] = bias ? __fadd_rn(a, bias[i0]) : a;
-      if (i1 != i0) z[t * N + i1] = bias ? __fadd_rn(b, bias[i1]) : b;
-    }
-  } else {
-    for (int p = threadIdx.x; p < T * N; p += blockDim.x) {
-      const int t = p / N, i = p - t * N;
-      const uint4* ut = reinterpret_cast<const uint4*>(u_s + (size_t)t * us_ld);
-      const float4* wi = reinterpret_cast<const float4*>(w_s + (size_t)i * ws_ld);
-      float a = 0.0f;
-      uint4 xu = ut[0];
-      float4 w0 = wi[0], w1 = wi[1];
-      for (int c = 0; c + 1 < steps; ++c) {  // next 8 elements loaded under this step's FMAs
-        const uint4 nxu = ut[c + 1];
-        const float4 nw0 = wi[2 * c + 2], nw1 = wi[2 * c + 3];
-        fma8(a, xu, w0, w1);
-        xu = nxu;
-        w0 = nw0;
-        w1 = nw1;
-      }
-      fma8(a, xu, w0, w1);
-      z[p] = bias ? __fadd_rn(a, bias[i]) : a;
-    }
+                             float* z, float* zp, const float* zb_g, int* sel, float* aw) {
+  const int nblk = (d + kRouteBlock - 1) / kRouteBlock, nt = blockDim.x;
+  if (!zb_g) {
+    if (T * N * nblk <= nt)
+      route_chains<1>(u_s, us_ld, w_s, ws_ld, T, d, N, zp);
+    else if (T * ((N + 1) / 2) * nblk <= nt)
+      route_chains<2>(u_s, us_ld, w_s, ws_ld, T, d, N, zp);
+    else
+      route_chains<4>(u_s, us_ld, w_s, ws_ld, T, d, N, zp);
+    __syncthreads();
+  }
+  for (int q = threadIdx.x; q < T * N; q += blockDim.x) {
+    const int i = q / T, t = q - i * T;
+    float zz = 0.0f;
+    if (zb_g)
+      for (int m = 0; m < nblk; ++m) zz = __fadd_rn(zz, __ldcg(zb_g + ((size_t)m * N + i) * T + t));
+    else
+      for (int m = 0; m < nblk; ++m) zz = __fadd_rn(zz, zp[((size_t)m * N + i) * T + t]);
+    z[t * N + i] = bias ? __fadd_rn(zz, bias[i]) : zz;
   }
   __syncthreads();
   for (int t = threadIdx.x; t < T; t += blockDim.x) {
-    if (N <= 8)
+    if (N == 8 && k == 2)
+      topk8_k2(z + t * N, renorm, sel + t * k, aw + t * k);
+    else if (N <= 8)
       topk_token<8>(z + t * N, N, k, renorm, sel + t * k, aw + t * k);
     else if (N <= 32)
       topk_token<32>(z + t * N, N, k, renorm, sel + t * k, aw + t * k);
@@ -298,6 +377,8 @@ struct Plan {
   int nbuf;      // router-weight buffers (2: next layer prefetched)
   int nsel_max;  // experts a layer can select: min(N, T*k)
   int part_cap;  // floats of the phase-A partial-sum buffer
+  int early;     // 1: phase B forms the next layer's router block sums (RB a
+                 // multiple of kRouteBlock, next router rows prefetched)
   uint32_t u, wr0, wr1, z, sel, aw, cnt, start, fill, list, esel, epos, misc;
   uint32_t aq, as, part, bq, bs, zs;
   uint32_t total;
@@ -315,6 +396,7 @@ struct Params {
   int32_t* top_idx;     // [n_layers][T][k] (nullable)
   float* top_w;         // [T][k] of the last layer (nullable)
   float* H;             // [N][T][h] fp32 scratch
+  float* zb;            // [d / kRouteBlock][N][T] next layer's router block sums
   unsigned* bar;        // [0] arrivals, [1] abort
   int* status;
   unsigned long long* stamps;  // nullable: [n_layers][kStamps] SM cycle stamps of CTA 0
@@ -357,7 +439,12 @@ bool make_plan(const moe_shape& s, int sms, Plan* out) {
       p.RB = RB;
       p.nbuf = nbuf;
       p.nsel_max = nsel_max;
-      p.part_cap = 2048 + 4 * RA * T;  // >= 2 (g, v) x units x 2 tokens
+      // >= 2 (g, v) x units x 2 tokens; the routing's block sums share it
+      p.part_cap = 2048 + 4 * RA * T;
+      const int route_parts = T * N * ((d + kRouteBlock - 1) / kRouteBlock);
+      if (p.part_cap < route_parts) p.part_cap = route_parts;
+      if (p.part_cap < RB) p.part_cap = RB;  // phase B's u_next rows (fp32)
+      p.early = nbuf == 2 && RB % kRouteBlock == 0 && d % kRouteBlock == 0;
       uint32_t off = 0;
       p.u = take(off, (size_t)T * (d + 8) * 2);
       p.wr0 = take(off, (size_t)N * (d + 4) * 4);
@@ -436,12 +523,23 @@ __global__ void __launch_bounds__(kThreads, 1) decode_persistent(const __grid_co
     stage_rows(reinterpret_cast<char*>(u_s), us_ld * 2, reinterpret_cast<const char*>(u_cur),
                (size_t)d * 2, T, d * 2);
     for (int e = tid; e < N; e += blockDim.x) cnt[e] = 0;
-    cp_wait_all();
-    __syncthreads();
-    stamp(p, l, 1);
-
-    // ---- routing (every CTA), then the pairs grouped by expert
-    route_in_cta(u_s, us_ld, wr_s, ws_ld, T, d, N, k, p.renorm, L.bias, z, sel, aw);
+    // ---- routing (every CTA), then the pairs grouped by expert.  With the
+    // block sums formed by the previous layer's phase B, routing runs while
+    // u_l is still being staged (and stamps 1 and 2 both follow it).
+    const bool early = P.early && l > 0;
+    if (early) {
+      __syncthreads();
+      route_in_cta(u_s, us_ld, wr_s, ws_ld, T, d, N, k, p.renorm, L.bias, z, part, p.zb, sel, aw);
+      cp_wait_all();
+      __syncthreads();
+      stamp(p, l, 1);
+    } else {
+      cp_wait_all();
+      __syncthreads();
+      stamp(p, l, 1);
+      route_in_cta(u_s, us_ld, wr_s, ws_ld, T, d, N, k, p.renorm, L.bias, z, part, nullptr, sel,
+                   aw);
+    }
     stamp(p, l, 2);
     if (b == 0) {
       for (int x = tid; x < Tk; x += blockDim.x) {
@@ -714,13 +812,40 @@ __global__ void __launch_bounds__(kThreads, 1) decode_persistent(const __grid_co
       }
       __syncthreads();
       if (un == b) stamp(p, l, 10);
+      const bool early_next = P.early && !last;
       for (int r = tid; r < RB; r += blockDim.x) {
         float acc = 0.0f;
         for (int q = 0; q < k; ++q) acc = fmaf(aw[t * k + q], zs[q * (RB + 1) + r], acc);
         const int m = sl * RB + r;
         const size_t o = (size_t)t * d + m;
         if (last && p.y) p.y[o] = __float2half_rn(acc);
-        if (u_next) u_next[o] = __float2half_rn(__half2float(u_s[(size_t)t * us_ld + m]) + acc);
+        const __half un = __float2half_rn(__half2float(u_s[(size_t)t * us_ld + m]) + acc);
+        if (u_next) u_next[o] = un;
+        if (early_next) part[r] = __half2float(un);
+      }
+      if (early_next) {
+        // the next layer's router block sums of this unit's kRouteBlock-wide
+        // blocks of u_{l+1}[t]: one ascending FMA chain per (expert, block)
+        // over the prefetched router rows, stored for every CTA to read
+        cp_wait_group<1>();  // the next router rows (the speculative item may be in flight)
+        __syncthreads();
+        const float* wn = reinterpret_cast<const float*>(sm + ((l & 1) ? P.wr0 : P.wr1));
+        for (int q = tid; q < N * (RB / kRouteBlock); q += blockDim.x) {
+          const int i = q % N, mb = q / N;
+          const int j0 = sl * RB + mb * kRouteBlock;
+          const float4* w4 = reinterpret_cast<const float4*>(wn + (size_t)i * ws_ld + j0);
+          const float4* x4 = reinterpret_cast<const float4*>(part + mb * kRouteBlock);
+          float c = 0.0f;
+#pragma unroll 8
+          for (int s4 = 0; s4 < kRouteBlock / 4; ++s4) {
+            const float4 w = w4[s4], x = x4[s4];
+            c = __fmaf_rn(w.x, x.x, c);
+            c = __fmaf_rn(w.y, x.y, c);
+            c = __fmaf_rn(w.z, x.z, c);
+            c = __fmaf_rn(w.w, x.w, c);
+          }
+          p.zb[((size_t)(j0 / kRouteBlock) * N + i) * T + t] = c;
+        }
       }
       __syncthreads();
     }
@@ -739,6 +864,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_persistent(const __grid_co
 // ------------------------------------------------------------------ host
 struct WsLayout {
   float* H;
+  float* zb;
   int32_t* idx;
   float* w;
   __half* work;
@@ -750,6 +876,7 @@ WsLayout carve_decode(const moe_shape& s, void* base) {
   Carver c(base);
   WsLayout L;
   L.H = c.take<float>((size_t)s.N * s.T * s.h);
+  L.zb = c.take<float>((size_t)((s.d + kRouteBlock - 1) / kRouteBlock) * s.N * s.T);
   L.idx = c.take<int32_t>((size_t)s.T * s.k);
   L.w = c.take<float>((size_t)s.T * s.k);
   L.work = c.take<__half>((size_t)s.T * s.d);
@@ -837,6 +964,7 @@ int launch_decode(const moe_shape& s, const moe_q4_layer* layers, int n, const _
   p.top_idx = top_idx;
   p.top_w = top_w;
   p.H = W.H;
+  p.zb = W.zb;
   p.bar = W.bar;
   p.status = status_word();
   p.stamps = stamps;

@@ -5,8 +5,10 @@
 //
 // Logits are a register-tiled SIMT GEMM: each thread owns 8 tokens x 8
 // experts and walks the input dimension in ascending order with one fused
-// multiply-add per step, so every logit is the same sequential fp32 chain
-// whatever the tiling (the reproducible order the routing decision needs).
+// multiply-add per step into a block partial, which it adds to the logit at
+// each kRouteBlock boundary, so every logit follows the same blocked fp32
+// order whatever the tiling (the reproducible order the routing decision
+// needs).
 // Top-k runs one warp per token with the logits in registers.  With at most
 // 16 experts a single fused kernel (router_fused_small) does all of it.
 #include <cfloat>
@@ -20,27 +22,13 @@ namespace {
 // Many experts (N > 16): a block tile of 8 TG tokens x 128 experts with
 // 16 TG threads, 8 x 8 logits per thread, K walked in steps of 16 through
 // double-buffered shared tiles (the next step's global loads are held in
-// registers while the current step computes).  Each logit is still one
-// thread's FMA chain over j in ascending order, so the result equals the
-// other router kernels bit for bit.  A thread's tokens are {4 ty + i,
+// registers while the current step computes).  Each logit's block partials
+// are one thread's FMA chains, added to the logit after every 128 inputs,
+// so the result equals the other router kernels bit for bit.  A thread's tokens are {4 ty + i,
 // 4 TG + 4 ty + i} and its experts {4 tx + j, 64 + 4 tx + j}, so the 16-byte
 // shared reads of a warp are broadcasts or consecutive.  TG (8..16) is picked
 // per launch so that the tiles fill whole waves of SMs (see pick_tg).
 constexpr int kBigBN = 128, kBigBK = 16;
-
-// (c0, c1) = (b0 * a + c0, b1 * a + c1), each a single-rounding fp32 fma:
-// the packed instruction gives the same results as two __fmaf_rn with half
-// the instructions to issue.
-__device__ __forceinline__ void fma2_rn(float& c0, float& c1, float b0, float b1, float a) {
-  asm("{\n\t.reg .b64 ra, rb, rc;\n\t"
-      "mov.b64 ra, {%2, %2};\n\t"
-      "mov.b64 rb, {%3, %4};\n\t"
-      "mov.b64 rc, {%0, %1};\n\t"
-      "fma.rn.f32x2 rc, rb, ra, rc;\n\t"
-      "mov.b64 {%0, %1}, rc;\n\t}"
-      : "+f"(c0), "+f"(c1)
-      : "f"(a), "f"(b0), "f"(b1));
-}
 
 template <typename TU, int TG>
 __global__ void __launch_bounds__(16 * TG)
@@ -54,11 +42,18 @@ __global__ void __launch_bounds__(16 * TG)
   __shared__ __align__(16) float wsm[2][kBigBK][kBigBN];
   const int t0 = blockIdx.x * BT, n0 = blockIdx.y * kBigBN;
   const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
-  float acc[8][8];
+  static_assert(kRouteBlock % kBigBK == 0, "K steps must not straddle a route block");
+  // the 64 running logits of a thread live in shared memory (its own float4
+  // column of acc_s [16][NT], so no synchronisation), the current block's
+  // partials in registers
+  extern __shared__ float4 acc_s[];
+  float part[8][8];
 #pragma unroll
   for (int i = 0; i < 8; ++i)
 #pragma unroll
-    for (int j = 0; j < 8; ++j) acc[i][j] = 0.0f;
+    for (int j = 0; j < 8; ++j) part[i][j] = 0.0f;
+#pragma unroll
+  for (int q = 0; q < 16; ++q) acc_s[q * NT + tid] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
   // a K step's loads: token row tid >> 1 (8 columns at (tid & 1) * 8), and
   // expert rows (tid + q NT) >> 1 for q < WU
   float ru[8], rw[WU][8];
@@ -116,7 +111,20 @@ __global__ void __launch_bounds__(16 * TG)
 #pragma unroll
       for (int i = 0; i < 8; ++i)
 #pragma unroll
-        for (int j = 0; j < 8; j += 2) fma2_rn(acc[i][j], acc[i][j + 1], b[j], b[j + 1], a[i]);
+        for (int j = 0; j < 8; j += 2) fma2_rn(part[i][j], part[i][j + 1], b[j], b[j + 1], a[i]);
+    }
+    if (!more || (k0 + kBigBK) % kRouteBlock == 0) {  // a block ends: add its partials
+#pragma unroll
+      for (int q = 0; q < 16; ++q) {
+        float* pq = &part[q >> 1][(q & 1) * 4];
+        float4 v = acc_s[q * NT + tid];
+        v.x = __fadd_rn(v.x, pq[0]);
+        v.y = __fadd_rn(v.y, pq[1]);
+        v.z = __fadd_rn(v.z, pq[2]);
+        v.w = __fadd_rn(v.w, pq[3]);
+        acc_s[q * NT + tid] = v;
+        pq[0] = pq[1] = pq[2] = pq[3] = 0.0f;
+      }
     }
     if (more) {
       put(buf ^ 1);
@@ -128,10 +136,12 @@ __global__ void __launch_bounds__(16 * TG)
   for (int i = 0; i < 8; ++i) {
     const int t = t0 + (i < 4 ? 4 * ty + i : HALF + 4 * ty + i - 4);
     if (t >= T) continue;
+    const float4 v0 = acc_s[(2 * i) * NT + tid], v1 = acc_s[(2 * i + 1) * NT + tid];
+    const float zi[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       const int n = n0 + (j < 4 ? 4 * tx + j : 64 + 4 * tx + j - 4);
-      if (n < N) z[(size_t)t * N + n] = bias ? __fadd_rn(acc[i][j], bias[n]) : acc[i][j];
+      if (n < N) z[(size_t)t * N + n] = bias ? __fadd_rn(zi[j], bias[n]) : zi[j];
     }
   }
 }
@@ -238,9 +248,27 @@ __global__ void __launch_bounds__(256)
   }
 }
 
+// One 8-element step of a block chain: c = w[j] x[j] + c for j ascending.
+template <typename TU>
+__device__ __forceinline__ float dot8(float c, const TU* x, const float* w) {
+  float xv[8];
+  load8(x, xv);
+  const float4 w0 = *reinterpret_cast<const float4*>(w);
+  const float4 w1 = *reinterpret_cast<const float4*>(w + 4);
+  c = __fmaf_rn(w0.x, xv[0], c);
+  c = __fmaf_rn(w0.y, xv[1], c);
+  c = __fmaf_rn(w0.z, xv[2], c);
+  c = __fmaf_rn(w0.w, xv[3], c);
+  c = __fmaf_rn(w1.x, xv[4], c);
+  c = __fmaf_rn(w1.y, xv[5], c);
+  c = __fmaf_rn(w1.z, xv[6], c);
+  c = __fmaf_rn(w1.w, xv[7], c);
+  return c;
+}
+
 // Few experts (N <= NP <= 16): a block routes 128 / NP tokens with one
-// thread per (token, expert) pair, each running its logit's sequential FMA
-// chain over j (the same order as the tiled kernel), then one thread per
+// thread per (token, expert) pair, each running its logit's block chains
+// over j (the same order as the tiled kernel), then one thread per
 // token does softmax, top-k and the combine weights from shared memory, so
 // routing is a single launch.  Per slab of inputs the block's token rows and
 // the router rows are copied with cp.async (every copy issued before one
@@ -297,19 +325,20 @@ __global__ void __launch_bounds__(kRouteThreads)
     if (t < T && e < N) {
       const TU* ut = reinterpret_cast<const TU*>(us + tl * kRowBytes);
       const float* wt = ws[e];
-      for (int j = 0; j < kw; j += 8) {
-        float x[8];
-        load8(ut + j, x);
-        const float4 w0 = *reinterpret_cast<const float4*>(wt + j);
-        const float4 w1 = *reinterpret_cast<const float4*>(wt + j + 4);
-        acc = __fmaf_rn(w0.x, x[0], acc);
-        acc = __fmaf_rn(w0.y, x[1], acc);
-        acc = __fmaf_rn(w0.z, x[2], acc);
-        acc = __fmaf_rn(w0.w, x[3], acc);
-        acc = __fmaf_rn(w1.x, x[4], acc);
-        acc = __fmaf_rn(w1.y, x[5], acc);
-        acc = __fmaf_rn(w1.z, x[6], acc);
-        acc = __fmaf_rn(w1.w, x[7], acc);
+      if (kSlab == 2 * kRouteBlock && kw == kSlab) {  // two blocks, chains interleaved
+        float c0 = 0.0f, c1 = 0.0f;
+        for (int j = 0; j < kRouteBlock; j += 8) {
+          c0 = dot8(c0, ut + j, wt + j);
+          c1 = dot8(c1, ut + kRouteBlock + j, wt + kRouteBlock + j);
+        }
+        acc = __fadd_rn(__fadd_rn(acc, c0), c1);
+      } else {
+        for (int jb = 0; jb < kw; jb += kRouteBlock) {
+          const int je = min(jb + kRouteBlock, kw);
+          float c = 0.0f;
+          for (int j = jb; j < je; j += 8) c = dot8(c, ut + j, wt + j);
+          acc = __fadd_rn(acc, c);
+        }
       }
     }
   }
@@ -358,8 +387,17 @@ template <typename TU, int TG>
 void launch_logits_tg(const TU* u, const float* w, const float* bias, float* z, int T, int d,
                       int N, cudaStream_t st) {
   dim3 grid((T + 8 * TG - 1) / (8 * TG), (N + kBigBN - 1) / kBigBN);
-  MOE_PREFER_SHARED((router_logits_big<TU, TG>));
-  launch_pdl(router_logits_big<TU, TG>, grid, dim3(16 * TG), 0, st, u, w, bias, z, T, d, N);
+  const size_t smem = (size_t)64 * 4 * 16 * TG;  // acc_s: 64 fp32 logits per thread
+  static std::atomic<bool> configured[kMaxDevices];
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (device_slot(dev) && needs_setup(configured, dev)) {
+    MOE_PREFER_SHARED((router_logits_big<TU, TG>));
+    cudaFuncSetAttribute(router_logits_big<TU, TG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)smem);
+    mark_setup(configured, dev);
+  }
+  launch_pdl(router_logits_big<TU, TG>, grid, dim3(16 * TG), smem, st, u, w, bias, z, T, d, N);
 }
 
 template <typename TU>

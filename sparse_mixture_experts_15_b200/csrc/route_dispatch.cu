@@ -5,8 +5,9 @@
 //
 // CTA b owns the contiguous tokens [b tpc, (b + 1) tpc):
 //   phase 1  stage its token rows and the router rows in shared memory, run
-//            every (token, expert) logit as the sequential fp32 FMA chain
-//            over j (the order of the other router kernels and the oracle),
+//            every (token, expert) logit in the blocked fp32 order of
+//            kRouteBlock-element FMA chains (the order of the other router
+//            kernels and the oracle),
 //            softmax / top-k / weights with one thread per token, and count
 //            its dispatches per expert -> hist[b][e].
 //   barrier  (bounded, grid-wide)
@@ -163,8 +164,29 @@ __global__ void __launch_bounds__(kRDThreads, 1) route_dispatch(const __grid_con
     const int tl = q / N, i = q - tl * N;
     const TU* x = reinterpret_cast<const TU*>(us + tl * ub);
     const float* wi = ws + i * wld;
+    // blocked order: four blocks' chains at a time (independent, so their
+    // FMAs overlap), each block sum added in ascending order
     float a = 0.0f;
-    for (int j = 0; j < d; j += 8) a = dot8_chain(a, x + j, wi + j);
+    int j0 = 0;
+    for (; j0 + 4 * kRouteBlock <= d; j0 += 4 * kRouteBlock) {
+      float c0 = 0.0f, c1 = 0.0f, c2 = 0.0f, c3 = 0.0f;
+      for (int j = j0; j < j0 + kRouteBlock; j += 8) {
+        c0 = dot8_chain(c0, x + j, wi + j);
+        c1 = dot8_chain(c1, x + j + kRouteBlock, wi + j + kRouteBlock);
+        c2 = dot8_chain(c2, x + j + 2 * kRouteBlock, wi + j + 2 * kRouteBlock);
+        c3 = dot8_chain(c3, x + j + 3 * kRouteBlock, wi + j + 3 * kRouteBlock);
+      }
+      a = __fadd_rn(a, c0);
+      a = __fadd_rn(a, c1);
+      a = __fadd_rn(a, c2);
+      a = __fadd_rn(a, c3);
+    }
+    for (; j0 < d; j0 += kRouteBlock) {
+      const int j1 = min(j0 + kRouteBlock, d);
+      float c = 0.0f;
+      for (int j = j0; j < j1; j += 8) c = dot8_chain(c, x + j, wi + j);
+      a = __fadd_rn(a, c);
+    }
     const float zz = p.bias ? __fadd_rn(a, p.bias[i]) : a;
     z[q] = zz;
     if (p.logits) p.logits[(size_t)(tb + tl) * N + i] = zz;
