@@ -37,7 +37,7 @@ struct RDPlan {
   int tpc;      // tokens per CTA
   int grid;     // CTAs
   int row_bytes;
-  uint32_t u, w, z, sel, aw, cnt, base, len, off, wcnt, hist, total;
+  uint32_t u, w, z, zp, sel, aw, cnt, base, len, off, wcnt, hist, total;
 };
 
 struct RDParams {
@@ -84,6 +84,7 @@ bool make_rd_plan(const moe_shape& s, int32_t dtype, int sms, RDPlan* out) {
   p.u = take(off, (size_t)tpc * (p.row_bytes + 16));
   p.w = take(off, (size_t)s.N * (s.d + 4) * 4);
   p.z = take(off, (size_t)tpc * s.N * 4);
+  p.zp = take(off, (size_t)((s.d + kRouteBlock - 1) / kRouteBlock) * tpc * s.N * 4);
   p.sel = take(off, (size_t)tpc * s.k * 4);
   p.aw = take(off, (size_t)tpc * s.k * 4);
   p.cnt = take(off, kRDMaxN * 4);
@@ -105,23 +106,6 @@ __device__ __forceinline__ void cp16(void* smem, const void* gmem) {
                : "memory");
 }
 
-template <typename TU>
-__device__ __forceinline__ float dot8_chain(float a, const TU* x, const float* w) {
-  float xv[8];
-  load8(x, xv);
-  const float4 w0 = *reinterpret_cast<const float4*>(w);
-  const float4 w1 = *reinterpret_cast<const float4*>(w + 4);
-  a = __fmaf_rn(w0.x, xv[0], a);
-  a = __fmaf_rn(w0.y, xv[1], a);
-  a = __fmaf_rn(w0.z, xv[2], a);
-  a = __fmaf_rn(w0.w, xv[3], a);
-  a = __fmaf_rn(w1.x, xv[4], a);
-  a = __fmaf_rn(w1.y, xv[5], a);
-  a = __fmaf_rn(w1.z, xv[6], a);
-  a = __fmaf_rn(w1.w, xv[7], a);
-  return a;
-}
-
 template <int NP, typename TU>
 __global__ void __launch_bounds__(kRDThreads, 1) route_dispatch(const __grid_constant__ RDParams p) {
   extern __shared__ __align__(16) char sm[];
@@ -134,6 +118,7 @@ __global__ void __launch_bounds__(kRDThreads, 1) route_dispatch(const __grid_con
   char* us = sm + P.u;
   float* ws = reinterpret_cast<float*>(sm + P.w);
   float* z = reinterpret_cast<float*>(sm + P.z);
+  float* zp = reinterpret_cast<float*>(sm + P.zp);
   int* sel = reinterpret_cast<int*>(sm + P.sel);
   float* aw = reinterpret_cast<float*>(sm + P.aw);
   int* cnt = reinterpret_cast<int*>(sm + P.cnt);
@@ -160,33 +145,51 @@ __global__ void __launch_bounds__(kRDThreads, 1) route_dispatch(const __grid_con
   for (int e = tid; e < kRDMaxN; e += blockDim.x) cnt[e] = 0;
   asm volatile("cp.async.wait_all;" ::: "memory");
   __syncthreads();
+  // block sums: unit = (token pair, expert quad, block m), whose eight
+  // chains share each loaded activation (four experts) and router value (two
+  // tokens); zp [m][nt][N]
+  const int nblk = (d + kRouteBlock - 1) / kRouteBlock;
+  {
+    const int ntp = (nt + 1) / 2, neq = (N + 3) / 4, units = ntp * neq * nblk;
+    for (int uu = tid; uu < units; uu += blockDim.x) {
+      const int tp = uu % ntp, r = uu / ntp, eq = r % neq, m = r / neq;
+      const int t0 = 2 * tp, t1 = min(t0 + 1, nt - 1), e0 = 4 * eq;
+      const int j0 = m * kRouteBlock, len = min(kRouteBlock, d - j0);
+      const TU* xa = reinterpret_cast<const TU*>(us + t0 * ub) + j0;
+      const TU* xb = reinterpret_cast<const TU*>(us + t1 * ub) + j0;
+      const float* wr[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) wr[e] = ws + min(e0 + e, N - 1) * wld + j0;
+      float ca[4] = {0.0f, 0.0f, 0.0f, 0.0f}, cb[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+      for (int j = 0; j < len; j += 8) {
+        float va[8], vb[8];
+        load8(xa + j, va);
+        load8(xb + j, vb);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float4 w0 = *reinterpret_cast<const float4*>(wr[e] + j);
+          const float4 w1 = *reinterpret_cast<const float4*>(wr[e] + j + 4);
+          const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            ca[e] = __fmaf_rn(wv[q], va[q], ca[e]);
+            cb[e] = __fmaf_rn(wv[q], vb[q], cb[e]);
+          }
+        }
+      }
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        if (e0 + e < N) {
+          zp[((size_t)m * nt + t0) * N + e0 + e] = ca[e];
+          if (t1 != t0) zp[((size_t)m * nt + t1) * N + e0 + e] = cb[e];
+        }
+    }
+  }
+  __syncthreads();
   for (int q = tid; q < nt * N; q += blockDim.x) {
     const int tl = q / N, i = q - tl * N;
-    const TU* x = reinterpret_cast<const TU*>(us + tl * ub);
-    const float* wi = ws + i * wld;
-    // blocked order: four blocks' chains at a time (independent, so their
-    // FMAs overlap), each block sum added in ascending order
     float a = 0.0f;
-    int j0 = 0;
-    for (; j0 + 4 * kRouteBlock <= d; j0 += 4 * kRouteBlock) {
-      float c0 = 0.0f, c1 = 0.0f, c2 = 0.0f, c3 = 0.0f;
-      for (int j = j0; j < j0 + kRouteBlock; j += 8) {
-        c0 = dot8_chain(c0, x + j, wi + j);
-        c1 = dot8_chain(c1, x + j + kRouteBlock, wi + j + kRouteBlock);
-        c2 = dot8_chain(c2, x + j + 2 * kRouteBlock, wi + j + 2 * kRouteBlock);
-        c3 = dot8_chain(c3, x + j + 3 * kRouteBlock, wi + j + 3 * kRouteBlock);
-      }
-      a = __fadd_rn(a, c0);
-      a = __fadd_rn(a, c1);
-      a = __fadd_rn(a, c2);
-      a = __fadd_rn(a, c3);
-    }
-    for (; j0 < d; j0 += kRouteBlock) {
-      const int j1 = min(j0 + kRouteBlock, d);
-      float c = 0.0f;
-      for (int j = j0; j < j1; j += 8) c = dot8_chain(c, x + j, wi + j);
-      a = __fadd_rn(a, c);
-    }
+    for (int m = 0; m < nblk; ++m) a = __fadd_rn(a, zp[(size_t)m * nt * N + q]);
     const float zz = p.bias ? __fadd_rn(a, p.bias[i]) : a;
     z[q] = zz;
     if (p.logits) p.logits[(size_t)(tb + tl) * N + i] = zz;
