@@ -91,8 +91,9 @@ __global__ void __launch_bounds__(256)
 
 // One warp per token; rows already carry their weights (fp32 a * F(u)), the
 // kept slots are added in ascending s in fp32 and rounded once.  The token's
-// k (<= 32) slot rows are read once into shared memory; the row loads of four
-// slots are issued before their adds, so a warp has several loads in flight.
+// k (<= 32) slot row indices are read once into shared memory; a lane loads
+// two slots' rows for four of its columns before adding them, so a warp has
+// eight loads per lane in flight.
 template <typename TY>
 __global__ void __launch_bounds__(256)
     combine_weighted(const float4* __restrict__ rows, int width4,
@@ -111,26 +112,37 @@ __global__ void __launch_bounds__(256)
     }
     srow[wib][lane] = r;
     __syncwarp();
-    for (int c = lane; c < width4; c += 32) {
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int s0 = 0; s0 < k; s0 += 4) {
-        float4 v[4];
-        int rs[4];
+    // four columns per lane at a time (c0 + 32 q), two slots per round: the
+    // eight row loads of a round are in flight together
+    for (int c0 = lane; c0 < width4; c0 += 32 * 4) {
+      float4 acc[4];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
+      for (int q = 0; q < 4; ++q) acc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int s0 = 0; s0 < k; s0 += 2) {
+        float4 v[2][4];
+        int rs[2];
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
           rs[j] = s0 + j < k ? srow[wib][s0 + j] : -1;
-          if (rs[j] >= 0) v[j] = rows[(size_t)rs[j] * width4 + c];
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            if (rs[j] >= 0 && c0 + 32 * q < width4)
+              v[j][q] = rows[(size_t)rs[j] * width4 + c0 + 32 * q];
         }
 #pragma unroll
-        for (int j = 0; j < 4; ++j)
-          if (rs[j] >= 0) {
-            acc.x += v[j].x;
-            acc.y += v[j].y;
-            acc.z += v[j].z;
-            acc.w += v[j].w;
-          }
+        for (int j = 0; j < 2; ++j)
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            if (rs[j] >= 0 && c0 + 32 * q < width4) {
+              acc[q].x += v[j][q].x;
+              acc[q].y += v[j][q].y;
+              acc[q].z += v[j][q].z;
+              acc[q].w += v[j][q].w;
+            }
       }
-      store4<TY>(y + ((size_t)t * width4 + c) * 4, acc);
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        if (c0 + 32 * q < width4) store4<TY>(y + ((size_t)t * width4 + c0 + 32 * q) * 4, acc[q]);
     }
     __syncwarp();  // srow is rewritten for the warp's next token
   }
