@@ -35,7 +35,7 @@ __global__ void __launch_bounds__(16 * TG)
     router_logits_big(const TU* __restrict__ u, const float* __restrict__ w,
                       const float* __restrict__ bias, float* __restrict__ z, int T, int d, int N) {
   constexpr int BT = 8 * TG, HALF = 4 * TG, NT = 16 * TG;
-  constexpr int WU = (2 * kBigBN + NT - 1) / NT;  // weight-row loads per thread (1 or 2)
+  constexpr int WQ = (kBigBN * kBigBK / 4 + NT - 1) / NT;  // weight float4 loads per thread
   pdl_wait();
   pdl_allow_next();
   __shared__ __align__(16) float us[2][kBigBK][BT];
@@ -55,8 +55,9 @@ __global__ void __launch_bounds__(16 * TG)
 #pragma unroll
   for (int q = 0; q < 16; ++q) acc_s[q * NT + tid] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
   // a K step's loads: token row tid >> 1 (8 columns at (tid & 1) * 8), and
-  // expert rows (tid + q NT) >> 1 for q < WU
-  float ru[8], rw[WU][8];
+  // 4 columns of expert row x >> 2 at (x & 3) * 4 for x = tid + q NT, q < WQ
+  float ru[8];
+  float4 rw[WQ];
   auto fetch = [&](int k0) {
     const int kw = min(kBigBK, d - k0);  // multiple of 8
     {
@@ -69,14 +70,11 @@ __global__ void __launch_bounds__(16 * TG)
       }
     }
 #pragma unroll
-    for (int q = 0; q < WU; ++q) {
-      const int x = tid + q * NT, lr = x >> 1, lc = (x & 1) * 8;
-      if (lr < kBigBN && n0 + lr < N && lc < kw) {
-        load8(w + (size_t)(n0 + lr) * d + k0 + lc, rw[q]);
-      } else {
-#pragma unroll
-        for (int j = 0; j < 8; ++j) rw[q][j] = 0.0f;
-      }
+    for (int q = 0; q < WQ; ++q) {
+      const int x = tid + q * NT, lr = x >> 2, lc = (x & 3) * 4;
+      rw[q] = (lr < kBigBN && n0 + lr < N && lc < kw)
+                  ? *reinterpret_cast<const float4*>(w + (size_t)(n0 + lr) * d + k0 + lc)
+                  : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
     }
   };
   auto put = [&](int buf) {
@@ -86,50 +84,58 @@ __global__ void __launch_bounds__(16 * TG)
       for (int j = 0; j < 8; ++j) us[buf][lc + j][lr] = ru[j];
     }
 #pragma unroll
-    for (int q = 0; q < WU; ++q) {
-      const int x = tid + q * NT, lr = x >> 1, lc = (x & 1) * 8;
-      if (lr < kBigBN)
-#pragma unroll
-        for (int j = 0; j < 8; ++j) wsm[buf][lc + j][lr] = rw[q][j];
+    for (int q = 0; q < WQ; ++q) {
+      const int x = tid + q * NT, lr = x >> 2, lc = (x & 3) * 4;
+      if (lr < kBigBN) {
+        wsm[buf][lc][lr] = rw[q].x;
+        wsm[buf][lc + 1][lr] = rw[q].y;
+        wsm[buf][lc + 2][lr] = rw[q].z;
+        wsm[buf][lc + 3][lr] = rw[q].w;
+      }
     }
   };
   fetch(0);
   put(0);
   __syncthreads();
   int buf = 0;
-  for (int k0 = 0; k0 < d; k0 += kBigBK) {
-    const bool more = k0 + kBigBK < d;
-    if (more) fetch(k0 + kBigBK);
-    const int kw = min(kBigBK, d - k0);
-    for (int kk = 0; kk < kw; ++kk) {
-      const float4 a0 = *reinterpret_cast<const float4*>(&us[buf][kk][4 * ty]);
-      const float4 a1 = *reinterpret_cast<const float4*>(&us[buf][kk][HALF + 4 * ty]);
-      const float4 b0 = *reinterpret_cast<const float4*>(&wsm[buf][kk][4 * tx]);
-      const float4 b1 = *reinterpret_cast<const float4*>(&wsm[buf][kk][64 + 4 * tx]);
-      const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-      const float b[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+  // blocks of kRouteBlock inputs; inside a block the K steps run as one loop
+  // (the same body for every step), the partials are added after it
+  for (int kb = 0; kb < d; kb += kRouteBlock) {
+    const int ke = min(kb + kRouteBlock, d);
+    for (int k0 = kb; k0 < ke; k0 += kBigBK) {
+      const bool more = k0 + kBigBK < d;
+      if (more) fetch(k0 + kBigBK);
+      // a short last step reads the zeros fetch() put past d: fma(0, 0, p)
+      // leaves p unchanged, so every step runs all kBigBK columns
+#pragma unroll 4
+      for (int kk = 0; kk < kBigBK; ++kk) {
+        const float4 a0 = *reinterpret_cast<const float4*>(&us[buf][kk][4 * ty]);
+        const float4 a1 = *reinterpret_cast<const float4*>(&us[buf][kk][HALF + 4 * ty]);
+        const float4 b0 = *reinterpret_cast<const float4*>(&wsm[buf][kk][4 * tx]);
+        const float4 b1 = *reinterpret_cast<const float4*>(&wsm[buf][kk][64 + 4 * tx]);
+        const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+        const float b[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
-      for (int i = 0; i < 8; ++i)
+        for (int i = 0; i < 8; ++i)
 #pragma unroll
-        for (int j = 0; j < 8; j += 2) fma2_rn(part[i][j], part[i][j + 1], b[j], b[j + 1], a[i]);
-    }
-    if (!more || (k0 + kBigBK) % kRouteBlock == 0) {  // a block ends: add its partials
-#pragma unroll
-      for (int q = 0; q < 16; ++q) {
-        float* pq = &part[q >> 1][(q & 1) * 4];
-        float4 v = acc_s[q * NT + tid];
-        v.x = __fadd_rn(v.x, pq[0]);
-        v.y = __fadd_rn(v.y, pq[1]);
-        v.z = __fadd_rn(v.z, pq[2]);
-        v.w = __fadd_rn(v.w, pq[3]);
-        acc_s[q * NT + tid] = v;
-        pq[0] = pq[1] = pq[2] = pq[3] = 0.0f;
+          for (int j = 0; j < 8; j += 2) fma2_rn(part[i][j], part[i][j + 1], b[j], b[j + 1], a[i]);
+      }
+      if (more) {
+        put(buf ^ 1);
+        __syncthreads();
+        buf ^= 1;
       }
     }
-    if (more) {
-      put(buf ^ 1);
-      __syncthreads();
-      buf ^= 1;
+#pragma unroll
+    for (int q = 0; q < 16; ++q) {  // the block ends: add its partials
+      float* pq = &part[q >> 1][(q & 1) * 4];
+      float4 v = acc_s[q * NT + tid];
+      v.x = __fadd_rn(v.x, pq[0]);
+      v.y = __fadd_rn(v.y, pq[1]);
+      v.z = __fadd_rn(v.z, pq[2]);
+      v.w = __fadd_rn(v.w, pq[3]);
+      acc_s[q * NT + tid] = v;
+      pq[0] = pq[1] = pq[2] = pq[3] = 0.0f;
     }
   }
 #pragma unroll
@@ -146,19 +152,20 @@ __global__ void __launch_bounds__(16 * TG)
   }
 }
 
-// Token-tile width 8 TG for the large router: one CTA's tile takes about the
-// same time whatever TG (FMA-bound per SM), so the step lasts about
-// ceil(tiles / SMs) tiles of 8 TG tokens; the TG with the least
-// ceil(tiles / SMs) * TG wins (larger TG on ties).  4096 tokens x 896
-// experts on 148 SMs: TG = 13 (280 tiles, 2 per SM) against TG = 16's 224
-// tiles, also 2 per SM but 128 tokens each.
-int pick_tg(int T, int N, int sms) {
+// Token-tile width 8 TG for the large router: a tile's time grows with TG
+// (its FMAs), and cps[TG] tiles run at once per SM (the kernel's occupancy,
+// set by its registers: 7-warp CTAs fit twice per SM only at <= 128
+// registers a thread), so the step lasts about ceil(tiles / (SMs cps)) * TG;
+// the least wins (larger TG on ties).  4096 tokens x 896 experts on 148
+// SMs: TG = 13, 280 tiles in one wave of 2 per SM.
+int pick_tg(int T, int N, int sms, const int* cps) {
   const int64_t nt = (N + kBigBN - 1) / kBigBN;
   int best = 16;
   int64_t best_cost = INT64_MAX;
   for (int tg = 16; tg >= 8; --tg) {
     const int64_t tiles = nt * ((T + 8 * tg - 1) / (8 * tg));
-    const int64_t cost = (tiles + sms - 1) / sms * tg;
+    const int64_t slots = (int64_t)sms * (cps[tg] > 0 ? cps[tg] : 1);
+    const int64_t cost = (tiles + slots - 1) / slots * tg;
     if (cost < best_cost) {
       best_cost = cost;
       best = tg;
@@ -383,27 +390,50 @@ __global__ void __launch_bounds__(kRouteThreads)
   }
 }
 
+template <int TG>
+constexpr size_t logits_smem() {
+  return (size_t)64 * 4 * 16 * TG;  // acc_s: 64 fp32 logits per thread
+}
+
+// Sets the instantiation's shared-memory attributes once per device and
+// returns its CTAs per SM (0 when unknown).
+template <typename TU, int TG>
+int logits_setup() {
+  static std::atomic<bool> configured[kMaxDevices];
+  static std::atomic<int> occupancy[kMaxDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || !device_slot(dev)) return 0;
+  if (needs_setup(configured, dev)) {
+    MOE_PREFER_SHARED((router_logits_big<TU, TG>));
+    cudaFuncSetAttribute(router_logits_big<TU, TG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)logits_smem<TG>());
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, router_logits_big<TU, TG>, 16 * TG,
+                                                      logits_smem<TG>()) != cudaSuccess)
+      n = 0;
+    occupancy[dev].store(n, std::memory_order_relaxed);
+    mark_setup(configured, dev);
+  }
+  return occupancy[dev].load(std::memory_order_relaxed);
+}
+
 template <typename TU, int TG>
 void launch_logits_tg(const TU* u, const float* w, const float* bias, float* z, int T, int d,
                       int N, cudaStream_t st) {
   dim3 grid((T + 8 * TG - 1) / (8 * TG), (N + kBigBN - 1) / kBigBN);
-  const size_t smem = (size_t)64 * 4 * 16 * TG;  // acc_s: 64 fp32 logits per thread
-  static std::atomic<bool> configured[kMaxDevices];
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (device_slot(dev) && needs_setup(configured, dev)) {
-    MOE_PREFER_SHARED((router_logits_big<TU, TG>));
-    cudaFuncSetAttribute(router_logits_big<TU, TG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)smem);
-    mark_setup(configured, dev);
-  }
-  launch_pdl(router_logits_big<TU, TG>, grid, dim3(16 * TG), smem, st, u, w, bias, z, T, d, N);
+  logits_setup<TU, TG>();
+  launch_pdl(router_logits_big<TU, TG>, grid, dim3(16 * TG), logits_smem<TG>(), st, u, w, bias,
+             z, T, d, N);
 }
 
 template <typename TU>
 void launch_logits(const TU* u, const float* w, const float* bias, float* z, int T, int d, int N,
                    cudaStream_t st) {
-  switch (pick_tg(T, N, sm_count())) {
+  const int cps[17] = {0, 0, 0, 0, 0, 0, 0, 0,
+                       logits_setup<TU, 8>(),  logits_setup<TU, 9>(),  logits_setup<TU, 10>(),
+                       logits_setup<TU, 11>(), logits_setup<TU, 12>(), logits_setup<TU, 13>(),
+                       logits_setup<TU, 14>(), logits_setup<TU, 15>(), logits_setup<TU, 16>()};
+  switch (pick_tg(T, N, sm_count(), cps)) {
     case 8: return launch_logits_tg<TU, 8>(u, w, bias, z, T, d, N, st);
     case 9: return launch_logits_tg<TU, 9>(u, w, bias, z, T, d, N, st);
     case 10: return launch_logits_tg<TU, 10>(u, w, bias, z, T, d, N, st);
