@@ -81,6 +81,33 @@ __device__ __forceinline__ void fma2_rn(float& c0, float& c1, float b0, float b1
       : "f"(a), "f"(b0), "f"(b1));
 }
 
+// The two largest of zr[0..n) (n >= 2, n <= NR) in the order of the
+// slot-by-slot top-k selection: larger first, ties to the lower index, and a
+// NaN kept only where that selection would keep it (a NaN first entry, or a
+// NaN second entry when nothing later compares larger).  One pass.
+template <int NR>
+__device__ __forceinline__ void top2_of(const float* zr, int n, int& b0, float& z0, int& b1,
+                                        float& z1) {
+  b0 = 0;
+  z0 = zr[0];
+  b1 = -1;
+  z1 = 0.0f;
+#pragma unroll
+  for (int i = 1; i < NR; ++i) {
+    if (i < n) {
+      if (zr[i] > z0) {
+        b1 = b0;
+        z1 = z0;
+        b0 = i;
+        z0 = zr[i];
+      } else if (b1 < 0 || zr[i] > z1) {
+        b1 = i;
+        z1 = zr[i];
+      }
+    }
+  }
+}
+
 // Load 8 consecutive elements (16 B for 16-bit types, 32 B for fp32) as fp32.
 __device__ __forceinline__ void load8(const float* p, float* o) {
   float4 a = *reinterpret_cast<const float4*>(p);

@@ -217,20 +217,9 @@ __device__ __forceinline__ void topk8_k2(const float* zt, int renorm, int* sel, 
   const float4 za = *reinterpret_cast<const float4*>(zt);
   const float4 zb = *reinterpret_cast<const float4*>(zt + 4);
   const float zr[8] = {za.x, za.y, za.z, za.w, zb.x, zb.y, zb.z, zb.w};
-  int b0 = 0, b1 = -1;
-  float z0 = zr[0], z1 = 0.0f;
-#pragma unroll
-  for (int i = 1; i < 8; ++i) {
-    if (zr[i] > z0) {
-      b1 = b0;
-      z1 = z0;
-      b0 = i;
-      z0 = zr[i];
-    } else if (b1 < 0 || zr[i] > z1) {
-      b1 = i;
-      z1 = zr[i];
-    }
-  }
+  int b0, b1;
+  float z0, z1;
+  top2_of<8>(zr, 8, b0, z0, b1, z1);
   const float e1 = expf(z1 - z0);
   float S = 1.0f + e1;
   if (!renorm) {

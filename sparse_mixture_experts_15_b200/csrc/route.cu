@@ -356,7 +356,34 @@ __global__ void __launch_bounds__(kRouteThreads)
   }
   if (hist && threadIdx.x < NP) cnt[threadIdx.x] = 0;
   __syncthreads();
-  if (threadIdx.x < TPB && t0 + threadIdx.x < T) {
+  if (threadIdx.x < TPB && t0 + threadIdx.x < T && k == 2 && !probs) {
+    // top-2 in one pass and weights from one reciprocal, as the fused
+    // route+dispatch kernel does, so both give the same weights bit for bit
+    const int tt = t0 + threadIdx.x;
+    float zr[NP];
+#pragma unroll
+    for (int i = 0; i < NP; ++i) zr[i] = i < N ? zs[threadIdx.x][i] : 0.0f;
+    int b0, b1;
+    float z0, z1;
+    top2_of<NP>(zr, N, b0, z0, b1, z1);
+    const float e1 = expf(z1 - z0);
+    float S = 1.0f + e1;
+    if (!renorm) {
+      S = 0.0f;
+#pragma unroll
+      for (int i = 0; i < NP; ++i)
+        if (i < N) S += expf(zr[i] - z0);
+    }
+    const float r = 1.0f / S;
+    top_idx[(size_t)tt * 2] = b0;
+    top_idx[(size_t)tt * 2 + 1] = b1;
+    top_w[(size_t)tt * 2] = expf(z0 - z0) * r;
+    top_w[(size_t)tt * 2 + 1] = e1 * r;
+    if (hist) {
+      atomicAdd(&cnt[b0], 1);
+      atomicAdd(&cnt[b1], 1);
+    }
+  } else if (threadIdx.x < TPB && t0 + threadIdx.x < T) {
     const int tt = t0 + threadIdx.x;
     const float* z = zs[threadIdx.x];
     float zmax = -FLT_MAX;

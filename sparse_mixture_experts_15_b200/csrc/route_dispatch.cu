@@ -200,6 +200,34 @@ __global__ void __launch_bounds__(kRDThreads, 1) route_dispatch(const __grid_con
     float zr[NP];
 #pragma unroll
     for (int i = 0; i < NP; ++i) zr[i] = i < N ? z[tl * N + i] : 0.0f;
+    if (k == 2 && !p.probs) {
+      // top-2 in one pass; e = exp(z - z_0), weights from one reciprocal
+      // (renormalised: a_s = e_s / (1 + e_1); otherwise a_s = e_s / sum e)
+      int b0, b1;
+      float z0, z1;
+      top2_of<NP>(zr, N, b0, z0, b1, z1);
+      const float e1 = expf(z1 - z0);
+      float S = 1.0f + e1;
+      if (!p.renorm) {
+        S = 0.0f;
+#pragma unroll
+        for (int i = 0; i < NP; ++i)
+          if (i < N) S += expf(zr[i] - z0);
+      }
+      const float r = 1.0f / S;
+      const float a0 = expf(z0 - z0) * r, a1 = e1 * r;
+      sel[tl * 2] = b0;
+      sel[tl * 2 + 1] = b1;
+      aw[tl * 2] = a0;
+      aw[tl * 2 + 1] = a1;
+      p.top_idx[(size_t)t * 2] = b0;
+      p.top_idx[(size_t)t * 2 + 1] = b1;
+      p.top_w[(size_t)t * 2] = a0;
+      p.top_w[(size_t)t * 2 + 1] = a1;
+      atomicAdd(&cnt[b0], 1);
+      atomicAdd(&cnt[b1], 1);
+      continue;
+    }
     float zmax = -FLT_MAX;
 #pragma unroll
     for (int i = 0; i < NP; ++i)

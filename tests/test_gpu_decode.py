@@ -165,6 +165,36 @@ def test_decode_layer_other_shapes(T, d, N, k, h):
     assert rel_err(y.float().cpu().numpy(), oy) < TOL_Q4
 
 
+@pytest.mark.parametrize("T,d,N,k,h", [
+    (32, 1024, 8, 2, 256),   # phase-B units of 256 rows: two router blocks each
+    (32, 512, 64, 8, 128),   # 64 experts: 64 block sums per unit
+    (16, 512, 8, 2, 128),    # units of 64 rows: every layer runs its own chains
+])
+def test_decode_step_equals_layers(T, d, N, k, h):
+    """A 3-layer chained step (where a phase-B unit covers whole 128-input
+    router blocks, layers 1.. route from the block sums the previous layer's
+    phase B formed) equals the layer calls made one by one, which always
+    form the block sums from their own input."""
+    import dataclasses
+    wl = dataclasses.replace(W.decode(T=T, n_layers=3), d=d, N=N, k=k, h=h)
+    layers = [Layer(wl, l) for l in range(wl.n_layers)]
+    s = moe.shape(T, d, N, k, h, 1, 0)
+    u0 = _f16(_u0(wl))
+    out = torch.empty_like(u0)
+    idx_all = torch.empty((wl.n_layers, T, k), dtype=torch.int32, device="cuda")
+    moe.moe_decode_step(s, [L.abi for L in layers], u0, out, idx_all)
+    cur = u0
+    for l, L in enumerate(layers):
+        y = torch.empty_like(cur)
+        nxt = torch.empty_like(cur)
+        idx = torch.empty((T, k), dtype=torch.int32, device="cuda")
+        moe.moe_decode_layer(s, L.abi, cur, y, nxt, idx)
+        assert torch.equal(idx, idx_all[l]), f"layer {l}"
+        cur = nxt
+    torch.cuda.synchronize()
+    assert np.array_equal(_codes(cur), _codes(out))
+
+
 def test_decode_step_chunks_and_graph_replay():
     """40 layers (more than one launch carries) at T=1: the chained call equals
     the layer calls made one by one, and a CUDA-graph replay of the chained
@@ -203,11 +233,12 @@ def test_decode_step_chunks_and_graph_replay():
         assert np.array_equal(_codes(out2), _codes(out))
 
 
-def test_decode_step_trace_matches_and_stamps_phases():
+@pytest.mark.parametrize("T", [8, 32])
+def test_decode_step_trace_matches_and_stamps_phases(T):
     """The traced step (40 layers, two launches) gives the same output and
     routing as moe_decode_step, and each layer's phase stamps are
     non-decreasing SM cycle counts (block 0 stays on one SM)."""
-    wl = W.decode(T=8, n_layers=40)
+    wl = W.decode(T=T, n_layers=40)
     layers = [Layer(wl, l) for l in range(wl.n_layers)]
     s = moe.shape(wl.T, wl.d, wl.N, wl.k, wl.h, 1, 0)
     u0 = _f16(_u0(wl))
