@@ -124,6 +124,62 @@ def test_route_ties_and_controlled_logits():
     assert idx.cpu().numpy().tolist() == [[1, 2, 4]] * 3
 
 
+def _block_order_router(N, d=256):
+    """Router rows whose fp32 logit depends on the summation order (u = 1):
+    expert 0: 2^25 at 0, -2^25 at 128, 1 at 129 (blocked order 0, one chain 1);
+    expert 1: 1 at 0, 2^25 at 128, -2^25 at 129 (blocked 1, one chain 0);
+    expert 2: 2^25 at 0, 1 at 8, -2^25 at 128 (blocked 0, a pairwise tree 1);
+    expert 3: 0.5 at 0; the rest zero."""
+    Wr = np.zeros((N, d), np.float32)
+    Wr[0, [0, 128, 129]] = [2.0 ** 25, -(2.0 ** 25), 1.0]
+    Wr[1, [0, 128, 129]] = [1.0, 2.0 ** 25, -(2.0 ** 25)]
+    Wr[2, [0, 8, 128]] = [2.0 ** 25, 1.0, -(2.0 ** 25)]
+    Wr[3, 0] = 0.5
+    return Wr
+
+
+@pytest.mark.parametrize("N", [4, 8, 32])
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16, torch.float16])
+def test_router_block_order_on_gpu(N, dtype):
+    """Every router kernel forms the logits in the blocked order of the oracle
+    (128-input chains, block sums in order): the hand-worked logits 0, 1, 0,
+    0.5 come out exactly and the top-2 is experts 1 and 3."""
+    T, d = 40, 256
+    Wr = _block_order_router(N, d)
+    u = np.ones((T, d), np.float32)
+    s = moe.shape(T, d, N, 2, 64, 1, 0)
+    idx = torch.empty((T, 2), dtype=torch.int32, device="cuda")
+    tw = torch.empty((T, 2), dtype=torch.float32, device="cuda")
+    z = torch.empty((T, N), dtype=torch.float32, device="cuda")
+    moe.moe_route(s, torch.from_numpy(u).to(dtype).cuda(), torch.from_numpy(Wr).cuda(), idx, tw,
+                  logits=z)
+    torch.cuda.synchronize()
+    zo, _, oidx, _ = O.route(u, Wr, 2, 1)
+    zn = z.cpu().numpy()
+    assert np.array_equal(zn, zo)
+    assert np.array_equal(zn[:, :4], np.tile([0.0, 1.0, 0.0, 0.5], (T, 1)))
+    assert np.array_equal(idx.cpu().numpy(), oidx)
+    assert np.all(idx.cpu().numpy() == [1, 3])
+
+
+def test_layer_routing_block_order():
+    """The layer path's own router (the fused route+dispatch kernel for few
+    experts) picks experts 1 and 3 on the order-sensitive router rows."""
+    T, d, N, k, h = 64, 256, 4, 2, 64
+    Wr = torch.from_numpy(_block_order_router(N, d)).cuda()
+    u = torch.ones((T, d), dtype=torch.bfloat16, device="cuda")
+    g = torch.Generator(device="cuda").manual_seed(11)
+    w_gate, w_up = ((torch.randn(N, h, d, device="cuda", generator=g) * 0.02).to(torch.bfloat16)
+                    for _ in range(2))
+    w_down = (torch.randn(N, d, h, device="cuda", generator=g) * 0.02).to(torch.bfloat16)
+    y = torch.empty((T, d), dtype=torch.bfloat16, device="cuda")
+    top_idx = torch.empty((T, k), dtype=torch.int32, device="cuda")
+    s = moe.shape(T, d, N, k, h, 1, 0)
+    moe.moe_layer_fwd(s, Wr, w_gate, w_up, w_down, u, y, outputs={"top_idx": top_idx})
+    torch.cuda.synchronize()
+    assert np.all(top_idx.cpu().numpy() == [1, 3])
+
+
 @pytest.mark.parametrize("name,T", [("small", 4096), ("latent", 2048)])
 def test_aux_stats_vs_oracle(name, T):
     wl = W.ALL[name](T=T)
