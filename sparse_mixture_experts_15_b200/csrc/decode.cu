@@ -850,14 +850,339 @@ __global__ void __launch_bounds__(kThreads, 1) decode_persistent(const __grid_co
   }
 }
 
+// Bulk prefetch of [p, p + bytes) into L2 (16-byte aligned start and size).
+__device__ __forceinline__ void l2_prefetch(const void* ptr, int bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(ptr), "r"(bytes) : "memory");
+}
+
+// ============================================= one grid barrier per layer
+// Items (token t, slot s, hidden slice j of S), T k S of them, spread over
+// the CTAs.  An item stages its token's row, the selected expert e's gate and
+// up rows of hidden slice j and the down projection's columns of that slice,
+// forms H_j = SiLU(W_gate u) * (W_up u) on chip and the partial output
+// W_down[:, slice j] H_j, and stores that row to global memory.  The CTA that
+// stores a token's last (k S-th) partial row, told by a per-token arrival
+// counter, sums the token's partials (slots in order, each slot's slices in
+// order), forms u_{l+1}[t] = fp16(u_l + y) and the next layer's router block
+// sums for that row.  One grid barrier then separates the layers: the next
+// layer routes from the block sums.  Compared with the two-phase kernel this
+// drops the barrier between the hidden and the output projection (a token's
+// H never leaves the CTA) at the cost of one dequantisation per weight per
+// token.  Only the selected experts' rows are read.
+struct Plan2 {
+  int S;       // hidden slices per (token, slot)
+  int hS;      // hidden units per slice
+  int nparts;  // parts of d per gate/up row (one thread each)
+  uint32_t u, wr, z, sel, aw, zp, uh, uf, gq, gs, dq, ds, part, hs, misc;
+  uint32_t total;
+};
+
+struct Params2 {
+  LayerPtrs layer[kLayersPerLaunch];
+  int n_layers;
+  int T, d, N, k, h, renorm;
+  Plan2 plan;
+  const __half* u_in;
+  __half* u_work;
+  __half* u_out;
+  __half* y;
+  int32_t* top_idx;
+  float* top_w;
+  float* ypart;  // [T][k S][d] partial output rows
+  int* tcnt;     // [T] partial rows stored this layer (zero between layers)
+  float* zb;     // [d / kRouteBlock][N][T] next layer's router block sums
+  unsigned* bar;
+  int* status;
+  unsigned long long* stamps;
+};
+
+// Stamps of the one-barrier kernel, in the same 13 slots: 0 layer start,
+// 1 input staged (layer 0) or block sums read, 2 routed, 3 = 2, 4 item's rows
+// staged, 5 = 4, 6 gate/up dots formed, 7 H formed, 8 = 7, 9 down slice
+// ready, 10 partial row stored and counted, 11 token assembled (or = 10),
+// 12 barrier passed.
+__device__ __forceinline__ void stamp2(const Params2& p, int l, int i) {
+  if (p.stamps && blockIdx.x == 0 && threadIdx.x == 0)
+    p.stamps[(size_t)l * kStamps + i] = clock64();
+}
+
+bool make_plan2(const moe_shape& s, int sms, Plan2* out) {
+  const int T = s.T, d = s.d, N = s.N, k = s.k, h = s.h;
+  const int nb = d / 32, nbh = h / 32, nblk = (d + kRouteBlock - 1) / kRouteBlock;
+  // the most slices that keep the T k S items within one wave of CTAs
+  int S0 = 1;
+  while (2 * S0 <= nbh && (int64_t)T * k * 2 * S0 <= sms) S0 *= 2;
+  for (int S = S0; S <= nbh; S *= 2) {
+    const int hS = h / S;
+    if (2 * hS > kThreads) continue;
+    Plan2 p{};
+    p.S = S;
+    p.hS = hS;
+    p.nparts = kThreads / (2 * hS);
+    if (p.nparts > nb) p.nparts = nb;
+    uint32_t off = 0;
+    p.u = take(off, (size_t)T * (d + 8) * 2);  // layer 0: every token's row for its chains
+    p.wr = take(off, (size_t)N * (d + 4) * 4);
+    p.z = take(off, (size_t)T * N * 4);
+    p.sel = take(off, (size_t)T * k * 4);
+    p.aw = take(off, (size_t)T * k * 4);
+    p.zp = take(off, (size_t)T * N * nblk * 4);
+    p.uh = take(off, (size_t)d * 2);
+    p.uf = take(off, (size_t)d * 4);
+    p.gq = take(off, (size_t)2 * hS * (d / 2));
+    p.gs = take(off, (size_t)2 * hS * nb * 2);
+    p.dq = take(off, (size_t)d * (hS / 2));
+    p.ds = take(off, (size_t)d * nbh * 2);
+    p.part = take(off, (size_t)2 * hS * p.nparts * 4);
+    p.hs = take(off, (size_t)hS * 4);
+    p.misc = take(off, 16);
+    p.total = off;
+    if (off <= kSmemLimit) {
+      *out = p;
+      return true;
+    }
+  }
+  return false;
+}
+
+__global__ void __launch_bounds__(kThreads, 1) decode_fused(const __grid_constant__ Params2 p) {
+  extern __shared__ __align__(16) char sm[];
+  const Plan2& P = p.plan;
+  const int T = p.T, d = p.d, N = p.N, k = p.k, h = p.h, Tk = T * k;
+  const int S = P.S, hS = P.hS, nparts = P.nparts, KS = k * S;
+  const int nb = d / 32, nbh = h / 32, nblk = (d + kRouteBlock - 1) / kRouteBlock;
+  const int us_ld = d + 8, ws_ld = d + 4;
+  const int G = gridDim.x, b = blockIdx.x, tid = threadIdx.x;
+  __half* u_s = reinterpret_cast<__half*>(sm + P.u);
+  float* wr = reinterpret_cast<float*>(sm + P.wr);
+  float* z = reinterpret_cast<float*>(sm + P.z);
+  int* sel = reinterpret_cast<int*>(sm + P.sel);
+  float* aw = reinterpret_cast<float*>(sm + P.aw);
+  float* zp = reinterpret_cast<float*>(sm + P.zp);
+  __half* uh = reinterpret_cast<__half*>(sm + P.uh);
+  float* uf = reinterpret_cast<float*>(sm + P.uf);
+  uint8_t* gq = reinterpret_cast<uint8_t*>(sm + P.gq);
+  uint16_t* gs = reinterpret_cast<uint16_t*>(sm + P.gs);
+  uint8_t* dq = reinterpret_cast<uint8_t*>(sm + P.dq);
+  uint16_t* ds = reinterpret_cast<uint16_t*>(sm + P.ds);
+  float* part = reinterpret_cast<float*>(sm + P.part);
+  float* hsv = reinterpret_cast<float*>(sm + P.hs);
+  int* flag = reinterpret_cast<int*>(sm + P.misc);
+  const int W = Tk * S;
+  unsigned n_bar = 0;
+
+  stage_rows(reinterpret_cast<char*>(wr), ws_ld * 4,
+             reinterpret_cast<const char*>(p.layer[0].w_route), (size_t)d * 4, N, d * 4);
+  for (int l = 0; l < p.n_layers; ++l) {
+    const LayerPtrs& L = p.layer[l];
+    const bool last = l == p.n_layers - 1;
+    const __half* u_cur = l == 0 ? p.u_in : p.u_work;
+    __half* u_next = last ? p.u_out : p.u_work;
+    stamp2(p, l, 0);
+    if (l == 0) {  // no block sums yet: every CTA runs the chains over u_0
+      stage_rows(reinterpret_cast<char*>(u_s), us_ld * 2, reinterpret_cast<const char*>(u_cur),
+                 (size_t)d * 2, T, d * 2);
+      cp_wait_all();
+      __syncthreads();
+      stamp2(p, l, 1);
+      route_in_cta(u_s, us_ld, wr, ws_ld, T, d, N, k, p.renorm, L.bias, z, zp, nullptr, sel, aw);
+    } else {
+      __syncthreads();
+      stamp2(p, l, 1);
+      route_in_cta(u_s, us_ld, wr, ws_ld, T, d, N, k, p.renorm, L.bias, z, zp, p.zb, sel, aw);
+    }
+    stamp2(p, l, 2);
+    stamp2(p, l, 3);
+    if (b == 0) {
+      for (int x = tid; x < Tk; x += blockDim.x) {
+        if (p.top_idx) p.top_idx[(size_t)l * Tk + x] = sel[x];
+        if (last && p.top_w) p.top_w[x] = aw[x];
+      }
+    }
+    bool rows_next = false;  // the next layer's router rows issued (into wr)
+    for (int w = b; w < W; w += G) {
+      const int pr = w / S, j = w - pr * S, t = pr / k, s = pr - t * k;
+      const int e = sel[pr];
+      // the token's row and the slice's gate and up rows (one group), the
+      // slice's down columns (another group, waited for after the dots)
+      stage_bytes(uh, u_cur + (size_t)t * d, d * 2);
+      const size_t grow = (size_t)e * h + (size_t)j * hS;
+      stage_bytes(gq, L.gq + grow * (d / 2), hS * (d / 2));
+      stage_bytes(gq + (size_t)hS * (d / 2), L.uq + grow * (d / 2), hS * (d / 2));
+      stage_bytes(gs, L.gs + grow * nb, hS * nb * 2);
+      stage_bytes(gs + (size_t)hS * nb, L.us + grow * nb, hS * nb * 2);
+      cp_commit();
+      const int cpr = hS / 32;  // 16-byte pieces of a down row's slice
+      for (int i = tid; i < d * cpr; i += blockDim.x) {
+        const int o = i / cpr, c = i - o * cpr;
+        cp16(dq + (size_t)o * (hS / 2) + c * 16,
+             L.dq + ((size_t)e * d + o) * (h / 2) + (size_t)j * (hS / 2) + c * 16);
+      }
+      stage_bytes(ds, L.ds + (size_t)e * d * nbh, d * nbh * 2);
+      cp_commit();
+      // the next layer's router rows, for the block sums of the tokens this
+      // CTA assembles (routing, above, was the last reader of the buffer);
+      // their own group, waited for before an assembly
+      if (!last && !rows_next)
+        stage_rows(reinterpret_cast<char*>(wr), ws_ld * 4,
+                   reinterpret_cast<const char*>(p.layer[l + 1].w_route), (size_t)d * 4, N,
+                   d * 4);
+      rows_next = true;
+      cp_commit();
+      cp_wait_group<2>();  // the row and the gate/up rows
+      __syncthreads();
+      if (w == b) {
+        stamp2(p, l, 4);
+        stamp2(p, l, 5);
+      }
+      for (int i = tid; i < d; i += blockDim.x) uf[i] = __half2float(uh[i]);
+      __syncthreads();
+      // gate/up dots: thread = (row r2 of the 2 hS gate/up rows, part pp of
+      // d), weights dequantised in registers
+      for (int u2 = tid; u2 < 2 * hS * nparts; u2 += blockDim.x) {
+        const int r2 = u2 % (2 * hS), pp = u2 / (2 * hS);
+        const int b0 = pp * nb / nparts, b1 = (pp + 1) * nb / nparts;
+        const uint8_t* q = gq + (size_t)r2 * (d / 2);
+        const uint16_t* sc = gs + (size_t)r2 * nb;
+        // per block: sum of (q - 8) x over its 32 weights in four chains,
+        // then one multiply-add by the block scale
+        float acc = 0.0f;
+        for (int blk = b0; blk < b1; ++blk) {
+          const uint4 raw = *reinterpret_cast<const uint4*>(q + blk * 16);
+          const uint32_t wd[4] = {raw.x, raw.y, raw.z, raw.w};
+          const float4* x4 = reinterpret_cast<const float4*>(uf + blk * 32);
+          float c0 = 0.0f, c1 = 0.0f, c2 = 0.0f, c3 = 0.0f;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const uint32_t lo = wd[i] & 0x0F0F0F0Fu, hi = (wd[i] >> 4) & 0x0F0F0F0Fu;
+            const float4 xl = x4[i], xh = x4[4 + i];  // elements 4i.. and 16+4i..
+            c0 = fmaf(nib(lo, 0), xl.x, c0);
+            c1 = fmaf(nib(lo, 1), xl.y, c1);
+            c2 = fmaf(nib(lo, 2), xl.z, c2);
+            c3 = fmaf(nib(lo, 3), xl.w, c3);
+            c0 = fmaf(nib(hi, 0), xh.x, c0);
+            c1 = fmaf(nib(hi, 1), xh.y, c1);
+            c2 = fmaf(nib(hi, 2), xh.z, c2);
+            c3 = fmaf(nib(hi, 3), xh.w, c3);
+          }
+          acc = fmaf(f16f(sc[blk]), (c0 + c1) + (c2 + c3), acc);
+        }
+        part[r2 * nparts + pp] = acc;
+      }
+      __syncthreads();
+      if (w == b) stamp2(p, l, 6);
+      for (int r = tid; r < hS; r += blockDim.x) {
+        float g = 0.0f, v = 0.0f;
+        for (int pp = 0; pp < nparts; ++pp) {
+          g += part[r * nparts + pp];
+          v += part[(hS + r) * nparts + pp];
+        }
+        hsv[r] = silu(g) * v;
+      }
+      cp_wait_group<1>();  // the down slice
+      __syncthreads();
+      if (w == b) {
+        stamp2(p, l, 7);
+        stamp2(p, l, 8);
+        stamp2(p, l, 9);
+      }
+      // partial output: row o of W_down[e] over the slice's hidden units
+      float* yp = p.ypart + ((size_t)t * KS + (size_t)s * S + j) * d;
+      for (int o = tid; o < d; o += blockDim.x) {
+        const uint8_t* q = dq + (size_t)o * (hS / 2);
+        float a0 = 0.0f, a1 = 0.0f;
+        for (int bl = 0; bl < cpr; ++bl) {
+          float wv[32];
+          dequant_block(q + bl * 16, ds[(size_t)o * nbh + (size_t)j * cpr + bl], wv);
+          const float* hb = hsv + bl * 32;
+#pragma unroll
+          for (int c = 0; c < 32; c += 2) {
+            a0 = fmaf(wv[c], hb[c], a0);
+            a1 = fmaf(wv[c + 1], hb[c + 1], a1);
+          }
+        }
+        yp[o] = a0 + a1;
+      }
+      __syncthreads();
+      if (tid == 0) {  // publish the row, count it; the last row's CTA assembles
+        __threadfence();
+        const int done = atomicAdd(p.tcnt + t, 1) == KS - 1;
+        if (done) __threadfence();
+        *flag = done;
+      }
+      __syncthreads();
+      if (w == b) stamp2(p, l, 10);
+      if (*flag) {
+        cp_wait_group<0>();  // the next layer's router rows
+        __syncthreads();
+        for (int o = tid; o < d; o += blockDim.x) {
+          float acc = 0.0f;
+          for (int s2 = 0; s2 < k; ++s2) {
+            float ys = 0.0f;
+            for (int j2 = 0; j2 < S; ++j2)
+              ys += __ldcg(p.ypart + ((size_t)t * KS + (size_t)s2 * S + j2) * d + o);
+            acc = fmaf(aw[t * k + s2], ys, acc);
+          }
+          if (last && p.y) p.y[(size_t)t * d + o] = __float2half_rn(acc);
+          const __half un = __float2half_rn(__half2float(uh[o]) + acc);
+          if (u_next) u_next[(size_t)t * d + o] = un;
+          uf[o] = __half2float(un);
+        }
+        if (tid == 0) p.tcnt[t] = 0;
+        if (!last) {
+          __syncthreads();
+          // the next layer's router block sums of u_{l+1}[t]: one ascending
+          // FMA chain per (expert, 128-input block)
+          for (int q = tid; q < N * nblk; q += blockDim.x) {
+            const int i = q % N, m = q / N, j0 = m * kRouteBlock;
+            const int len = min(kRouteBlock, d - j0);
+            const float4* w4 = reinterpret_cast<const float4*>(wr + (size_t)i * ws_ld + j0);
+            const float4* x4 = reinterpret_cast<const float4*>(uf + j0);
+            float c = 0.0f;
+#pragma unroll 4
+            for (int s4 = 0; s4 < len / 4; ++s4) {
+              const float4 wv = w4[s4], x = x4[s4];
+              c = __fmaf_rn(wv.x, x.x, c);
+              c = __fmaf_rn(wv.y, x.y, c);
+              c = __fmaf_rn(wv.z, x.z, c);
+              c = __fmaf_rn(wv.w, x.w, c);
+            }
+            p.zb[((size_t)m * N + i) * T + t] = c;
+          }
+        }
+      }
+      if (w == b) stamp2(p, l, 11);
+      __syncthreads();  // the staging buffers are refilled by the next item
+    }
+    if (b >= W)
+      for (int i = 4; i < 12; ++i) stamp2(p, l, i);
+    cp_wait_all();  // (a CTA without items still has the router rows in flight)
+    grid_arrive(p.bar);
+    // while the barrier completes: CTA b < N S pulls the next layer's gate/up
+    // rows of (expert b / S, slice b % S) and, for slice 0, the expert's down
+    // rows into L2, so that the items' copies after routing hit L2
+    if (!last && b < N * S && tid == 0) {
+      const LayerPtrs& Ln = p.layer[l + 1];
+      const int e = b / S, j = b - (b / S) * S;
+      const size_t grow = (size_t)e * h + (size_t)j * hS;
+      l2_prefetch(Ln.gq + grow * (d / 2), hS * (d / 2));
+      l2_prefetch(Ln.uq + grow * (d / 2), hS * (d / 2));
+      if (j == 0) l2_prefetch(Ln.dq + (size_t)e * d * (h / 2), d * (h / 2));
+    }
+    if (!grid_wait(p.bar, (unsigned)G * ++n_bar, p.status)) return;
+    stamp2(p, l, 12);
+  }
+}
+
 // ------------------------------------------------------------------ host
 struct WsLayout {
   float* H;
+  float* ypart;  // one-barrier kernel: [T][k h/32][d] partial rows (at most h/32 slices)
   float* zb;
   int32_t* idx;
   float* w;
   __half* work;
-  unsigned* bar;
+  unsigned* bar;  // [0..3] barrier words, then [T] per-token counters
   size_t bytes;
 };
 
@@ -865,11 +1190,12 @@ WsLayout carve_decode(const moe_shape& s, void* base) {
   Carver c(base);
   WsLayout L;
   L.H = c.take<float>((size_t)s.N * s.T * s.h);
+  L.ypart = c.take<float>((size_t)s.T * s.k * (s.h / 32) * s.d);
   L.zb = c.take<float>((size_t)((s.d + kRouteBlock - 1) / kRouteBlock) * s.N * s.T);
   L.idx = c.take<int32_t>((size_t)s.T * s.k);
   L.w = c.take<float>((size_t)s.T * s.k);
   L.work = c.take<__half>((size_t)s.T * s.d);
-  L.bar = c.take<unsigned>(4);
+  L.bar = c.take<unsigned>(4 + (size_t)s.T);
   L.bytes = c.used();
   return L;
 }
@@ -885,9 +1211,12 @@ bool device_info(int* sms) {
     int n = 0;
     if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
         cudaFuncSetAttribute(decode_persistent, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)kSmemLimit) != cudaSuccess ||
+        cudaFuncSetAttribute(decode_fused, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)kSmemLimit) != cudaSuccess)
       return false;
     MOE_PREFER_SHARED((decode_persistent));
+    MOE_PREFER_SHARED((decode_fused));
     sm_count[dev].store(n, std::memory_order_relaxed);
     mark_setup(configured, dev);
   }
@@ -922,12 +1251,74 @@ LayerPtrs layer_ptrs(const moe_q4_layer& L) {
                    L.up_qs,   L.up_scales, L.down_qs, L.down_scales};
 }
 
-// One cooperative launch over layers [0, n) of `layers`.
+cudaError_t launch_coop(const void* kernel, int grid, size_t smem, cudaStream_t st, void* params) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  void* args[] = {params};
+  return cudaLaunchKernelExC(&cfg, kernel, args);
+}
+
+// The one-barrier kernel over layers [0, n) when its plan fits.
+int launch_decode_fused(const moe_shape& s, const Plan2& plan, int sms, const moe_q4_layer* layers,
+                        int n, const __half* u_in, __half* u_out, __half* y, int32_t* top_idx,
+                        float* top_w, const WsLayout& W, cudaStream_t st,
+                        unsigned long long* stamps) {
+  int occ = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, decode_fused, kThreads, plan.total) !=
+      cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (occ < 1) return MOE_ERR_UNSUPPORTED;
+  Params2 p{};
+  p.plan = plan;
+  const int items = s.T * s.k * plan.S;
+  const int grid = items < sms ? items : sms;
+  for (int l = 0; l < n; ++l) p.layer[l] = layer_ptrs(layers[l]);
+  p.n_layers = n;
+  p.T = s.T;
+  p.d = s.d;
+  p.N = s.N;
+  p.k = s.k;
+  p.h = s.h;
+  p.renorm = s.renorm;
+  p.u_in = u_in;
+  p.u_work = W.work;
+  p.u_out = u_out;
+  p.y = y;
+  p.top_idx = top_idx;
+  p.top_w = top_w;
+  p.ypart = W.ypart;
+  p.tcnt = reinterpret_cast<int*>(W.bar + 4);
+  p.zb = W.zb;
+  p.bar = W.bar;
+  p.status = status_word();
+  p.stamps = stamps;
+  if (cudaMemsetAsync(W.bar, 0, (4 + (size_t)s.T) * sizeof(unsigned), st) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  return launch_coop(reinterpret_cast<const void*>(decode_fused), grid, plan.total, st, &p) ==
+                 cudaSuccess
+             ? MOE_OK
+             : MOE_ERR_CUDA;
+}
+
+// One cooperative launch over layers [0, n) of `layers`: the one-barrier
+// kernel when its shared-memory plan fits, else the two-phase kernel.
 int launch_decode(const moe_shape& s, const moe_q4_layer* layers, int n, const __half* u_in,
                   __half* u_out, __half* y, int32_t* top_idx, float* top_w, const WsLayout& W,
                   cudaStream_t st, unsigned long long* stamps = nullptr) {
   int sms = 0;
   if (!device_info(&sms)) return MOE_ERR_CUDA;
+  Plan2 plan2;
+  if (make_plan2(s, sms, &plan2))
+    return launch_decode_fused(s, plan2, sms, layers, n, u_in, u_out, y, top_idx, top_w, W, st,
+                               stamps);
   Params p{};
   if (!make_plan(s, sms, &p.plan)) return MOE_ERR_UNSUPPORTED;
   int occ = 0;
