@@ -1047,6 +1047,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused(const __grid_constan
         // per block: sum of (q - 8) x over its 32 weights in four chains,
         // then one multiply-add by the block scale
         float acc = 0.0f;
+#pragma unroll 2
         for (int blk = b0; blk < b1; ++blk) {
           const uint4 raw = *reinterpret_cast<const uint4*>(q + blk * 16);
           const uint32_t wd[4] = {raw.x, raw.y, raw.z, raw.w};
@@ -1091,6 +1092,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused(const __grid_constan
       for (int o = tid; o < d; o += blockDim.x) {
         const uint8_t* q = dq + (size_t)o * (hS / 2);
         float a0 = 0.0f, a1 = 0.0f;
+#pragma unroll 2
         for (int bl = 0; bl < cpr; ++bl) {
           float wv[32];
           dequant_block(q + bl * 16, ds[(size_t)o * nbh + (size_t)j * cpr + bl], wv);
@@ -1105,16 +1107,19 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused(const __grid_constan
       }
       __syncthreads();
       if (tid == 0) {  // publish the row, count it; the last row's CTA assembles
-        __threadfence();
-        const int done = atomicAdd(p.tcnt + t, 1) == KS - 1;
-        if (done) __threadfence();
-        *flag = done;
+        int old;
+        // release: the CTA's partial-row stores (ordered before by the
+        // barrier above) become visible with the count; acquire: the last
+        // counter sees every other partial row
+        asm volatile("atom.add.acq_rel.gpu.s32 %0, [%1], 1;"
+                     : "=r"(old)
+                     : "l"(p.tcnt + t)
+                     : "memory");
+        *flag = old == KS - 1;
       }
       __syncthreads();
       if (w == b) stamp2(p, l, 10);
       if (*flag) {
-        cp_wait_group<0>();  // the next layer's router rows
-        __syncthreads();
         for (int o = tid; o < d; o += blockDim.x) {
           float acc = 0.0f;
           for (int s2 = 0; s2 < k; ++s2) {
@@ -1130,6 +1135,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused(const __grid_constan
         }
         if (tid == 0) p.tcnt[t] = 0;
         if (!last) {
+          cp_wait_group<0>();  // the next layer's router rows
           __syncthreads();
           // the next layer's router block sums of u_{l+1}[t]: one ascending
           // FMA chain per (expert, 128-input block)
