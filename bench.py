@@ -607,9 +607,11 @@ class DecodeReplica:
         return sum(t.numel() * t.element_size() for t in self.keep)
 
 
-DECODE_PHASES = ("stage u", "route", "group pairs", "stage gate/up rows", "dequantise",
-                 "gate/up dots", "H store", "barrier 1", "down rows ready", "down dots",
-                 "combine + u_next", "barrier 2")
+# Intervals between the 13 per-layer stamps of the one-barrier decode kernel
+# (the kernel the benchmark shapes run); the bracketed ones are empty there.
+DECODE_PHASES = ("start", "route", "(stamps 2-3)", "stage item rows", "(stamps 4-5)",
+                 "gate/up dots", "H", "(stamps 7-8)", "down columns ready",
+                 "down partial + count", "token assembly", "barrier")
 
 
 def decode_phases(wl, moe, s, rep, out, ws, torch, sm_mhz: float):

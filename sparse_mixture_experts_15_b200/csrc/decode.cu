@@ -9,7 +9,10 @@
 //
 // At decode sizes a layer moves well under a megabyte, so the step is bound
 // by its chain of dependent phases, not by HBM.  All layers of a call run in
-// ONE persistent cooperative launch (one CTA per SM, all co-resident), with
+// ONE persistent cooperative launch (at most one CTA per SM, all
+// co-resident).  Two kernels: the one-barrier kernel (further below: items
+// of (token, slot, hidden slice), one grid barrier per layer) when its
+// shared-memory plan fits, else the two-phase kernel described here, with
 // two grid barriers per layer instead of two kernel boundaries:
 //   route   every CTA stages u_l and W_route (fp32) in shared memory and
 //           routes all T tokens itself (identical, deterministic code, so

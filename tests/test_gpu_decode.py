@@ -147,6 +147,7 @@ def test_decode_reads_only_selected_experts():
     (32, 1024, 8, 2, 256),   # 8 output rows per phase-B slice, h/32 = 8 parts
     (5, 64, 4, 2, 32),       # tiny: one q4 block per hidden row, ragged T
     (3, 96, 4, 3, 64),       # d/32 = 3 blocks: uneven phase-A parts
+    (16, 2048, 8, 2, 128),   # too wide for the one-barrier plan: the two-phase kernel
 ])
 def test_decode_layer_other_shapes(T, d, N, k, h):
     import dataclasses
@@ -169,12 +170,13 @@ def test_decode_layer_other_shapes(T, d, N, k, h):
     (32, 1024, 8, 2, 256),   # phase-B units of 256 rows: two router blocks each
     (32, 512, 64, 8, 128),   # 64 experts: 64 block sums per unit
     (16, 512, 8, 2, 128),    # units of 64 rows: every layer runs its own chains
+    (16, 2048, 8, 2, 128),   # the two-phase kernel (the one-barrier plan does not fit)
 ])
 def test_decode_step_equals_layers(T, d, N, k, h):
-    """A 3-layer chained step (where a phase-B unit covers whole 128-input
-    router blocks, layers 1.. route from the block sums the previous layer's
-    phase B formed) equals the layer calls made one by one, which always
-    form the block sums from their own input."""
+    """A 3-layer chained step (layers 1.. route from the router block sums
+    that the previous layer formed, in either decode kernel) equals the
+    layer calls made one by one, which form the block sums from their own
+    input."""
     import dataclasses
     wl = dataclasses.replace(W.decode(T=T, n_layers=3), d=d, N=N, k=k, h=h)
     layers = [Layer(wl, l) for l in range(wl.n_layers)]
