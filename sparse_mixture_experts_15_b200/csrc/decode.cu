@@ -893,6 +893,7 @@ struct Params2 {
   float* top_w;
   float* ypart;  // [T][k S][d] partial output rows
   int* tcnt;     // [T] partial rows stored this layer (zero between layers)
+  int* tflag;    // [T] layers whose output row (and block sums) token t has
   float* zb;     // [d / kRouteBlock][N][T] next layer's router block sums
   unsigned* bar;
   int* status;
@@ -948,6 +949,34 @@ bool make_plan2(const moe_shape& s, int sms, Plan2* out) {
   return false;
 }
 
+// Thread 0 waits (bounded, like the grid barrier) until *f >= target, then
+// the CTA proceeds; false (every CTA then returns) on timeout or abort.
+__device__ bool token_wait(const int* f, int target, unsigned* bar, int* status) {
+  __shared__ int ok;
+  if (threadIdx.x == 0) {
+    int good = 1;
+    const unsigned long long t0 = global_ns();
+    unsigned polls = 0;
+    while ((int)ld_acquire(reinterpret_cast<const unsigned*>(f)) < target) {
+      if ((++polls & 15u) == 0) {
+        if (ld_acquire(bar + 1) != 0u) {
+          good = 0;
+          break;
+        }
+        if (global_ns() - t0 > kBarrierBudgetNs) {
+          record_error(status, MOE_ERR_TIMEOUT);
+          atomicExch(bar + 1, 1u);
+          good = 0;
+          break;
+        }
+      }
+    }
+    ok = good;
+  }
+  __syncthreads();
+  return ok != 0;
+}
+
 __global__ void __launch_bounds__(kThreads, 1) decode_fused(const __grid_constant__ Params2 p) {
   extern __shared__ __align__(16) char sm[];
   const Plan2& P = p.plan;
@@ -972,7 +1001,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused(const __grid_constan
   float* hsv = reinterpret_cast<float*>(sm + P.hs);
   int* flag = reinterpret_cast<int*>(sm + P.misc);
   const int W = Tk * S;
-  unsigned n_bar = 0;
 
   stage_rows(reinterpret_cast<char*>(wr), ws_ld * 4,
              reinterpret_cast<const char*>(p.layer[0].w_route), (size_t)d * 4, N, d * 4);
@@ -989,22 +1017,55 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused(const __grid_constan
       __syncthreads();
       stamp2(p, l, 1);
       route_in_cta(u_s, us_ld, wr, ws_ld, T, d, N, k, p.renorm, L.bias, z, zp, nullptr, sel, aw);
-    } else {
-      __syncthreads();
-      stamp2(p, l, 1);
-      route_in_cta(u_s, us_ld, wr, ws_ld, T, d, N, k, p.renorm, L.bias, z, zp, p.zb, sel, aw);
-    }
-    stamp2(p, l, 2);
-    stamp2(p, l, 3);
-    if (b == 0) {
-      for (int x = tid; x < Tk; x += blockDim.x) {
-        if (p.top_idx) p.top_idx[(size_t)l * Tk + x] = sel[x];
-        if (last && p.top_w) p.top_w[x] = aw[x];
+      stamp2(p, l, 2);
+      stamp2(p, l, 3);
+      if (b == 0) {
+        for (int x = tid; x < Tk; x += blockDim.x) {
+          if (p.top_idx) p.top_idx[(size_t)l * Tk + x] = sel[x];
+          if (last && p.top_w) p.top_w[x] = aw[x];
+        }
       }
     }
     bool rows_next = false;  // the next layer's router rows issued (into wr)
     for (int w = b; w < W; w += G) {
       const int pr = w / S, j = w - pr * S, t = pr / k, s = pr - t * k;
+      if (l > 0) {
+        // tokens are independent: wait only for token t's layer-l input (its
+        // row and router block sums, released by the CTA that assembled it),
+        // then route token t alone
+        if (!token_wait(p.tflag + t, l, p.bar, p.status)) {
+          cp_wait_all();
+          return;
+        }
+        if (w == b) stamp2(p, l, 1);
+        for (int i = tid; i < N; i += blockDim.x) {
+          float zz = 0.0f;
+          for (int m = 0; m < nblk; ++m)
+            zz = __fadd_rn(zz, __ldcg(p.zb + ((size_t)m * N + i) * T + t));
+          z[t * N + i] = L.bias ? __fadd_rn(zz, L.bias[i]) : zz;
+        }
+        __syncthreads();
+        if (tid == 0) {
+          if (N == 8 && k == 2)
+            topk8_k2(z + t * N, p.renorm, sel + t * k, aw + t * k);
+          else if (N <= 8)
+            topk_token<8>(z + t * N, N, k, p.renorm, sel + t * k, aw + t * k);
+          else if (N <= 32)
+            topk_token<32>(z + t * N, N, k, p.renorm, sel + t * k, aw + t * k);
+          else
+            topk_wide(z + t * N, N, k, p.renorm, sel + t * k, aw + t * k);
+        }
+        __syncthreads();
+        if (s == 0 && j == 0)  // one of the token's items writes its routing
+          for (int x = tid; x < k; x += blockDim.x) {
+            if (p.top_idx) p.top_idx[(size_t)l * Tk + t * k + x] = sel[t * k + x];
+            if (last && p.top_w) p.top_w[t * k + x] = aw[t * k + x];
+          }
+        if (w == b) {
+          stamp2(p, l, 2);
+          stamp2(p, l, 3);
+        }
+      }
       const int e = sel[pr];
       // the token's row and the slice's gate and up rows (one group), the
       // slice's down columns (another group, waited for after the dots)
@@ -1159,15 +1220,19 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused(const __grid_constan
             p.zb[((size_t)m * N + i) * T + t] = c;
           }
         }
+        __syncthreads();  // the row and its block sums stored by every thread
+        if (tid == 0)
+          asm volatile("st.release.gpu.global.s32 [%0], %1;" ::"l"(p.tflag + t), "r"(l + 1)
+                       : "memory");
       }
       if (w == b) stamp2(p, l, 11);
       __syncthreads();  // the staging buffers are refilled by the next item
     }
     if (b >= W)
-      for (int i = 4; i < 12; ++i) stamp2(p, l, i);
-    cp_wait_all();  // (a CTA without items still has the router rows in flight)
-    grid_arrive(p.bar);
-    // while the barrier completes: CTA b < N S pulls the next layer's gate/up
+      for (int i = 1; i < 12; ++i) stamp2(p, l, i);
+    // the router rows must land before the next layer refills the buffer
+    cp_wait_all();
+    // CTA b < N S pulls the next layer's gate/up
     // rows of (expert b / S, slice b % S) and, for slice 0, the expert's down
     // rows into L2, so that the items' copies after routing hit L2
     if (!last && b < N * S && tid == 0) {
@@ -1178,7 +1243,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused(const __grid_constan
       l2_prefetch(Ln.uq + grow * (d / 2), hS * (d / 2));
       if (j == 0) l2_prefetch(Ln.dq + (size_t)e * d * (h / 2), d * (h / 2));
     }
-    if (!grid_wait(p.bar, (unsigned)G * ++n_bar, p.status)) return;
     stamp2(p, l, 12);
   }
 }
@@ -1191,7 +1255,7 @@ struct WsLayout {
   int32_t* idx;
   float* w;
   __half* work;
-  unsigned* bar;  // [0..3] barrier words, then [T] per-token counters
+  unsigned* bar;  // [0..3] barrier words, then [T] per-token counters, [T] per-token flags
   size_t bytes;
 };
 
@@ -1204,7 +1268,7 @@ WsLayout carve_decode(const moe_shape& s, void* base) {
   L.idx = c.take<int32_t>((size_t)s.T * s.k);
   L.w = c.take<float>((size_t)s.T * s.k);
   L.work = c.take<__half>((size_t)s.T * s.d);
-  L.bar = c.take<unsigned>(4 + (size_t)s.T);
+  L.bar = c.take<unsigned>(4 + 2 * (size_t)s.T);
   L.bytes = c.used();
   return L;
 }
@@ -1305,11 +1369,12 @@ int launch_decode_fused(const moe_shape& s, const Plan2& plan, int sms, const mo
   p.top_w = top_w;
   p.ypart = W.ypart;
   p.tcnt = reinterpret_cast<int*>(W.bar + 4);
+  p.tflag = reinterpret_cast<int*>(W.bar + 4 + s.T);
   p.zb = W.zb;
   p.bar = W.bar;
   p.status = status_word();
   p.stamps = stamps;
-  if (cudaMemsetAsync(W.bar, 0, (4 + (size_t)s.T) * sizeof(unsigned), st) != cudaSuccess)
+  if (cudaMemsetAsync(W.bar, 0, (4 + 2 * (size_t)s.T) * sizeof(unsigned), st) != cudaSuccess)
     return MOE_ERR_CUDA;
   return launch_coop(reinterpret_cast<const void*>(decode_fused), grid, plan.total, st, &p) ==
                  cudaSuccess
