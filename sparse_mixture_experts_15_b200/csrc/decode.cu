@@ -853,30 +853,27 @@ __global__ void __launch_bounds__(kThreads, 1) decode_persistent(const __grid_co
   }
 }
 
-// Bulk prefetch of [p, p + bytes) into L2 (16-byte aligned start and size).
-__device__ __forceinline__ void l2_prefetch(const void* ptr, int bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(ptr), "r"(bytes) : "memory");
-}
-
-// ============================================= one grid barrier per layer
-// Items (token t, slot s, hidden slice j of S), T k S of them, spread over
-// the CTAs.  An item stages its token's row, the selected expert e's gate and
-// up rows of hidden slice j and the down projection's columns of that slice,
-// forms H_j = SiLU(W_gate u) * (W_up u) on chip and the partial output
-// W_down[:, slice j] H_j, and stores that row to global memory.  The CTA that
-// stores a token's last (k S-th) partial row, told by a per-token arrival
-// counter, sums the token's partials (slots in order, each slot's slices in
-// order), forms u_{l+1}[t] = fp16(u_l + y) and the next layer's router block
-// sums for that row.  One grid barrier then separates the layers: the next
-// layer routes from the block sums.  Compared with the two-phase kernel this
-// drops the barrier between the hidden and the output projection (a token's
-// H never leaves the CTA) at the cost of one dequantisation per weight per
-// token.  Only the selected experts' rows are read.
+// ================================================ per-token decode kernel
+// Tokens are independent through the layer stack, so this kernel needs no
+// grid barrier.  CTA b owns the item (token t, slot s, hidden slice j of S)
+// for every layer (T k S CTAs, at most one per SM) and keeps its token's
+// row u_l[t] in shared memory.  Per layer it routes token t itself (the
+// 128-input block chains of its logits, top-k), stages the selected
+// expert's gate and up rows of slice j and the slice's down columns, forms
+// H_j = SiLU(W_gate u) * (W_up u) on chip and the partial output row
+// W_down[:, slice j] H_j, stores that row and counts it on the token's
+// counter.  Once the token's k S rows are counted, each of the token's CTAs
+// sums them in one fixed order (slots in order, each slot's slices in
+// order) into u_{l+1}[t] = fp16(u_l + y), so all of them hold the same next
+// row and route it to the same experts.  Partial rows alternate between two
+// buffers by layer parity: a CTA can start layer l+1 only after every item
+// of its token counted layer l, i.e. after every reader of layer l-1's rows
+// has moved on.  Only the selected experts' rows are read.
 struct Plan2 {
   int S;       // hidden slices per (token, slot)
   int hS;      // hidden units per slice
   int nparts;  // parts of d per gate/up row (one thread each)
-  uint32_t u, wr, z, sel, aw, zp, uh, uf, gq, gs, dq, ds, part, hs, misc;
+  uint32_t wr, z, sel, aw, zp, uh, uf, gq, gs, dq, ds, part, hs, misc;
   uint32_t total;
 };
 
@@ -886,51 +883,53 @@ struct Params2 {
   int T, d, N, k, h, renorm;
   Plan2 plan;
   const __half* u_in;
-  __half* u_work;
   __half* u_out;
   __half* y;
   int32_t* top_idx;
   float* top_w;
-  float* ypart;  // [T][k S][d] partial output rows
-  int* tcnt;     // [T] partial rows stored this layer (zero between layers)
-  int* tflag;    // [T] layers whose output row (and block sums) token t has
-  float* zb;     // [d / kRouteBlock][N][T] next layer's router block sums
-  unsigned* bar;
+  float* ypart;  // [2][T][k S][d] partial output rows, by layer parity
+  int* tcnt;     // [T] partial rows counted so far (k S per layer)
+  unsigned* bar;  // [1]: abort flag
   int* status;
   unsigned long long* stamps;
 };
 
-// Stamps of the one-barrier kernel, in the same 13 slots: 0 layer start,
-// 1 input staged (layer 0) or block sums read, 2 routed, 3 = 2, 4 item's rows
-// staged, 5 = 4, 6 gate/up dots formed, 7 H formed, 8 = 7, 9 down slice
-// ready, 10 partial row stored and counted, 11 token assembled (or = 10),
-// 12 barrier passed.
+// Stamps of the per-token kernel, in the same 13 slots (block 0's item):
+// 0 layer start, 1 = 0, 2 routed, 3 = 2, 4 the item's gate/up rows staged,
+// 5 = 4, 6 gate/up dots formed, 7 H formed, 8 = 7, 9 down columns ready,
+// 10 partial row stored and counted, 11 the token's rows all counted,
+// 12 next row formed.
 __device__ __forceinline__ void stamp2(const Params2& p, int l, int i) {
   if (p.stamps && blockIdx.x == 0 && threadIdx.x == 0)
     p.stamps[(size_t)l * kStamps + i] = clock64();
 }
 
+// Bulk prefetch of [p, p + bytes) into L2 (16-byte aligned start and size).
+__device__ __forceinline__ void l2_prefetch(const void* ptr, int bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(ptr), "r"(bytes) : "memory");
+}
+
 bool make_plan2(const moe_shape& s, int sms, Plan2* out) {
   const int T = s.T, d = s.d, N = s.N, k = s.k, h = s.h;
   const int nb = d / 32, nbh = h / 32, nblk = (d + kRouteBlock - 1) / kRouteBlock;
-  // the most slices that keep the T k S items within one wave of CTAs
+  if ((int64_t)T * k > sms) return false;  // one CTA per item
+  // the most slices that keep one CTA per item
   int S0 = 1;
   while (2 * S0 <= nbh && (int64_t)T * k * 2 * S0 <= sms) S0 *= 2;
-  for (int S = S0; S <= nbh; S *= 2) {
+  for (int S = S0; S >= 1; S /= 2) {
     const int hS = h / S;
-    if (2 * hS > kThreads) continue;
+    if (2 * hS > kThreads) break;
     Plan2 p{};
     p.S = S;
     p.hS = hS;
     p.nparts = kThreads / (2 * hS);
     if (p.nparts > nb) p.nparts = nb;
     uint32_t off = 0;
-    p.u = take(off, (size_t)T * (d + 8) * 2);  // layer 0: every token's row for its chains
     p.wr = take(off, (size_t)N * (d + 4) * 4);
-    p.z = take(off, (size_t)T * N * 4);
-    p.sel = take(off, (size_t)T * k * 4);
-    p.aw = take(off, (size_t)T * k * 4);
-    p.zp = take(off, (size_t)T * N * nblk * 4);
+    p.z = take(off, (size_t)N * 4);
+    p.sel = take(off, (size_t)k * 4);
+    p.aw = take(off, (size_t)k * 4);
+    p.zp = take(off, (size_t)N * nblk * 4);
     p.uh = take(off, (size_t)d * 2);
     p.uf = take(off, (size_t)d * 4);
     p.gq = take(off, (size_t)2 * hS * (d / 2));
@@ -949,9 +948,9 @@ bool make_plan2(const moe_shape& s, int sms, Plan2* out) {
   return false;
 }
 
-// Thread 0 waits (bounded, like the grid barrier) until *f >= target, then
-// the CTA proceeds; false (every CTA then returns) on timeout or abort.
-__device__ bool token_wait(const int* f, int target, unsigned* bar, int* status) {
+// Thread 0 waits (bounded, 2 s of device time) until *f >= target, then the
+// CTA proceeds; false on timeout (MOE_ERR_TIMEOUT, abort raised) or abort.
+__device__ bool count_wait(const int* f, int target, unsigned* abort_flag, int* status) {
   __shared__ int ok;
   if (threadIdx.x == 0) {
     int good = 1;
@@ -959,13 +958,13 @@ __device__ bool token_wait(const int* f, int target, unsigned* bar, int* status)
     unsigned polls = 0;
     while ((int)ld_acquire(reinterpret_cast<const unsigned*>(f)) < target) {
       if ((++polls & 15u) == 0) {
-        if (ld_acquire(bar + 1) != 0u) {
+        if (ld_acquire(abort_flag) != 0u) {
           good = 0;
           break;
         }
         if (global_ns() - t0 > kBarrierBudgetNs) {
           record_error(status, MOE_ERR_TIMEOUT);
-          atomicExch(bar + 1, 1u);
+          atomicExch(abort_flag, 1u);
           good = 0;
           break;
         }
@@ -977,15 +976,14 @@ __device__ bool token_wait(const int* f, int target, unsigned* bar, int* status)
   return ok != 0;
 }
 
-__global__ void __launch_bounds__(kThreads, 1) decode_fused(const __grid_constant__ Params2 p) {
+__global__ void __launch_bounds__(kThreads, 1) decode_token(const __grid_constant__ Params2 p) {
   extern __shared__ __align__(16) char sm[];
   const Plan2& P = p.plan;
   const int T = p.T, d = p.d, N = p.N, k = p.k, h = p.h, Tk = T * k;
   const int S = P.S, hS = P.hS, nparts = P.nparts, KS = k * S;
   const int nb = d / 32, nbh = h / 32, nblk = (d + kRouteBlock - 1) / kRouteBlock;
-  const int us_ld = d + 8, ws_ld = d + 4;
-  const int G = gridDim.x, b = blockIdx.x, tid = threadIdx.x;
-  __half* u_s = reinterpret_cast<__half*>(sm + P.u);
+  const int ws_ld = d + 4, cpr = hS / 32;
+  const int b = blockIdx.x, tid = threadIdx.x;
   float* wr = reinterpret_cast<float*>(sm + P.wr);
   float* z = reinterpret_cast<float*>(sm + P.z);
   int* sel = reinterpret_cast<int*>(sm + P.sel);
@@ -999,250 +997,193 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused(const __grid_constan
   uint16_t* ds = reinterpret_cast<uint16_t*>(sm + P.ds);
   float* part = reinterpret_cast<float*>(sm + P.part);
   float* hsv = reinterpret_cast<float*>(sm + P.hs);
-  int* flag = reinterpret_cast<int*>(sm + P.misc);
-  const int W = Tk * S;
+  if (b >= Tk * S) return;
+  const int pr = b / S, j = b - pr * S, t = pr / k, s = pr - t * k;
+  const bool writer = s == 0 && j == 0;  // writes the token's routing and outputs
 
+  // the token's input row and layer 0's router rows
+  stage_bytes(uh, p.u_in + (size_t)t * d, d * 2);
   stage_rows(reinterpret_cast<char*>(wr), ws_ld * 4,
              reinterpret_cast<const char*>(p.layer[0].w_route), (size_t)d * 4, N, d * 4);
+  cp_wait_all();
+  __syncthreads();
+  for (int i = tid; i < d; i += blockDim.x) uf[i] = __half2float(uh[i]);
+  __syncthreads();
   for (int l = 0; l < p.n_layers; ++l) {
     const LayerPtrs& L = p.layer[l];
     const bool last = l == p.n_layers - 1;
-    const __half* u_cur = l == 0 ? p.u_in : p.u_work;
-    __half* u_next = last ? p.u_out : p.u_work;
     stamp2(p, l, 0);
-    if (l == 0) {  // no block sums yet: every CTA runs the chains over u_0
-      stage_rows(reinterpret_cast<char*>(u_s), us_ld * 2, reinterpret_cast<const char*>(u_cur),
-                 (size_t)d * 2, T, d * 2);
-      cp_wait_all();
-      __syncthreads();
-      stamp2(p, l, 1);
-      route_in_cta(u_s, us_ld, wr, ws_ld, T, d, N, k, p.renorm, L.bias, z, zp, nullptr, sel, aw);
-      stamp2(p, l, 2);
-      stamp2(p, l, 3);
-      if (b == 0) {
-        for (int x = tid; x < Tk; x += blockDim.x) {
-          if (p.top_idx) p.top_idx[(size_t)l * Tk + x] = sel[x];
-          if (last && p.top_w) p.top_w[x] = aw[x];
-        }
-      }
-    }
-    bool rows_next = false;  // the next layer's router rows issued (into wr)
-    for (int w = b; w < W; w += G) {
-      const int pr = w / S, j = w - pr * S, t = pr / k, s = pr - t * k;
-      if (l > 0) {
-        // tokens are independent: wait only for token t's layer-l input (its
-        // row and router block sums, released by the CTA that assembled it),
-        // then route token t alone
-        if (!token_wait(p.tflag + t, l, p.bar, p.status)) {
-          cp_wait_all();
-          return;
-        }
-        if (w == b) stamp2(p, l, 1);
-        for (int i = tid; i < N; i += blockDim.x) {
-          float zz = 0.0f;
-          for (int m = 0; m < nblk; ++m)
-            zz = __fadd_rn(zz, __ldcg(p.zb + ((size_t)m * N + i) * T + t));
-          z[t * N + i] = L.bias ? __fadd_rn(zz, L.bias[i]) : zz;
-        }
-        __syncthreads();
-        if (tid == 0) {
-          if (N == 8 && k == 2)
-            topk8_k2(z + t * N, p.renorm, sel + t * k, aw + t * k);
-          else if (N <= 8)
-            topk_token<8>(z + t * N, N, k, p.renorm, sel + t * k, aw + t * k);
-          else if (N <= 32)
-            topk_token<32>(z + t * N, N, k, p.renorm, sel + t * k, aw + t * k);
-          else
-            topk_wide(z + t * N, N, k, p.renorm, sel + t * k, aw + t * k);
-        }
-        __syncthreads();
-        if (s == 0 && j == 0)  // one of the token's items writes its routing
-          for (int x = tid; x < k; x += blockDim.x) {
-            if (p.top_idx) p.top_idx[(size_t)l * Tk + t * k + x] = sel[t * k + x];
-            if (last && p.top_w) p.top_w[t * k + x] = aw[t * k + x];
-          }
-        if (w == b) {
-          stamp2(p, l, 2);
-          stamp2(p, l, 3);
-        }
-      }
-      const int e = sel[pr];
-      // the token's row and the slice's gate and up rows (one group), the
-      // slice's down columns (another group, waited for after the dots)
-      stage_bytes(uh, u_cur + (size_t)t * d, d * 2);
-      const size_t grow = (size_t)e * h + (size_t)j * hS;
-      stage_bytes(gq, L.gq + grow * (d / 2), hS * (d / 2));
-      stage_bytes(gq + (size_t)hS * (d / 2), L.uq + grow * (d / 2), hS * (d / 2));
-      stage_bytes(gs, L.gs + grow * nb, hS * nb * 2);
-      stage_bytes(gs + (size_t)hS * nb, L.us + grow * nb, hS * nb * 2);
-      cp_commit();
-      const int cpr = hS / 32;  // 16-byte pieces of a down row's slice
-      for (int i = tid; i < d * cpr; i += blockDim.x) {
-        const int o = i / cpr, c = i - o * cpr;
-        cp16(dq + (size_t)o * (hS / 2) + c * 16,
-             L.dq + ((size_t)e * d + o) * (h / 2) + (size_t)j * (hS / 2) + c * 16);
-      }
-      stage_bytes(ds, L.ds + (size_t)e * d * nbh, d * nbh * 2);
-      cp_commit();
-      // the next layer's router rows, for the block sums of the tokens this
-      // CTA assembles (routing, above, was the last reader of the buffer);
-      // their own group, waited for before an assembly
-      if (!last && !rows_next)
-        stage_rows(reinterpret_cast<char*>(wr), ws_ld * 4,
-                   reinterpret_cast<const char*>(p.layer[l + 1].w_route), (size_t)d * 4, N,
-                   d * 4);
-      rows_next = true;
-      cp_commit();
-      cp_wait_group<2>();  // the row and the gate/up rows
-      __syncthreads();
-      if (w == b) {
-        stamp2(p, l, 4);
-        stamp2(p, l, 5);
-      }
-      for (int i = tid; i < d; i += blockDim.x) uf[i] = __half2float(uh[i]);
-      __syncthreads();
-      // gate/up dots: thread = (row r2 of the 2 hS gate/up rows, part pp of
-      // d), weights dequantised in registers
-      for (int u2 = tid; u2 < 2 * hS * nparts; u2 += blockDim.x) {
-        const int r2 = u2 % (2 * hS), pp = u2 / (2 * hS);
-        const int b0 = pp * nb / nparts, b1 = (pp + 1) * nb / nparts;
-        const uint8_t* q = gq + (size_t)r2 * (d / 2);
-        const uint16_t* sc = gs + (size_t)r2 * nb;
-        // per block: sum of (q - 8) x over its 32 weights in four chains,
-        // then one multiply-add by the block scale
-        float acc = 0.0f;
-#pragma unroll 2
-        for (int blk = b0; blk < b1; ++blk) {
-          const uint4 raw = *reinterpret_cast<const uint4*>(q + blk * 16);
-          const uint32_t wd[4] = {raw.x, raw.y, raw.z, raw.w};
-          const float4* x4 = reinterpret_cast<const float4*>(uf + blk * 32);
-          float c0 = 0.0f, c1 = 0.0f, c2 = 0.0f, c3 = 0.0f;
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const uint32_t lo = wd[i] & 0x0F0F0F0Fu, hi = (wd[i] >> 4) & 0x0F0F0F0Fu;
-            const float4 xl = x4[i], xh = x4[4 + i];  // elements 4i.. and 16+4i..
-            c0 = fmaf(nib(lo, 0), xl.x, c0);
-            c1 = fmaf(nib(lo, 1), xl.y, c1);
-            c2 = fmaf(nib(lo, 2), xl.z, c2);
-            c3 = fmaf(nib(lo, 3), xl.w, c3);
-            c0 = fmaf(nib(hi, 0), xh.x, c0);
-            c1 = fmaf(nib(hi, 1), xh.y, c1);
-            c2 = fmaf(nib(hi, 2), xh.z, c2);
-            c3 = fmaf(nib(hi, 3), xh.w, c3);
-          }
-          acc = fmaf(f16f(sc[blk]), (c0 + c1) + (c2 + c3), acc);
-        }
-        part[r2 * nparts + pp] = acc;
-      }
-      __syncthreads();
-      if (w == b) stamp2(p, l, 6);
-      for (int r = tid; r < hS; r += blockDim.x) {
-        float g = 0.0f, v = 0.0f;
-        for (int pp = 0; pp < nparts; ++pp) {
-          g += part[r * nparts + pp];
-          v += part[(hS + r) * nparts + pp];
-        }
-        hsv[r] = silu(g) * v;
-      }
-      cp_wait_group<1>();  // the down slice
-      __syncthreads();
-      if (w == b) {
-        stamp2(p, l, 7);
-        stamp2(p, l, 8);
-        stamp2(p, l, 9);
-      }
-      // partial output: row o of W_down[e] over the slice's hidden units
-      float* yp = p.ypart + ((size_t)t * KS + (size_t)s * S + j) * d;
-      for (int o = tid; o < d; o += blockDim.x) {
-        const uint8_t* q = dq + (size_t)o * (hS / 2);
-        float a0 = 0.0f, a1 = 0.0f;
-#pragma unroll 2
-        for (int bl = 0; bl < cpr; ++bl) {
-          float wv[32];
-          dequant_block(q + bl * 16, ds[(size_t)o * nbh + (size_t)j * cpr + bl], wv);
-          const float* hb = hsv + bl * 32;
-#pragma unroll
-          for (int c = 0; c < 32; c += 2) {
-            a0 = fmaf(wv[c], hb[c], a0);
-            a1 = fmaf(wv[c + 1], hb[c + 1], a1);
-          }
-        }
-        yp[o] = a0 + a1;
-      }
-      __syncthreads();
-      if (tid == 0) {  // publish the row, count it; the last row's CTA assembles
-        int old;
-        // release: the CTA's partial-row stores (ordered before by the
-        // barrier above) become visible with the count; acquire: the last
-        // counter sees every other partial row
-        asm volatile("atom.add.acq_rel.gpu.s32 %0, [%1], 1;"
-                     : "=r"(old)
-                     : "l"(p.tcnt + t)
-                     : "memory");
-        *flag = old == KS - 1;
-      }
-      __syncthreads();
-      if (w == b) stamp2(p, l, 10);
-      if (*flag) {
-        for (int o = tid; o < d; o += blockDim.x) {
-          float acc = 0.0f;
-          for (int s2 = 0; s2 < k; ++s2) {
-            float ys = 0.0f;
-            for (int j2 = 0; j2 < S; ++j2)
-              ys += __ldcg(p.ypart + ((size_t)t * KS + (size_t)s2 * S + j2) * d + o);
-            acc = fmaf(aw[t * k + s2], ys, acc);
-          }
-          if (last && p.y) p.y[(size_t)t * d + o] = __float2half_rn(acc);
-          const __half un = __float2half_rn(__half2float(uh[o]) + acc);
-          if (u_next) u_next[(size_t)t * d + o] = un;
-          uf[o] = __half2float(un);
-        }
-        if (tid == 0) p.tcnt[t] = 0;
-        if (!last) {
-          cp_wait_group<0>();  // the next layer's router rows
-          __syncthreads();
-          // the next layer's router block sums of u_{l+1}[t]: one ascending
-          // FMA chain per (expert, 128-input block)
-          for (int q = tid; q < N * nblk; q += blockDim.x) {
-            const int i = q % N, m = q / N, j0 = m * kRouteBlock;
-            const int len = min(kRouteBlock, d - j0);
-            const float4* w4 = reinterpret_cast<const float4*>(wr + (size_t)i * ws_ld + j0);
-            const float4* x4 = reinterpret_cast<const float4*>(uf + j0);
-            float c = 0.0f;
+    stamp2(p, l, 1);
+    // ---- route token t: block chains over its row, sums in block order, top-k
+    for (int q = tid; q < N * nblk; q += blockDim.x) {
+      const int i = q % N, m = q / N, j0 = m * kRouteBlock;
+      const int len = min(kRouteBlock, d - j0);
+      const float4* w4 = reinterpret_cast<const float4*>(wr + (size_t)i * ws_ld + j0);
+      const float4* x4 = reinterpret_cast<const float4*>(uf + j0);
+      float c = 0.0f;
 #pragma unroll 4
-            for (int s4 = 0; s4 < len / 4; ++s4) {
-              const float4 wv = w4[s4], x = x4[s4];
-              c = __fmaf_rn(wv.x, x.x, c);
-              c = __fmaf_rn(wv.y, x.y, c);
-              c = __fmaf_rn(wv.z, x.z, c);
-              c = __fmaf_rn(wv.w, x.w, c);
-            }
-            p.zb[((size_t)m * N + i) * T + t] = c;
-          }
-        }
-        __syncthreads();  // the row and its block sums stored by every thread
-        if (tid == 0)
-          asm volatile("st.release.gpu.global.s32 [%0], %1;" ::"l"(p.tflag + t), "r"(l + 1)
-                       : "memory");
+      for (int s4 = 0; s4 < len / 4; ++s4) {
+        const float4 wv = w4[s4], x = x4[s4];
+        c = __fmaf_rn(wv.x, x.x, c);
+        c = __fmaf_rn(wv.y, x.y, c);
+        c = __fmaf_rn(wv.z, x.z, c);
+        c = __fmaf_rn(wv.w, x.w, c);
       }
-      if (w == b) stamp2(p, l, 11);
-      __syncthreads();  // the staging buffers are refilled by the next item
+      zp[m * N + i] = c;
     }
-    if (b >= W)
-      for (int i = 1; i < 12; ++i) stamp2(p, l, i);
-    // the router rows must land before the next layer refills the buffer
-    cp_wait_all();
-    // CTA b < N S pulls the next layer's gate/up
-    // rows of (expert b / S, slice b % S) and, for slice 0, the expert's down
-    // rows into L2, so that the items' copies after routing hit L2
+    __syncthreads();
+    for (int i = tid; i < N; i += blockDim.x) {
+      float zz = 0.0f;
+      for (int m = 0; m < nblk; ++m) zz = __fadd_rn(zz, zp[m * N + i]);
+      z[i] = L.bias ? __fadd_rn(zz, L.bias[i]) : zz;
+    }
+    __syncthreads();
+    if (tid == 0) {
+      if (N == 8 && k == 2)
+        topk8_k2(z, p.renorm, sel, aw);
+      else if (N <= 8)
+        topk_token<8>(z, N, k, p.renorm, sel, aw);
+      else if (N <= 32)
+        topk_token<32>(z, N, k, p.renorm, sel, aw);
+      else
+        topk_wide(z, N, k, p.renorm, sel, aw);
+    }
+    __syncthreads();
+    if (writer)
+      for (int x = tid; x < k; x += blockDim.x) {
+        if (p.top_idx) p.top_idx[(size_t)l * Tk + t * k + x] = sel[x];
+        if (last && p.top_w) p.top_w[t * k + x] = aw[x];
+      }
+    stamp2(p, l, 2);
+    stamp2(p, l, 3);
+    const int e = sel[s];
+    // ---- the slice's gate and up rows (one group), its down columns
+    // (another), the next layer's router rows (a third; routing above was
+    // the last reader of the buffer)
+    const size_t grow = (size_t)e * h + (size_t)j * hS;
+    stage_bytes(gq, L.gq + grow * (d / 2), hS * (d / 2));
+    stage_bytes(gq + (size_t)hS * (d / 2), L.uq + grow * (d / 2), hS * (d / 2));
+    stage_bytes(gs, L.gs + grow * nb, hS * nb * 2);
+    stage_bytes(gs + (size_t)hS * nb, L.us + grow * nb, hS * nb * 2);
+    cp_commit();
+    for (int i = tid; i < d * cpr; i += blockDim.x) {
+      const int o = i / cpr, c = i - o * cpr;
+      cp16(dq + (size_t)o * (hS / 2) + c * 16,
+           L.dq + ((size_t)e * d + o) * (h / 2) + (size_t)j * (hS / 2) + c * 16);
+    }
+    stage_bytes(ds, L.ds + (size_t)e * d * nbh, d * nbh * 2);
+    cp_commit();
+    if (!last)
+      stage_rows(reinterpret_cast<char*>(wr), ws_ld * 4,
+                 reinterpret_cast<const char*>(p.layer[l + 1].w_route), (size_t)d * 4, N,
+                 d * 4);
+    cp_commit();
+    cp_wait_group<2>();  // the gate/up rows
+    __syncthreads();
+    stamp2(p, l, 4);
+    stamp2(p, l, 5);
+    // ---- gate/up dots: thread = (row r2 of the 2 hS gate/up rows, part pp
+    // of d); per q4 block the sum of (q - 8) x, then one multiply-add by the
+    // block scale
+    for (int u2 = tid; u2 < 2 * hS * nparts; u2 += blockDim.x) {
+      const int r2 = u2 % (2 * hS), pp = u2 / (2 * hS);
+      const int b0 = pp * nb / nparts, b1 = (pp + 1) * nb / nparts;
+      const uint8_t* q = gq + (size_t)r2 * (d / 2);
+      const uint16_t* sc = gs + (size_t)r2 * nb;
+      float acc = 0.0f;
+#pragma unroll 2
+      for (int blk = b0; blk < b1; ++blk) {
+        const uint4 raw = *reinterpret_cast<const uint4*>(q + blk * 16);
+        const uint32_t wd[4] = {raw.x, raw.y, raw.z, raw.w};
+        const float4* x4 = reinterpret_cast<const float4*>(uf + blk * 32);
+        float c0 = 0.0f, c1 = 0.0f, c2 = 0.0f, c3 = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const uint32_t lo = wd[i] & 0x0F0F0F0Fu, hi = (wd[i] >> 4) & 0x0F0F0F0Fu;
+          const float4 xl = x4[i], xh = x4[4 + i];  // elements 4i.. and 16+4i..
+          c0 = fmaf(nib(lo, 0), xl.x, c0);
+          c1 = fmaf(nib(lo, 1), xl.y, c1);
+          c2 = fmaf(nib(lo, 2), xl.z, c2);
+          c3 = fmaf(nib(lo, 3), xl.w, c3);
+          c0 = fmaf(nib(hi, 0), xh.x, c0);
+          c1 = fmaf(nib(hi, 1), xh.y, c1);
+          c2 = fmaf(nib(hi, 2), xh.z, c2);
+          c3 = fmaf(nib(hi, 3), xh.w, c3);
+        }
+        acc = fmaf(f16f(sc[blk]), (c0 + c1) + (c2 + c3), acc);
+      }
+      part[r2 * nparts + pp] = acc;
+    }
+    __syncthreads();
+    stamp2(p, l, 6);
+    for (int r = tid; r < hS; r += blockDim.x) {
+      float g = 0.0f, v = 0.0f;
+      for (int pp = 0; pp < nparts; ++pp) {
+        g += part[r * nparts + pp];
+        v += part[(hS + r) * nparts + pp];
+      }
+      hsv[r] = silu(g) * v;
+    }
+    cp_wait_group<1>();  // the down columns
+    __syncthreads();
+    stamp2(p, l, 7);
+    stamp2(p, l, 8);
+    stamp2(p, l, 9);
+    // ---- partial output row: row o of W_down[e] over the slice's hidden units
+    float* ybuf = p.ypart + (size_t)(l & 1) * Tk * S * d + (size_t)t * KS * d;
+    for (int o = tid; o < d; o += blockDim.x) {
+      const uint8_t* q = dq + (size_t)o * (hS / 2);
+      float a0 = 0.0f, a1 = 0.0f;
+#pragma unroll 2
+      for (int bl = 0; bl < cpr; ++bl) {
+        float wv[32];
+        dequant_block(q + bl * 16, ds[(size_t)o * nbh + (size_t)j * cpr + bl], wv);
+        const float* hb = hsv + bl * 32;
+#pragma unroll
+        for (int c = 0; c < 32; c += 2) {
+          a0 = fmaf(wv[c], hb[c], a0);
+          a1 = fmaf(wv[c + 1], hb[c + 1], a1);
+        }
+      }
+      ybuf[(size_t)(s * S + j) * d + o] = a0 + a1;
+    }
+    __syncthreads();
+    if (tid == 0)  // release: the CTA's stores (ordered by the barrier above) with the count
+      asm volatile("red.release.gpu.global.add.s32 [%0], 1;" ::"l"(p.tcnt + t) : "memory");
+    stamp2(p, l, 10);
+    // while the token's other items finish: CTA b < N S pulls the next
+    // layer's gate/up rows of (expert b / S, slice b % S) into L2
     if (!last && b < N * S && tid == 0) {
       const LayerPtrs& Ln = p.layer[l + 1];
-      const int e = b / S, j = b - (b / S) * S;
-      const size_t grow = (size_t)e * h + (size_t)j * hS;
-      l2_prefetch(Ln.gq + grow * (d / 2), hS * (d / 2));
-      l2_prefetch(Ln.uq + grow * (d / 2), hS * (d / 2));
-      if (j == 0) l2_prefetch(Ln.dq + (size_t)e * d * (h / 2), d * (h / 2));
+      const int ep = b / S, jp = b - (b / S) * S;
+      const size_t gp = (size_t)ep * h + (size_t)jp * hS;
+      l2_prefetch(Ln.gq + gp * (d / 2), hS * (d / 2));
+      l2_prefetch(Ln.uq + gp * (d / 2), hS * (d / 2));
+      if (jp == 0) l2_prefetch(Ln.dq + (size_t)ep * d * (h / 2), d * (h / 2));
     }
+    if (!count_wait(p.tcnt + t, KS * (l + 1), p.bar + 1, p.status)) {
+      cp_wait_all();
+      return;
+    }
+    stamp2(p, l, 11);
+    // ---- the token's next row, the same in each of its CTAs
+    for (int o = tid; o < d; o += blockDim.x) {
+      float acc = 0.0f;
+      for (int s2 = 0; s2 < k; ++s2) {
+        float ys = 0.0f;
+        for (int j2 = 0; j2 < S; ++j2) ys += __ldcg(ybuf + (size_t)(s2 * S + j2) * d + o);
+        acc = fmaf(aw[s2], ys, acc);
+      }
+      const __half un = __float2half_rn(__half2float(uh[o]) + acc);
+      if (last && writer) {
+        if (p.y) p.y[(size_t)t * d + o] = __float2half_rn(acc);
+        if (p.u_out) p.u_out[(size_t)t * d + o] = un;
+      }
+      uh[o] = un;
+      uf[o] = __half2float(un);
+    }
+    cp_wait_group<0>();  // the next layer's router rows
+    __syncthreads();
     stamp2(p, l, 12);
   }
 }
@@ -1250,12 +1191,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused(const __grid_constan
 // ------------------------------------------------------------------ host
 struct WsLayout {
   float* H;
-  float* ypart;  // one-barrier kernel: [T][k h/32][d] partial rows (at most h/32 slices)
+  float* ypart;  // per-token kernel: [2][T][k h/32][d] partial rows (at most h/32 slices)
   float* zb;
   int32_t* idx;
   float* w;
   __half* work;
-  unsigned* bar;  // [0..3] barrier words, then [T] per-token counters, [T] per-token flags
+  unsigned* bar;  // [0..3] barrier words, then [T] per-token counters
   size_t bytes;
 };
 
@@ -1263,12 +1204,12 @@ WsLayout carve_decode(const moe_shape& s, void* base) {
   Carver c(base);
   WsLayout L;
   L.H = c.take<float>((size_t)s.N * s.T * s.h);
-  L.ypart = c.take<float>((size_t)s.T * s.k * (s.h / 32) * s.d);
+  L.ypart = c.take<float>((size_t)2 * s.T * s.k * (s.h / 32) * s.d);
   L.zb = c.take<float>((size_t)((s.d + kRouteBlock - 1) / kRouteBlock) * s.N * s.T);
   L.idx = c.take<int32_t>((size_t)s.T * s.k);
   L.w = c.take<float>((size_t)s.T * s.k);
   L.work = c.take<__half>((size_t)s.T * s.d);
-  L.bar = c.take<unsigned>(4 + 2 * (size_t)s.T);
+  L.bar = c.take<unsigned>(4 + (size_t)s.T);
   L.bytes = c.used();
   return L;
 }
@@ -1285,11 +1226,11 @@ bool device_info(int* sms) {
     if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
         cudaFuncSetAttribute(decode_persistent, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)kSmemLimit) != cudaSuccess ||
-        cudaFuncSetAttribute(decode_fused, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaFuncSetAttribute(decode_token, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)kSmemLimit) != cudaSuccess)
       return false;
     MOE_PREFER_SHARED((decode_persistent));
-    MOE_PREFER_SHARED((decode_fused));
+    MOE_PREFER_SHARED((decode_token));
     sm_count[dev].store(n, std::memory_order_relaxed);
     mark_setup(configured, dev);
   }
@@ -1340,19 +1281,19 @@ cudaError_t launch_coop(const void* kernel, int grid, size_t smem, cudaStream_t 
 }
 
 // The one-barrier kernel over layers [0, n) when its plan fits.
-int launch_decode_fused(const moe_shape& s, const Plan2& plan, int sms, const moe_q4_layer* layers,
-                        int n, const __half* u_in, __half* u_out, __half* y, int32_t* top_idx,
+// The per-token kernel over layers [0, n): T k S CTAs, one item each.
+int launch_decode_token(const moe_shape& s, const Plan2& plan, const moe_q4_layer* layers, int n,
+                        const __half* u_in, __half* u_out, __half* y, int32_t* top_idx,
                         float* top_w, const WsLayout& W, cudaStream_t st,
                         unsigned long long* stamps) {
   int occ = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, decode_fused, kThreads, plan.total) !=
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, decode_token, kThreads, plan.total) !=
       cudaSuccess)
     return MOE_ERR_CUDA;
   if (occ < 1) return MOE_ERR_UNSUPPORTED;
   Params2 p{};
   p.plan = plan;
-  const int items = s.T * s.k * plan.S;
-  const int grid = items < sms ? items : sms;
+  const int grid = s.T * s.k * plan.S;  // <= the SM count by the plan
   for (int l = 0; l < n; ++l) p.layer[l] = layer_ptrs(layers[l]);
   p.n_layers = n;
   p.T = s.T;
@@ -1362,28 +1303,27 @@ int launch_decode_fused(const moe_shape& s, const Plan2& plan, int sms, const mo
   p.h = s.h;
   p.renorm = s.renorm;
   p.u_in = u_in;
-  p.u_work = W.work;
   p.u_out = u_out;
   p.y = y;
   p.top_idx = top_idx;
   p.top_w = top_w;
   p.ypart = W.ypart;
   p.tcnt = reinterpret_cast<int*>(W.bar + 4);
-  p.tflag = reinterpret_cast<int*>(W.bar + 4 + s.T);
-  p.zb = W.zb;
   p.bar = W.bar;
   p.status = status_word();
   p.stamps = stamps;
-  if (cudaMemsetAsync(W.bar, 0, (4 + 2 * (size_t)s.T) * sizeof(unsigned), st) != cudaSuccess)
+  if (cudaMemsetAsync(W.bar, 0, (4 + (size_t)s.T) * sizeof(unsigned), st) != cudaSuccess)
     return MOE_ERR_CUDA;
-  return launch_coop(reinterpret_cast<const void*>(decode_fused), grid, plan.total, st, &p) ==
+  // cooperative: every CTA resident at once, which the bounded count waits need
+  return launch_coop(reinterpret_cast<const void*>(decode_token), grid, plan.total, st, &p) ==
                  cudaSuccess
              ? MOE_OK
              : MOE_ERR_CUDA;
 }
 
-// One cooperative launch over layers [0, n) of `layers`: the one-barrier
-// kernel when its shared-memory plan fits, else the two-phase kernel.
+// One cooperative launch over layers [0, n) of `layers`: the per-token
+// kernel when its items fit one per SM and its shared-memory plan fits,
+// else the two-phase kernel.
 int launch_decode(const moe_shape& s, const moe_q4_layer* layers, int n, const __half* u_in,
                   __half* u_out, __half* y, int32_t* top_idx, float* top_w, const WsLayout& W,
                   cudaStream_t st, unsigned long long* stamps = nullptr) {
@@ -1391,7 +1331,7 @@ int launch_decode(const moe_shape& s, const moe_q4_layer* layers, int n, const _
   if (!device_info(&sms)) return MOE_ERR_CUDA;
   Plan2 plan2;
   if (make_plan2(s, sms, &plan2))
-    return launch_decode_fused(s, plan2, sms, layers, n, u_in, u_out, y, top_idx, top_w, W, st,
+    return launch_decode_token(s, plan2, layers, n, u_in, u_out, y, top_idx, top_w, W, st,
                                stamps);
   Params p{};
   if (!make_plan(s, sms, &p.plan)) return MOE_ERR_UNSUPPORTED;
