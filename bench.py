@@ -607,11 +607,11 @@ class DecodeReplica:
         return sum(t.numel() * t.element_size() for t in self.keep)
 
 
-# Intervals between the 13 per-layer stamps of the one-barrier decode kernel
+# Intervals between the 13 per-layer stamps of the per-token decode kernel
 # (the kernel the benchmark shapes run); the bracketed ones are empty there.
-DECODE_PHASES = ("start", "route", "(stamps 2-3)", "stage item rows", "(stamps 4-5)",
+DECODE_PHASES = ("(stamps 0-1)", "route", "(stamps 2-3)", "stage item rows", "(stamps 4-5)",
                  "gate/up dots", "H", "(stamps 7-8)", "down columns ready",
-                 "down partial + count", "token assembly", "barrier")
+                 "down partial + count", "wait for the token's rows", "next row")
 
 
 def decode_phases(wl, moe, s, rep, out, ws, torch, sm_mhz: float):

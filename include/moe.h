@@ -457,27 +457,27 @@ MOE_API int moe_decode_layer(const moe_shape* shape, const moe_q4_layer* layer, 
 /* n_layers chained layers: u_{l+1} = fp16(u_l + y_l), u_out = u_{n_layers}.
  * `layers` is a host array of n_layers structs.  top_idx_all [n_layers][T][k]
  * (nullable) receives every layer's routing.  Up to 32 layers run in one
- * cooperative launch (at most one CTA per SM, every grid-barrier wait
- * bounded: MOE_ERR_TIMEOUT in the device status word).  When its
- * shared-memory plan fits, the launch takes (token, slot, hidden slice)
- * items with one grid barrier per layer (the last CTA to store a token's
- * partial output row assembles the token); otherwise it runs a two-phase
- * kernel (selected-expert hidden slices, barrier, (token, output rows)
- * units, barrier).  The kernel is chosen from the shape, so a chain and
- * moe_decode_layer use the same per-layer arithmetic and a chain equals the
- * layer calls made one by one.  Capturable in a CUDA graph. */
+ * cooperative launch (at most one CTA per SM, every wait bounded:
+ * MOE_ERR_TIMEOUT in the device status word).  When the T k (token, slot)
+ * pairs fit one CTA each and its shared-memory plan fits, the launch runs
+ * the per-token kernel (CTA = (token, slot, hidden slice) for all layers,
+ * the token's CTAs exchanging partial output rows through a per-token
+ * counter, no grid barrier); otherwise a two-phase kernel (selected-expert
+ * hidden slices, grid barrier, (token, output rows) units, grid barrier).
+ * The kernel is chosen from the shape, so a chain and moe_decode_layer use
+ * the same per-layer arithmetic and a chain equals the layer calls made one
+ * by one.  Capturable in a CUDA graph. */
 MOE_API int moe_decode_step(const moe_shape* shape, int32_t n_layers, const moe_q4_layer* layers,
                             const uint16_t* u0, uint16_t* u_out, int32_t* top_idx_all, void* ws,
                             size_t ws_bytes, void* stream);
 
 /* moe_decode_step that also records, for each layer, 13 SM-cycle stamps
  * (clock64 of block 0, thread 0) into stamps [n_layers][13] (device memory,
- * 8-byte aligned; caller-owned).  One-barrier kernel: 0 layer start,
- * 1 input staged (first layer of a launch) or ready to read the router
- * block sums, 2 routed, 3 = 2, 4 the item's token row and gate/up rows
- * staged, 5 = 4, 6 gate/up dots formed, 7 H formed, 8 = 7, 9 down columns
- * ready, 10 partial output row stored and counted, 11 token assembled
- * (= 10 when block 0 was not the token's last), 12 grid barrier passed.
+ * 8-byte aligned; caller-owned).  Per-token kernel (block 0 = token 0,
+ * slot 0, slice 0): 0 layer start, 1 = 0, 2 routed, 3 = 2, 4 the slice's
+ * gate/up rows staged, 5 = 4, 6 gate/up dots formed, 7 H formed, 8 = 7,
+ * 9 down columns ready, 10 partial output row stored and counted, 11 all of
+ * the token's partial rows counted, 12 next row formed.
  * Two-phase kernel: 0 layer start, 1 input rows staged, 2 routed, 3
  * dispatch pairs grouped by expert, 4 gate/up q4 rows staged, 5 = 4, 6
  * gate/up dots formed, 7 hidden phase done (H stored), 8 first grid barrier

@@ -143,11 +143,11 @@ def test_decode_reads_only_selected_experts():
 
 
 @pytest.mark.parametrize("T,d,N,k,h", [
-    (32, 512, 64, 8, 128),   # 64 experts top-8: several phase-A items per CTA
-    (32, 1024, 8, 2, 256),   # 8 output rows per phase-B slice, h/32 = 8 parts
+    (32, 512, 64, 8, 128),   # 64 experts top-8: more items than SMs, the two-phase kernel
+    (32, 1024, 8, 2, 256),   # h = 256: the two-phase kernel (the per-token plan is too large)
     (5, 64, 4, 2, 32),       # tiny: one q4 block per hidden row, ragged T
     (3, 96, 4, 3, 64),       # d/32 = 3 blocks: uneven phase-A parts
-    (16, 2048, 8, 2, 128),   # too wide for the one-barrier plan: the two-phase kernel
+    (16, 2048, 8, 2, 128),   # wide rows: per-token kernel with 4 hidden slices of 32
 ])
 def test_decode_layer_other_shapes(T, d, N, k, h):
     import dataclasses
@@ -167,10 +167,10 @@ def test_decode_layer_other_shapes(T, d, N, k, h):
 
 
 @pytest.mark.parametrize("T,d,N,k,h", [
-    (32, 1024, 8, 2, 256),   # phase-B units of 256 rows: two router blocks each
-    (32, 512, 64, 8, 128),   # 64 experts: 64 block sums per unit
-    (16, 512, 8, 2, 128),    # units of 64 rows: every layer runs its own chains
-    (16, 2048, 8, 2, 128),   # the two-phase kernel (the one-barrier plan does not fit)
+    (32, 1024, 8, 2, 256),   # two-phase kernel, output units of 256 rows: two router blocks each
+    (32, 512, 64, 8, 128),   # two-phase kernel, 64 experts: 64 block sums per unit
+    (16, 512, 8, 2, 128),    # per-token kernel, 16 tokens x 2 slots x 4 slices
+    (16, 2048, 8, 2, 128),   # per-token kernel, wide rows
 ])
 def test_decode_step_equals_layers(T, d, N, k, h):
     """A 3-layer chained step (layers 1.. route from the router block sums
