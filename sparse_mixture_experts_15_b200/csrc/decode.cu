@@ -861,19 +861,21 @@ __global__ void __launch_bounds__(kThreads, 1) decode_persistent(const __grid_co
 // 128-input block chains of its logits, top-k), stages the selected
 // expert's gate and up rows of slice j and the slice's down columns, forms
 // H_j = SiLU(W_gate u) * (W_up u) on chip and the partial output row
-// W_down[:, slice j] H_j, stores that row and counts it on the token's
-// counter.  Once the token's k S rows are counted, each of the token's CTAs
-// sums them in one fixed order (slots in order, each slot's slices in
-// order) into u_{l+1}[t] = fp16(u_l + y), so all of them hold the same next
-// row and route it to the same experts.  Partial rows alternate between two
-// buffers by layer parity: a CTA can start layer l+1 only after every item
-// of its token counted layer l, i.e. after every reader of layer l-1's rows
-// has moved on.  Only the selected experts' rows are read.
+// W_down[:, slice j] H_j in its own shared memory.  A token's k S CTAs form
+// one thread-block cluster: after a cluster barrier each of them reads the
+// token's k S partial rows from the cluster's shared memory and sums them in
+// one fixed order (slots in order, each slot's slices in order) into
+// u_{l+1}[t] = fp16(u_l + y), so all of them hold the same next row and
+// route it to the same experts.  Partial rows alternate between two buffers
+// by layer parity: a CTA passes the next layer's cluster barrier only after
+// every peer has read this layer's rows.  Nothing waits across clusters, so
+// the launch needs no co-residency beyond the cluster's.  Only the selected
+// experts' rows are read.
 struct Plan2 {
   int S;       // hidden slices per (token, slot)
   int hS;      // hidden units per slice
   int nparts;  // parts of d per gate/up row (one thread each)
-  uint32_t wr, z, sel, aw, zp, uh, uf, gq, gs, dq, ds, part, hs, misc;
+  uint32_t wr, z, sel, aw, zp, uh, uf, gq, gs, dq, ds, part, hs, yr, misc;
   uint32_t total;
 };
 
@@ -887,18 +889,14 @@ struct Params2 {
   __half* y;
   int32_t* top_idx;
   float* top_w;
-  float* ypart;  // [2][T][k S][d] partial output rows, by layer parity
-  int* tcnt;     // [T] partial rows counted so far (k S per layer)
-  unsigned* bar;  // [1]: abort flag
-  int* status;
   unsigned long long* stamps;
 };
 
 // Stamps of the per-token kernel, in the same 13 slots (block 0's item):
 // 0 layer start, 1 = 0, 2 routed, 3 = 2, 4 the item's gate/up rows staged,
 // 5 = 4, 6 gate/up dots formed, 7 H formed, 8 = 7, 9 down columns ready,
-// 10 partial row stored and counted, 11 the token's rows all counted,
-// 12 next row formed.
+// 10 partial row in shared memory, 11 cluster barrier passed (every row of
+// the token there), 12 next row formed.
 __device__ __forceinline__ void stamp2(const Params2& p, int l, int i) {
   if (p.stamps && blockIdx.x == 0 && threadIdx.x == 0)
     p.stamps[(size_t)l * kStamps + i] = clock64();
@@ -912,10 +910,11 @@ __device__ __forceinline__ void l2_prefetch(const void* ptr, int bytes) {
 bool make_plan2(const moe_shape& s, int sms, Plan2* out) {
   const int T = s.T, d = s.d, N = s.N, k = s.k, h = s.h;
   const int nb = d / 32, nbh = h / 32, nblk = (d + kRouteBlock - 1) / kRouteBlock;
-  if ((int64_t)T * k > sms) return false;  // one CTA per item
-  // the most slices that keep one CTA per item
+  if ((int64_t)T * k > sms || k > 8) return false;  // one CTA per item, clusters <= 8
+  // the most slices that keep one CTA per item and k S within a portable
+  // cluster
   int S0 = 1;
-  while (2 * S0 <= nbh && (int64_t)T * k * 2 * S0 <= sms) S0 *= 2;
+  while (2 * S0 <= nbh && (int64_t)T * k * 2 * S0 <= sms && k * 2 * S0 <= 8) S0 *= 2;
   for (int S = S0; S >= 1; S /= 2) {
     const int hS = h / S;
     if (2 * hS > kThreads) break;
@@ -938,6 +937,7 @@ bool make_plan2(const moe_shape& s, int sms, Plan2* out) {
     p.ds = take(off, (size_t)d * nbh * 2);
     p.part = take(off, (size_t)2 * hS * p.nparts * 4);
     p.hs = take(off, (size_t)hS * 4);
+    p.yr = take(off, (size_t)2 * d * 4);
     p.misc = take(off, 16);
     p.total = off;
     if (off <= kSmemLimit) {
@@ -948,32 +948,22 @@ bool make_plan2(const moe_shape& s, int sms, Plan2* out) {
   return false;
 }
 
-// Thread 0 waits (bounded, 2 s of device time) until *f >= target, then the
-// CTA proceeds; false on timeout (MOE_ERR_TIMEOUT, abort raised) or abort.
-__device__ bool count_wait(const int* f, int target, unsigned* abort_flag, int* status) {
-  __shared__ int ok;
-  if (threadIdx.x == 0) {
-    int good = 1;
-    const unsigned long long t0 = global_ns();
-    unsigned polls = 0;
-    while ((int)ld_acquire(reinterpret_cast<const unsigned*>(f)) < target) {
-      if ((++polls & 15u) == 0) {
-        if (ld_acquire(abort_flag) != 0u) {
-          good = 0;
-          break;
-        }
-        if (global_ns() - t0 > kBarrierBudgetNs) {
-          record_error(status, MOE_ERR_TIMEOUT);
-          atomicExch(abort_flag, 1u);
-          good = 0;
-          break;
-        }
-      }
-    }
-    ok = good;
-  }
-  __syncthreads();
-  return ok != 0;
+// Cluster barrier of all threads (release / acquire, so shared-memory stores
+// before it are seen by the cluster's loads after it), a shared-memory
+// address of the cluster's CTA `rank`, and a load from it.
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
+                   : "memory");
+}
+__device__ __forceinline__ uint32_t cluster_addr(uint32_t local, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ float ld_cluster_f32(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+  return v;
 }
 
 __global__ void __launch_bounds__(kThreads, 1) decode_token(const __grid_constant__ Params2 p) {
@@ -997,7 +987,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_token(const __grid_constan
   uint16_t* ds = reinterpret_cast<uint16_t*>(sm + P.ds);
   float* part = reinterpret_cast<float*>(sm + P.part);
   float* hsv = reinterpret_cast<float*>(sm + P.hs);
-  if (b >= Tk * S) return;
+  float* yr = reinterpret_cast<float*>(sm + P.yr);
+  if (b >= Tk * S) return;  // (the grid is exactly T k S)
   const int pr = b / S, j = b - pr * S, t = pr / k, s = pr - t * k;
   const bool writer = s == 0 && j == 0;  // writes the token's routing and outputs
 
@@ -1129,8 +1120,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_token(const __grid_constan
     stamp2(p, l, 7);
     stamp2(p, l, 8);
     stamp2(p, l, 9);
-    // ---- partial output row: row o of W_down[e] over the slice's hidden units
-    float* ybuf = p.ypart + (size_t)(l & 1) * Tk * S * d + (size_t)t * KS * d;
+    // ---- partial output row: row o of W_down[e] over the slice's hidden
+    // units, into this CTA's buffer of the layer's parity
+    float* ymine = yr + (size_t)(l & 1) * d;
     for (int o = tid; o < d; o += blockDim.x) {
       const uint8_t* q = dq + (size_t)o * (hS / 2);
       float a0 = 0.0f, a1 = 0.0f;
@@ -1145,14 +1137,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_token(const __grid_constan
           a1 = fmaf(wv[c + 1], hb[c + 1], a1);
         }
       }
-      ybuf[(size_t)(s * S + j) * d + o] = a0 + a1;
+      ymine[o] = a0 + a1;
     }
-    __syncthreads();
-    if (tid == 0)  // release: the CTA's stores (ordered by the barrier above) with the count
-      asm volatile("red.release.gpu.global.add.s32 [%0], 1;" ::"l"(p.tcnt + t) : "memory");
     stamp2(p, l, 10);
-    // while the token's other items finish: CTA b < N S pulls the next
-    // layer's gate/up rows of (expert b / S, slice b % S) into L2
+    // while the cluster meets: CTA b < N S pulls the next layer's gate/up
+    // rows of (expert b / S, slice b % S) into L2
     if (!last && b < N * S && tid == 0) {
       const LayerPtrs& Ln = p.layer[l + 1];
       const int ep = b / S, jp = b - (b / S) * S;
@@ -1161,17 +1150,19 @@ __global__ void __launch_bounds__(kThreads, 1) decode_token(const __grid_constan
       l2_prefetch(Ln.uq + gp * (d / 2), hS * (d / 2));
       if (jp == 0) l2_prefetch(Ln.dq + (size_t)ep * d * (h / 2), d * (h / 2));
     }
-    if (!count_wait(p.tcnt + t, KS * (l + 1), p.bar + 1, p.status)) {
-      cp_wait_all();
-      return;
-    }
+    cluster_sync_all();  // every partial row of the token is in the cluster
     stamp2(p, l, 11);
-    // ---- the token's next row, the same in each of its CTAs
+    // ---- the token's next row, the same in each of its CTAs: cluster rank
+    // s2 S + j2 holds slot s2's slice j2
+    uint32_t peer[8];
+    const uint32_t ymine_a = static_cast<uint32_t>(__cvta_generic_to_shared(ymine));
+#pragma unroll
+    for (int r = 0; r < 8; ++r) peer[r] = r < KS ? cluster_addr(ymine_a, r) : 0u;
     for (int o = tid; o < d; o += blockDim.x) {
       float acc = 0.0f;
       for (int s2 = 0; s2 < k; ++s2) {
         float ys = 0.0f;
-        for (int j2 = 0; j2 < S; ++j2) ys += __ldcg(ybuf + (size_t)(s2 * S + j2) * d + o);
+        for (int j2 = 0; j2 < S; ++j2) ys += ld_cluster_f32(peer[s2 * S + j2] + 4u * o);
         acc = fmaf(aw[s2], ys, acc);
       }
       const __half un = __float2half_rn(__half2float(uh[o]) + acc);
@@ -1186,17 +1177,17 @@ __global__ void __launch_bounds__(kThreads, 1) decode_token(const __grid_constan
     __syncthreads();
     stamp2(p, l, 12);
   }
+  cluster_sync_all();  // no CTA leaves while a peer may still read its rows
 }
 
 // ------------------------------------------------------------------ host
 struct WsLayout {
   float* H;
-  float* ypart;  // per-token kernel: [2][T][k h/32][d] partial rows (at most h/32 slices)
   float* zb;
   int32_t* idx;
   float* w;
   __half* work;
-  unsigned* bar;  // [0..3] barrier words, then [T] per-token counters
+  unsigned* bar;  // [0] arrivals, [1] abort of the two-phase kernel's barriers
   size_t bytes;
 };
 
@@ -1204,12 +1195,11 @@ WsLayout carve_decode(const moe_shape& s, void* base) {
   Carver c(base);
   WsLayout L;
   L.H = c.take<float>((size_t)s.N * s.T * s.h);
-  L.ypart = c.take<float>((size_t)2 * s.T * s.k * (s.h / 32) * s.d);
   L.zb = c.take<float>((size_t)((s.d + kRouteBlock - 1) / kRouteBlock) * s.N * s.T);
   L.idx = c.take<int32_t>((size_t)s.T * s.k);
   L.w = c.take<float>((size_t)s.T * s.k);
   L.work = c.take<__half>((size_t)s.T * s.d);
-  L.bar = c.take<unsigned>(4 + (size_t)s.T);
+  L.bar = c.take<unsigned>(4);
   L.bytes = c.used();
   return L;
 }
@@ -1265,35 +1255,15 @@ LayerPtrs layer_ptrs(const moe_q4_layer& L) {
                    L.up_qs,   L.up_scales, L.down_qs, L.down_scales};
 }
 
-cudaError_t launch_coop(const void* kernel, int grid, size_t smem, cudaStream_t st, void* params) {
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeCooperative;
-  attr[0].val.cooperative = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  void* args[] = {params};
-  return cudaLaunchKernelExC(&cfg, kernel, args);
-}
-
 // The one-barrier kernel over layers [0, n) when its plan fits.
-// The per-token kernel over layers [0, n): T k S CTAs, one item each.
+// The per-token kernel over layers [0, n): T k S CTAs, one item each, in
+// clusters of k S (one token each).
 int launch_decode_token(const moe_shape& s, const Plan2& plan, const moe_q4_layer* layers, int n,
                         const __half* u_in, __half* u_out, __half* y, int32_t* top_idx,
-                        float* top_w, const WsLayout& W, cudaStream_t st,
-                        unsigned long long* stamps) {
-  int occ = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, decode_token, kThreads, plan.total) !=
-      cudaSuccess)
-    return MOE_ERR_CUDA;
-  if (occ < 1) return MOE_ERR_UNSUPPORTED;
+                        float* top_w, cudaStream_t st, unsigned long long* stamps) {
+  const int ks = s.k * plan.S;
   Params2 p{};
   p.plan = plan;
-  const int grid = s.T * s.k * plan.S;  // <= the SM count by the plan
   for (int l = 0; l < n; ++l) p.layer[l] = layer_ptrs(layers[l]);
   p.n_layers = n;
   p.T = s.T;
@@ -1307,23 +1277,29 @@ int launch_decode_token(const moe_shape& s, const Plan2& plan, const moe_q4_laye
   p.y = y;
   p.top_idx = top_idx;
   p.top_w = top_w;
-  p.ypart = W.ypart;
-  p.tcnt = reinterpret_cast<int*>(W.bar + 4);
-  p.bar = W.bar;
-  p.status = status_word();
   p.stamps = stamps;
-  if (cudaMemsetAsync(W.bar, 0, (4 + (size_t)s.T) * sizeof(unsigned), st) != cudaSuccess)
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(s.T * ks);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = plan.total;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = ks;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int clusters = 0;
+  if (cudaOccupancyMaxActiveClusters(&clusters, decode_token, &cfg) != cudaSuccess)
     return MOE_ERR_CUDA;
-  // cooperative: every CTA resident at once, which the bounded count waits need
-  return launch_coop(reinterpret_cast<const void*>(decode_token), grid, plan.total, st, &p) ==
-                 cudaSuccess
-             ? MOE_OK
-             : MOE_ERR_CUDA;
+  if (clusters < 1) return MOE_ERR_UNSUPPORTED;
+  return cudaLaunchKernelEx(&cfg, decode_token, p) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
-// One cooperative launch over layers [0, n) of `layers`: the per-token
-// kernel when its items fit one per SM and its shared-memory plan fits,
-// else the two-phase kernel.
+// One launch over layers [0, n) of `layers`: the per-token kernel (thread-
+// block clusters, one per token) when its items fit one per SM and its
+// shared-memory plan fits, else the cooperative two-phase kernel.
 int launch_decode(const moe_shape& s, const moe_q4_layer* layers, int n, const __half* u_in,
                   __half* u_out, __half* y, int32_t* top_idx, float* top_w, const WsLayout& W,
                   cudaStream_t st, unsigned long long* stamps = nullptr) {
@@ -1331,8 +1307,7 @@ int launch_decode(const moe_shape& s, const moe_q4_layer* layers, int n, const _
   if (!device_info(&sms)) return MOE_ERR_CUDA;
   Plan2 plan2;
   if (make_plan2(s, sms, &plan2))
-    return launch_decode_token(s, plan2, layers, n, u_in, u_out, y, top_idx, top_w, W, st,
-                               stamps);
+    return launch_decode_token(s, plan2, layers, n, u_in, u_out, y, top_idx, top_w, st, stamps);
   Params p{};
   if (!make_plan(s, sms, &p.plan)) return MOE_ERR_UNSUPPORTED;
   int occ = 0;
