@@ -1154,16 +1154,24 @@ __global__ void __launch_bounds__(kThreads, 1) decode_token(const __grid_constan
     stamp2(p, l, 11);
     // ---- the token's next row, the same in each of its CTAs: cluster rank
     // s2 S + j2 holds slot s2's slice j2
-    uint32_t peer[8];
     const uint32_t ymine_a = static_cast<uint32_t>(__cvta_generic_to_shared(ymine));
-#pragma unroll
-    for (int r = 0; r < 8; ++r) peer[r] = r < KS ? cluster_addr(ymine_a, r) : 0u;
+    const int lgS = __ffs(S) - 1;
     for (int o = tid; o < d; o += blockDim.x) {
-      float acc = 0.0f;
-      for (int s2 = 0; s2 < k; ++s2) {
-        float ys = 0.0f;
-        for (int j2 = 0; j2 < S; ++j2) ys += ld_cluster_f32(peer[s2 * S + j2] + 4u * o);
-        acc = fmaf(aw[s2], ys, acc);
+      // the k S rows' values of column o, loaded together, then summed in order
+      float yv[8];
+#pragma unroll
+      for (int r = 0; r < 8; ++r)
+        yv[r] = r < KS ? ld_cluster_f32(cluster_addr(ymine_a + 4u * o, r)) : 0.0f;
+      float acc = 0.0f, ys = 0.0f;
+#pragma unroll
+      for (int r = 0; r < 8; ++r) {
+        if (r < KS) {
+          ys += yv[r];
+          if (((r + 1) & (S - 1)) == 0) {  // slot r / S complete (S a power of 2)
+            acc = fmaf(aw[r >> lgS], ys, acc);
+            ys = 0.0f;
+          }
+        }
       }
       const __half un = __float2half_rn(__half2float(uh[o]) + acc);
       if (last && writer) {
