@@ -931,7 +931,7 @@ bool make_plan2(const moe_shape& s, int sms, Plan2* out) {
     p.zp = take(off, (size_t)N * nblk * 4);
     p.uh = take(off, (size_t)d * 2);
     p.uf = take(off, (size_t)d * 4);
-    p.gq = take(off, (size_t)2 * hS * (d / 2));
+    p.gq = take(off, (size_t)2 * hS * (d / 2 + 16));  // rows padded 16 B: no bank conflicts
     p.gs = take(off, (size_t)2 * hS * nb * 2);
     p.dq = take(off, (size_t)d * (hS / 2));
     p.ds = take(off, (size_t)d * nbh * 2);
@@ -1052,8 +1052,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_token(const __grid_constan
     // (another), the next layer's router rows (a third; routing above was
     // the last reader of the buffer)
     const size_t grow = (size_t)e * h + (size_t)j * hS;
-    stage_bytes(gq, L.gq + grow * (d / 2), hS * (d / 2));
-    stage_bytes(gq + (size_t)hS * (d / 2), L.uq + grow * (d / 2), hS * (d / 2));
+    stage_rows(reinterpret_cast<char*>(gq), d / 2 + 16,
+               reinterpret_cast<const char*>(L.gq + grow * (d / 2)), d / 2, hS, d / 2);
+    stage_rows(reinterpret_cast<char*>(gq) + (size_t)hS * (d / 2 + 16), d / 2 + 16,
+               reinterpret_cast<const char*>(L.uq + grow * (d / 2)), d / 2, hS, d / 2);
     stage_bytes(gs, L.gs + grow * nb, hS * nb * 2);
     stage_bytes(gs + (size_t)hS * nb, L.us + grow * nb, hS * nb * 2);
     cp_commit();
@@ -1079,7 +1081,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_token(const __grid_constan
     for (int u2 = tid; u2 < 2 * hS * nparts; u2 += blockDim.x) {
       const int r2 = u2 % (2 * hS), pp = u2 / (2 * hS);
       const int b0 = pp * nb / nparts, b1 = (pp + 1) * nb / nparts;
-      const uint8_t* q = gq + (size_t)r2 * (d / 2);
+      const uint8_t* q = gq + (size_t)r2 * (d / 2 + 16);
       const uint16_t* sc = gs + (size_t)r2 * nb;
       float acc = 0.0f;
 #pragma unroll 2
