@@ -106,6 +106,13 @@ __device__ __forceinline__ void cp_wait_group() {
 __device__ __forceinline__ void stage_rows(char* smem, int s_stride, const char* gmem,
                                            size_t g_stride, int rows, int row_bytes) {
   const int per_row = row_bytes / 16;
+  if (per_row <= (int)blockDim.x && blockDim.x % per_row == 0) {
+    // a thread keeps one 16-byte column and walks the rows: no division per copy
+    const int c = threadIdx.x % per_row, step = blockDim.x / per_row;
+    for (int r = threadIdx.x / per_row; r < rows; r += step)
+      cp16(smem + (size_t)r * s_stride + c * 16, gmem + r * g_stride + (size_t)c * 16);
+    return;
+  }
   for (int i = threadIdx.x; i < rows * per_row; i += blockDim.x) {
     const int r = i / per_row, c = i - r * per_row;
     cp16(smem + (size_t)r * s_stride + c * 16, gmem + r * g_stride + (size_t)c * 16);
@@ -1059,11 +1066,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_token(const __grid_constan
     stage_bytes(gs, L.gs + grow * nb, hS * nb * 2);
     stage_bytes(gs + (size_t)hS * nb, L.us + grow * nb, hS * nb * 2);
     cp_commit();
-    for (int i = tid; i < d * cpr; i += blockDim.x) {
-      const int o = i / cpr, c = i - o * cpr;
-      cp16(dq + (size_t)o * (hS / 2) + c * 16,
-           L.dq + ((size_t)e * d + o) * (h / 2) + (size_t)j * (hS / 2) + c * 16);
-    }
+    stage_rows(reinterpret_cast<char*>(dq), hS / 2,
+               reinterpret_cast<const char*>(L.dq + (size_t)e * d * (h / 2) + (size_t)j * (hS / 2)),
+               h / 2, d, hS / 2);
     stage_bytes(ds, L.ds + (size_t)e * d * nbh, d * nbh * 2);
     cp_commit();
     if (!last)
