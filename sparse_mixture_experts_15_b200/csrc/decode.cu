@@ -914,6 +914,13 @@ __device__ __forceinline__ void l2_prefetch(const void* ptr, int bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(ptr), "r"(bytes) : "memory");
 }
 
+// Shared row stride of a down row's slice (hS / 2 bytes): padded by 16 bytes
+// when it is a multiple of 32, so the 16-byte loads of a warp's 32 rows hit
+// distinct banks.
+__host__ __device__ __forceinline__ int dq_ld(int hS) {
+  return (hS / 2) % 32 == 0 ? hS / 2 + 16 : hS / 2;
+}
+
 bool make_plan2(const moe_shape& s, int sms, Plan2* out) {
   const int T = s.T, d = s.d, N = s.N, k = s.k, h = s.h;
   const int nb = d / 32, nbh = h / 32, nblk = (d + kRouteBlock - 1) / kRouteBlock;
@@ -940,7 +947,7 @@ bool make_plan2(const moe_shape& s, int sms, Plan2* out) {
     p.uf = take(off, (size_t)d * 4);
     p.gq = take(off, (size_t)2 * hS * (d / 2 + 16));  // rows padded 16 B: no bank conflicts
     p.gs = take(off, (size_t)2 * hS * nb * 2);
-    p.dq = take(off, (size_t)d * (hS / 2));
+    p.dq = take(off, (size_t)d * dq_ld(hS));
     p.ds = take(off, (size_t)d * nbh * 2);
     p.part = take(off, (size_t)2 * hS * p.nparts * 4);
     p.hs = take(off, (size_t)hS * 4);
@@ -1066,7 +1073,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_token(const __grid_constan
     stage_bytes(gs, L.gs + grow * nb, hS * nb * 2);
     stage_bytes(gs + (size_t)hS * nb, L.us + grow * nb, hS * nb * 2);
     cp_commit();
-    stage_rows(reinterpret_cast<char*>(dq), hS / 2,
+    stage_rows(reinterpret_cast<char*>(dq), dq_ld(hS),
                reinterpret_cast<const char*>(L.dq + (size_t)e * d * (h / 2) + (size_t)j * (hS / 2)),
                h / 2, d, hS / 2);
     stage_bytes(ds, L.ds + (size_t)e * d * nbh, d * nbh * 2);
@@ -1131,7 +1138,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_token(const __grid_constan
     // units, into this CTA's buffer of the layer's parity
     float* ymine = yr + (size_t)(l & 1) * d;
     for (int o = tid; o < d; o += blockDim.x) {
-      const uint8_t* q = dq + (size_t)o * (hS / 2);
+      const uint8_t* q = dq + (size_t)o * dq_ld(hS);
       float a0 = 0.0f, a1 = 0.0f;
 #pragma unroll 2
       for (int bl = 0; bl < cpr; ++bl) {
