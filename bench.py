@@ -607,11 +607,21 @@ class DecodeReplica:
         return sum(t.numel() * t.element_size() for t in self.keep)
 
 
-# Intervals between the 13 per-layer stamps of the per-token decode kernel
-# (the kernel the benchmark shapes run); the bracketed ones are empty there.
-DECODE_PHASES = ("(stamps 0-1)", "route", "(stamps 2-3)", "stage item rows", "(stamps 4-5)",
-                 "gate/up dots", "H", "(stamps 7-8)", "down columns ready",
-                 "down partial + count", "wait for the token's rows", "next row")
+# Intervals between the 13 per-layer stamps of each decode kernel (the
+# bracketed ones are empty in the per-token kernel).
+DECODE_PHASES = {
+    1: ("(stamps 0-1)", "route", "(stamps 2-3)", "stage item rows", "(stamps 4-5)",
+        "gate/up dots", "H", "(stamps 7-8)", "down columns ready", "down partial row",
+        "cluster barrier", "next row"),
+    2: ("stage u", "route", "group pairs", "stage gate/up rows", "(stamps 4-5)", "gate/up dots",
+        "H store", "grid barrier 1", "down rows ready", "down dots", "combine + u_next",
+        "grid barrier 2"),
+}
+DECODE_KERNELS = {
+    1: "decode_token: all layers of the step in one launch, one thread-block cluster per token",
+    2: "decode_persistent: all layers of the step in one cooperative launch, two grid barriers "
+       "per layer",
+}
 
 
 def decode_phases(wl, moe, s, rep, out, ws, torch, sm_mhz: float):
@@ -626,7 +636,7 @@ def decode_phases(wl, moe, s, rep, out, ws, torch, sm_mhz: float):
     per = np.median(cyc, axis=0) / sm_mhz
     layer = np.median(st[1:, -1] - st[1:, 0] if wl.n_layers > 1 else st[:, -1] - st[:, 0]) / sm_mhz
     return {"layer_us": float(layer), "sm_mhz": sm_mhz,
-            **{name: float(v) for name, v in zip(DECODE_PHASES, per)}}
+            **{name: float(v) for name, v in zip(DECODE_PHASES[moe.moe_decode_kernel(s)], per)}}
 
 
 def decode_main(args, wl, torch, moe, rank, world, dist):
@@ -724,8 +734,7 @@ def decode_main(args, wl, torch, moe, rank, world, dist):
                                  f"({n_rep * one.nbytes() / 2**20:.0f} MiB > L2)"},
                 "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
                              "frac": achieved / hbm, "traffic": None,
-                             "kernel": "decode_persistent: all layers of the step in one "
-                                       "cooperative launch",
+                             "kernel": DECODE_KERNELS[moe.moe_decode_kernel(s)],
                              "phases_us": phases,
                              "bytes_per_step": bytes_timed / args.steps,
                              "peak_source": f"{src} hbm_gbs",

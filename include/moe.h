@@ -454,15 +454,23 @@ MOE_API int moe_decode_layer(const moe_shape* shape, const moe_q4_layer* layer, 
                              uint16_t* y, uint16_t* u_next, int32_t* top_idx, float* top_w,
                              void* ws, size_t ws_bytes, void* stream);
 
+/* Which kernel moe_decode_layer and moe_decode_step run for this shape on
+ * the current device: 1 the per-token kernel, 2 the two-phase kernel, 0 the
+ * shape is outside the limits above (or no device is visible). */
+MOE_API int moe_decode_kernel(const moe_shape* shape);
+
 /* n_layers chained layers: u_{l+1} = fp16(u_l + y_l), u_out = u_{n_layers}.
  * `layers` is a host array of n_layers structs.  top_idx_all [n_layers][T][k]
  * (nullable) receives every layer's routing.  Up to 32 layers run in one
- * cooperative launch (at most one CTA per SM, every wait bounded:
- * MOE_ERR_TIMEOUT in the device status word).  When the T k (token, slot)
- * pairs fit one CTA each and its shared-memory plan fits, the launch runs
+ * launch (at most one CTA per SM; the two-phase kernel is a cooperative
+ * launch whose grid-barrier waits are bounded: MOE_ERR_TIMEOUT in the device
+ * status word).  When the T k (token, slot)
+ * pairs fit one CTA each, its shared-memory plan fits and a cluster of a
+ * token's CTAs can be resident, the launch runs
  * the per-token kernel (CTA = (token, slot, hidden slice) for all layers,
- * the token's CTAs exchanging partial output rows through a per-token
- * counter, no grid barrier); otherwise a two-phase kernel (selected-expert
+ * the token's k S CTAs one thread-block cluster that exchanges partial
+ * output rows through distributed shared memory, no grid barrier);
+ * otherwise a two-phase kernel (selected-expert
  * hidden slices, grid barrier, (token, output rows) units, grid barrier).
  * The kernel is chosen from the shape, so a chain and moe_decode_layer use
  * the same per-layer arithmetic and a chain equals the layer calls made one
@@ -476,8 +484,9 @@ MOE_API int moe_decode_step(const moe_shape* shape, int32_t n_layers, const moe_
  * 8-byte aligned; caller-owned).  Per-token kernel (block 0 = token 0,
  * slot 0, slice 0): 0 layer start, 1 = 0, 2 routed, 3 = 2, 4 the slice's
  * gate/up rows staged, 5 = 4, 6 gate/up dots formed, 7 H formed, 8 = 7,
- * 9 down columns ready, 10 partial output row stored and counted, 11 all of
- * the token's partial rows counted, 12 next row formed.
+ * 9 down columns ready, 10 partial output row in shared memory, 11 the
+ * cluster barrier passed (every partial row of the token stored), 12 next
+ * row formed.
  * Two-phase kernel: 0 layer start, 1 input rows staged, 2 routed, 3
  * dispatch pairs grouped by expert, 4 gate/up q4 rows staged, 5 = 4, 6
  * gate/up dots formed, 7 hidden phase done (H stored), 8 first grid barrier

@@ -115,6 +115,7 @@ _PROTOS = {
                                    ctypes.POINTER(MoeE4M3Scales),
                                    ctypes.POINTER(MoeLatentWeights), _vp, _vp,
                                    ctypes.POINTER(MoeLayerOutputs), _vp, _sz, _vp]),
+    "moe_decode_kernel": (_i32, [_P_SHAPE]),
     "moe_decode_workspace_bytes": (_sz, [_P_SHAPE]),
     "moe_decode_layer": (_i32, [_P_SHAPE, ctypes.POINTER(MoeQ4Layer), _vp, _vp, _vp, _vp, _vp,
                                 _vp, _sz, _vp]),
@@ -528,6 +529,13 @@ def q4_layer(w_route, gate_qs, gate_scales, up_qs, up_scales, down_qs, down_scal
         _need(*args)
     return MoeQ4Layer(_ptr(w_route), _ptr(bias), _ptr(gate_qs), _ptr(gate_scales), _ptr(up_qs),
                       _ptr(up_scales), _ptr(down_qs), _ptr(down_scales))
+
+
+DECODE_PER_TOKEN, DECODE_TWO_PHASE = 1, 2  # moe_decode_kernel's answers (0: unsupported)
+
+
+def moe_decode_kernel(s: MoeShape) -> int:
+    return int(_lib.moe_decode_kernel(ctypes.byref(s)))
 
 
 def moe_decode_workspace_bytes(s: MoeShape) -> int:

@@ -1277,13 +1277,32 @@ LayerPtrs layer_ptrs(const moe_q4_layer& L) {
                    L.up_qs,   L.up_scales, L.down_qs, L.down_scales};
 }
 
-// The one-barrier kernel over layers [0, n) when its plan fits.
+enum class DecodeKind { kNone = 0, kPerToken = 1, kTwoPhase = 2 };
+
+// Launch configuration of the per-token kernel: T k S CTAs in clusters of
+// k S (one token each); attr must outlive the returned configuration.
+cudaLaunchConfig_t token_launch_cfg(const moe_shape& s, const Plan2& plan, cudaStream_t st,
+                                    cudaLaunchAttribute* attr) {
+  const int ks = s.k * plan.S;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(s.T * ks);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = plan.total;
+  cfg.stream = st;
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = ks;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cfg;
+}
+
 // The per-token kernel over layers [0, n): T k S CTAs, one item each, in
 // clusters of k S (one token each).
 int launch_decode_token(const moe_shape& s, const Plan2& plan, const moe_q4_layer* layers, int n,
                         const __half* u_in, __half* u_out, __half* y, int32_t* top_idx,
                         float* top_w, cudaStream_t st, unsigned long long* stamps) {
-  const int ks = s.k * plan.S;
   Params2 p{};
   p.plan = plan;
   for (int l = 0; l < n; ++l) p.layer[l] = layer_ptrs(layers[l]);
@@ -1300,23 +1319,26 @@ int launch_decode_token(const moe_shape& s, const Plan2& plan, const moe_q4_laye
   p.top_idx = top_idx;
   p.top_w = top_w;
   p.stamps = stamps;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(s.T * ks);
-  cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = plan.total;
-  cfg.stream = st;
   cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = ks;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  int clusters = 0;
-  if (cudaOccupancyMaxActiveClusters(&clusters, decode_token, &cfg) != cudaSuccess)
-    return MOE_ERR_CUDA;
-  if (clusters < 1) return MOE_ERR_UNSUPPORTED;
+  const cudaLaunchConfig_t cfg = token_launch_cfg(s, plan, st, attr);
   return cudaLaunchKernelEx(&cfg, decode_token, p) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+// Which kernel a shape runs on this device: the per-token kernel when its
+// plan fits and a cluster of the token's k S CTAs can be resident, else the
+// two-phase kernel when its plan fits, else none.
+DecodeKind choose_decode(const moe_shape& s, int sms, Plan2* plan2) {
+  if (make_plan2(s, sms, plan2)) {
+    cudaLaunchAttribute attr[1];
+    const cudaLaunchConfig_t cfg = token_launch_cfg(s, *plan2, nullptr, attr);
+    int clusters = 0;
+    if (cudaOccupancyMaxActiveClusters(&clusters, decode_token, &cfg) == cudaSuccess &&
+        clusters >= 1)
+      return DecodeKind::kPerToken;
+    cudaGetLastError();  // clear the error a failed query recorded
+  }
+  Plan p;
+  return make_plan(s, sms, &p) ? DecodeKind::kTwoPhase : DecodeKind::kNone;
 }
 
 // One launch over layers [0, n) of `layers`: the per-token kernel (thread-
@@ -1328,7 +1350,9 @@ int launch_decode(const moe_shape& s, const moe_q4_layer* layers, int n, const _
   int sms = 0;
   if (!device_info(&sms)) return MOE_ERR_CUDA;
   Plan2 plan2;
-  if (make_plan2(s, sms, &plan2))
+  const DecodeKind kind = choose_decode(s, sms, &plan2);
+  if (kind == DecodeKind::kNone) return MOE_ERR_UNSUPPORTED;
+  if (kind == DecodeKind::kPerToken)
     return launch_decode_token(s, plan2, layers, n, u_in, u_out, y, top_idx, top_w, st, stamps);
   Params p{};
   if (!make_plan(s, sms, &p.plan)) return MOE_ERR_UNSUPPORTED;
@@ -1375,6 +1399,14 @@ int launch_decode(const moe_shape& s, const moe_q4_layer* layers, int n, const _
 
 }  // namespace
 }  // namespace moe
+
+extern "C" int moe_decode_kernel(const moe_shape* shape) {
+  if (!moe::decode_shape_ok(shape)) return 0;
+  int sms = 0;
+  if (!moe::device_info(&sms) || sms <= 0) return 0;
+  moe::Plan2 plan2;
+  return static_cast<int>(moe::choose_decode(*shape, sms, &plan2));
+}
 
 extern "C" size_t moe_decode_workspace_bytes(const moe_shape* shape) {
   if (!moe::decode_shape_ok(shape)) return 0;

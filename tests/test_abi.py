@@ -278,3 +278,19 @@ def test_decode_shape_support_query(T, d, N, k, h, ok):
     for the shapes the persistent kernel's shared-memory plan can hold."""
     n = moe.moe_decode_workspace_bytes(moe.shape(T, d, N, k, h, 1, 0))
     assert (n > 0) == ok
+
+
+def test_decode_kernel_query_on_the_host():
+    """The decode kernel query answers 0 for a shape outside the limits, and
+    0 for every shape where no device is visible; with a device the benchmark
+    shapes run the per-token kernel and 64 experts top-8 (more (token, slot)
+    pairs than SMs) the two-phase kernel."""
+    import torch
+    assert moe.moe_decode_kernel(moe.shape(33, 512, 8, 2, 128, 1, 0)) == 0
+    assert moe.moe_decode_kernel(moe.shape(32, 500, 8, 2, 128, 1, 0)) == 0
+    if not torch.cuda.is_available():
+        assert moe.moe_decode_kernel(moe.shape(32, 512, 8, 2, 128, 1, 0)) == 0
+        return
+    for T in (1, 8, 32):
+        assert moe.moe_decode_kernel(moe.shape(T, 512, 8, 2, 128, 1, 0)) == moe.DECODE_PER_TOKEN
+    assert moe.moe_decode_kernel(moe.shape(32, 512, 64, 8, 128, 1, 0)) == moe.DECODE_TWO_PHASE

@@ -166,21 +166,25 @@ def test_decode_layer_other_shapes(T, d, N, k, h):
     assert rel_err(y.float().cpu().numpy(), oy) < TOL_Q4
 
 
-@pytest.mark.parametrize("T,d,N,k,h", [
-    (32, 1024, 8, 2, 256),   # two-phase kernel, output units of 256 rows: two router blocks each
-    (32, 512, 64, 8, 128),   # two-phase kernel, 64 experts: 64 block sums per unit
-    (16, 512, 8, 2, 128),    # per-token kernel, 16 tokens x 2 slots x 4 slices
-    (16, 2048, 8, 2, 128),   # per-token kernel, wide rows
+PER_TOKEN, TWO_PHASE = 1, 2  # moe_decode_kernel's answers
+
+
+@pytest.mark.parametrize("T,d,N,k,h,kind", [
+    (32, 1024, 8, 2, 256, TWO_PHASE),  # output units of 256 rows: two router blocks each
+    (32, 512, 64, 8, 128, TWO_PHASE),  # 64 experts: 64 block sums per unit
+    (16, 512, 8, 2, 128, PER_TOKEN),   # 16 tokens x 2 slots x 4 slices
+    (16, 2048, 8, 2, 128, PER_TOKEN),  # wide rows
 ])
-def test_decode_step_equals_layers(T, d, N, k, h):
+def test_decode_step_equals_layers(T, d, N, k, h, kind):
     """A 3-layer chained step (layers 1.. route from the router block sums
-    that the previous layer formed, in either decode kernel) equals the
-    layer calls made one by one, which form the block sums from their own
-    input."""
+    that the previous layer formed, in either decode kernel, the one the
+    shape runs checked by the kernel query) equals the layer calls made one
+    by one, which form the block sums from their own input."""
     import dataclasses
     wl = dataclasses.replace(W.decode(T=T, n_layers=3), d=d, N=N, k=k, h=h)
     layers = [Layer(wl, l) for l in range(wl.n_layers)]
     s = moe.shape(T, d, N, k, h, 1, 0)
+    assert moe.moe_decode_kernel(s) == kind
     u0 = _f16(_u0(wl))
     out = torch.empty_like(u0)
     idx_all = torch.empty((wl.n_layers, T, k), dtype=torch.int32, device="cuda")
