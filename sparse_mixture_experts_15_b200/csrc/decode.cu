@@ -1136,22 +1136,52 @@ __global__ void __launch_bounds__(kThreads, 1) decode_token(const __grid_constan
     stamp2(p, l, 9);
     // ---- partial output row: row o of W_down[e] over the slice's hidden
     // units, into this CTA's buffer of the layer's parity
+    // A thread takes rows o0 and o0 + blockDim.x together, so each H value
+    // it loads feeds both; per q4 block the sum of (q - 8) h, then one
+    // multiply-add by the block scale.
     float* ymine = yr + (size_t)(l & 1) * d;
-    for (int o = tid; o < d; o += blockDim.x) {
-      const uint8_t* q = dq + (size_t)o * dq_ld(hS);
-      float a0 = 0.0f, a1 = 0.0f;
+    const int dld = dq_ld(hS);
+    for (int o0 = tid; o0 < d; o0 += 2 * blockDim.x) {
+      const int o1 = o0 + blockDim.x < d ? o0 + blockDim.x : o0;
+      const uint8_t* q0 = dq + (size_t)o0 * dld;
+      const uint8_t* q1 = dq + (size_t)o1 * dld;
+      const uint16_t* s0 = ds + (size_t)o0 * nbh + (size_t)j * cpr;
+      const uint16_t* s1 = ds + (size_t)o1 * nbh + (size_t)j * cpr;
+      float y0 = 0.0f, y1 = 0.0f;
 #pragma unroll 2
       for (int bl = 0; bl < cpr; ++bl) {
-        float wv[32];
-        dequant_block(q + bl * 16, ds[(size_t)o * nbh + (size_t)j * cpr + bl], wv);
-        const float* hb = hsv + bl * 32;
+        const uint4 r0 = *reinterpret_cast<const uint4*>(q0 + bl * 16);
+        const uint4 r1 = *reinterpret_cast<const uint4*>(q1 + bl * 16);
+        const uint32_t w0[4] = {r0.x, r0.y, r0.z, r0.w}, w1[4] = {r1.x, r1.y, r1.z, r1.w};
+        const float4* h4 = reinterpret_cast<const float4*>(hsv + bl * 32);
+        float c00 = 0.0f, c01 = 0.0f, c10 = 0.0f, c11 = 0.0f;
 #pragma unroll
-        for (int c = 0; c < 32; c += 2) {
-          a0 = fmaf(wv[c], hb[c], a0);
-          a1 = fmaf(wv[c + 1], hb[c + 1], a1);
+        for (int i = 0; i < 4; ++i) {
+          const uint32_t lo0 = w0[i] & 0x0F0F0F0Fu, hi0 = (w0[i] >> 4) & 0x0F0F0F0Fu;
+          const uint32_t lo1 = w1[i] & 0x0F0F0F0Fu, hi1 = (w1[i] >> 4) & 0x0F0F0F0Fu;
+          const float4 hl = h4[i], hh = h4[4 + i];  // elements 4i.. and 16+4i..
+          c00 = fmaf(nib(lo0, 0), hl.x, c00);
+          c10 = fmaf(nib(lo1, 0), hl.x, c10);
+          c01 = fmaf(nib(lo0, 1), hl.y, c01);
+          c11 = fmaf(nib(lo1, 1), hl.y, c11);
+          c00 = fmaf(nib(lo0, 2), hl.z, c00);
+          c10 = fmaf(nib(lo1, 2), hl.z, c10);
+          c01 = fmaf(nib(lo0, 3), hl.w, c01);
+          c11 = fmaf(nib(lo1, 3), hl.w, c11);
+          c00 = fmaf(nib(hi0, 0), hh.x, c00);
+          c10 = fmaf(nib(hi1, 0), hh.x, c10);
+          c01 = fmaf(nib(hi0, 1), hh.y, c01);
+          c11 = fmaf(nib(hi1, 1), hh.y, c11);
+          c00 = fmaf(nib(hi0, 2), hh.z, c00);
+          c10 = fmaf(nib(hi1, 2), hh.z, c10);
+          c01 = fmaf(nib(hi0, 3), hh.w, c01);
+          c11 = fmaf(nib(hi1, 3), hh.w, c11);
         }
+        y0 = fmaf(f16f(s0[bl]), c00 + c01, y0);
+        y1 = fmaf(f16f(s1[bl]), c10 + c11, y1);
       }
-      ymine[o] = a0 + a1;
+      ymine[o0] = y0;
+      if (o1 != o0) ymine[o1] = y1;
     }
     stamp2(p, l, 10);
     // while the cluster meets: CTA b < N S pulls the next layer's gate/up
