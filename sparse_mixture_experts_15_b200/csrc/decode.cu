@@ -58,20 +58,26 @@ __device__ __forceinline__ float nib(uint32_t v, int b) {
   return __uint_as_float(__byte_perm(v, 0x4B000000u, 0x7540 | b)) - 8388616.0f;
 }
 
-// 32 weights of one q4_0 block: byte j -> element j (low nibble), j+16 (high).
-__device__ __forceinline__ void dequant_block(const uint8_t* qs, uint16_t scale, float* w) {
+// Sum over one q4_0 block of (q - 8) x (byte j of the block holds element j
+// in its low nibble and element j + 16 in its high one): four chains, added
+// pairwise; the caller applies the block scale once.
+__device__ __forceinline__ float q4_block_dot(const uint8_t* qs, const float* x) {
   const uint4 raw = *reinterpret_cast<const uint4*>(qs);
-  const float s = f16f(scale);
   const uint32_t wd[4] = {raw.x, raw.y, raw.z, raw.w};
+  float a0 = 0.0f, a1 = 0.0f, a2 = 0.0f, a3 = 0.0f;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const uint32_t lo = wd[i] & 0x0F0F0F0Fu, hi = (wd[i] >> 4) & 0x0F0F0F0Fu;
-#pragma unroll
-    for (int b = 0; b < 4; ++b) {
-      w[4 * i + b] = nib(lo, b) * s;
-      w[16 + 4 * i + b] = nib(hi, b) * s;
-    }
+    a0 = fmaf(nib(lo, 0), x[4 * i], a0);
+    a1 = fmaf(nib(lo, 1), x[4 * i + 1], a1);
+    a2 = fmaf(nib(lo, 2), x[4 * i + 2], a2);
+    a3 = fmaf(nib(lo, 3), x[4 * i + 3], a3);
+    a0 = fmaf(nib(hi, 0), x[16 + 4 * i], a0);
+    a1 = fmaf(nib(hi, 1), x[16 + 4 * i + 1], a1);
+    a2 = fmaf(nib(hi, 2), x[16 + 4 * i + 2], a2);
+    a3 = fmaf(nib(hi, 3), x[16 + 4 * i + 3], a3);
   }
+  return (a0 + a1) + (a2 + a3);
 }
 
 
@@ -791,20 +797,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_persistent(const __grid_co
           for (int c = 0; c < 32; ++c) hc[c] = 0.f;
         }
         for (int r = g * rper; r < (g + 1) * rper; ++r) {
-          float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-          if (valid) {
-            float wv[32];
-            dequant_block(bq + ((size_t)s2 * RB + r) * (h / 2) + pp * 16,
-                          bs[((size_t)s2 * RB + r) * nbh + pp], wv);
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-              a0 = fmaf(wv[4 * c], hc[4 * c], a0);
-              a1 = fmaf(wv[4 * c + 1], hc[4 * c + 1], a1);
-              a2 = fmaf(wv[4 * c + 2], hc[4 * c + 2], a2);
-              a3 = fmaf(wv[4 * c + 3], hc[4 * c + 3], a3);
-            }
-          }
-          float zz = (a0 + a1) + (a2 + a3);
+          // the block's sum of (q - 8) h times its scale
+          float zz = 0.0f;
+          if (valid)
+            zz = f16f(bs[((size_t)s2 * RB + r) * nbh + pp]) *
+                 q4_block_dot(bq + ((size_t)s2 * RB + r) * (h / 2) + pp * 16, hc);
           for (int o = nbh / 2; o >= 1; o >>= 1) zz += __shfl_xor_sync(0xffffffffu, zz, o);
           if (valid && pp == 0) zs[s2 * (RB + 1) + r] = zz;
         }
