@@ -150,9 +150,17 @@ __device__ __noinline__ void topk_wide(const float* zt, int N, int k, int renorm
   float ps = 0.0f;
   float a[8];
   for (int s = 0; s < k; ++s) {
+    // the running best kept in a register (bv == zt[bi]), so no comparison
+    // waits on a load whose address depends on the previous one
     int bi = -1;
-    for (int i = 0; i < N; ++i)
-      if (!((taken >> i) & 1ull) && (bi < 0 || zt[i] > zt[bi])) bi = i;
+    float bv = 0.0f;
+    for (int i = 0; i < N; ++i) {
+      const float zi = zt[i];
+      if (!((taken >> i) & 1ull) && (bi < 0 || zi > bv)) {
+        bi = i;
+        bv = zi;
+      }
+    }
     if (bi < 0) bi = __ffsll((long long)~taken) - 1;  // only NaN logits left
     taken |= 1ull << bi;
     sel[s] = bi;
