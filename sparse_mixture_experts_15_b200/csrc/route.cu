@@ -397,9 +397,15 @@ __global__ void __launch_bounds__(kRouteThreads)
     int isel[16];
     float ps = 0.0f;
     for (int s = 0; s < k; ++s) {
-      int bi = -1;
-      for (int i = 0; i < N; ++i)
-        if (!((taken >> i) & 1u) && (bi < 0 || z[i] > z[bi])) bi = i;
+      int bi = -1;  // the running best's value kept in a register (bv == z[bi])
+      float bv = 0.0f;
+      for (int i = 0; i < N; ++i) {
+        const float zi = z[i];
+        if (!((taken >> i) & 1u) && (bi < 0 || zi > bv)) {
+          bi = i;
+          bv = zi;
+        }
+      }
       taken |= 1u << bi;
       isel[s] = bi;
       psel[s] = expf(z[bi] - zmax) / den;
