@@ -439,11 +439,17 @@ bool make_plan(const moe_shape& s, int sms, Plan* out) {
   const int nb = d / 32, nbh = h / 32;
   // phase-B units are (token, RB output rows): ideally the T * d / RB units
   // fill at most one wave of CTAs, and each unit reads only its token's k
-  // rows of H; RB divides d.  Smaller RB (more units per CTA), then a single
-  // router buffer, then fewer hidden rows per item when shared memory is short.
+  // rows of H; RB divides d.  Of the plans that fit shared memory (RB, then
+  // the router buffers, then RA descending), the one with the fewest phase-A
+  // items plus phase-B units per CTA wins, a plan without routing from the
+  // previous layer's block sums counting two more (a CTA runs its items and
+  // units one after another, each a staging round trip and its dots); ties
+  // keep the earlier plan.
   int RB_max = 4;
   while (RB_max < d && d % (2 * RB_max) == 0 && (int64_t)T * (d / RB_max) > sms) RB_max *= 2;
   const int nsel_max = N < T * k ? N : T * k;
+  bool found = false;
+  int best = 0;
   for (int RB = RB_max; RB >= 4; RB /= 2)
   for (int nbuf = 2; nbuf >= 1; --nbuf) {
     for (int RA = 8; RA >= 2; RA /= 2) {
@@ -479,13 +485,20 @@ bool make_plan(const moe_shape& s, int sms, Plan* out) {
       p.bs = take(off, (size_t)k * RB * nbh * 2);
       p.zs = take(off, (size_t)k * (RB + 1) * 4);
       p.total = off;
-      if (off <= kSmemLimit) {
+      if (off > kSmemLimit) continue;
+      const int items = nsel_max * (h / RA), units = T * (d / RB);
+      int grid = items > units ? items : units;
+      if (grid > sms) grid = sms;
+      if (grid < 1) grid = 1;  // T = 0: no items and no units
+      const int score = (items + grid - 1) / grid + (units + grid - 1) / grid + (p.early ? 0 : 2);
+      if (!found || score < best) {
         *out = p;
-        return true;
+        best = score;
+        found = true;
       }
     }
   }
-  return false;
+  return found;
 }
 
 // ---------------------------------------------------------------- kernel

@@ -294,3 +294,10 @@ def test_decode_kernel_query_on_the_host():
     for T in (1, 8, 32):
         assert moe.moe_decode_kernel(moe.shape(T, 512, 8, 2, 128, 1, 0)) == moe.DECODE_PER_TOKEN
     assert moe.moe_decode_kernel(moe.shape(32, 512, 64, 8, 128, 1, 0)) == moe.DECODE_TWO_PHASE
+
+
+@pytest.mark.parametrize("N,k", [(8, 2), (64, 8)])
+def test_decode_plan_for_an_empty_batch(N, k):
+    """The decode shape check plans T = 0 too (no items, no units): the
+    workspace query answers on the host instead of failing."""
+    assert moe.moe_decode_workspace_bytes(moe.shape(0, 512, N, k, 128, 1, 0)) > 0
